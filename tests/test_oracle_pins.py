@@ -493,3 +493,51 @@ def test_attention_brute_force_decimal():
 def test_attention_empty_is_zero():
     out = orc.attention(np.ones((1, 2, 128)), np.zeros((1, 0, 1, 128)), np.zeros((1, 0, 1, 128)), 1.0)
     assert (out == 0).all()
+
+
+def test_encoded_records_quantize_the_rotated_residual():
+    """Record-level check with an independent path: y = R (x_l - s_hat a_hat)
+    computed here by a butterfly, then every residual group's scale/min must
+    be the FP8 values nearest (max-min)/3 and min (table search), and every
+    code the nearest grid point (exhaustive search).  The anchor record is
+    checked the same way against x_L itself."""
+    rng = np.random.default_rng(71)
+    n, d, L, seed = 24, 128, 4, 0xA11CE
+    anchor = rng.standard_normal((n, d))
+    anchor[:, [3, 40, 77, 100]] *= 10.0
+    loops = [rng.uniform(0.8, 1.2, (n, 1)) * anchor + s * rng.standard_normal((n, d)) for s in (0.3, 0.2, 0.02)]
+    x = np.stack([_bf16(a) for a in loops + [anchor]])
+    e = orc.encode(x, 16, 4, 2, True, seed)
+    rec = orc.reconstruct(e.a_codes, e.a_meta, e.r_codes, e.r_meta, e.r_coef, L, d, 16, 4, 2, True, seed)
+    table = _fp8_table()
+    sigma = orc.rotation_signs(seed, d)
+
+    def nearest_fp8(v):
+        return min(table, key=lambda cv: (abs(cv[1] - v), cv[0] & 1))[1]
+
+    def check(vec, packed, meta, bits, eflag, mflag):
+        qmax = (1 << bits) - 1
+        codes = orc.unpack(packed, d, bits)
+        for grp in range(d // 16):
+            seg = vec[grp * 16:(grp + 1) * 16]
+            s8, m8 = orc.fp8_value(int(meta[2 * grp])), orc.fp8_value(int(meta[2 * grp + 1]))
+            if not mflag[grp] & 1:
+                assert s8 == nearest_fp8((seg.max() - seg.min()) / qmax)
+            if not mflag[grp] & 2:
+                assert m8 == nearest_fp8(seg.min())
+            if mflag[grp]:
+                continue
+            for i in range(16):
+                if eflag[grp * 16 + i] or s8 == 0:
+                    continue
+                errs = [abs(seg[i] - (m8 + c * s8)) for c in range(qmax + 1)]
+                assert codes[grp * 16 + i] == int(np.argmin(errs))
+
+    xf = orc.bf16_bits_to_f64(x)
+    for t in range(n):
+        check(xf[L - 1, t], e.a_codes[t], e.a_meta[t], 4, e.a_eflag[t], e.a_mflag[t])
+        ahat = rec[L - 1, t]
+        for l in range(L - 1):
+            sh = orc.bf16_value(int(e.r_coef[l, t]))
+            y = _fwht(sigma * (xf[l, t] - sh * ahat)) / math.sqrt(d)
+            check(y, e.r_codes[l, t], e.r_meta[l, t], 2, e.r_eflag[l, t], e.r_mflag[l, t])
