@@ -1,0 +1,464 @@
+"""Benchmark of the ResidualQuant decode step on B200.
+
+A step is one decode step of a looped Transformer over a cache already
+holding T-1 committed tokens per sequence: for every loop (outer) and layer
+(inner) it appends the new token's K/V (rq_append: tail copy for loops 1..L-1,
+fp64 encode + commit at the anchor loop) and runs single-token decode
+attention (rq_decode_attn) over T keys.  The metric is decode-attention
+tokens/s = batch / step time (whole job: all ranks' sequences / max-over-ranks
+time), plus achieved HBM GB/s of the decode calls over their algorithmic
+compressed bytes.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+Multi-GPU: launched by torchrun, one rank per GPU; every rank owns its own
+batch (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CONFIGS = {
+    # name: (layers, loops, loops_per_group, batch, T, H_kv, H_q, g, ba, br, sigma by distance)
+    "tiny": dict(layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, sigma=(0.1, 0.2, 0.3)),
+    "ouro8k_b4": dict(layers=24, loops=4, Lg=4, B=4, T=8192, H=16, Hq=16, g=16, ba=4, br=2, sigma=(0.1, 0.2, 0.3)),
+    "long16k_b2": dict(layers=24, loops=4, Lg=4, B=2, T=16384, H=16, Hq=16, g=16, ba=4, br=2, sigma=(0.1, 0.2, 0.3)),
+    "long16k_b4": dict(layers=24, loops=4, Lg=4, B=4, T=16384, H=16, Hq=16, g=16, ba=4, br=2, sigma=(0.1, 0.2, 0.3)),
+    "deep": dict(layers=4, loops=32, Lg=4, B=8, T=4096, H=40, Hq=40, g=16, ba=4, br=2, sigma=(0.1, 0.25, 0.4)),
+}
+CONFIG_SEED = {"tiny": 0x5EED0000, "ouro8k_b4": 0x5EED0001, "long16k_b2": 0x5EED0002,
+               "long16k_b4": 0x5EED0002, "deep": 0x5EED0003}
+FILL_CHUNK = 512
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling (every 50 ms) around the
+    timed region; summarise() keeps only the samples taken inside a host
+    wall-clock window."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+
+    def summarise(self, t0: float, t1: float):
+        import datetime
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for n, v in zip(names, r[3]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": max(r[2] for r in inside),
+                "samples": len(inside), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, cfgd, rank, world, local_rank):
+    import torch
+    import decode_attention_14_b200 as rq
+    from decode_attention_14_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    name = args.config
+    layers = args.layers or cfgd["layers"]
+    loops, Lg, B, T, H, Hq = cfgd["loops"], cfgd["Lg"], cfgd["B"], cfgd["T"], cfgd["H"], cfgd["Hq"]
+    seed = CONFIG_SEED[name] + 1000 * rank
+    fmt = rq.RQ_FMT_BF16 if args.bf16 else rq.RQ_FMT_RESIDUAL
+    cfg = rq.make_config(num_layers=layers, num_loops=loops, loops_per_group=Lg, batch=B, max_tokens=T,
+                         max_tail_tokens=FILL_CHUNK, num_kv_heads=H, num_q_heads=Hq, group_size=cfgd["g"],
+                         anchor_bits=cfgd["ba"], resid_bits=cfgd["br"], rotate=True, format=fmt, seed=0xA11CE)
+    cache = rq.Cache(cfg, device=dev)
+    T0 = T - 1
+    groups = loops // Lg
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- fill: T-1 committed tokens per (layer, group) (untimed)
+    for layer in range(layers):
+        for grp in range(groups):
+            for t0 in range(0, T0, FILL_CHUNK):
+                n = min(FILL_CHUNK, T0 - t0)
+                Kg, Vg = synth.group_kv(seed, layer, grp, Lg, cfgd["sigma"], B, n, H, t0=t0, device=dev)
+                for j in range(Lg):
+                    cache.append(layer, grp * Lg + j, Kg[j], Vg[j])
+                del Kg, Vg
+    torch.cuda.synchronize(dev)
+
+    # ---- per-step inputs: the new token of every (layer, loop), one query each
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(synth.mix_seed(seed, 99))
+    new_k = torch.randn((layers, loops, B, 1, H, 128), generator=gen, device=dev).to(torch.bfloat16)
+    new_v = torch.randn((layers, loops, B, 1, H, 128), generator=gen, device=dev).to(torch.bfloat16)
+    qs = torch.stack([torch.stack([synth.queries(seed, l, lp, 0, B, Hq, device=dev) for lp in range(loops)])
+                      for l in range(layers)])
+    outs = torch.empty((layers, loops, B, Hq, 128), dtype=torch.float32, device=dev)
+
+    decode = rq.rq_decode_attn_bf16 if args.bf16 else rq.rq_decode_attn
+    h = cache.h
+
+    def reset():
+        # host-side only: roll every (layer, group) back to T-1 committed tokens
+        n_groups = loops if args.bf16 else groups
+        for layer in range(layers):
+            for grp in range(n_groups):
+                cache.truncate(layer, grp, T0)
+
+    def step(ev=None, k=None, v=None, q=None):
+        k = new_k if k is None else k
+        v = new_v if v is None else v
+        q = qs if q is None else q
+        reset()
+        cur = torch.cuda.current_stream(dev)
+        sptr = int(cur.cuda_stream)
+        for lp in range(loops):
+            for layer in range(layers):
+                st = rq.rq_append(h, layer, lp, k[layer, lp], v[layer, lp], 1, sptr)
+                if st != 0:
+                    raise rq.RQError(st, "rq_append")
+                if ev is not None:
+                    ev[0][lp * layers + layer].record(cur)
+                st = decode(h, layer, lp, q[layer, lp], outs[layer, lp], 0.0, sptr)
+                if ev is not None:
+                    ev[1][lp * layers + layer].record(cur)
+                if st != 0:
+                    raise rq.RQError(st, "rq_decode_attn")
+
+    # algorithmic bytes of each decode call during a step (lengths as in the step)
+    reset()
+    call_bytes = []
+    for lp in range(loops):
+        for layer in range(layers):
+            rq.rq_append(h, layer, lp, new_k[layer, lp], new_v[layer, lp], 1, int(stream.cuda_stream))
+            call_bytes.append(cache.decode_bytes(layer, lp))
+    torch.cuda.synchronize(dev)
+    step_decode_bytes = sum(call_bytes)
+
+    # The timed region replays one CUDA graph holding K identical steps (the
+    # host-side state is reset to T-1 committed tokens before each captured
+    # step, so every step launches the same work); external timing events
+    # around every decode call become graph nodes.
+    ncalls = loops * layers
+    evs = [([torch.cuda.Event(enable_timing=True, external=True) for _ in range(ncalls)],
+            [torch.cuda.Event(enable_timing=True, external=True) for _ in range(ncalls)]) for _ in range(args.steps)]
+    for _ in range(2):
+        step()   # eager warm-up before capture
+    torch.cuda.synchronize(dev)
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1):
+        step()
+    gK = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gK):
+        for s_ in range(args.steps):
+            step(evs[s_])
+    torch.cuda.synchronize(dev)
+    for _ in range(args.warmup):
+        g1.replay()
+    torch.cuda.synchronize(dev)
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        tdist.barrier()
+    sampler = ClockSampler(local_rank) if rank == 0 and not args.no_clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    w0 = time.time()
+    t_start.record(stream)
+    gK.replay()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    clocks = None
+    if sampler:
+        clock_src = "timed region"
+        probe_until = w1
+        if (w1 - w0) < 1.0:
+            # too short for the sampler: replay the same graph for ~1.5 s more
+            # (after the timed region, same load) and take the clocks there
+            clock_src = "replays of the timed graph right after the timed region"
+            pw0 = time.time()
+            while time.time() - pw0 < 1.5:
+                gK.replay()
+                torch.cuda.synchronize(dev)
+            probe_until = time.time()
+            sampler.stop()
+            clocks = sampler.summarise(pw0, probe_until)
+        else:
+            sampler.stop()
+            clocks = sampler.summarise(w0, w1)
+        if clocks is not None:
+            clocks["sampled_during"] = clock_src
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for ev in evs for a, b in zip(ev[0], ev[1]))
+    if dist:
+        t = torch.tensor([elapsed_ms, dec_ms], device=dev, dtype=torch.float64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        elapsed_ms, dec_ms = float(t[0]), float(t[1])
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hk = new_k.cpu().pin_memory()
+        hv = new_v.cpu().pin_memory()
+        hq = qs.cpu().pin_memory()
+        ho = torch.empty(outs.shape, dtype=torch.float32).pin_memory()
+        dk, dv, dq = torch.empty_like(new_k), torch.empty_like(new_v), torch.empty_like(qs)
+        h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
+        d2h = ho.numel() * 4
+
+        def e2e_step():
+            # eager public-API calls, inputs copied in from pinned host memory
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            step(k=dk, v=dv, q=dq)
+            ho.copy_(outs, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if dist:
+            tdist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a.elapsed_time(b)
+        if dist:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": world * B * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    cache.check()
+
+    ms_step = elapsed_ms / args.steps
+    value = world * B * args.steps / (elapsed_ms / 1e3)
+    dec_ms_call = dec_ms / (args.steps * ncalls)
+    achieved = step_decode_bytes * args.steps / (dec_ms / 1e3) / 1e9
+    peak, peak_kind = _peaks()
+    bf16_bytes = None
+    res = {
+        "metric": "decode-attention tokens/s (" + ("BF16 cache" if args.bf16 else "INT4 anchor/INT2 resid") + ")",
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4/int2 codes, fp8 meta, fp32 math" if not args.bf16 else "bf16 in, fp32 math",
+        "data": "synthetic (seeded; anchor N(0,1) with 4 outlier channels x10, loops c*anchor+sigma*N(0,1))",
+        "config": {"workload": name, "layers": layers, "loops": loops, "loops_per_group": Lg, "batch": B,
+                   "seq_len": T, "kv_heads": H, "q_heads": Hq, "head_dim": 128, "group": cfgd["g"],
+                   "anchor_bits": cfgd["ba"], "resid_bits": cfgd["br"], "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: %.1f GB of records read per step, loop-major over %d layers"
+                         % (step_decode_bytes / 1e9, layers)},
+        "decode_attn": {"ms_per_step": round(dec_ms / args.steps, 4), "us_per_call": round(dec_ms_call * 1e3, 3),
+                        "bytes_per_step": int(step_decode_bytes), "gbs": round(achieved, 1),
+                        "tokens_per_s_decode_only": round(world * B * args.steps / (dec_ms / 1e3), 2)},
+        "append": {"ms_per_step": round(ms_step - dec_ms / args.steps, 4)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "rq_decode_attn call (split kernel + combine)", "peak_kind": peak_kind},
+        "e2e": e2e,
+        "gpu_launches": int(args.steps * loops * layers * 3),
+        "clocks": clocks,
+    }
+    return res, cache, call_bytes
+
+
+# ---------------------------------------------------------------- cpu baseline (oracle)
+def oracle_unit_decode_seconds(cfgd, seed, n_units: int, T: int | None = None):
+    """Times the oracle's decode of `n_units` (sequence, kv head) units: for
+    each unit, reconstruct the 4 loops' K/V over T tokens from its records and
+    run the direct fp64 softmax for each loop's query.  Returns (seconds per
+    unit-step, description).  Records are produced by the oracle's own
+    encoder from CPU-generated synthetic inputs (untimed)."""
+    import torch
+    from decode_attention_14_b200 import synth
+    from oracle import oracle as orc
+
+    T = T or cfgd["T"]
+    Lg, g, ba, br = cfgd["Lg"], cfgd["g"], cfgd["ba"], cfgd["br"]
+    total = 0.0
+    for u in range(n_units):
+        Kg, Vg = synth.group_kv(seed + u, 0, 0, Lg, cfgd["sigma"], 1, T, 1, device="cpu")
+        recs = []
+        for X in (Kg, Vg):
+            x = np.stack([synth.bf16_to_u16(X[j]).reshape(-1, 128) for j in range(Lg)])
+            recs.append(orc.encode(x, g, ba, br, True, 0xA11CE))
+        q = torch.randn((1, 1, 128)).to(torch.bfloat16)
+        qf = orc.bf16_bits_to_f64(synth.bf16_to_u16(q))
+        t0 = time.perf_counter()
+        kvhat = [orc.reconstruct(e.a_codes, e.a_meta, e.r_codes, e.r_meta, e.r_coef, Lg, 128, g, ba, br, True, 0xA11CE)
+                 for e in recs]
+        for j in range(Lg):
+            orc.attention(qf, kvhat[0][j][None, :, None, :], kvhat[1][j][None, :, None, :], 1 / math.sqrt(128))
+        total += time.perf_counter() - t0
+    return total / n_units
+
+
+def cpu_baseline(cfgd, seed, budget_s: float = 15.0):
+    # one unit at full T to size the sample, then as many as fit the budget
+    per_unit = oracle_unit_decode_seconds(cfgd, seed, 1)
+    n = int(max(1, min(8, budget_s // max(per_unit, 1e-3) - 1)))
+    if n > 1:
+        per_unit = oracle_unit_decode_seconds(cfgd, seed + 7, n)
+    units_per_step = cfgd["layers"] * (cfgd["loops"] // cfgd["Lg"]) * cfgd["B"] * cfgd["H"]
+    step_s = per_unit * units_per_step
+    return {"value": round(cfgd["B"] / step_s, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} (sequence, kv head) unit(s) x {cfgd['loops']} loops at T={cfgd['T']} "
+                      f"(reconstruct + fp64 softmax), {per_unit:.2f} s/unit, scaled to "
+                      f"{units_per_step} units per step (extrapolated)"}
+
+
+def run_reference(args, cfgd):
+    """The oracle, timed as it stands on the host cores: each step a bounded
+    sample (one (sequence, kv head) unit of one layer group), scaled to the
+    workload's metric."""
+    seed = CONFIG_SEED[args.config]
+    for w in range(args.warmup):
+        oracle_unit_decode_seconds(cfgd, seed + 100 + w, 1, T=min(cfgd["T"], 1024))
+    per = [oracle_unit_decode_seconds(cfgd, seed + s, 1) for s in range(args.steps)]
+    per_unit = float(np.mean(per))
+    units_per_step = cfgd["layers"] * (cfgd["loops"] // cfgd["Lg"]) * cfgd["B"] * cfgd["H"]
+    step_s = per_unit * units_per_step
+    value = cfgd["B"] / step_s
+    sample = (f"1 (sequence, kv head) unit x {cfgd['loops']} loops at T={cfgd['T']} per step "
+              f"(oracle reconstruct + fp64 softmax), scaled to {units_per_step} units per decode step")
+    return {
+        "impl": "reference",
+        "metric": "decode-attention tokens/s (INT4 anchor/INT2 resid)",
+        "value": round(value, 6), "unit": "tokens/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
+        "config": {"workload": args.config, "layers": cfgd["layers"], "loops": cfgd["loops"], "batch": cfgd["B"],
+                   "seq_len": cfgd["T"], "kv_heads": cfgd["H"], "q_heads": cfgd["Hq"], "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="ouro8k_b4", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--bf16", action="store_true", help="time the uncompressed BF16 comparison kernel")
+    ap.add_argument("--layers", type=int, default=0, help="override layer count (profiling runs only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--json-out", default="")
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.layers:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    cfgd = CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            res = run_reference(args, cfgd)
+            print(json.dumps(res))
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    res, cache, _ = run_ours(args, cfgd, rank, world, local_rank)
+    if rank == 0 and not args.no_cpu_baseline and not args.layers:
+        res["cpu_baseline"] = cpu_baseline(cfgd, CONFIG_SEED[args.config])
+    if rank == 0:
+        line = json.dumps(res)
+        print(line)
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(line + "\n")
+    cache.close()
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,523 @@
+// api.cpp -- the C ABI declared in include/rq.h: argument validation, the
+// cache's host-side state (committed lengths, tail counts), arena layout and
+// kernel launches.  Every arithmetic step of the method runs in the CUDA
+// kernels; this file only moves pointers and sizes around.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "rq_internal.h"
+
+using namespace rq;
+
+struct rq_cache {
+    Layout lay;
+    uint8_t *base = nullptr;
+    bool owned = false;
+    int device = 0;
+    int sms = 148;
+    std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]
+    std::vector<int> ntail;   // [layer][loop]
+    uint32_t sigma[4] = {0, 0, 0, 0};
+};
+
+namespace {
+
+// splitmix64 (Steele, Lea & Flood, OOPSLA 2014): golden-gamma increment and
+// the 30/27/31 xor-shift-multiply finaliser.
+uint64_t splitmix64(uint64_t x) {
+    uint64_t z = x + 0x9E3779B97F4A7C15ULL;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+bool is_anchor_loop(const Layout &L, int loop) { return (loop % L.Lg) == L.Lg - 1; }
+
+uint8_t *group_base(const rq_cache *c, int layer, int group) {
+    const Layout &L = c->lay;
+    return c->base + L.off_records + ((size_t)layer * L.groups + group) * L.group_block;
+}
+
+uint8_t *anchor_codes(const rq_cache *c, int layer, int group, int kv) {
+    const Layout &L = c->lay;
+    return group_base(c, layer, group) + kv * (L.anchor_codes_bytes + L.anchor_meta_bytes);
+}
+uint8_t *anchor_meta(const rq_cache *c, int layer, int group, int kv) {
+    return anchor_codes(c, layer, group, kv) + c->lay.anchor_codes_bytes;
+}
+size_t resid_side(const Layout &L) { return L.resid_codes_bytes + L.resid_meta_bytes + L.resid_coef_bytes; }
+uint8_t *resid_codes(const rq_cache *c, int layer, int group, int j, int kv) {
+    const Layout &L = c->lay;
+    return group_base(c, layer, group) + L.anchor_block + (size_t)j * L.resid_block + kv * resid_side(L);
+}
+uint8_t *resid_meta(const rq_cache *c, int layer, int group, int j, int kv) {
+    return resid_codes(c, layer, group, j, kv) + c->lay.resid_codes_bytes;
+}
+uint8_t *resid_coef(const rq_cache *c, int layer, int group, int j, int kv) {
+    return resid_meta(c, layer, group, j, kv) + c->lay.resid_meta_bytes;
+}
+uint8_t *tail_ptr(const rq_cache *c, int layer, int group, int j, int kv) {
+    const Layout &L = c->lay;
+    return group_base(c, layer, group) + L.anchor_block + (size_t)(L.Lg - 1) * L.resid_block +
+           (size_t)j * L.tail_block + kv * L.tail_bytes;
+}
+uint16_t *bf16_ptr(const rq_cache *c, int layer, int loop, int kv) {
+    const Layout &L = c->lay;
+    return (uint16_t *)(c->base + L.off_records + ((size_t)layer * L.cfg.num_loops + loop) * L.bf16_block +
+                        kv * L.bf16_side);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt((float)kHeadDim); }
+
+// Split-KV partition: enough CTAs to cover the SMs a few times over, chunks
+// that are a multiple of 16 tokens.
+void choose_splits(const rq_cache *c, int T, int units, int *S, int *chunk) {
+    if (T <= 0) {
+        *S = 0;
+        *chunk = 16;
+        return;
+    }
+    int target = c->sms * 4;
+    int s = (target + units - 1) / units;
+    int smax = std::min(c->lay.splits_max, (T + 63) / 64);
+    s = std::max(1, std::min(s, smax));
+    s = std::max(s, (T + kMaxChunk - 1) / kMaxChunk);   // bounded per-CTA logit buffer
+    int ch = (T + s - 1) / s;
+    ch = (ch + 15) / 16 * 16;
+    *chunk = ch;
+    *S = (T + ch - 1) / ch;
+}
+
+}  // namespace
+
+namespace rq {
+
+bool make_layout(const rq_config &cfg, Layout *out) {
+    Layout L;
+    std::memset(&L, 0, sizeof(L));
+    L.cfg = cfg;
+    const size_t B = cfg.batch, H = cfg.num_kv_heads, Hq = cfg.num_q_heads;
+    if (cfg.format == RQ_FMT_RESIDUAL) {
+        L.rec.a_codes = kHeadDim * cfg.anchor_bits / 8;
+        L.rec.r_codes = kHeadDim * cfg.resid_bits / 8;
+        L.rec.meta = (kHeadDim / cfg.group_size) * 2;
+    }
+    L.Lg = cfg.loops_per_group;
+    L.groups = cfg.num_loops / cfg.loops_per_group;
+    L.Tp = (int)align_up((size_t)cfg.max_tokens, kTokTile);
+    L.tail_cap = cfg.max_tail_tokens;
+    L.splits_max = std::min(kMaxSplits, L.Tp / kTokTile);
+    const size_t bht = B * H * (size_t)L.Tp;
+    if (cfg.format == RQ_FMT_RESIDUAL) {
+        L.anchor_codes_bytes = align_up(bht * L.rec.a_codes, kAlign);
+        L.anchor_meta_bytes = align_up(bht * L.rec.meta, kAlign);
+        L.anchor_block = 2 * (L.anchor_codes_bytes + L.anchor_meta_bytes);
+        L.resid_codes_bytes = align_up(bht * L.rec.r_codes, kAlign);
+        L.resid_meta_bytes = align_up(bht * L.rec.meta, kAlign);
+        L.resid_coef_bytes = align_up(bht * 2, kAlign);
+        L.resid_block = 2 * (L.resid_codes_bytes + L.resid_meta_bytes + L.resid_coef_bytes);
+        L.tail_bytes = align_up(B * (size_t)L.tail_cap * H * kHeadDim * 2, kAlign);
+        L.tail_block = 2 * L.tail_bytes;
+        L.group_block = L.anchor_block + (size_t)(L.Lg - 1) * (L.resid_block + L.tail_block);
+        L.records_bytes = (size_t)cfg.num_layers * L.groups * L.group_block;
+    } else {
+        L.bf16_side = align_up(bht * kHeadDim * 2, kAlign);
+        L.bf16_block = 2 * L.bf16_side;
+        L.records_bytes = (size_t)cfg.num_layers * cfg.num_loops * L.bf16_block;
+    }
+    L.off_records = 0;
+    L.off_partials = align_up(L.records_bytes, kAlign);
+    size_t partial_bytes = align_up(B * Hq * (size_t)L.splits_max * kPartialStride * sizeof(float), kAlign);
+    L.off_counters = L.off_partials + partial_bytes;
+    L.off_err = L.off_counters + align_up(B * H * sizeof(int), kAlign);
+    L.total = L.off_err + kAlign;
+    *out = L;
+    return true;
+}
+
+}  // namespace rq
+
+extern "C" {
+
+const char *rq_status_string(int status) {
+    switch (status) {
+    case RQ_OK: return "ok";
+    case RQ_ERR_INVALID: return "invalid argument";
+    case RQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RQ_ERR_NOMEM: return "out of memory / arena too small";
+    case RQ_ERR_CAPACITY: return "capacity exceeded";
+    case RQ_ERR_STATE: return "call out of order / wrong cache format";
+    case RQ_ERR_CUDA: return "CUDA error";
+    case RQ_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int rq_config_check(const rq_config *c) {
+    if (!c) return RQ_ERR_INVALID;
+    if (c->num_layers < 1 || c->num_loops < 1 || c->loops_per_group < 1 || c->batch < 1 ||
+        c->max_tokens < 1 || c->max_tail_tokens < 0 || c->num_kv_heads < 1 || c->num_q_heads < 1)
+        return RQ_ERR_INVALID;
+    if (c->num_loops % c->loops_per_group != 0) return RQ_ERR_INVALID;
+    if (c->num_q_heads % c->num_kv_heads != 0) return RQ_ERR_INVALID;
+    if (c->format != RQ_FMT_RESIDUAL && c->format != RQ_FMT_BF16) return RQ_ERR_INVALID;
+    if (c->rotate != 0 && c->rotate != 1) return RQ_ERR_INVALID;
+    int G = c->num_q_heads / c->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return RQ_ERR_UNSUPPORTED;
+    if (c->head_dim != kHeadDim) return RQ_ERR_UNSUPPORTED;
+    if (c->format == RQ_FMT_RESIDUAL) {
+        if (c->group_size != 16 && c->group_size != 32) return RQ_ERR_UNSUPPORTED;
+        if (c->anchor_bits != 2 && c->anchor_bits != 4) return RQ_ERR_UNSUPPORTED;
+        if (c->resid_bits != 2 && c->resid_bits != 4) return RQ_ERR_UNSUPPORTED;
+        if (c->loops_per_group > 1 && c->max_tail_tokens < 1) return RQ_ERR_INVALID;
+    }
+    // size sanity: every per-stream offset must fit the kernels' 64-bit math
+    // and the token index the kernels' 32-bit math
+    if (c->max_tokens > (1 << 20) || c->max_tail_tokens > (1 << 20)) return RQ_ERR_UNSUPPORTED;
+    return RQ_OK;
+}
+
+size_t rq_cache_required_bytes(const rq_config *cfg) {
+    if (rq_config_check(cfg) != RQ_OK) return 0;
+    Layout L;
+    make_layout(*cfg, &L);
+    return L.total;
+}
+
+size_t rq_cache_token_bytes(const rq_config *c) {
+    if (rq_config_check(c) != RQ_OK) return 0;
+    const size_t heads = (size_t)c->num_kv_heads, layers = (size_t)c->num_layers;
+    if (c->format == RQ_FMT_BF16)
+        return layers * c->num_loops * heads * 2 * kHeadDim * 2;
+    const size_t meta = (kHeadDim / c->group_size) * 2;
+    const size_t a = kHeadDim * c->anchor_bits / 8 + meta;
+    const size_t r = kHeadDim * c->resid_bits / 8 + meta + 2;
+    const size_t groups = c->num_loops / c->loops_per_group;
+    return layers * heads * 2 * groups * (a + (size_t)(c->loops_per_group - 1) * r);
+}
+
+int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache **out) {
+    if (!out) return RQ_ERR_INVALID;
+    *out = nullptr;
+    int st = rq_config_check(cfg);
+    if (st != RQ_OK) return st;
+    rq_cache *c = new (std::nothrow) rq_cache();
+    if (!c) return RQ_ERR_NOMEM;
+    make_layout(*cfg, &c->lay);
+    if (cudaGetDevice(&c->device) != cudaSuccess) {
+        delete c;
+        return RQ_ERR_CUDA;
+    }
+    cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device);
+    if (dev_mem) {
+        if (bytes < c->lay.total || ((uintptr_t)dev_mem % kAlign) != 0) {
+            delete c;
+            return RQ_ERR_NOMEM;
+        }
+        c->base = (uint8_t *)dev_mem;
+        c->owned = false;
+    } else {
+        void *p = nullptr;
+        if (cudaMalloc(&p, c->lay.total) != cudaSuccess) {
+            cudaGetLastError();
+            delete c;
+            return RQ_ERR_NOMEM;
+        }
+        c->base = (uint8_t *)p;
+        c->owned = true;
+    }
+    if (cudaMemset(c->base, 0, c->lay.total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        if (c->owned) cudaFree(c->base);
+        delete c;
+        return RQ_ERR_CUDA;
+    }
+    const Layout &L = c->lay;
+    c->len.assign((size_t)cfg->num_layers * (cfg->format == RQ_FMT_RESIDUAL ? L.groups : cfg->num_loops), 0);
+    c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
+    if (cfg->rotate)
+        for (int j = 0; j < kHeadDim; j++)
+            if (splitmix64(cfg->seed + (uint64_t)j) >> 63) c->sigma[j / 32] |= 1u << (j % 32);
+    *out = c;
+    return RQ_OK;
+}
+
+int rq_cache_destroy(rq_cache *c) {
+    if (!c) return RQ_OK;
+    int st = RQ_OK;
+    if (c->owned) {
+        if (cudaDeviceSynchronize() != cudaSuccess) st = RQ_ERR_CUDA;
+        cudaFree(c->base);
+    }
+    delete c;
+    return st;
+}
+
+int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, int n, void *stream) {
+    if (!c || !k || !v || n < 1) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cfg.format == RQ_FMT_BF16) {
+        int &len = c->len[(size_t)layer * cfg.num_loops + loop];
+        if (len + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
+        Bf16StoreArgs a;
+        a.src[0] = (const uint16_t *)k;
+        a.src[1] = (const uint16_t *)v;
+        a.dst[0] = bf16_ptr(c, layer, loop, 0);
+        a.dst[1] = bf16_ptr(c, layer, loop, 1);
+        a.B = cfg.batch;
+        a.H = cfg.num_kv_heads;
+        a.n = n;
+        a.pos0 = len;
+        a.Tp = L.Tp;
+        int s = cuda_status(launch_bf16_store(a, st));
+        if (s == RQ_OK) len += n;
+        return s;
+    }
+    const int group = loop / L.Lg, j = loop % L.Lg;
+    int &len = c->len[(size_t)layer * L.groups + group];
+    if (!is_anchor_loop(L, loop)) {
+        int &nt = c->ntail[(size_t)layer * cfg.num_loops + loop];
+        if (nt + n > L.tail_cap) return RQ_ERR_CAPACITY;
+        TailArgs a;
+        a.src[0] = (const uint16_t *)k;
+        a.src[1] = (const uint16_t *)v;
+        a.dst[0] = (uint16_t *)tail_ptr(c, layer, group, j, 0);
+        a.dst[1] = (uint16_t *)tail_ptr(c, layer, group, j, 1);
+        a.B = cfg.batch;
+        a.H = cfg.num_kv_heads;
+        a.n = n;
+        a.pos0 = nt;
+        a.cap = L.tail_cap;
+        int s = cuda_status(launch_tail_copy(a, st));
+        if (s == RQ_OK) nt += n;
+        return s;
+    }
+    // anchor loop: every other loop of the group must hold exactly these n tokens
+    for (int jj = 0; jj < L.Lg - 1; jj++)
+        if (c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] != n) return RQ_ERR_STATE;
+    if (len + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
+    AppendArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.x_anchor[0] = (const uint16_t *)k;
+    a.x_anchor[1] = (const uint16_t *)v;
+    a.nres = L.Lg - 1;
+    if (a.nres > 0) {
+        a.tail0 = tail_ptr(c, layer, group, 0, 0);
+        a.tail_loop_stride = L.tail_block;
+        a.tail_kv_stride = L.tail_bytes;
+        a.r_codes0 = resid_codes(c, layer, group, 0, 0);
+        a.r_meta0 = resid_meta(c, layer, group, 0, 0);
+        a.r_coef0 = resid_coef(c, layer, group, 0, 0);
+        a.resid_loop_stride = L.resid_block;
+        a.resid_kv_stride = resid_side(L);
+    }
+    a.a_codes0 = anchor_codes(c, layer, group, 0);
+    a.a_meta0 = anchor_meta(c, layer, group, 0);
+    a.anchor_kv_stride = L.anchor_codes_bytes + L.anchor_meta_bytes;
+    a.B = cfg.batch;
+    a.H = cfg.num_kv_heads;
+    a.n = n;
+    a.pos0 = len;
+    a.Tp = L.Tp;
+    a.tail_cap = L.tail_cap;
+    a.g = cfg.group_size;
+    a.ba = cfg.anchor_bits;
+    a.br = cfg.resid_bits;
+    a.rotate = cfg.rotate;
+    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    int s = cuda_status(launch_append(a, st));
+    if (s != RQ_OK) return s;
+    len += n;
+    for (int jj = 0; jj < L.Lg - 1; jj++) c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] = 0;
+    return RQ_OK;
+}
+
+static int decode_common(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
+                         void *stream, bool bf16) {
+    if (!c || !q || !out) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
+    if ((cfg.format == RQ_FMT_BF16) != bf16) return RQ_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const uint16_t *)q;
+    a.partials = (float *)(c->base + L.off_partials);
+    a.B = cfg.batch;
+    a.H = cfg.num_kv_heads;
+    a.Hq = cfg.num_q_heads;
+    a.G = cfg.num_q_heads / cfg.num_kv_heads;
+    a.Tp = L.Tp;
+    a.splits_max = L.splits_max;
+    a.g = cfg.group_size;
+    a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
+    a.rotate = cfg.rotate;
+    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    CombineArgs cb;
+    std::memset(&cb, 0, sizeof(cb));
+    int n_tail = 0;
+    bool resid = false;
+    if (bf16) {
+        a.T = c->len[(size_t)layer * cfg.num_loops + loop];
+        a.bf[0] = bf16_ptr(c, layer, loop, 0);
+        a.bf[1] = bf16_ptr(c, layer, loop, 1);
+    } else {
+        const int group = loop / L.Lg, j = loop % L.Lg;
+        a.T = c->len[(size_t)layer * L.groups + group];
+        for (int kv = 0; kv < 2; kv++) {
+            a.a_codes[kv] = anchor_codes(c, layer, group, kv);
+            a.a_meta[kv] = anchor_meta(c, layer, group, kv);
+        }
+        if (!is_anchor_loop(L, loop)) {
+            resid = true;
+            for (int kv = 0; kv < 2; kv++) {
+                a.r_codes[kv] = resid_codes(c, layer, group, j, kv);
+                a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
+                a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, j, kv);
+            }
+            n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
+            cb.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
+            cb.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
+        }
+    }
+    const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
+    choose_splits(c, a.T, units, &a.S, &a.chunk);
+    if (a.S > 0) {
+        cudaError_t e = bf16 ? launch_decode_bf16(a, st)
+                             : launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st);
+        if (e != cudaSuccess) return RQ_ERR_CUDA;
+    }
+    cb.partials = a.partials;
+    cb.q = a.q;
+    cb.out = out;
+    cb.B = a.B;
+    cb.H = a.H;
+    cb.Hq = a.Hq;
+    cb.G = a.G;
+    cb.S = a.S;
+    cb.splits_max = a.splits_max;
+    cb.n_tail = n_tail;
+    cb.tail_cap = L.tail_cap;
+    cb.scale_log2 = a.scale_log2;
+    return cuda_status(launch_combine(cb, st));
+}
+
+int rq_decode_attn(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream) {
+    return decode_common(c, layer, loop, q, out, scale, stream, false);
+}
+
+int rq_decode_attn_bf16(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
+                        void *stream) {
+    return decode_common(c, layer, loop, q, out, scale, stream, true);
+}
+
+int rq_cache_length(const rq_cache *c, int layer, int group, int *len) {
+    if (!c || !len) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    int ngroups = L.cfg.format == RQ_FMT_RESIDUAL ? L.groups : L.cfg.num_loops;
+    if (layer < 0 || layer >= L.cfg.num_layers || group < 0 || group >= ngroups) return RQ_ERR_INVALID;
+    *len = c->len[(size_t)layer * ngroups + group];
+    return RQ_OK;
+}
+
+int rq_cache_tail_length(const rq_cache *c, int layer, int loop, int *n) {
+    if (!c || !n) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    if (layer < 0 || layer >= L.cfg.num_layers || loop < 0 || loop >= L.cfg.num_loops) return RQ_ERR_INVALID;
+    *n = c->ntail[(size_t)layer * L.cfg.num_loops + loop];
+    return RQ_OK;
+}
+
+int rq_cache_truncate(rq_cache *c, int layer, int group, int new_len) {
+    if (!c) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    int ngroups = L.cfg.format == RQ_FMT_RESIDUAL ? L.groups : L.cfg.num_loops;
+    if (layer < 0 || layer >= L.cfg.num_layers || group < 0 || group >= ngroups) return RQ_ERR_INVALID;
+    int &len = c->len[(size_t)layer * ngroups + group];
+    if (new_len < 0 || new_len > len) return RQ_ERR_INVALID;
+    if (L.cfg.format == RQ_FMT_RESIDUAL)
+        for (int jj = 0; jj < L.Lg - 1; jj++)
+            if (c->ntail[(size_t)layer * L.cfg.num_loops + group * L.Lg + jj] != 0) return RQ_ERR_STATE;
+    len = new_len;
+    return RQ_OK;
+}
+
+int rq_cache_export(const rq_cache *c, int layer, int loop, void *host_codes, void *host_meta, void *host_coef,
+                    void *stream) {
+    if (!c || !host_codes || !host_meta) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
+    if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
+    const int group = loop / L.Lg, j = loop % L.Lg;
+    const bool anchor = is_anchor_loop(L, loop);
+    if (!anchor && !host_coef) return RQ_ERR_INVALID;
+    const int len = c->len[(size_t)layer * L.groups + group];
+    const size_t bh = (size_t)cfg.batch * cfg.num_kv_heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (len == 0) return RQ_OK;
+    const size_t crec = anchor ? L.rec.a_codes : L.rec.r_codes;
+    for (int kv = 0; kv < 2; kv++) {
+        const uint8_t *codes = anchor ? anchor_codes(c, layer, group, kv) : resid_codes(c, layer, group, j, kv);
+        const uint8_t *meta = anchor ? anchor_meta(c, layer, group, kv) : resid_meta(c, layer, group, j, kv);
+        uint8_t *hc = (uint8_t *)host_codes + kv * bh * len * crec;
+        uint8_t *hm = (uint8_t *)host_meta + kv * bh * len * L.rec.meta;
+        cudaError_t e = cudaMemcpy2DAsync(hc, len * crec, codes, (size_t)L.Tp * crec, len * crec, bh,
+                                          cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(hm, len * (size_t)L.rec.meta, meta, (size_t)L.Tp * L.rec.meta,
+                                  len * (size_t)L.rec.meta, bh, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess && !anchor) {
+            uint8_t *hf = (uint8_t *)host_coef + kv * bh * len * 2;
+            e = cudaMemcpy2DAsync(hf, len * 2, resid_coef(c, layer, group, j, kv), (size_t)L.Tp * 2, len * 2, bh,
+                                  cudaMemcpyDeviceToHost, st);
+        }
+        if (e != cudaSuccess) return RQ_ERR_CUDA;
+    }
+    return cuda_status(cudaStreamSynchronize(st));
+}
+
+size_t rq_decode_bytes(const rq_cache *c, int layer, int loop) {
+    if (!c) return 0;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return 0;
+    const size_t bh = (size_t)cfg.batch * cfg.num_kv_heads;
+    const size_t qo = (size_t)cfg.batch * cfg.num_q_heads * kHeadDim * (2 + 4);
+    if (cfg.format == RQ_FMT_BF16) {
+        const size_t T = c->len[(size_t)layer * cfg.num_loops + loop];
+        return T * bh * 2 * kHeadDim * 2 + qo;
+    }
+    const int group = loop / L.Lg;
+    const size_t T = c->len[(size_t)layer * L.groups + group];
+    size_t per = 2 * (size_t)(L.rec.a_codes + L.rec.meta);
+    size_t tail = 0;
+    if (!is_anchor_loop(L, loop)) {
+        per += 2 * (size_t)(L.rec.r_codes + L.rec.meta + 2);
+        tail = (size_t)c->ntail[(size_t)layer * cfg.num_loops + loop] * bh * 2 * kHeadDim * 2;
+    }
+    return T * bh * per + tail + qo;
+}
+
+int rq_check(rq_cache *c) {
+    if (!c) return RQ_ERR_INVALID;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
+    int err = 0;
+    if (cudaMemcpy(&err, c->base + c->lay.off_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RQ_ERR_CUDA;
+    if (err != 0) {
+        int zero = 0;
+        cudaMemcpy(c->base + c->lay.off_err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return RQ_ERR_TIMEOUT;
+    }
+    return RQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,131 @@
+// rq_internal.h -- layout of the cache arena and the launch interface shared
+// by the host API (api.cpp) and the CUDA kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/rq.h"
+
+namespace rq {
+
+constexpr int kHeadDim = 128;
+constexpr int kTokTile = 64;        // padding granule of every token stream
+constexpr int kMaxSplits = 256;     // split-KV partitions per (b, kv head)
+constexpr int kMaxChunk = 4096;     // tokens per CTA (bounds the logit buffer)
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Byte sizes of one record (one token-head, K or V).
+struct RecordSizes {
+    int a_codes;   // anchor codes: d * anchor_bits / 8
+    int r_codes;   // residual codes: d * resid_bits / 8
+    int meta;      // (d / g) * 2: [scale e4m3, min e4m3] per group
+};
+
+// Where every array of the arena lives.  All token streams are laid out
+// [B][H_kv][Tp][record] so that the records of one (sequence, head) are one
+// contiguous, 16-byte-aligned run of Tp records (Tp = max_tokens rounded up
+// to kTokTile).
+struct Layout {
+    rq_config cfg;
+    RecordSizes rec;
+    int groups;          // anchor groups per layer = num_loops / loops_per_group
+    int Lg;              // loops per group
+    int Tp;              // padded token capacity of a stream
+    int tail_cap;        // max_tail_tokens
+    int splits_max;      // partial slots per (b, q head)
+    // residual format: per (layer, group)
+    size_t anchor_codes_bytes;   // one kv side: B*H*Tp*a_codes
+    size_t anchor_meta_bytes;    // one kv side: B*H*Tp*meta
+    size_t anchor_block;         // both kv sides, aligned
+    size_t resid_codes_bytes, resid_meta_bytes, resid_coef_bytes;
+    size_t resid_block;          // one non-anchor loop, both kv sides
+    size_t tail_bytes;           // one kv side of one loop: B*tail_cap*H*d*2
+    size_t tail_block;           // one non-anchor loop, both kv sides
+    size_t group_block;          // anchor + (Lg-1) residual + (Lg-1) tail blocks
+    // BF16 format: per (layer, loop)
+    size_t bf16_side;            // B*H*Tp*d*2
+    size_t bf16_block;           // both kv sides
+    // workspace
+    size_t off_records;          // start of the record area (0)
+    size_t records_bytes;
+    size_t off_partials;         // float [B][Hq][splits_max][kPartialStride]
+    size_t off_counters;         // int [B][H_kv]
+    size_t off_err;              // int error word (+ pad)
+    size_t total;
+};
+
+constexpr int kPartialStride = kHeadDim + 4;   // o[128], m, l, pad, pad
+
+bool make_layout(const rq_config &cfg, Layout *out);
+
+// --------------------------------------------------------------- kernels
+struct AppendArgs {
+    // inputs: anchor-loop K/V (kv = 0 K, 1 V), [B][n][H][d] bf16
+    const uint16_t *x_anchor[2];
+    // tails of the non-anchor loops of the group: tail(kv, j) = tail0 +
+    // j*tail_loop_stride + kv*tail_kv_stride (bytes); layout [B][cap][H][d]
+    const uint8_t *tail0;
+    size_t tail_loop_stride, tail_kv_stride;
+    // anchor records: codes/meta of side kv at anchor0 + kv*anchor_kv_stride
+    uint8_t *a_codes0, *a_meta0;
+    size_t anchor_kv_stride;
+    // residual records of loop j: r_*0 + j*resid_loop_stride + kv*resid_kv_stride
+    uint8_t *r_codes0, *r_meta0, *r_coef0;
+    size_t resid_loop_stride, resid_kv_stride;
+    int B, H, n, pos0, Tp, tail_cap, nres;   // nres = Lg - 1
+    int g, ba, br, rotate;
+    uint32_t sigma[4];
+};
+
+struct TailArgs {
+    const uint16_t *src[2];   // [B][n][H][d]
+    uint16_t *dst[2];         // [B][cap][H][d]
+    int B, H, n, pos0, cap;
+};
+
+struct Bf16StoreArgs {
+    const uint16_t *src[2];   // [B][n][H][d]
+    uint16_t *dst[2];         // [B][H][Tp][d]
+    int B, H, n, pos0, Tp;
+};
+
+struct DecodeArgs {
+    // anchor streams (kv 0 = K, 1 = V)
+    const uint8_t *a_codes[2], *a_meta[2];
+    // residual streams (null for the anchor loop)
+    const uint8_t *r_codes[2], *r_meta[2];
+    const uint16_t *r_coef[2];
+    // BF16 format streams
+    const uint16_t *bf[2];
+    const uint16_t *q;        // [B][Hq][d] bf16
+    float *partials;          // [B][Hq][splits_max][kPartialStride]
+    int B, H, Hq, G, T, Tp, S, chunk, splits_max;
+    int g;
+    float scale_log2;         // softmax_scale * log2(e)
+    int rotate;
+    uint32_t sigma[4];
+};
+
+struct CombineArgs {
+    const float *partials;
+    const uint16_t *q;
+    const uint16_t *tail_k, *tail_v;   // [B][cap][H][d] or null
+    float *out;               // [B][Hq][d]
+    int B, H, Hq, G, S, splits_max, n_tail, tail_cap;
+    float scale_log2;
+};
+
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t st);
+cudaError_t launch_tail_copy(const TailArgs &a, cudaStream_t st);
+cudaError_t launch_bf16_store(const Bf16StoreArgs &a, cudaStream_t st);
+cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st);
+cudaError_t launch_decode_bf16(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
+
+}  // namespace rq

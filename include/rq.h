@@ -1,0 +1,214 @@
+/*
+ * rq.h -- C ABI of the B200 (sm_100a) ResidualQuant decode-attention library.
+ *
+ * Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
+ * 2-Bit Residuals" (arXiv 2610.10381; abstract, and the ai4snews summary,
+ * paragraphs 1-4).  A looped Transformer produces its own K/V per (layer,
+ * loop); the cache keeps the final loop of each loop group as an INT4
+ * "anchor" and every other loop as a BF16 least-squares coefficient plus an
+ * INT2 residual of the rotated difference, so that
+ *     K_l ~= s_l * a_hat + R^T r_hat          (two cache reads per loop)
+ * Decode attention returns softmax(q K^T * scale) V over that cache.
+ *
+ * Conventions shared by every call:
+ *   - All device pointers are CUDA global-memory pointers of the current
+ *     device.  "stream" is a cudaStream_t passed as void* (NULL = the legacy
+ *     default stream).  Work is enqueued asynchronously; no call
+ *     synchronises the host except rq_cache_create/destroy and
+ *     rq_cache_export (which copies to host memory).
+ *   - BF16 arrays hold IEEE bfloat16 bit patterns (uint16).
+ *   - Calls return an rq_status (0 = RQ_OK, negative = error) and never
+ *     throw; a failing call leaves the cache state unchanged.
+ *   - Calls that touch one cache must not run concurrently with each other
+ *     (the cache owns one split-combine workspace); enqueue them on one
+ *     stream, or order the streams.
+ *   - Ownership: the caller owns q, k, v, out and (optionally) the cache's
+ *     device arena; the library owns the host-side handle and, when it
+ *     allocated the arena itself, the arena.
+ */
+#ifndef RQ_H
+#define RQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RQ_OK = 0,
+    RQ_ERR_INVALID = -1,      /* bad argument (null pointer, index out of range, ...) */
+    RQ_ERR_UNSUPPORTED = -2,  /* configuration outside what the kernels implement */
+    RQ_ERR_NOMEM = -3,        /* caller arena too small, or device allocation failed */
+    RQ_ERR_CAPACITY = -4,     /* append would exceed max_tokens / max_tail_tokens */
+    RQ_ERR_STATE = -5,        /* call out of order (e.g. anchor append before its loops) */
+    RQ_ERR_CUDA = -6,         /* a CUDA runtime call failed (sticky errors included) */
+    RQ_ERR_TIMEOUT = -7       /* a device-side bounded wait gave up (see rq_check) */
+} rq_status;
+
+typedef enum {
+    RQ_FMT_RESIDUAL = 0,      /* INT anchor + INT residuals (the compressed cache) */
+    RQ_FMT_BF16 = 1           /* every loop stored uncompressed in BF16 (comparison) */
+} rq_format;
+
+/*
+ * Cache shape and format.
+ *   num_layers       layers sharing the cache object
+ *   num_loops        recurrent loops per layer (Ouro-1.4B: 4; Huginn: 32)
+ *   loops_per_group  loops per anchor group; the anchor is the LAST loop of
+ *                    each group (Ouro 4/4; Huginn-style 32 loops in 8 groups
+ *                    of 4, per the ai4snews summary, paragraph 1).
+ *                    num_loops % loops_per_group == 0.
+ *   batch            sequences B; every sequence has the same length
+ *   max_tokens       committed-token capacity per (layer, group)
+ *   max_tail_tokens  in-flight tokens a non-anchor loop may hold before the
+ *                    group's anchor commits them
+ *   num_kv_heads     H_kv
+ *   num_q_heads      H_q; H_q % H_kv == 0 and H_q/H_kv in {1,2,4,8};
+ *                    query head h reads kv head h / (H_q/H_kv)
+ *   head_dim         d; must be 128
+ *   group_size       g in {16, 32}: quantization groups along head_dim, each
+ *                    with an FP8-E4M3 scale and an FP8-E4M3 minimum
+ *   anchor_bits      {4, 2};  resid_bits {2, 4}
+ *   rotate           1: residuals rotated by R = H_d diag(sigma)/sqrt(d)
+ *                    (Sylvester Hadamard; sigma_j = -1 iff the top bit of
+ *                    splitmix64(seed + j) is set); 0: R = I
+ *   format           rq_format
+ *   seed             rotation seed (one rotation per cache, shared by K and
+ *                    V, all layers and loops)
+ */
+typedef struct rq_config {
+    int32_t num_layers;
+    int32_t num_loops;
+    int32_t loops_per_group;
+    int32_t batch;
+    int32_t max_tokens;
+    int32_t max_tail_tokens;
+    int32_t num_kv_heads;
+    int32_t num_q_heads;
+    int32_t head_dim;
+    int32_t group_size;
+    int32_t anchor_bits;
+    int32_t resid_bits;
+    int32_t rotate;
+    int32_t format;
+    uint64_t seed;
+} rq_config;
+
+typedef struct rq_cache rq_cache;
+
+/* Human-readable name of a status code (static string). */
+const char *rq_status_string(int status);
+
+/* Validates cfg.  RQ_OK, RQ_ERR_INVALID or RQ_ERR_UNSUPPORTED. */
+int rq_config_check(const rq_config *cfg);
+
+/* Device bytes rq_cache_create needs for cfg (records, BF16 tails, split
+ * workspace, alignment padding); 0 if cfg is invalid. */
+size_t rq_cache_required_bytes(const rq_config *cfg);
+
+/* Committed storage per token: bytes of all records one token occupies over
+ * all layers, loops, heads, K and V (codes + FP8 scale/min + BF16
+ * coefficients; BF16 format: 2 bytes per element).  This is the figure behind
+ * the pages' effective-bitwidth accounting (ai4snews summary, paragraph 2):
+ * for 4 loops, INT4 anchor, INT2 residuals, g = 32 it is 19.34% of BF16
+ * (the 80.7% reduction).  0 if cfg is invalid. */
+size_t rq_cache_token_bytes(const rq_config *cfg);
+
+/* Creates a cache.  dev_mem: caller-owned device arena of at least
+ * rq_cache_required_bytes(cfg) bytes, 256-byte aligned, or NULL to let the
+ * library cudaMalloc it.  The arena is zeroed (synchronously).  On success
+ * *out receives the handle.  Errors: INVALID, UNSUPPORTED, NOMEM, CUDA. */
+int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache **out);
+
+/* Frees the handle and, if the library allocated it, the arena
+ * (synchronises the device first).  NULL is accepted. */
+int rq_cache_destroy(rq_cache *cache);
+
+/*
+ * Append n_tokens tokens of one (layer, loop) for every sequence.
+ *   k_bf16, v_bf16: device, [batch][n_tokens][num_kv_heads][head_dim] BF16.
+ * RQ_FMT_RESIDUAL:
+ *   - a non-anchor loop copies its K/V into that loop's BF16 tail (the
+ *     in-flight tokens, read by decode as they are);
+ *   - the anchor loop (last loop of its group) requires every other loop of
+ *     the group to hold exactly n_tokens tail tokens (else RQ_ERR_STATE);
+ *     it quantizes the anchor to INT<anchor_bits> (groups of g, FP8 scale
+ *     and min), and for each other loop computes the least-squares
+ *     coefficient s = <x_l, a_hat>/<a_hat, a_hat> (BF16), the residual
+ *     x_l - s_hat a_hat, rotates it by R and quantizes it to
+ *     INT<resid_bits> the same way (ai4snews summary, paragraph 1); then it
+ *     commits the tokens and empties the group's tails.  The encoding
+ *     decisions are taken in fp64.
+ * RQ_FMT_BF16: the tokens are stored in that loop's BF16 cache directly.
+ * Errors: INVALID, CAPACITY, STATE, CUDA.  The input buffers may be reused
+ * once the enqueued work has run.
+ */
+int rq_append(rq_cache *cache, int layer, int loop, const void *k_bf16, const void *v_bf16,
+              int n_tokens, void *stream);
+
+/*
+ * Single-token decode attention for one (layer, loop) over the compressed
+ * cache (format RQ_FMT_RESIDUAL).
+ *   q_bf16: device, [batch][num_q_heads][head_dim] BF16.
+ *   out:    device, [batch][num_q_heads][head_dim] fp32.
+ *   softmax_scale: logits are scale * <q, k>; <= 0 selects 1/sqrt(head_dim).
+ * Keys/values seen: the committed tokens of the loop's group (anchor loop:
+ * the dequantized anchor; other loops: s_hat a_hat + R^T r_hat), followed by
+ * the loop's BF16 tail tokens.  With no key at all the output is zero.
+ * Errors: INVALID, STATE (wrong format), CUDA.
+ */
+int rq_decode_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
+                   float softmax_scale, void *stream);
+
+/* The same attention over an RQ_FMT_BF16 cache: the uncompressed comparison
+ * kernel (the role BF16 FlashAttention plays in the ai4snews summary,
+ * paragraph 4).  Errors: INVALID, STATE (wrong format), CUDA. */
+int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
+                        float softmax_scale, void *stream);
+
+/* Committed length of (layer, group).  group = loop / loops_per_group for
+ * the residual format; for the BF16 format pass the loop index. */
+int rq_cache_length(const rq_cache *cache, int layer, int group, int *len);
+
+/* In-flight (tail) tokens of (layer, loop); 0 for anchor loops and for the
+ * BF16 format. */
+int rq_cache_tail_length(const rq_cache *cache, int layer, int loop, int *n);
+
+/* Roll the committed length of (layer, group) back to new_len (<= current),
+ * e.g. to discard rejected tokens.  The group's tails must be empty (else
+ * RQ_ERR_STATE).  Host-side only: no device work. */
+int rq_cache_truncate(rq_cache *cache, int layer, int group, int new_len);
+
+/*
+ * Copy the committed records of (layer, loop) to host memory in the logical
+ * record format (for tests and inspection; synchronises `stream`):
+ *   anchor loop:   host_codes [2][B][H_kv][len][d*anchor_bits/8]  (K then V)
+ *                  host_meta  [2][B][H_kv][len][2*d/g]  ([scale, min] per group)
+ *                  host_coef  unused (may be NULL)
+ *   other loops:   host_codes [2][B][H_kv][len][d*resid_bits/8]
+ *                  host_meta  [2][B][H_kv][len][2*d/g]
+ *                  host_coef  [2][B][H_kv][len] BF16
+ * Code packing: element i at byte i*b/8, bit (i*b)%8, LSB first.
+ * Errors: INVALID, STATE (BF16 format), CUDA.
+ */
+int rq_cache_export(const rq_cache *cache, int layer, int loop, void *host_codes, void *host_meta,
+                    void *host_coef, void *stream);
+
+/* Algorithmic bytes one decode call of (layer, loop) moves at the current
+ * lengths: codes + FP8 meta + BF16 coefficients of the records read (anchor
+ * and, for non-anchor loops, the loop's residual), BF16 tail tokens, BF16 q
+ * and fp32 out.  Split-combine traffic is not counted.  0 on bad input. */
+size_t rq_decode_bytes(const rq_cache *cache, int layer, int loop);
+
+/* Reports asynchronous failures: RQ_ERR_TIMEOUT if a kernel's bounded wait
+ * gave up, RQ_ERR_CUDA if the context holds a sticky error, else RQ_OK.
+ * Synchronises the device. */
+int rq_check(rq_cache *cache);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RQ_H */

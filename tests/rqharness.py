@@ -1,0 +1,241 @@
+"""Test harness: builds caches on the GPU through the C ABI from seeded
+synthetic inputs, and checks the GPU results against the fp64 oracle.
+
+Parity contract (stated for the ResidualQuant hot path):
+  * packed codes, FP8 scale/min and BF16 coefficients bit-exact, except
+    values the oracle flags as lying within 1e-6 (relative) of a rounding
+    boundary; a flagged coefficient excludes its residual record, a flagged
+    scale/min excludes its group's codes, and any anchor flag excludes the
+    token-head's residual records (they depend on the anchor);
+  * attention output against the oracle fed the GPU's own records: relative
+    L2 error <= 1e-3 and max abs error <= 2e-3;
+  * reconstruction MSE of the GPU's records within 1% of the oracle's.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+import decode_attention_14_b200 as rq
+from decode_attention_14_b200 import synth
+from oracle import oracle as orc
+
+REL_L2_TOL = 1e-3
+MAX_ABS_TOL = 2e-3
+MSE_REL_TOL = 0.01
+D = 128
+
+
+@dataclass
+class Built:
+    cache: rq.Cache
+    cfg: object
+    seed: int
+    T: int
+    n_tail: int
+    # inputs[layer][group] = (K list of Lg bf16 [B][T+n_tail][H][d], V list)
+    inputs: dict = field(default_factory=dict)
+
+
+def scale32() -> float:
+    return float(np.float32(1.0 / math.sqrt(D)))
+
+
+def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, rotate=True,
+          n_tail=0, seed=0x5EED0000, sigma=(0.1, 0.2, 0.3), chunk=128, fmt=rq.RQ_FMT_RESIDUAL,
+          only_layers=None, only_groups=None, max_tokens=None) -> Built:
+    """Fills `layers` x (loops/Lg) groups with T committed tokens (appended in
+    chunks through the tail), then n_tail in-flight tokens on every
+    non-anchor loop."""
+    tail_cap = max(chunk, n_tail, 1)
+    cfg = rq.make_config(num_layers=layers, num_loops=loops, loops_per_group=Lg, batch=B,
+                         max_tokens=max_tokens or max(T, 1), max_tail_tokens=tail_cap, num_kv_heads=H,
+                         num_q_heads=Hq, group_size=g, anchor_bits=ba, resid_bits=br, rotate=rotate,
+                         format=fmt, seed=0xA11CE)
+    cache = rq.Cache(cfg)
+    bt = Built(cache, cfg, seed, T, n_tail)
+    for layer in range(layers):
+        if only_layers is not None and layer not in only_layers:
+            continue
+        for grp in range(loops // Lg):
+            if only_groups is not None and grp not in only_groups:
+                continue
+            K, V = synth.group_kv(seed, layer, grp, Lg, sigma, B, T + n_tail, H, device="cuda")
+            bt.inputs[(layer, grp)] = (K, V)
+            for t0 in range(0, T, chunk):
+                t1 = min(T, t0 + chunk)
+                for j in range(Lg):
+                    loop = grp * Lg + j
+                    k = K[j][:, t0:t1].contiguous()
+                    v = V[j][:, t0:t1].contiguous()
+                    cache.append(layer, loop, k, v)
+            if n_tail and fmt == rq.RQ_FMT_RESIDUAL:
+                for j in range(Lg - 1):
+                    cache.append(layer, grp * Lg + j, K[j][:, T:].contiguous(), V[j][:, T:].contiguous())
+    torch.cuda.synchronize()
+    return bt
+
+
+# ------------------------------------------------------------------ records
+def oracle_encode(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> orc.Encoded:
+    """Oracle encoding of the committed tokens of one group and side.
+    Token-heads ordered (b, h, t) like the export; bh_sel restricts to a list
+    of (b, h)."""
+    K, V = bt.inputs[(layer, grp)]
+    X = K if kv == 0 else V
+    Lg = len(X)
+    T = bt.T
+    arrs = []
+    for j in range(Lg):
+        u = synth.bf16_to_u16(X[j][:, :T])            # [B][T][H][d]
+        u = np.ascontiguousarray(u.transpose(0, 2, 1, 3))   # [B][H][T][d]
+        if bh_sel is not None:
+            u = np.stack([u[b, h] for (b, h) in bh_sel])     # [nsel][T][d]
+        arrs.append(u.reshape(-1, D))
+    x = np.stack(arrs)
+    cfg = bt.cfg
+    return orc.encode(x, cfg.group_size, cfg.anchor_bits, cfg.resid_bits, bool(cfg.rotate), cfg.seed)
+
+
+def gpu_records(bt: Built, layer: int, loop: int, kv: int, bh_sel=None):
+    codes, meta, coef = bt.cache.export(layer, loop)
+    c, m = codes[kv], meta[kv]
+    f = None if coef is None else coef[kv]
+    if bh_sel is not None:
+        c = np.stack([c[b, h] for (b, h) in bh_sel])
+        m = np.stack([m[b, h] for (b, h) in bh_sel])
+        if f is not None:
+            f = np.stack([f[b, h] for (b, h) in bh_sel])
+    c = c.reshape(-1, c.shape[-1])
+    m = m.reshape(-1, m.shape[-1])
+    if f is not None:
+        f = f.reshape(-1)
+    return c, m, f
+
+
+def _elem_codes(packed: np.ndarray, bits: int) -> np.ndarray:
+    per = 8 // bits
+    return np.stack([(packed >> (bits * k)) & ((1 << bits) - 1) for k in range(per)], -1).reshape(
+        packed.shape[0], -1)
+
+
+def compare_records(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
+    """Bit-exact comparison with exclusions.  Returns dict of counts."""
+    cfg = bt.cfg
+    Lg = cfg.loops_per_group
+    e = oracle_encode(bt, layer, grp, kv, bh_sel)
+    G = D // cfg.group_size
+    res = dict(mismatch=0, flagged=0, compared=0)
+    anchor_loop = grp * Lg + Lg - 1
+    gc, gm, _ = gpu_records(bt, layer, anchor_loop, kv, bh_sel)
+    a_bad = (e.a_eflag.any(1) | (e.a_mflag != 0).any(1))      # token-heads with any anchor flag
+
+    def cmp(gpu_c, gpu_m, orc_c, orc_m, eflag, mflag, bits, skip_rows):
+        ge, oe = _elem_codes(gpu_c, bits), _elem_codes(orc_c, bits)
+        grp_of = np.arange(D) // cfg.group_size
+        excl = eflag.astype(bool) | (mflag[:, grp_of] != 0) | skip_rows[:, None]
+        res["flagged"] += int(excl.sum())
+        res["compared"] += int((~excl).sum())
+        res["mismatch"] += int(((ge != oe) & ~excl).sum())
+        sc_ok = ((mflag & 1) == 0) & ~skip_rows[:, None]
+        mn_ok = ((mflag & 2) == 0) & ~skip_rows[:, None]
+        res["mismatch"] += int(((gpu_m[:, 0::2] != orc_m[:, 0::2]) & sc_ok).sum())
+        res["mismatch"] += int(((gpu_m[:, 1::2] != orc_m[:, 1::2]) & mn_ok).sum())
+
+    cmp(gc, gm, e.a_codes, e.a_meta, e.a_eflag, e.a_mflag, cfg.anchor_bits, np.zeros(len(gc), bool))
+    for j in range(Lg - 1):
+        rc, rm, rf = gpu_records(bt, layer, grp * Lg + j, kv, bh_sel)
+        skip = a_bad | (e.r_cflag[j] != 0)
+        res["mismatch"] += int(((rf != e.r_coef[j]) & ~skip).sum())
+        res["flagged"] += int(skip.sum())
+        cmp(rc, rm, e.r_codes[j], e.r_meta[j], e.r_eflag[j], e.r_mflag[j], cfg.resid_bits, skip)
+    return res
+
+
+def reconstruct_gpu(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> np.ndarray:
+    """Oracle reconstruction of the GPU's exported records: [Lg][n][d]."""
+    cfg = bt.cfg
+    Lg = cfg.loops_per_group
+    ac, am, _ = gpu_records(bt, layer, grp * Lg + Lg - 1, kv, bh_sel)
+    if Lg > 1:
+        rs = [gpu_records(bt, layer, grp * Lg + j, kv, bh_sel) for j in range(Lg - 1)]
+        rc = np.stack([r[0] for r in rs])
+        rm = np.stack([r[1] for r in rs])
+        rf = np.stack([r[2] for r in rs])
+    else:
+        rc = rm = rf = None
+    return orc.reconstruct(ac, am, rc, rm, rf, Lg, D, cfg.group_size, cfg.anchor_bits, cfg.resid_bits,
+                           bool(cfg.rotate), cfg.seed)
+
+
+def mse_check(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
+    cfg = bt.cfg
+    e = oracle_encode(bt, layer, grp, kv, bh_sel)
+    Lg = cfg.loops_per_group
+    mine = orc.reconstruct(e.a_codes, e.a_meta, e.r_codes if Lg > 1 else None, e.r_meta if Lg > 1 else None,
+                           e.r_coef if Lg > 1 else None, Lg, D, cfg.group_size, cfg.anchor_bits, cfg.resid_bits,
+                           bool(cfg.rotate), cfg.seed)
+    gpu = reconstruct_gpu(bt, layer, grp, kv, bh_sel)
+    K, V = bt.inputs[(layer, grp)]
+    X = K if kv == 0 else V
+    xs = []
+    for j in range(Lg):
+        u = synth.bf16_to_u16(X[j][:, :bt.T]).transpose(0, 2, 1, 3)
+        if bh_sel is not None:
+            u = np.stack([u[b, h] for (b, h) in bh_sel])
+        xs.append(orc.bf16_bits_to_f64(np.ascontiguousarray(u).reshape(-1, D)))
+    x = np.stack(xs)
+    return orc.mse(gpu, x), orc.mse(mine, x)
+
+
+# ------------------------------------------------------------------ attention
+def oracle_decode(bt: Built, layer: int, loop: int, q_bf16: torch.Tensor, bh_sel=None, bf16_cache=False):
+    """Oracle attention for (layer, loop), keys/values from the GPU's own
+    records (or, for the BF16 format, the BF16 inputs).  Returns
+    [len(bh_sel) or B*Hq ...] as [B][Hq][d] restricted to selected (b, kv)."""
+    cfg = bt.cfg
+    Lg = cfg.loops_per_group
+    grp, j = loop // Lg, loop % Lg
+    B, H, Hq = cfg.batch, cfg.num_kv_heads, cfg.num_q_heads
+    Gq = Hq // H
+    K, V = bt.inputs[(layer, grp)]
+    sel = bh_sel if bh_sel is not None else [(b, h) for b in range(B) for h in range(H)]
+    n_tail = bt.n_tail if (j != Lg - 1 and not bf16_cache) else 0
+    T = bt.T
+    qf = orc.bf16_bits_to_f64(synth.bf16_to_u16(q_bf16))          # [B][Hq][d]
+    kv_vals = []
+    for kv, X in ((0, K), (1, V)):
+        if bf16_cache:
+            u = synth.bf16_to_u16(X[j][:, :T]).transpose(0, 2, 1, 3)
+            vals = orc.bf16_bits_to_f64(np.stack([u[b, h] for (b, h) in sel]))     # [nsel][T][d]
+        else:
+            rec = reconstruct_gpu(bt, layer, grp, kv, sel)[j].reshape(len(sel), T, D)
+            vals = rec
+        if n_tail:
+            tu = synth.bf16_to_u16(X[j][:, T:T + n_tail]).transpose(0, 2, 1, 3)
+            tv = orc.bf16_bits_to_f64(np.stack([tu[b, h] for (b, h) in sel]))
+            vals = np.concatenate([vals, tv], axis=1)
+        kv_vals.append(vals)
+    out = {}
+    for i, (b, h) in enumerate(sel):
+        q = qf[b:b + 1, h * Gq:(h + 1) * Gq]                       # [1][Gq][d]
+        k = kv_vals[0][i][None, :, None, :]
+        v = kv_vals[1][i][None, :, None, :]
+        o = orc.attention(q, k, v, scale32())
+        out[(b, h)] = o[0]                                          # [Gq][d]
+    return out
+
+
+def attn_errors(gpu_out: np.ndarray, ref: dict, Gq: int):
+    g, r = [], []
+    for (b, h), o in ref.items():
+        g.append(gpu_out[b, h * Gq:(h + 1) * Gq])
+        r.append(o)
+    g = np.concatenate(g).astype(np.float64)
+    r = np.concatenate(r)
+    rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
+    mx = float(np.abs(g - r).max())
+    return rel, mx
