@@ -20,6 +20,8 @@ struct rq_cache {
     std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]
     std::vector<int> ntail;   // [layer][loop]
     uint32_t sigma[4] = {0, 0, 0, 0};
+    // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
+    int occ[2][kMaxChunk / kTokTile];
 };
 
 namespace {
@@ -73,23 +75,36 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; 
 
 float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt((float)kHeadDim); }
 
-// Split-KV partition: enough CTAs to cover the SMs a few times over, chunks
-// that are a multiple of 16 tokens.
-void choose_splits(const rq_cache *c, int T, int units, int *S, int *chunk) {
+// Split-KV partition of T tokens over `units` independent (sequence, kv head
+// [, q-head pair]) problems.  Chunks are whole 64-token tiles, at most
+// kMaxChunk.  Among the admissible split counts the one with the least
+// wave-quantised work (waves x tokens per CTA, plus a fixed per-CTA cost)
+// is taken, waves counted from the kernel's measured occupancy.
+void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *chunk) {
     if (T <= 0) {
         *S = 0;
-        *chunk = 16;
+        *chunk = kTokTile;
         return;
     }
-    int target = c->sms * 4;
-    int s = (target + units - 1) / units;
-    int smax = std::min(c->lay.splits_max, (T + 63) / 64);
-    s = std::max(1, std::min(s, smax));
-    s = std::max(s, (T + kMaxChunk - 1) / kMaxChunk);   // bounded per-CTA logit buffer
-    int ch = (T + s - 1) / s;
-    ch = (ch + 15) / 16 * 16;
-    *chunk = ch;
-    *S = (T + ch - 1) / ch;
+    const int s_lo = (T + kMaxChunk - 1) / kMaxChunk;
+    const int s_hi = std::min(c->lay.splits_max, (T + kTokTile - 1) / kTokTile);
+    long best_cost = -1;
+    int best_s = s_lo, best_ch = kMaxChunk;
+    for (int s = s_lo; s <= std::max(s_lo, s_hi); s++) {
+        int ch = (T + s - 1) / s;
+        ch = (ch + kTokTile - 1) / kTokTile * kTokTile;
+        const int ss = (T + ch - 1) / ch;
+        const int slots = std::max(1, c->occ[which][ch / kTokTile - 1] * c->sms);
+        const long waves = ((long)ss * units + slots - 1) / slots;
+        const long cost = waves * (ch + 2 * kTokTile);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_s = ss;
+            best_ch = ch;
+        }
+    }
+    *S = best_s;
+    *chunk = best_ch;
 }
 
 }  // namespace
@@ -238,6 +253,19 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
     const Layout &L = c->lay;
     c->len.assign((size_t)cfg->num_layers * (cfg->format == RQ_FMT_RESIDUAL ? L.groups : cfg->num_loops), 0);
     c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
+    {
+        const int G = cfg->num_q_heads / cfg->num_kv_heads;
+        for (int i = 0; i < kMaxChunk / kTokTile; i++) {
+            const int ch = kTokTile * (i + 1);
+            if (cfg->format == RQ_FMT_BF16) {
+                c->occ[0][i] = c->occ[1][i] = decode_bf16_occupancy(G, ch);
+            } else {
+                c->occ[0][i] = decode_rq_occupancy(G, cfg->anchor_bits, cfg->resid_bits, false, cfg->group_size, ch);
+                c->occ[1][i] = decode_rq_occupancy(G, cfg->anchor_bits, cfg->resid_bits, true, cfg->group_size, ch);
+            }
+        }
+        cudaGetLastError();
+    }
     if (cfg->rotate)
         for (int j = 0; j < kHeadDim; j++)
             if (splitmix64(cfg->seed + (uint64_t)j) >> 63) c->sigma[j / 32] |= 1u << (j % 32);
@@ -350,6 +378,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     std::memset(&a, 0, sizeof(a));
     a.q = (const uint16_t *)q;
     a.partials = (float *)(c->base + L.off_partials);
+    a.err = (int *)(c->base + L.off_err);
     a.B = cfg.batch;
     a.H = cfg.num_kv_heads;
     a.Hq = cfg.num_q_heads;
@@ -388,7 +417,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
-    choose_splits(c, a.T, units, &a.S, &a.chunk);
+    choose_splits(c, a.T, units, resid ? 1 : 0, &a.S, &a.chunk);
     if (a.S > 0) {
         cudaError_t e = bf16 ? launch_decode_bf16(a, st)
                              : launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st);

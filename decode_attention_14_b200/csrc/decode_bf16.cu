@@ -184,6 +184,14 @@ cudaError_t launch_decode_bf16(const DecodeArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+int decode_bf16_occupancy(int G, int chunk) {
+    int n = 0;
+    const size_t smem = (size_t)chunk * sizeof(float) * (G == 1 ? 1 : 2);
+    cudaError_t e = G == 1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_bf16_kernel<1>, 128, smem)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_bf16_kernel<2>, 128, smem);
+    return (e == cudaSuccess && n > 0) ? n : 1;
+}
+
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     combine_kernel<<<dim3(a.Hq, a.B), 128, 0, st>>>(a);
     return cudaGetLastError();

@@ -15,7 +15,7 @@ namespace rq {
 constexpr int kHeadDim = 128;
 constexpr int kTokTile = 64;        // padding granule of every token stream
 constexpr int kMaxSplits = 256;     // split-KV partitions per (b, kv head)
-constexpr int kMaxChunk = 4096;     // tokens per CTA (bounds the logit buffer)
+constexpr int kMaxChunk = 1024;     // tokens per CTA (bounds the per-CTA shared-memory buffers)
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -105,6 +105,7 @@ struct DecodeArgs {
     const uint16_t *bf[2];
     const uint16_t *q;        // [B][Hq][d] bf16
     float *partials;          // [B][Hq][splits_max][kPartialStride]
+    int *err;                 // device error word (bounded waits that gave up)
     int B, H, Hq, G, T, Tp, S, chunk, splits_max;
     int g;
     float scale_log2;         // softmax_scale * log2(e)
@@ -127,5 +128,8 @@ cudaError_t launch_bf16_store(const Bf16StoreArgs &a, cudaStream_t st);
 cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st);
 cudaError_t launch_decode_bf16(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
+// resident CTAs per SM of the decode kernels for a given chunk (tokens per CTA)
+int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk);
+int decode_bf16_occupancy(int G, int chunk);
 
 }  // namespace rq

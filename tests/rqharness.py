@@ -2,11 +2,12 @@
 synthetic inputs, and checks the GPU results against the fp64 oracle.
 
 Parity contract (stated for the ResidualQuant hot path):
-  * packed codes, FP8 scale/min and BF16 coefficients bit-exact, except
-    values the oracle flags as lying within 1e-6 (relative) of a rounding
-    boundary; a flagged coefficient excludes its residual record, a flagged
-    scale/min excludes its group's codes, and any anchor flag excludes the
-    token-head's residual records (they depend on the anchor);
+  * every packed code, FP8 scale/min and BF16 coefficient is compared and
+    must be bit-exact; a difference is tolerated (and counted) only at a
+    value the oracle flags as lying within 1e-6 (relative) of a rounding
+    boundary, exact ties included.  A tolerated difference excludes what
+    depends on it: a scale/min its group's codes, a coefficient its residual
+    record, an anchor record the token-head's residual records;
   * attention output against the oracle fed the GPU's own records: relative
     L2 error <= 1e-3 and max abs error <= 2e-3;
   * reconstruction MSE of the GPU's records within 1% of the oracle's.
@@ -123,35 +124,50 @@ def _elem_codes(packed: np.ndarray, bits: int) -> np.ndarray:
 
 
 def compare_records(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
-    """Bit-exact comparison with exclusions.  Returns dict of counts."""
+    """Compares every code, FP8 scale/min and BF16 coefficient.  A difference
+    at a value the oracle flags as within 1e-6 (relative) of a rounding
+    boundary (exact ties included) is tolerated and counted; a tolerated
+    difference in an anchor record or a coefficient excludes the records that
+    depend on it (the token-head's residuals / that residual record).  Any
+    other difference is a mismatch.  Returns counts."""
     cfg = bt.cfg
     Lg = cfg.loops_per_group
     e = oracle_encode(bt, layer, grp, kv, bh_sel)
-    G = D // cfg.group_size
-    res = dict(mismatch=0, flagged=0, compared=0)
+    res = dict(mismatch=0, tolerated=0, flagged=0, excluded=0, compared=0)
     anchor_loop = grp * Lg + Lg - 1
     gc, gm, _ = gpu_records(bt, layer, anchor_loop, kv, bh_sel)
-    a_bad = (e.a_eflag.any(1) | (e.a_mflag != 0).any(1))      # token-heads with any anchor flag
+    grp_of = np.arange(D) // cfg.group_size
 
     def cmp(gpu_c, gpu_m, orc_c, orc_m, eflag, mflag, bits, skip_rows):
+        """returns per-row bool: some tolerated difference in this record"""
         ge, oe = _elem_codes(gpu_c, bits), _elem_codes(orc_c, bits)
-        grp_of = np.arange(D) // cfg.group_size
-        excl = eflag.astype(bool) | (mflag[:, grp_of] != 0) | skip_rows[:, None]
-        res["flagged"] += int(excl.sum())
+        live = ~skip_rows[:, None]
+        # meta
+        sc_diff = (gpu_m[:, 0::2] != orc_m[:, 0::2]) & live
+        mn_diff = (gpu_m[:, 1::2] != orc_m[:, 1::2]) & live
+        sc_flag = (mflag & 1) != 0
+        mn_flag = (mflag & 2) != 0
+        res["mismatch"] += int((sc_diff & ~sc_flag).sum() + (mn_diff & ~mn_flag).sum())
+        meta_tol = (sc_diff & sc_flag) | (mn_diff & mn_flag)             # [rows][groups]
+        # codes: a group whose meta legitimately differs is excluded
+        excl = meta_tol[:, grp_of] | skip_rows[:, None]
+        diff = (ge != oe) & ~excl
+        fl = eflag.astype(bool)
+        res["mismatch"] += int((diff & ~fl).sum())
+        res["tolerated"] += int((diff & fl).sum() + meta_tol.sum())
+        res["flagged"] += int((fl & ~excl).sum() + ((sc_flag | mn_flag) & live).sum())
+        res["excluded"] += int(excl.sum())
         res["compared"] += int((~excl).sum())
-        res["mismatch"] += int(((ge != oe) & ~excl).sum())
-        sc_ok = ((mflag & 1) == 0) & ~skip_rows[:, None]
-        mn_ok = ((mflag & 2) == 0) & ~skip_rows[:, None]
-        res["mismatch"] += int(((gpu_m[:, 0::2] != orc_m[:, 0::2]) & sc_ok).sum())
-        res["mismatch"] += int(((gpu_m[:, 1::2] != orc_m[:, 1::2]) & mn_ok).sum())
+        return (diff & fl).any(1) | meta_tol.any(1)
 
-    cmp(gc, gm, e.a_codes, e.a_meta, e.a_eflag, e.a_mflag, cfg.anchor_bits, np.zeros(len(gc), bool))
+    a_tol = cmp(gc, gm, e.a_codes, e.a_meta, e.a_eflag, e.a_mflag, cfg.anchor_bits, np.zeros(len(gc), bool))
     for j in range(Lg - 1):
         rc, rm, rf = gpu_records(bt, layer, grp * Lg + j, kv, bh_sel)
-        skip = a_bad | (e.r_cflag[j] != 0)
-        res["mismatch"] += int(((rf != e.r_coef[j]) & ~skip).sum())
-        res["flagged"] += int(skip.sum())
-        cmp(rc, rm, e.r_codes[j], e.r_meta[j], e.r_eflag[j], e.r_mflag[j], cfg.resid_bits, skip)
+        cdiff = (rf != e.r_coef[j]) & ~a_tol
+        cflag = e.r_cflag[j] != 0
+        res["mismatch"] += int((cdiff & ~cflag).sum())
+        res["tolerated"] += int((cdiff & cflag).sum())
+        cmp(rc, rm, e.r_codes[j], e.r_meta[j], e.r_eflag[j], e.r_mflag[j], cfg.resid_bits, a_tol | cdiff)
     return res
 
 
