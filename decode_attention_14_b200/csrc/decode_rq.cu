@@ -13,13 +13,18 @@
 // basis, the residual part in the rotated basis, and R^T is applied once per
 // CTA to the rotated accumulator.
 //
-// Arithmetic.  The per-code products run on the integer dot-product unit
-// (dp2a: two 16-bit x 8-bit products per instruction): q (and R q) are
-// converted once per CTA to 16-bit fixed point with a power-of-two scale,
-// and the V weights p_t * s_t * sc_{g,t} to 16-bit fixed point with one
-// power-of-two scale per quantization group, chosen from the chunk's largest
-// weight bound (so every weight keeps >= 14 significant bits).  Per-group
-// scales, minima, softmax and the final rotation stay in fp32.
+// Arithmetic.  The per-code products run on the integer dot-product units,
+// which consume packed codes with no conversion to floating point:
+//  - logits: q (and R q) are converted once per CTA to 24-bit fixed point
+//    (power-of-two scale, |q| < 2^22) split into three byte planes, and
+//    sum_i q_i c_i is three dp4a (4 products each) per 4 codes, exact;
+//  - values: each weight p_t s_t sc_{g,t} becomes 32-bit fixed point with a
+//    power-of-two scale per quantization group (the chunk's bound of the
+//    weight mapped into [2^29, 2^30)) split into 16-bit halves, and
+//    sum_t w_t c_t,i is two dp2a (2 products each) per 2 codes, exact.
+// The fixed-point rounding of q and of the weights is the only deviation from
+// fp32 arithmetic (relative 2^-21 of max|q|, 2^-29 of the weight bound).
+// Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
 // Data movement.  Each CTA owns a chunk of one (sequence, kv head), streamed
 // in 64-token tiles through a 3-stage shared-memory ring filled by one
@@ -47,7 +52,6 @@ constexpr int kStages = 3;
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
-constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: float(x) + kMagic holds round(x) in its low bits
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait
 
 // ---------------------------------------------------------------- PTX helpers
@@ -119,81 +123,82 @@ __device__ __forceinline__ Seg<BITS> lds_seg(const uint8_t *p) {
     return s;
 }
 
-// Which two segment elements sit in the 16-bit halves of q pair register r,
-// matching the byte lanes the unpacking below produces (dp2a .lo uses code
-// bytes 0,1; .hi bytes 2,3).
+// Byte lanes of the unpacked code words of a 16-element segment.  Unpacked
+// word r holds four codes, one per byte; elem_of<BITS>(r, m) is the segment
+// element in byte m of word r.
+//   BITS=4: r = 2u + hi: nibbles of word u; bytes = elements 8u + hi + {0,2,4,6}
+//   BITS=2: r = c: (w >> 2c) & 0x03030303; bytes = elements c + {0,4,8,12}
 template <int BITS>
-__device__ __forceinline__ void qpair_index(int r, int &i0, int &i1) {
-    if (BITS == 4) {
-        // lo nibbles of word u: bytes = elements 8u+{0,2,4,6}; hi nibbles: 8u+{1,3,5,7}
-        const int u = r >> 2, hi = (r >> 1) & 1, upper = r & 1;
-        i0 = 8 * u + hi + 4 * upper;
-        i1 = i0 + 2;
-    } else {
-        // (w >> 2c) & 0x03030303: bytes = elements c, 4+c, 8+c, 12+c
-        const int c = r >> 1, upper = r & 1;
-        i0 = c + 8 * upper;
-        i1 = i0 + 4;
-    }
+__device__ __forceinline__ int elem_of(int r, int m) {
+    return BITS == 4 ? 8 * (r >> 1) + (r & 1) + 2 * m : r + 4 * m;
 }
 
-// sum_i q_i c_i over a segment, q as 16-bit pairs in the order of qpair_index.
 template <int BITS>
-__device__ __forceinline__ int dot_seg(const Seg<BITS> &s, const uint32_t qp[8]) {
-    int acc = 0;
-    if (BITS == 4) {
-#pragma unroll
-        for (int u = 0; u < 2; u++) {
-            const int lo = (int)(s.w[u] & 0x0F0F0F0Fu);
-            const int hi = (int)((s.w[u] >> 4) & 0x0F0F0F0Fu);
-            acc = __dp2a_lo((int)qp[4 * u + 0], lo, acc);
-            acc = __dp2a_hi((int)qp[4 * u + 1], lo, acc);
-            acc = __dp2a_lo((int)qp[4 * u + 2], hi, acc);
-            acc = __dp2a_hi((int)qp[4 * u + 3], hi, acc);
-        }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const int b = (int)((s.w[0] >> (2 * c)) & 0x03030303u);
-            acc = __dp2a_lo((int)qp[2 * c + 0], b, acc);
-            acc = __dp2a_hi((int)qp[2 * c + 1], b, acc);
-        }
-    }
-    return acc;
+__device__ __forceinline__ uint32_t unpack_word(const Seg<BITS> &s, int r) {
+    if (BITS == 4) return (r & 1) ? ((s.w[r >> 1] >> 4) & 0x0F0F0F0Fu) : (s.w[r >> 1] & 0x0F0F0F0Fu);
+    return (s.w[0] >> (2 * r)) & 0x03030303u;
 }
 
-// acc[i] += w0 * c0_i + w1 * c1_i for the 16 elements of a segment, codes of
-// two tokens, weights packed as (w0 | w1 << 16).
+// q of one segment in 24-bit fixed point as three byte planes laid out like
+// the unpacked code words: plane 0 and 1 unsigned, plane 2 signed.
+struct QPlanes {
+    uint32_t p[3][4];
+};
+
+// sum_i q_i c_i of one segment, exact in int32 (|q| < 2^22).
 template <int BITS>
-__device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b, uint32_t wp, int acc[16]) {
-    const int W = (int)wp;
+__device__ __forceinline__ int dot_seg(const Seg<BITS> &s, const QPlanes &q) {
+    unsigned lo = 0, mid = 0;
+    int hi = 0;
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+        const uint32_t c = unpack_word<BITS>(s, r);
+        lo = __dp4a(q.p[0][r], c, lo);
+        mid = __dp4a(q.p[1][r], c, mid);
+        hi = __dp4a((int)q.p[2][r], (int)c, hi);
+    }
+    return (int)(((unsigned)hi << 16) + (mid << 8) + lo);
+}
+
+// acc{Lo,Hi}[i] += w0 * c0_i + w1 * c1_i for the 16 elements of a segment,
+// codes of two tokens; weights as 16-bit halves: wlo = (w0 & 0xFFFF) |
+// (w1 << 16) (unsigned), whi = (w0 >> 16) | (w1 >> 16) << 16 (signed).
+template <int BITS>
+__device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b, uint32_t wlo, uint32_t whi,
+                                         unsigned accLo[16], int accHi[16]) {
+    const int Wh = (int)whi;
     if (BITS == 4) {
 #pragma unroll
         for (int u = 0; u < 2; u++) {
             const uint32_t X = __byte_perm(a.w[u], b.w[u], 0x5140);   // bytes 0,1 of both tokens
             const uint32_t Y = __byte_perm(a.w[u], b.w[u], 0x7362);   // bytes 2,3 of both tokens
-            const int xl = (int)(X & 0x0F0F0F0Fu), xh = (int)((X >> 4) & 0x0F0F0F0Fu);
-            const int yl = (int)(Y & 0x0F0F0F0Fu), yh = (int)((Y >> 4) & 0x0F0F0F0Fu);
-            acc[8 * u + 0] = __dp2a_lo(W, xl, acc[8 * u + 0]);
-            acc[8 * u + 2] = __dp2a_hi(W, xl, acc[8 * u + 2]);
-            acc[8 * u + 1] = __dp2a_lo(W, xh, acc[8 * u + 1]);
-            acc[8 * u + 3] = __dp2a_hi(W, xh, acc[8 * u + 3]);
-            acc[8 * u + 4] = __dp2a_lo(W, yl, acc[8 * u + 4]);
-            acc[8 * u + 6] = __dp2a_hi(W, yl, acc[8 * u + 6]);
-            acc[8 * u + 5] = __dp2a_lo(W, yh, acc[8 * u + 5]);
-            acc[8 * u + 7] = __dp2a_hi(W, yh, acc[8 * u + 7]);
+            const uint32_t c[4] = {X & 0x0F0F0F0Fu, (X >> 4) & 0x0F0F0F0Fu, Y & 0x0F0F0F0Fu, (Y >> 4) & 0x0F0F0F0Fu};
+            // c[0]: elements 8u+0 (bytes 0,1), 8u+2 (bytes 2,3); c[1]: 8u+1, 8u+3; c[2]: 8u+4, 8u+6; c[3]: 8u+5, 8u+7
+            const int e0[4] = {0, 1, 4, 5};
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const int e = 8 * u + e0[k];
+                accLo[e] = __dp2a_lo(wlo, c[k], accLo[e]);
+                accHi[e] = __dp2a_lo(Wh, (int)c[k], accHi[e]);
+                accLo[e + 2] = __dp2a_hi(wlo, c[k], accLo[e + 2]);
+                accHi[e + 2] = __dp2a_hi(Wh, (int)c[k], accHi[e + 2]);
+            }
         }
     } else {
         const uint32_t X = __byte_perm(a.w[0], b.w[0], 0x5140);   // bytes 0,1: elements 0-7
         const uint32_t Y = __byte_perm(a.w[0], b.w[0], 0x7362);   // bytes 2,3: elements 8-15
 #pragma unroll
         for (int c = 0; c < 4; c++) {
-            const int x = (int)((X >> (2 * c)) & 0x03030303u);
-            const int y = (int)((Y >> (2 * c)) & 0x03030303u);
-            acc[c] = __dp2a_lo(W, x, acc[c]);
-            acc[4 + c] = __dp2a_hi(W, x, acc[4 + c]);
-            acc[8 + c] = __dp2a_lo(W, y, acc[8 + c]);
-            acc[12 + c] = __dp2a_hi(W, y, acc[12 + c]);
+            const uint32_t x = (X >> (2 * c)) & 0x03030303u;
+            const uint32_t y = (Y >> (2 * c)) & 0x03030303u;
+            accLo[c] = __dp2a_lo(wlo, x, accLo[c]);
+            accHi[c] = __dp2a_lo(Wh, (int)x, accHi[c]);
+            accLo[4 + c] = __dp2a_hi(wlo, x, accLo[4 + c]);
+            accHi[4 + c] = __dp2a_hi(Wh, (int)x, accHi[4 + c]);
+            accLo[8 + c] = __dp2a_lo(wlo, y, accLo[8 + c]);
+            accHi[8 + c] = __dp2a_lo(Wh, (int)y, accHi[8 + c]);
+            accLo[12 + c] = __dp2a_hi(wlo, y, accLo[12 + c]);
+            accHi[12 + c] = __dp2a_hi(Wh, (int)y, accHi[12 + c]);
         }
     }
 }
@@ -203,12 +208,6 @@ __device__ __forceinline__ float2 meta_pair(uint32_t m16) {
     const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)m16, __NV_E4M3);
     return __half22float2(__half2(h));
 }
-
-// exact int -> float for |x| < 2^22 on the ALU pipes
-__device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(x + 0x4B400000) - kMagic; }
-
-// round(x * y) (|x * y| < 2^15) in the low 16 bits, one rounding, ties to even
-__device__ __forceinline__ uint32_t fix16_bits_fma(float x, float y) { return __float_as_uint(fmaf(x, y, kMagic)); }
 
 // power-of-two scale 2^F putting a positive bound into [2^(top-1), 2^top)
 __device__ __forceinline__ float fixed_scale(float bound, int top) {
@@ -239,8 +238,8 @@ __device__ __forceinline__ Layout2 make_layout2(int g, int chunk_tiles) {
     L.k_rm = L.k_rc + (RESID ? kTile * L.R_C : 0);
     L.k_cf = L.k_rm + (RESID ? kTile * L.MR : 0);
     L.k_bytes = L.k_cf + (RESID ? kTile * 2 : 0);
-    L.v_rc = kTile * L.A_C;
-    L.v_bytes = L.v_rc + (RESID ? kTile * L.R_C : 0);
+    L.v_rc = 0;                                   // residual V sub-pass stage: codes only
+    L.v_bytes = kTile * L.A_C;                    // anchor V sub-pass stage: codes only
     L.stage_bytes = ((max(L.k_bytes, L.v_bytes) + 127) / 128) * 128;
     const int ct = chunk_tiles * kTile;
     L.vm_r = ct * L.MR;
@@ -251,7 +250,7 @@ __device__ __forceinline__ Layout2 make_layout2(int g, int chunk_tiles) {
 }
 
 template <int GK, int BA, int BR, bool RESID>
-__global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kStages];
     __shared__ __align__(8) uint64_t bar_empty[kStages];
@@ -304,7 +303,8 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
                 }
             }
             int issued = 0;
-            for (int it = 0; it < 2 * ntiles; it++) {
+            const int nitems = (RESID ? 3 : 2) * ntiles;   // K tiles, V anchor tiles, V residual tiles
+            for (int it = 0; it < nitems; it++) {
                 const int stage = it % kStages;
                 if (it >= kStages && !mbar_wait(&bar_empty[stage], ((it / kStages) - 1) & 1, &s_abort)) {
                     s_abort = 1;
@@ -312,9 +312,9 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
                     break;
                 }
                 uint8_t *st = ring + stage * L.stage_bytes;
-                const bool kpass = it < ntiles;
-                const size_t tk = tok0 + (size_t)(kpass ? it : it - ntiles) * kTile;
-                if (kpass) {
+                const int pass = it / ntiles;
+                const size_t tk = tok0 + (size_t)(it - pass * ntiles) * kTile;
+                if (pass == 0) {
                     mbar_expect_tx(&bar_full[stage], (uint32_t)L.k_bytes);
                     bulk_g2s(st, a.a_codes[0] + tk * L.A_C, kTile * L.A_C, &bar_full[stage]);
                     bulk_g2s(st + L.k_am, a.a_meta[0] + tk * L.MR, kTile * L.MR, &bar_full[stage]);
@@ -323,10 +323,12 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
                         bulk_g2s(st + L.k_rm, a.r_meta[0] + tk * L.MR, kTile * L.MR, &bar_full[stage]);
                         bulk_g2s(st + L.k_cf, a.r_coef[0] + tk, kTile * 2, &bar_full[stage]);
                     }
-                } else {
-                    mbar_expect_tx(&bar_full[stage], (uint32_t)L.v_bytes);
+                } else if (pass == 1) {
+                    mbar_expect_tx(&bar_full[stage], (uint32_t)(kTile * L.A_C));
                     bulk_g2s(st, a.a_codes[1] + tk * L.A_C, kTile * L.A_C, &bar_full[stage]);
-                    if (RESID) bulk_g2s(st + L.v_rc, a.r_codes[1] + tk * L.R_C, kTile * L.R_C, &bar_full[stage]);
+                } else {
+                    mbar_expect_tx(&bar_full[stage], (uint32_t)(kTile * L.R_C));
+                    bulk_g2s(st, a.r_codes[1] + tk * L.R_C, kTile * L.R_C, &bar_full[stage]);
                 }
                 issued = it + 1;
             }
@@ -374,29 +376,35 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
     }
     consumer_sync();
     const float qmax = fmaxf(fmaxf(s_red[0][0], s_red[1][0]), fmaxf(s_red[2][0], s_red[3][0]));
-    const float qscale = fixed_scale(qmax, 14);  // q_int = round(q * qscale), |q_int| <= 2^14
+    const float qscale = fixed_scale(qmax, 22);  // q_int = round(q * qscale), |q_int| < 2^22
     const float qinv = 1.f / qscale;             // exact (power of two)
-    uint32_t qpA[GK][8], qpR[GK][8];
+    QPlanes qA[GK], qR[GK];
     float QA[GK], QR[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
         QA[gq] = QR[gq] = 0.f;
 #pragma unroll
-        for (int r = 0; r < 8; r++) {
-            int i0, i1;
-            qpair_index<BA>(r, i0, i1);
-            const float x0 = rintf(s_q[gq][0][seg * 16 + i0] * qscale);
-            const float x1 = rintf(s_q[gq][0][seg * 16 + i1] * qscale);
-            QA[gq] += x0 + x1;
-            qpA[gq][r] = ((uint32_t)(int)x0 & 0xFFFFu) | ((uint32_t)(int)x1 << 16);
-            if (RESID) {
-                qpair_index<BR>(r, i0, i1);
-                const float y0 = rintf(s_q[gq][1][seg * 16 + i0] * qscale);
-                const float y1 = rintf(s_q[gq][1][seg * 16 + i1] * qscale);
-                QR[gq] += y0 + y1;
-                qpR[gq][r] = ((uint32_t)(int)y0 & 0xFFFFu) | ((uint32_t)(int)y1 << 16);
-            } else {
-                qpR[gq][r] = 0;
+        for (int r = 0; r < 4; r++) {
+            uint32_t pa[3] = {0, 0, 0}, pr[3] = {0, 0, 0};
+#pragma unroll
+            for (int m = 0; m < 4; m++) {
+                const int xa = __float2int_rn(s_q[gq][0][seg * 16 + elem_of<BA>(r, m)] * qscale);
+                QA[gq] += (float)xa;
+                pa[0] |= (uint32_t)(xa & 0xFF) << (8 * m);
+                pa[1] |= (uint32_t)((xa >> 8) & 0xFF) << (8 * m);
+                pa[2] |= (uint32_t)((xa >> 16) & 0xFF) << (8 * m);
+                if (RESID) {
+                    const int xr = __float2int_rn(s_q[gq][1][seg * 16 + elem_of<BR>(r, m)] * qscale);
+                    QR[gq] += (float)xr;
+                    pr[0] |= (uint32_t)(xr & 0xFF) << (8 * m);
+                    pr[1] |= (uint32_t)((xr >> 8) & 0xFF) << (8 * m);
+                    pr[2] |= (uint32_t)((xr >> 16) & 0xFF) << (8 * m);
+                }
+            }
+#pragma unroll
+            for (int pl = 0; pl < 3; pl++) {
+                qA[gq].p[pl][r] = pa[pl];
+                qR[gq].p[pl][r] = pr[pl];
             }
         }
     }
@@ -429,10 +437,10 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
             }
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
-                const float A = fmaf(ma.y, QA[gq], ma.x * i2f_exact(dot_seg<BA>(ca, qpA[gq])));
+                const float A = fmaf(ma.y, QA[gq], ma.x * __int2float_rn(dot_seg<BA>(ca, qA[gq])));
                 float v = A;
                 if (RESID) {
-                    const float R = fmaf(mr.y, QR[gq], mr.x * i2f_exact(dot_seg<BR>(cr, qpR[gq])));
+                    const float R = fmaf(mr.y, QR[gq], mr.x * __int2float_rn(dot_seg<BR>(cr, qR[gq])));
                     v = fmaf(shat, A, R);
                 }
                 part[gq][k] = v;
@@ -444,8 +452,10 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
         const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
-            float r0 = (b4 ? part[gq][2] : part[gq][0]) + __shfl_xor_sync(0xffffffffu, b4 ? part[gq][0] : part[gq][2], 4);
-            float r1 = (b4 ? part[gq][3] : part[gq][1]) + __shfl_xor_sync(0xffffffffu, b4 ? part[gq][1] : part[gq][3], 4);
+            float r0 = (b4 ? part[gq][2] : part[gq][0]) +
+                       __shfl_xor_sync(0xffffffffu, b4 ? part[gq][0] : part[gq][2], 4);
+            float r1 = (b4 ? part[gq][3] : part[gq][1]) +
+                       __shfl_xor_sync(0xffffffffu, b4 ? part[gq][1] : part[gq][3], 4);
             float r = (b2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b2 ? r0 : r1, 2);
             r += __shfl_xor_sync(0xffffffffu, r, 1);
             r *= qinv;
@@ -476,25 +486,25 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
     for (int gq = 0; gq < GK; gq++)
         M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
     consumer_sync();   // everyone has read s_red
-    // p = exp2(z - M); the scores buffer is overwritten with P = p * s_hat(V);
-    // bounds of |s_hat| and of every group's scale for the fixed-point V weights
+    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V weight);
+    // bounds of |s_hat| and of every group's scale for the fixed-point weights
     float lsum[GK];
-    uint32_t cf_max = 0, sc_max_a = 0, sc_max_r = 0;   // |coef| bits, scale bytes (per group: thread's group = tid & 7)
+    uint32_t cf_max = 0, sc_max_a = 0, sc_max_r = 0;
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
-    const int G8 = 128 / a.g;   // groups per record
     for (int t = tid; t < n; t += kConsumers) {
-        const float shv = RESID ? bf16_to_f32(reinterpret_cast<const uint16_t *>(vm + L.vm_cf)[t]) : 1.f;
+        const uint16_t cf = RESID ? reinterpret_cast<const uint16_t *>(vm + L.vm_cf)[t] : (uint16_t)0x3F80;
+        const float shv = bf16_to_f32(cf);
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
             const float p = exp2f(s_sc[gq * a.chunk + t] - M[gq]);
             lsum[gq] += p;
-            s_sc[gq * a.chunk + t] = p;                       // residual V weight
-            s_P[gq * a.chunk + t] = p * shv;                  // anchor V weight (carries s_hat)
+            s_sc[gq * a.chunk + t] = p;
+            s_P[gq * a.chunk + t] = p * shv;
         }
-        if (RESID) cf_max = max(cf_max, (uint32_t)reinterpret_cast<const uint16_t *>(vm + L.vm_cf)[t] & 0x7FFFu);
+        cf_max = max(cf_max, (uint32_t)cf & 0x7FFFu);
     }
-    // scale-byte maxima: thread handles group (tid % G8) of tokens tid/G8, +128/G8, ...
+    const int G8 = kHeadDim / a.g;   // groups per record
     {
         const int grp = tid % G8;
         for (int t = tid / G8; t < n; t += kConsumers / G8) {
@@ -502,7 +512,6 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
             if (RESID) sc_max_r = max(sc_max_r, (uint32_t)vm[L.vm_r + t * L.MR + 2 * grp]);
         }
     }
-    // reduce: lsum over all; cf_max over all; scale maxima over threads with the same group
     {
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
@@ -538,100 +547,111 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
             sa = max(sa, __float_as_uint(s_red[w][2 * GK + mgrp]));
             sr = max(sr, __float_as_uint(s_red[w][2 * GK + 8 + mgrp]));
         }
-        const float shmax = RESID ? bf16_to_f32((uint16_t)cfm) : 1.f;
-        // the bound is an exact product of a BF16 and an FP8 value (<= 12
-        // significant bits), so bound * 2^F <= 2^15 - 8 and no rounded weight
-        // can reach 2^15
-        cA = fixed_scale(shmax * e4m3_to_f32(sa), 15);
-        cR = fixed_scale(e4m3_to_f32(sr), 15);
+        // weight <= |s_hat|max * scale max = bound; 2^F puts the bound into
+        // [2^29, 2^30): every rounded weight fits int32 with room to spare
+        cA = fixed_scale(bf16_to_f32((uint16_t)cfm) * e4m3_to_f32(sa), 30);
+        cR = fixed_scale(e4m3_to_f32(sr), 30);
     }
 
-    // ------------------------------------------------------------ pass 2: values
-    int accA[GK][16], accR[GK][16];
-    float mA[GK], mR[GK];
+    // ------------------------------------------------------------ pass 2: values (anchor, then residual)
+    const int npass = RESID ? 2 : 1;
+    for (int vp = 0; vp < npass; vp++) {
+        const float cW = vp == 0 ? cA : cR;
+        const float *wsrc = vp == 0 ? s_P : s_sc;
+        const uint8_t *vmeta = vm + (vp == 0 ? 0 : L.vm_r);
+        unsigned accLo[GK][16];
+        int accHi[GK][16];
+        float mS[GK];
 #pragma unroll
-    for (int gq = 0; gq < GK; gq++) {
-        mA[gq] = mR[gq] = 0.f;
+        for (int gq = 0; gq < GK; gq++) {
+            mS[gq] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; e++) accA[gq][e] = accR[gq][e] = 0;
-    }
-    for (int i = 0; i < ntiles; i++) {
-        const int it = ntiles + i;
-        const int stage = it % kStages;
-        if (!mbar_wait(&bar_full[stage], (it / kStages) & 1, &s_abort)) {
-            s_abort = 1;
-            atomicExch(a.err, 4);
+            for (int e = 0; e < 16; e++) {
+                accLo[gq][e] = 0u;
+                accHi[gq][e] = 0;
+            }
         }
-        const uint8_t *st = ring + stage * L.stage_bytes;
-        Seg<BA> ca[4];
-        Seg<BR> cr[4];
-        float P[GK][4], p[GK][4];
-        float2 ma[4], mr[4];
+        for (int i = 0; i < ntiles; i++) {
+            const int it = (1 + vp) * ntiles + i;
+            const int stage = it % kStages;
+            if (!mbar_wait(&bar_full[stage], (it / kStages) & 1, &s_abort)) {
+                s_abort = 1;
+                atomicExch(a.err, 4);
+            }
+            const uint8_t *st = ring + stage * L.stage_bytes;
+            uint32_t wlo[GK][2], whi[GK][2];
+            float2 mm[4];
+            float W[GK][4];
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-            const int tok = 16 * warp + sub + 4 * k;
-            const bool valid = (i * kTile + tok) < n;
-            const int tl = min(i * kTile + tok, n - 1);     // weights of tokens >= n are zero
-            ca[k] = lds_seg<BA>(st + tok * L.A_C + seg * (2 * BA));
-            ma[k] = meta_pair(*reinterpret_cast<const uint16_t *>(vm + tl * L.MR + 2 * mgrp));
-            if (RESID) {
-                cr[k] = lds_seg<BR>(st + L.v_rc + tok * L.R_C + seg * (2 * BR));
-                mr[k] = meta_pair(*reinterpret_cast<const uint16_t *>(vm + L.vm_r + tl * L.MR + 2 * mgrp));
+            for (int k = 0; k < 4; k++) {
+                const int tok = 16 * warp + sub + 4 * k;
+                const bool valid = (i * kTile + tok) < n;
+                const int tl = min(i * kTile + tok, n - 1);     // weights of tokens >= n are zero
+                mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(vmeta + tl * L.MR + 2 * mgrp));
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) W[gq][k] = valid ? wsrc[gq * a.chunk + tl] : 0.f;
             }
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
-                P[gq][k] = valid ? s_P[gq * a.chunk + tl] : 0.f;
-                p[gq][k] = valid ? s_sc[gq * a.chunk + tl] : 0.f;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_empty[stage]);
-#pragma unroll
-        for (int gq = 0; gq < GK; gq++) {
-            uint32_t wa[4], wr[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                wa[k] = fix16_bits_fma(P[gq][k] * cA, ma[k].x);
-                mA[gq] = fmaf(P[gq][k], ma[k].y, mA[gq]);
-            }
-            acc_pair<BA>(ca[0], ca[1], __byte_perm(wa[0], wa[1], 0x5410), accA[gq]);
-            acc_pair<BA>(ca[2], ca[3], __byte_perm(wa[2], wa[3], 0x5410), accA[gq]);
-            if (RESID) {
+                int wi[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    wr[k] = fix16_bits_fma(p[gq][k] * cR, mr[k].x);
-                    mR[gq] = fmaf(p[gq][k], mr[k].y, mR[gq]);
+                    wi[k] = __float2int_rn(W[gq][k] * cW * mm[k].x);
+                    mS[gq] = fmaf(W[gq][k], mm[k].y, mS[gq]);
                 }
-                acc_pair<BR>(cr[0], cr[1], __byte_perm(wr[0], wr[1], 0x5410), accR[gq]);
-                acc_pair<BR>(cr[2], cr[3], __byte_perm(wr[2], wr[3], 0x5410), accR[gq]);
+#pragma unroll
+                for (int pr = 0; pr < 2; pr++) {
+                    wlo[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x5410);
+                    whi[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x7632);
+                }
+            }
+            if (vp == 0) {
+                Seg<BA> c[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) c[k] = lds_seg<BA>(st + (16 * warp + sub + 4 * k) * L.A_C + seg * (2 * BA));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_empty[stage]);
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) {
+                    acc_pair<BA>(c[0], c[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                    acc_pair<BA>(c[2], c[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                }
+            } else {
+                Seg<BR> c[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) c[k] = lds_seg<BR>(st + (16 * warp + sub + 4 * k) * L.R_C + seg * (2 * BR));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_empty[stage]);
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) {
+                    acc_pair<BR>(c[0], c[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                    acc_pair<BR>(c[2], c[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                }
+            }
+        }
+        // fixed point -> fp32, minimum term, reduce over sub-groups (lanes xor 8, 16)
+        const float iW = 1.f / cW;
+#pragma unroll
+        for (int gq = 0; gq < GK; gq++) {
+#pragma unroll
+            for (int e = 0; e < 16; e++) {
+                float v = fmaf((float)accHi[gq][e], 65536.f, (float)accLo[gq][e]);
+                v = fmaf(v, iW, mS[gq]);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                if (sub == 0) s_acc[warp][gq][vp][seg * 16 + e] = v;
             }
         }
     }
 
-    // ------------------------------------------------------------ reduce and write the partial
-    const float iA = 1.f / cA, iR = 1.f / cR;
-#pragma unroll
-    for (int gq = 0; gq < GK; gq++) {
-#pragma unroll
-        for (int e = 0; e < 16; e++) {
-            float va = fmaf((float)accA[gq][e], iA, mA[gq]);
-            float vr = RESID ? fmaf((float)accR[gq][e], iR, mR[gq]) : 0.f;
-            va += __shfl_xor_sync(0xffffffffu, va, 8);
-            va += __shfl_xor_sync(0xffffffffu, va, 16);
-            vr += __shfl_xor_sync(0xffffffffu, vr, 8);
-            vr += __shfl_xor_sync(0xffffffffu, vr, 16);
-            if (sub == 0) {
-                s_acc[warp][gq][0][seg * 16 + e] = va;
-                s_acc[warp][gq][1][seg * 16 + e] = vr;
-            }
-        }
-    }
+    // ------------------------------------------------------------ reduce over warps, write the partial
     consumer_sync();
     float oA[GK], oR[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
         oA[gq] = s_acc[0][gq][0][tid] + s_acc[1][gq][0][tid] + s_acc[2][gq][0][tid] + s_acc[3][gq][0][tid];
-        oR[gq] = s_acc[0][gq][1][tid] + s_acc[1][gq][1][tid] + s_acc[2][gq][1][tid] + s_acc[3][gq][1][tid];
+        oR[gq] = RESID ? s_acc[0][gq][1][tid] + s_acc[1][gq][1][tid] + s_acc[2][gq][1][tid] + s_acc[3][gq][1][tid]
+                       : 0.f;
     }
     if (RESID && a.rotate) {
         // o += R^T o_rot = sigma . (H o_rot) / sqrt(d)
@@ -658,7 +678,7 @@ __global__ void __launch_bounds__(kThreads) decode_rq_kernel(const DecodeArgs a)
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
         float *part = a.partials + (((size_t)b * a.Hq + hq0 + gq) * a.splits_max + split) * kPartialStride;
-        part[tid] = oA[gq] + (RESID ? oR[gq] : 0.f);
+        part[tid] = oA[gq] + oR[gq];
         if (tid == 0) {
             part[kHeadDim] = M[gq];
             part[kHeadDim + 1] = Lsum[gq];
@@ -670,7 +690,7 @@ template <int GK, int BA, int BR, bool RESID>
 size_t smem_bytes(int g, int chunk) {
     const int A_C = 16 * BA, R_C = 16 * BR, MR = 256 / g;
     int k_bytes = kTile * (A_C + MR) + (RESID ? kTile * (R_C + MR + 2) : 0);
-    int v_bytes = kTile * A_C + (RESID ? kTile * R_C : 0);
+    int v_bytes = kTile * A_C;
     int stage = ((std::max(k_bytes, v_bytes) + 127) / 128) * 128;
     int vm = chunk * MR + (RESID ? chunk * (MR + 2) : 0);
     return (size_t)kStages * stage + ((vm + 127) / 128) * 128 + (size_t)2 * GK * chunk * sizeof(float);
