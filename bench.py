@@ -227,10 +227,14 @@ def run_ours(args, cfgd, rank, world, local_rank):
     t_end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     w0 = time.time()
+    if args.profile:
+        torch.cuda.cudart().cudaProfilerStart()   # ncu --profile-from-start off captures this region only
     t_start.record(stream)
     gK.replay()
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    if args.profile:
+        torch.cuda.cudart().cudaProfilerStop()
     w1 = time.time()
     clocks = None
     if sampler:
@@ -422,6 +426,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--json-out", default="")
+    ap.add_argument("--profile", action="store_true",
+                    help="bracket the timed region with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     args = ap.parse_args()
     if args.warmup < 3 and not args.layers:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
