@@ -1,5 +1,6 @@
 """Builds ``librq.so`` (the C-ABI library of include/rq.h) in-tree with nvcc
-for sm_100a.  Run ``python -m decode_attention_14_b200.build``."""
+for sm_100a.  Run ``python decode_attention_14_b200/build.py`` (standalone:
+it imports nothing from the package, whose import loads the library)."""
 from __future__ import annotations
 
 import os
