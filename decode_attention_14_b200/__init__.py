@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
     L.rq_decode_attn.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
     L.rq_decode_attn_bf16.restype = i32
     L.rq_decode_attn_bf16.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
+    L.rq_decode_attn_noalloc.restype = i32
+    L.rq_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
     L.rq_cache_length.restype = i32
     L.rq_cache_length.argtypes = [vp, i32, i32, ctypes.POINTER(i32)]
     L.rq_cache_tail_length.restype = i32
@@ -182,6 +184,11 @@ def rq_decode_attn(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0,
 def rq_decode_attn_bf16(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0, stream=None) -> int:
     return lib.rq_decode_attn_bf16(h, layer, loop, ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(out)),
                                    softmax_scale, ctypes.c_void_p(_stream(stream)))
+
+
+def rq_decode_attn_noalloc(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0, stream=None) -> int:
+    return lib.rq_decode_attn_noalloc(h, layer, loop, ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(out)),
+                                      softmax_scale, ctypes.c_void_p(_stream(stream)))
 
 
 def rq_cache_length(h, layer: int, group: int) -> int:

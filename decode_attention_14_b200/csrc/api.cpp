@@ -366,8 +366,11 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     return RQ_OK;
 }
 
+// partials == nullptr: the split partials go to the cache's own workspace
+// (stride splits_max).  Otherwise to `partials` (capacity partial_floats,
+// stride = the split count actually used).
 static int decode_common(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
-                         void *stream, bool bf16) {
+                         void *stream, bool bf16, float *partials = nullptr, size_t partial_floats = 0) {
     if (!c || !q || !out) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
@@ -418,6 +421,11 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
     choose_splits(c, a.T, units, resid ? 1 : 0, &a.S, &a.chunk);
+    if (partials) {
+        a.splits_max = std::max(a.S, 1);
+        if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;
+        a.partials = partials;
+    }
     if (a.S > 0) {
         cudaError_t e = bf16 ? launch_decode_bf16(a, st)
                              : launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st);
@@ -437,6 +445,18 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     cb.scale_log2 = a.scale_log2;
     return cuda_status(launch_combine(cb, st));
 }
+
+}  // extern "C"
+
+namespace rq {
+int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
+                        float *partials, size_t partial_floats) {
+    if (!partials) return RQ_ERR_INVALID;
+    return decode_common(c, layer, loop, q, out, scale, stream, false, partials, partial_floats);
+}
+}  // namespace rq
+
+extern "C" {
 
 int rq_decode_attn(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream) {
     return decode_common(c, layer, loop, q, out, scale, stream, false);

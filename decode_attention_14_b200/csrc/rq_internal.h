@@ -132,4 +132,9 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk);
 int decode_bf16_occupancy(int G, int chunk);
 
+// rq_decode_attn with the split partials written to caller-supplied device
+// scratch (capacity in floats) instead of the cache's workspace.
+int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
+                        float *partials, size_t partial_floats);
+
 }  // namespace rq

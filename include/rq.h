@@ -168,6 +168,27 @@ int rq_decode_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, flo
 int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
                         float softmax_scale, void *stream);
 
+/*
+ * rq_decode_attn without any allocation: identical arguments, results and
+ * errors, except that the split-combine partials go to a fixed array the
+ * library holds in device memory (8 MiB per GPU that loads the library, kept
+ * until process exit) instead of the cache's workspace.  The paper has no
+ * counterpart to this call; it is a deployment convenience.
+ *   For callers that must not allocate device memory after start-up: a plugin
+ *   inside a host framework that owns all device memory and offers no
+ *   allocator, a serving loop whose memory is planned once, or work issued
+ *   during stream capture, where allocation calls are refused.
+ *   Limit: batch * num_q_heads * S * 132 floats must fit in 2^21 floats, S
+ *   being the split count the call chooses (at most ceil(T/64)); beyond it the
+ *   call returns RQ_ERR_CAPACITY and enqueues nothing.
+ *   The first call on a device looks up the array's device address; make it
+ *   before any stream capture.  All calls on a device share the array: calls
+ *   whose GPU work overlaps race on it and must be ordered by the caller.
+ *   Format must be RQ_FMT_RESIDUAL (else RQ_ERR_STATE).
+ */
+int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
+                           float softmax_scale, void *stream);
+
 /* Committed length of (layer, group).  group = loop / loops_per_group for
  * the residual format; for the BF16 format pass the loop index. */
 int rq_cache_length(const rq_cache *cache, int layer, int group, int *len);
