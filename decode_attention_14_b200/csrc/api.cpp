@@ -148,7 +148,7 @@ bool make_layout(const rq_config &cfg, Layout *out) {
     L.off_partials = align_up(L.records_bytes, kAlign);
     size_t partial_bytes = align_up(B * Hq * (size_t)L.splits_max * kPartialStride * sizeof(float), kAlign);
     L.off_counters = L.off_partials + partial_bytes;
-    L.off_err = L.off_counters + align_up(B * H * sizeof(int), kAlign);
+    L.off_err = L.off_counters + align_up(B * Hq * sizeof(int), kAlign);
     L.total = L.off_err + kAlign;
     *out = L;
     return true;
@@ -369,8 +369,12 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
 // partials == nullptr: the split partials go to the cache's own workspace
 // (stride splits_max).  Otherwise to `partials` (capacity partial_floats,
 // stride = the split count actually used).
+// partials == nullptr: split partials and combine counters in the cache's
+// workspace (partial stride splits_max).  Otherwise in the caller's scratch
+// (stride = the split count this call uses).
 static int decode_common(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
-                         void *stream, bool bf16, float *partials = nullptr, size_t partial_floats = 0) {
+                         void *stream, bool bf16, float *partials = nullptr, size_t partial_floats = 0,
+                         int *counters = nullptr, size_t max_units = 0) {
     if (!c || !q || !out) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
@@ -380,7 +384,9 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
     a.q = (const uint16_t *)q;
+    a.out = out;
     a.partials = (float *)(c->base + L.off_partials);
+    a.counters = (int *)(c->base + L.off_counters);
     a.err = (int *)(c->base + L.off_err);
     a.B = cfg.batch;
     a.H = cfg.num_kv_heads;
@@ -391,10 +397,8 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     a.g = cfg.group_size;
     a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
     a.rotate = cfg.rotate;
+    a.tail_cap = L.tail_cap;
     std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
-    CombineArgs cb;
-    std::memset(&cb, 0, sizeof(cb));
-    int n_tail = 0;
     bool resid = false;
     if (bf16) {
         a.T = c->len[(size_t)layer * cfg.num_loops + loop];
@@ -414,9 +418,9 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
                 a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
                 a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, j, kv);
             }
-            n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
-            cb.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
-            cb.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
+            a.n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
+            a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
+            a.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
@@ -424,39 +428,34 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     if (partials) {
         a.splits_max = std::max(a.S, 1);
         if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;
+        if ((size_t)a.B * a.Hq > max_units) return RQ_ERR_CAPACITY;
         a.partials = partials;
+        a.counters = counters;
     }
-    if (a.S > 0) {
-        cudaError_t e = bf16 ? launch_decode_bf16(a, st)
-                             : launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st);
+    if (!bf16 && a.S > 0)   // the decode kernel merges its splits and the tail itself
+        return cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st));
+    if (bf16 && a.S > 0) {
+        cudaError_t e = launch_decode_bf16(a, st);
         if (e != cudaSuccess) return RQ_ERR_CUDA;
     }
+    CombineArgs cb;
+    std::memset(&cb, 0, sizeof(cb));
     cb.partials = a.partials;
     cb.q = a.q;
     cb.out = out;
+    cb.tail_k = a.tail_k;
+    cb.tail_v = a.tail_v;
     cb.B = a.B;
     cb.H = a.H;
     cb.Hq = a.Hq;
     cb.G = a.G;
     cb.S = a.S;
     cb.splits_max = a.splits_max;
-    cb.n_tail = n_tail;
+    cb.n_tail = a.n_tail;
     cb.tail_cap = L.tail_cap;
     cb.scale_log2 = a.scale_log2;
     return cuda_status(launch_combine(cb, st));
 }
-
-}  // extern "C"
-
-namespace rq {
-int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
-                        float *partials, size_t partial_floats) {
-    if (!partials) return RQ_ERR_INVALID;
-    return decode_common(c, layer, loop, q, out, scale, stream, false, partials, partial_floats);
-}
-}  // namespace rq
-
-extern "C" {
 
 int rq_decode_attn(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream) {
     return decode_common(c, layer, loop, q, out, scale, stream, false);

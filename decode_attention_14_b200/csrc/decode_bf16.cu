@@ -9,6 +9,7 @@
 // BF16 tail tokens.
 #include <math_constants.h>
 
+#include "combine.cuh"
 #include "common.cuh"
 #include "rq_internal.h"
 
@@ -134,42 +135,21 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     }
 }
 
-// One CTA per (sequence, query head): merges the split partials (m_s, l_s,
-// o_s) and then the BF16 tail tokens one by one with the online-softmax
-// rescaling rule, and writes o / l (zero when nothing was attended).
+struct BlockSync {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+
+// One CTA per (sequence, query head): merges the split partials and the BF16
+// tail tokens (combine_row) and writes o / l (zero when nothing was attended).
 __global__ void __launch_bounds__(128) combine_kernel(const CombineArgs a) {
     __shared__ float s_red[4];
-    const int hq = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hq = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const int h = hq / a.G;
-    float M = -CUDART_INF_F, l = 0.f, o = 0.f;
-    const float *part = a.partials + ((size_t)b * a.Hq + hq) * a.splits_max * kPartialStride;
-    for (int s = 0; s < a.S; s++) {
-        const float *p = part + (size_t)s * kPartialStride;
-        const float ms = p[kHeadDim], ls = p[kHeadDim + 1], os = p[tid];
-        const float nm = fmaxf(M, ms);
-        const float c0 = exp2f(M - nm), c1 = exp2f(ms - nm);
-        o = o * c0 + os * c1;
-        l = l * c0 + ls * c1;
-        M = nm;
-    }
-    if (a.n_tail > 0) {
-        const float q = bf16_to_f32(a.q[((size_t)b * a.Hq + hq) * kHeadDim + tid]) * a.scale_log2;
-        for (int j = 0; j < a.n_tail; j++) {
-            const size_t row = (((size_t)b * a.tail_cap + j) * a.H + h) * kHeadDim;
-            float z = q * bf16_to_f32(a.tail_k[row + tid]);
-            for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
-            __syncthreads();
-            if (lane == 0) s_red[warp] = z;
-            __syncthreads();
-            z = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-            const float nm = fmaxf(M, z);
-            const float c0 = exp2f(M - nm), c1 = exp2f(z - nm);
-            o = o * c0 + bf16_to_f32(a.tail_v[row + tid]) * c1;
-            l = l * c0 + c1;
-            M = nm;
-        }
-    }
-    a.out[((size_t)b * a.Hq + hq) * kHeadDim + tid] = (l > 0.f) ? o / l : 0.f;
+    const size_t row = (size_t)b * a.Hq + hq;
+    const size_t trow = ((size_t)b * a.tail_cap * a.H + h) * kHeadDim;
+    combine_row(a.partials + row * a.splits_max * kPartialStride, a.S, a.q + row * kHeadDim, a.scale_log2,
+                a.tail_k ? a.tail_k + trow : nullptr, a.tail_v ? a.tail_v + trow : nullptr, (size_t)a.H * kHeadDim,
+                a.n_tail, a.out + row * kHeadDim, tid, s_red, BlockSync());
 }
 
 }  // namespace

@@ -10,8 +10,8 @@
 // (FP8 scale sc, FP8 minimum mn, integer codes c):
 //   q_seg . x_hat_seg = mn * sum(q_seg) + sc * sum(q_i c_i)
 // The V sum is accumulated the same way: the anchor part in the original
-// basis, the residual part in the rotated basis, and R^T is applied once per
-// CTA to the rotated accumulator.
+// basis, the residual part in the rotated basis; R^T is applied once per CTA
+// to the rotated accumulator.
 //
 // Arithmetic.  The per-code products run on the integer dot-product units,
 // which consume packed codes with no conversion to floating point:
@@ -19,28 +19,34 @@
 //    (power-of-two scale, |q| < 2^22) split into three byte planes, and
 //    sum_i q_i c_i is three dp4a (4 products each) per 4 codes, exact;
 //  - values: each weight p_t s_t sc_{g,t} becomes 32-bit fixed point with a
-//    power-of-two scale per quantization group (the chunk's bound of the
-//    weight mapped into [2^29, 2^30)) split into 16-bit halves, and
-//    sum_t w_t c_t,i is two dp2a (2 products each) per 2 codes, exact.
-// The fixed-point rounding of q and of the weights is the only deviation from
-// fp32 arithmetic (relative 2^-21 of max|q|, 2^-29 of the weight bound).
+//    power-of-two scale chosen from a bound of every weight of the chunk
+//    (max |s_t| x 448, the largest FP8 scale; mapped into [2^29, 2^30)),
+//    split into 16-bit halves; sum_t w_t c_t,i is two dp2a (2 products each)
+//    per 2 codes, exact.
+// The fixed-point rounding of q and of the weights is the only departure from
+// fp32 arithmetic (relative 2^-21 of max|q|; absolute 2^-29 of the bound).
 // Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
-// Data movement.  Each CTA owns a chunk of one (sequence, kv head), streamed
-// in 64-token tiles through a 3-stage shared-memory ring filled by one
-// producer warp with 1-D bulk asynchronous copies (cp.async.bulk, completion
-// counted on mbarriers; no multicast).  Pass 1 streams the K records and
-// writes the chunk's logits; pass 2 streams the V codes (the V scales,
-// minima and coefficients were fetched once at CTA start) and sums
-// exp2(z - chunk max) * v.  Every mbarrier wait is bounded: on timeout the
-// kernel records an error word, stops issuing copies, drains what it issued
-// and finishes without touching further data.
+// Data movement.  Each CTA owns a chunk of one (sequence, kv head) and
+// streams it in 64-token items through a 4-stage shared-memory ring filled
+// by one producer warp with 1-D bulk asynchronous copies (cp.async.bulk,
+// completion counted on mbarriers; no multicast): first the K records of
+// every tile (pass 1: logits), then the anchor V codes + meta of every tile,
+// then the residual V codes + meta (pass 2: values).  Only the V coefficients
+// of the chunk (2 bytes per token) are fetched once up front.  Every mbarrier
+// wait is bounded: on timeout the kernel records an error word, stops issuing
+// copies, drains what it issued and finishes without touching further data.
 //
-// Thread map (pass 1 and 2): 4 consumer warps x 16 tokens of each tile;
+// Split combine.  Each CTA writes its partial (max, sum, o); the last CTA of
+// a (sequence, kv head) -- found with a device-wide counter, no waiting --
+// merges all partials plus the loop's BF16 tail tokens and writes the output.
+//
+// Thread map (both passes): 4 consumer warps x 16 tokens of each item;
 // lane 8s+j takes head_dim segment j (elements 16j..16j+15) of tokens
 // s, s+4, s+8, s+12 of its warp's 16.
 #include <math_constants.h>
 
+#include "combine.cuh"
 #include "common.cuh"
 #include "rq_internal.h"
 
@@ -48,7 +54,7 @@ namespace rq {
 namespace {
 
 constexpr int kTile = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
@@ -103,6 +109,10 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 }
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
 
+struct ConsumerSync {
+    __device__ __forceinline__ void operator()() const { consumer_sync(); }
+};
+
 // ---------------------------------------------------------------- codes
 // A 16-element segment: BITS=4 -> 2 words (elements 0-7, 8-15), BITS=2 -> 1 word.
 template <int BITS>
@@ -123,9 +133,8 @@ __device__ __forceinline__ Seg<BITS> lds_seg(const uint8_t *p) {
     return s;
 }
 
-// Byte lanes of the unpacked code words of a 16-element segment.  Unpacked
-// word r holds four codes, one per byte; elem_of<BITS>(r, m) is the segment
-// element in byte m of word r.
+// Unpacked code word r of a segment holds four codes, one per byte;
+// elem_of<BITS>(r, m) is the segment element in byte m of word r.
 //   BITS=4: r = 2u + hi: nibbles of word u; bytes = elements 8u + hi + {0,2,4,6}
 //   BITS=2: r = c: (w >> 2c) & 0x03030303; bytes = elements c + {0,4,8,12}
 template <int BITS>
@@ -140,7 +149,7 @@ __device__ __forceinline__ uint32_t unpack_word(const Seg<BITS> &s, int r) {
 }
 
 // q of one segment in 24-bit fixed point as three byte planes laid out like
-// the unpacked code words: plane 0 and 1 unsigned, plane 2 signed.
+// the unpacked code words: planes 0 and 1 unsigned, plane 2 signed.
 struct QPlanes {
     uint32_t p[3][4];
 };
@@ -172,8 +181,10 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
         for (int u = 0; u < 2; u++) {
             const uint32_t X = __byte_perm(a.w[u], b.w[u], 0x5140);   // bytes 0,1 of both tokens
             const uint32_t Y = __byte_perm(a.w[u], b.w[u], 0x7362);   // bytes 2,3 of both tokens
-            const uint32_t c[4] = {X & 0x0F0F0F0Fu, (X >> 4) & 0x0F0F0F0Fu, Y & 0x0F0F0F0Fu, (Y >> 4) & 0x0F0F0F0Fu};
-            // c[0]: elements 8u+0 (bytes 0,1), 8u+2 (bytes 2,3); c[1]: 8u+1, 8u+3; c[2]: 8u+4, 8u+6; c[3]: 8u+5, 8u+7
+            // c[0]: elements 8u+0 (bytes 0,1), 8u+2 (bytes 2,3); c[1]: 8u+1, 8u+3;
+            // c[2]: 8u+4, 8u+6; c[3]: 8u+5, 8u+7
+            const uint32_t c[4] = {X & 0x0F0F0F0Fu, (X >> 4) & 0x0F0F0F0Fu, Y & 0x0F0F0F0Fu,
+                                   (Y >> 4) & 0x0F0F0F0Fu};
             const int e0[4] = {0, 1, 4, 5};
 #pragma unroll
             for (int k = 0; k < 4; k++) {
@@ -218,46 +229,42 @@ __device__ __forceinline__ float fixed_scale(float bound, int top) {
     return ldexpf(1.f, F);
 }
 
-struct Layout2 {
-    int A_C, R_C, MR;
-    int k_am, k_rc, k_rm, k_cf, k_bytes;
-    int v_rc, v_bytes;
-    int stage_bytes;
-    int vm_r, vm_cf, vm_bytes;   // retained V meta: anchor meta, resid meta, coef
-    int sc_off;
+// Shared-memory plan of one CTA (bytes).  Items are 64 tokens.
+template <int BA, int BR, int GS, bool RESID>
+struct Plan {
+    static constexpr int A_C = 16 * BA;              // anchor codes per record
+    static constexpr int R_C = 16 * BR;              // residual codes per record
+    static constexpr int MR = 2 * (kHeadDim / GS);   // meta bytes per record
+    // K item: anchor codes | anchor meta | residual codes | residual meta | coefficients
+    static constexpr int K_AM = kTile * A_C;
+    static constexpr int K_RC = K_AM + kTile * MR;
+    static constexpr int K_RM = K_RC + (RESID ? kTile * R_C : 0);
+    static constexpr int K_CF = K_RM + (RESID ? kTile * MR : 0);
+    static constexpr int K_BYTES = K_CF + (RESID ? kTile * 2 : 0);
+    // V items: codes | meta, anchor items then residual items
+    static constexpr int VA_M = kTile * A_C;
+    static constexpr int VA_BYTES = VA_M + kTile * MR;
+    static constexpr int VR_M = kTile * R_C;
+    static constexpr int VR_BYTES = VR_M + kTile * MR;
+    static constexpr int STAGE = ((K_BYTES > VA_BYTES ? K_BYTES : VA_BYTES) + 127) / 128 * 128;
+    static constexpr int RING = kStages * STAGE;
+    // then: V coefficients [chunk] (RESID), logits/p [GK][chunk], p*s_hat [GK][chunk]
+    __host__ __device__ static int coef_bytes(int chunk) { return RESID ? (chunk * 2 + 127) / 128 * 128 : 0; }
+    __host__ __device__ static size_t smem(int GK, int chunk) {
+        return (size_t)RING + coef_bytes(chunk) + (size_t)2 * GK * chunk * sizeof(float);
+    }
 };
 
-template <int BA, int BR, bool RESID>
-__device__ __forceinline__ Layout2 make_layout2(int g, int chunk_tiles) {
-    Layout2 L;
-    L.A_C = 16 * BA;
-    L.R_C = 16 * BR;
-    L.MR = 256 / g;
-    L.k_am = kTile * L.A_C;
-    L.k_rc = L.k_am + kTile * L.MR;
-    L.k_rm = L.k_rc + (RESID ? kTile * L.R_C : 0);
-    L.k_cf = L.k_rm + (RESID ? kTile * L.MR : 0);
-    L.k_bytes = L.k_cf + (RESID ? kTile * 2 : 0);
-    L.v_rc = 0;                                   // residual V sub-pass stage: codes only
-    L.v_bytes = kTile * L.A_C;                    // anchor V sub-pass stage: codes only
-    L.stage_bytes = ((max(L.k_bytes, L.v_bytes) + 127) / 128) * 128;
-    const int ct = chunk_tiles * kTile;
-    L.vm_r = ct * L.MR;
-    L.vm_cf = L.vm_r + (RESID ? ct * L.MR : 0);
-    L.vm_bytes = L.vm_cf + (RESID ? ct * 2 : 0);
-    L.sc_off = kStages * L.stage_bytes + ((L.vm_bytes + 127) / 128) * 128;
-    return L;
-}
-
-template <int GK, int BA, int BR, bool RESID>
+template <int GK, int BA, int BR, int GS, bool RESID>
 __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs a) {
+    using P = Plan<BA, BR, GS, RESID>;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kStages];
     __shared__ __align__(8) uint64_t bar_empty[kStages];
-    __shared__ __align__(8) uint64_t bar_vm;
-    __shared__ int s_abort;
+    __shared__ __align__(8) uint64_t bar_cf;
+    __shared__ int s_abort, s_last;
     __shared__ float s_q[GK][2][kHeadDim];
-    __shared__ float s_red[4][2 * GK + 16];
+    __shared__ float s_red[4][2 * GK + 2];
     __shared__ float s_acc[4][GK][2][kHeadDim];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -268,20 +275,18 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
     const int t0 = split * a.chunk;
     const int n = min(a.chunk, a.T - t0);
     const int ntiles = (n + kTile - 1) / kTile;
-    const int chunk_tiles = a.chunk / kTile;
     const size_t bh = (size_t)b * a.H + h;
-    const Layout2 L = make_layout2<BA, BR, RESID>(a.g, chunk_tiles);
     uint8_t *ring = smem;
-    uint8_t *vm = smem + kStages * L.stage_bytes;
-    float *s_sc = reinterpret_cast<float *>(smem + L.sc_off);   // [GK][chunk] logits, then p
-    float *s_P = s_sc + GK * a.chunk;                           // [GK][chunk] p * s_hat(V)
+    const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);        // V coefficients
+    float *s_sc = reinterpret_cast<float *>(smem + P::RING + P::coef_bytes(a.chunk));  // [GK][chunk] logits -> p
+    float *s_P = s_sc + GK * a.chunk;                                                  // [GK][chunk] p * s_hat
 
     if (tid == 0) {
         for (int i = 0; i < kStages; i++) {
             mbar_init(&bar_full[i], 1);
             mbar_init(&bar_empty[i], 4);
         }
-        mbar_init(&bar_vm, 1);
+        mbar_init(&bar_cf, 1);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -291,19 +296,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
     if (warp == 4) {
         if (lane == 0) {
             const size_t tok0 = bh * a.Tp + (size_t)t0;
-            const uint32_t ntok = (uint32_t)(ntiles * kTile);
-            // V scales/minima (+ coefficients) of the whole chunk, fetched once
-            {
-                uint32_t bytes = ntok * L.MR + (RESID ? ntok * (L.MR + 2) : 0);
-                mbar_expect_tx(&bar_vm, bytes);
-                bulk_g2s(vm, a.a_meta[1] + tok0 * L.MR, ntok * L.MR, &bar_vm);
-                if (RESID) {
-                    bulk_g2s(vm + L.vm_r, a.r_meta[1] + tok0 * L.MR, ntok * L.MR, &bar_vm);
-                    bulk_g2s(vm + L.vm_cf, a.r_coef[1] + tok0, ntok * 2, &bar_vm);
-                }
+            if (RESID) {
+                mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
+                bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
             }
             int issued = 0;
-            const int nitems = (RESID ? 3 : 2) * ntiles;   // K tiles, V anchor tiles, V residual tiles
+            const int nitems = (RESID ? 3 : 2) * ntiles;   // K tiles, anchor V tiles, residual V tiles
             for (int it = 0; it < nitems; it++) {
                 const int stage = it % kStages;
                 if (it >= kStages && !mbar_wait(&bar_empty[stage], ((it / kStages) - 1) & 1, &s_abort)) {
@@ -311,29 +309,32 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
                     atomicExch(a.err, 1);
                     break;
                 }
-                uint8_t *st = ring + stage * L.stage_bytes;
+                uint8_t *st = ring + stage * P::STAGE;
+                uint64_t *bar = &bar_full[stage];
                 const int pass = it / ntiles;
                 const size_t tk = tok0 + (size_t)(it - pass * ntiles) * kTile;
                 if (pass == 0) {
-                    mbar_expect_tx(&bar_full[stage], (uint32_t)L.k_bytes);
-                    bulk_g2s(st, a.a_codes[0] + tk * L.A_C, kTile * L.A_C, &bar_full[stage]);
-                    bulk_g2s(st + L.k_am, a.a_meta[0] + tk * L.MR, kTile * L.MR, &bar_full[stage]);
+                    mbar_expect_tx(bar, (uint32_t)P::K_BYTES);
+                    bulk_g2s(st, a.a_codes[0] + tk * P::A_C, kTile * P::A_C, bar);
+                    bulk_g2s(st + P::K_AM, a.a_meta[0] + tk * P::MR, kTile * P::MR, bar);
                     if (RESID) {
-                        bulk_g2s(st + L.k_rc, a.r_codes[0] + tk * L.R_C, kTile * L.R_C, &bar_full[stage]);
-                        bulk_g2s(st + L.k_rm, a.r_meta[0] + tk * L.MR, kTile * L.MR, &bar_full[stage]);
-                        bulk_g2s(st + L.k_cf, a.r_coef[0] + tk, kTile * 2, &bar_full[stage]);
+                        bulk_g2s(st + P::K_RC, a.r_codes[0] + tk * P::R_C, kTile * P::R_C, bar);
+                        bulk_g2s(st + P::K_RM, a.r_meta[0] + tk * P::MR, kTile * P::MR, bar);
+                        bulk_g2s(st + P::K_CF, a.r_coef[0] + tk, kTile * 2, bar);
                     }
                 } else if (pass == 1) {
-                    mbar_expect_tx(&bar_full[stage], (uint32_t)(kTile * L.A_C));
-                    bulk_g2s(st, a.a_codes[1] + tk * L.A_C, kTile * L.A_C, &bar_full[stage]);
+                    mbar_expect_tx(bar, (uint32_t)P::VA_BYTES);
+                    bulk_g2s(st, a.a_codes[1] + tk * P::A_C, kTile * P::A_C, bar);
+                    bulk_g2s(st + P::VA_M, a.a_meta[1] + tk * P::MR, kTile * P::MR, bar);
                 } else {
-                    mbar_expect_tx(&bar_full[stage], (uint32_t)(kTile * L.R_C));
-                    bulk_g2s(st, a.r_codes[1] + tk * L.R_C, kTile * L.R_C, &bar_full[stage]);
+                    mbar_expect_tx(bar, (uint32_t)P::VR_BYTES);
+                    bulk_g2s(st, a.r_codes[1] + tk * P::R_C, kTile * P::R_C, bar);
+                    bulk_g2s(st + P::VR_M, a.r_meta[1] + tk * P::MR, kTile * P::MR, bar);
                 }
                 issued = it + 1;
             }
             // drain: every issued copy must have landed before the CTA exits
-            mbar_wait(&bar_vm, 0, &s_abort);
+            if (RESID) mbar_wait(&bar_cf, 0, &s_abort);
             for (int it = max(0, issued - kStages); it < issued; it++)
                 mbar_wait(&bar_full[it % kStages], (it / kStages) & 1, &s_abort);
         }
@@ -342,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
 
     // ------------------------------------------------------------ consumers
     const int sub = lane >> 3, seg = lane & 7;
-    const int mgrp = (seg * 16) / a.g;
+    const int mg = (seg * 16) / GS;   // quantization group of this lane's segment
 
-    // q (log2-domain scale folded in) and R q, then 16-bit fixed point
+    // q (log2-domain scale folded in) and R q, then 24-bit fixed-point planes
     for (int gq = 0; gq < GK; gq++)
         s_q[gq][0][tid] = bf16_to_f32(a.q[((size_t)b * a.Hq + hq0 + gq) * kHeadDim + tid]) * a.scale_log2;
     consumer_sync();
@@ -413,6 +414,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
     float mloc[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
+    const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
+    const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
     for (int i = 0; i < ntiles; i++) {
         const int stage = i % kStages;
         const bool ok = mbar_wait(&bar_full[stage], (i / kStages) & 1, &s_abort);
@@ -420,20 +423,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
             s_abort = 1;
             atomicExch(a.err, 2);
         }
-        const uint8_t *st = ring + stage * L.stage_bytes;
+        const uint8_t *st = ring + stage * P::STAGE;
         float part[GK][4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
             const int tok = 16 * warp + sub + 4 * k;
-            const Seg<BA> ca = lds_seg<BA>(st + tok * L.A_C + seg * (2 * BA));
-            const float2 ma = meta_pair(*reinterpret_cast<const uint16_t *>(st + L.k_am + tok * L.MR + 2 * mgrp));
+            const Seg<BA> ca = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
+            const float2 ma = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_AM + tok * P::MR + 2 * mg));
             float shat = 1.f;
             Seg<BR> cr;
             float2 mr = make_float2(0.f, 0.f);
             if (RESID) {
-                cr = lds_seg<BR>(st + L.k_rc + tok * L.R_C + seg * (2 * BR));
-                mr = meta_pair(*reinterpret_cast<const uint16_t *>(st + L.k_rm + tok * L.MR + 2 * mgrp));
-                shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + L.k_cf + 2 * tok));
+                cr = lds_seg<BR>(st + P::K_RC + tok * P::R_C + seg * (2 * BR));
+                mr = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_RM + tok * P::MR + 2 * mg));
+                shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + P::K_CF + 2 * tok));
             }
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
@@ -449,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_empty[stage]);
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
-        const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
+        const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
             float r0 = (b4 ? part[gq][2] : part[gq][0]) +
@@ -459,12 +462,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
             float r = (b2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b2 ? r0 : r1, 2);
             r += __shfl_xor_sync(0xffffffffu, r, 1);
             r *= qinv;
-            const int k = (b4 ? 2 : 0) + (b2 ? 1 : 0);
-            const int tl = i * kTile + 16 * warp + sub + 4 * k;
-            if (tl < n && ok) {
-                if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;
-                mloc[gq] = fmaxf(mloc[gq], r);
-            }
+            if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;   // tl < ntiles*64 <= chunk
+            if (tl < n && ok) mloc[gq] = fmaxf(mloc[gq], r);
         }
     }
 
@@ -475,8 +474,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
         for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
         if (lane == 0) s_red[warp][gq] = v;
     }
-    const bool vm_ok = mbar_wait(&bar_vm, 0, &s_abort);
-    if (!vm_ok) {
+    if (RESID && !mbar_wait(&bar_cf, 0, &s_abort)) {
         s_abort = 1;
         atomicExch(a.err, 3);
     }
@@ -486,71 +484,45 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
     for (int gq = 0; gq < GK; gq++)
         M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
     consumer_sync();   // everyone has read s_red
-    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V weight);
-    // bounds of |s_hat| and of every group's scale for the fixed-point weights
+    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V weight),
+    // zero beyond the chunk's tokens; the bound of |s_hat| for the fixed point
     float lsum[GK];
-    uint32_t cf_max = 0, sc_max_a = 0, sc_max_r = 0;
+    uint32_t cf_max = 0;
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
-    for (int t = tid; t < n; t += kConsumers) {
-        const uint16_t cf = RESID ? reinterpret_cast<const uint16_t *>(vm + L.vm_cf)[t] : (uint16_t)0x3F80;
+    for (int t = tid; t < ntiles * kTile; t += kConsumers) {
+        const bool valid = t < n;
+        const uint16_t cf = RESID ? s_cf[t] : (uint16_t)0x3F80;
         const float shv = bf16_to_f32(cf);
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
-            const float p = exp2f(s_sc[gq * a.chunk + t] - M[gq]);
+            const float p = valid ? exp2f(s_sc[gq * a.chunk + t] - M[gq]) : 0.f;
             lsum[gq] += p;
             s_sc[gq * a.chunk + t] = p;
             s_P[gq * a.chunk + t] = p * shv;
         }
-        cf_max = max(cf_max, (uint32_t)cf & 0x7FFFu);
+        if (valid) cf_max = max(cf_max, (uint32_t)cf & 0x7FFFu);
     }
-    const int G8 = kHeadDim / a.g;   // groups per record
-    {
-        const int grp = tid % G8;
-        for (int t = tid / G8; t < n; t += kConsumers / G8) {
-            sc_max_a = max(sc_max_a, (uint32_t)vm[t * L.MR + 2 * grp]);
-            if (RESID) sc_max_r = max(sc_max_r, (uint32_t)vm[L.vm_r + t * L.MR + 2 * grp]);
-        }
-    }
-    {
 #pragma unroll
-        for (int gq = 0; gq < GK; gq++) {
-            float v = lsum[gq];
-            for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-            lsum[gq] = v;
-        }
-        for (int m = 16; m >= 1; m >>= 1) cf_max = max(cf_max, __shfl_xor_sync(0xffffffffu, cf_max, m));
-        for (int m = 16; m >= G8; m >>= 1) {
-            sc_max_a = max(sc_max_a, __shfl_xor_sync(0xffffffffu, sc_max_a, m));
-            sc_max_r = max(sc_max_r, __shfl_xor_sync(0xffffffffu, sc_max_r, m));
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int gq = 0; gq < GK; gq++) s_red[warp][gq] = lsum[gq];
-            s_red[warp][GK] = __uint_as_float(cf_max);
-        }
-        if (lane < G8) {
-            s_red[warp][2 * GK + lane] = __uint_as_float(sc_max_a);
-            s_red[warp][2 * GK + 8 + lane] = __uint_as_float(sc_max_r);
-        }
+    for (int gq = 0; gq < GK; gq++) {
+        float v = lsum[gq];
+        for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+        if (lane == 0) s_red[warp][gq] = v;
     }
+    for (int m = 16; m >= 1; m >>= 1) cf_max = max(cf_max, __shfl_xor_sync(0xffffffffu, cf_max, m));
+    if (lane == 0) s_red[warp][GK] = __uint_as_float(cf_max);
     consumer_sync();
     float Lsum[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) Lsum[gq] = s_red[0][gq] + s_red[1][gq] + s_red[2][gq] + s_red[3][gq];
-    float cA, cR;   // fixed-point scales of this lane's group: anchor and residual V weights
+    // weights w = P * sc (anchor) or p * sc (residual), |P| <= max|s_hat|, p <= 1, sc <= 448
+    float cA, cR;
     {
-        uint32_t cfm = 0, sa = 0, sr = 0;
+        uint32_t cfm = 0;
 #pragma unroll
-        for (int w = 0; w < 4; w++) {
-            cfm = max(cfm, __float_as_uint(s_red[w][GK]));
-            sa = max(sa, __float_as_uint(s_red[w][2 * GK + mgrp]));
-            sr = max(sr, __float_as_uint(s_red[w][2 * GK + 8 + mgrp]));
-        }
-        // weight <= |s_hat|max * scale max = bound; 2^F puts the bound into
-        // [2^29, 2^30): every rounded weight fits int32 with room to spare
-        cA = fixed_scale(bf16_to_f32((uint16_t)cfm) * e4m3_to_f32(sa), 30);
-        cR = fixed_scale(e4m3_to_f32(sr), 30);
+        for (int w = 0; w < 4; w++) cfm = max(cfm, __float_as_uint(s_red[w][GK]));
+        cA = fixed_scale(bf16_to_f32((uint16_t)cfm) * 448.f, 30);
+        cR = fixed_scale(448.f, 30);
     }
 
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
@@ -558,7 +530,6 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
     for (int vp = 0; vp < npass; vp++) {
         const float cW = vp == 0 ? cA : cR;
         const float *wsrc = vp == 0 ? s_P : s_sc;
-        const uint8_t *vmeta = vm + (vp == 0 ? 0 : L.vm_r);
         unsigned accLo[GK][16];
         int accHi[GK][16];
         float mS[GK];
@@ -578,19 +549,27 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
                 s_abort = 1;
                 atomicExch(a.err, 4);
             }
-            const uint8_t *st = ring + stage * L.stage_bytes;
+            const uint8_t *st = ring + stage * P::STAGE;
             uint32_t wlo[GK][2], whi[GK][2];
             float2 mm[4];
             float W[GK][4];
+            Seg<BA> ca[4];
+            Seg<BR> cr[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 const int tok = 16 * warp + sub + 4 * k;
-                const bool valid = (i * kTile + tok) < n;
-                const int tl = min(i * kTile + tok, n - 1);     // weights of tokens >= n are zero
-                mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(vmeta + tl * L.MR + 2 * mgrp));
+                if (vp == 0) {
+                    ca[k] = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
+                    mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VA_M + tok * P::MR + 2 * mg));
+                } else {
+                    cr[k] = lds_seg<BR>(st + tok * P::R_C + seg * (2 * BR));
+                    mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VR_M + tok * P::MR + 2 * mg));
+                }
 #pragma unroll
-                for (int gq = 0; gq < GK; gq++) W[gq][k] = valid ? wsrc[gq * a.chunk + tl] : 0.f;
+                for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + i * kTile + tok];
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_empty[stage]);
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
                 int wi[4];
@@ -604,28 +583,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
                     wlo[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x5410);
                     whi[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x7632);
                 }
-            }
-            if (vp == 0) {
-                Seg<BA> c[4];
-#pragma unroll
-                for (int k = 0; k < 4; k++) c[k] = lds_seg<BA>(st + (16 * warp + sub + 4 * k) * L.A_C + seg * (2 * BA));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar_empty[stage]);
-#pragma unroll
-                for (int gq = 0; gq < GK; gq++) {
-                    acc_pair<BA>(c[0], c[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                    acc_pair<BA>(c[2], c[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
-                }
-            } else {
-                Seg<BR> c[4];
-#pragma unroll
-                for (int k = 0; k < 4; k++) c[k] = lds_seg<BR>(st + (16 * warp + sub + 4 * k) * L.R_C + seg * (2 * BR));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar_empty[stage]);
-#pragma unroll
-                for (int gq = 0; gq < GK; gq++) {
-                    acc_pair<BR>(c[0], c[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                    acc_pair<BR>(c[2], c[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                if (vp == 0) {
+                    acc_pair<BA>(ca[0], ca[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                    acc_pair<BA>(ca[2], ca[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                } else {
+                    acc_pair<BR>(cr[0], cr[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                    acc_pair<BR>(cr[2], cr[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
                 }
             }
         }
@@ -684,76 +647,99 @@ __global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs
             part[kHeadDim + 1] = Lsum[gq];
         }
     }
+
+    // ------------------------------------------------------------ last CTA of the unit combines
+    __threadfence();
+    consumer_sync();
+    const int unit = (b * a.H + h) * npairs + pair;
+    if (tid == 0) s_last = (atomicAdd(&a.counters[unit], 1) == a.S - 1);
+    consumer_sync();
+    if (s_last) {
+        __threadfence();
+        if (tid == 0) a.counters[unit] = 0;   // ready for the next call
+#pragma unroll 1
+        for (int gq = 0; gq < GK; gq++) {
+            const size_t row = (size_t)b * a.Hq + hq0 + gq;
+            const size_t trow = ((size_t)b * a.tail_cap * a.H + h) * kHeadDim;
+            combine_row(a.partials + row * a.splits_max * kPartialStride, a.S, a.q + row * kHeadDim, a.scale_log2,
+                        a.tail_k ? a.tail_k + trow : nullptr, a.tail_v ? a.tail_v + trow : nullptr,
+                        (size_t)a.H * kHeadDim, a.n_tail, a.out + row * kHeadDim, tid, &s_red[0][0],
+                        ConsumerSync());
+        }
+    }
 }
 
-template <int GK, int BA, int BR, bool RESID>
-size_t smem_bytes(int g, int chunk) {
-    const int A_C = 16 * BA, R_C = 16 * BR, MR = 256 / g;
-    int k_bytes = kTile * (A_C + MR) + (RESID ? kTile * (R_C + MR + 2) : 0);
-    int v_bytes = kTile * A_C;
-    int stage = ((std::max(k_bytes, v_bytes) + 127) / 128) * 128;
-    int vm = chunk * MR + (RESID ? chunk * (MR + 2) : 0);
-    return (size_t)kStages * stage + ((vm + 127) / 128) * 128 + (size_t)2 * GK * chunk * sizeof(float);
-}
-
-template <int GK, int BA, int BR, bool RESID>
+template <int GK, int BA, int BR, int GS, bool RESID>
 cudaError_t configure() {
     static bool configured = false;   // the largest dynamic shared memory any launch can ask for
     if (configured) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, RESID>,
+    cudaError_t e = cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<GK, BA, BR, RESID>(16, kMaxChunk));
+                                         (int)Plan<BA, BR, GS, RESID>::smem(GK, kMaxChunk));
     if (e == cudaSuccess) configured = true;
     return e;
 }
 
-template <int GK, int BA, int BR, bool RESID>
+template <int GK, int BA, int BR, int GS, bool RESID>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
     const dim3 grid(a.S, a.H, a.B * (a.G / GK));
-    const size_t smem = smem_bytes<GK, BA, BR, RESID>(a.g, a.chunk);
-    cudaError_t e = configure<GK, BA, BR, RESID>();
+    cudaError_t e = configure<GK, BA, BR, GS, RESID>();
     if (e != cudaSuccess) return e;
-    decode_rq_kernel<GK, BA, BR, RESID><<<grid, kThreads, smem, st>>>(a);
+    decode_rq_kernel<GK, BA, BR, GS, RESID>
+        <<<grid, kThreads, Plan<BA, BR, GS, RESID>::smem(GK, a.chunk), st>>>(a);
     return cudaGetLastError();
 }
 
-template <int GK, int BA, int BR, bool RESID>
-int occupancy_t(int g, int chunk) {
-    if (configure<GK, BA, BR, RESID>() != cudaSuccess) return 1;
+template <int GK, int BA, int BR, int GS, bool RESID>
+int occupancy_t(int chunk) {
+    if (configure<GK, BA, BR, GS, RESID>() != cudaSuccess) return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, RESID>, kThreads,
-                                                      smem_bytes<GK, BA, BR, RESID>(g, chunk)) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, RESID>, kThreads,
+                                                      Plan<BA, BR, GS, RESID>::smem(GK, chunk)) != cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
 }
 
-template <int GK>
-int occupancy_g(int ba, int br, bool resid, int g, int chunk) {
-    if (!resid) return ba == 4 ? occupancy_t<GK, 4, 2, false>(g, chunk) : occupancy_t<GK, 2, 2, false>(g, chunk);
-    if (ba == 4 && br == 2) return occupancy_t<GK, 4, 2, true>(g, chunk);
-    if (ba == 4 && br == 4) return occupancy_t<GK, 4, 4, true>(g, chunk);
-    if (ba == 2 && br == 2) return occupancy_t<GK, 2, 2, true>(g, chunk);
-    return occupancy_t<GK, 2, 4, true>(g, chunk);
-}
+// Variant dispatch: one instantiation per (q heads per CTA, bits, group, loop kind).
+template <int GK, int GS>
+struct Dispatch {
+    template <typename F>
+    static auto run(int ba, int br, bool resid, F f) {
+        if (!resid) return ba == 4 ? f.template go<GK, 4, 2, GS, false>() : f.template go<GK, 2, 2, GS, false>();
+        if (ba == 4 && br == 2) return f.template go<GK, 4, 2, GS, true>();
+        if (ba == 4 && br == 4) return f.template go<GK, 4, 4, GS, true>();
+        if (ba == 2 && br == 2) return f.template go<GK, 2, 2, GS, true>();
+        return f.template go<GK, 2, 4, GS, true>();
+    }
+};
 
-template <int GK>
-cudaError_t launch_g(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st) {
-    if (!resid) return ba == 4 ? launch_t<GK, 4, 2, false>(a, st) : launch_t<GK, 2, 2, false>(a, st);
-    if (ba == 4 && br == 2) return launch_t<GK, 4, 2, true>(a, st);
-    if (ba == 4 && br == 4) return launch_t<GK, 4, 4, true>(a, st);
-    if (ba == 2 && br == 2) return launch_t<GK, 2, 2, true>(a, st);
-    return launch_t<GK, 2, 4, true>(a, st);
+struct LaunchF {
+    const DecodeArgs *a;
+    cudaStream_t st;
+    template <int GK, int BA, int BR, int GS, bool RESID>
+    cudaError_t go() const { return launch_t<GK, BA, BR, GS, RESID>(*a, st); }
+};
+struct OccF {
+    int chunk;
+    template <int GK, int BA, int BR, int GS, bool RESID>
+    int go() const { return occupancy_t<GK, BA, BR, GS, RESID>(chunk); }
+};
+
+template <typename F>
+auto dispatch(int G, int g, int ba, int br, bool resid, F f) {
+    if (G == 1) return g == 16 ? Dispatch<1, 16>::run(ba, br, resid, f) : Dispatch<1, 32>::run(ba, br, resid, f);
+    return g == 16 ? Dispatch<2, 16>::run(ba, br, resid, f) : Dispatch<2, 32>::run(ba, br, resid, f);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st) {
-    if (a.G == 1) return launch_g<1>(a, ba, br, resid, st);
-    return launch_g<2>(a, ba, br, resid, st);   // G = 2, 4, 8: pairs of query heads
+    // G = 2, 4, 8 run as pairs of query heads per CTA
+    return dispatch(a.G, a.g, ba, br, resid, LaunchF{&a, st});
 }
 
 int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk) {
-    return G == 1 ? occupancy_g<1>(ba, br, resid, g, chunk) : occupancy_g<2>(ba, br, resid, g, chunk);
+    return dispatch(G, g, ba, br, resid, OccF{chunk});
 }
 
 }  // namespace rq

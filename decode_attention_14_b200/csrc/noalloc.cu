@@ -16,15 +16,19 @@
 // current) and caches it; make that first call before any stream capture.
 // All calls on a device share the one array and it keeps the last call's
 // contents: calls whose GPU work overlaps (other streams, other threads) race
-// on it and must be ordered by the caller.  Nothing in it needs to start at
-// zero: every partial slot is written before it is read within a call.
+// on it and must be ordered by the caller.  The split partials need no
+// clearing (each slot is written before it is read within a call); the last
+// 64 Ki words hold the split-combine counters, zeroed once at set-up and
+// returned to zero by every call.
 #include <mutex>
 
 #include "rq_internal.h"
 
 namespace {
 
-constexpr size_t kScratchFloats = size_t(2) << 20;   // 2 Mi floats = 8 MiB
+constexpr size_t kScratchFloats = size_t(2) << 20;   // 2 Mi floats = 8 MiB in all
+constexpr size_t kCounterInts = 65536;               // combine counters, at the end of the array
+constexpr size_t kPartialFloats = kScratchFloats - kCounterInts;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_decode_scratch[kScratchFloats];
@@ -44,6 +48,12 @@ int scratch_for_current_device(float **out) {
             cudaGetLastError();
             return RQ_ERR_CUDA;
         }
+        // the combine counters must start at zero (each call leaves them at zero)
+        if (cudaMemset(static_cast<float *>(p) + kPartialFloats, 0, kCounterInts * sizeof(int)) != cudaSuccess ||
+            cudaDeviceSynchronize() != cudaSuccess) {
+            cudaGetLastError();
+            return RQ_ERR_CUDA;
+        }
         g_scratch_ptr[dev] = static_cast<float *>(p);
     }
     *out = g_scratch_ptr[dev];
@@ -58,5 +68,6 @@ extern "C" int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, cons
     float *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);
     if (st != RQ_OK) return st;
-    return rq::decode_with_scratch(cache, layer, loop, q_bf16, out, softmax_scale, stream, scratch, kScratchFloats);
+    return rq::decode_with_scratch(cache, layer, loop, q_bf16, out, softmax_scale, stream, scratch, kPartialFloats,
+                                   reinterpret_cast<int *>(scratch + kPartialFloats), kCounterInts);
 }

@@ -105,7 +105,11 @@ struct DecodeArgs {
     const uint16_t *bf[2];
     const uint16_t *q;        // [B][Hq][d] bf16
     float *partials;          // [B][Hq][splits_max][kPartialStride]
+    int *counters;            // [B * Hq] arrival counters of the fused split combine (zero between calls)
     int *err;                 // device error word (bounded waits that gave up)
+    float *out;               // [B][Hq][d] fp32
+    const uint16_t *tail_k, *tail_v;   // [B][tail_cap][H][d] BF16 in-flight tokens, or null
+    int n_tail, tail_cap;
     int B, H, Hq, G, T, Tp, S, chunk, splits_max;
     int g;
     float scale_log2;         // softmax_scale * log2(e)
@@ -132,9 +136,11 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk);
 int decode_bf16_occupancy(int G, int chunk);
 
-// rq_decode_attn with the split partials written to caller-supplied device
-// scratch (capacity in floats) instead of the cache's workspace.
+// rq_decode_attn with the split partials and the combine counters in
+// caller-supplied device scratch instead of the cache's workspace: `partials`
+// holds partial_floats floats, `counters` max_units ints that are zero
+// between calls.
 int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
-                        float *partials, size_t partial_floats);
+                        float *partials, size_t partial_floats, int *counters, size_t max_units);
 
 }  // namespace rq
