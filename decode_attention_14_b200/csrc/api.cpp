@@ -457,6 +457,19 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     return cuda_status(launch_combine(cb, st));
 }
 
+}  // extern "C"
+
+namespace rq {
+int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
+                        float *partials, size_t partial_floats, int *counters, size_t max_units) {
+    if (!partials || !counters) return RQ_ERR_INVALID;
+    return decode_common(c, layer, loop, q, out, scale, stream, false, partials, partial_floats, counters,
+                         max_units);
+}
+}  // namespace rq
+
+extern "C" {
+
 int rq_decode_attn(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream) {
     return decode_common(c, layer, loop, q, out, scale, stream, false);
 }
