@@ -28,7 +28,7 @@
 // Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
 // Data movement.  Each CTA owns a chunk of one (sequence, kv head) and
-// streams it in 64-token items through a 4-stage shared-memory ring filled
+// streams it in 64-token items through a 3-stage shared-memory ring filled
 // by one producer warp with 1-D bulk asynchronous copies (cp.async.bulk,
 // completion counted on mbarriers; no multicast): first the K records of
 // every tile (pass 1: logits), then the anchor V codes + meta of every tile,
@@ -54,7 +54,7 @@ namespace rq {
 namespace {
 
 constexpr int kTile = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
@@ -256,7 +256,7 @@ struct Plan {
 };
 
 template <int GK, int BA, int BR, int GS, bool RESID>
-__global__ void __launch_bounds__(kThreads, 3) decode_rq_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, GK == 1 ? 5 : 3) decode_rq_kernel(const DecodeArgs a) {
     using P = Plan<BA, BR, GS, RESID>;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kStages];
