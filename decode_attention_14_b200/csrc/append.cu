@@ -4,8 +4,9 @@
 // to the residuals only, INT4 anchor / INT2 residuals; paragraph 2: group
 // size 16 with FP8 scales and offsets, BF16 least-squares coefficients).
 //
-// One warp encodes one (K|V, sequence, token, kv head): lane l holds the four
-// head_dim elements 4l..4l+3.  Every encoding decision (group min/max, the
+// One warp encodes one record (the anchor or one loop's residual) of one
+// (K|V, sequence, token, kv head): lane l holds the four head_dim elements
+// 4l..4l+3.  Every encoding decision (group min/max, the
 // scale and minimum before their FP8 rounding, the code quotient, the
 // least-squares coefficient before its BF16 rounding, the rotated residual)
 // is computed in fp64, so the integer codes come out the same as from an
@@ -80,13 +81,20 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
+// One warp per record: (K|V, sequence, token, kv head, j), j < nres the
+// residual of loop j, j == nres the anchor.  Every warp re-derives the anchor
+// (a few fp64 operations) so that the records of one token are encoded in
+// parallel rather than one after another.
 __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     const int lane = threadIdx.x & 31;
     const long long wid = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
-    const long long total = 2LL * a.B * a.n * a.H;
+    const int nrec = a.nres + 1;
+    const long long total = 2LL * a.B * a.n * a.H * nrec;
     if (wid >= total) return;   // uniform per warp
-    const int h = (int)(wid % a.H);
-    long long r = wid / a.H;
+    const int j = (int)(wid % nrec);
+    long long r = wid / nrec;
+    const int h = (int)(r % a.H);
+    r /= a.H;
     const int t = (int)(r % a.n);
     r /= a.n;
     const int b = (int)(r % a.B);
@@ -99,50 +107,51 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     const uint32_t apack = quantize4(x, a.ba, a.g, lane, ahat, &s8, &m8);
     const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0 + t);
     const int meta_rec = 2 * (kHeadDim / a.g);
-    uint8_t *ac = a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8);
-    uint8_t *am = a.a_meta0 + kv * a.anchor_kv_stride + rec * meta_rec;
-    store_record(ac, am, apack, s8, m8, a.ba, a.g, lane);
+    if (j == a.nres) {
+        uint8_t *ac = a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8);
+        uint8_t *am = a.a_meta0 + kv * a.anchor_kv_stride + rec * meta_rec;
+        store_record(ac, am, apack, s8, m8, a.ba, a.g, lane);
+        return;
+    }
 
     double aa = 0.0;
 #pragma unroll
     for (int k = 0; k < 4; k++) aa = __dadd_rn(aa, __dmul_rn(ahat[k], ahat[k]));
     const double den = warp_sum(aa);
 
-    for (int j = 0; j < a.nres; j++) {
-        const uint16_t *tail = reinterpret_cast<const uint16_t *>(a.tail0 + j * a.tail_loop_stride +
-                                                                   kv * a.tail_kv_stride);
-        double xl[4];
-        load4_bf16(tail + (((size_t)b * a.tail_cap + t) * a.H + h) * kHeadDim + lane * 4, xl);
-        // least-squares coefficient against the dequantized anchor, stored in BF16
-        double xa = 0.0;
+    const uint16_t *tail = reinterpret_cast<const uint16_t *>(a.tail0 + j * a.tail_loop_stride +
+                                                               kv * a.tail_kv_stride);
+    double xl[4];
+    load4_bf16(tail + (((size_t)b * a.tail_cap + t) * a.H + h) * kHeadDim + lane * 4, xl);
+    // least-squares coefficient against the dequantized anchor, stored in BF16
+    double xa = 0.0;
 #pragma unroll
-        for (int k = 0; k < 4; k++) xa = __dadd_rn(xa, __dmul_rn(xl[k], ahat[k]));
-        const double num = warp_sum(xa);
-        const double s = (den != 0.0) ? __ddiv_rn(num, den) : 0.0;
-        const __nv_bfloat16 sb = __double2bfloat16(s);
-        const double sh = (double)__bfloat162float(sb);
-        // residual with the stored coefficient, then y = R r = H (sigma . r) / sqrt(d)
-        double y[4];
+    for (int k = 0; k < 4; k++) xa = __dadd_rn(xa, __dmul_rn(xl[k], ahat[k]));
+    const double num = warp_sum(xa);
+    const double s = (den != 0.0) ? __ddiv_rn(num, den) : 0.0;
+    const __nv_bfloat16 sb = __double2bfloat16(s);
+    const double sh = (double)__bfloat162float(sb);
+    // residual with the stored coefficient, then y = R r = H (sigma . r) / sqrt(d)
+    double y[4];
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-            double rr = __dsub_rn(xl[k], __dmul_rn(sh, ahat[k]));
-            if (a.rotate && sigma_neg(a.sigma, lane * 4 + k)) rr = -rr;
-            y[k] = rr;
-        }
-        if (a.rotate) {
-            wht128_warp<double>(y, lane);
+    for (int k = 0; k < 4; k++) {
+        double rr = __dsub_rn(xl[k], __dmul_rn(sh, ahat[k]));
+        if (a.rotate && sigma_neg(a.sigma, lane * 4 + k)) rr = -rr;
+        y[k] = rr;
+    }
+    if (a.rotate) {
+        wht128_warp<double>(y, lane);
 #pragma unroll
-            for (int k = 0; k < 4; k++) y[k] = __dmul_rn(y[k], kInvSqrt128);
-        }
-        double yhat[4];
-        const uint32_t rpack = quantize4(y, a.br, a.g, lane, yhat, &s8, &m8);
-        uint8_t *rc = a.r_codes0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * (kHeadDim * a.br / 8);
-        uint8_t *rm = a.r_meta0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * meta_rec;
-        store_record(rc, rm, rpack, s8, m8, a.br, a.g, lane);
-        if (lane == 0) {
-            uint16_t *rf = reinterpret_cast<uint16_t *>(a.r_coef0 + j * a.resid_loop_stride + kv * a.resid_kv_stride);
-            rf[rec] = __bfloat16_as_ushort(sb);
-        }
+        for (int k = 0; k < 4; k++) y[k] = __dmul_rn(y[k], kInvSqrt128);
+    }
+    double yhat[4];
+    const uint32_t rpack = quantize4(y, a.br, a.g, lane, yhat, &s8, &m8);
+    uint8_t *rc = a.r_codes0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * (kHeadDim * a.br / 8);
+    uint8_t *rm = a.r_meta0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * meta_rec;
+    store_record(rc, rm, rpack, s8, m8, a.br, a.g, lane);
+    if (lane == 0) {
+        uint16_t *rf = reinterpret_cast<uint16_t *>(a.r_coef0 + j * a.resid_loop_stride + kv * a.resid_kv_stride);
+        rf[rec] = __bfloat16_as_ushort(sb);
     }
 }
 
@@ -184,7 +193,7 @@ __global__ void bf16_store_kernel(const Bf16StoreArgs a) {
 }  // namespace
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st) {
-    const long long warps = 2LL * a.B * a.n * a.H;
+    const long long warps = 2LL * a.B * a.n * a.H * (a.nres + 1);
     const long long blocks = (warps + 3) / 4;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     append_kernel<<<(unsigned)blocks, 128, 0, st>>>(a);
