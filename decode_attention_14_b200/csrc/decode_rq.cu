@@ -54,7 +54,13 @@ namespace rq {
 namespace {
 
 constexpr int kTile = 64;
-constexpr int kStages = 3;
+#ifndef RQ_DECODE_STAGES
+#define RQ_DECODE_STAGES 3
+#endif
+#ifndef RQ_DECODE_MIN_CTAS
+#define RQ_DECODE_MIN_CTAS 5
+#endif
+constexpr int kStages = RQ_DECODE_STAGES;
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
@@ -256,7 +262,7 @@ struct Plan {
 };
 
 template <int GK, int BA, int BR, int GS, bool RESID>
-__global__ void __launch_bounds__(kThreads, GK == 1 ? 5 : 3) decode_rq_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) decode_rq_kernel(const DecodeArgs a) {
     using P = Plan<BA, BR, GS, RESID>;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kStages];
