@@ -112,6 +112,29 @@ class ClockSampler:
                 "samples": len(inside), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings (all ranks must call it).  With
+    one process (no process group) the values come back unchanged."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_rate(world: int, per_rank_items: int, steps: int, max_elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own per_rank_items per
+    step; the job's time is the slowest rank's."""
+    return world * per_rank_items * steps / (max_elapsed_ms / 1e3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own sequences (independent batches, no data-path exchange)."""
+    return base + 1000 * rank
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, cfgd, rank, world, local_rank):
     import torch
@@ -123,7 +146,7 @@ def run_ours(args, cfgd, rank, world, local_rank):
     name = args.config
     layers = args.layers or cfgd["layers"]
     loops, Lg, B, T, H, Hq = cfgd["loops"], cfgd["Lg"], cfgd["B"], cfgd["T"], cfgd["H"], cfgd["Hq"]
-    seed = CONFIG_SEED[name] + 1000 * rank
+    seed = rank_seed(CONFIG_SEED[name], rank)
     fmt = rq.RQ_FMT_BF16 if args.bf16 else rq.RQ_FMT_RESIDUAL
     cfg = rq.make_config(num_layers=layers, num_loops=loops, loops_per_group=Lg, batch=B, max_tokens=T,
                          max_tail_tokens=FILL_CHUNK, num_kv_heads=H, num_q_heads=Hq, group_size=cfgd["g"],
@@ -281,10 +304,7 @@ def run_ours(args, cfgd, rank, world, local_rank):
     d1.record(stream)
     torch.cuda.synchronize(dev)
     dec_ms = d0.elapsed_time(d1)
-    if dist:
-        t = torch.tensor([elapsed_ms, dec_ms], device=dev, dtype=torch.float64)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        elapsed_ms, dec_ms = float(t[0]), float(t[1])
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dev)
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -316,17 +336,13 @@ def run_ours(args, cfgd, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a.elapsed_time(b)
-        if dist:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e_ms = float(t[0])
-        e2e = {"value": world * B * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+        e_ms = max_over_ranks([a.elapsed_time(b)], dev)[0]
+        e2e = {"value": weak_scaling_rate(world, B, args.steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     cache.check()
 
     ms_step = elapsed_ms / args.steps
-    value = world * B * args.steps / (elapsed_ms / 1e3)
+    value = weak_scaling_rate(world, B, args.steps, elapsed_ms)
     dec_ms_call = dec_ms / (args.steps * ncalls)
     achieved = step_decode_bytes * args.steps / (dec_ms / 1e3) / 1e9
     peak, peak_kind = _peaks()

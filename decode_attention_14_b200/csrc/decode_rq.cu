@@ -28,7 +28,7 @@
 // Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
 // Data movement.  Each CTA owns a chunk of one (sequence, kv head) and
-// streams it in 64-token items through a 3-stage shared-memory ring filled
+// streams it in 64-token items through a 4-stage shared-memory ring filled
 // by one producer warp with 1-D bulk asynchronous copies (cp.async.bulk,
 // completion counted on mbarriers; no multicast): first the K records of
 // every tile (pass 1: logits), then the anchor V codes + meta of every tile,
@@ -55,10 +55,10 @@ namespace {
 
 constexpr int kTile = 64;
 #ifndef RQ_DECODE_STAGES
-#define RQ_DECODE_STAGES 3
+#define RQ_DECODE_STAGES 4
 #endif
 #ifndef RQ_DECODE_MIN_CTAS
-#define RQ_DECODE_MIN_CTAS 5
+#define RQ_DECODE_MIN_CTAS 4
 #endif
 constexpr int kStages = RQ_DECODE_STAGES;
 constexpr int kConsumers = 128;

@@ -39,6 +39,8 @@ class Built:
     n_tail: int
     # inputs[layer][group] = (K list of Lg bf16 [B][T+n_tail][H][d], V list)
     inputs: dict = field(default_factory=dict)
+    # memoised oracle reconstructions of the GPU records (keyed by what they depend on)
+    recon: dict = field(default_factory=dict)
 
 
 def scale32() -> float:
@@ -173,6 +175,13 @@ def compare_records(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
 
 def reconstruct_gpu(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> np.ndarray:
     """Oracle reconstruction of the GPU's exported records: [Lg][n][d]."""
+    key = (layer, grp, kv, None if bh_sel is None else tuple(bh_sel), bt.T)
+    if key not in bt.recon:
+        bt.recon[key] = _reconstruct_gpu(bt, layer, grp, kv, bh_sel)
+    return bt.recon[key]
+
+
+def _reconstruct_gpu(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> np.ndarray:
     cfg = bt.cfg
     Lg = cfg.loops_per_group
     ac, am, _ = gpu_records(bt, layer, grp * Lg + Lg - 1, kv, bh_sel)
