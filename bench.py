@@ -41,6 +41,32 @@ CONFIG_SEED = {"tiny": 0x5EED0000, "ouro8k_b4": 0x5EED0001, "long16k_b2": 0x5EED
 FILL_CHUNK = 512
 
 
+KERNEL_SOURCES = ["decode_attention_14_b200/csrc/decode_rq.cu", "decode_attention_14_b200/csrc/combine.cuh",
+                  "decode_attention_14_b200/csrc/common.cuh", "decode_attention_14_b200/csrc/rq_internal.h"]
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(config_name: str):
+    """DRAM bytes (read + write) per decode launch from the committed ncu
+    summary, only if it was taken on the kernel sources as they are now."""
+    p = os.path.join(ROOT, "profiles", "decode_rq_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return j.get("bytes_per_launch", {}).get(config_name)
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -358,7 +384,8 @@ def run_ours(args, cfgd, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4/int2 codes, fp8 meta, fp32 math" if not args.bf16 else "bf16 in, fp32 math",
+        "dtype": ("u4/u2 codes, int32 dp4a/dp2a dot products, fp32 softmax" if not args.bf16
+                  else "bf16 in, fp32 math"),
         "data": "synthetic (seeded; anchor N(0,1) with 4 outlier channels x10, loops c*anchor+sigma*N(0,1))",
         "config": {"workload": name, "layers": layers, "loops": loops, "loops_per_group": Lg, "batch": B,
                    "seq_len": T, "kv_heads": H, "q_heads": Hq, "head_dim": 128, "group": cfgd["g"],
@@ -371,7 +398,8 @@ def run_ours(args, cfgd, rank, world, local_rank):
                         "tokens_per_s_decode_only": round(world * B * args.steps / (dec_ms / 1e3), 2)},
         "append": {"ms_per_step_est": round(max(ms_step - dec_ms / args.steps, 0.0), 4)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": measured_traffic(name) if not args.bf16 else None,
+                     "algorithmic_bytes_per_launch": int(step_decode_bytes / ncalls),
                      "kernel": "rq_decode_attn call (split kernel + combine)", "peak_kind": peak_kind},
         "e2e": e2e,
         "gpu_launches": int(args.steps * loops * layers * 3),
@@ -456,7 +484,7 @@ def run_reference(args, cfgd):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="ouro8k_b4", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -178,7 +178,8 @@ __device__ __forceinline__ int dot_seg(const Seg<BITS> &s, const QPlanes &q) {
 // acc{Lo,Hi}[i] += w0 * c0_i + w1 * c1_i for the 16 elements of a segment,
 // codes of two tokens; weights as 16-bit halves: wlo = (w0 & 0xFFFF) |
 // (w1 << 16) (unsigned), whi = (w0 >> 16) | (w1 >> 16) << 16 (signed).
-template <int BITS>
+// HI = false skips the high halves (exact when they are zero).
+template <int BITS, bool HI = true>
 __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b, uint32_t wlo, uint32_t whi,
                                          unsigned accLo[16], int accHi[16]) {
     const int Wh = (int)whi;
@@ -196,9 +197,11 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
             for (int k = 0; k < 4; k++) {
                 const int e = 8 * u + e0[k];
                 accLo[e] = __dp2a_lo(wlo, c[k], accLo[e]);
-                accHi[e] = __dp2a_lo(Wh, (int)c[k], accHi[e]);
                 accLo[e + 2] = __dp2a_hi(wlo, c[k], accLo[e + 2]);
-                accHi[e + 2] = __dp2a_hi(Wh, (int)c[k], accHi[e + 2]);
+                if (HI) {
+                    accHi[e] = __dp2a_lo(Wh, (int)c[k], accHi[e]);
+                    accHi[e + 2] = __dp2a_hi(Wh, (int)c[k], accHi[e + 2]);
+                }
             }
         }
     } else {
@@ -209,13 +212,15 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
             const uint32_t x = (X >> (2 * c)) & 0x03030303u;
             const uint32_t y = (Y >> (2 * c)) & 0x03030303u;
             accLo[c] = __dp2a_lo(wlo, x, accLo[c]);
-            accHi[c] = __dp2a_lo(Wh, (int)x, accHi[c]);
             accLo[4 + c] = __dp2a_hi(wlo, x, accLo[4 + c]);
-            accHi[4 + c] = __dp2a_hi(Wh, (int)x, accHi[4 + c]);
             accLo[8 + c] = __dp2a_lo(wlo, y, accLo[8 + c]);
-            accHi[8 + c] = __dp2a_lo(Wh, (int)y, accHi[8 + c]);
             accLo[12 + c] = __dp2a_hi(wlo, y, accLo[12 + c]);
-            accHi[12 + c] = __dp2a_hi(Wh, (int)y, accHi[12 + c]);
+            if (HI) {
+                accHi[c] = __dp2a_lo(Wh, (int)x, accHi[c]);
+                accHi[4 + c] = __dp2a_hi(Wh, (int)x, accHi[4 + c]);
+                accHi[8 + c] = __dp2a_lo(Wh, (int)y, accHi[8 + c]);
+                accHi[12 + c] = __dp2a_hi(Wh, (int)y, accHi[12 + c]);
+            }
         }
     }
 }
@@ -531,10 +536,20 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         cR = fixed_scale(448.f, 30);
     }
 
+    // weights pre-multiplied by their fixed-point scale (powers of two: exact)
+    for (int t = tid; t < ntiles * kTile; t += kConsumers) {
+#pragma unroll
+        for (int gq = 0; gq < GK; gq++) {
+            s_P[gq * a.chunk + t] *= cA;
+            s_sc[gq * a.chunk + t] *= cR;
+        }
+    }
+    consumer_sync();
+
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
     const int npass = RESID ? 2 : 1;
     for (int vp = 0; vp < npass; vp++) {
-        const float cW = vp == 0 ? cA : cR;
+        const float cW = vp == 0 ? cA : cR;   // weights in s_P / s_sc already carry it
         const float *wsrc = vp == 0 ? s_P : s_sc;
         unsigned accLo[GK][16];
         int accHi[GK][16];
@@ -576,25 +591,43 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_empty[stage]);
+            uint32_t hi_any = 0;
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
                 int wi[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    wi[k] = __float2int_rn(W[gq][k] * cW * mm[k].x);
+                    wi[k] = __float2int_rn(W[gq][k] * mm[k].x);   // W carries the scale 2^F
                     mS[gq] = fmaf(W[gq][k], mm[k].y, mS[gq]);
                 }
 #pragma unroll
                 for (int pr = 0; pr < 2; pr++) {
                     wlo[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x5410);
                     whi[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x7632);
+                    hi_any |= whi[gq][pr];
                 }
+            }
+            // small weights (most tokens of a peaked softmax) have zero high
+            // halves; when no lane of the warp has one, skip their products
+            const bool need_hi = __any_sync(0xffffffffu, hi_any != 0);
+#pragma unroll
+            for (int gq = 0; gq < GK; gq++) {
                 if (vp == 0) {
-                    acc_pair<BA>(ca[0], ca[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                    acc_pair<BA>(ca[2], ca[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                    if (need_hi) {
+                        acc_pair<BA>(ca[0], ca[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                        acc_pair<BA>(ca[2], ca[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                    } else {
+                        acc_pair<BA, false>(ca[0], ca[1], wlo[gq][0], 0u, accLo[gq], accHi[gq]);
+                        acc_pair<BA, false>(ca[2], ca[3], wlo[gq][1], 0u, accLo[gq], accHi[gq]);
+                    }
                 } else {
-                    acc_pair<BR>(cr[0], cr[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                    acc_pair<BR>(cr[2], cr[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                    if (need_hi) {
+                        acc_pair<BR>(cr[0], cr[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
+                        acc_pair<BR>(cr[2], cr[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                    } else {
+                        acc_pair<BR, false>(cr[0], cr[1], wlo[gq][0], 0u, accLo[gq], accHi[gq]);
+                        acc_pair<BR, false>(cr[2], cr[3], wlo[gq][1], 0u, accLo[gq], accHi[gq]);
+                    }
                 }
             }
         }
@@ -605,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
             for (int e = 0; e < 16; e++) {
                 float v = fmaf((float)accHi[gq][e], 65536.f, (float)accLo[gq][e]);
-                v = fmaf(v, iW, mS[gq]);
+                v = (v + mS[gq]) * iW;   // both in units of 2^-F
                 v += __shfl_xor_sync(0xffffffffu, v, 8);
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 if (sub == 0) s_acc[warp][gq][vp][seg * 16 + e] = v;
