@@ -402,71 +402,98 @@ def run_ours(args, cfgd, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": int(step_decode_bytes / ncalls),
                      "kernel": "rq_decode_attn call (split kernel + combine)", "peak_kind": peak_kind},
         "e2e": e2e,
-        "gpu_launches": int(args.steps * loops * layers * 3),
+        # per (layer, loop): one append-side kernel (tail copy, encoder or BF16 store) and one
+        # decode kernel that merges its own splits; the BF16 path adds a combine kernel
+        "gpu_launches": int(args.steps * loops * layers * (3 if args.bf16 else 2)),
         "clocks": clocks,
     }
     return res, cache, call_bytes
 
 
 # ---------------------------------------------------------------- cpu baseline (oracle)
-def oracle_unit_decode_seconds(cfgd, seed, n_units: int, T: int | None = None):
-    """Times the oracle's decode of `n_units` (sequence, kv head) units: for
-    each unit, reconstruct the 4 loops' K/V over T tokens from its records and
-    run the direct fp64 softmax for each loop's query.  Returns (seconds per
-    unit-step, description).  Records are produced by the oracle's own
-    encoder from CPU-generated synthetic inputs (untimed)."""
-    import torch
-    from decode_attention_14_b200 import synth
-    from oracle import oracle as orc
+class OracleUnits:
+    """Records of a few (sequence, kv head) units at full T, encoded by the
+    oracle from CPU-generated synthetic inputs (setup, untimed)."""
 
-    T = T or cfgd["T"]
-    Lg, g, ba, br = cfgd["Lg"], cfgd["g"], cfgd["ba"], cfgd["br"]
-    total = 0.0
-    for u in range(n_units):
-        Kg, Vg = synth.group_kv(seed + u, 0, 0, Lg, cfgd["sigma"], 1, T, 1, device="cpu")
-        recs = []
-        for X in (Kg, Vg):
-            x = np.stack([synth.bf16_to_u16(X[j]).reshape(-1, 128) for j in range(Lg)])
-            recs.append(orc.encode(x, g, ba, br, True, 0xA11CE))
-        q = torch.randn((1, 1, 128)).to(torch.bfloat16)
-        qf = orc.bf16_bits_to_f64(synth.bf16_to_u16(q))
+    def __init__(self, cfgd, seed, n_units: int, T: int | None = None):
+        import torch
+        from decode_attention_14_b200 import synth
+        from oracle import oracle as orc
+        self.cfgd, self.T = cfgd, T or cfgd["T"]
+        Lg = cfgd["Lg"]
+        self.units = []
+        for u in range(n_units):
+            Kg, Vg = synth.group_kv(seed + u, 0, 0, Lg, cfgd["sigma"], 1, self.T, 1, device="cpu")
+            recs = []
+            for X in (Kg, Vg):
+                x = np.stack([synth.bf16_to_u16(X[j]).reshape(-1, 128) for j in range(Lg)])
+                recs.append(orc.encode(x, cfgd["g"], cfgd["ba"], cfgd["br"], True, 0xA11CE))
+            q = torch.randn((1, 1, 128)).to(torch.bfloat16)
+            self.units.append((recs, orc.bf16_bits_to_f64(synth.bf16_to_u16(q))))
+
+    def decode_seconds(self, u: int, loop: int) -> float:
+        """One decode call of one unit, timed: reconstruct the loop's K and V
+        from its two reads (anchor + the loop's residual; the anchor alone for
+        the anchor loop) and run the direct fp64 softmax."""
+        from oracle import oracle as orc
+        c = self.cfgd
+        Lg = c["Lg"]
+        recs, qf = self.units[u % len(self.units)]
         t0 = time.perf_counter()
-        kvhat = [orc.reconstruct(e.a_codes, e.a_meta, e.r_codes, e.r_meta, e.r_coef, Lg, 128, g, ba, br, True, 0xA11CE)
-                 for e in recs]
-        for j in range(Lg):
-            orc.attention(qf, kvhat[0][j][None, :, None, :], kvhat[1][j][None, :, None, :], 1 / math.sqrt(128))
-        total += time.perf_counter() - t0
-    return total / n_units
+        kv = []
+        for e in recs:
+            if loop == Lg - 1:
+                x = orc.reconstruct(e.a_codes, e.a_meta, None, None, None, 1, 128, c["g"], c["ba"], c["br"], True,
+                                    0xA11CE)[0]
+            else:
+                x = orc.reconstruct(e.a_codes, e.a_meta, e.r_codes[loop:loop + 1], e.r_meta[loop:loop + 1],
+                                    e.r_coef[loop:loop + 1], 2, 128, c["g"], c["ba"], c["br"], True, 0xA11CE)[0]
+            kv.append(x)
+        orc.attention(qf, kv[0][None, :, None, :], kv[1][None, :, None, :], 1 / math.sqrt(128))
+        return time.perf_counter() - t0
+
+
+def calls_per_step(cfgd) -> int:
+    return cfgd["layers"] * cfgd["loops"] * cfgd["B"] * cfgd["H"]   # (unit, loop) decodes per step
 
 
 def cpu_baseline(cfgd, seed, budget_s: float = 15.0):
-    # one unit at full T to size the sample, then as many as fit the budget
-    per_unit = oracle_unit_decode_seconds(cfgd, seed, 1)
-    n = int(max(1, min(8, budget_s // max(per_unit, 1e-3) - 1)))
-    if n > 1:
-        per_unit = oracle_unit_decode_seconds(cfgd, seed + 7, n)
-    units_per_step = cfgd["layers"] * (cfgd["loops"] // cfgd["Lg"]) * cfgd["B"] * cfgd["H"]
-    step_s = per_unit * units_per_step
+    """The oracle as it stands, one host core, on a bounded sample of the
+    workload: every loop of a few (sequence, kv head) units at full T,
+    scaled to a decode step."""
+    ou = OracleUnits(cfgd, seed, 2)
+    Lg = cfgd["Lg"]
+    times, t_start = [], time.perf_counter()
+    while time.perf_counter() - t_start < budget_s or len(times) < Lg:
+        i = len(times)
+        times.append(ou.decode_seconds(i // Lg, i % Lg))
+        if len(times) >= 8 * Lg:
+            break
+    # average over whole groups of loops (anchor and residual loops in proportion)
+    n = len(times) // Lg * Lg
+    per = float(np.mean(times[:n]))
+    step_s = per * calls_per_step(cfgd)
     return {"value": round(cfgd["B"] / step_s, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} (sequence, kv head) unit(s) x {cfgd['loops']} loops at T={cfgd['T']} "
-                      f"(reconstruct + fp64 softmax), {per_unit:.2f} s/unit, scaled to "
-                      f"{units_per_step} units per step (extrapolated)"}
+            "sample": f"{n} unit-loop decodes ({n // Lg} (sequence, kv head) unit pass(es) over all {Lg} loops) "
+                      f"at T={cfgd['T']}, {per:.3f} s each (reconstruct from records + fp64 softmax), scaled to "
+                      f"{calls_per_step(cfgd)} unit-loops per decode step (extrapolated)"}
 
 
 def run_reference(args, cfgd):
-    """The oracle, timed as it stands on the host cores: each step a bounded
-    sample (one (sequence, kv head) unit of one layer group), scaled to the
-    workload's metric."""
+    """The oracle, timed as it stands on one host core: each step is a
+    bounded sample -- one (sequence, kv head) unit of one loop at full T
+    (reconstruct from records + direct fp64 softmax), loops taken in turn --
+    scaled to the workload's decode step."""
     seed = CONFIG_SEED[args.config]
+    ou = OracleUnits(cfgd, seed, 2)
+    Lg = cfgd["Lg"]
     for w in range(args.warmup):
-        oracle_unit_decode_seconds(cfgd, seed + 100 + w, 1, T=min(cfgd["T"], 1024))
-    per = [oracle_unit_decode_seconds(cfgd, seed + s, 1) for s in range(args.steps)]
-    per_unit = float(np.mean(per))
-    units_per_step = cfgd["layers"] * (cfgd["loops"] // cfgd["Lg"]) * cfgd["B"] * cfgd["H"]
-    step_s = per_unit * units_per_step
+        ou.decode_seconds(w, w % Lg)
+    per = float(np.mean([ou.decode_seconds(s // Lg, s % Lg) for s in range(args.steps)]))
+    step_s = per * calls_per_step(cfgd)
     value = cfgd["B"] / step_s
-    sample = (f"1 (sequence, kv head) unit x {cfgd['loops']} loops at T={cfgd['T']} per step "
-              f"(oracle reconstruct + fp64 softmax), scaled to {units_per_step} units per decode step")
+    sample = (f"per step: 1 (sequence, kv head) unit x 1 loop (loops in turn) at T={cfgd['T']} (oracle reconstruct "
+              f"+ fp64 softmax, {per:.3f} s), scaled to {calls_per_step(cfgd)} unit-loops per decode step")
     return {
         "impl": "reference",
         "metric": "decode-attention tokens/s (INT4 anchor/INT2 resid)",

@@ -366,9 +366,6 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     return RQ_OK;
 }
 
-// partials == nullptr: the split partials go to the cache's own workspace
-// (stride splits_max).  Otherwise to `partials` (capacity partial_floats,
-// stride = the split count actually used).
 // partials == nullptr: split partials and combine counters in the cache's
 // workspace (partial stride splits_max).  Otherwise in the caller's scratch
 // (stride = the split count this call uses).
