@@ -54,13 +54,18 @@ namespace rq {
 namespace {
 
 constexpr int kTile = 64;
-#ifndef RQ_DECODE_STAGES
-#define RQ_DECODE_STAGES 4
+#ifndef RQ_DECODE_PRODUCER_SLEEP_NS
+#define RQ_DECODE_PRODUCER_SLEEP_NS 0
+#endif
+#ifndef RQ_DECODE_RING_BYTES
+#define RQ_DECODE_RING_BYTES 39936
 #endif
 #ifndef RQ_DECODE_MIN_CTAS
 #define RQ_DECODE_MIN_CTAS 4
 #endif
-constexpr int kStages = RQ_DECODE_STAGES;
+constexpr int kRingBytes = RQ_DECODE_RING_BYTES;   // byte ring of one CTA (multiple of 128)
+constexpr int kSlots = 16;                         // mbarrier pairs: at most 16 items in flight
+static_assert(kRingBytes % 128 == 0, "ring must be a multiple of 128 bytes");
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
@@ -96,11 +101,14 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 // Bounded wait on an mbarrier phase; gives up after kWaitNs or as soon as
-// another warp of the CTA has given up.
+// another warp of the CTA has given up.  SLEEP_NS > 0 backs off between
+// polls (for waits whose latency does not matter).
+template <unsigned SLEEP_NS = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (;;) {
+        if (SLEEP_NS) __nanosleep(SLEEP_NS);
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
         if (global_ns() - t0 > kWaitNs) return false;
@@ -148,6 +156,12 @@ __device__ __forceinline__ int elem_of(int r, int m) {
     return BITS == 4 ? 8 * (r >> 1) + (r & 1) + 2 * m : r + 4 * m;
 }
 
+// Inverse of elem_of: the (word, byte) slot 4r + m of segment element i.
+template <int BITS>
+__device__ __forceinline__ int slot_of(int i) {
+    return BITS == 4 ? 4 * (2 * (i >> 3) + (i & 1)) + ((i & 7) >> 1) : 4 * (i & 3) + (i >> 2);
+}
+
 template <int BITS>
 __device__ __forceinline__ uint32_t unpack_word(const Seg<BITS> &s, int r) {
     if (BITS == 4) return (r & 1) ? ((s.w[r >> 1] >> 4) & 0x0F0F0F0Fu) : (s.w[r >> 1] & 0x0F0F0F0Fu);
@@ -175,10 +189,31 @@ __device__ __forceinline__ int dot_seg(const Seg<BITS> &s, const QPlanes &q) {
     return (int)(((unsigned)hi << 16) + (mid << 8) + lo);
 }
 
-// acc{Lo,Hi}[i] += w0 * c0_i + w1 * c1_i for the 16 elements of a segment,
-// codes of two tokens; weights as 16-bit halves: wlo = (w0 & 0xFFFF) |
-// (w1 << 16) (unsigned), whi = (w0 >> 16) | (w1 >> 16) << 16 (signed).
+// acc{Lo,Hi}[i] += 2^acc_shift(i) (w0 * c0_i + w1 * c1_i) for the 16 elements
+// of a segment, codes of two tokens; weights as 16-bit halves: wlo =
+// (w0 & 0xFFFF) | (w1 << 16) (unsigned), whi = (w0 >> 16) | (w1 >> 16) << 16
+// (signed).  Codes are masked in place rather than shifted down, so element
+// i's sums carry the factor 2^acc_shift(i), removed once at the end (the sums
+// stay below 2^30 for the 64 tokens a lane takes per chunk).
 // HI = false skips the high halves (exact when they are zero).
+// dp2a with signed 16-bit halves of a and UNSIGNED bytes of b (the masked
+// codes reach 240, beyond int8).
+__device__ __forceinline__ int dp2a_lo_su(int a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi_su(int a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+template <int BITS>
+__host__ __device__ constexpr int acc_shift(int e) {
+    return BITS == 4 ? ((e & 1) ? 4 : 0) : 2 * (e & 3);
+}
+
 template <int BITS, bool HI = true>
 __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b, uint32_t wlo, uint32_t whi,
                                          unsigned accLo[16], int accHi[16]) {
@@ -190,8 +225,7 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
             const uint32_t Y = __byte_perm(a.w[u], b.w[u], 0x7362);   // bytes 2,3 of both tokens
             // c[0]: elements 8u+0 (bytes 0,1), 8u+2 (bytes 2,3); c[1]: 8u+1, 8u+3;
             // c[2]: 8u+4, 8u+6; c[3]: 8u+5, 8u+7
-            const uint32_t c[4] = {X & 0x0F0F0F0Fu, (X >> 4) & 0x0F0F0F0Fu, Y & 0x0F0F0F0Fu,
-                                   (Y >> 4) & 0x0F0F0F0Fu};
+            const uint32_t c[4] = {X & 0x0F0F0F0Fu, X & 0xF0F0F0F0u, Y & 0x0F0F0F0Fu, Y & 0xF0F0F0F0u};
             const int e0[4] = {0, 1, 4, 5};
 #pragma unroll
             for (int k = 0; k < 4; k++) {
@@ -199,8 +233,8 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
                 accLo[e] = __dp2a_lo(wlo, c[k], accLo[e]);
                 accLo[e + 2] = __dp2a_hi(wlo, c[k], accLo[e + 2]);
                 if (HI) {
-                    accHi[e] = __dp2a_lo(Wh, (int)c[k], accHi[e]);
-                    accHi[e + 2] = __dp2a_hi(Wh, (int)c[k], accHi[e + 2]);
+                    accHi[e] = dp2a_lo_su(Wh, c[k], accHi[e]);
+                    accHi[e + 2] = dp2a_hi_su(Wh, c[k], accHi[e + 2]);
                 }
             }
         }
@@ -209,17 +243,17 @@ __device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b,
         const uint32_t Y = __byte_perm(a.w[0], b.w[0], 0x7362);   // bytes 2,3: elements 8-15
 #pragma unroll
         for (int c = 0; c < 4; c++) {
-            const uint32_t x = (X >> (2 * c)) & 0x03030303u;
-            const uint32_t y = (Y >> (2 * c)) & 0x03030303u;
+            const uint32_t x = X & (0x03030303u << (2 * c));
+            const uint32_t y = Y & (0x03030303u << (2 * c));
             accLo[c] = __dp2a_lo(wlo, x, accLo[c]);
             accLo[4 + c] = __dp2a_hi(wlo, x, accLo[4 + c]);
             accLo[8 + c] = __dp2a_lo(wlo, y, accLo[8 + c]);
             accLo[12 + c] = __dp2a_hi(wlo, y, accLo[12 + c]);
             if (HI) {
-                accHi[c] = __dp2a_lo(Wh, (int)x, accHi[c]);
-                accHi[4 + c] = __dp2a_hi(Wh, (int)x, accHi[4 + c]);
-                accHi[8 + c] = __dp2a_lo(Wh, (int)y, accHi[8 + c]);
-                accHi[12 + c] = __dp2a_hi(Wh, (int)y, accHi[12 + c]);
+                accHi[c] = dp2a_lo_su(Wh, x, accHi[c]);
+                accHi[4 + c] = dp2a_hi_su(Wh, x, accHi[4 + c]);
+                accHi[8 + c] = dp2a_lo_su(Wh, y, accHi[8 + c]);
+                accHi[12 + c] = dp2a_hi_su(Wh, y, accHi[12 + c]);
             }
         }
     }
@@ -240,7 +274,10 @@ __device__ __forceinline__ float fixed_scale(float bound, int top) {
     return ldexpf(1.f, F);
 }
 
-// Shared-memory plan of one CTA (bytes).  Items are 64 tokens.
+// Shared-memory plan of one CTA (bytes).  Items are 64 tokens; they are placed
+// back to back in a byte ring (an item never straddles its end), so the
+// number in flight follows their size: about 4 K items, 7 anchor V items or
+// 12 residual V items at once.
 template <int BA, int BR, int GS, bool RESID>
 struct Plan {
     static constexpr int A_C = 16 * BA;              // anchor codes per record
@@ -257,8 +294,17 @@ struct Plan {
     static constexpr int VA_BYTES = VA_M + kTile * MR;
     static constexpr int VR_M = kTile * R_C;
     static constexpr int VR_BYTES = VR_M + kTile * MR;
-    static constexpr int STAGE = ((K_BYTES > VA_BYTES ? K_BYTES : VA_BYTES) + 127) / 128 * 128;
-    static constexpr int RING = kStages * STAGE;
+    static constexpr int RING = kRingBytes;
+    static_assert(K_BYTES % 128 == 0 && VA_BYTES % 128 == 0 && VR_BYTES % 128 == 0, "item alignment");
+    static_assert(K_BYTES <= RING && VA_BYTES <= RING, "ring too small");
+    __host__ __device__ static constexpr int item_bytes(int pass) {
+        return pass == 0 ? K_BYTES : pass == 1 ? VA_BYTES : VR_BYTES;
+    }
+    // ring offset of the item after one of `cur` bytes at offset `off`, when the next has `next` bytes
+    __host__ __device__ static int advance(int off, int cur, int next) {
+        off += cur;
+        return off + next > RING ? 0 : off;
+    }
     // then: V coefficients [chunk] (RESID), logits/p [GK][chunk], p*s_hat [GK][chunk]
     __host__ __device__ static int coef_bytes(int chunk) { return RESID ? (chunk * 2 + 127) / 128 * 128 : 0; }
     __host__ __device__ static size_t smem(int GK, int chunk) {
@@ -270,11 +316,13 @@ template <int GK, int BA, int BR, int GS, bool RESID>
 __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) decode_rq_kernel(const DecodeArgs a) {
     using P = Plan<BA, BR, GS, RESID>;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bar_full[kStages];
-    __shared__ __align__(8) uint64_t bar_empty[kStages];
+    __shared__ __align__(8) uint64_t bar_full[kSlots];
+    __shared__ __align__(8) uint64_t bar_empty[kSlots];
     __shared__ __align__(8) uint64_t bar_cf;
     __shared__ int s_abort, s_last;
     __shared__ float s_q[GK][2][kHeadDim];
+    __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
+    __shared__ int s_qsum[GK][2][8];                             // sum of each segment's fixed-point q
     __shared__ float s_red[4][2 * GK + 2];
     __shared__ float s_acc[4][GK][2][kHeadDim];
 
@@ -293,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     float *s_P = s_sc + GK * a.chunk;                                                  // [GK][chunk] p * s_hat
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; i++) {
+        for (int i = 0; i < kSlots; i++) {
             mbar_init(&bar_full[i], 1);
-            mbar_init(&bar_empty[i], 4);
+            mbar_init(&bar_empty[i], kConsumers);   // every consumer thread arrives
         }
         mbar_init(&bar_cf, 1);
         s_abort = 0;
@@ -311,43 +359,95 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
                 bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
             }
-            int issued = 0;
-            const int nitems = (RESID ? 3 : 2) * ntiles;   // K tiles, anchor V tiles, residual V tiles
-            for (int it = 0; it < nitems; it++) {
-                const int stage = it % kStages;
-                if (it >= kStages && !mbar_wait(&bar_empty[stage], ((it / kStages) - 1) & 1, &s_abort)) {
-                    s_abort = 1;
-                    atomicExch(a.err, 1);
-                    break;
-                }
-                uint8_t *st = ring + stage * P::STAGE;
-                uint64_t *bar = &bar_full[stage];
-                const int pass = it / ntiles;
-                const size_t tk = tok0 + (size_t)(it - pass * ntiles) * kTile;
+            // Items in order: K tiles, anchor V tiles, residual V tiles.  Item it
+            // occupies [virt, virt + bytes) of an unbounded virtual byte
+            // sequence, padded so that no item straddles the ring's end; its
+            // ring offset is phys = virt mod RING.  Before it is issued, every
+            // older item starting below virt + bytes - RING must have been
+            // released, and at most kSlots items may be outstanding.  The
+            // loop keeps all of this in running counters (no division).
+            const int npass = RESID ? 3 : 2;
+            int it = 0, virt = 0, phys = 0;
+            int rel = 0, vrel = 0, rphys = 0, rtile = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
+            bool ok = true;
+            for (int pass = 0; pass < npass && ok; pass++) {
+                const int bytes = P::item_bytes(pass);
+                const uint8_t *c0, *c1 = nullptr;   // code and meta sources of this pass's first tile
+                int cstride = 0, c1stride = P::MR * kTile;
                 if (pass == 0) {
-                    mbar_expect_tx(bar, (uint32_t)P::K_BYTES);
-                    bulk_g2s(st, a.a_codes[0] + tk * P::A_C, kTile * P::A_C, bar);
-                    bulk_g2s(st + P::K_AM, a.a_meta[0] + tk * P::MR, kTile * P::MR, bar);
-                    if (RESID) {
-                        bulk_g2s(st + P::K_RC, a.r_codes[0] + tk * P::R_C, kTile * P::R_C, bar);
-                        bulk_g2s(st + P::K_RM, a.r_meta[0] + tk * P::MR, kTile * P::MR, bar);
-                        bulk_g2s(st + P::K_CF, a.r_coef[0] + tk, kTile * 2, bar);
-                    }
+                    c0 = a.a_codes[0] + tok0 * P::A_C;
+                    c1 = a.a_meta[0] + tok0 * P::MR;
+                    cstride = P::A_C * kTile;
                 } else if (pass == 1) {
-                    mbar_expect_tx(bar, (uint32_t)P::VA_BYTES);
-                    bulk_g2s(st, a.a_codes[1] + tk * P::A_C, kTile * P::A_C, bar);
-                    bulk_g2s(st + P::VA_M, a.a_meta[1] + tk * P::MR, kTile * P::MR, bar);
+                    c0 = a.a_codes[1] + tok0 * P::A_C;
+                    c1 = a.a_meta[1] + tok0 * P::MR;
+                    cstride = P::A_C * kTile;
                 } else {
-                    mbar_expect_tx(bar, (uint32_t)P::VR_BYTES);
-                    bulk_g2s(st, a.r_codes[1] + tk * P::R_C, kTile * P::R_C, bar);
-                    bulk_g2s(st + P::VR_M, a.r_meta[1] + tk * P::MR, kTile * P::MR, bar);
+                    c0 = a.r_codes[1] + tok0 * P::R_C;
+                    c1 = a.r_meta[1] + tok0 * P::MR;
+                    cstride = P::R_C * kTile;
                 }
-                issued = it + 1;
+                const uint8_t *r0 = RESID ? a.r_codes[0] + tok0 * P::R_C : nullptr;
+                const uint8_t *r1 = RESID ? a.r_meta[0] + tok0 * P::MR : nullptr;
+                const uint8_t *r2 = RESID ? reinterpret_cast<const uint8_t *>(a.r_coef[0] + tok0) : nullptr;
+                for (int i = 0; i < ntiles; i++, it++) {
+                    if (phys + bytes > P::RING) {
+                        virt += P::RING - phys;
+                        phys = 0;
+                    }
+                    while (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING)) {
+                        if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
+                                                                    &s_abort)) {
+                            ok = false;
+                            break;
+                        }
+                        vrel += rbytes;
+                        rphys += rbytes;
+                        if (++rtile == ntiles) {
+                            rtile = 0;
+                            rbytes = P::item_bytes(++rpass);
+                        }
+                        if (rphys + rbytes > P::RING) {
+                            vrel += P::RING - rphys;
+                            rphys = 0;
+                        }
+                        rel++;
+                    }
+                    if (!ok) {
+                        s_abort = 1;
+                        atomicExch(a.err, 1);
+                        break;
+                    }
+                    uint8_t *st = ring + phys;
+                    uint64_t *bar = &bar_full[it % kSlots];
+                    mbar_expect_tx(bar, (uint32_t)bytes);
+                    if (pass == 0) {
+                        bulk_g2s(st, c0, kTile * P::A_C, bar);
+                        bulk_g2s(st + P::K_AM, c1, kTile * P::MR, bar);
+                        if (RESID) {
+                            bulk_g2s(st + P::K_RC, r0, kTile * P::R_C, bar);
+                            bulk_g2s(st + P::K_RM, r1, kTile * P::MR, bar);
+                            bulk_g2s(st + P::K_CF, r2, kTile * 2, bar);
+                            r0 += kTile * P::R_C;
+                            r1 += kTile * P::MR;
+                            r2 += kTile * 2;
+                        }
+                    } else {
+                        bulk_g2s(st, c0, (uint32_t)cstride, bar);
+                        bulk_g2s(st + cstride, c1, kTile * P::MR, bar);
+                    }
+                    c0 += cstride;
+                    c1 += c1stride;
+                    virt += bytes;
+                    phys += bytes;
+                }
             }
+            const int issued = it;
             // drain: every issued copy must have landed before the CTA exits
-            if (RESID) mbar_wait(&bar_cf, 0, &s_abort);
-            for (int it = max(0, issued - kStages); it < issued; it++)
-                mbar_wait(&bar_full[it % kStages], (it / kStages) & 1, &s_abort);
+            // (the consumers stop waiting once the CTA has given up)
+            if (RESID) mbar_wait<256>(&bar_cf, 0, &s_abort);
+            for (int it = max(0, issued - kSlots); it < issued; it++)
+                mbar_wait<256>(&bar_full[it % kSlots], (it / kSlots) & 1, &s_abort);
         }
         return;
     }
@@ -390,35 +490,50 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const float qmax = fmaxf(fmaxf(s_red[0][0], s_red[1][0]), fmaxf(s_red[2][0], s_red[3][0]));
     const float qscale = fixed_scale(qmax, 22);  // q_int = round(q * qscale), |q_int| < 2^22
     const float qinv = 1.f / qscale;             // exact (power of two)
+    // Each consumer thread converts element tid of q (and of R q) and stores
+    // its three bytes where the lanes of its segment pick them up as plane
+    // words; the integer sum of each segment's 16 values comes from a
+    // 16-lane shuffle reduction.
+    {
+        const int sg = tid >> 4, i = tid & 15;
+#pragma unroll
+        for (int gq = 0; gq < GK; gq++) {
+#pragma unroll
+            for (int ab = 0; ab < (RESID ? 2 : 1); ab++) {
+                const int x = __float2int_rn(s_q[gq][ab][tid] * qscale);
+                uint8_t *dst = &s_qp[gq][ab][0][sg * 16 + (ab == 0 ? slot_of<BA>(i) : slot_of<BR>(i))];
+                dst[0] = (uint8_t)(x & 0xFF);
+                dst[kHeadDim] = (uint8_t)((x >> 8) & 0xFF);
+                dst[2 * kHeadDim] = (uint8_t)((x >> 16) & 0xFF);
+                int sum = x;
+#pragma unroll
+                for (int m = 1; m < 16; m <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+                if (i == 0) s_qsum[gq][ab][sg] = sum;
+            }
+        }
+    }
+    consumer_sync();
     QPlanes qA[GK], qR[GK];
     float QA[GK], QR[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
-        QA[gq] = QR[gq] = 0.f;
 #pragma unroll
-        for (int r = 0; r < 4; r++) {
-            uint32_t pa[3] = {0, 0, 0}, pr[3] = {0, 0, 0};
-#pragma unroll
-            for (int m = 0; m < 4; m++) {
-                const int xa = __float2int_rn(s_q[gq][0][seg * 16 + elem_of<BA>(r, m)] * qscale);
-                QA[gq] += (float)xa;
-                pa[0] |= (uint32_t)(xa & 0xFF) << (8 * m);
-                pa[1] |= (uint32_t)((xa >> 8) & 0xFF) << (8 * m);
-                pa[2] |= (uint32_t)((xa >> 16) & 0xFF) << (8 * m);
-                if (RESID) {
-                    const int xr = __float2int_rn(s_q[gq][1][seg * 16 + elem_of<BR>(r, m)] * qscale);
-                    QR[gq] += (float)xr;
-                    pr[0] |= (uint32_t)(xr & 0xFF) << (8 * m);
-                    pr[1] |= (uint32_t)((xr >> 8) & 0xFF) << (8 * m);
-                    pr[2] |= (uint32_t)((xr >> 16) & 0xFF) << (8 * m);
-                }
-            }
-#pragma unroll
-            for (int pl = 0; pl < 3; pl++) {
-                qA[gq].p[pl][r] = pa[pl];
-                qR[gq].p[pl][r] = pr[pl];
+        for (int pl = 0; pl < 3; pl++) {
+            const uint4 wa = *reinterpret_cast<const uint4 *>(&s_qp[gq][0][pl][seg * 16]);
+            qA[gq].p[pl][0] = wa.x;
+            qA[gq].p[pl][1] = wa.y;
+            qA[gq].p[pl][2] = wa.z;
+            qA[gq].p[pl][3] = wa.w;
+            if (RESID) {
+                const uint4 wr = *reinterpret_cast<const uint4 *>(&s_qp[gq][1][pl][seg * 16]);
+                qR[gq].p[pl][0] = wr.x;
+                qR[gq].p[pl][1] = wr.y;
+                qR[gq].p[pl][2] = wr.z;
+                qR[gq].p[pl][3] = wr.w;
             }
         }
+        QA[gq] = (float)s_qsum[gq][0][seg];
+        QR[gq] = RESID ? (float)s_qsum[gq][1][seg] : 0.f;
     }
 
     // ------------------------------------------------------------ pass 1: logits
@@ -427,14 +542,15 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
     const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
     const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
+    int c_off = 0;   // ring offset of the current item (the producer's placement rule)
     for (int i = 0; i < ntiles; i++) {
-        const int stage = i % kStages;
-        const bool ok = mbar_wait(&bar_full[stage], (i / kStages) & 1, &s_abort);
+        const int slot = i % kSlots;
+        const bool ok = mbar_wait(&bar_full[slot], (i / kSlots) & 1, &s_abort);
         if (!ok) {
             s_abort = 1;
             atomicExch(a.err, 2);
         }
-        const uint8_t *st = ring + stage * P::STAGE;
+        const uint8_t *st = ring + c_off;
         float part[GK][4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
@@ -460,8 +576,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 part[gq][k] = v;
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_empty[stage]);
+        mbar_arrive(&bar_empty[slot]);
+        c_off = P::advance(c_off, P::K_BYTES, i + 1 < ntiles ? P::K_BYTES : P::VA_BYTES);
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
         const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
@@ -565,12 +681,12 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         }
         for (int i = 0; i < ntiles; i++) {
             const int it = (1 + vp) * ntiles + i;
-            const int stage = it % kStages;
-            if (!mbar_wait(&bar_full[stage], (it / kStages) & 1, &s_abort)) {
+            const int slot = it % kSlots;
+            if (!mbar_wait(&bar_full[slot], (it / kSlots) & 1, &s_abort)) {
                 s_abort = 1;
                 atomicExch(a.err, 4);
             }
-            const uint8_t *st = ring + stage * P::STAGE;
+            const uint8_t *st = ring + c_off;
             uint32_t wlo[GK][2], whi[GK][2];
             float2 mm[4];
             float W[GK][4];
@@ -589,8 +705,11 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
                 for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + i * kTile + tok];
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_empty[stage]);
+            mbar_arrive(&bar_empty[slot]);
+            {
+                const int cur = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
+                c_off = P::advance(c_off, cur, i + 1 < ntiles ? cur : P::VR_BYTES);
+            }
             uint32_t hi_any = 0;
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
@@ -637,8 +756,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         for (int gq = 0; gq < GK; gq++) {
 #pragma unroll
             for (int e = 0; e < 16; e++) {
+                const int sh = vp == 0 ? acc_shift<BA>(e) : acc_shift<BR>(e);
                 float v = fmaf((float)accHi[gq][e], 65536.f, (float)accLo[gq][e]);
-                v = (v + mS[gq]) * iW;   // both in units of 2^-F
+                v = fmaf(v, __int_as_float((127 - sh) << 23), mS[gq]) * iW;   // 2^-sh; both in units of 2^-F
                 v += __shfl_xor_sync(0xffffffffu, v, 8);
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 if (sub == 0) s_acc[warp][gq][vp][seg * 16 + e] = v;
