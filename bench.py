@@ -2,9 +2,10 @@
 
 A step is one decode step of a looped Transformer over a cache already
 holding T-1 committed tokens per sequence: for every loop (outer) and layer
-(inner) it appends the new token's K/V (rq_append: tail copy for loops 1..L-1,
-fp64 encode + commit at the anchor loop) and runs single-token decode
-attention (rq_decode_attn) over T keys.  The metric is decode-attention
+(inner) it appends the new token's K/V and runs single-token decode attention
+over T keys: rq_append_decode_attn, one launch for loops 1..L-1 (the decode
+kernel writes the tail row), the fp64 encode + commit and then the decode at
+the anchor loop (--separate-append: rq_append and rq_decode_attn as two calls).  The metric is decode-attention
 tokens/s = batch / step time (whole job: all ranks' sequences / max-over-ranks
 time), plus achieved HBM GB/s of the decode calls over their algorithmic
 compressed bytes.
@@ -212,7 +213,9 @@ def run_ours(args, cfgd, rank, world, local_rank):
             for grp in range(n_groups):
                 cache.truncate(layer, grp, T0)
 
-    def step(ev=None, k=None, v=None, q=None):
+    fused = not args.bf16 and not args.separate_append
+
+    def step(k=None, v=None, q=None):
         k = new_k if k is None else k
         v = new_v if v is None else v
         q = qs if q is None else q
@@ -221,14 +224,16 @@ def run_ours(args, cfgd, rank, world, local_rank):
         sptr = int(cur.cuda_stream)
         for lp in range(loops):
             for layer in range(layers):
+                if fused:
+                    st = rq.rq_append_decode_attn(h, layer, lp, k[layer, lp], v[layer, lp], 1, q[layer, lp],
+                                                  outs[layer, lp], 0.0, sptr)
+                    if st != 0:
+                        raise rq.RQError(st, "rq_append_decode_attn")
+                    continue
                 st = rq.rq_append(h, layer, lp, k[layer, lp], v[layer, lp], 1, sptr)
                 if st != 0:
                     raise rq.RQError(st, "rq_append")
-                if ev is not None:
-                    ev[0][lp * layers + layer].record(cur)
                 st = decode(h, layer, lp, q[layer, lp], outs[layer, lp], 0.0, sptr)
-                if ev is not None:
-                    ev[1][lp * layers + layer].record(cur)
                 if st != 0:
                     raise rq.RQError(st, "rq_decode_attn")
 
@@ -390,6 +395,8 @@ def run_ours(args, cfgd, rank, world, local_rank):
         "config": {"workload": name, "layers": layers, "loops": loops, "loops_per_group": Lg, "batch": B,
                    "seq_len": T, "kv_heads": H, "q_heads": Hq, "head_dim": 128, "group": cfgd["g"],
                    "anchor_bits": cfgd["ba"], "resid_bits": cfgd["br"], "parallelism": f"replicas x{world}",
+                   "step_calls": ("rq_append + rq_decode_attn_bf16" if args.bf16 else
+                                  "rq_append + rq_decode_attn" if args.separate_append else "rq_append_decode_attn"),
                    "l2": "inputs larger than L2: %.1f GB of records read per step, loop-major over %d layers"
                          % (step_decode_bytes / 1e9, layers)},
         "decode_attn": {"ms_per_step": round(dec_ms / args.steps, 4), "us_per_call": round(dec_ms_call * 1e3, 3),
@@ -402,9 +409,11 @@ def run_ours(args, cfgd, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": int(step_decode_bytes / ncalls),
                      "kernel": "rq_decode_attn call (split kernel + combine)", "peak_kind": peak_kind},
         "e2e": e2e,
-        # per (layer, loop): one append-side kernel (tail copy, encoder or BF16 store) and one
-        # decode kernel that merges its own splits; the BF16 path adds a combine kernel
-        "gpu_launches": int(args.steps * loops * layers * (3 if args.bf16 else 2)),
+        # per (layer, loop): the fused call is one kernel for a non-anchor loop and the encoder +
+        # decode kernel at the anchor loop; separate calls add the tail-copy kernel; the BF16
+        # path is store + decode + combine
+        "gpu_launches": int(args.steps * layers * (3 * loops if args.bf16 else
+                                                    2 * loops if args.separate_append else loops + groups)),
         "clocks": clocks,
     }
     return res, cache, call_bytes
@@ -516,6 +525,8 @@ def main():
     ap.add_argument("--config", default="ouro8k_b4", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--bf16", action="store_true", help="time the uncompressed BF16 comparison kernel")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="rq_append then rq_decode_attn instead of the fused rq_append_decode_attn")
     ap.add_argument("--layers", type=int, default=0, help="override layer count (profiling runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

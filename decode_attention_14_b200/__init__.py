@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
     L.rq_append.argtypes = [vp, i32, i32, vp, vp, i32, vp]
     L.rq_decode_attn.restype = i32
     L.rq_decode_attn.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
+    L.rq_append_decode_attn.restype = i32
+    L.rq_append_decode_attn.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, ctypes.c_float, vp]
     L.rq_decode_attn_bf16.restype = i32
     L.rq_decode_attn_bf16.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
     L.rq_decode_attn_noalloc.restype = i32
@@ -181,6 +183,13 @@ def rq_decode_attn(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0,
                               softmax_scale, ctypes.c_void_p(_stream(stream)))
 
 
+def rq_append_decode_attn(h, layer: int, loop: int, k, v, n_tokens: int, q, out, softmax_scale: float = 0.0,
+                          stream=None) -> int:
+    return lib.rq_append_decode_attn(h, layer, loop, ctypes.c_void_p(_ptr(k)), ctypes.c_void_p(_ptr(v)), n_tokens,
+                                     ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(out)), softmax_scale,
+                                     ctypes.c_void_p(_stream(stream)))
+
+
 def rq_decode_attn_bf16(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0, stream=None) -> int:
     return lib.rq_decode_attn_bf16(h, layer, loop, ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(out)),
                                    softmax_scale, ctypes.c_void_p(_stream(stream)))
@@ -259,6 +268,20 @@ class Cache:
         _check_dev(out, "float32", (self.B, self.Hq, HEAD_DIM), "out")
         fn = rq_decode_attn_bf16 if bf16 else rq_decode_attn
         _ok(fn(self.h, layer, loop, q, out, scale, stream), fn.__name__)
+        return out
+
+    def append_decode(self, layer: int, loop: int, k, v, q, out=None, scale: float = 0.0, stream=None):
+        """rq_append then rq_decode_attn, fused into one launch where possible."""
+        import torch
+        n = k.shape[1]
+        shape = (self.B, n, self.H, HEAD_DIM)
+        _check_dev(k, "bfloat16", shape, "k")
+        _check_dev(v, "bfloat16", shape, "v")
+        _check_dev(q, "bfloat16", (self.B, self.Hq, HEAD_DIM), "q")
+        if out is None:
+            out = torch.empty((self.B, self.Hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+        _check_dev(out, "float32", (self.B, self.Hq, HEAD_DIM), "out")
+        _ok(rq_append_decode_attn(self.h, layer, loop, k, v, n, q, out, scale, stream), "rq_append_decode_attn")
         return out
 
     def length(self, layer: int, group: int) -> int:

@@ -76,10 +76,11 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; 
 float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt((float)kHeadDim); }
 
 // Split-KV partition of T tokens over `units` independent (sequence, kv head
-// [, q-head pair]) problems.  Chunks are whole 64-token tiles, at most
-// kMaxChunk.  Among the admissible split counts the one with the least
-// wave-quantised work (waves x tokens per CTA, plus a fixed per-CTA cost)
-// is taken, waves counted from the kernel's measured occupancy.
+// [, q-head pair]) problems.  The ceil(T/64) tiles are dealt out evenly over
+// S splits (split_range); chunk is the largest split, at most kMaxChunk.
+// Among the admissible split counts the one with the least wave-quantised
+// work (waves x tokens of the largest CTA, plus a fixed per-CTA cost) is
+// taken, waves counted from the kernel's measured occupancy.
 void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *chunk) {
     if (T <= 0) {
         *S = 0;
@@ -90,10 +91,10 @@ void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *
     const int s_hi = std::min(c->lay.splits_max, (T + kTokTile - 1) / kTokTile);
     long best_cost = -1;
     int best_s = s_lo, best_ch = kMaxChunk;
+    const int nt = (T + kTokTile - 1) / kTokTile;
     for (int s = s_lo; s <= std::max(s_lo, s_hi); s++) {
-        int ch = (T + s - 1) / s;
-        ch = (ch + kTokTile - 1) / kTokTile * kTokTile;
-        const int ss = (T + ch - 1) / ch;
+        const int ch = (nt + s - 1) / s * kTokTile;
+        const int ss = s;
         const int slots = std::max(1, c->occ[which][ch / kTokTile - 1] * c->sms);
         const long waves = ((long)ss * units + slots - 1) / slots;
         const long cost = waves * (ch + 2 * kTokTile);
@@ -369,9 +370,11 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
 // partials == nullptr: split partials and combine counters in the cache's
 // workspace (partial stride splits_max).  Otherwise in the caller's scratch
 // (stride = the split count this call uses).
+// app_k != nullptr: append app_n tokens to the loop first (rq_append_decode_attn).
 static int decode_common(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
                          void *stream, bool bf16, float *partials = nullptr, size_t partial_floats = 0,
-                         int *counters = nullptr, size_t max_units = 0) {
+                         int *counters = nullptr, size_t max_units = 0, const void *app_k = nullptr,
+                         const void *app_v = nullptr, int app_n = 0) {
     if (!c || !q || !out) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
@@ -429,6 +432,28 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         a.partials = partials;
         a.counters = counters;
     }
+    if (app_k) {
+        // one launch when the loop keeps the tokens in its tail and the split
+        // kernel runs (it writes the rows, then merges them); else append first
+        if (!(resid && a.S > 0)) {
+            int s = rq_append(c, layer, loop, app_k, app_v, app_n, stream);
+            if (s != RQ_OK) return s;
+            return decode_common(c, layer, loop, q, out, scale, stream, bf16);
+        }
+        int &nt = c->ntail[(size_t)layer * cfg.num_loops + loop];
+        if (nt + app_n > L.tail_cap) return RQ_ERR_CAPACITY;
+        const int group = loop / L.Lg, j = loop % L.Lg;
+        a.new_k = (const uint16_t *)app_k;
+        a.new_v = (const uint16_t *)app_v;
+        a.tail_k_w = (uint16_t *)tail_ptr(c, layer, group, j, 0);
+        a.tail_v_w = (uint16_t *)tail_ptr(c, layer, group, j, 1);
+        a.n_new = app_n;
+        a.tail_pos = nt;
+        a.n_tail = nt + app_n;
+        int s = cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st));
+        if (s == RQ_OK) nt += app_n;
+        return s;
+    }
     if (!bf16 && a.S > 0)   // the decode kernel merges its splits and the tail itself
         return cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st));
     if (bf16 && a.S > 0) {
@@ -469,6 +494,13 @@ extern "C" {
 
 int rq_decode_attn(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream) {
     return decode_common(c, layer, loop, q, out, scale, stream, false);
+}
+
+int rq_append_decode_attn(rq_cache *c, int layer, int loop, const void *k, const void *v, int n,
+                          const void *q, float *out, float scale, void *stream) {
+    if (!c || !k || !v || n <= 0) return RQ_ERR_INVALID;
+    if (c->lay.cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
+    return decode_common(c, layer, loop, q, out, scale, stream, false, nullptr, 0, nullptr, 0, k, v, n);
 }
 
 int rq_decode_attn_bf16(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,

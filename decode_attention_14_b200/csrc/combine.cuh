@@ -1,7 +1,8 @@
 // combine.cuh -- merging split-KV partials (max m_s, sum l_s, unnormalised
 // o_s, log2 domain) and BF16 tail tokens into one attention output row:
 //   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
-// with the tail tokens folded in one by one by the same rescaling rule.
+// with M = max_s m_s, then the tail tokens folded in one by one with a
+// running maximum.
 #pragma once
 
 #include <math_constants.h>
@@ -20,32 +21,61 @@ __device__ __forceinline__ void combine_row(const float *part, int S, const uint
                                             const uint16_t *tail_k, const uint16_t *tail_v, size_t tail_stride,
                                             int n_tail, float *out_row, int tid, float *red, Sync sync) {
     const int lane = tid & 31, warp = tid >> 5;
-    float M = -CUDART_INF_F, l = 0.f, o = 0.f;
-    for (int s = 0; s < S; s++) {
-        const float *p = part + (size_t)s * kPartialStride;
-        const float ms = __ldcg(p + kHeadDim), ls = __ldcg(p + kHeadDim + 1), os = __ldcg(p + tid);
-        const float nm = fmaxf(M, ms);
-        const float c0 = exp2f(M - nm), c1 = exp2f(ms - nm);
-        o = o * c0 + os * c1;
-        l = l * c0 + ls * c1;
-        M = nm;
-    }
+    // q and the first tail token are fetched first, so that their latency
+    // overlaps the partials' (L2 loads: the tail rows may have been written
+    // during this kernel by another CTA)
+    float q = 0.f, k0 = 0.f, v0 = 0.f;
     if (n_tail > 0) {
-        const float q = bf16_to_f32(q_row[tid]) * scale_log2;
-        for (int j = 0; j < n_tail; j++) {
-            const size_t row = (size_t)j * tail_stride;
-            float z = q * bf16_to_f32(tail_k[row + tid]);
-            for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
-            sync();
-            if (lane == 0) red[warp] = z;
-            sync();
-            z = red[0] + red[1] + red[2] + red[3];
-            const float nm = fmaxf(M, z);
-            const float c0 = exp2f(M - nm), c1 = exp2f(z - nm);
-            o = o * c0 + bf16_to_f32(tail_v[row + tid]) * c1;
-            l = l * c0 + c1;
-            M = nm;
+        q = bf16_to_f32(q_row[tid]) * scale_log2;
+        k0 = bf16_to_f32(__ldcg(tail_k + tid));
+        v0 = bf16_to_f32(__ldcg(tail_v + tid));
+    }
+    // partials, kBatch splits per round of loads: first M = max_s m_s, then
+    // the sums rescaled to it (padding slots carry m = -inf, weight 0)
+    constexpr int kBatch = 8;
+    float M = -CUDART_INF_F;
+    for (int s0 = 0; s0 < S; s0 += kBatch) {
+        float m[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; u++)
+            m[u] = (s0 + u < S) ? __ldcg(part + (size_t)(s0 + u) * kPartialStride + kHeadDim) : -CUDART_INF_F;
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) M = fmaxf(M, m[u]);
+    }
+    float l = 0.f, o = 0.f;
+    for (int s0 = 0; s0 < S; s0 += kBatch) {
+        float m[kBatch], ls[kBatch], os[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const bool in = s0 + u < S;
+            const float *p = part + (size_t)(s0 + u) * kPartialStride;
+            m[u] = in ? __ldcg(p + kHeadDim) : -CUDART_INF_F;
+            ls[u] = in ? __ldcg(p + kHeadDim + 1) : 0.f;
+            os[u] = in ? __ldcg(p + tid) : 0.f;
         }
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const float c = exp2f(m[u] - M);
+            l = fmaf(ls[u], c, l);
+            o = fmaf(os[u], c, o);
+        }
+    }
+    // tail tokens, folded in one by one with the running-max rule
+    for (int j = 0; j < n_tail; j++) {
+        const size_t row = (size_t)j * tail_stride;
+        const float kj = j == 0 ? k0 : bf16_to_f32(__ldcg(tail_k + row + tid));
+        const float vj = j == 0 ? v0 : bf16_to_f32(__ldcg(tail_v + row + tid));
+        float z = q * kj;
+        for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+        sync();
+        if (lane == 0) red[warp] = z;
+        sync();
+        z = red[0] + red[1] + red[2] + red[3];
+        const float nm = fmaxf(M, z);
+        const float c0 = exp2f(M - nm), c1 = exp2f(z - nm);
+        o = o * c0 + vj * c1;
+        l = l * c0 + c1;
+        M = nm;
     }
     out_row[tid] = (l > 0.f) ? o / l : 0.f;
 }

@@ -39,8 +39,8 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, sub = lane >> 3, seg = lane & 7;
     const int hq0 = h * a.G + pair * GK;
-    const int t0 = split * a.chunk;
-    const int n = min(a.chunk, a.T - t0);
+    int t0, n;
+    split_range(split, a.S, a.T, &t0, &n);
     const size_t bh = (size_t)b * a.H + h;
 
 #pragma unroll

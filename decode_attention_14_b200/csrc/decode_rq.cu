@@ -53,7 +53,15 @@
 namespace rq {
 namespace {
 
-constexpr int kTile = 64;
+constexpr int kTile = 64;   // tokens of one thread-map pass: 4 consumer warps x 16
+#ifndef RQ_DECODE_ITEM_TILES
+#define RQ_DECODE_ITEM_TILES 2
+#endif
+constexpr int kItemTiles = RQ_DECODE_ITEM_TILES;   // tiles per ring item
+constexpr int kItem = kTile * kItemTiles;          // tokens per ring item
+#ifndef RQ_DECODE_PAIR_VOTE
+#define RQ_DECODE_PAIR_VOTE 1
+#endif
 #ifndef RQ_DECODE_PRODUCER_SLEEP_NS
 #define RQ_DECODE_PRODUCER_SLEEP_NS 0
 #endif
@@ -274,7 +282,7 @@ __device__ __forceinline__ float fixed_scale(float bound, int top) {
     return ldexpf(1.f, F);
 }
 
-// Shared-memory plan of one CTA (bytes).  Items are 64 tokens; they are placed
+// Shared-memory plan of one CTA (bytes).  Items are kItem tokens; they are placed
 // back to back in a byte ring (an item never straddles its end), so the
 // number in flight follows their size: about 4 K items, 7 anchor V items or
 // 12 residual V items at once.
@@ -284,16 +292,16 @@ struct Plan {
     static constexpr int R_C = 16 * BR;              // residual codes per record
     static constexpr int MR = 2 * (kHeadDim / GS);   // meta bytes per record
     // K item: anchor codes | anchor meta | residual codes | residual meta | coefficients
-    static constexpr int K_AM = kTile * A_C;
-    static constexpr int K_RC = K_AM + kTile * MR;
-    static constexpr int K_RM = K_RC + (RESID ? kTile * R_C : 0);
-    static constexpr int K_CF = K_RM + (RESID ? kTile * MR : 0);
-    static constexpr int K_BYTES = K_CF + (RESID ? kTile * 2 : 0);
+    static constexpr int K_AM = kItem * A_C;
+    static constexpr int K_RC = K_AM + kItem * MR;
+    static constexpr int K_RM = K_RC + (RESID ? kItem * R_C : 0);
+    static constexpr int K_CF = K_RM + (RESID ? kItem * MR : 0);
+    static constexpr int K_BYTES = K_CF + (RESID ? kItem * 2 : 0);
     // V items: codes | meta, anchor items then residual items
-    static constexpr int VA_M = kTile * A_C;
-    static constexpr int VA_BYTES = VA_M + kTile * MR;
-    static constexpr int VR_M = kTile * R_C;
-    static constexpr int VR_BYTES = VR_M + kTile * MR;
+    static constexpr int VA_M = kItem * A_C;
+    static constexpr int VA_BYTES = VA_M + kItem * MR;
+    static constexpr int VR_M = kItem * R_C;
+    static constexpr int VR_BYTES = VR_M + kItem * MR;
     static constexpr int RING = kRingBytes;
     static_assert(K_BYTES % 128 == 0 && VA_BYTES % 128 == 0 && VR_BYTES % 128 == 0, "item alignment");
     static_assert(K_BYTES <= RING && VA_BYTES <= RING, "ring too small");
@@ -331,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int npairs = a.G / GK;
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int hq0 = h * a.G + pair * GK;
-    const int t0 = split * a.chunk;
-    const int n = min(a.chunk, a.T - t0);
+    int t0, n;
+    split_range(split, a.S, a.T, &t0, &n);
     const int ntiles = (n + kTile - 1) / kTile;
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
                 bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
             }
-            // Items in order: K tiles, anchor V tiles, residual V tiles.  Item it
+            // Items in order: K items, anchor V items, residual V items.  Item it
             // occupies [virt, virt + bytes) of an unbounded virtual byte
             // sequence, padded so that no item straddles the ring's end; its
             // ring offset is phys = virt mod RING.  Before it is issued, every
@@ -368,29 +376,30 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // loop keeps all of this in running counters (no division).
             const int npass = RESID ? 3 : 2;
             int it = 0, virt = 0, phys = 0;
-            int rel = 0, vrel = 0, rphys = 0, rtile = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
+            const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // items per pass
+            int rel = 0, vrel = 0, rphys = 0, ritem = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
             bool ok = true;
             for (int pass = 0; pass < npass && ok; pass++) {
                 const int bytes = P::item_bytes(pass);
                 const uint8_t *c0, *c1 = nullptr;   // code and meta sources of this pass's first tile
-                int cstride = 0, c1stride = P::MR * kTile;
+                int cstride = 0, c1stride = P::MR * kItem;
                 if (pass == 0) {
                     c0 = a.a_codes[0] + tok0 * P::A_C;
                     c1 = a.a_meta[0] + tok0 * P::MR;
-                    cstride = P::A_C * kTile;
+                    cstride = P::A_C * kItem;
                 } else if (pass == 1) {
                     c0 = a.a_codes[1] + tok0 * P::A_C;
                     c1 = a.a_meta[1] + tok0 * P::MR;
-                    cstride = P::A_C * kTile;
+                    cstride = P::A_C * kItem;
                 } else {
                     c0 = a.r_codes[1] + tok0 * P::R_C;
                     c1 = a.r_meta[1] + tok0 * P::MR;
-                    cstride = P::R_C * kTile;
+                    cstride = P::R_C * kItem;
                 }
                 const uint8_t *r0 = RESID ? a.r_codes[0] + tok0 * P::R_C : nullptr;
                 const uint8_t *r1 = RESID ? a.r_meta[0] + tok0 * P::MR : nullptr;
                 const uint8_t *r2 = RESID ? reinterpret_cast<const uint8_t *>(a.r_coef[0] + tok0) : nullptr;
-                for (int i = 0; i < ntiles; i++, it++) {
+                for (int j = 0; j < nitems; j++, it++) {
                     if (phys + bytes > P::RING) {
                         virt += P::RING - phys;
                         phys = 0;
@@ -403,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         }
                         vrel += rbytes;
                         rphys += rbytes;
-                        if (++rtile == ntiles) {
-                            rtile = 0;
+                        if (++ritem == nitems) {
+                            ritem = 0;
                             rbytes = P::item_bytes(++rpass);
                         }
                         if (rphys + rbytes > P::RING) {
@@ -418,23 +427,27 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         atomicExch(a.err, 1);
                         break;
                     }
+                    // the last item of a pass may hold fewer tiles: copy only those
+                    const int toks = min(kItem, (ntiles - j * kItemTiles) * kTile);
                     uint8_t *st = ring + phys;
                     uint64_t *bar = &bar_full[it % kSlots];
-                    mbar_expect_tx(bar, (uint32_t)bytes);
                     if (pass == 0) {
-                        bulk_g2s(st, c0, kTile * P::A_C, bar);
-                        bulk_g2s(st + P::K_AM, c1, kTile * P::MR, bar);
+                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + (RESID ? P::R_C + P::MR + 2 : 0))));
+                        bulk_g2s(st, c0, toks * P::A_C, bar);
+                        bulk_g2s(st + P::K_AM, c1, toks * P::MR, bar);
                         if (RESID) {
-                            bulk_g2s(st + P::K_RC, r0, kTile * P::R_C, bar);
-                            bulk_g2s(st + P::K_RM, r1, kTile * P::MR, bar);
-                            bulk_g2s(st + P::K_CF, r2, kTile * 2, bar);
-                            r0 += kTile * P::R_C;
-                            r1 += kTile * P::MR;
-                            r2 += kTile * 2;
+                            bulk_g2s(st + P::K_RC, r0, toks * P::R_C, bar);
+                            bulk_g2s(st + P::K_RM, r1, toks * P::MR, bar);
+                            bulk_g2s(st + P::K_CF, r2, toks * 2, bar);
+                            r0 += kItem * P::R_C;
+                            r1 += kItem * P::MR;
+                            r2 += kItem * 2;
                         }
                     } else {
-                        bulk_g2s(st, c0, (uint32_t)cstride, bar);
-                        bulk_g2s(st + cstride, c1, kTile * P::MR, bar);
+                        const int cb = pass == 1 ? P::A_C : P::R_C;
+                        mbar_expect_tx(bar, (uint32_t)(toks * (cb + P::MR)));
+                        bulk_g2s(st, c0, toks * cb, bar);
+                        bulk_g2s(st + cstride, c1, toks * P::MR, bar);
                     }
                     c0 += cstride;
                     c1 += c1stride;
@@ -453,6 +466,20 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     }
 
     // ------------------------------------------------------------ consumers
+    if (a.n_new > 0 && split == 0) {
+        // fused append: this unit's new tail rows (K and V, 16-byte vectors);
+        // the fence before the arrival count below publishes them to the
+        // CTA that combines
+        const int nvec = a.n_new * 2 * (kHeadDim / 8);
+        for (int i = tid; i < nvec; i += kConsumers) {
+            const int vec = i % (kHeadDim / 8), r = i / (kHeadDim / 8), kv = r & 1, t = r >> 1;
+            const uint4 *src = reinterpret_cast<const uint4 *>((kv ? a.new_v : a.new_k) +
+                                                               (((size_t)b * a.n_new + t) * a.H + h) * kHeadDim);
+            uint4 *dst = reinterpret_cast<uint4 *>((kv ? a.tail_v_w : a.tail_k_w) +
+                                                   (((size_t)b * a.tail_cap + a.tail_pos + t) * a.H + h) * kHeadDim);
+            dst[vec] = src[vec];
+        }
+    }
     const int sub = lane >> 3, seg = lane & 7;
     const int mg = (seg * 16) / GS;   // quantization group of this lane's segment
 
@@ -542,55 +569,66 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
     const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
     const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
+    const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // ring items per pass
     int c_off = 0;   // ring offset of the current item (the producer's placement rule)
-    for (int i = 0; i < ntiles; i++) {
-        const int slot = i % kSlots;
-        const bool ok = mbar_wait(&bar_full[slot], (i / kSlots) & 1, &s_abort);
+    for (int j = 0; j < nitems; j++) {
+        const int slot = j % kSlots;
+        const bool ok = mbar_wait(&bar_full[slot], (j / kSlots) & 1, &s_abort);
         if (!ok) {
             s_abort = 1;
             atomicExch(a.err, 2);
         }
         const uint8_t *st = ring + c_off;
-        float part[GK][4];
+        float part[kItemTiles][GK][4];
 #pragma unroll
-        for (int k = 0; k < 4; k++) {
-            const int tok = 16 * warp + sub + 4 * k;
-            const Seg<BA> ca = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
-            const float2 ma = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_AM + tok * P::MR + 2 * mg));
-            float shat = 1.f;
-            Seg<BR> cr;
-            float2 mr = make_float2(0.f, 0.f);
-            if (RESID) {
-                cr = lds_seg<BR>(st + P::K_RC + tok * P::R_C + seg * (2 * BR));
-                mr = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_RM + tok * P::MR + 2 * mg));
-                shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + P::K_CF + 2 * tok));
-            }
+        for (int u = 0; u < kItemTiles; u++) {
+            if (j * kItemTiles + u >= ntiles) break;   // uniform: a short last item
 #pragma unroll
-            for (int gq = 0; gq < GK; gq++) {
-                const float A = fmaf(ma.y, QA[gq], ma.x * __int2float_rn(dot_seg<BA>(ca, qA[gq])));
-                float v = A;
+            for (int k = 0; k < 4; k++) {
+                const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
+                const Seg<BA> ca = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
+                const float2 ma =
+                    meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_AM + tok * P::MR + 2 * mg));
+                float shat = 1.f;
+                Seg<BR> cr;
+                float2 mr = make_float2(0.f, 0.f);
                 if (RESID) {
-                    const float R = fmaf(mr.y, QR[gq], mr.x * __int2float_rn(dot_seg<BR>(cr, qR[gq])));
-                    v = fmaf(shat, A, R);
+                    cr = lds_seg<BR>(st + P::K_RC + tok * P::R_C + seg * (2 * BR));
+                    mr = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_RM + tok * P::MR + 2 * mg));
+                    shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + P::K_CF + 2 * tok));
                 }
-                part[gq][k] = v;
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) {
+                    const float A = fmaf(ma.y, QA[gq], ma.x * __int2float_rn(dot_seg<BA>(ca, qA[gq])));
+                    float v = A;
+                    if (RESID) {
+                        const float R = fmaf(mr.y, QR[gq], mr.x * __int2float_rn(dot_seg<BR>(cr, qR[gq])));
+                        v = fmaf(shat, A, R);
+                    }
+                    part[u][gq][k] = v;
+                }
             }
         }
         mbar_arrive(&bar_empty[slot]);
-        c_off = P::advance(c_off, P::K_BYTES, i + 1 < ntiles ? P::K_BYTES : P::VA_BYTES);
+        c_off = P::advance(c_off, P::K_BYTES, j + 1 < nitems ? P::K_BYTES : P::VA_BYTES);
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
-        const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
-        for (int gq = 0; gq < GK; gq++) {
-            float r0 = (b4 ? part[gq][2] : part[gq][0]) +
-                       __shfl_xor_sync(0xffffffffu, b4 ? part[gq][0] : part[gq][2], 4);
-            float r1 = (b4 ? part[gq][3] : part[gq][1]) +
-                       __shfl_xor_sync(0xffffffffu, b4 ? part[gq][1] : part[gq][3], 4);
-            float r = (b2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b2 ? r0 : r1, 2);
-            r += __shfl_xor_sync(0xffffffffu, r, 1);
-            r *= qinv;
-            if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;   // tl < ntiles*64 <= chunk
-            if (tl < n && ok) mloc[gq] = fmaxf(mloc[gq], r);
+        for (int u = 0; u < kItemTiles; u++) {
+            const int i = j * kItemTiles + u;
+            if (i >= ntiles) break;
+            const int tl = i * kTile + 16 * warp + sub + 4 * kown;
+#pragma unroll
+            for (int gq = 0; gq < GK; gq++) {
+                float r0 = (b4 ? part[u][gq][2] : part[u][gq][0]) +
+                           __shfl_xor_sync(0xffffffffu, b4 ? part[u][gq][0] : part[u][gq][2], 4);
+                float r1 = (b4 ? part[u][gq][3] : part[u][gq][1]) +
+                           __shfl_xor_sync(0xffffffffu, b4 ? part[u][gq][1] : part[u][gq][3], 4);
+                float r = (b2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b2 ? r0 : r1, 2);
+                r += __shfl_xor_sync(0xffffffffu, r, 1);
+                r *= qinv;
+                if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;   // tl < ntiles*64 <= chunk
+                if (tl < n && ok) mloc[gq] = fmaxf(mloc[gq], r);
+            }
         }
     }
 
@@ -679,73 +717,81 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 accHi[gq][e] = 0;
             }
         }
-        for (int i = 0; i < ntiles; i++) {
-            const int it = (1 + vp) * ntiles + i;
+        for (int j = 0; j < nitems; j++) {
+            const int it = (1 + vp) * nitems + j;
             const int slot = it % kSlots;
             if (!mbar_wait(&bar_full[slot], (it / kSlots) & 1, &s_abort)) {
                 s_abort = 1;
                 atomicExch(a.err, 4);
             }
             const uint8_t *st = ring + c_off;
-            uint32_t wlo[GK][2], whi[GK][2];
-            float2 mm[4];
-            float W[GK][4];
-            Seg<BA> ca[4];
-            Seg<BR> cr[4];
+            const int last_u = min(kItemTiles, ntiles - j * kItemTiles) - 1;   // a short last item
 #pragma unroll
-            for (int k = 0; k < 4; k++) {
-                const int tok = 16 * warp + sub + 4 * k;
-                if (vp == 0) {
-                    ca[k] = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
-                    mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VA_M + tok * P::MR + 2 * mg));
-                } else {
-                    cr[k] = lds_seg<BR>(st + tok * P::R_C + seg * (2 * BR));
-                    mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VR_M + tok * P::MR + 2 * mg));
-                }
-#pragma unroll
-                for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + i * kTile + tok];
-            }
-            mbar_arrive(&bar_empty[slot]);
-            {
-                const int cur = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
-                c_off = P::advance(c_off, cur, i + 1 < ntiles ? cur : P::VR_BYTES);
-            }
-            uint32_t hi_any = 0;
-#pragma unroll
-            for (int gq = 0; gq < GK; gq++) {
-                int wi[4];
+            for (int u = 0; u < kItemTiles; u++) {
+                if (u > last_u) break;   // uniform
+                uint32_t wlo[GK][2], whi[GK][2];
+                float2 mm[4];
+                float W[GK][4];
+                Seg<BA> ca[4];
+                Seg<BR> cr[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    wi[k] = __float2int_rn(W[gq][k] * mm[k].x);   // W carries the scale 2^F
-                    mS[gq] = fmaf(W[gq][k], mm[k].y, mS[gq]);
-                }
-#pragma unroll
-                for (int pr = 0; pr < 2; pr++) {
-                    wlo[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x5410);
-                    whi[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x7632);
-                    hi_any |= whi[gq][pr];
-                }
-            }
-            // small weights (most tokens of a peaked softmax) have zero high
-            // halves; when no lane of the warp has one, skip their products
-            const bool need_hi = __any_sync(0xffffffffu, hi_any != 0);
-#pragma unroll
-            for (int gq = 0; gq < GK; gq++) {
-                if (vp == 0) {
-                    if (need_hi) {
-                        acc_pair<BA>(ca[0], ca[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                        acc_pair<BA>(ca[2], ca[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
+                    const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
+                    if (vp == 0) {
+                        ca[k] = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
+                        mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VA_M + tok * P::MR + 2 * mg));
                     } else {
-                        acc_pair<BA, false>(ca[0], ca[1], wlo[gq][0], 0u, accLo[gq], accHi[gq]);
-                        acc_pair<BA, false>(ca[2], ca[3], wlo[gq][1], 0u, accLo[gq], accHi[gq]);
+                        cr[k] = lds_seg<BR>(st + tok * P::R_C + seg * (2 * BR));
+                        mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VR_M + tok * P::MR + 2 * mg));
                     }
+#pragma unroll
+                    for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + j * kItem + tok];
+                }
+                if (u == last_u) {   // every read of the item is done: release it
+                    mbar_arrive(&bar_empty[slot]);
+                    const int cur = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
+                    c_off = P::advance(c_off, cur, j + 1 < nitems ? cur : P::VR_BYTES);
+                }
+                uint32_t hi_any[2] = {0u, 0u};   // per token pair
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) {
+                    int wi[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        wi[k] = __float2int_rn(W[gq][k] * mm[k].x);   // W carries the scale 2^F
+                        mS[gq] = fmaf(W[gq][k], mm[k].y, mS[gq]);
+                    }
+#pragma unroll
+                    for (int pr = 0; pr < 2; pr++) {
+                        wlo[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x5410);
+                        whi[gq][pr] = __byte_perm((uint32_t)wi[2 * pr], (uint32_t)wi[2 * pr + 1], 0x7632);
+                        hi_any[pr] |= whi[gq][pr];
+                    }
+                }
+                // small weights (most tokens of a peaked softmax) have zero high
+                // halves; when no lane of the warp has one, skip their products
+                bool need_hi[2];
+                if (RQ_DECODE_PAIR_VOTE) {
+                    need_hi[0] = __any_sync(0xffffffffu, hi_any[0] != 0);
+                    need_hi[1] = __any_sync(0xffffffffu, hi_any[1] != 0);
                 } else {
-                    if (need_hi) {
-                        acc_pair<BR>(cr[0], cr[1], wlo[gq][0], whi[gq][0], accLo[gq], accHi[gq]);
-                        acc_pair<BR>(cr[2], cr[3], wlo[gq][1], whi[gq][1], accLo[gq], accHi[gq]);
-                    } else {
-                        acc_pair<BR, false>(cr[0], cr[1], wlo[gq][0], 0u, accLo[gq], accHi[gq]);
-                        acc_pair<BR, false>(cr[2], cr[3], wlo[gq][1], 0u, accLo[gq], accHi[gq]);
+                    need_hi[0] = need_hi[1] = __any_sync(0xffffffffu, (hi_any[0] | hi_any[1]) != 0);
+                }
+#pragma unroll
+                for (int gq = 0; gq < GK; gq++) {
+#pragma unroll
+                    for (int pr = 0; pr < 2; pr++) {
+                        if (vp == 0) {
+                            if (need_hi[pr])
+                                acc_pair<BA>(ca[2 * pr], ca[2 * pr + 1], wlo[gq][pr], whi[gq][pr], accLo[gq], accHi[gq]);
+                            else
+                                acc_pair<BA, false>(ca[2 * pr], ca[2 * pr + 1], wlo[gq][pr], 0u, accLo[gq], accHi[gq]);
+                        } else {
+                            if (need_hi[pr])
+                                acc_pair<BR>(cr[2 * pr], cr[2 * pr + 1], wlo[gq][pr], whi[gq][pr], accLo[gq], accHi[gq]);
+                            else
+                                acc_pair<BR, false>(cr[2 * pr], cr[2 * pr + 1], wlo[gq][pr], 0u, accLo[gq], accHi[gq]);
+                        }
                     }
                 }
             }

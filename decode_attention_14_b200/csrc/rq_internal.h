@@ -110,12 +110,26 @@ struct DecodeArgs {
     float *out;               // [B][Hq][d] fp32
     const uint16_t *tail_k, *tail_v;   // [B][tail_cap][H][d] BF16 in-flight tokens, or null
     int n_tail, tail_cap;
+    // fused append: n_new tokens [B][n_new][H][d] written to tail rows
+    // tail_pos.. (included in n_tail) by split 0 of each unit before the combine
+    const uint16_t *new_k, *new_v;
+    uint16_t *tail_k_w, *tail_v_w;
+    int n_new, tail_pos;
     int B, H, Hq, G, T, Tp, S, chunk, splits_max;
     int g;
     float scale_log2;         // softmax_scale * log2(e)
     int rotate;
     uint32_t sigma[4];
 };
+
+// Tokens [*t0, *t0 + *n) of split `split` of S: the ceil(T/64) tiles are
+// dealt out evenly (tile counts differ by at most one; chunk >= the largest).
+__host__ __device__ inline void split_range(int split, int S, int T, int *t0, int *n) {
+    const int nt = (T + kTokTile - 1) / kTokTile;
+    const int lo = (int)((long long)split * nt / S), hi = (int)((long long)(split + 1) * nt / S);
+    *t0 = lo * kTokTile;
+    *n = (hi * kTokTile < T ? hi * kTokTile : T) - *t0;
+}
 
 struct CombineArgs {
     const float *partials;

@@ -162,6 +162,22 @@ int rq_append(rq_cache *cache, int layer, int loop, const void *k_bf16, const vo
 int rq_decode_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
                    float softmax_scale, void *stream);
 
+/*
+ * rq_append(cache, layer, loop, k, v, n_tokens) followed by
+ * rq_decode_attn(cache, layer, loop, q, out, softmax_scale) on the same
+ * stream, with the same results, state changes and errors.  For a non-anchor
+ * loop of an RQ_FMT_RESIDUAL cache holding committed tokens, it is one kernel
+ * launch: the decode kernel writes the new tokens into the loop's BF16 tail
+ * itself before merging the tail (the per-step order of the ai4snews
+ * summary's decode: the new token's earlier loops are kept uncompressed and
+ * attended to).  Otherwise it enqueues the two calls.  The paper has no
+ * counterpart to the fusion; it saves a launch per non-anchor loop.
+ *   k_bf16, v_bf16: as for rq_append; q_bf16, out: as for rq_decode_attn.
+ * Errors: INVALID, CAPACITY, STATE, CUDA; on error nothing is appended.
+ */
+int rq_append_decode_attn(rq_cache *cache, int layer, int loop, const void *k_bf16, const void *v_bf16,
+                          int n_tokens, const void *q_bf16, float *out, float softmax_scale, void *stream);
+
 /* The same attention over an RQ_FMT_BF16 cache: the uncompressed comparison
  * kernel (the role BF16 FlashAttention plays in the ai4snews summary,
  * paragraph 4).  Errors: INVALID, STATE (wrong format), CUDA. */
