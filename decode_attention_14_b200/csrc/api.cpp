@@ -193,7 +193,7 @@ int rq_config_check(const rq_config *c) {
     }
     // size sanity: every per-stream offset must fit the kernels' 64-bit math
     // and the token index the kernels' 32-bit math
-    if (c->max_tokens > (1 << 20) || c->max_tail_tokens > (1 << 20)) return RQ_ERR_UNSUPPORTED;
+    if (c->max_tokens > kMaxSplits * kMaxChunk || c->max_tail_tokens > (1 << 20)) return RQ_ERR_UNSUPPORTED;
     return RQ_OK;
 }
 
@@ -603,8 +603,10 @@ int rq_check(rq_cache *c) {
     if (cudaMemcpy(&err, c->base + c->lay.off_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return RQ_ERR_CUDA;
     if (err != 0) {
-        int zero = 0;
-        cudaMemcpy(c->base + c->lay.off_err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        // a call that gave up may have left its arrival counters part-way:
+        // clear them with the error word so that the next call starts clean
+        cudaMemset(c->base + c->lay.off_counters, 0, c->lay.off_err + sizeof(int) - c->lay.off_counters);
+        cudaDeviceSynchronize();
         return RQ_ERR_TIMEOUT;
     }
     return RQ_OK;

@@ -61,7 +61,8 @@ typedef enum {
  *                    of 4, per the ai4snews summary, paragraph 1).
  *                    num_loops % loops_per_group == 0.
  *   batch            sequences B; every sequence has the same length
- *   max_tokens       committed-token capacity per (layer, group)
+ *   max_tokens       committed-token capacity per (layer, group), at most
+ *                    262144 (256 split partials of up to 1024 tokens)
  *   max_tail_tokens  in-flight tokens a non-anchor loop may hold before the
  *                    group's anchor commits them
  *   num_kv_heads     H_kv

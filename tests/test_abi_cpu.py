@@ -47,6 +47,9 @@ def test_config_validation():
     assert rq.rq_config_check(_cfg(loops_per_group=1, max_tail_tokens=0)) == rq.RQ_OK
     assert rq.rq_config_check(_cfg(format=rq.RQ_FMT_BF16, group_size=0)) == rq.RQ_OK
     assert rq.rq_cache_required_bytes(_cfg(head_dim=64)) == 0
+    # at most 256 split partials of at most 1024 tokens per (sequence, head)
+    assert rq.rq_config_check(_cfg(batch=1, max_tokens=262144)) == rq.RQ_OK
+    assert rq.rq_config_check(_cfg(batch=1, max_tokens=262145)) == rq.RQ_ERR_UNSUPPORTED
 
 
 def test_token_bytes_reproduce_storage_reduction():
