@@ -197,13 +197,6 @@ __device__ __forceinline__ int dot_seg(const Seg<BITS> &s, const QPlanes &q) {
     return (int)(((unsigned)hi << 16) + (mid << 8) + lo);
 }
 
-// acc{Lo,Hi}[i] += 2^acc_shift(i) (w0 * c0_i + w1 * c1_i) for the 16 elements
-// of a segment, codes of two tokens; weights as 16-bit halves: wlo =
-// (w0 & 0xFFFF) | (w1 << 16) (unsigned), whi = (w0 >> 16) | (w1 >> 16) << 16
-// (signed).  Codes are masked in place rather than shifted down, so element
-// i's sums carry the factor 2^acc_shift(i), removed once at the end (the sums
-// stay below 2^30 for the 64 tokens a lane takes per chunk).
-// HI = false skips the high halves (exact when they are zero).
 // dp2a with signed 16-bit halves of a and UNSIGNED bytes of b (the masked
 // codes reach 240, beyond int8).
 __device__ __forceinline__ int dp2a_lo_su(int a, uint32_t b, int c) {
@@ -222,48 +215,71 @@ __host__ __device__ constexpr int acc_shift(int e) {
     return BITS == 4 ? ((e & 1) ? 4 : 0) : 2 * (e & 3);
 }
 
-template <int BITS, bool HI = true>
-__device__ __forceinline__ void acc_pair(const Seg<BITS> &a, const Seg<BITS> &b, uint32_t wlo, uint32_t whi,
-                                         unsigned accLo[16], int accHi[16]) {
-    const int Wh = (int)whi;
+// The code words of one segment for a pair of tokens, masked in place:
+// word i feeds the dp2a of elements pair_elem(i) (low half of the word) and
+// pair_elem(i) + pair_step (high half), codes of both tokens side by side.
+template <int BITS>
+struct PairCodes {
+    uint32_t c[8];
+};
+template <int BITS>
+__host__ __device__ constexpr int pair_elem(int i) {
+    return BITS == 4 ? 8 * (i >> 2) + ((i & 3) < 2 ? (i & 3) : (i & 3) + 2) : (i < 4 ? i : i + 4);
+}
+template <int BITS>
+__host__ __device__ constexpr int pair_step() {
+    return BITS == 4 ? 2 : 4;
+}
+
+template <int BITS>
+__device__ __forceinline__ PairCodes<BITS> pair_codes(const Seg<BITS> &a, const Seg<BITS> &b) {
+    PairCodes<BITS> p;
     if (BITS == 4) {
 #pragma unroll
         for (int u = 0; u < 2; u++) {
             const uint32_t X = __byte_perm(a.w[u], b.w[u], 0x5140);   // bytes 0,1 of both tokens
             const uint32_t Y = __byte_perm(a.w[u], b.w[u], 0x7362);   // bytes 2,3 of both tokens
-            // c[0]: elements 8u+0 (bytes 0,1), 8u+2 (bytes 2,3); c[1]: 8u+1, 8u+3;
-            // c[2]: 8u+4, 8u+6; c[3]: 8u+5, 8u+7
-            const uint32_t c[4] = {X & 0x0F0F0F0Fu, X & 0xF0F0F0F0u, Y & 0x0F0F0F0Fu, Y & 0xF0F0F0F0u};
-            const int e0[4] = {0, 1, 4, 5};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                const int e = 8 * u + e0[k];
-                accLo[e] = __dp2a_lo(wlo, c[k], accLo[e]);
-                accLo[e + 2] = __dp2a_hi(wlo, c[k], accLo[e + 2]);
-                if (HI) {
-                    accHi[e] = dp2a_lo_su(Wh, c[k], accHi[e]);
-                    accHi[e + 2] = dp2a_hi_su(Wh, c[k], accHi[e + 2]);
-                }
-            }
+            p.c[4 * u + 0] = X & 0x0F0F0F0Fu;   // elements 8u+0, 8u+2
+            p.c[4 * u + 1] = X & 0xF0F0F0F0u;   // elements 8u+1, 8u+3 (x16)
+            p.c[4 * u + 2] = Y & 0x0F0F0F0Fu;   // elements 8u+4, 8u+6
+            p.c[4 * u + 3] = Y & 0xF0F0F0F0u;   // elements 8u+5, 8u+7 (x16)
         }
     } else {
         const uint32_t X = __byte_perm(a.w[0], b.w[0], 0x5140);   // bytes 0,1: elements 0-7
         const uint32_t Y = __byte_perm(a.w[0], b.w[0], 0x7362);   // bytes 2,3: elements 8-15
 #pragma unroll
         for (int c = 0; c < 4; c++) {
-            const uint32_t x = X & (0x03030303u << (2 * c));
-            const uint32_t y = Y & (0x03030303u << (2 * c));
-            accLo[c] = __dp2a_lo(wlo, x, accLo[c]);
-            accLo[4 + c] = __dp2a_hi(wlo, x, accLo[4 + c]);
-            accLo[8 + c] = __dp2a_lo(wlo, y, accLo[8 + c]);
-            accLo[12 + c] = __dp2a_hi(wlo, y, accLo[12 + c]);
-            if (HI) {
-                accHi[c] = dp2a_lo_su(Wh, x, accHi[c]);
-                accHi[4 + c] = dp2a_hi_su(Wh, x, accHi[4 + c]);
-                accHi[8 + c] = dp2a_lo_su(Wh, y, accHi[8 + c]);
-                accHi[12 + c] = dp2a_hi_su(Wh, y, accHi[12 + c]);
-            }
+            p.c[c] = X & (0x03030303u << (2 * c));       // elements c, 4+c (x4^c)
+            p.c[4 + c] = Y & (0x03030303u << (2 * c));   // elements 8+c, 12+c (x4^c)
         }
+    }
+    return p;
+}
+
+// accLo[i] += 2^acc_shift(i) (w0 * c0_i + w1 * c1_i) with the low 16-bit
+// halves wlo = (w0 & 0xFFFF) | (w1 << 16); acc_hi the same with the signed
+// high halves whi = (w0 >> 16) | (w1 >> 16) << 16.  Codes are masked in
+// place rather than shifted down, so element i's sums carry the factor
+// 2^acc_shift(i), removed once at the end (the sums stay below 2^30 for the
+// 64 tokens a lane takes per chunk).
+template <int BITS>
+__device__ __forceinline__ void acc_lo(const PairCodes<BITS> &p, uint32_t wlo, unsigned accLo[16]) {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        constexpr int s = pair_step<BITS>();
+        const int e = pair_elem<BITS>(i);
+        accLo[e] = __dp2a_lo(wlo, p.c[i], accLo[e]);
+        accLo[e + s] = __dp2a_hi(wlo, p.c[i], accLo[e + s]);
+    }
+}
+template <int BITS>
+__device__ __forceinline__ void acc_hi(const PairCodes<BITS> &p, uint32_t whi, int accHi[16]) {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        constexpr int s = pair_step<BITS>();
+        const int e = pair_elem<BITS>(i);
+        accHi[e] = dp2a_lo_su((int)whi, p.c[i], accHi[e]);
+        accHi[e + s] = dp2a_hi_su((int)whi, p.c[i], accHi[e + s]);
     }
 }
 
@@ -778,19 +794,22 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     need_hi[0] = need_hi[1] = __any_sync(0xffffffffu, (hi_any[0] | hi_any[1]) != 0);
                 }
 #pragma unroll
-                for (int gq = 0; gq < GK; gq++) {
+                for (int pr = 0; pr < 2; pr++) {
+                    if (vp == 0) {
+                        const PairCodes<BA> pc = pair_codes<BA>(ca[2 * pr], ca[2 * pr + 1]);
 #pragma unroll
-                    for (int pr = 0; pr < 2; pr++) {
-                        if (vp == 0) {
-                            if (need_hi[pr])
-                                acc_pair<BA>(ca[2 * pr], ca[2 * pr + 1], wlo[gq][pr], whi[gq][pr], accLo[gq], accHi[gq]);
-                            else
-                                acc_pair<BA, false>(ca[2 * pr], ca[2 * pr + 1], wlo[gq][pr], 0u, accLo[gq], accHi[gq]);
-                        } else {
-                            if (need_hi[pr])
-                                acc_pair<BR>(cr[2 * pr], cr[2 * pr + 1], wlo[gq][pr], whi[gq][pr], accLo[gq], accHi[gq]);
-                            else
-                                acc_pair<BR, false>(cr[2 * pr], cr[2 * pr + 1], wlo[gq][pr], 0u, accLo[gq], accHi[gq]);
+                        for (int gq = 0; gq < GK; gq++) acc_lo<BA>(pc, wlo[gq][pr], accLo[gq]);
+                        if (need_hi[pr]) {
+#pragma unroll
+                            for (int gq = 0; gq < GK; gq++) acc_hi<BA>(pc, whi[gq][pr], accHi[gq]);
+                        }
+                    } else {
+                        const PairCodes<BR> pc = pair_codes<BR>(cr[2 * pr], cr[2 * pr + 1]);
+#pragma unroll
+                        for (int gq = 0; gq < GK; gq++) acc_lo<BR>(pc, wlo[gq][pr], accLo[gq]);
+                        if (need_hi[pr]) {
+#pragma unroll
+                            for (int gq = 0; gq < GK; gq++) acc_hi<BR>(pc, whi[gq][pr], accHi[gq]);
                         }
                     }
                 }
