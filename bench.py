@@ -517,6 +517,100 @@ def run_reference(args, cfgd):
     }
 
 
+# ---------------------------------------------------------------- batch / format sweep
+SWEEP_FORMATS = [
+    # name, (group, anchor bits, residual bits, rotate) or None for the BF16 cache
+    ("mixed_g16", (16, 4, 2, True)),
+    ("mixed_g32", (32, 4, 2, True)),
+    ("mixed_g16_rotation_off", (16, 4, 2, False)),
+    ("uniform_int2_g16", (16, 2, 2, True)),
+    ("bf16", None),
+]
+
+
+def run_sweep(args):
+    """Ouro-1.4B shape at T = 8192: for each format, batch 1, 2, 4, ... up
+    to the largest power of two whose 24-layer cache fits in free device
+    memory (at most 128).  Each row times the decode calls of one filled
+    layer (every layer issues the same calls) and scales to the 24 x 4 calls
+    of a decode step: tokens/s = batch / step time; GB/s over the calls'
+    algorithmic bytes."""
+    import torch
+    import decode_attention_14_b200 as rq
+    from decode_attention_14_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = CONFIGS["ouro8k_b4"]
+    loops, Lg, T, H, Hq, layers = base["loops"], base["Lg"], base["T"], base["H"], base["Hq"], base["layers"]
+    peak, peak_kind = _peaks()
+    reps = 20
+    rows = []
+    for name, fmt in SWEEP_FORMATS:
+        kw = dict(num_layers=layers, num_loops=loops, loops_per_group=Lg, max_tokens=T, max_tail_tokens=FILL_CHUNK,
+                  num_kv_heads=H, num_q_heads=Hq, seed=0xA11CE)
+        if fmt is None:
+            kw.update(format=rq.RQ_FMT_BF16)
+        else:
+            kw.update(group_size=fmt[0], anchor_bits=fmt[1], resid_bits=fmt[2], rotate=fmt[3])
+        free, _ = torch.cuda.mem_get_info(dev)
+        token_bytes = rq.rq_cache_token_bytes(rq.make_config(batch=1, **kw))
+        bf16_token_bytes = rq.rq_cache_token_bytes(rq.make_config(batch=1, **dict(kw, format=rq.RQ_FMT_BF16)))
+        fit = 0
+        b = 1
+        while b <= 128 and rq.rq_cache_required_bytes(rq.make_config(batch=b, **kw)) <= free:
+            fit = b
+            b *= 2
+        b = 1
+        while b <= fit:
+            cfg = rq.make_config(batch=b, **dict(kw, num_layers=1))
+            cache = rq.Cache(cfg, device=dev)
+            seed = 0x5EED0005 + b
+            for t0 in range(0, T, FILL_CHUNK):
+                n = min(FILL_CHUNK, T - t0)
+                Kg, Vg = synth.group_kv(seed, 0, 0, Lg, base["sigma"], b, n, H, t0=t0, device=dev)
+                for j in range(Lg):
+                    cache.append(0, j, Kg[j], Vg[j])
+                del Kg, Vg
+            torch.cuda.synchronize(dev)
+            q = synth.queries(seed, 0, 0, 0, b, Hq, device=dev)
+            out = torch.empty((b, Hq, 128), dtype=torch.float32, device=dev)
+            fn = rq.rq_decode_attn_bf16 if fmt is None else rq.rq_decode_attn
+            us, byt = [], []
+            for lp in range(loops):
+                for _ in range(3):
+                    assert fn(cache.h, 0, lp, q, out, 0.0) == 0
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for _ in range(reps):
+                        st = fn(cache.h, 0, lp, q, out, 0.0)
+                        if st != 0:
+                            raise rq.RQError(st, fn.__name__)
+                g.replay()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                us.append(e0.elapsed_time(e1) * 1e3 / reps)
+                byt.append(cache.decode_bytes(0, lp))
+                del g
+            cache.check()
+            cache.close()
+            step_us = layers * sum(us)
+            gbs = sum(byt) / (sum(us) * 1e-6) / 1e9
+            row = {"sweep": "ouro8k", "format": name, "batch": b, "seq_len": T,
+                   "tokens_per_s": round(b / (step_us * 1e-6), 2), "decode_step_ms": round(step_us / 1e3, 4),
+                   "us_per_call": [round(x, 2) for x in us], "gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                   "peak": peak, "peak_kind": peak_kind, "largest_batch_fits": fit,
+                   "cache_bytes_per_token": token_bytes, "vs_bf16_bytes": round(token_bytes / bf16_token_bytes, 4),
+                   "timing": "CUDA graph of %d calls per loop on one filled layer, scaled to %d layers" % (reps, layers)}
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+            b *= 2
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -532,6 +626,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--json-out", default="")
+    ap.add_argument("--sweep", action="store_true",
+                    help="batch x format sweep of the Ouro shape at T=8192 (one JSON line per row)")
     ap.add_argument("--profile", action="store_true",
                     help="bracket the timed region with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     args = ap.parse_args()
@@ -542,6 +638,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         if rank == 0:
             res = run_reference(args, cfgd)
