@@ -556,9 +556,11 @@ def run_sweep(args):
         free, _ = torch.cuda.mem_get_info(dev)
         token_bytes = rq.rq_cache_token_bytes(rq.make_config(batch=1, **kw))
         bf16_token_bytes = rq.rq_cache_token_bytes(rq.make_config(batch=1, **dict(kw, format=rq.RQ_FMT_BF16)))
+        # the largest batch whose full cache (24 layers, a decode-time tail of
+        # 8 tokens per loop) fits in free device memory
         fit = 0
         b = 1
-        while b <= 128 and rq.rq_cache_required_bytes(rq.make_config(batch=b, **kw)) <= free:
+        while b <= 128 and rq.rq_cache_required_bytes(rq.make_config(batch=b, **dict(kw, max_tail_tokens=8))) <= free:
             fit = b
             b *= 2
         b = 1

@@ -104,6 +104,18 @@ def test_deep_recurrence_groups_small():
         _decode_and_check(bt, 0, loop)
 
 
+@pytest.mark.parametrize("Lg", [8, 16])
+def test_larger_loop_groups(Lg):
+    """Loop groups of 8 and 16 (one anchor per group, Lg - 1 residual loops
+    per anchor), sigma growing linearly with distance from the anchor."""
+    sigma = tuple(0.1 + 0.3 * d / (Lg - 2) for d in range(Lg - 1))
+    bt = H.build(layers=1, loops=2 * Lg, Lg=Lg, B=1, T=90, H=2, Hq=2, n_tail=1, sigma=sigma, seed=0x5EED6100 + Lg)
+    for grp in (0, 1):
+        _records_and_mse(bt, 0, grp)
+    for loop in (0, Lg // 2, Lg - 1, Lg, 2 * Lg - 2, 2 * Lg - 1):
+        _decode_and_check(bt, 0, loop)
+
+
 def test_bf16_comparison_kernel():
     bt = H.build(layers=1, loops=2, Lg=1, B=2, T=300, H=2, Hq=4, fmt=rq.RQ_FMT_BF16, seed=0x5EED7000)
     for loop in range(2):
