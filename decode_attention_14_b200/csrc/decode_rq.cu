@@ -347,7 +347,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     __shared__ __align__(8) uint64_t bar_full[kSlots];
     __shared__ __align__(8) uint64_t bar_empty[kSlots];
     __shared__ __align__(8) uint64_t bar_cf;
+    __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
     __shared__ int s_abort, s_last;
+    __shared__ unsigned s_cfmax;
     __shared__ float s_q[GK][2][kHeadDim];
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
     __shared__ int s_qsum[GK][2][8];                             // sum of each segment's fixed-point q
@@ -374,7 +376,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             mbar_init(&bar_empty[i], kConsumers);   // every consumer thread arrives
         }
         mbar_init(&bar_cf, 1);
+        mbar_init(&bar_cfmax, 31);
         s_abort = 0;
+        s_cfmax = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -481,6 +485,17 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             if (RESID) mbar_wait<256>(&bar_cf, 0, &s_abort);
             for (int it = max(0, issued - kSlots); it < issued; it++)
                 mbar_wait<256>(&bar_full[it % kSlots], (it / kSlots) & 1, &s_abort);
+        } else {
+            // the other lanes: the bound max |s_hat(V)| of the chunk's V
+            // coefficients (for the weights' fixed point), ready before the
+            // softmax needs it
+            unsigned m = 0;
+            if (RESID && mbar_wait<64>(&bar_cf, 0, &s_abort)) {
+                const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING);
+                for (int t = lane - 1; t < n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
+            }
+            atomicMax(&s_cfmax, m);
+            mbar_arrive(&bar_cfmax);
         }
         return;
     }
@@ -669,24 +684,29 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++)
         M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
     consumer_sync();   // everyone has read s_red
-    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V weight),
-    // zero beyond the chunk's tokens; the bound of |s_hat| for the fixed point
+    // the weights' fixed-point scales: w = P * sc (anchor) or p * sc
+    // (residual), |P| <= max|s_hat|, p <= 1, sc <= 448 (powers of two)
+    if (!mbar_wait(&bar_cfmax, 0, &s_abort)) {
+        s_abort = 1;
+        atomicExch(a.err, 3);
+    }
+    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax) * 448.f : 448.f, kWeightTop);
+    const float cR = fixed_scale(448.f, kWeightTop);
+    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V
+    // weight), zero beyond the chunk's tokens, stored with their scales
     float lsum[GK];
-    uint32_t cf_max = 0;
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
     for (int t = tid; t < ntiles * kTile; t += kConsumers) {
         const bool valid = t < n;
-        const uint16_t cf = RESID ? s_cf[t] : (uint16_t)0x3F80;
-        const float shv = bf16_to_f32(cf);
+        const float shv = RESID ? bf16_to_f32(s_cf[t]) : 1.f;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
             const float p = valid ? exp2f(s_sc[gq * a.chunk + t] - M[gq]) : 0.f;
             lsum[gq] += p;
-            s_sc[gq * a.chunk + t] = p;
-            s_P[gq * a.chunk + t] = p * shv;
+            s_sc[gq * a.chunk + t] = p * cR;
+            s_P[gq * a.chunk + t] = p * shv * cA;
         }
-        if (valid) cf_max = max(cf_max, (uint32_t)cf & 0x7FFFu);
     }
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
@@ -694,31 +714,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
         if (lane == 0) s_red[warp][gq] = v;
     }
-    for (int m = 16; m >= 1; m >>= 1) cf_max = max(cf_max, __shfl_xor_sync(0xffffffffu, cf_max, m));
-    if (lane == 0) s_red[warp][GK] = __uint_as_float(cf_max);
     consumer_sync();
     float Lsum[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) Lsum[gq] = s_red[0][gq] + s_red[1][gq] + s_red[2][gq] + s_red[3][gq];
-    // weights w = P * sc (anchor) or p * sc (residual), |P| <= max|s_hat|, p <= 1, sc <= 448
-    float cA, cR;
-    {
-        uint32_t cfm = 0;
-#pragma unroll
-        for (int w = 0; w < 4; w++) cfm = max(cfm, __float_as_uint(s_red[w][GK]));
-        cA = fixed_scale(bf16_to_f32((uint16_t)cfm) * 448.f, kWeightTop);
-        cR = fixed_scale(448.f, kWeightTop);
-    }
-
-    // weights pre-multiplied by their fixed-point scale (powers of two: exact)
-    for (int t = tid; t < ntiles * kTile; t += kConsumers) {
-#pragma unroll
-        for (int gq = 0; gq < GK; gq++) {
-            s_P[gq * a.chunk + t] *= cA;
-            s_sc[gq * a.chunk + t] *= cR;
-        }
-    }
-    consumer_sync();
 
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
     const int npass = RESID ? 2 : 1;
