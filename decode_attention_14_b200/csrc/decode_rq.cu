@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
     __shared__ int s_qsum[GK][2][8];                             // sum of each segment's fixed-point q
     __shared__ float s_red[4][2 * GK + 2];
-    __shared__ float s_acc[4][GK][2][kHeadDim];
+    __shared__ __align__(16) float s_acc[4][GK][2][kHeadDim];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, h = blockIdx.y;
@@ -683,7 +683,6 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
     for (int gq = 0; gq < GK; gq++)
         M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
-    consumer_sync();   // everyone has read s_red
     // the weights' fixed-point scales: w = P * sc (anchor) or p * sc
     // (residual), |P| <= max|s_hat|, p <= 1, sc <= 448 (powers of two)
     if (!mbar_wait(&bar_cfmax, 0, &s_abort)) {
@@ -712,12 +711,13 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++) {
         float v = lsum[gq];
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-        if (lane == 0) s_red[warp][gq] = v;
+        if (lane == 0) s_red[warp][GK + gq] = v;   // beside the maxima, which are read until here
     }
     consumer_sync();
     float Lsum[GK];
 #pragma unroll
-    for (int gq = 0; gq < GK; gq++) Lsum[gq] = s_red[0][gq] + s_red[1][gq] + s_red[2][gq] + s_red[3][gq];
+    for (int gq = 0; gq < GK; gq++)
+        Lsum[gq] = s_red[0][GK + gq] + s_red[1][GK + gq] + s_red[2][GK + gq] + s_red[3][GK + gq];
 
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
     const int npass = RESID ? 2 : 1;
@@ -818,19 +818,31 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 }
             }
         }
-        // fixed point -> fp32, minimum term, reduce over sub-groups (lanes xor 8, 16)
-        const float iW = 1.f / cW;
+        // fixed point -> fp32 (the 2^-acc_shift and 2^-F factors and the
+        // minimum term folded into one FMA), then a reduce-scatter over the
+        // 4 sub-groups (lanes xor 8, xor 16): each lane ends with 4 elements
+        const float iW = 1.f / cW;   // exact (power of two)
+        const bool hb8 = (sub & 1) != 0, hb16 = (sub & 2) != 0;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
+            const float mSi = mS[gq] * iW;
+            float v[16];
 #pragma unroll
             for (int e = 0; e < 16; e++) {
                 const int sh = vp == 0 ? acc_shift<BA>(e) : acc_shift<BR>(e);
-                float v = fmaf((float)accHi[gq][e], 65536.f, (float)accLo[gq][e]);
-                v = fmaf(v, __int_as_float((127 - sh) << 23), mS[gq]) * iW;   // 2^-sh; both in units of 2^-F
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                if (sub == 0) s_acc[warp][gq][vp][seg * 16 + e] = v;
+                const float f = fmaf((float)accHi[gq][e], 65536.f, (float)accLo[gq][e]);
+                v[e] = fmaf(f, __int_as_float((127 - sh) << 23) * iW, mSi);
             }
+            float r1[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                r1[i] = (hb8 ? v[8 + i] : v[i]) + __shfl_xor_sync(0xffffffffu, hb8 ? v[i] : v[8 + i], 8);
+            float4 r2;
+            r2.x = (hb16 ? r1[4] : r1[0]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[0] : r1[4], 16);
+            r2.y = (hb16 ? r1[5] : r1[1]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[1] : r1[5], 16);
+            r2.z = (hb16 ? r1[6] : r1[2]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[2] : r1[6], 16);
+            r2.w = (hb16 ? r1[7] : r1[3]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[3] : r1[7], 16);
+            *reinterpret_cast<float4 *>(&s_acc[warp][gq][vp][seg * 16 + (hb8 ? 8 : 0) + (hb16 ? 4 : 0)]) = r2;
         }
     }
 
