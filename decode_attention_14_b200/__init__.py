@@ -91,6 +91,10 @@ def _load() -> ctypes.CDLL:
     L.rq_cache_tail_length.argtypes = [vp, i32, i32, ctypes.POINTER(i32)]
     L.rq_cache_truncate.restype = i32
     L.rq_cache_truncate.argtypes = [vp, i32, i32, i32]
+    L.rq_cache_truncate_seq.restype = i32
+    L.rq_cache_truncate_seq.argtypes = [vp, i32, i32, i32, i32]
+    L.rq_cache_length_seq.restype = i32
+    L.rq_cache_length_seq.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32)]
     L.rq_cache_export.restype = i32
     L.rq_cache_export.argtypes = [vp, i32, i32, vp, vp, vp, vp]
     L.rq_decode_bytes.restype = ctypes.c_size_t
@@ -216,6 +220,16 @@ def rq_cache_truncate(h, layer: int, group: int, new_len: int) -> int:
     return lib.rq_cache_truncate(h, layer, group, new_len)
 
 
+def rq_cache_truncate_seq(h, layer: int, group: int, seq: int, new_len: int) -> int:
+    return lib.rq_cache_truncate_seq(h, layer, group, seq, new_len)
+
+
+def rq_cache_length_seq(h, layer: int, group: int, seq: int) -> int:
+    n = ctypes.c_int(0)
+    _ok(lib.rq_cache_length_seq(h, layer, group, seq, ctypes.byref(n)), "rq_cache_length_seq")
+    return n.value
+
+
 def rq_decode_bytes(h, layer: int, loop: int) -> int:
     return int(lib.rq_decode_bytes(h, layer, loop))
 
@@ -292,6 +306,12 @@ class Cache:
 
     def truncate(self, layer: int, group: int, new_len: int) -> None:
         _ok(rq_cache_truncate(self.h, layer, group, new_len), "rq_cache_truncate")
+
+    def truncate_seq(self, layer: int, group: int, seq: int, new_len: int) -> None:
+        _ok(rq_cache_truncate_seq(self.h, layer, group, seq, new_len), "rq_cache_truncate_seq")
+
+    def length_seq(self, layer: int, group: int, seq: int) -> int:
+        return rq_cache_length_seq(self.h, layer, group, seq)
 
     def decode_bytes(self, layer: int, loop: int) -> int:
         return rq_decode_bytes(self.h, layer, loop)

@@ -17,7 +17,8 @@ struct rq_cache {
     bool owned = false;
     int device = 0;
     int sms = 148;
-    std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]
+    std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]; the longest sequence
+    std::vector<int> seq;     // the same, per sequence: [layer][group or loop][batch]
     std::vector<int> ntail;   // [layer][loop]
     uint32_t sigma[4] = {0, 0, 0, 0};
     // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
@@ -72,6 +73,19 @@ uint16_t *bf16_ptr(const rq_cache *c, int layer, int loop, int kv) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+// per-sequence lengths of length slot `slot` (= layer * groups + group, or
+// layer * loops + loop for the BF16 format)
+int *seq_lens(rq_cache *c, size_t slot) { return c->seq.data() + slot * c->lay.cfg.batch; }
+const int *seq_lens(const rq_cache *c, size_t slot) { return c->seq.data() + slot * c->lay.cfg.batch; }
+void fill_lens(const int *v, int B, SeqLens *out) {
+    for (int b = 0; b < B; b++) out->v[b] = v[b];
+}
+void grow(rq_cache *c, size_t slot, int n) {
+    int *v = seq_lens(c, slot);
+    for (int b = 0; b < c->lay.cfg.batch; b++) v[b] += n;
+    c->len[slot] += n;
+}
 
 float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt((float)kHeadDim); }
 
@@ -194,6 +208,7 @@ int rq_config_check(const rq_config *c) {
     // size sanity: every per-stream offset must fit the kernels' 64-bit math
     // and the token index the kernels' 32-bit math
     if (c->max_tokens > kMaxSplits * kMaxChunk || c->max_tail_tokens > (1 << 20)) return RQ_ERR_UNSUPPORTED;
+    if (c->batch > kMaxBatch) return RQ_ERR_UNSUPPORTED;
     return RQ_OK;
 }
 
@@ -253,6 +268,7 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
     }
     const Layout &L = c->lay;
     c->len.assign((size_t)cfg->num_layers * (cfg->format == RQ_FMT_RESIDUAL ? L.groups : cfg->num_loops), 0);
+    c->seq.assign(c->len.size() * (size_t)cfg->batch, 0);
     c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
     {
         const int G = cfg->num_q_heads / cfg->num_kv_heads;
@@ -292,8 +308,8 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
     cudaStream_t st = (cudaStream_t)stream;
     if (cfg.format == RQ_FMT_BF16) {
-        int &len = c->len[(size_t)layer * cfg.num_loops + loop];
-        if (len + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
+        const size_t slot = (size_t)layer * cfg.num_loops + loop;
+        if (c->len[slot] + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
         Bf16StoreArgs a;
         a.src[0] = (const uint16_t *)k;
         a.src[1] = (const uint16_t *)v;
@@ -302,14 +318,14 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
         a.B = cfg.batch;
         a.H = cfg.num_kv_heads;
         a.n = n;
-        a.pos0 = len;
+        fill_lens(seq_lens(c, slot), cfg.batch, &a.pos0);
         a.Tp = L.Tp;
         int s = cuda_status(launch_bf16_store(a, st));
-        if (s == RQ_OK) len += n;
+        if (s == RQ_OK) grow(c, slot, n);
         return s;
     }
     const int group = loop / L.Lg, j = loop % L.Lg;
-    int &len = c->len[(size_t)layer * L.groups + group];
+    const size_t slot = (size_t)layer * L.groups + group;
     if (!is_anchor_loop(L, loop)) {
         int &nt = c->ntail[(size_t)layer * cfg.num_loops + loop];
         if (nt + n > L.tail_cap) return RQ_ERR_CAPACITY;
@@ -330,7 +346,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     // anchor loop: every other loop of the group must hold exactly these n tokens
     for (int jj = 0; jj < L.Lg - 1; jj++)
         if (c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] != n) return RQ_ERR_STATE;
-    if (len + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
+    if (c->len[slot] + n > cfg.max_tokens) return RQ_ERR_CAPACITY;
     AppendArgs a;
     std::memset(&a, 0, sizeof(a));
     a.x_anchor[0] = (const uint16_t *)k;
@@ -352,7 +368,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     a.B = cfg.batch;
     a.H = cfg.num_kv_heads;
     a.n = n;
-    a.pos0 = len;
+    fill_lens(seq_lens(c, slot), cfg.batch, &a.pos0);
     a.Tp = L.Tp;
     a.tail_cap = L.tail_cap;
     a.g = cfg.group_size;
@@ -362,7 +378,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
     int s = cuda_status(launch_append(a, st));
     if (s != RQ_OK) return s;
-    len += n;
+    grow(c, slot, n);
     for (int jj = 0; jj < L.Lg - 1; jj++) c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] = 0;
     return RQ_OK;
 }
@@ -402,11 +418,13 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     bool resid = false;
     if (bf16) {
         a.T = c->len[(size_t)layer * cfg.num_loops + loop];
+        fill_lens(seq_lens(c, (size_t)layer * cfg.num_loops + loop), cfg.batch, &a.seqT);
         a.bf[0] = bf16_ptr(c, layer, loop, 0);
         a.bf[1] = bf16_ptr(c, layer, loop, 1);
     } else {
         const int group = loop / L.Lg, j = loop % L.Lg;
         a.T = c->len[(size_t)layer * L.groups + group];
+        fill_lens(seq_lens(c, (size_t)layer * L.groups + group), cfg.batch, &a.seqT);
         for (int kv = 0; kv < 2; kv++) {
             a.a_codes[kv] = anchor_codes(c, layer, group, kv);
             a.a_meta[kv] = anchor_meta(c, layer, group, kv);
@@ -530,12 +548,43 @@ int rq_cache_truncate(rq_cache *c, int layer, int group, int new_len) {
     const Layout &L = c->lay;
     int ngroups = L.cfg.format == RQ_FMT_RESIDUAL ? L.groups : L.cfg.num_loops;
     if (layer < 0 || layer >= L.cfg.num_layers || group < 0 || group >= ngroups) return RQ_ERR_INVALID;
-    int &len = c->len[(size_t)layer * ngroups + group];
-    if (new_len < 0 || new_len > len) return RQ_ERR_INVALID;
+    const size_t slot = (size_t)layer * ngroups + group;
+    if (new_len < 0 || new_len > c->len[slot]) return RQ_ERR_INVALID;
     if (L.cfg.format == RQ_FMT_RESIDUAL)
         for (int jj = 0; jj < L.Lg - 1; jj++)
             if (c->ntail[(size_t)layer * L.cfg.num_loops + group * L.Lg + jj] != 0) return RQ_ERR_STATE;
-    len = new_len;
+    int *v = seq_lens(c, slot), mx = 0;
+    for (int b = 0; b < L.cfg.batch; b++) mx = std::max(mx, v[b] = std::min(v[b], new_len));
+    c->len[slot] = mx;
+    return RQ_OK;
+}
+
+int rq_cache_truncate_seq(rq_cache *c, int layer, int group, int seq, int new_len) {
+    if (!c) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    int ngroups = L.cfg.format == RQ_FMT_RESIDUAL ? L.groups : L.cfg.num_loops;
+    if (layer < 0 || layer >= L.cfg.num_layers || group < 0 || group >= ngroups || seq < 0 || seq >= L.cfg.batch)
+        return RQ_ERR_INVALID;
+    const size_t slot = (size_t)layer * ngroups + group;
+    int *v = seq_lens(c, slot);
+    if (new_len < 0 || new_len > v[seq]) return RQ_ERR_INVALID;
+    if (L.cfg.format == RQ_FMT_RESIDUAL)
+        for (int jj = 0; jj < L.Lg - 1; jj++)
+            if (c->ntail[(size_t)layer * L.cfg.num_loops + group * L.Lg + jj] != 0) return RQ_ERR_STATE;
+    v[seq] = new_len;
+    int mx = 0;
+    for (int b = 0; b < L.cfg.batch; b++) mx = std::max(mx, v[b]);
+    c->len[slot] = mx;
+    return RQ_OK;
+}
+
+int rq_cache_length_seq(const rq_cache *c, int layer, int group, int seq, int *len) {
+    if (!c || !len) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    int ngroups = L.cfg.format == RQ_FMT_RESIDUAL ? L.groups : L.cfg.num_loops;
+    if (layer < 0 || layer >= L.cfg.num_layers || group < 0 || group >= ngroups || seq < 0 || seq >= L.cfg.batch)
+        return RQ_ERR_INVALID;
+    *len = seq_lens(c, (size_t)layer * ngroups + group)[seq];
     return RQ_OK;
 }
 
@@ -581,19 +630,22 @@ size_t rq_decode_bytes(const rq_cache *c, int layer, int loop) {
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return 0;
     const size_t bh = (size_t)cfg.batch * cfg.num_kv_heads;
     const size_t qo = (size_t)cfg.batch * cfg.num_q_heads * kHeadDim * (2 + 4);
-    if (cfg.format == RQ_FMT_BF16) {
-        const size_t T = c->len[(size_t)layer * cfg.num_loops + loop];
-        return T * bh * 2 * kHeadDim * 2 + qo;
-    }
+    auto tokens = [&](size_t slot) {   // committed tokens summed over the sequences
+        size_t t = 0;
+        for (int b = 0; b < cfg.batch; b++) t += (size_t)seq_lens(c, slot)[b];
+        return t;
+    };
+    if (cfg.format == RQ_FMT_BF16)
+        return tokens((size_t)layer * cfg.num_loops + loop) * cfg.num_kv_heads * 2 * kHeadDim * 2 + qo;
     const int group = loop / L.Lg;
-    const size_t T = c->len[(size_t)layer * L.groups + group];
+    const size_t T = tokens((size_t)layer * L.groups + group);
     size_t per = 2 * (size_t)(L.rec.a_codes + L.rec.meta);
     size_t tail = 0;
     if (!is_anchor_loop(L, loop)) {
         per += 2 * (size_t)(L.rec.r_codes + L.rec.meta + 2);
         tail = (size_t)c->ntail[(size_t)layer * cfg.num_loops + loop] * bh * 2 * kHeadDim * 2;
     }
-    return T * bh * per + tail + qo;
+    return T * cfg.num_kv_heads * per + tail + qo;
 }
 
 int rq_check(rq_cache *c) {

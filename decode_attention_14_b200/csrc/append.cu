@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     load4_bf16(a.x_anchor[kv] + (((size_t)b * a.n + t) * a.H + h) * kHeadDim + lane * 4, x);
     uint32_t s8, m8;
     const uint32_t apack = quantize4(x, a.ba, a.g, lane, ahat, &s8, &m8);
-    const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0 + t);
+    const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0.v[b] + t);
     const int meta_rec = 2 * (kHeadDim / a.g);
     if (j == a.nres) {
         uint8_t *ac = a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8);
@@ -186,7 +186,7 @@ __global__ void bf16_store_kernel(const Bf16StoreArgs a) {
     const int t = (int)(r % a.n);
     const int b = (int)(r / a.n);
     const uint4 *src = reinterpret_cast<const uint4 *>(a.src[kv] + (((size_t)b * a.n + t) * a.H + h) * kHeadDim);
-    uint4 *dst = reinterpret_cast<uint4 *>(a.dst[kv] + (((size_t)b * a.H + h) * a.Tp + a.pos0 + t) * kHeadDim);
+    uint4 *dst = reinterpret_cast<uint4 *>(a.dst[kv] + (((size_t)b * a.H + h) * a.Tp + a.pos0.v[b] + t) * kHeadDim);
     dst[vec] = src[vec];
 }
 

@@ -55,7 +55,8 @@ __device__ __forceinline__ void combine_row(const float *part, int S, const uint
         }
 #pragma unroll
         for (int u = 0; u < kBatch; u++) {
-            const float c = exp2f(m[u] - M);
+            // a split with no key (a short sequence) has m = -inf: weight 0
+            const float c = m[u] == -CUDART_INF_F ? 0.f : exp2f(m[u] - M);
             l = fmaf(ls[u], c, l);
             o = fmaf(os[u], c, o);
         }

@@ -31,7 +31,7 @@ template <int GK>
 __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     extern __shared__ float s_scores[];   // [GK][chunk]
     __shared__ float s_q[GK][kHeadDim];
-    __shared__ float s_red[4][GK];
+    __shared__ float s_red[4][GK], s_lsum[4][GK];
     __shared__ float s_acc[4][GK][kHeadDim];
 
     const int split = blockIdx.x, h = blockIdx.y;
@@ -39,8 +39,9 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, sub = lane >> 3, seg = lane & 7;
     const int hq0 = h * a.G + pair * GK;
+    const int Tb = a.seqT.v[b];   // this sequence's committed tokens
     int t0, n;
-    split_range(split, a.S, a.T, &t0, &n);
+    split_range(split, a.S, Tb, &t0, &n);
     const size_t bh = (size_t)b * a.H + h;
 
 #pragma unroll
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     for (int it = warp * 4; it < n; it += 16) {
         const int tl = it + sub;
         const bool valid = tl < n;
-        const size_t rec = bh * a.Tp + (size_t)min(t0 + tl, a.T - 1);
+        const size_t rec = bh * a.Tp + (size_t)min(t0 + tl, Tb - 1);
         float k[16];
         load16_bf16(a.bf[0] + rec * kHeadDim + seg * 16, k);
 #pragma unroll
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
     for (int it = warp * 4; it < n; it += 16) {
         const int tl = it + sub;
         const bool valid = tl < n;
-        const size_t rec = bh * a.Tp + (size_t)min(t0 + tl, a.T - 1);
+        const size_t rec = bh * a.Tp + (size_t)min(t0 + tl, Tb - 1);
         float v[16];
         load16_bf16(a.bf[1] + rec * kHeadDim + seg * 16, v);
 #pragma unroll
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
         float l = lsum[gq];
         l += __shfl_xor_sync(0xffffffffu, l, 8);
         l += __shfl_xor_sync(0xffffffffu, l, 16);
-        if (lane == 0) s_red[warp][gq] = l;
+        if (lane == 0) s_lsum[warp][gq] = l;
     }
     __syncthreads();
 #pragma unroll
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(128) decode_bf16_kernel(const DecodeArgs a) {
         part[tid] = s_acc[0][gq][tid] + s_acc[1][gq][tid] + s_acc[2][gq][tid] + s_acc[3][gq][tid];
         if (tid == 0) {
             part[kHeadDim] = M[gq];
-            part[kHeadDim + 1] = s_red[0][gq] + s_red[1][gq] + s_red[2][gq] + s_red[3][gq];
+            part[kHeadDim + 1] = s_lsum[0][gq] + s_lsum[1][gq] + s_lsum[2][gq] + s_lsum[3][gq];
         }
     }
 }

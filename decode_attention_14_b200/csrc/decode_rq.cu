@@ -361,8 +361,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int npairs = a.G / GK;
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int hq0 = h * a.G + pair * GK;
-    int t0, n;
-    split_range(split, a.S, a.T, &t0, &n);
+    int t0, n;   // this split's tokens of its sequence (none when the sequence is short)
+    split_range(split, a.S, a.seqT.v[b], &t0, &n);
     const int ntiles = (n + kTile - 1) / kTile;
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
@@ -387,9 +387,11 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     if (warp == 4) {
         if (lane == 0) {
             const size_t tok0 = bh * a.Tp + (size_t)t0;
-            if (RESID) {
+            if (RESID && ntiles > 0) {
                 mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
                 bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
+            } else if (RESID) {
+                mbar_arrive(&bar_cf);   // nothing to fetch
             }
             // Items in order: K items, anchor V items, residual V items.  Item it
             // occupies [virt, virt + bytes) of an unbounded virtual byte

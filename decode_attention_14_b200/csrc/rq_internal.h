@@ -16,6 +16,7 @@ constexpr int kHeadDim = 128;
 constexpr int kTokTile = 64;        // padding granule of every token stream
 constexpr int kMaxSplits = 256;     // split-KV partitions per (b, kv head)
 constexpr int kMaxChunk = 1024;     // tokens per CTA (bounds the per-CTA shared-memory buffers)
+constexpr int kMaxBatch = 256;      // sequences per cache (their lengths travel in the launch arguments)
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -65,6 +66,11 @@ constexpr int kPartialStride = kHeadDim + 4;   // o[128], m, l, pad, pad
 bool make_layout(const rq_config &cfg, Layout *out);
 
 // --------------------------------------------------------------- kernels
+// Per-sequence token counts (committed length, or the position a write starts at).
+struct SeqLens {
+    int v[kMaxBatch];
+};
+
 struct AppendArgs {
     // inputs: anchor-loop K/V (kv = 0 K, 1 V), [B][n][H][d] bf16
     const uint16_t *x_anchor[2];
@@ -78,7 +84,8 @@ struct AppendArgs {
     // residual records of loop j: r_*0 + j*resid_loop_stride + kv*resid_kv_stride
     uint8_t *r_codes0, *r_meta0, *r_coef0;
     size_t resid_loop_stride, resid_kv_stride;
-    int B, H, n, pos0, Tp, tail_cap, nres;   // nres = Lg - 1
+    SeqLens pos0;                              // first token position written, per sequence
+    int B, H, n, Tp, tail_cap, nres;           // nres = Lg - 1
     int g, ba, br, rotate;
     uint32_t sigma[4];
 };
@@ -92,7 +99,8 @@ struct TailArgs {
 struct Bf16StoreArgs {
     const uint16_t *src[2];   // [B][n][H][d]
     uint16_t *dst[2];         // [B][H][Tp][d]
-    int B, H, n, pos0, Tp;
+    SeqLens pos0;             // first token position written, per sequence
+    int B, H, n, Tp;
 };
 
 struct DecodeArgs {
@@ -115,6 +123,7 @@ struct DecodeArgs {
     const uint16_t *new_k, *new_v;
     uint16_t *tail_k_w, *tail_v_w;
     int n_new, tail_pos;
+    SeqLens seqT;             // committed tokens of each sequence (T = their maximum)
     int B, H, Hq, G, T, Tp, S, chunk, splits_max;
     int g;
     float scale_log2;         // softmax_scale * log2(e)

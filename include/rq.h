@@ -60,7 +60,9 @@ typedef enum {
  *                    each group (Ouro 4/4; Huginn-style 32 loops in 8 groups
  *                    of 4, per the ai4snews summary, paragraph 1).
  *                    num_loops % loops_per_group == 0.
- *   batch            sequences B; every sequence has the same length
+ *   batch            sequences B (at most 256); appends add the same number
+ *                    of tokens to every sequence, while committed lengths may
+ *                    differ per sequence (rq_cache_truncate_seq)
  *   max_tokens       committed-token capacity per (layer, group), at most
  *                    262144 (256 split partials of up to 1024 tokens)
  *   max_tail_tokens  in-flight tokens a non-anchor loop may hold before the
@@ -206,22 +208,36 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
 int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
                            float softmax_scale, void *stream);
 
-/* Committed length of (layer, group).  group = loop / loops_per_group for
- * the residual format; for the BF16 format pass the loop index. */
+/* Committed length of (layer, group): the longest sequence's.  group =
+ * loop / loops_per_group for the residual format; for the BF16 format pass
+ * the loop index. */
 int rq_cache_length(const rq_cache *cache, int layer, int group, int *len);
+
+/* Committed length of sequence `seq` of (layer, group). */
+int rq_cache_length_seq(const rq_cache *cache, int layer, int group, int seq, int *len);
 
 /* In-flight (tail) tokens of (layer, loop); 0 for anchor loops and for the
  * BF16 format. */
 int rq_cache_tail_length(const rq_cache *cache, int layer, int loop, int *n);
 
 /* Roll the committed length of (layer, group) back to new_len (<= current),
- * e.g. to discard rejected tokens.  The group's tails must be empty (else
- * RQ_ERR_STATE).  Host-side only: no device work. */
+ * e.g. to discard rejected tokens: every sequence keeps min(its length,
+ * new_len).  The group's tails must be empty (else RQ_ERR_STATE).
+ * Host-side only: no device work. */
 int rq_cache_truncate(rq_cache *cache, int layer, int group, int new_len);
+
+/* The same for one sequence: its committed length becomes new_len (<= its
+ * current length).  Sequences of one cache may so hold different numbers of
+ * committed tokens (a ragged batch); decode attends, for each sequence, to
+ * its own committed tokens (plus the loop's tail tokens), and later appends
+ * write each sequence's tokens after its own last one.  Errors: INVALID,
+ * STATE (non-empty tails).  Host-side only. */
+int rq_cache_truncate_seq(rq_cache *cache, int layer, int group, int seq, int new_len);
 
 /*
  * Copy the committed records of (layer, loop) to host memory in the logical
  * record format (for tests and inspection; synchronises `stream`):
+ * (len = rq_cache_length; rows past a shorter sequence's length hold no token of it)
  *   anchor loop:   host_codes [2][B][H_kv][len][d*anchor_bits/8]  (K then V)
  *                  host_meta  [2][B][H_kv][len][2*d/g]  ([scale, min] per group)
  *                  host_coef  unused (may be NULL)

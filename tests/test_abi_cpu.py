@@ -50,6 +50,9 @@ def test_config_validation():
     # at most 256 split partials of at most 1024 tokens per (sequence, head)
     assert rq.rq_config_check(_cfg(batch=1, max_tokens=262144)) == rq.RQ_OK
     assert rq.rq_config_check(_cfg(batch=1, max_tokens=262145)) == rq.RQ_ERR_UNSUPPORTED
+    # sequences' lengths travel in the launch arguments: at most 256 per cache
+    assert rq.rq_config_check(_cfg(batch=256, max_tokens=64)) == rq.RQ_OK
+    assert rq.rq_config_check(_cfg(batch=257, max_tokens=64)) == rq.RQ_ERR_UNSUPPORTED
 
 
 def test_token_bytes_reproduce_storage_reduction():
