@@ -392,13 +392,11 @@ def run_ours(args, cfgd, rank, world, local_rank):
         "dtype": ("u4/u2 codes, int32 dp4a/dp2a dot products, fp32 softmax" if not args.bf16
                   else "bf16 in, fp32 math"),
         "data": "synthetic (seeded; anchor N(0,1) with 4 outlier channels x10, loops c*anchor+sigma*N(0,1))",
-        "config": {"workload": name, "layers": layers, "loops": loops, "loops_per_group": Lg, "batch": B,
-                   "seq_len": T, "kv_heads": H, "q_heads": Hq, "head_dim": 128, "group": cfgd["g"],
-                   "anchor_bits": cfgd["ba"], "resid_bits": cfgd["br"], "parallelism": f"replicas x{world}",
+        "config": dict(workload_config(name, cfgd, layers, world), **{
                    "step_calls": ("rq_append + rq_decode_attn_bf16" if args.bf16 else
                                   "rq_append + rq_decode_attn" if args.separate_append else "rq_append_decode_attn"),
                    "l2": "inputs larger than L2: %.1f GB of records read per step, loop-major over %d layers"
-                         % (step_decode_bytes / 1e9, layers)},
+                         % (step_decode_bytes / 1e9, layers)}),
         "decode_attn": {"ms_per_step": round(dec_ms / args.steps, 4), "us_per_call": round(dec_ms_call * 1e3, 3),
                         "timing": "CUDA events around a graph of the timed steps' decode calls only",
                         "bytes_per_step": int(step_decode_bytes), "gbs": round(achieved, 1),
@@ -488,6 +486,14 @@ def cpu_baseline(cfgd, seed, budget_s: float = 15.0):
                       f"{calls_per_step(cfgd)} unit-loops per decode step (extrapolated)"}
 
 
+def workload_config(name: str, cfgd, layers: int, world: int) -> dict:
+    """The `config` keys both arms report for a workload."""
+    return {"workload": name, "layers": layers, "loops": cfgd["loops"], "loops_per_group": cfgd["Lg"],
+            "batch": cfgd["B"], "seq_len": cfgd["T"], "kv_heads": cfgd["H"], "q_heads": cfgd["Hq"], "head_dim": 128,
+            "group": cfgd["g"], "anchor_bits": cfgd["ba"], "resid_bits": cfgd["br"],
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, cfgd):
     """The oracle, timed as it stands on one host core: each step is a
     bounded sample -- one (sequence, kv head) unit of one loop at full T
@@ -506,11 +512,12 @@ def run_reference(args, cfgd):
     return {
         "impl": "reference",
         "metric": "decode-attention tokens/s (INT4 anchor/INT2 resid)",
-        "value": round(value, 6), "unit": "tokens/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "value": round(value, 6), "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
-        "config": {"workload": args.config, "layers": cfgd["layers"], "loops": cfgd["loops"], "batch": cfgd["B"],
-                   "seq_len": cfgd["T"], "kv_heads": cfgd["H"], "q_heads": cfgd["Hq"], "parallelism": "cpu"},
+        "config": dict(workload_config(args.config, cfgd, cfgd["layers"], int(os.environ.get("WORLD_SIZE", "1"))),
+                       host="the oracle on one host core (rank 0)"),
         "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
