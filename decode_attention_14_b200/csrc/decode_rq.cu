@@ -30,23 +30,25 @@
 // dominant key, against the 2e-3 parity bound).
 // Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
-// Data movement.  Each CTA owns a chunk of one (sequence, kv head) and
-// streams it in 64-token items through a 4-stage shared-memory ring filled
-// by one producer warp with 1-D bulk asynchronous copies (cp.async.bulk,
-// completion counted on mbarriers; no multicast): first the K records of
-// every tile (pass 1: logits), then the anchor V codes + meta of every tile,
-// then the residual V codes + meta (pass 2: values).  Only the V coefficients
-// of the chunk (2 bytes per token) are fetched once up front.  Every mbarrier
-// wait is bounded: on timeout the kernel records an error word, stops issuing
-// copies, drains what it issued and finishes without touching further data.
+// Data movement.  Each CTA owns a chunk of one (sequence, kv head) (the
+// sequence's 64-token tiles dealt evenly over the splits) and streams it in
+// 128-token items through a byte-addressed shared-memory ring filled by one
+// producer warp with 1-D bulk asynchronous copies (cp.async.bulk, completion
+// counted on mbarriers; no multicast): first the K records of every item
+// (pass 1: logits), then the anchor V codes + meta, then the residual V codes
+// + meta (pass 2: values).  Only the V coefficients of the chunk (2 bytes per
+// token) are fetched once up front; the producer warp's other lanes take
+// their maximum for the weights' fixed point.  Every mbarrier wait is
+// bounded: on timeout the kernel records an error word, stops issuing copies,
+// drains what it issued and finishes without touching further data.
 //
 // Split combine.  Each CTA writes its partial (max, sum, o); the last CTA of
 // a (sequence, kv head) -- found with a device-wide counter, no waiting --
 // merges all partials plus the loop's BF16 tail tokens and writes the output.
 //
-// Thread map (both passes): 4 consumer warps x 16 tokens of each item;
-// lane 8s+j takes head_dim segment j (elements 16j..16j+15) of tokens
-// s, s+4, s+8, s+12 of its warp's 16.
+// Thread map (both passes): 4 consumer warps x 16 tokens of each 64-token
+// tile of an item; lane 8s+j takes head_dim segment j (elements 16j..16j+15)
+// of tokens s, s+4, s+8, s+12 of its warp's 16.
 #include <math_constants.h>
 
 #include "combine.cuh"
