@@ -1,8 +1,8 @@
 // combine.cuh -- merging split-KV partials (max m_s, sum l_s, unnormalised
 // o_s, log2 domain) and BF16 tail tokens into one attention output row:
 //   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
-// with M = max_s m_s, then the tail tokens folded in one by one with a
-// running maximum.
+// with M = max_s m_s (kept as a running maximum over batches of splits),
+// then the tail tokens folded in one by one by the same rule.
 #pragma once
 
 #include <math_constants.h>
@@ -30,19 +30,11 @@ __device__ __forceinline__ void combine_row(const float *part, int S, const uint
         k0 = bf16_to_f32(__ldcg(tail_k + tid));
         v0 = bf16_to_f32(__ldcg(tail_v + tid));
     }
-    // partials, kBatch splits per round of loads: first M = max_s m_s, then
-    // the sums rescaled to it (padding slots carry m = -inf, weight 0)
-    constexpr int kBatch = 8;
-    float M = -CUDART_INF_F;
-    for (int s0 = 0; s0 < S; s0 += kBatch) {
-        float m[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; u++)
-            m[u] = (s0 + u < S) ? __ldcg(part + (size_t)(s0 + u) * kPartialStride + kHeadDim) : -CUDART_INF_F;
-#pragma unroll
-        for (int u = 0; u < kBatch; u++) M = fmaxf(M, m[u]);
-    }
-    float l = 0.f, o = 0.f;
+    // partials, kBatch splits per round of loads (one round for up to kBatch
+    // splits): the batch's maximum, the running sums rescaled to it, then the
+    // batch folded in (a split with no key has m = -inf: weight 0)
+    constexpr int kBatch = 16;
+    float M = -CUDART_INF_F, l = 0.f, o = 0.f;
     for (int s0 = 0; s0 < S; s0 += kBatch) {
         float m[kBatch], ls[kBatch], os[kBatch];
 #pragma unroll
@@ -53,13 +45,20 @@ __device__ __forceinline__ void combine_row(const float *part, int S, const uint
             ls[u] = in ? __ldcg(p + kHeadDim + 1) : 0.f;
             os[u] = in ? __ldcg(p + tid) : 0.f;
         }
+        float Mn = M;
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) Mn = fmaxf(Mn, m[u]);
+        if (Mn == -CUDART_INF_F) continue;   // nothing attended yet
+        const float c0 = exp2f(M - Mn);      // 0 while M = -inf
+        l *= c0;
+        o *= c0;
 #pragma unroll
         for (int u = 0; u < kBatch; u++) {
-            // a split with no key (a short sequence) has m = -inf: weight 0
-            const float c = m[u] == -CUDART_INF_F ? 0.f : exp2f(m[u] - M);
+            const float c = m[u] == -CUDART_INF_F ? 0.f : exp2f(m[u] - Mn);
             l = fmaf(ls[u], c, l);
             o = fmaf(os[u], c, o);
         }
+        M = Mn;
     }
     // tail tokens, folded in one by one with the running-max rule
     for (int j = 0; j < n_tail; j++) {
