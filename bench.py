@@ -86,13 +86,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, path: str = ""):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(), f"rq_clocks_rank{index}.csv")
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        if os.path.dirname(self.path):
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -289,7 +291,7 @@ def run_ours(args, cfgd, rank, world, local_rank):
     if dist:
         import torch.distributed as tdist
         tdist.barrier()
-    sampler = ClockSampler(local_rank) if rank == 0 and not args.no_clocks else None
+    sampler = ClockSampler(local_rank, args.clocks_csv) if rank == 0 and not args.no_clocks else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
@@ -634,6 +636,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--clocks-csv", default="", help="where the raw nvidia-smi samples go (default: a temp file)")
     ap.add_argument("--json-out", default="")
     ap.add_argument("--sweep", action="store_true",
                     help="batch x format sweep of the Ouro shape at T=8192 (one JSON line per row)")

@@ -14,15 +14,15 @@
  *   - the final loop of a loop group is the shared anchor, stored at INT4;
  *   - every other loop is stored as a low-bit (INT2) residual against it;
  *   - least-squares scaling of the anchor before subtraction, with the
- *     coefficient stored in BF16 (ai4snews para. 2: "extra BF16
- *     least-squares coefficients");
+ *     coefficient stored in BF16 (ai4snews para. 2 counts these BF16
+ *     coefficients in the storage budget);
  *   - an orthogonal rotation applied to the residuals only, never to the
  *     KV states (ai4snews para. 1);
  *   - grouped quantization, group size 16, with an FP8 scale and an FP8
  *     offset per group (ai4snews para. 2);
  *   - reconstruction from two reads: anchor + one residual (ai4snews
  *     para. 3).
- * Readings where the pages are silent (all stated in the design notes):
+ * Readings where the pages are silent:
  *   FP8 = OCP E4M3 (bias 7, max 448, no inf), round-to-nearest-even with
  *   saturation to +-448; "offset" = the group minimum; scale =
  *   (max-min)/(2^b-1) taken from the unrounded min/max; codes are computed
@@ -58,9 +58,9 @@
 
 #define ORC_EXPORT __attribute__((visibility("default")))
 
-/* Relative width of the "near a rounding boundary" window (stated in the
- * parity contract: elements whose pre-rounding value lies within 1e-6
- * relative of a boundary are excluded from bit-exact comparison). */
+/* Relative width of the window around a rounding boundary: elements whose
+ * pre-rounding value lies within 1e-6 relative of a boundary are flagged and
+ * left out of the bit-exact comparison of codes. */
 static const double ORC_NEAR_REL = 1e-6;
 
 /* ------------------------------------------------------------------ */
