@@ -83,6 +83,8 @@ def _load() -> ctypes.CDLL:
     L.rq_append_decode_attn.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, ctypes.c_float, vp]
     L.rq_decode_attn_bf16.restype = i32
     L.rq_decode_attn_bf16.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
+    L.rq_prefill_attn.restype = i32
+    L.rq_prefill_attn.argtypes = [vp, i32, i32, vp, i32, vp, ctypes.c_float, vp]
     L.rq_decode_attn_noalloc.restype = i32
     L.rq_decode_attn_noalloc.argtypes = [vp, i32, i32, vp, vp, ctypes.c_float, vp]
     L.rq_cache_length.restype = i32
@@ -199,6 +201,12 @@ def rq_decode_attn_bf16(h, layer: int, loop: int, q, out, softmax_scale: float =
                                    softmax_scale, ctypes.c_void_p(_stream(stream)))
 
 
+def rq_prefill_attn(h, layer: int, loop: int, q, n_tokens: int, out, softmax_scale: float = 0.0,
+                    stream=None) -> int:
+    return lib.rq_prefill_attn(h, layer, loop, ctypes.c_void_p(_ptr(q)), n_tokens, ctypes.c_void_p(_ptr(out)),
+                               softmax_scale, ctypes.c_void_p(_stream(stream)))
+
+
 def rq_decode_attn_noalloc(h, layer: int, loop: int, q, out, softmax_scale: float = 0.0, stream=None) -> int:
     return lib.rq_decode_attn_noalloc(h, layer, loop, ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(out)),
                                       softmax_scale, ctypes.c_void_p(_stream(stream)))
@@ -282,6 +290,18 @@ class Cache:
         _check_dev(out, "float32", (self.B, self.Hq, HEAD_DIM), "out")
         fn = rq_decode_attn_bf16 if bf16 else rq_decode_attn
         _ok(fn(self.h, layer, loop, q, out, scale, stream), fn.__name__)
+        return out
+
+    def prefill(self, layer: int, loop: int, q, out=None, scale: float = 0.0, stream=None):
+        """rq_prefill_attn: causal attention of the n most recent tokens,
+        q [batch][n][num_q_heads][128] bf16 -> fp32 of the same shape."""
+        import torch
+        n = q.shape[1]
+        _check_dev(q, "bfloat16", (self.B, n, self.Hq, HEAD_DIM), "q")
+        if out is None:
+            out = torch.empty((self.B, n, self.Hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+        _check_dev(out, "float32", (self.B, n, self.Hq, HEAD_DIM), "out")
+        _ok(rq_prefill_attn(self.h, layer, loop, q, n, out, scale, stream), "rq_prefill_attn")
         return out
 
     def append_decode(self, layer: int, loop: int, k, v, q, out=None, scale: float = 0.0, stream=None):

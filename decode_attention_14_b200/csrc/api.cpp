@@ -7,6 +7,7 @@
 #include <cstring>
 #include <new>
 
+#include "prefill.h"
 #include "rq_internal.h"
 
 using namespace rq;
@@ -23,6 +24,9 @@ struct rq_cache {
     uint32_t sigma[4] = {0, 0, 0, 0};
     // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
     int occ[2][kMaxChunk / kTokTile];
+    // split partials of rq_prefill_attn, allocated on first use and grown on demand
+    float *prefill_ws = nullptr;
+    size_t prefill_ws_floats = 0;
 };
 
 namespace {
@@ -293,10 +297,11 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
 int rq_cache_destroy(rq_cache *c) {
     if (!c) return RQ_OK;
     int st = RQ_OK;
-    if (c->owned) {
+    if (c->owned || c->prefill_ws) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = RQ_ERR_CUDA;
-        cudaFree(c->base);
     }
+    if (c->owned) cudaFree(c->base);
+    if (c->prefill_ws) cudaFree(c->prefill_ws);
     delete c;
     return st;
 }
@@ -524,6 +529,72 @@ int rq_append_decode_attn(rq_cache *c, int layer, int loop, const void *k, const
 int rq_decode_attn_bf16(rq_cache *c, int layer, int loop, const void *q, float *out, float scale,
                         void *stream) {
     return decode_common(c, layer, loop, q, out, scale, stream, true);
+}
+
+int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, float *out, float scale,
+                    void *stream) {
+    if (!c || !q || !out || n <= 0) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
+    if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
+    PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int group = loop / L.Lg, j = loop % L.Lg;
+    const size_t slot = (size_t)layer * L.groups + group;
+    const int T = c->len[slot];
+    fill_lens(seq_lens(c, slot), cfg.batch, &a.seqT);
+    for (int kv = 0; kv < 2; kv++) {
+        a.a_codes[kv] = anchor_codes(c, layer, group, kv);
+        a.a_meta[kv] = anchor_meta(c, layer, group, kv);
+    }
+    if (!is_anchor_loop(L, loop)) {
+        for (int kv = 0; kv < 2; kv++) {
+            a.r_codes[kv] = resid_codes(c, layer, group, j, kv);
+            a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
+            a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, j, kv);
+        }
+        a.n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
+        a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
+        a.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
+    }
+    // the n new tokens must be the most recent of every sequence
+    for (int b = 0; b < cfg.batch; b++)
+        if (a.seqT.v[b] + a.n_tail < n) return RQ_ERR_STATE;
+    a.q = (const uint16_t *)q;
+    a.out = out;
+    a.B = cfg.batch;
+    a.H = cfg.num_kv_heads;
+    a.Hq = cfg.num_q_heads;
+    a.G = cfg.num_q_heads / cfg.num_kv_heads;
+    a.n = n;
+    a.tail_cap = L.tail_cap;
+    a.Tp = L.Tp;
+    a.g = cfg.group_size;
+    a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
+    a.rotate = cfg.rotate;
+    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    a.nqb = (n * a.G + kPrefillRows - 1) / kPrefillRows;
+    if (n > 65535 || (long)a.B * a.nqb > 65535) return RQ_ERR_UNSUPPORTED;   // grid limits
+    a.S = prefill_splits(T, a.B * a.H * a.nqb, c->sms);
+    const size_t need = (size_t)a.B * n * a.Hq * std::max(a.S, 1) * kPartialStride;
+    if (need > c->prefill_ws_floats) {
+        if (c->prefill_ws) {
+            if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
+            cudaFree(c->prefill_ws);
+            c->prefill_ws = nullptr;
+            c->prefill_ws_floats = 0;
+        }
+        void *p = nullptr;
+        if (cudaMalloc(&p, need * sizeof(float)) != cudaSuccess) {
+            cudaGetLastError();
+            return RQ_ERR_NOMEM;
+        }
+        c->prefill_ws = (float *)p;
+        c->prefill_ws_floats = need;
+    }
+    a.partials = c->prefill_ws;
+    return cuda_status(launch_prefill(a, cfg.anchor_bits, cfg.resid_bits, (cudaStream_t)stream));
 }
 
 int rq_cache_length(const rq_cache *c, int layer, int group, int *len) {

@@ -1,0 +1,269 @@
+// prefill.cu -- multi-token causal attention over the ResidualQuant cache: the
+// step before decode (chunked prefill, or verifying several drafted tokens),
+// which the ai4snews summary's throughput study (paragraph 4) leaves out of
+// its decode timing.  Query row (i, hq) of sequence b, i < n, attends to the
+// first T_b + n_tail - n + 1 + i tokens of [the group's committed tokens, the
+// loop's BF16 tail tokens]: the n new tokens are the most recent ones,
+// committed already at an anchor loop, in the tail at the other loops.
+//
+// Design.  With n query tokens per sequence the keys are shared by n * G
+// query rows, so a CTA dequantizes each record once into shared memory in
+// fp32 (k_hat = s_hat a_hat + R^T y_hat; the inverse rotation is one warp
+// Walsh-Hadamard transform per token, cheaper than rotating n * G queries
+// once the rows outnumber a few) and runs both products, logits and p V, on
+// the FP32 pipes from shared memory:
+//  - CTA = (split of the committed tokens, kv head, sequence x block of up to
+//    64 query rows), 8 warps; warp w owns rows w, w + 8, ..., w + 56;
+//  - per 32-token step: dequantize K (warp per token), logits (lane = token,
+//    a row's 32 logits in one warp), online softmax per row, dequantize V,
+//    o += p V (lane = 4 columns of head_dim);
+//  - each CTA writes a partial (m, l, o) per row; a second kernel merges the
+//    partials and the tail tokens of each row (combine_row) under the row's
+//    causal limit.
+// This is a CUDA-core kernel: the contraction per step is 64 x 32 x 128
+// twice, too small and too oddly shaped (fp32 reconstruction) to pay for a
+// tensor-core pipeline at these row counts.
+#include <math_constants.h>
+
+#include <algorithm>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "prefill.h"
+
+namespace rq {
+namespace {
+
+constexpr int kThreadsP = 256;
+constexpr int kQStride = kHeadDim + 4;   // float4-aligned query rows
+constexpr int kKStride = kHeadDim + 1;   // lane = token reads a column without bank conflicts
+constexpr int kPStride = kPrefillTile + 1;
+constexpr size_t kSmemBytes =
+    (size_t)(kPrefillRows * kQStride + kPrefillTile * kKStride + kPrefillRows * kPStride) * sizeof(float);
+constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
+
+// The codes of elements 4 lane .. 4 lane + 3 of a record, LSB first.
+template <int BITS>
+__device__ __forceinline__ uint32_t lane_codes(const uint8_t *rec, int lane) {
+    if (BITS == 4) return *reinterpret_cast<const uint16_t *>(rec + 2 * lane);
+    return rec[lane];
+}
+
+// Reconstruct the K (kv = 0) or V (kv = 1) rows of tokens rec0 .. rec0 + tn - 1
+// into rows 0 .. tn - 1 of sK (rows tn .. 31 zeroed); warp per token, lane
+// holds elements 4 lane .. 4 lane + 3.
+template <int BA, int BR>
+__device__ __forceinline__ void dequant_tile(const PrefillArgs &a, int kv, size_t rec0, int tn, float *sK, int warp,
+                                             int lane) {
+    const int MR = 2 * (kHeadDim / a.g);
+    const int gi = (4 * lane) / a.g;   // quantization group of this lane's elements
+    const bool resid = a.r_codes[kv] != nullptr;
+    for (int u = warp; u < kPrefillTile; u += kThreadsP / 32) {
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (u < tn) {
+            const size_t rec = rec0 + u;
+            const uint32_t w = lane_codes<BA>(a.a_codes[kv] + rec * (16 * BA), lane);
+            const uint8_t *mp = a.a_meta[kv] + rec * MR + 2 * gi;
+            const float sc = e4m3_to_f32(mp[0]), mn = e4m3_to_f32(mp[1]);
+#pragma unroll
+            for (int k = 0; k < 4; k++) x[k] = fmaf((float)((w >> (BA * k)) & ((1u << BA) - 1)), sc, mn);
+            if (resid) {
+                const float sh = bf16_to_f32(a.r_coef[kv][rec]);
+                const uint32_t wr = lane_codes<BR>(a.r_codes[kv] + rec * (16 * BR), lane);
+                const uint8_t *mr = a.r_meta[kv] + rec * MR + 2 * gi;
+                const float rs = e4m3_to_f32(mr[0]), rm = e4m3_to_f32(mr[1]);
+                float y[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) y[k] = fmaf((float)((wr >> (BR * k)) & ((1u << BR) - 1)), rs, rm);
+                if (a.rotate) {
+                    // R^T y = diag(sigma) H y / sqrt(d)
+                    wht128_warp(y, lane);
+#pragma unroll
+                    for (int k = 0; k < 4; k++) y[k] *= sigma_neg(a.sigma, 4 * lane + k) ? -kInvSqrtD : kInvSqrtD;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; k++) x[k] = fmaf(sh, x[k], y[k]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; k++) sK[u * kKStride + 4 * lane + k] = x[k];
+    }
+}
+
+template <int BA, int BR>
+__global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillArgs a) {
+    extern __shared__ __align__(16) float smem[];
+    float *sQ = smem;                                  // [64][kQStride] q * scale * log2(e)
+    float *sK = sQ + kPrefillRows * kQStride;          // [32][kKStride] reconstructed K, then V
+    float *sP = sK + kPrefillTile * kKStride;          // [64][kPStride] probabilities of the step
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, h = blockIdx.y;
+    const int b = blockIdx.z / a.nqb, qb = blockIdx.z % a.nqb;
+    const int r0 = qb * kPrefillRows;                           // first query row (i * G + gq) of the CTA
+    const int nr = min(kPrefillRows, a.n * a.G - r0);           // rows of the CTA
+    const int Tb = a.seqT.v[b];
+    int t0, cnt;
+    split_range(split, a.S, Tb, &t0, &cnt);
+    const size_t bh = (size_t)b * a.H + h;
+
+    for (int idx = tid; idx < kPrefillRows * kHeadDim; idx += kThreadsP) {
+        const int r = idx / kHeadDim, d = idx % kHeadDim;
+        float v = 0.f;
+        if (r < nr) {
+            const int rg = r0 + r, i = rg / a.G, gq = rg % a.G;
+            v = bf16_to_f32(a.q[(((size_t)b * a.n + i) * a.Hq + h * a.G + gq) * kHeadDim + d]) * a.scale_log2;
+        }
+        sQ[r * kQStride + d] = v;
+    }
+    // this warp's rows: warp + 8 j for j < jn
+    const int jn = nr > warp ? (nr - warp + 7) / 8 : 0;
+    int lim[8];   // committed tokens each row may see
+    float m[8], l[8], acc[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int i = (r0 + warp + 8 * j) / a.G;
+        lim[j] = min(Tb, Tb + a.n_tail - a.n + 1 + i);
+        m[j] = -CUDART_INF_F;
+        l[j] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; k++) acc[j][k] = 0.f;
+    }
+    __syncthreads();
+
+    for (int tt = 0; tt < cnt; tt += kPrefillTile) {
+        const int tn = min(kPrefillTile, cnt - tt);
+        const size_t rec0 = bh * a.Tp + t0 + tt;
+        dequant_tile<BA, BR>(a, 0, rec0, tn, sK, warp, lane);
+        __syncthreads();
+        // logits of token lane for the warp's rows
+        float s[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) s[j] = 0.f;
+        const float *kr = sK + lane * kKStride;
+#pragma unroll 2
+        for (int d = 0; d < kHeadDim; d += 4) {
+            const float k0 = kr[d], k1 = kr[d + 1], k2 = kr[d + 2], k3 = kr[d + 3];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j < jn) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(sQ + (warp + 8 * j) * kQStride + d);
+                    s[j] = fmaf(qv.x, k0, fmaf(qv.y, k1, fmaf(qv.z, k2, fmaf(qv.w, k3, s[j]))));
+                }
+            }
+        }
+        // online softmax per row (log2 domain); masked tokens weigh 0
+        const int tabs = t0 + tt + lane;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (j < jn) {
+                const bool valid = lane < tn && tabs < lim[j];
+                const float z = valid ? s[j] : -CUDART_INF_F;
+                float mx = z;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                const float mn = fmaxf(m[j], mx);
+                float p = 0.f, alpha = 1.f;
+                if (mn != -CUDART_INF_F) {
+                    alpha = exp2f(m[j] - mn);   // 0 while nothing was seen
+                    p = valid ? exp2f(z - mn) : 0.f;
+                }
+                float ps = p;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+                l[j] = fmaf(l[j], alpha, ps);
+                m[j] = mn;
+#pragma unroll
+                for (int k = 0; k < 4; k++) acc[j][k] *= alpha;
+                sP[(warp + 8 * j) * kPStride + lane] = p;
+            }
+        }
+        __syncthreads();   // every logit has read sK; sP is complete
+        dequant_tile<BA, BR>(a, 1, rec0, tn, sK, warp, lane);
+        __syncthreads();
+        for (int t = 0; t < tn; t++) {
+            const float *vr = sK + t * kKStride;
+            const float v0 = vr[lane], v1 = vr[lane + 32], v2 = vr[lane + 64], v3 = vr[lane + 96];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (j < jn) {
+                    const float p = sP[(warp + 8 * j) * kPStride + t];
+                    acc[j][0] = fmaf(p, v0, acc[j][0]);
+                    acc[j][1] = fmaf(p, v1, acc[j][1]);
+                    acc[j][2] = fmaf(p, v2, acc[j][2]);
+                    acc[j][3] = fmaf(p, v3, acc[j][3]);
+                }
+            }
+        }
+        __syncthreads();   // sK and sP are rewritten by the next step
+    }
+
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        if (j < jn) {
+            const int rg = r0 + warp + 8 * j, i = rg / a.G, gq = rg % a.G;
+            const size_t row = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
+            float *part = a.partials + (row * a.S + split) * kPartialStride;
+#pragma unroll
+            for (int k = 0; k < 4; k++) part[lane + 32 * k] = acc[j][k];
+            if (lane == 0) {
+                part[kHeadDim] = m[j];
+                part[kHeadDim + 1] = l[j];
+            }
+        }
+    }
+}
+
+struct Sync128 {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+
+// One CTA per (q head, query token, sequence): the row's partials, then the
+// tail tokens it may see.
+__global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs a) {
+    __shared__ float s_red[4];
+    const int hq = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
+    const int h = hq / a.G;
+    const size_t row = ((size_t)b * a.n + i) * a.Hq + hq;
+    // of [committed, tail] the row sees T_b + n_tail - n + 1 + i tokens: all
+    // committed ones when the new tokens are in the tail
+    const int nt = a.tail_k ? max(0, a.n_tail - a.n + 1 + i) : 0;
+    const size_t trow = ((size_t)b * a.tail_cap * a.H + h) * kHeadDim;
+    combine_row(a.partials + row * a.S * kPartialStride, a.S, a.q + row * kHeadDim, a.scale_log2,
+                a.tail_k ? a.tail_k + trow : nullptr, a.tail_v ? a.tail_v + trow : nullptr,
+                (size_t)a.H * kHeadDim, nt, a.out + row * kHeadDim, threadIdx.x, s_red, Sync128());
+}
+
+template <int BA, int BR>
+cudaError_t launch_t(const PrefillArgs &a, cudaStream_t st) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_rq_kernel<BA, BR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    if (a.S > 0) prefill_rq_kernel<BA, BR><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, kSmemBytes, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int prefill_splits(int T, int units, int sms) {
+    if (T <= 0 || units <= 0) return 0;
+    const int nt = (T + kTokTile - 1) / kTokTile;
+    const int want = (4 * sms + units - 1) / units;   // about two waves at two CTAs per SM
+    return std::max(1, std::min(std::min(nt, kMaxSplits), want));
+}
+
+cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st) {
+    if (ba == 4 && br == 2) return launch_t<4, 2>(a, st);
+    if (ba == 2 && br == 2) return launch_t<2, 2>(a, st);
+    if (ba == 4 && br == 4) return launch_t<4, 4>(a, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rq

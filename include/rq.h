@@ -188,6 +188,34 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
                         float softmax_scale, void *stream);
 
 /*
+ * Multi-token causal attention for one (layer, loop) over the compressed
+ * cache (format RQ_FMT_RESIDUAL): the attention of a chunked prefill, or of
+ * several drafted tokens, after their K/V were appended (rq_append with
+ * n_tokens = n on every loop so far).  The ai4snews summary's decode study
+ * (paragraph 4) times decode only; this call is the step before it, reading
+ * the same records the decode reads.
+ *   q_bf16: device, [batch][n_tokens][num_q_heads][head_dim] BF16: the n most
+ *           recent tokens of every sequence, oldest first.
+ *   out:    device, [batch][n_tokens][num_q_heads][head_dim] fp32.
+ *   softmax_scale: as for rq_decode_attn.
+ * Keys/values: the sequence of the loop's group's committed tokens (as
+ * rq_decode_attn reconstructs them) followed by the loop's BF16 tail tokens;
+ * query token i (0-based) of sequence b sees its first
+ * len_b + n_tail - n_tokens + 1 + i tokens (len_b: b's committed tokens), so
+ * the n new tokens are the last ones -- committed at an anchor loop, in the
+ * tail at the other loops -- and each sees itself and the ones before it.
+ * The split partials live in a device buffer the cache allocates on the
+ * first call (and grows when a later call needs more:
+ * batch * n_tokens * num_q_heads * splits * 132 floats), freed by
+ * rq_cache_destroy; that allocation synchronises the device.
+ * Errors: INVALID (null pointer, n_tokens < 1, index out of range), STATE
+ * (wrong format, or a sequence holds fewer than n_tokens tokens),
+ * UNSUPPORTED (n_tokens > 65535), NOMEM, CUDA.
+ */
+int rq_prefill_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, int n_tokens, float *out,
+                    float softmax_scale, void *stream);
+
+/*
  * rq_decode_attn without any allocation: identical arguments, results and
  * errors, except that the split-combine partials go to a fixed array the
  * library holds in device memory (8 MiB per GPU that loads the library, kept
