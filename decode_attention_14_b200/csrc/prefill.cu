@@ -38,9 +38,55 @@ constexpr int kThreadsP = 256;
 constexpr int kQStride = kHeadDim + 4;   // float4-aligned query rows
 constexpr int kKStride = kHeadDim + 1;   // lane = token reads a column without bank conflicts
 constexpr int kPStride = kPrefillTile + 1;
-constexpr size_t kSmemBytes =
-    (size_t)(kPrefillRows * kQStride + kPrefillTile * kKStride + kPrefillRows * kPStride) * sizeof(float);
+constexpr int kFloatSmem = kPrefillRows * kQStride + kPrefillTile * kKStride + kPrefillRows * kPStride;
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
+
+// Raw records of one 32-token tile, K then V, each side laid out
+// [anchor codes][anchor meta][residual codes][residual meta][coefficients]
+// (meta sized for the largest, group 16); two such stages are in flight.
+template <int BA, int BR>
+struct Stage {
+    static constexpr int A_C = 16 * BA, R_C = 16 * BR, MR_MAX = 16;
+    static constexpr int SIDE = kPrefillTile * (A_C + R_C + 2 * MR_MAX) + 2 * kPrefillTile;
+    static constexpr int BYTES = 2 * SIDE;
+    static constexpr size_t smem() { return (size_t)kFloatSmem * sizeof(float) + 2 * (size_t)BYTES; }
+};
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// bytes (a multiple of 16, both addresses 16-byte aligned) spread over the CTA
+__device__ __forceinline__ void copy_async(uint8_t *dst, const uint8_t *src, int bytes, int tid) {
+    for (int o = 16 * tid; o < bytes; o += 16 * kThreadsP) cp_async16(dst + o, src + o);
+}
+
+// Issue the copies of the tile whose first record is rec0 (a multiple of 32:
+// every source is 16-byte aligned, and a whole tile lies inside the stream's
+// padded capacity).
+template <int BA, int BR>
+__device__ __forceinline__ void stage_tile(const PrefillArgs &a, uint8_t *st, size_t rec0, int MR, bool resid,
+                                           int tid) {
+    using SG = Stage<BA, BR>;
+    constexpr int TT = kPrefillTile;
+#pragma unroll
+    for (int kv = 0; kv < 2; kv++) {
+        uint8_t *d = st + kv * SG::SIDE;
+        copy_async(d, a.a_codes[kv] + rec0 * SG::A_C, TT * SG::A_C, tid);
+        copy_async(d + TT * SG::A_C, a.a_meta[kv] + rec0 * MR, TT * MR, tid);
+        if (resid) {
+            copy_async(d + TT * (SG::A_C + MR), a.r_codes[kv] + rec0 * SG::R_C, TT * SG::R_C, tid);
+            copy_async(d + TT * (SG::A_C + MR + SG::R_C), a.r_meta[kv] + rec0 * MR, TT * MR, tid);
+            copy_async(d + TT * (SG::A_C + SG::R_C + 2 * MR), reinterpret_cast<const uint8_t *>(a.r_coef[kv] + rec0),
+                       2 * TT, tid);
+        }
+    }
+}
 
 // The codes of elements 4 lane .. 4 lane + 3 of a record, LSB first.
 template <int BITS>
@@ -49,28 +95,30 @@ __device__ __forceinline__ uint32_t lane_codes(const uint8_t *rec, int lane) {
     return rec[lane];
 }
 
-// Reconstruct the K (kv = 0) or V (kv = 1) rows of tokens rec0 .. rec0 + tn - 1
-// into rows 0 .. tn - 1 of sK (rows tn .. 31 zeroed); warp per token, lane
-// holds elements 4 lane .. 4 lane + 3.
+// Reconstruct side kv of the staged tile, tokens 0 .. tn - 1, into rows
+// 0 .. tn - 1 of sK (rows tn .. 31 zeroed); warp per token, lane holds
+// elements 4 lane .. 4 lane + 3.
 template <int BA, int BR>
-__device__ __forceinline__ void dequant_tile(const PrefillArgs &a, int kv, size_t rec0, int tn, float *sK, int warp,
-                                             int lane) {
-    const int MR = 2 * (kHeadDim / a.g);
+__device__ __forceinline__ void dequant_tile(const PrefillArgs &a, const uint8_t *st, int kv, int MR, bool resid,
+                                             int tn, float *sK, int warp, int lane) {
+    using SG = Stage<BA, BR>;
+    constexpr int TT = kPrefillTile;
+    const uint8_t *d = st + kv * SG::SIDE;
     const int gi = (4 * lane) / a.g;   // quantization group of this lane's elements
-    const bool resid = a.r_codes[kv] != nullptr;
-    for (int u = warp; u < kPrefillTile; u += kThreadsP / 32) {
+#pragma unroll
+    for (int u = warp; u < TT; u += kThreadsP / 32) {
         float x[4] = {0.f, 0.f, 0.f, 0.f};
         if (u < tn) {
-            const size_t rec = rec0 + u;
-            const uint32_t w = lane_codes<BA>(a.a_codes[kv] + rec * (16 * BA), lane);
-            const uint8_t *mp = a.a_meta[kv] + rec * MR + 2 * gi;
+            const uint32_t w = lane_codes<BA>(d + u * SG::A_C, lane);
+            const uint8_t *mp = d + TT * SG::A_C + u * MR + 2 * gi;
             const float sc = e4m3_to_f32(mp[0]), mn = e4m3_to_f32(mp[1]);
 #pragma unroll
             for (int k = 0; k < 4; k++) x[k] = fmaf((float)((w >> (BA * k)) & ((1u << BA) - 1)), sc, mn);
             if (resid) {
-                const float sh = bf16_to_f32(a.r_coef[kv][rec]);
-                const uint32_t wr = lane_codes<BR>(a.r_codes[kv] + rec * (16 * BR), lane);
-                const uint8_t *mr = a.r_meta[kv] + rec * MR + 2 * gi;
+                const float sh =
+                    bf16_to_f32(reinterpret_cast<const uint16_t *>(d + TT * (SG::A_C + SG::R_C + 2 * MR))[u]);
+                const uint32_t wr = lane_codes<BR>(d + TT * (SG::A_C + MR) + u * SG::R_C, lane);
+                const uint8_t *mr = d + TT * (SG::A_C + MR + SG::R_C) + u * MR + 2 * gi;
                 const float rs = e4m3_to_f32(mr[0]), rm = e4m3_to_f32(mr[1]);
                 float y[4];
 #pragma unroll
@@ -92,10 +140,12 @@ __device__ __forceinline__ void dequant_tile(const PrefillArgs &a, int kv, size_
 
 template <int BA, int BR>
 __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillArgs a) {
+    using SG = Stage<BA, BR>;
     extern __shared__ __align__(16) float smem[];
     float *sQ = smem;                                  // [64][kQStride] q * scale * log2(e)
     float *sK = sQ + kPrefillRows * kQStride;          // [32][kKStride] reconstructed K, then V
     float *sP = sK + kPrefillTile * kKStride;          // [64][kPStride] probabilities of the step
+    uint8_t *sRaw = reinterpret_cast<uint8_t *>(smem + kFloatSmem);   // 2 stages of raw records
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, h = blockIdx.y;
@@ -106,6 +156,12 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
     int t0, cnt;
     split_range(split, a.S, Tb, &t0, &cnt);
     const size_t bh = (size_t)b * a.H + h;
+    const int MR = 2 * (kHeadDim / a.g);
+    const bool resid = a.r_codes[0] != nullptr;
+    const int ntl = (cnt + kPrefillTile - 1) / kPrefillTile;
+
+    if (ntl > 0) stage_tile<BA, BR>(a, sRaw, bh * a.Tp + t0, MR, resid, tid);
+    cp_async_commit();
 
     for (int idx = tid; idx < kPrefillRows * kHeadDim; idx += kThreadsP) {
         const int r = idx / kHeadDim, d = idx % kHeadDim;
@@ -129,12 +185,20 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
 #pragma unroll
         for (int k = 0; k < 4; k++) acc[j][k] = 0.f;
     }
-    __syncthreads();
 
-    for (int tt = 0; tt < cnt; tt += kPrefillTile) {
+    for (int kt = 0; kt < ntl; kt++) {
+        const int tt = kt * kPrefillTile;
         const int tn = min(kPrefillTile, cnt - tt);
-        const size_t rec0 = bh * a.Tp + t0 + tt;
-        dequant_tile<BA, BR>(a, 0, rec0, tn, sK, warp, lane);
+        const uint8_t *st = sRaw + (kt & 1) * SG::BYTES;
+        // the next tile's copies overlap this tile's work; its stage was
+        // released by the barrier that ended the step before
+        if (kt + 1 < ntl)
+            stage_tile<BA, BR>(a, sRaw + ((kt + 1) & 1) * SG::BYTES, bh * a.Tp + t0 + tt + kPrefillTile, MR,
+                               resid, tid);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();   // this tile's records (and, first time, sQ) are visible
+        dequant_tile<BA, BR>(a, st, 0, MR, resid, tn, sK, warp, lane);
         __syncthreads();
         // logits of token lane for the warp's rows
         float s[8];
@@ -179,7 +243,7 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
             }
         }
         __syncthreads();   // every logit has read sK; sP is complete
-        dequant_tile<BA, BR>(a, 1, rec0, tn, sK, warp, lane);
+        dequant_tile<BA, BR>(a, st, 1, MR, resid, tn, sK, warp, lane);
         __syncthreads();
         for (int t = 0; t < tn; t++) {
             const float *vr = sK + t * kKStride;
@@ -195,8 +259,9 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
                 }
             }
         }
-        __syncthreads();   // sK and sP are rewritten by the next step
+        __syncthreads();   // sK, sP and this stage are rewritten by the next steps
     }
+    cp_async_wait<0>();
 
 #pragma unroll
     for (int j = 0; j < 8; j++) {
@@ -239,11 +304,12 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t st) {
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(prefill_rq_kernel<BA, BR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
+                                             (int)Stage<BA, BR>::smem());
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (a.S > 0) prefill_rq_kernel<BA, BR><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, kSmemBytes, st>>>(a);
+    if (a.S > 0)
+        prefill_rq_kernel<BA, BR><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, Stage<BA, BR>::smem(), st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
