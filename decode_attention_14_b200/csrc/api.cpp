@@ -574,9 +574,9 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
     a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
     a.rotate = cfg.rotate;
     std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
-    a.nqb = (n * a.G + kPrefillRows - 1) / kPrefillRows;
-    if (n > 65535 || (long)a.B * a.nqb > 65535) return RQ_ERR_UNSUPPORTED;   // grid limits
-    a.S = prefill_splits(T, a.B * a.H * a.nqb, c->sms);
+    if (n > 65535) return RQ_ERR_UNSUPPORTED;   // grid limit
+    prefill_plan(&a, T, cfg.anchor_bits, cfg.resid_bits, c->sms);
+    if ((long)a.B * a.nqb > 65535) return RQ_ERR_UNSUPPORTED;
     const size_t need = (size_t)a.B * n * a.Hq * std::max(a.S, 1) * kPartialStride;
     if (need > c->prefill_ws_floats) {
         if (c->prefill_ws) {

@@ -12,8 +12,9 @@
 // Walsh-Hadamard transform per token, cheaper than rotating n * G queries
 // once the rows outnumber a few) and runs both products, logits and p V, on
 // the FP32 pipes from shared memory:
-//  - CTA = (split of the committed tokens, kv head, sequence x block of up to
-//    64 query rows), 8 warps; warp w owns rows w, w + 8, ..., w + 56;
+//  - CTA = (split of the committed tokens, kv head, sequence x block of
+//    8 RPW query rows, RPW in {1, 2, 4, 8} the fewest that hold a kv head's
+//    n * G rows), 8 warps; warp w owns rows w, w + 8, ...;
 //  - per 32-token step: dequantize K (warp per token), logits (lane = token,
 //    a row's 32 logits in one warp), online softmax per row, dequantize V,
 //    o += p V (lane = 4 columns of head_dim);
@@ -38,7 +39,10 @@ constexpr int kThreadsP = 256;
 constexpr int kQStride = kHeadDim + 4;   // float4-aligned query rows
 constexpr int kKStride = kHeadDim + 1;   // lane = token reads a column without bank conflicts
 constexpr int kPStride = kPrefillTile + 1;
-constexpr int kFloatSmem = kPrefillRows * kQStride + kPrefillTile * kKStride + kPrefillRows * kPStride;
+// shared floats of a CTA of `rows` query rows: q, one reconstructed tile, probabilities
+__host__ __device__ constexpr int float_smem(int rows) {
+    return rows * kQStride + kPrefillTile * kKStride + rows * kPStride;
+}
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
 
 // Raw records of one 32-token tile, K then V, each side laid out
@@ -49,7 +53,7 @@ struct Stage {
     static constexpr int A_C = 16 * BA, R_C = 16 * BR, MR_MAX = 16;
     static constexpr int SIDE = kPrefillTile * (A_C + R_C + 2 * MR_MAX) + 2 * kPrefillTile;
     static constexpr int BYTES = 2 * SIDE;
-    static constexpr size_t smem() { return (size_t)kFloatSmem * sizeof(float) + 2 * (size_t)BYTES; }
+    static constexpr size_t smem(int rows) { return (size_t)float_smem(rows) * sizeof(float) + 2 * (size_t)BYTES; }
 };
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -138,20 +142,22 @@ __device__ __forceinline__ void dequant_tile(const PrefillArgs &a, const uint8_t
     }
 }
 
-template <int BA, int BR>
-__global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillArgs a) {
+// RPW query rows per warp (8 RPW per CTA); fewer rows leave room for more CTAs per SM
+template <int BA, int BR, int RPW>
+__global__ void __launch_bounds__(kThreadsP, RPW <= 2 ? 4 : RPW == 4 ? 3 : 2) prefill_rq_kernel(const PrefillArgs a) {
     using SG = Stage<BA, BR>;
+    constexpr int ROWS = 8 * RPW;
     extern __shared__ __align__(16) float smem[];
-    float *sQ = smem;                                  // [64][kQStride] q * scale * log2(e)
-    float *sK = sQ + kPrefillRows * kQStride;          // [32][kKStride] reconstructed K, then V
-    float *sP = sK + kPrefillTile * kKStride;          // [64][kPStride] probabilities of the step
-    uint8_t *sRaw = reinterpret_cast<uint8_t *>(smem + kFloatSmem);   // 2 stages of raw records
+    float *sQ = smem;                                  // [ROWS][kQStride] q * scale * log2(e)
+    float *sK = sQ + ROWS * kQStride;                  // [32][kKStride] reconstructed K, then V
+    float *sP = sK + kPrefillTile * kKStride;          // [ROWS][kPStride] probabilities of the step
+    uint8_t *sRaw = reinterpret_cast<uint8_t *>(smem + float_smem(ROWS));   // 2 stages of raw records
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, h = blockIdx.y;
     const int b = blockIdx.z / a.nqb, qb = blockIdx.z % a.nqb;
-    const int r0 = qb * kPrefillRows;                           // first query row (i * G + gq) of the CTA
-    const int nr = min(kPrefillRows, a.n * a.G - r0);           // rows of the CTA
+    const int r0 = qb * ROWS;                                   // first query row (i * G + gq) of the CTA
+    const int nr = min(ROWS, a.n * a.G - r0);                   // rows of the CTA
     const int Tb = a.seqT.v[b];
     int t0, cnt;
     split_range(split, a.S, Tb, &t0, &cnt);
@@ -163,7 +169,7 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
     if (ntl > 0) stage_tile<BA, BR>(a, sRaw, bh * a.Tp + t0, MR, resid, tid);
     cp_async_commit();
 
-    for (int idx = tid; idx < kPrefillRows * kHeadDim; idx += kThreadsP) {
+    for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreadsP) {
         const int r = idx / kHeadDim, d = idx % kHeadDim;
         float v = 0.f;
         if (r < nr) {
@@ -174,10 +180,10 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
     }
     // this warp's rows: warp + 8 j for j < jn
     const int jn = nr > warp ? (nr - warp + 7) / 8 : 0;
-    int lim[8];   // committed tokens each row may see
-    float m[8], l[8], acc[8][4];
+    int lim[RPW];   // committed tokens each row may see
+    float m[RPW], l[RPW], acc[RPW][4];
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
+    for (int j = 0; j < RPW; j++) {
         const int i = (r0 + warp + 8 * j) / a.G;
         lim[j] = min(Tb, Tb + a.n_tail - a.n + 1 + i);
         m[j] = -CUDART_INF_F;
@@ -201,15 +207,15 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
         dequant_tile<BA, BR>(a, st, 0, MR, resid, tn, sK, warp, lane);
         __syncthreads();
         // logits of token lane for the warp's rows
-        float s[8];
+        float s[RPW];
 #pragma unroll
-        for (int j = 0; j < 8; j++) s[j] = 0.f;
+        for (int j = 0; j < RPW; j++) s[j] = 0.f;
         const float *kr = sK + lane * kKStride;
 #pragma unroll 2
         for (int d = 0; d < kHeadDim; d += 4) {
             const float k0 = kr[d], k1 = kr[d + 1], k2 = kr[d + 2], k3 = kr[d + 3];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < RPW; j++) {
                 if (j < jn) {
                     const float4 qv = *reinterpret_cast<const float4 *>(sQ + (warp + 8 * j) * kQStride + d);
                     s[j] = fmaf(qv.x, k0, fmaf(qv.y, k1, fmaf(qv.z, k2, fmaf(qv.w, k3, s[j]))));
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
         // online softmax per row (log2 domain); masked tokens weigh 0
         const int tabs = t0 + tt + lane;
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
+        for (int j = 0; j < RPW; j++) {
             if (j < jn) {
                 const bool valid = lane < tn && tabs < lim[j];
                 const float z = valid ? s[j] : -CUDART_INF_F;
@@ -249,7 +255,7 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
             const float *vr = sK + t * kKStride;
             const float v0 = vr[lane], v1 = vr[lane + 32], v2 = vr[lane + 64], v3 = vr[lane + 96];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < RPW; j++) {
                 if (j < jn) {
                     const float p = sP[(warp + 8 * j) * kPStride + t];
                     acc[j][0] = fmaf(p, v0, acc[j][0]);
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(kThreadsP, 2) prefill_rq_kernel(const PrefillA
     cp_async_wait<0>();
 
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
+    for (int j = 0; j < RPW; j++) {
         if (j < jn) {
             const int rg = r0 + warp + 8 * j, i = rg / a.G, gq = rg % a.G;
             const size_t row = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
@@ -299,37 +305,84 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
                 (size_t)a.H * kHeadDim, nt, a.out + row * kHeadDim, threadIdx.x, s_red, Sync128());
 }
 
-template <int BA, int BR>
-cudaError_t launch_t(const PrefillArgs &a, cudaStream_t st) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_rq_kernel<BA, BR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)Stage<BA, BR>::smem());
-        if (e != cudaSuccess) return e;
-        configured = true;
+template <int BA, int BR, int RPW>
+struct Variant {
+    static cudaError_t configure() {
+        static bool done = false;
+        if (done) return cudaSuccess;
+        cudaError_t e = cudaFuncSetAttribute(prefill_rq_kernel<BA, BR, RPW>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)Stage<BA, BR>::smem(8 * RPW));
+        if (e == cudaSuccess) done = true;
+        return e;
     }
-    if (a.S > 0)
-        prefill_rq_kernel<BA, BR><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, Stage<BA, BR>::smem(), st>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
-    return cudaGetLastError();
+    static int occupancy() {
+        static int occ = 0;
+        if (occ == 0 && configure() == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prefill_rq_kernel<BA, BR, RPW>, kThreadsP,
+                                                          Stage<BA, BR>::smem(8 * RPW)) != cudaSuccess)
+            occ = 0;
+        return occ > 0 ? occ : 1;
+    }
+    static cudaError_t launch(const PrefillArgs &a, cudaStream_t st) {
+        cudaError_t e = configure();
+        if (e != cudaSuccess) return e;
+        if (a.S > 0)
+            prefill_rq_kernel<BA, BR, RPW>
+                <<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, Stage<BA, BR>::smem(8 * RPW), st>>>(a);
+        return cudaGetLastError();
+    }
+};
+
+// f(Variant) for the (bits, rows per warp) of a
+template <typename F>
+auto with_variant(int ba, int br, int rpw, F f) -> decltype(f(Variant<4, 2, 1>())) {
+#define RQ_PREFILL_RPW(BA, BR)                      \
+    switch (rpw) {                                  \
+        case 1: return f(Variant<BA, BR, 1>());     \
+        case 2: return f(Variant<BA, BR, 2>());     \
+        case 4: return f(Variant<BA, BR, 4>());     \
+        default: return f(Variant<BA, BR, 8>());    \
+    }
+    if (ba == 2 && br == 2) RQ_PREFILL_RPW(2, 2)
+    if (ba == 4 && br == 4) RQ_PREFILL_RPW(4, 4)
+    RQ_PREFILL_RPW(4, 2)
+#undef RQ_PREFILL_RPW
 }
 
 }  // namespace
 
-int prefill_splits(int T, int units, int sms) {
-    if (T <= 0 || units <= 0) return 0;
+// Rows per warp: the fewest that hold every query row of a kv head (at most
+// 8, 64 rows per CTA).  Splits: the count with the least wave-quantised work
+// (waves x 64-token tiles of the largest split, plus one tile of fixed cost),
+// waves counted from the variant's measured occupancy.
+void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
+    const int nq = a->n * a->G;
+    a->rpw = nq <= 8 ? 1 : nq <= 16 ? 2 : nq <= 32 ? 4 : 8;
+    a->nqb = (nq + 8 * a->rpw - 1) / (8 * a->rpw);
+    a->S = 0;
+    if (T <= 0) return;
+    const int occ = with_variant(ba, br, a->rpw, [](auto v) { return decltype(v)::occupancy(); });
+    const long slots = (long)std::max(1, occ) * std::max(1, sms);
+    const long units = (long)a->B * a->H * a->nqb;
     const int nt = (T + kTokTile - 1) / kTokTile;
-    const int want = (4 * sms + units - 1) / units;   // about two waves at two CTAs per SM
-    return std::max(1, std::min(std::min(nt, kMaxSplits), want));
+    long best = -1;
+    for (int S = 1; S <= std::min(nt, kMaxSplits); S++) {
+        const long waves = (S * units + slots - 1) / slots;
+        const long cost = waves * ((nt + S - 1) / S + 1);
+        if (best < 0 || cost < best) {
+            best = cost;
+            a->S = S;
+        }
+    }
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st) {
-    if (ba == 4 && br == 2) return launch_t<4, 2>(a, st);
-    if (ba == 2 && br == 2) return launch_t<2, 2>(a, st);
-    if (ba == 4 && br == 4) return launch_t<4, 4>(a, st);
-    return cudaErrorInvalidValue;
+    if (!((ba == 4 && br == 2) || (ba == 2 && br == 2) || (ba == 4 && br == 4))) return cudaErrorInvalidValue;
+    cudaError_t e = with_variant(ba, br, a.rpw, [&](auto v) { return decltype(v)::launch(a, st); });
+    if (e != cudaSuccess) return e;
+    prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace rq

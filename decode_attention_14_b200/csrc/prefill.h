@@ -6,7 +6,6 @@
 
 namespace rq {
 
-constexpr int kPrefillRows = 64;   // query rows (token x q head of one kv head) per CTA
 constexpr int kPrefillTile = 32;   // committed tokens per step of a CTA
 
 // Causal attention of the n most recent tokens of every sequence: query row
@@ -22,16 +21,17 @@ struct PrefillArgs {
     float *partials;                   // [B][n][Hq][S][kPartialStride]
     float *out;                        // [B][n][Hq][d] fp32
     SeqLens seqT;                      // committed tokens of each sequence
-    int B, H, Hq, G, n, n_tail, tail_cap, Tp, S, nqb;
+    int B, H, Hq, G, n, n_tail, tail_cap, Tp, S;
+    int rpw, nqb;                      // query rows per warp (8 per CTA), row blocks per kv head
     int g;                             // quantization group size
     float scale_log2;                  // softmax_scale * log2(e)
     int rotate;
     uint32_t sigma[4];
 };
 
-// Splits over the committed tokens (and so the partial slots per query row)
-// for a prefill of `units` = B * H * nqb CTAs per split.
-int prefill_splits(int T, int units, int sms);
+// Sets a->rpw, a->nqb and the split count a->S over the committed tokens (T
+// = the longest sequence); a->B, H, G and n must be set.
+void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms);
 cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st);
 
 }  // namespace rq

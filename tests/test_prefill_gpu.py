@@ -91,11 +91,13 @@ def _f64(t):
     return orc.bf16_bits_to_f64(synth.bf16_to_u16(t))
 
 
-@pytest.mark.parametrize("n", [1, 5, 33])
-def test_prefill_chunk_through_a_group(n):
+@pytest.mark.parametrize("n,Hq", [(1, 4), (5, 4), (7, 8), (33, 4)])
+def test_prefill_chunk_through_a_group(n, Hq):
     """A chunk of n tokens through loops 0..3: tails at loops 0-2, committed
-    at the anchor loop; then loop 0 again with the chunk committed."""
-    B, Hkv, Hq, T = 2, 2, 4, 300
+    at the anchor loop; then loop 0 again with the chunk committed.  n * G
+    query rows per kv head: 2, 10, 28 and 66 (1, 2, 4 and 8 rows per warp,
+    the last over two row blocks)."""
+    B, Hkv, T = 2, 2, 300
     G = Hq // Hkv
     bt = H.build(layers=1, loops=4, Lg=4, B=B, T=T, H=Hkv, Hq=Hq, n_tail=0, chunk=64, seed=0x5EED9000,
                  max_tokens=T + n)
