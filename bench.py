@@ -622,6 +622,82 @@ def run_sweep(args):
     return rows
 
 
+# FP32 lanes x 2 flops x SMs x maximum SM clock of a B200: the ALU roofline of
+# a kernel whose products run as fp32 FMAs
+FP32_PEAK_TFLOPS = 128 * 2 * 148 * 1.965e9 / 1e12
+
+
+def run_prefill(args):
+    """rq_prefill_attn on the Ouro-1.4B-shaped cache (B = 4, T = 8192, H = 16):
+    n new tokens per sequence, timed at a residual loop (the chunk in the BF16
+    tail) and at the anchor loop (the chunk committed).  One JSON line per
+    (n, loop kind).  FLOPs counted: 2 x 128 for q.k and 2 x 128 for p v per
+    (query row, committed token)."""
+    import torch
+    import decode_attention_14_b200 as rq
+    from decode_attention_14_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = CONFIGS["ouro8k_b4"]
+    loops, Lg, T, H, Hq, B = base["loops"], base["Lg"], base["T"], base["H"], base["Hq"], base["B"]
+    reps = 10
+    rows = []
+    for n in [int(x) for x in args.prefill.split(",")]:
+        cfg = rq.make_config(num_layers=1, num_loops=loops, loops_per_group=Lg, batch=B, max_tokens=T + n,
+                             max_tail_tokens=max(FILL_CHUNK, n), num_kv_heads=H, num_q_heads=Hq, seed=0xA11CE)
+        cache = rq.Cache(cfg, device=dev)
+        seed = 0x5EED0007 + n
+        for t0 in range(0, T, FILL_CHUNK):
+            Kg, Vg = synth.group_kv(seed, 0, 0, Lg, base["sigma"], B, FILL_CHUNK, H, t0=t0, device=dev)
+            for j in range(Lg):
+                cache.append(0, j, Kg[j], Vg[j])
+        Kn, Vn = synth.group_kv(seed, 0, 0, Lg, base["sigma"], B, n, H, t0=T, device=dev)
+        q = torch.randn((B, n, Hq, 128), generator=torch.Generator(device=dev).manual_seed(seed), device=dev)
+        q = q.to(torch.bfloat16)
+        out = torch.empty((B, n, Hq, 128), dtype=torch.float32, device=dev)
+        for kind in ("residual", "anchor"):
+            if kind == "residual":
+                cache.append(0, 0, Kn[0], Vn[0])
+                loop = 0
+            else:
+                for j in range(1, Lg):
+                    cache.append(0, j, Kn[j], Vn[j])
+                loop = Lg - 1
+            for _ in range(3):
+                assert rq.rq_prefill_attn(cache.h, 0, loop, q, n, out, 0.0) == 0
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(reps):
+                    st = rq.rq_prefill_attn(cache.h, 0, loop, q, n, out, 0.0)
+                    if st != 0:
+                        raise rq.RQError(st, "rq_prefill_attn")
+            g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            del g
+            committed = T if kind == "residual" else T + n
+            flops = 4.0 * 128 * n * Hq * B * committed
+            tflops = flops / (us * 1e-6) / 1e12
+            row = {"prefill": "ouro8k_b4", "n_tokens": n, "loop": kind, "batch": B, "seq_len": committed,
+                   "us_per_call": round(us, 1), "query_tokens_per_s": round(B * n / (us * 1e-6), 1),
+                   "decode_bytes_per_call": cache.decode_bytes(0, loop),
+                   "roofline": {"bound": "alu", "achieved": round(tflops, 2), "peak": round(FP32_PEAK_TFLOPS, 1),
+                                "unit": "TFLOP/s", "frac": round(tflops / FP32_PEAK_TFLOPS, 4),
+                                "peak_kind": "fp32 FMA lanes x clock (derived)"},
+                   "timing": "CUDA graph of %d calls, CUDA events" % reps}
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+        cache.check()
+        cache.close()
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -640,6 +716,8 @@ def main():
     ap.add_argument("--json-out", default="")
     ap.add_argument("--sweep", action="store_true",
                     help="batch x format sweep of the Ouro shape at T=8192 (one JSON line per row)")
+    ap.add_argument("--prefill", default="",
+                    help="comma-separated chunk sizes: time rq_prefill_attn on the Ouro shape instead")
     ap.add_argument("--profile", action="store_true",
                     help="bracket the timed region with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     args = ap.parse_args()
@@ -652,6 +730,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.prefill:
+        run_prefill(args)
         return
     if args.impl == "reference":
         if rank == 0:
