@@ -71,6 +71,9 @@ def lib():
         L.orc_attention.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [ctypes.c_void_p] * 4 + [ctypes.c_int]
         L.orc_mse.restype = ctypes.c_double
         L.orc_mse.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
+        L.orc_encode_ablation.restype = None
+        L.orc_encode_ablation.argtypes = [ctypes.c_int] * 7 + [ctypes.c_uint64] + [ctypes.c_int] * 2 + \
+            [ctypes.c_void_p] * 4
         _lib = L
     return _lib
 
@@ -202,6 +205,25 @@ def reconstruct(a_codes, a_meta, r_codes, r_meta, r_coef, L: int, d: int, g: int
     lib().orc_reconstruct(n, L, d, g, ba, br, int(rotate), seed, _p(a_codes), _p(a_meta),
                           _p(r_codes), _p(r_meta), _p(r_coef), _p(out))
     return out
+
+
+ANCHOR_LAST, ANCHOR_PREVIOUS = 0, 1
+SCALE_LEAST_SQUARES, SCALE_NORM_RATIO, SCALE_NONE = 0, 1, 2
+
+
+def encode_ablation(x_bf16: np.ndarray, g: int, ba: int, br: int, rotate: bool, seed: int,
+                    anchor_mode: int, scale_mode: int):
+    """Ablation encoders of one loop group (orc_encode_ablation): x_bf16
+    uint16 [L][n][d] -> (reconstruction float64 [L][n][d], stored
+    coefficients float64 [L][n], records read to rebuild each loop [L])."""
+    x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)
+    L, n, d = x_bf16.shape
+    xhat = np.zeros((L, n, d), np.float64)
+    coef = np.zeros((L, n), np.float64)
+    reads = np.zeros(L, np.int32)
+    lib().orc_encode_ablation(n, L, d, g, ba, br, int(rotate), seed, int(anchor_mode), int(scale_mode),
+                              _p(x_bf16), _p(xhat), _p(coef), _p(reads))
+    return xhat, coef, reads
 
 
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, threads: int = 1) -> np.ndarray:

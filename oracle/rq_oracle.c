@@ -453,6 +453,97 @@ ORC_EXPORT void orc_reconstruct(int n, int L, int d, int g, int ba, int br, int 
 }
 
 /* ------------------------------------------------------------------ */
+/* Ablation encoders (the arXiv abstract's comparison of reference      */
+/* choice and scaling method): encode one loop group of n token-heads   */
+/* and return the reconstruction, for reconstruction-error studies.     */
+/*   anchor_mode 0: last-loop anchor, shared -- loop L-1 is quantized   */
+/*                  at ba bits; every other loop l is a residual        */
+/*                  against a_hat (the method; identical to orc_encode  */
+/*                  followed by orc_reconstruct);                        */
+/*   anchor_mode 1: previous-loop anchor, chained -- loop 0 is          */
+/*                  quantized at ba bits; loop l >= 1 is a residual     */
+/*                  against the reconstruction of loop l-1, so its      */
+/*                  reconstruction reads l+1 records.                    */
+/*   scale_mode  0: least squares  s = <x, ref>/<ref, ref> (0 if ref=0);*/
+/*   scale_mode  1: norm ratio     s = |x| / |ref| (0 if ref=0);        */
+/*   scale_mode  2: none           s = 1.                                */
+/* In every mode s is stored as BF16, the residual x - s_hat ref is     */
+/* rotated by R and quantized at br bits, and the reconstruction is     */
+/* s_hat ref + R^T y_hat.                                                */
+/*   x_bf16 [L][n][d]; xhat out [L][n][d]; coef out [L][n] (s_hat, 0 for */
+/*   the anchor loop); reads out [L]: records read to rebuild each loop. */
+/* Readings (the pages name the variants only): the previous-loop       */
+/* anchor is the first loop of the group, so that every loop but one    */
+/* has a reference; norm-ratio scaling keeps s >= 0.                     */
+/* ------------------------------------------------------------------ */
+ORC_EXPORT void orc_encode_ablation(int n, int L, int d, int g, int ba, int br, int rotate, uint64_t seed,
+                                    int anchor_mode, int scale_mode, const uint16_t *x_bf16,
+                                    double *xhat, double *coef, int *reads)
+{
+    int t, l, i, j;
+    int G = d / g;
+    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double *x = (double *)malloc(sizeof(double) * (size_t)d);
+    double *r = (double *)malloc(sizeof(double) * (size_t)d);
+    double *y = (double *)malloc(sizeof(double) * (size_t)d);
+    double *yhat = (double *)malloc(sizeof(double) * (size_t)d);
+    uint8_t *packed = (uint8_t *)malloc((size_t)d);
+    uint8_t *meta = (uint8_t *)malloc((size_t)(2 * G));
+    const int first = anchor_mode == 0 ? L - 1 : 0;   /* the anchor loop */
+    orc_rotation_matrix(seed, d, rotate, R);
+    for (l = 0; l < L; l++)
+        reads[l] = l == first ? 1 : (anchor_mode == 0 ? 2 : l + 1);
+    for (t = 0; t < n; t++) {
+        double *ahat = xhat + ((size_t)first * n + t) * d;
+        for (i = 0; i < d; i++)
+            x[i] = orc_bf16_value(x_bf16[((size_t)first * n + t) * d + i]);
+        quantize_record(x, d, g, ba, packed, meta, NULL, NULL);
+        orc_dequant(packed, meta, d, g, ba, ahat);
+        coef[(size_t)first * n + t] = 0.0;
+        for (l = 0; l < L; l++) {
+            double num = 0.0, den = 0.0, xx = 0.0, s = 0.0, shat;
+            const double *ref;
+            double *o;
+            if (l == first)
+                continue;
+            /* chained: loops 1, 2, ... in order, each against the one before */
+            ref = anchor_mode == 0 ? ahat : xhat + ((size_t)(l - 1) * n + t) * d;
+            o = xhat + ((size_t)l * n + t) * d;
+            for (i = 0; i < d; i++)
+                x[i] = orc_bf16_value(x_bf16[((size_t)l * n + t) * d + i]);
+            for (i = 0; i < d; i++) {
+                num += x[i] * ref[i];
+                den += ref[i] * ref[i];
+                xx += x[i] * x[i];
+            }
+            if (scale_mode == 2)
+                s = 1.0;
+            else if (den != 0.0)
+                s = scale_mode == 0 ? num / den : sqrt(xx) / sqrt(den);
+            shat = orc_bf16_value(orc_bf16_round(s, NULL));
+            coef[(size_t)l * n + t] = shat;
+            for (i = 0; i < d; i++)
+                r[i] = x[i] - shat * ref[i];
+            for (i = 0; i < d; i++) {
+                double acc = 0.0;
+                for (j = 0; j < d; j++)
+                    acc += R[i * d + j] * r[j];
+                y[i] = acc;
+            }
+            quantize_record(y, d, g, br, packed, meta, NULL, NULL);
+            orc_dequant(packed, meta, d, g, br, yhat);
+            for (i = 0; i < d; i++) {
+                double acc = 0.0;
+                for (j = 0; j < d; j++)
+                    acc += R[j * d + i] * yhat[j];
+                o[i] = shat * ref[i] + acc;
+            }
+        }
+    }
+    free(R); free(x); free(r); free(y); free(yhat); free(packed); free(meta);
+}
+
+/* ------------------------------------------------------------------ */
 /* Direct softmax attention in fp64 (two passes: max, then weights).    */
 /*   q   [B][Hq][d]                                                      */
 /*   k,v [B][T][Hkv][d]  (all keys this query may see, in token order)   */
