@@ -36,7 +36,9 @@
  * fp64, with no blocking, fusion or reordering.  The rotation is applied as
  * an explicit O(d^2) matrix product (not a butterfly).
  *
- * Parity pins: see tests/test_oracle_pins.py.  Every function below is
+ * Parity pins: see tests/test_oracle_pins.py (and tests/test_oracle_ablation.py
+ * for orc_encode_ablation, the abstract's ablation variants: previous-loop
+ * chained anchor, norm-ratio and no scaling).  Every function below is
  * pinned there against something other than itself.
  *
  * Logical record format (what this oracle produces and what the CUDA
