@@ -99,6 +99,10 @@ def test_null_arguments_rejected_without_device():
     assert rq.lib.rq_append(None, 0, 0, None, None, 1, None) == rq.RQ_ERR_INVALID
     assert rq.lib.rq_decode_attn(None, 0, 0, None, None, 0.0, None) == rq.RQ_ERR_INVALID
     assert rq.lib.rq_decode_attn_bf16(None, 0, 0, None, None, 0.0, None) == rq.RQ_ERR_INVALID
+    assert rq.lib.rq_prefill_attn(None, 0, 0, None, 4, None, 0.0, None) == rq.RQ_ERR_INVALID
+    assert rq.lib.rq_append_decode_attn(None, 0, 0, None, None, 1, None, None, 0.0, None) == rq.RQ_ERR_INVALID
+    assert rq.lib.rq_decode_attn_noalloc(None, 0, 0, None, None, 0.0, None) == rq.RQ_ERR_INVALID
+    assert rq.lib.rq_cache_truncate_seq(None, 0, 0, 0, 0) == rq.RQ_ERR_INVALID
     assert rq.lib.rq_cache_export(None, 0, 0, None, None, None, None) == rq.RQ_ERR_INVALID
     assert rq.lib.rq_cache_truncate(None, 0, 0, 0) == rq.RQ_ERR_INVALID
     assert rq.lib.rq_check(None) == rq.RQ_ERR_INVALID
