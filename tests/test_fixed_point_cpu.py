@@ -14,8 +14,7 @@ Ouro-shaped synthetic workload and bounds its error against exact fp64
 attention over the same records: the rounding alone must stay well inside the
 parity bound (max abs 2e-3) that the GPU tests apply, with room left for the
 fp32 arithmetic around it.  It exercises no GPU code; it documents why 24 and
-28 bits were chosen (16-bit q or weights exceed the bound, see the design
-notes' precision paragraph).
+28 bits were chosen: with 16-bit weights the same arithmetic breaks the bound.
 """
 import math
 
