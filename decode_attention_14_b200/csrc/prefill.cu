@@ -17,13 +17,14 @@
 //    n * G rows), 8 warps; warp w owns rows w, w + 8, ...;
 //  - per 32-token step: dequantize K (warp per token), logits (lane = token,
 //    a row's 32 logits in one warp), online softmax per row, dequantize V,
-//    o += p V (lane = 4 columns of head_dim);
+//    o += p V (lane = 4 columns of head_dim); the raw records of the next
+//    step are copied into a second shared buffer (cp.async) meanwhile;
 //  - each CTA writes a partial (m, l, o) per row; a second kernel merges the
 //    partials and the tail tokens of each row (combine_row) under the row's
 //    causal limit.
-// This is a CUDA-core kernel: the contraction per step is 64 x 32 x 128
-// twice, too small and too oddly shaped (fp32 reconstruction) to pay for a
-// tensor-core pipeline at these row counts.
+// This is a CUDA-core kernel: the contraction per step is at most 64 x 32 x
+// 128 twice, on fp32 reconstructions; BF16 tensor-core operands would add a
+// rounding of every reconstructed key and value.
 #include <math_constants.h>
 
 #include <algorithm>
