@@ -168,7 +168,7 @@ def rank_seed(base: int, rank: int) -> int:
 def run_ours(args, cfgd, rank, world, local_rank):
     import torch
     import decode_attention_14_b200 as rq
-    from decode_attention_14_b200 import synth
+    import synth
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -426,19 +426,22 @@ class OracleUnits:
 
     def __init__(self, cfgd, seed, n_units: int, T: int | None = None):
         import torch
-        from decode_attention_14_b200 import synth
+        import synth
         from oracle import oracle as orc
+        from concurrent.futures import ThreadPoolExecutor
         self.cfgd, self.T = cfgd, T or cfgd["T"]
         Lg = cfgd["Lg"]
-        self.units = []
+        inputs = []
         for u in range(n_units):
             Kg, Vg = synth.group_kv(seed + u, 0, 0, Lg, cfgd["sigma"], 1, self.T, 1, device="cpu")
-            recs = []
-            for X in (Kg, Vg):
-                x = np.stack([synth.bf16_to_u16(X[j]).reshape(-1, 128) for j in range(Lg)])
-                recs.append(orc.encode(x, cfgd["g"], cfgd["ba"], cfgd["br"], True, 0xA11CE))
-            q = torch.randn((1, 1, 128)).to(torch.bfloat16)
-            self.units.append((recs, orc.bf16_bits_to_f64(synth.bf16_to_u16(q))))
+            xs = [np.stack([synth.bf16_to_u16(X[j]).reshape(-1, 128) for j in range(Lg)]) for X in (Kg, Vg)]
+            q = torch.randn((1, 1, 128), generator=torch.Generator().manual_seed(seed + u)).to(torch.bfloat16)
+            inputs.append((xs, orc.bf16_bits_to_f64(synth.bf16_to_u16(q))))
+        # encode the units' records concurrently (the oracle's C calls release the interpreter lock)
+        with ThreadPoolExecutor(max_workers=2 * n_units) as ex:
+            recs = list(ex.map(lambda x: orc.encode(x, cfgd["g"], cfgd["ba"], cfgd["br"], True, 0xA11CE),
+                               [x for xs, _ in inputs for x in xs]))
+        self.units = [(recs[2 * u:2 * u + 2], inputs[u][1]) for u in range(n_units)]
 
     def decode_seconds(self, u: int, loop: int) -> float:
         """One decode call of one unit, timed: reconstruct the loop's K and V
@@ -466,25 +469,44 @@ def calls_per_step(cfgd) -> int:
     return cfgd["layers"] * cfgd["loops"] * cfgd["B"] * cfgd["H"]   # (unit, loop) decodes per step
 
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_round(ou: "OracleUnits", threads: int, first: int) -> float:
+    """Wall seconds of `threads` unit-loop decodes run at once, one per host
+    thread (the oracle's C calls release the interpreter lock): unit-loop i
+    is unit i // Lg, loop i % Lg, for i = first .. first + threads - 1."""
+    from concurrent.futures import ThreadPoolExecutor
+    Lg = ou.cfgd["Lg"]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda i: ou.decode_seconds(i // Lg, i % Lg), range(first, first + threads)))
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(cfgd, seed, budget_s: float = 15.0):
-    """The oracle as it stands, one host core, on a bounded sample of the
-    workload: every loop of a few (sequence, kv head) units at full T,
-    scaled to a decode step."""
-    ou = OracleUnits(cfgd, seed, 2)
+    """The oracle as it stands on all host cores, on a bounded sample of the
+    workload: rounds of one unit-loop decode per core ((sequence, kv head)
+    units at full T, every loop in turn), scaled to a decode step."""
+    threads = host_cores()
+    ou = OracleUnits(cfgd, seed, min(4, threads))
     Lg = cfgd["Lg"]
-    times, t_start = [], time.perf_counter()
-    while time.perf_counter() - t_start < budget_s or len(times) < Lg:
-        i = len(times)
-        times.append(ou.decode_seconds(i // Lg, i % Lg))
-        if len(times) >= 8 * Lg:
+    walls, done, t_start = [], 0, time.perf_counter()
+    while time.perf_counter() - t_start < budget_s or done < Lg:
+        walls.append(oracle_round(ou, threads, done))
+        done += threads
+        if len(walls) >= 64:
             break
-    # average over whole groups of loops (anchor and residual loops in proportion)
-    n = len(times) // Lg * Lg
-    per = float(np.mean(times[:n]))
-    step_s = per * calls_per_step(cfgd)
-    return {"value": round(cfgd["B"] / step_s, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} unit-loop decodes ({n // Lg} (sequence, kv head) unit pass(es) over all {Lg} loops) "
-                      f"at T={cfgd['T']}, {per:.3f} s each (reconstruct from records + fp64 softmax), scaled to "
+    rate = done / sum(walls)                      # unit-loop decodes per second, all cores
+    step_s = calls_per_step(cfgd) / rate
+    return {"value": round(cfgd["B"] / step_s, 6), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} unit-loop decodes in {len(walls)} round(s) of {threads} concurrent ones (one per "
+                      f"host core; {len(ou.units)} distinct (sequence, kv head) units at T={cfgd['T']}, all {Lg} loops "
+                      f"in turn; reconstruct from records + fp64 softmax), {sum(walls):.1f} s, scaled to "
                       f"{calls_per_step(cfgd)} unit-loops per decode step (extrapolated)"}
 
 
@@ -497,20 +519,22 @@ def workload_config(name: str, cfgd, layers: int, world: int) -> dict:
 
 
 def run_reference(args, cfgd):
-    """The oracle, timed as it stands on one host core: each step is a
-    bounded sample -- one (sequence, kv head) unit of one loop at full T
-    (reconstruct from records + direct fp64 softmax), loops taken in turn --
-    scaled to the workload's decode step."""
+    """The oracle, timed as it stands on all host cores: each step is a
+    bounded sample -- one round of unit-loop decodes, one per host core
+    ((sequence, kv head) units at full T, loops in turn; reconstruct from
+    records + direct fp64 softmax) -- scaled to the workload's decode step."""
     seed = CONFIG_SEED[args.config]
-    ou = OracleUnits(cfgd, seed, 2)
-    Lg = cfgd["Lg"]
+    threads = host_cores()
+    ou = OracleUnits(cfgd, seed, min(4, threads))
     for w in range(args.warmup):
-        ou.decode_seconds(w, w % Lg)
-    per = float(np.mean([ou.decode_seconds(s // Lg, s % Lg) for s in range(args.steps)]))
-    step_s = per * calls_per_step(cfgd)
+        oracle_round(ou, threads, w * threads)
+    walls = [oracle_round(ou, threads, (args.warmup + s) * threads) for s in range(args.steps)]
+    rate = threads * args.steps / sum(walls)
+    step_s = calls_per_step(cfgd) / rate
     value = cfgd["B"] / step_s
-    sample = (f"per step: 1 (sequence, kv head) unit x 1 loop (loops in turn) at T={cfgd['T']} (oracle reconstruct "
-              f"+ fp64 softmax, {per:.3f} s), scaled to {calls_per_step(cfgd)} unit-loops per decode step")
+    sample = (f"per step: {threads} concurrent unit-loop decodes (one per host core, loops in turn) at "
+              f"T={cfgd['T']} (oracle reconstruct + fp64 softmax, {np.mean(walls):.3f} s per round), scaled to "
+              f"{calls_per_step(cfgd)} unit-loops per decode step")
     return {
         "impl": "reference",
         "metric": "decode-attention tokens/s (INT4 anchor/INT2 resid)",
@@ -519,8 +543,8 @@ def run_reference(args, cfgd):
         "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded, CPU generator)",
         "config": dict(workload_config(args.config, cfgd, cfgd["layers"], int(os.environ.get("WORLD_SIZE", "1"))),
-                       host="the oracle on one host core (rank 0)"),
-        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                       host=f"the oracle on {threads} host cores (rank 0)"),
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -546,7 +570,7 @@ def run_sweep(args):
     algorithmic bytes."""
     import torch
     import decode_attention_14_b200 as rq
-    from decode_attention_14_b200 import synth
+    import synth
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -635,7 +659,7 @@ def run_prefill(args):
     (query row, committed token)."""
     import torch
     import decode_attention_14_b200 as rq
-    from decode_attention_14_b200 import synth
+    import synth
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)

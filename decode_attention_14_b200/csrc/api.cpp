@@ -21,6 +21,10 @@ struct rq_cache {
     std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]; the longest sequence
     std::vector<int> seq;     // the same, per sequence: [layer][group or loop][batch]
     std::vector<int> ntail;   // [layer][loop]
+    // per length slot: the first token position the most recent record write
+    // (an anchor append) started at, over the sequences; records below it are
+    // not touched by any append still in flight
+    std::vector<int> wstart;
     uint32_t sigma[4] = {0, 0, 0, 0};
     // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
     int occ[2][kMaxChunk / kTokTile];
@@ -76,6 +80,14 @@ uint16_t *bf16_ptr(const rq_cache *c, int layer, int loop, int kv) {
                         kv * L.bf16_side);
 }
 
+// largest V scale byte of record r (r < Lg - 1: residual of loop r; r = Lg - 1:
+// the anchor) of every (sequence, kv head) of (layer, group): int [B][H]
+int *vmax_ptr(const rq_cache *c, int layer, int group, int r) {
+    const Layout &L = c->lay;
+    const size_t bh = (size_t)L.cfg.batch * L.cfg.num_kv_heads;
+    return (int *)(c->base + L.off_vmax) + (((size_t)layer * L.groups + group) * L.Lg + r) * bh;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
 
 // per-sequence lengths of length slot `slot` (= layer * groups + group, or
@@ -92,6 +104,17 @@ void grow(rq_cache *c, size_t slot, int n) {
 }
 
 float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt((float)kHeadDim); }
+
+// Kernels run on the current device and address the cache's arena, so the
+// two must be the same device.
+bool on_cache_device(const rq_cache *c) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return dev == c->device;
+}
 
 // Split-KV partition of T tokens over `units` independent (sequence, kv head
 // [, q-head pair]) problems.  The ceil(T/64) tiles are dealt out evenly over
@@ -168,7 +191,11 @@ bool make_layout(const rq_config &cfg, Layout *out) {
     size_t partial_bytes = align_up(B * Hq * (size_t)L.splits_max * kPartialStride * sizeof(float), kAlign);
     L.off_counters = L.off_partials + partial_bytes;
     L.off_err = L.off_counters + align_up(B * Hq * sizeof(int), kAlign);
-    L.total = L.off_err + kAlign;
+    L.off_vmax = L.off_err + kAlign;
+    const size_t vmax_bytes = cfg.format == RQ_FMT_RESIDUAL
+                                  ? align_up((size_t)cfg.num_layers * L.groups * L.Lg * B * H * sizeof(int), kAlign)
+                                  : 0;
+    L.total = L.off_vmax + vmax_bytes;
     *out = L;
     return true;
 }
@@ -274,6 +301,7 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
     c->len.assign((size_t)cfg->num_layers * (cfg->format == RQ_FMT_RESIDUAL ? L.groups : cfg->num_loops), 0);
     c->seq.assign(c->len.size() * (size_t)cfg->batch, 0);
     c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
+    c->wstart.assign(c->len.size(), 0x7FFFFFFF);
     {
         const int G = cfg->num_q_heads / cfg->num_kv_heads;
         for (int i = 0; i < kMaxChunk / kTokTile; i++) {
@@ -308,6 +336,7 @@ int rq_cache_destroy(rq_cache *c) {
 
 int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, int n, void *stream) {
     if (!c || !k || !v || n < 1) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
@@ -370,6 +399,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     a.a_codes0 = anchor_codes(c, layer, group, 0);
     a.a_meta0 = anchor_meta(c, layer, group, 0);
     a.anchor_kv_stride = L.anchor_codes_bytes + L.anchor_meta_bytes;
+    a.vmax = vmax_ptr(c, layer, group, 0);
     a.B = cfg.batch;
     a.H = cfg.num_kv_heads;
     a.n = n;
@@ -383,6 +413,9 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
     int s = cuda_status(launch_append(a, st));
     if (s != RQ_OK) return s;
+    int w0 = 0x7FFFFFFF;
+    for (int b = 0; b < cfg.batch; b++) w0 = std::min(w0, a.pos0.v[b]);
+    c->wstart[slot] = w0;
     grow(c, slot, n);
     for (int jj = 0; jj < L.Lg - 1; jj++) c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] = 0;
     return RQ_OK;
@@ -397,6 +430,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
                          int *counters = nullptr, size_t max_units = 0, const void *app_k = nullptr,
                          const void *app_v = nullptr, int app_n = 0) {
     if (!c || !q || !out) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
@@ -434,8 +468,11 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
             a.a_codes[kv] = anchor_codes(c, layer, group, kv);
             a.a_meta[kv] = anchor_meta(c, layer, group, kv);
         }
+        a.vmax_a = vmax_ptr(c, layer, group, L.Lg - 1);
+        a.stable = c->wstart[(size_t)layer * L.groups + group];
         if (!is_anchor_loop(L, loop)) {
             resid = true;
+            a.vmax_r = vmax_ptr(c, layer, group, j);
             for (int kv = 0; kv < 2; kv++) {
                 a.r_codes[kv] = resid_codes(c, layer, group, j, kv);
                 a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
@@ -505,6 +542,8 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
 }  // extern "C"
 
 namespace rq {
+int cache_device(const rq_cache *c) { return c->device; }
+
 int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
                         float *partials, size_t partial_floats, int *counters, size_t max_units) {
     if (!partials || !counters) return RQ_ERR_INVALID;
@@ -534,10 +573,13 @@ int rq_decode_attn_bf16(rq_cache *c, int layer, int loop, const void *q, float *
 int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, float *out, float scale,
                     void *stream) {
     if (!c || !q || !out || n <= 0) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
     if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
+    // the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4
+    if (cfg.anchor_bits == 2 && cfg.resid_bits == 4) return RQ_ERR_UNSUPPORTED;
     PrefillArgs a;
     std::memset(&a, 0, sizeof(a));
     const int group = loop / L.Lg, j = loop % L.Lg;
@@ -662,6 +704,7 @@ int rq_cache_length_seq(const rq_cache *c, int layer, int group, int seq, int *l
 int rq_cache_export(const rq_cache *c, int layer, int loop, void *host_codes, void *host_meta, void *host_coef,
                     void *stream) {
     if (!c || !host_codes || !host_meta) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
     const Layout &L = c->lay;
     const rq_config &cfg = L.cfg;
     if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
@@ -721,15 +764,21 @@ size_t rq_decode_bytes(const rq_cache *c, int layer, int loop) {
 
 int rq_check(rq_cache *c) {
     if (!c) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
     if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
     int err = 0;
     if (cudaMemcpy(&err, c->base + c->lay.off_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return RQ_ERR_CUDA;
     if (err != 0) {
-        // a call that gave up may have left its arrival counters part-way:
-        // clear them with the error word so that the next call starts clean
+        // A call whose bounded wait gave up still counts every CTA's arrival
+        // (consumers finish their pass over the data they have and reach the
+        // counter), so its counters return to zero; they are cleared here
+        // anyway, with the error word -- the cache's and the allocation-free
+        // entry point's -- so that the next call starts clean whatever
+        // happened.
         cudaMemset(c->base + c->lay.off_counters, 0, c->lay.off_err + sizeof(int) - c->lay.off_counters);
-        cudaDeviceSynchronize();
+        noalloc_reset_counters();
+        if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
         return RQ_ERR_TIMEOUT;
     }
     return RQ_OK;

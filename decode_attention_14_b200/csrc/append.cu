@@ -67,6 +67,14 @@ __device__ __forceinline__ void store_record(uint8_t *codes, uint8_t *meta, uint
     }
 }
 
+// Raise the stream's largest V scale byte (FP8 E4M3 scales are never
+// negative, and for non-negative E4M3 values the byte order is the value
+// order) to the record's largest.
+__device__ __forceinline__ void raise_vmax(int *slot, uint32_t s8, int lane) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, s8);
+    if (lane == 0) atomicMax(slot, (int)m);
+}
+
 __device__ __forceinline__ void load4_bf16(const uint16_t *p, double x[4]) {
     const uint2 raw = *reinterpret_cast<const uint2 *>(p);
     x[0] = (double)bf16_to_f32((uint16_t)(raw.x & 0xFFFF));
@@ -111,6 +119,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         uint8_t *ac = a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8);
         uint8_t *am = a.a_meta0 + kv * a.anchor_kv_stride + rec * meta_rec;
         store_record(ac, am, apack, s8, m8, a.ba, a.g, lane);
+        if (kv == 1) raise_vmax(a.vmax + ((size_t)a.nres * a.B + b) * a.H + h, s8, lane);
         return;
     }
 
@@ -149,6 +158,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     uint8_t *rc = a.r_codes0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * (kHeadDim * a.br / 8);
     uint8_t *rm = a.r_meta0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * meta_rec;
     store_record(rc, rm, rpack, s8, m8, a.br, a.g, lane);
+    if (kv == 1) raise_vmax(a.vmax + ((size_t)j * a.B + b) * a.H + h, s8, lane);
     if (lane == 0) {
         uint16_t *rf = reinterpret_cast<uint16_t *>(a.r_coef0 + j * a.resid_loop_stride + kv * a.resid_kv_stride);
         rf[rec] = __bfloat16_as_ushort(sb);

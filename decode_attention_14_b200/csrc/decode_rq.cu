@@ -20,14 +20,24 @@
 //    sum_i q_i c_i is three dp4a (4 products each) per 4 codes, exact;
 //  - values: each weight p_t s_t sc_{g,t} becomes fixed point with a
 //    power-of-two scale chosen from a bound of every weight of the chunk
-//    (max |s_t| x 448, the largest FP8 scale; mapped into [2^27, 2^28)),
+//    (max |s_t| of the chunk times the largest V scale the encoder has
+//    written to the (sequence, head) stream; mapped into [2^21, 2^22)),
 //    split into 16-bit halves; sum_t w_t c_t,i is two dp2a (2 products each)
 //    per 2 codes, exact.  The high halves are nonzero only for the largest
 //    weights, and skipped when a warp has none for a token pair.
 // The fixed-point rounding of q and of the weights is the only departure from
-// fp32 arithmetic (relative 2^-21 of max|q|; absolute 2^-27 of the bound:
-// below 1e-4 of the output on the synthetic workloads, 2e-4 with one
-// dominant key, against the 2e-3 parity bound).
+// fp32 arithmetic (relative 2^-21 of max|q|; absolute 2^-22 of the bound,
+// which follows the actual V scales, so small-magnitude V keeps its relative
+// precision).
+//
+// Programmatic launch.  The kernel may start while the previous kernel on
+// its stream is still running (the host launches it with programmatic stream
+// serialization): the producer streams committed records below a.stable --
+// which no in-flight work writes -- before its grid-dependency wait; every
+// other global access (q, the V scale bounds, records from a.stable on, the
+// tail, partials, counters, out) comes after the wait.  A thread signals
+// that the next kernel may start only after its own wait has returned, so at
+// most one earlier kernel is ever still running.
 // Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
 // Data movement.  Each CTA owns a chunk of one (sequence, kv head) (the
@@ -83,7 +93,10 @@ constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait
-constexpr int kWeightTop = 28;                          // V weights below 2^28 (fixed point)
+constexpr int kWeightTop = 22;                          // V weight bound in [2^21, 2^22) (fixed point)
+#ifndef RQ_DECODE_PDL
+#define RQ_DECODE_PDL 1
+#endif
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -134,6 +147,13 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+// Grid-dependency control (programmatic dependent launch): wait for the
+// previous kernel on the stream to complete (its writes visible), then allow
+// the next one to start.  Both are no-ops without a programmatic launch.
+__device__ __forceinline__ void griddep_wait_then_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
 
@@ -389,6 +409,17 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     if (warp == 4) {
         if (lane == 0) {
             const size_t tok0 = bh * a.Tp + (size_t)t0;
+            // records of tokens [.., tok_end) may be read before the grid
+            // dependency wait only if all of them lie below a.stable (padding
+            // beyond the sequence's length is read but never used)
+            bool waited = false;
+            auto dep = [&](int tok_end) {
+                if (!waited && t0 + tok_end > a.stable) {
+                    griddep_wait_then_release();
+                    waited = true;
+                }
+            };
+            dep(RESID && ntiles > 0 ? n : 0);
             if (RESID && ntiles > 0) {
                 mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
                 bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
@@ -432,6 +463,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         virt += P::RING - phys;
                         phys = 0;
                     }
+                    if (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING))
+                        dep(0x7FFFFFFF);   // about to block on the consumers, who run after their wait
+                    dep(min((j + 1) * kItem, n));
                     while (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING)) {
                         if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
                                                                     &s_abort)) {
@@ -483,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     phys += bytes;
                 }
             }
+            dep(0x7FFFFFFF);
             const int issued = it;
             // drain: every issued copy must have landed before the CTA exits
             // (the consumers stop waiting once the CTA has given up)
@@ -493,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // the other lanes: the bound max |s_hat(V)| of the chunk's V
             // coefficients (for the weights' fixed point), ready before the
             // softmax needs it
+            griddep_wait_then_release();
             unsigned m = 0;
             if (RESID && mbar_wait<64>(&bar_cf, 0, &s_abort)) {
                 const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING);
@@ -505,6 +541,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     }
 
     // ------------------------------------------------------------ consumers
+    griddep_wait_then_release();
+    // upper bounds of this stream's V scales (anchor; the loop's residual)
+    const float vA = e4m3_to_f32((uint32_t)a.vmax_a[bh]);
+    const float vR = RESID ? e4m3_to_f32((uint32_t)a.vmax_r[bh]) : 0.f;
     if (a.n_new > 0 && split == 0) {
         // fused append: this unit's new tail rows (K and V, 16-byte vectors);
         // the fence before the arrival count below publishes them to the
@@ -688,13 +728,14 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++)
         M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
     // the weights' fixed-point scales: w = P * sc (anchor) or p * sc
-    // (residual), |P| <= max|s_hat|, p <= 1, sc <= 448 (powers of two)
+    // (residual), |P| <= max|s_hat|, p <= 1, sc <= the stream's largest V
+    // scale (powers of two)
     if (!mbar_wait(&bar_cfmax, 0, &s_abort)) {
         s_abort = 1;
         atomicExch(a.err, 3);
     }
-    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax) * 448.f : 448.f, kWeightTop);
-    const float cR = fixed_scale(448.f, kWeightTop);
+    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax) * vA : vA, kWeightTop);
+    const float cR = fixed_scale(vR, kWeightTop);
     // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V
     // weight), zero beyond the chunk's tokens, stored with their scales
     float lsum[GK];
@@ -914,13 +955,12 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 
 template <int GK, int BA, int BR, int GS, bool RESID>
 cudaError_t configure() {
-    static bool configured = false;   // the largest dynamic shared memory any launch can ask for
-    if (configured) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Plan<BA, BR, GS, RESID>::smem(GK, kMaxChunk));
-    if (e == cudaSuccess) configured = true;
-    return e;
+    static bool done[kMaxDevices] = {};   // the largest dynamic shared memory any launch can ask for
+    return once_per_device(done, [] {
+        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)Plan<BA, BR, GS, RESID>::smem(GK, kMaxChunk));
+    });
 }
 
 template <int GK, int BA, int BR, int GS, bool RESID>
@@ -928,8 +968,18 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
     const dim3 grid(a.S, a.H, a.B * (a.G / GK));
     cudaError_t e = configure<GK, BA, BR, GS, RESID>();
     if (e != cudaSuccess) return e;
-    decode_rq_kernel<GK, BA, BR, GS, RESID>
-        <<<grid, kThreads, Plan<BA, BR, GS, RESID>::smem(GK, a.chunk), st>>>(a);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = Plan<BA, BR, GS, RESID>::smem(GK, a.chunk);
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = RQ_DECODE_PDL ? 1 : 0;
+    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, RESID>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -29,18 +29,17 @@ namespace {
 constexpr size_t kScratchFloats = size_t(2) << 20;   // 2 Mi floats = 8 MiB in all
 constexpr size_t kCounterInts = 65536;               // combine counters, at the end of the array
 constexpr size_t kPartialFloats = kScratchFloats - kCounterInts;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_decode_scratch[kScratchFloats];
 
 std::mutex g_setup_mutex;
-float *g_scratch_ptr[kMaxDevices] = {nullptr};
+float *g_scratch_ptr[rq::kMaxDevices] = {nullptr};
 
 // Device address of g_decode_scratch on the current device (resolved once).
 int scratch_for_current_device(float **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return RQ_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return RQ_ERR_UNSUPPORTED;
+    if (dev < 0 || dev >= rq::kMaxDevices) return RQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
     if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
@@ -62,9 +61,28 @@ int scratch_for_current_device(float **out) {
 
 }  // namespace
 
+namespace rq {
+void noalloc_reset_counters() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return;
+    }
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (g_scratch_ptr[dev]) cudaMemset(g_scratch_ptr[dev] + kPartialFloats, 0, kCounterInts * sizeof(int));
+}
+}  // namespace rq
+
 extern "C" int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
                                       float softmax_scale, void *stream) {
     if (!cache || !q_bf16 || !out) return RQ_ERR_INVALID;
+    // the scratch address is per device: the current device must be the cache's
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return RQ_ERR_CUDA;
+    }
+    if (dev != rq::cache_device(cache)) return RQ_ERR_INVALID;
     float *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);
     if (st != RQ_OK) return st;

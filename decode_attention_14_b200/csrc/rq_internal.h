@@ -17,7 +17,22 @@ constexpr int kTokTile = 64;        // padding granule of every token stream
 constexpr int kMaxSplits = 256;     // split-KV partitions per (b, kv head)
 constexpr int kMaxChunk = 1024;     // tokens per CTA (bounds the per-CTA shared-memory buffers)
 constexpr int kMaxBatch = 256;      // sequences per cache (their lengths travel in the launch arguments)
+constexpr int kMaxDevices = 64;     // devices a process may drive (per-device function attributes)
 constexpr size_t kAlign = 256;
+
+// Runs `set` (a cudaFuncSetAttribute call) once per device: function
+// attributes are per-device state.  `done` is the caller's static flag array.
+template <typename F>
+cudaError_t once_per_device(bool (&done)[kMaxDevices], F set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -58,6 +73,7 @@ struct Layout {
     size_t off_partials;         // float [B][Hq][splits_max][kPartialStride]
     size_t off_counters;         // int [B][H_kv]
     size_t off_err;              // int error word (+ pad)
+    size_t off_vmax;             // int [layers][groups][Lg][B][H_kv]: largest V scale byte per stream
     size_t total;
 };
 
@@ -84,6 +100,10 @@ struct AppendArgs {
     // residual records of loop j: r_*0 + j*resid_loop_stride + kv*resid_kv_stride
     uint8_t *r_codes0, *r_meta0, *r_coef0;
     size_t resid_loop_stride, resid_kv_stride;
+    // largest FP8 scale byte of each V stream of the group, [Lg][B][H]
+    // (record j < nres: residual of loop j; j = nres: the anchor), raised
+    // with atomicMax as records are written
+    int *vmax;
     SeqLens pos0;                              // first token position written, per sequence
     int B, H, n, Tp, tail_cap, nres;           // nres = Lg - 1
     int g, ba, br, rotate;
@@ -117,6 +137,15 @@ struct DecodeArgs {
     int *err;                 // device error word (bounded waits that gave up)
     float *out;               // [B][Hq][d] fp32
     const uint16_t *tail_k, *tail_v;   // [B][tail_cap][H][d] BF16 in-flight tokens, or null
+    // largest FP8 scale byte of the anchor V and (residual loops) the loop's
+    // residual V stream of every (sequence, kv head), [B][H]: upper bounds of
+    // the V scales, from which the weights' fixed point is chosen
+    const int *vmax_a, *vmax_r;
+    // committed records below token `stable` are not written by any work
+    // that may still run when this kernel starts (see the programmatic
+    // launch in api.cpp); records from `stable` on are read only after the
+    // kernel's grid-dependency wait
+    int stable;
     int n_tail, tail_cap;
     // fused append: n_new tokens [B][n_new][H][d] written to tail rows
     // tail_pos.. (included in n_tail) by split 0 of each unit before the combine
@@ -165,5 +194,13 @@ int decode_bf16_occupancy(int G, int chunk);
 // between calls.
 int decode_with_scratch(rq_cache *c, int layer, int loop, const void *q, float *out, float scale, void *stream,
                         float *partials, size_t partial_floats, int *counters, size_t max_units);
+
+// The device the cache's arena lives on.
+int cache_device(const rq_cache *c);
+
+// Zeroes the allocation-free entry point's combine counters on the current
+// device if that device's scratch address has been resolved (after a
+// bounded wait gave up; see rq_check).  Enqueued on the legacy stream.
+void noalloc_reset_counters();
 
 }  // namespace rq

@@ -12,8 +12,9 @@
  *
  * Conventions shared by every call:
  *   - All device pointers are CUDA global-memory pointers of the current
- *     device.  "stream" is a cudaStream_t passed as void* (NULL = the legacy
- *     default stream).  Work is enqueued asynchronously; no call
+ *     device, which must be the device the cache was created on (else
+ *     RQ_ERR_INVALID).  "stream" is a cudaStream_t passed as void* (NULL =
+ *     the legacy default stream).  Work is enqueued asynchronously; no call
  *     synchronises the host except rq_cache_create/destroy and
  *     rq_cache_export (which copies to host memory).
  *   - BF16 arrays hold IEEE bfloat16 bit patterns (uint16).
@@ -24,7 +25,9 @@
  *     stream, or order the streams.
  *   - Ownership: the caller owns q, k, v, out and (optionally) the cache's
  *     device arena; the library owns the host-side handle and, when it
- *     allocated the arena itself, the arena.
+ *     allocated the arena itself, the arena.  Once created, the arena is
+ *     written only by this library's calls (the decode kernel relies on it:
+ *     see rq_decode_attn).
  */
 #ifndef RQ_H
 #define RQ_H
@@ -160,6 +163,12 @@ int rq_append(rq_cache *cache, int layer, int loop, const void *k_bf16, const vo
  * Keys/values seen: the committed tokens of the loop's group (anchor loop:
  * the dequantized anchor; other loops: s_hat a_hat + R^T r_hat), followed by
  * the loop's BF16 tail tokens.  With no key at all the output is zero.
+ * Overlap: the kernel is launched so that it may start while the previous
+ * work on `stream` is still running (programmatic dependent launch).  Before
+ * that work has completed it reads only committed records that no append
+ * enqueued earlier can still be writing; q, the tail, out and everything else
+ * are touched only after it.  The observable results are those of plain
+ * stream order.
  * Errors: INVALID, STATE (wrong format), CUDA.
  */
 int rq_decode_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
@@ -213,7 +222,9 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
  * the caller.
  * Errors: INVALID (null pointer, n_tokens < 1, index out of range), STATE
  * (wrong format, or a sequence holds fewer than n_tokens tokens),
- * UNSUPPORTED (n_tokens > 65535), NOMEM, CUDA.
+ * UNSUPPORTED (n_tokens > 65535, or an INT2 anchor with INT4 residuals --
+ * the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4),
+ * NOMEM, CUDA.  UNSUPPORTED is returned before any allocation.
  */
 int rq_prefill_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, int n_tokens, float *out,
                     float softmax_scale, void *stream);
@@ -228,12 +239,16 @@ int rq_prefill_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, in
  *   inside a host framework that owns all device memory and offers no
  *   allocator, a serving loop whose memory is planned once, or work issued
  *   during stream capture, where allocation calls are refused.
- *   Limit: batch * num_q_heads * S * 132 floats must fit in 2^21 floats, S
- *   being the split count the call chooses (at most ceil(T/64)); beyond it the
- *   call returns RQ_ERR_CAPACITY and enqueues nothing.
- *   The first call on a device looks up the array's device address; make it
- *   before any stream capture.  All calls on a device share the array: calls
- *   whose GPU work overlaps race on it and must be ordered by the caller.
+ *   Limits: batch * num_q_heads * S * 132 floats must fit in 2^21 - 2^16
+ *   floats (the last 2^16 words of the array hold the combine counters), S
+ *   being the split count the call chooses (at most ceil(T/64)), and
+ *   batch * num_q_heads must not exceed 65536; beyond either the call returns
+ *   RQ_ERR_CAPACITY and enqueues nothing.
+ *   The first call on a device looks up the array's device address (and
+ *   zeroes its counters, synchronously); make it before any stream capture.
+ *   The current device must be the cache's (else RQ_ERR_INVALID).  All calls
+ *   on a device share the array: calls whose GPU work overlaps race on it and
+ *   must be ordered by the caller.
  *   Format must be RQ_FMT_RESIDUAL (else RQ_ERR_STATE).
  */
 int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
@@ -288,7 +303,9 @@ int rq_cache_export(const rq_cache *cache, int layer, int loop, void *host_codes
 size_t rq_decode_bytes(const rq_cache *cache, int layer, int loop);
 
 /* Reports asynchronous failures: RQ_ERR_TIMEOUT if a kernel's bounded wait
- * gave up, RQ_ERR_CUDA if the context holds a sticky error, else RQ_OK.
+ * gave up (the error word and the split-combine counters -- the cache's and
+ * rq_decode_attn_noalloc's on this device -- are then cleared, so later calls
+ * start clean), RQ_ERR_CUDA if the context holds a sticky error, else RQ_OK.
  * Synchronises the device. */
 int rq_check(rq_cache *cache);
 

@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 from oracle import oracle as orc
 
 REL_L2_TOL = 1e-3
@@ -67,17 +67,37 @@ def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, r
             if only_groups is not None and grp not in only_groups:
                 continue
             K, V = synth.group_kv(seed, layer, grp, Lg, sigma, B, T + n_tail, H, device="cuda")
-            bt.inputs[(layer, grp)] = (K, V)
-            for t0 in range(0, T, chunk):
-                t1 = min(T, t0 + chunk)
-                for j in range(Lg):
-                    loop = grp * Lg + j
-                    k = K[j][:, t0:t1].contiguous()
-                    v = V[j][:, t0:t1].contiguous()
-                    cache.append(layer, loop, k, v)
-            if n_tail and fmt == rq.RQ_FMT_RESIDUAL:
-                for j in range(Lg - 1):
-                    cache.append(layer, grp * Lg + j, K[j][:, T:].contiguous(), V[j][:, T:].contiguous())
+            fill_group(bt, layer, grp, K, V, chunk)
+    torch.cuda.synchronize()
+    return bt
+
+
+def fill_group(bt: Built, layer: int, grp: int, K, V, chunk: int = 128) -> None:
+    """Appends the given K/V of one loop group (lists of Lg BF16 CUDA tensors
+    [B][T + n_tail][H][d], index Lg - 1 the anchor): the first bt.T tokens
+    committed in chunks through the tails, the rest left in the tails."""
+    cache, T, Lg = bt.cache, bt.T, bt.cfg.loops_per_group
+    bt.inputs[(layer, grp)] = (K, V)
+    for t0 in range(0, T, chunk):
+        t1 = min(T, t0 + chunk)
+        for j in range(Lg):
+            cache.append(layer, grp * Lg + j, K[j][:, t0:t1].contiguous(), V[j][:, t0:t1].contiguous())
+    if bt.n_tail and bt.cfg.format == rq.RQ_FMT_RESIDUAL:
+        for j in range(Lg - 1):
+            cache.append(layer, grp * Lg + j, K[j][:, T:].contiguous(), V[j][:, T:].contiguous())
+
+
+def build_from(K, V, *, Hq: int, g=16, ba=4, br=2, rotate=True, T: int, n_tail=0, chunk=128,
+               seed=0) -> Built:
+    """A one-layer, one-group cache holding the given K/V (lists of Lg BF16
+    CUDA tensors [B][T + n_tail][H][d]; index Lg - 1 is the anchor)."""
+    Lg = len(K)
+    B, _, Hkv, _ = K[0].shape
+    cfg = rq.make_config(num_layers=1, num_loops=Lg, loops_per_group=Lg, batch=B, max_tokens=max(T, 1),
+                         max_tail_tokens=max(chunk, n_tail, 1), num_kv_heads=Hkv, num_q_heads=Hq, group_size=g,
+                         anchor_bits=ba, resid_bits=br, rotate=rotate, seed=0xA11CE)
+    bt = Built(rq.Cache(cfg), cfg, seed, T, n_tail)
+    fill_group(bt, 0, 0, K, V, chunk)
     torch.cuda.synchronize()
     return bt
 

@@ -21,7 +21,7 @@ import pytest
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 
 import rqharness as H
 
@@ -35,7 +35,7 @@ def _check(bt, groups, sel, loops_to_check=None):
         for kv in (0, 1):
             r = H.compare_records(bt, 0, grp, kv, sel)
             assert r["mismatch"] == 0, r
-            assert r["tolerated"] <= 1e-3 * r["compared"] + 4, r
+            assert r["tolerated"] == 0, r   # none on the synthetic workloads (reported when nonzero)
         loops = loops_to_check if loops_to_check is not None else range(grp * Lg, grp * Lg + Lg)
         for loop in loops:
             q = synth.queries(bt.seed, 0, loop, 0, cfg.batch, cfg.num_q_heads)

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 
 import rqharness as H
 

@@ -129,7 +129,7 @@ def test_study_on_synthetic_loops():
     seeded synthetic loop group (4 loops, H = 4, T = 256; loops at distance k
     from the last one carry noise 0.1 k on top of a scaled copy of it).
     Printed with -s; asserted: scaling beats none for both references."""
-    from decode_attention_14_b200 import synth
+    import synth
     rows = {}
     for kv in (0, 1):
         K, V = synth.group_kv(0x5EED0001, 0, 0, 4, (0.1, 0.2, 0.3), 1, 256, 4, device="cpu")

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 
 import rqharness as H
 
@@ -34,7 +34,7 @@ def _records_and_mse(bt, layer, grp, bh_sel=None):
         assert r["compared"] > 0
         # differences are only tolerated at flagged boundary values; they and
         # the records they exclude must stay rare
-        assert r["tolerated"] <= 1e-3 * r["compared"] + 4, r
+        assert r["tolerated"] == 0, r   # none on the synthetic workloads (reported when nonzero)
         assert r["excluded"] <= 1e-2 * r["compared"] + 64, r
         g, o = H.mse_check(bt, layer, grp, kv, bh_sel)
         assert abs(g / o - 1.0) <= H.MSE_REL_TOL, (kv, g, o)

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 from oracle import oracle as orc
 
 import rqharness as H

@@ -6,9 +6,10 @@ a serving loop whose memory is planned at start-up, or work issued while a
 stream is being captured.  For them the library keeps the split-combine
 scratch of this entry point in a fixed device array of its own (8 MiB per
 GPU).  This file checks, through the C ABI, that it returns what
-rq_decode_attn returns (within the parity tolerance) on two calls in a row,
-and that it refuses, without enqueuing work, a call whose scratch would not
-fit.  It is named to run last so that a failure here cannot hide the other
+rq_decode_attn (and the fp64 oracle) return (within the parity tolerance) on
+two calls in a row, that a call captured into a CUDA graph after a first
+eager call replays correctly, and that it refuses, without enqueuing work, a
+call whose scratch would not fit.  It is named to run last so that a failure here cannot hide the other
 tests' results.
 """
 import numpy as np
@@ -16,7 +17,7 @@ import pytest
 import torch
 
 import decode_attention_14_b200 as rq
-from decode_attention_14_b200 import synth
+import synth
 
 import rqharness as H
 
@@ -36,6 +37,7 @@ def test_noalloc_matches_rq_decode_attn_twice():
     for loop in (0, 2, 3):          # residual loops with BF16 tail tokens, and the anchor loop
         q = synth.queries(bt.seed, 0, loop, 0, cfg.batch, cfg.num_q_heads)
         ref = bt.cache.decode(0, loop, q)
+        orc_ref = H.oracle_decode(bt, 0, loop, q)
         for _ in range(2):
             out = torch.full_like(ref, float("nan"))
             st = rq.rq_decode_attn_noalloc(bt.cache.h, 0, loop, q, out)
@@ -43,6 +45,38 @@ def test_noalloc_matches_rq_decode_attn_twice():
             torch.cuda.synchronize()
             rel, mx = _errors(out, ref)
             assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (loop, rel, mx)
+            # and against the fp64 oracle over the same records
+            rel, mx = H.attn_errors(out.cpu().numpy(), orc_ref, cfg.num_q_heads // cfg.num_kv_heads)
+            assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (loop, rel, mx)
+    bt.cache.check()
+
+
+def test_noalloc_inside_stream_capture():
+    """After one eager call (which looks up the scratch address), a call
+    captured into a CUDA graph on a side stream allocates nothing and replays
+    with the same results, twice."""
+    bt = H.build(layers=1, loops=4, Lg=4, B=2, T=500, H=2, Hq=4, n_tail=1, seed=0x5EEDA100)
+    cfg = bt.cfg
+    loop = 1
+    q = synth.queries(bt.seed, 0, loop, 0, cfg.batch, cfg.num_q_heads)
+    ref = bt.cache.decode(0, loop, q)
+    out = torch.zeros_like(ref)
+    assert rq.rq_decode_attn_noalloc(bt.cache.h, 0, loop, q, out) == rq.RQ_OK
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            st = rq.rq_decode_attn_noalloc(bt.cache.h, 0, loop, q, out, 0.0, side)
+    assert st == rq.RQ_OK, rq.rq_status_string(st)
+    for _ in range(2):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        rel, mx = _errors(out, ref)
+        assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (rel, mx)
+    del g
     bt.cache.check()
 
 
