@@ -51,6 +51,8 @@ def lib():
         L.orc_splitmix64.argtypes = [ctypes.c_uint64]
         L.orc_rotation_signs.restype = None
         L.orc_rotation_signs.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+        L.orc_rotation_scale.restype = ctypes.c_double
+        L.orc_rotation_scale.argtypes = [ctypes.c_int, ctypes.c_int]
         L.orc_rotation_matrix.restype = None
         L.orc_rotation_matrix.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
         L.orc_quantize_group.restype = None
@@ -112,6 +114,11 @@ def rotation_signs(seed: int, d: int) -> np.ndarray:
     out = np.zeros(d, np.float64)
     lib().orc_rotation_signs(seed, d, _p(out))
     return out
+
+
+def rotation_scale(d: int, rotate: bool = True) -> float:
+    """The scalar c of R = c * H diag(sigma): 1/sqrt(d), correctly rounded."""
+    return float(lib().orc_rotation_scale(d, int(rotate)))
 
 
 def rotation_matrix(seed: int, d: int, rotate: bool = True) -> np.ndarray:

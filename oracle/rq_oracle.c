@@ -34,7 +34,9 @@
  *
  * Every function here is written from those definitions, step by step, in
  * fp64, with no blocking, fusion or reordering.  The rotation is applied as
- * an explicit O(d^2) matrix product (not a butterfly).
+ * an explicit O(d^2) matrix product (not a butterfly), in the factored form
+ * of its definition: the +-1 matrix H diag(sigma) times the vector (an exact
+ * signed sum for the cache's values), then the scalar 1/sqrt(d) once.
  *
  * Parity pins: see tests/test_oracle_pins.py (and tests/test_oracle_ablation.py
  * for orc_encode_ablation, the abstract's ablation variants: previous-loop
@@ -215,21 +217,71 @@ static int popcount_int(unsigned x)
     return c;
 }
 
-/* R[i*d + j]; rotate == 0 gives the identity. */
-ORC_EXPORT void orc_rotation_matrix(uint64_t seed, int d, int rotate, double *R)
+/* R = c * S with S = H_d diag(sigma) (entries +-1) and c = 1/sqrt(d) when
+ * rotating; S = I and c = 1 otherwise.  d is a power of two (Sylvester), so
+ * 1/sqrt(d) = 2^(-k/2) for d = 2^k: an exact power of two for even k, else
+ * sqrt(1/2) (correctly rounded by IEEE sqrt) times an exact power of two --
+ * the correctly rounded value either way. */
+ORC_EXPORT double orc_rotation_scale(int d, int rotate)
+{
+    int k = 0;
+    if (!rotate)
+        return 1.0;
+    while ((1 << k) < d)
+        k++;
+    return (k % 2) ? sqrt(0.5) * ldexp(1.0, -(k - 1) / 2) : ldexp(1.0, -k / 2);
+}
+
+/* S[i*d + j]: the +-1 matrix H_d diag(sigma), or the identity. */
+ORC_EXPORT void orc_rotation_signs_matrix(uint64_t seed, int d, int rotate, double *S)
 {
     int i, j;
     double *sigma = (double *)malloc(sizeof(double) * (size_t)d);
-    double inv = 1.0 / sqrt((double)d);
     orc_rotation_signs(seed, d, sigma);
     for (i = 0; i < d; i++)
         for (j = 0; j < d; j++) {
             if (!rotate)
-                R[i * d + j] = (i == j) ? 1.0 : 0.0;
+                S[i * d + j] = (i == j) ? 1.0 : 0.0;
             else
-                R[i * d + j] = ((popcount_int((unsigned)(i & j)) & 1) ? -1.0 : 1.0) * sigma[j] * inv;
+                S[i * d + j] = ((popcount_int((unsigned)(i & j)) & 1) ? -1.0 : 1.0) * sigma[j];
         }
     free(sigma);
+}
+
+/* R[i*d + j] = c * S[i*d + j]; rotate == 0 gives the identity. */
+ORC_EXPORT void orc_rotation_matrix(uint64_t seed, int d, int rotate, double *R)
+{
+    int i;
+    double c = orc_rotation_scale(d, rotate);
+    orc_rotation_signs_matrix(seed, d, rotate, R);
+    for (i = 0; i < d * d; i++)
+        R[i] *= c;
+}
+
+/* y = R v = c * (S v): the signed sum of S's +-1 entries times v first, then
+ * one multiplication by c.  For the cache's values (sums of a bounded number
+ * of binary digits) the signed sum is exact, so y carries a single rounding. */
+static void rotate_vec(const double *S, double c, int d, const double *v, double *y)
+{
+    int i, j;
+    for (i = 0; i < d; i++) {
+        double acc = 0.0;
+        for (j = 0; j < d; j++)
+            acc += S[i * d + j] * v[j];
+        y[i] = c * acc;
+    }
+}
+
+/* x = R^T v = c * (S^T v): (R^T v)_i = sum_j R_ji v_j. */
+static void rotate_back(const double *S, double c, int d, const double *v, double *x)
+{
+    int i, j;
+    for (i = 0; i < d; i++) {
+        double acc = 0.0;
+        for (j = 0; j < d; j++)
+            acc += S[j * d + i] * v[j];
+        x[i] = c * acc;
+    }
 }
 
 /* ------------------------------------------------------------------ */
@@ -364,16 +416,17 @@ ORC_EXPORT void orc_encode(int n, int L, int d, int g, int ba, int br, int rotat
                            uint8_t *a_eflag, uint8_t *a_mflag,
                            uint8_t *r_eflag, uint8_t *r_mflag, uint8_t *r_cflag)
 {
-    int t, l, i, j;
+    int t, l, i;
     int G = d / g;
     size_t ab = (size_t)(d * ba / 8), rb = (size_t)(d * br / 8);
-    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double c = orc_rotation_scale(d, rotate);
     double *xa = (double *)malloc(sizeof(double) * (size_t)d);
     double *ahat = (double *)malloc(sizeof(double) * (size_t)d);
     double *xl = (double *)malloc(sizeof(double) * (size_t)d);
     double *r = (double *)malloc(sizeof(double) * (size_t)d);
     double *y = (double *)malloc(sizeof(double) * (size_t)d);
-    orc_rotation_matrix(seed, d, rotate, R);
+    orc_rotation_signs_matrix(seed, d, rotate, S);
     for (t = 0; t < n; t++) {
         const uint16_t *xa_bits = x_bf16 + ((size_t)(L - 1) * n + t) * d;
         for (i = 0; i < d; i++)
@@ -403,18 +456,13 @@ ORC_EXPORT void orc_encode(int n, int L, int d, int g, int ba, int br, int rotat
                 r_cflag[rec] = (uint8_t)cnear;
             for (i = 0; i < d; i++)
                 r[i] = xl[i] - shat * ahat[i];
-            for (i = 0; i < d; i++) {
-                double acc = 0.0;
-                for (j = 0; j < d; j++)
-                    acc += R[i * d + j] * r[j];
-                y[i] = acc;
-            }
+            rotate_vec(S, c, d, r, y);
             quantize_record(y, d, g, br, r_codes + rec * rb, r_meta + rec * 2 * G,
                             r_eflag ? r_eflag + rec * d : NULL,
                             r_mflag ? r_mflag + rec * G : NULL);
         }
     }
-    free(R); free(xa); free(ahat); free(xl); free(r); free(y);
+    free(S); free(xa); free(ahat); free(xl); free(r); free(y);
 }
 
 /* ------------------------------------------------------------------ */
@@ -428,13 +476,15 @@ ORC_EXPORT void orc_reconstruct(int n, int L, int d, int g, int ba, int br, int 
                                 const uint8_t *r_codes, const uint8_t *r_meta, const uint16_t *r_coef,
                                 double *out)
 {
-    int t, l, i, j;
+    int t, l, i;
     int G = d / g;
     size_t ab = (size_t)(d * ba / 8), rb = (size_t)(d * br / 8);
-    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double c = orc_rotation_scale(d, rotate);
     double *ahat = (double *)malloc(sizeof(double) * (size_t)d);
     double *yhat = (double *)malloc(sizeof(double) * (size_t)d);
-    orc_rotation_matrix(seed, d, rotate, R);
+    double *back = (double *)malloc(sizeof(double) * (size_t)d);
+    orc_rotation_signs_matrix(seed, d, rotate, S);
     for (t = 0; t < n; t++) {
         orc_dequant(a_codes + (size_t)t * ab, a_meta + (size_t)t * 2 * G, d, g, ba, ahat);
         memcpy(out + ((size_t)(L - 1) * n + t) * d, ahat, sizeof(double) * (size_t)d);
@@ -443,15 +493,12 @@ ORC_EXPORT void orc_reconstruct(int n, int L, int d, int g, int ba, int br, int 
             double shat = orc_bf16_value(r_coef[rec]);
             double *o = out + rec * d;
             orc_dequant(r_codes + rec * rb, r_meta + rec * 2 * G, d, g, br, yhat);
-            for (i = 0; i < d; i++) {
-                double acc = 0.0;
-                for (j = 0; j < d; j++)
-                    acc += R[j * d + i] * yhat[j];  /* (R^T y)_i = sum_j R_ji y_j */
-                o[i] = shat * ahat[i] + acc;
-            }
+            rotate_back(S, c, d, yhat, back);
+            for (i = 0; i < d; i++)
+                o[i] = shat * ahat[i] + back[i];
         }
     }
-    free(R); free(ahat); free(yhat);
+    free(S); free(ahat); free(yhat); free(back);
 }
 
 /* ------------------------------------------------------------------ */
@@ -482,17 +529,19 @@ ORC_EXPORT void orc_encode_ablation(int n, int L, int d, int g, int ba, int br, 
                                     int anchor_mode, int scale_mode, const uint16_t *x_bf16,
                                     double *xhat, double *coef, int *reads)
 {
-    int t, l, i, j;
+    int t, l, i;
     int G = d / g;
-    double *R = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double c = orc_rotation_scale(d, rotate);
     double *x = (double *)malloc(sizeof(double) * (size_t)d);
     double *r = (double *)malloc(sizeof(double) * (size_t)d);
     double *y = (double *)malloc(sizeof(double) * (size_t)d);
     double *yhat = (double *)malloc(sizeof(double) * (size_t)d);
+    double *back = (double *)malloc(sizeof(double) * (size_t)d);
     uint8_t *packed = (uint8_t *)malloc((size_t)d);
     uint8_t *meta = (uint8_t *)malloc((size_t)(2 * G));
     const int first = anchor_mode == 0 ? L - 1 : 0;   /* the anchor loop */
-    orc_rotation_matrix(seed, d, rotate, R);
+    orc_rotation_signs_matrix(seed, d, rotate, S);
     for (l = 0; l < L; l++)
         reads[l] = l == first ? 1 : (anchor_mode == 0 ? 2 : l + 1);
     for (t = 0; t < n; t++) {
@@ -526,23 +575,15 @@ ORC_EXPORT void orc_encode_ablation(int n, int L, int d, int g, int ba, int br, 
             coef[(size_t)l * n + t] = shat;
             for (i = 0; i < d; i++)
                 r[i] = x[i] - shat * ref[i];
-            for (i = 0; i < d; i++) {
-                double acc = 0.0;
-                for (j = 0; j < d; j++)
-                    acc += R[i * d + j] * r[j];
-                y[i] = acc;
-            }
+            rotate_vec(S, c, d, r, y);
             quantize_record(y, d, g, br, packed, meta, NULL, NULL);
             orc_dequant(packed, meta, d, g, br, yhat);
-            for (i = 0; i < d; i++) {
-                double acc = 0.0;
-                for (j = 0; j < d; j++)
-                    acc += R[j * d + i] * yhat[j];
-                o[i] = shat * ref[i] + acc;
-            }
+            rotate_back(S, c, d, yhat, back);
+            for (i = 0; i < d; i++)
+                o[i] = shat * ref[i] + back[i];
         }
     }
-    free(R); free(x); free(r); free(y); free(yhat); free(packed); free(meta);
+    free(S); free(x); free(r); free(y); free(yhat); free(back); free(packed); free(meta);
 }
 
 /* ------------------------------------------------------------------ */

@@ -541,3 +541,17 @@ def test_encoded_records_quantize_the_rotated_residual():
             sh = orc.bf16_value(int(e.r_coef[l, t]))
             y = _fwht(sigma * (xf[l, t] - sh * ahat)) / math.sqrt(d)
             check(y, e.r_codes[l, t], e.r_meta[l, t], 2, e.r_eflag[l, t], e.r_mflag[l, t])
+
+
+def test_rotation_scale_is_correctly_rounded():
+    """1/sqrt(d) for d = 2^k is the double nearest the exact value (decimal
+    arithmetic at 60 digits), so the oracle's rotation carries one rounding,
+    as the definition R = H diag(sigma)/sqrt(d) does when applied in exact
+    arithmetic and rounded once."""
+    import decimal
+    decimal.getcontext().prec = 60
+    for k in range(0, 12):
+        d = 2 ** k
+        exact = decimal.Decimal(1) / decimal.Decimal(d).sqrt()
+        assert orc.rotation_scale(d) == float(exact), k
+    assert orc.rotation_scale(128, False) == 1.0
