@@ -153,7 +153,8 @@ def test_constant_groups_anchor():
     for X in (K, V):
         for grp in range(D // 16):
             sel = (np.arange(T + NTAIL) + grp) % 4 == 0
-            vals = rng.standard_normal((B, int(sel.sum()), HKV, 1))
+            # (the boolean index moves the token axis first: [tokens][B][H][16])
+            vals = rng.standard_normal((int(sel.sum()), B, HKV, 1))
             X[LG - 1, :, sel, :, grp * 16:(grp + 1) * 16] = np.round(vals * 8) / 8   # BF16-exact constants
     bt = build(K, V)
     check_records(bt, strict=True)
@@ -194,14 +195,14 @@ def test_constant_groups_residual_without_rotation():
 
 @pytest.mark.parametrize("scaled", ["K", "KV"])
 def test_beyond_fp8_range(scaled):
-    """Two channels x 1000 and x -700 (|x| up to thousands): minima below
+    """Two channels x 10^4 and x -7000 (|x| up to ~10^5): minima below
     -448 and ranges above 15 x 448 saturate.  Attention is checked when only
     K is scaled (V of thousands would put the output beyond what an absolute
     2e-3 bound can measure in fp32)."""
     K, V = synthetic(0x5EED0102)
     for X in ((K, V) if scaled == "KV" else (K,)):
-        X[..., 5] *= 1000.0
-        X[..., 77] *= -700.0
+        X[..., 5] *= 1.0e4
+        X[..., 77] *= -7.0e3
     bt = build(K, V)
     check_records(bt, strict=True)
     _, meta, _ = bt.cache.export(0, LG - 1)
