@@ -53,6 +53,11 @@ class rq_config(ctypes.Structure):
         ("rotate", ctypes.c_int32),
         ("format", ctypes.c_int32),
         ("seed", ctypes.c_uint64),
+        ("scale_mode", ctypes.c_int32),
+        ("anchor_mode", ctypes.c_int32),
+        ("rotation_per_layer", ctypes.c_int32),
+        ("block_tokens", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32),
     ]
 
 
@@ -120,13 +125,25 @@ def _ok(status: int, what: str) -> None:
         raise RQError(status, what)
 
 
+SCALE_LEAST_SQUARES, SCALE_NORM_RATIO, SCALE_NONE = 0, 1, 2
+ANCHOR_LAST, ANCHOR_CHAINED = 0, 1
+
+
 def make_config(*, num_layers: int, num_loops: int, loops_per_group: int, batch: int, max_tokens: int,
                 max_tail_tokens: int, num_kv_heads: int, num_q_heads: int, head_dim: int = HEAD_DIM,
                 group_size: int = 16, anchor_bits: int = 4, resid_bits: int = 2, rotate: bool = True,
-                format: int = RQ_FMT_RESIDUAL, seed: int = 0xA11CE) -> rq_config:
+                format: int = RQ_FMT_RESIDUAL, seed: int = 0xA11CE, scale_mode: int = SCALE_LEAST_SQUARES,
+                anchor_mode: int = ANCHOR_LAST, rotation_per_layer: bool = False, block_tokens: int = 0,
+                num_blocks: int = 0) -> rq_config:
     return rq_config(num_layers, num_loops, loops_per_group, batch, max_tokens, max_tail_tokens,
                      num_kv_heads, num_q_heads, head_dim, group_size, anchor_bits, resid_bits,
-                     int(bool(rotate)), format, seed)
+                     int(bool(rotate)), format, seed, scale_mode, anchor_mode, int(bool(rotation_per_layer)),
+                     block_tokens, num_blocks)
+
+
+def layer_seed(cfg: rq_config, layer: int) -> int:
+    """The rotation seed of a layer (seed + layer * 2^32 with per-layer rotations)."""
+    return (cfg.seed + (layer << 32 if cfg.rotation_per_layer else 0)) & ((1 << 64) - 1)
 
 
 # ------------------------------------------------------------ C-ABI mirrors

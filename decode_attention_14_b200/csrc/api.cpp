@@ -25,7 +25,7 @@ struct rq_cache {
     // (an anchor append) started at, over the sequences; records below it are
     // not touched by any append still in flight
     std::vector<int> wstart;
-    uint32_t sigma[4] = {0, 0, 0, 0};
+    std::vector<uint32_t> sigma;   // [layer][4]: sign bits of the layer's rotation
     // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
     int occ[2][kMaxChunk / kTokTile];
     // split partials of rq_prefill_attn, allocated on first use and grown on demand
@@ -44,7 +44,20 @@ uint64_t splitmix64(uint64_t x) {
     return z ^ (z >> 31);
 }
 
-bool is_anchor_loop(const Layout &L, int loop) { return (loop % L.Lg) == L.Lg - 1; }
+// The last loop of its group: its append commits the group's tokens (the
+// other loops keep theirs in BF16 tails until then).
+bool is_commit_loop(const Layout &L, int loop) { return (loop % L.Lg) == L.Lg - 1; }
+
+// The record a loop's own K/V is stored in: -1 the anchor record, else the
+// index of its residual record.  Last-loop reference: the commit loop is the
+// anchor and loop j < Lg - 1 is residual j.  Chained reference: loop 0 is
+// the anchor and loop j >= 1 is residual j - 1 (its reconstruction reads
+// the anchor and residuals 0 .. j - 1).
+int record_slot(const Layout &L, int loop) {
+    const int j = loop % L.Lg;
+    if (L.cfg.anchor_mode == 1) return j == 0 ? -1 : j - 1;
+    return j == L.Lg - 1 ? -1 : j;
+}
 
 uint8_t *group_base(const rq_cache *c, int layer, int group) {
     const Layout &L = c->lay;
@@ -227,6 +240,17 @@ int rq_config_check(const rq_config *c) {
     if (c->num_q_heads % c->num_kv_heads != 0) return RQ_ERR_INVALID;
     if (c->format != RQ_FMT_RESIDUAL && c->format != RQ_FMT_BF16) return RQ_ERR_INVALID;
     if (c->rotate != 0 && c->rotate != 1) return RQ_ERR_INVALID;
+    if (c->scale_mode < 0 || c->scale_mode > 2 || c->anchor_mode < 0 || c->anchor_mode > 1 ||
+        c->rotation_per_layer < 0 || c->rotation_per_layer > 1 || c->block_tokens < 0 || c->num_blocks < 0)
+        return RQ_ERR_INVALID;
+    if (c->block_tokens != 0) {
+        if (c->block_tokens != 128 && c->block_tokens != 256) return RQ_ERR_UNSUPPORTED;
+        if (c->format != RQ_FMT_RESIDUAL) return RQ_ERR_UNSUPPORTED;
+        if (c->num_blocks < 1) return RQ_ERR_INVALID;
+    } else if (c->num_blocks != 0) {
+        return RQ_ERR_INVALID;
+    }
+    if (c->format == RQ_FMT_BF16 && (c->scale_mode != 0 || c->anchor_mode != 0)) return RQ_ERR_INVALID;
     int G = c->num_q_heads / c->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return RQ_ERR_UNSUPPORTED;
     if (c->head_dim != kHeadDim) return RQ_ERR_UNSUPPORTED;
@@ -315,9 +339,13 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
         }
         cudaGetLastError();
     }
+    c->sigma.assign((size_t)cfg->num_layers * 4, 0u);
     if (cfg->rotate)
-        for (int j = 0; j < kHeadDim; j++)
-            if (splitmix64(cfg->seed + (uint64_t)j) >> 63) c->sigma[j / 32] |= 1u << (j % 32);
+        for (int layer = 0; layer < cfg->num_layers; layer++) {
+            const uint64_t seed = cfg->seed + (cfg->rotation_per_layer ? (uint64_t)layer << 32 : 0);
+            for (int j = 0; j < kHeadDim; j++)
+                if (splitmix64(seed + (uint64_t)j) >> 63) c->sigma[(size_t)layer * 4 + j / 32] |= 1u << (j % 32);
+        }
     *out = c;
     return RQ_OK;
 }
@@ -360,7 +388,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     }
     const int group = loop / L.Lg, j = loop % L.Lg;
     const size_t slot = (size_t)layer * L.groups + group;
-    if (!is_anchor_loop(L, loop)) {
+    if (!is_commit_loop(L, loop)) {
         int &nt = c->ntail[(size_t)layer * cfg.num_loops + loop];
         if (nt + n > L.tail_cap) return RQ_ERR_CAPACITY;
         TailArgs a;
@@ -410,7 +438,9 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     a.ba = cfg.anchor_bits;
     a.br = cfg.resid_bits;
     a.rotate = cfg.rotate;
-    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    a.scale_mode = cfg.scale_mode;
+    a.chained = cfg.anchor_mode;
+    std::memcpy(a.sigma, &c->sigma[(size_t)layer * 4], sizeof(a.sigma));
     int s = cuda_status(launch_append(a, st));
     if (s != RQ_OK) return s;
     int w0 = 0x7FFFFFFF;
@@ -453,7 +483,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
     a.rotate = cfg.rotate;
     a.tail_cap = L.tail_cap;
-    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    std::memcpy(a.sigma, &c->sigma[(size_t)layer * 4], sizeof(a.sigma));
     bool resid = false;
     if (bf16) {
         a.T = c->len[(size_t)layer * cfg.num_loops + loop];
@@ -470,17 +500,21 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
         a.vmax_a = vmax_ptr(c, layer, group, L.Lg - 1);
         a.stable = c->wstart[(size_t)layer * L.groups + group];
-        if (!is_anchor_loop(L, loop)) {
-            resid = true;
-            a.vmax_r = vmax_ptr(c, layer, group, j);
-            for (int kv = 0; kv < 2; kv++) {
-                a.r_codes[kv] = resid_codes(c, layer, group, j, kv);
-                a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
-                a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, j, kv);
-            }
+        if (!is_commit_loop(L, loop)) {
             a.n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
             a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
             a.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
+        }
+        const int slot = record_slot(L, loop);
+        if (slot >= 0) {
+            if (cfg.anchor_mode == 1) return RQ_ERR_UNSUPPORTED;   // chained reference: rq_decode_attn_chain
+            resid = true;
+            a.vmax_r = vmax_ptr(c, layer, group, slot);
+            for (int kv = 0; kv < 2; kv++) {
+                a.r_codes[kv] = resid_codes(c, layer, group, slot, kv);
+                a.r_meta[kv] = resid_meta(c, layer, group, slot, kv);
+                a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, slot, kv);
+            }
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
@@ -495,7 +529,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     if (app_k) {
         // one launch when the loop keeps the tokens in its tail and the split
         // kernel runs (it writes the rows, then merges them); else append first
-        if (!(resid && a.S > 0)) {
+        if (!(!bf16 && !is_commit_loop(L, loop) && a.S > 0)) {
             int s = rq_append(c, layer, loop, app_k, app_v, app_n, stream);
             if (s != RQ_OK) return s;
             return decode_common(c, layer, loop, q, out, scale, stream, bf16);
@@ -578,8 +612,10 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
     const rq_config &cfg = L.cfg;
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
     if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
-    // the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4
+    // the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4,
+    // the last-loop reference and contiguous records
     if (cfg.anchor_bits == 2 && cfg.resid_bits == 4) return RQ_ERR_UNSUPPORTED;
+    if (cfg.anchor_mode != 0 || cfg.block_tokens != 0) return RQ_ERR_UNSUPPORTED;
     PrefillArgs a;
     std::memset(&a, 0, sizeof(a));
     const int group = loop / L.Lg, j = loop % L.Lg;
@@ -590,7 +626,7 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
         a.a_codes[kv] = anchor_codes(c, layer, group, kv);
         a.a_meta[kv] = anchor_meta(c, layer, group, kv);
     }
-    if (!is_anchor_loop(L, loop)) {
+    if (!is_commit_loop(L, loop)) {
         for (int kv = 0; kv < 2; kv++) {
             a.r_codes[kv] = resid_codes(c, layer, group, j, kv);
             a.r_meta[kv] = resid_meta(c, layer, group, j, kv);
@@ -615,7 +651,7 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
     a.g = cfg.group_size;
     a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
     a.rotate = cfg.rotate;
-    std::memcpy(a.sigma, c->sigma, sizeof(a.sigma));
+    std::memcpy(a.sigma, &c->sigma[(size_t)layer * 4], sizeof(a.sigma));
     if (n > 65535) return RQ_ERR_UNSUPPORTED;   // grid limit
     prefill_plan(&a, T, cfg.anchor_bits, cfg.resid_bits, c->sms);
     if ((long)a.B * a.nqb > 65535) return RQ_ERR_UNSUPPORTED;
@@ -709,8 +745,8 @@ int rq_cache_export(const rq_cache *c, int layer, int loop, void *host_codes, vo
     const rq_config &cfg = L.cfg;
     if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
-    const int group = loop / L.Lg, j = loop % L.Lg;
-    const bool anchor = is_anchor_loop(L, loop);
+    const int group = loop / L.Lg, j = record_slot(L, loop);
+    const bool anchor = j < 0;
     if (!anchor && !host_coef) return RQ_ERR_INVALID;
     const int len = c->len[(size_t)layer * L.groups + group];
     const size_t bh = (size_t)cfg.batch * cfg.num_kv_heads;
@@ -755,10 +791,13 @@ size_t rq_decode_bytes(const rq_cache *c, int layer, int loop) {
     const size_t T = tokens((size_t)layer * L.groups + group);
     size_t per = 2 * (size_t)(L.rec.a_codes + L.rec.meta);
     size_t tail = 0;
-    if (!is_anchor_loop(L, loop)) {
-        per += 2 * (size_t)(L.rec.r_codes + L.rec.meta + 2);
+    // residual records read: the loop's own (last-loop reference) or all up
+    // to its own (chained reference)
+    const int slot = record_slot(L, loop);
+    const int nres = slot < 0 ? 0 : cfg.anchor_mode == 1 ? slot + 1 : 1;
+    per += 2 * (size_t)nres * (L.rec.r_codes + L.rec.meta + 2);
+    if (!is_commit_loop(L, loop))
         tail = (size_t)c->ntail[(size_t)layer * cfg.num_loops + loop] * bh * 2 * kHeadDim * 2;
-    }
     return T * cfg.num_kv_heads * per + tail + qo;
 }
 

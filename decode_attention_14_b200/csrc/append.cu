@@ -89,6 +89,77 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
+// The residual record j of one token-head against the reference ref (the
+// dequantized anchor, or in the chained reference the previous loop's
+// reconstruction): coefficient s (least squares <x, ref>/<ref, ref>, norm
+// ratio |x|/|ref|, or 1; 0 when ref = 0 in the first two), stored in BF16;
+// residual x - s_hat ref with the stored coefficient; y = R r =
+// H (sigma . r) / sqrt(d); y quantized at resid_bits.  If next != nullptr it
+// receives the reconstruction s_hat ref + R^T y_hat.
+__device__ __forceinline__ void encode_residual(const AppendArgs &a, const double xl[4], const double ref[4],
+                                                int j, int kv, int b, int h, size_t rec, int lane,
+                                                double next[4]) {
+    double rr = 0.0, xr = 0.0, xx = 0.0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        rr = __dadd_rn(rr, __dmul_rn(ref[k], ref[k]));
+        xr = __dadd_rn(xr, __dmul_rn(xl[k], ref[k]));
+        xx = __dadd_rn(xx, __dmul_rn(xl[k], xl[k]));
+    }
+    const double den = warp_sum(rr);
+    const double num = warp_sum(xr);
+    double s;
+    if (a.scale_mode == 2) {
+        s = 1.0;
+    } else if (den == 0.0) {
+        s = 0.0;
+    } else if (a.scale_mode == 0) {
+        s = __ddiv_rn(num, den);
+    } else {
+        s = __ddiv_rn(__dsqrt_rn(warp_sum(xx)), __dsqrt_rn(den));
+    }
+    const __nv_bfloat16 sb = __double2bfloat16(s);
+    const double sh = (double)__bfloat162float(sb);
+    double y[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        double r = __dsub_rn(xl[k], __dmul_rn(sh, ref[k]));
+        if (a.rotate && sigma_neg(a.sigma, lane * 4 + k)) r = -r;
+        y[k] = r;
+    }
+    if (a.rotate) {
+        wht128_warp<double>(y, lane);
+#pragma unroll
+        for (int k = 0; k < 4; k++) y[k] = __dmul_rn(y[k], kInvSqrt128);
+    }
+    double yhat[4];
+    uint32_t s8, m8;
+    const uint32_t rpack = quantize4(y, a.br, a.g, lane, yhat, &s8, &m8);
+    const int meta_rec = 2 * (kHeadDim / a.g);
+    uint8_t *rc = a.r_codes0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * (kHeadDim * a.br / 8);
+    uint8_t *rm = a.r_meta0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * meta_rec;
+    store_record(rc, rm, rpack, s8, m8, a.br, a.g, lane);
+    if (kv == 1) raise_vmax(a.vmax + ((size_t)j * a.B + b) * a.H + h, s8, lane);
+    if (lane == 0) {
+        uint16_t *rf = reinterpret_cast<uint16_t *>(a.r_coef0 + j * a.resid_loop_stride + kv * a.resid_kv_stride);
+        rf[rec] = __bfloat16_as_ushort(sb);
+    }
+    if (next) {
+        // R^T y_hat = sigma . (H y_hat) / sqrt(d), then s_hat ref + that
+        double back[4] = {yhat[0], yhat[1], yhat[2], yhat[3]};
+        if (a.rotate) {
+            wht128_warp<double>(back, lane);
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                back[k] = __dmul_rn(back[k], kInvSqrt128);
+                if (sigma_neg(a.sigma, lane * 4 + k)) back[k] = -back[k];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; k++) next[k] = __dadd_rn(__dmul_rn(sh, ref[k]), back[k]);
+    }
+}
+
 // One warp per record: (K|V, sequence, token, kv head, j), j < nres the
 // residual of loop j, j == nres the anchor.  Every warp re-derives the anchor
 // (a few fp64 operations) so that the records of one token are encoded in
@@ -123,45 +194,52 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
         return;
     }
 
-    double aa = 0.0;
-#pragma unroll
-    for (int k = 0; k < 4; k++) aa = __dadd_rn(aa, __dmul_rn(ahat[k], ahat[k]));
-    const double den = warp_sum(aa);
-
     const uint16_t *tail = reinterpret_cast<const uint16_t *>(a.tail0 + j * a.tail_loop_stride +
                                                                kv * a.tail_kv_stride);
     double xl[4];
     load4_bf16(tail + (((size_t)b * a.tail_cap + t) * a.H + h) * kHeadDim + lane * 4, xl);
-    // least-squares coefficient against the dequantized anchor, stored in BF16
-    double xa = 0.0;
-#pragma unroll
-    for (int k = 0; k < 4; k++) xa = __dadd_rn(xa, __dmul_rn(xl[k], ahat[k]));
-    const double num = warp_sum(xa);
-    const double s = (den != 0.0) ? __ddiv_rn(num, den) : 0.0;
-    const __nv_bfloat16 sb = __double2bfloat16(s);
-    const double sh = (double)__bfloat162float(sb);
-    // residual with the stored coefficient, then y = R r = H (sigma . r) / sqrt(d)
-    double y[4];
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-        double rr = __dsub_rn(xl[k], __dmul_rn(sh, ahat[k]));
-        if (a.rotate && sigma_neg(a.sigma, lane * 4 + k)) rr = -rr;
-        y[k] = rr;
-    }
-    if (a.rotate) {
-        wht128_warp<double>(y, lane);
-#pragma unroll
-        for (int k = 0; k < 4; k++) y[k] = __dmul_rn(y[k], kInvSqrt128);
-    }
-    double yhat[4];
-    const uint32_t rpack = quantize4(y, a.br, a.g, lane, yhat, &s8, &m8);
-    uint8_t *rc = a.r_codes0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * (kHeadDim * a.br / 8);
-    uint8_t *rm = a.r_meta0 + j * a.resid_loop_stride + kv * a.resid_kv_stride + rec * meta_rec;
-    store_record(rc, rm, rpack, s8, m8, a.br, a.g, lane);
-    if (kv == 1) raise_vmax(a.vmax + ((size_t)j * a.B + b) * a.H + h, s8, lane);
-    if (lane == 0) {
-        uint16_t *rf = reinterpret_cast<uint16_t *>(a.r_coef0 + j * a.resid_loop_stride + kv * a.resid_kv_stride);
-        rf[rec] = __bfloat16_as_ushort(sb);
+    encode_residual(a, xl, ahat, j, kv, b, h, rec, lane, nullptr);
+}
+
+// One token-head's records in the chained (previous-loop) reference: loop 0
+// is quantized at anchor_bits into the anchor record; loop l >= 1 is encoded
+// as a residual (record l - 1) against the reconstruction of loop l - 1,
+// which then becomes the reference of loop l + 1.  One warp per (K|V,
+// sequence, token, kv head): the chain is sequential.
+__global__ void __launch_bounds__(128) append_chain_kernel(const AppendArgs a) {
+    const int lane = threadIdx.x & 31;
+    const long long wid = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    const long long total = 2LL * a.B * a.n * a.H;
+    if (wid >= total) return;   // uniform per warp
+    long long r = wid;
+    const int h = (int)(r % a.H);
+    r /= a.H;
+    const int t = (int)(r % a.n);
+    r /= a.n;
+    const int b = (int)(r % a.B);
+    const int kv = (int)(r / a.B);
+    const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0.v[b] + t);
+    const int meta_rec = 2 * (kHeadDim / a.g);
+    // loop l's input: the tails hold loops 0 .. nres-1, the call's input the last loop
+    auto load_loop = [&](int l, double v[4]) {
+        if (l == a.nres) {
+            load4_bf16(a.x_anchor[kv] + (((size_t)b * a.n + t) * a.H + h) * kHeadDim + lane * 4, v);
+        } else {
+            const uint16_t *tail =
+                reinterpret_cast<const uint16_t *>(a.tail0 + l * a.tail_loop_stride + kv * a.tail_kv_stride);
+            load4_bf16(tail + (((size_t)b * a.tail_cap + t) * a.H + h) * kHeadDim + lane * 4, v);
+        }
+    };
+    double x[4], ref[4];
+    load_loop(0, x);
+    uint32_t s8, m8;
+    const uint32_t apack = quantize4(x, a.ba, a.g, lane, ref, &s8, &m8);
+    store_record(a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8),
+                 a.a_meta0 + kv * a.anchor_kv_stride + rec * meta_rec, apack, s8, m8, a.ba, a.g, lane);
+    if (kv == 1) raise_vmax(a.vmax + ((size_t)a.nres * a.B + b) * a.H + h, s8, lane);
+    for (int l = 1; l <= a.nres; l++) {
+        load_loop(l, x);
+        encode_residual(a, x, ref, l - 1, kv, b, h, rec, lane, ref);   // ref becomes x_hat_l
     }
 }
 
@@ -203,10 +281,13 @@ __global__ void bf16_store_kernel(const Bf16StoreArgs a) {
 }  // namespace
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st) {
-    const long long warps = 2LL * a.B * a.n * a.H * (a.nres + 1);
+    const long long warps = 2LL * a.B * a.n * a.H * (a.chained ? 1 : a.nres + 1);
     const long long blocks = (warps + 3) / 4;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-    append_kernel<<<(unsigned)blocks, 128, 0, st>>>(a);
+    if (a.chained)
+        append_chain_kernel<<<(unsigned)blocks, 128, 0, st>>>(a);
+    else
+        append_kernel<<<(unsigned)blocks, 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 

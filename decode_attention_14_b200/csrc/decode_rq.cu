@@ -81,19 +81,16 @@ constexpr int kItem = kTile * kItemTiles;          // tokens per ring item
 #define RQ_DECODE_PRODUCER_SLEEP_NS 0
 #endif
 #ifndef RQ_DECODE_RING_BYTES
-#define RQ_DECODE_RING_BYTES 36864
+#define RQ_DECODE_RING_BYTES 39936
 #endif
-// consumer warp-groups per CTA (one query head per CTA; two per CTA)
-#ifndef RQ_DECODE_NWG1
-#define RQ_DECODE_NWG1 4
+#ifndef RQ_DECODE_MIN_CTAS
+#define RQ_DECODE_MIN_CTAS 4
 #endif
-#ifndef RQ_DECODE_NWG2
-#define RQ_DECODE_NWG2 3
-#endif
-constexpr int kRingBytes = RQ_DECODE_RING_BYTES;   // byte ring of one warp-group (multiple of 128)
-constexpr int kSlots = 16;                         // mbarrier pairs per warp-group: at most 16 items in flight
+constexpr int kRingBytes = RQ_DECODE_RING_BYTES;   // byte ring of one CTA (multiple of 128)
+constexpr int kSlots = 16;                         // mbarrier pairs: at most 16 items in flight
 static_assert(kRingBytes % 128 == 0, "ring must be a multiple of 128 bytes");
-constexpr int kConsumers = 128;                    // threads of one consumer warp-group
+constexpr int kConsumers = 128;
+constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait
 constexpr int kWeightTop = 22;                          // V weight bound in [2^21, 2^22) (fixed point)
@@ -158,12 +155,10 @@ __device__ __forceinline__ void griddep_wait_then_release() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
-// Barrier over the 128 threads of consumer warp-group wg (named barrier 1 + wg).
-__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, %1;" ::"r"(1 + wg), "n"(kConsumers) : "memory"); }
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
 
-struct WgSync {
-    int wg;
-    __device__ __forceinline__ void operator()() const { wg_sync(wg); }
+struct ConsumerSync {
+    __device__ __forceinline__ void operator()() const { consumer_sync(); }
 };
 
 // ---------------------------------------------------------------- codes
@@ -362,233 +357,190 @@ struct Plan {
     }
     // then: V coefficients [chunk] (RESID), logits/p [GK][chunk], p*s_hat [GK][chunk]
     __host__ __device__ static int coef_bytes(int chunk) { return RESID ? (chunk * 2 + 127) / 128 * 128 : 0; }
-    // dynamic shared memory of one warp-group (a multiple of 128 bytes)
-    __host__ __device__ static size_t wg_smem(int GK, int chunk) {
-        return ((size_t)RING + coef_bytes(chunk) + (size_t)2 * GK * chunk * sizeof(float) + 127) / 128 * 128;
+    __host__ __device__ static size_t smem(int GK, int chunk) {
+        return (size_t)RING + coef_bytes(chunk) + (size_t)2 * GK * chunk * sizeof(float);
     }
 };
 
-// Chunk c of the call: split c % S of unit c / S, unit = (sequence, kv head,
-// pair of query heads) in that order (split fastest).
-struct Chunk {
-    int b, h, pair, split, t0, n, ntiles, nitems;
-    size_t bh;
-};
-
-__device__ __forceinline__ Chunk chunk_of(const DecodeArgs &a, int c, int npairs) {
-    Chunk k;
-    k.split = c % a.S;
-    const int u = c / a.S;
-    k.h = u % a.H;
-    const int bz = u / a.H;
-    k.b = bz / npairs;
-    k.pair = bz % npairs;
-    split_range(k.split, a.S, a.seqT.v[k.b], &k.t0, &k.n);
-    k.ntiles = (k.n + kTile - 1) / kTile;
-    k.nitems = (k.ntiles + kItemTiles - 1) / kItemTiles;
-    k.bh = (size_t)k.b * a.H + k.h;
-    return k;
-}
-
-template <int GK, int NWG>
-constexpr int min_ctas() {
-    return NWG == 1 ? (GK == 1 ? 4 : 3) : NWG == 2 ? (GK == 1 ? 2 : 1) : 1;
-}
-
-// NWG consumer warp-groups (4 warps each) and one producer warp per CTA.
-// Warp-group w works on chunk blockIdx.x * NWG + w; the producer fills the
-// warp-groups' rings round-robin, item by item, so the chunks of a CTA
-// advance together and finish together (co-resident CTAs, by contrast, are
-// scheduled unevenly: the last one to arrive on an SM would finish alone).
-template <int GK, int BA, int BR, int GS, bool RESID, int NWG>
-__global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
-    decode_rq_kernel(const DecodeArgs a) {
+template <int GK, int BA, int BR, int GS, bool RESID>
+__global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) decode_rq_kernel(const DecodeArgs a) {
     using P = Plan<BA, BR, GS, RESID>;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bar_full[NWG][kSlots];
-    __shared__ __align__(8) uint64_t bar_empty[NWG][kSlots];
-    __shared__ __align__(8) uint64_t bar_cf[NWG];
-    __shared__ __align__(8) uint64_t bar_cfmax[NWG];   // the chunk's max |s_hat(V)| is known
-    __shared__ int s_start[NWG][kSlots];               // producer: virtual ring start of the item in each slot
-    __shared__ int s_abort;
-    __shared__ int s_last[NWG];
-    __shared__ unsigned s_cfmax[NWG];
-    __shared__ float s_q[NWG][GK][2][kHeadDim];
-    __shared__ __align__(16) uint8_t s_qp[NWG][GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
-    __shared__ int s_qsum[NWG][GK][2][8];                             // sum of each segment's fixed-point q
-    __shared__ float s_red[NWG][4][2 * GK + 2];
-    __shared__ __align__(16) float s_acc[NWG][4][GK][2][kHeadDim];
+    __shared__ __align__(8) uint64_t bar_full[kSlots];
+    __shared__ __align__(8) uint64_t bar_empty[kSlots];
+    __shared__ __align__(8) uint64_t bar_cf;
+    __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
+    __shared__ int s_abort, s_last;
+    __shared__ unsigned s_cfmax;
+    __shared__ float s_q[GK][2][kHeadDim];
+    __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
+    __shared__ int s_qsum[GK][2][8];                             // sum of each segment's fixed-point q
+    __shared__ float s_red[4][2 * GK + 2];
+    __shared__ __align__(16) float s_acc[4][GK][2][kHeadDim];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, h = blockIdx.y;
     const int npairs = a.G / GK;
-    const int nchunks = a.S * a.H * a.B * npairs;
-    const size_t wg_bytes = P::wg_smem(GK, a.chunk);
+    const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
+    const int hq0 = h * a.G + pair * GK;
+    int t0, n;   // this split's tokens of its sequence (none when the sequence is short)
+    split_range(split, a.S, a.seqT.v[b], &t0, &n);
+    const int ntiles = (n + kTile - 1) / kTile;
+    const size_t bh = (size_t)b * a.H + h;
+    uint8_t *ring = smem;
+    const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);        // V coefficients
+    float *s_sc = reinterpret_cast<float *>(smem + P::RING + P::coef_bytes(a.chunk));  // [GK][chunk] logits -> p
+    float *s_P = s_sc + GK * a.chunk;                                                  // [GK][chunk] p * s_hat
 
     if (tid == 0) {
-        for (int w = 0; w < NWG; w++) {
-            for (int i = 0; i < kSlots; i++) {
-                mbar_init(&bar_full[w][i], 1);
-                mbar_init(&bar_empty[w][i], kConsumers);   // every consumer thread of the group arrives
-            }
-            mbar_init(&bar_cf[w], 1);
-            mbar_init(&bar_cfmax[w], 31);
-            s_cfmax[w] = 0;
+        for (int i = 0; i < kSlots; i++) {
+            mbar_init(&bar_full[i], 1);
+            mbar_init(&bar_empty[i], kConsumers);   // every consumer thread arrives
         }
+        mbar_init(&bar_cf, 1);
+        mbar_init(&bar_cfmax, 31);
         s_abort = 0;
+        s_cfmax = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
     // ------------------------------------------------------------ producer
-    if (warp == 4 * NWG) {
+    if (warp == 4) {
         if (lane == 0) {
-            // records of tokens [.., tok_end) of a chunk may be read before the
-            // grid dependency wait only if all of them lie below a.stable
-            // (padding beyond the sequence's length is read but never used)
+            const size_t tok0 = bh * a.Tp + (size_t)t0;
+            // records of tokens [.., tok_end) may be read before the grid
+            // dependency wait only if all of them lie below a.stable (padding
+            // beyond the sequence's length is read but never used)
             bool waited = false;
-            auto dep = [&](int t0, int tok_end) {
+            auto dep = [&](int tok_end) {
                 if (!waited && t0 + tok_end > a.stable) {
                     griddep_wait_then_release();
                     waited = true;
                 }
             };
-            Chunk ck[NWG];
-            int it[NWG], virt[NWG], phys[NWG], rel[NWG], pass[NWG], jj[NWG];
-            const int npass = RESID ? 3 : 2;
-#pragma unroll
-            for (int w = 0; w < NWG; w++) {
-                const int c = blockIdx.x * NWG + w;
-                ck[w] = chunk_of(a, c < nchunks ? c : 0, npairs);
-                if (c >= nchunks) ck[w].ntiles = ck[w].nitems = 0;
-                it[w] = virt[w] = phys[w] = rel[w] = jj[w] = 0;
-                pass[w] = (c < nchunks && ck[w].nitems > 0) ? 0 : npass;   // nothing to stream
-                if (c < nchunks && RESID) {
-                    if (ck[w].ntiles > 0) {
-                        dep(ck[w].t0, ck[w].n);
-                        const uint32_t bytes = (uint32_t)(ck[w].ntiles * kTile * 2);
-                        mbar_expect_tx(&bar_cf[w], bytes);
-                        bulk_g2s(smem + w * wg_bytes + P::RING, a.r_coef[1] + ck[w].bh * a.Tp + ck[w].t0, bytes,
-                                 &bar_cf[w]);
-                    } else {
-                        mbar_arrive(&bar_cf[w]);   // nothing to fetch
-                    }
-                }
+            dep(RESID && ntiles > 0 ? n : 0);
+            if (RESID && ntiles > 0) {
+                mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
+                bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
+            } else if (RESID) {
+                mbar_arrive(&bar_cf);   // nothing to fetch
             }
-            // Items of a group, in order: K items, anchor V items, residual V
-            // items.  Item `it` occupies [virt, virt + bytes) of an unbounded
-            // virtual byte sequence, padded so that no item straddles the
-            // ring's end; its ring offset is phys = virt mod RING.  Before it is
-            // issued, every older item starting below virt + bytes - RING must
-            // have been released, and at most kSlots items may be outstanding.
-            // One item per group per round.
-            bool ok = true, more = true;
-            while (more && ok) {
-                more = false;
-#pragma unroll
-                for (int w = 0; w < NWG; w++) {
-                    if (pass[w] >= npass || !ok) continue;
-                    more = true;
-                    const Chunk &k = ck[w];
-                    const int bytes = P::item_bytes(pass[w]);
-                    if (phys[w] + bytes > P::RING) {
-                        virt[w] += P::RING - phys[w];
-                        phys[w] = 0;
+            // Items in order: K items, anchor V items, residual V items.  Item it
+            // occupies [virt, virt + bytes) of an unbounded virtual byte
+            // sequence, padded so that no item straddles the ring's end; its
+            // ring offset is phys = virt mod RING.  Before it is issued, every
+            // older item starting below virt + bytes - RING must have been
+            // released, and at most kSlots items may be outstanding.  The
+            // loop keeps all of this in running counters (no division).
+            const int npass = RESID ? 3 : 2;
+            int it = 0, virt = 0, phys = 0;
+            const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // items per pass
+            int rel = 0, vrel = 0, rphys = 0, ritem = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
+            bool ok = true;
+            for (int pass = 0; pass < npass && ok; pass++) {
+                const int bytes = P::item_bytes(pass);
+                const uint8_t *c0, *c1 = nullptr;   // code and meta sources of this pass's first tile
+                int cstride = 0, c1stride = P::MR * kItem;
+                if (pass == 0) {
+                    c0 = a.a_codes[0] + tok0 * P::A_C;
+                    c1 = a.a_meta[0] + tok0 * P::MR;
+                    cstride = P::A_C * kItem;
+                } else if (pass == 1) {
+                    c0 = a.a_codes[1] + tok0 * P::A_C;
+                    c1 = a.a_meta[1] + tok0 * P::MR;
+                    cstride = P::A_C * kItem;
+                } else {
+                    c0 = a.r_codes[1] + tok0 * P::R_C;
+                    c1 = a.r_meta[1] + tok0 * P::MR;
+                    cstride = P::R_C * kItem;
+                }
+                const uint8_t *r0 = RESID ? a.r_codes[0] + tok0 * P::R_C : nullptr;
+                const uint8_t *r1 = RESID ? a.r_meta[0] + tok0 * P::MR : nullptr;
+                const uint8_t *r2 = RESID ? reinterpret_cast<const uint8_t *>(a.r_coef[0] + tok0) : nullptr;
+                for (int j = 0; j < nitems; j++, it++) {
+                    if (phys + bytes > P::RING) {
+                        virt += P::RING - phys;
+                        phys = 0;
                     }
-                    while (rel[w] < it[w] &&
-                           (it[w] - rel[w] >= kSlots || s_start[w][rel[w] % kSlots] < virt[w] + bytes - P::RING)) {
-                        dep(0, 0x7FFFFFFF);   // about to block on the consumers, who run after their wait
-                        if (!mbar_wait(&bar_empty[w][rel[w] % kSlots], (rel[w] / kSlots) & 1, &s_abort)) {
+                    if (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING))
+                        dep(0x7FFFFFFF);   // about to block on the consumers, who run after their wait
+                    dep(min((j + 1) * kItem, n));
+                    while (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING)) {
+                        if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
+                                                                    &s_abort)) {
                             ok = false;
                             break;
                         }
-                        rel[w]++;
+                        vrel += rbytes;
+                        rphys += rbytes;
+                        if (++ritem == nitems) {
+                            ritem = 0;
+                            rbytes = P::item_bytes(++rpass);
+                        }
+                        if (rphys + rbytes > P::RING) {
+                            vrel += P::RING - rphys;
+                            rphys = 0;
+                        }
+                        rel++;
                     }
                     if (!ok) {
                         s_abort = 1;
                         atomicExch(a.err, 1);
                         break;
                     }
-                    const int j = jj[w];
-                    dep(k.t0, min((j + 1) * kItem, k.n));
                     // the last item of a pass may hold fewer tiles: copy only those
-                    const int toks = min(kItem, (k.ntiles - j * kItemTiles) * kTile);
-                    const size_t tok = k.bh * a.Tp + (size_t)k.t0 + (size_t)j * kItem;
-                    uint8_t *st = smem + w * wg_bytes + phys[w];
-                    uint64_t *bar = &bar_full[w][it[w] % kSlots];
-                    s_start[w][it[w] % kSlots] = virt[w];
-                    if (pass[w] == 0) {
+                    const int toks = min(kItem, (ntiles - j * kItemTiles) * kTile);
+                    uint8_t *st = ring + phys;
+                    uint64_t *bar = &bar_full[it % kSlots];
+                    if (pass == 0) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + (RESID ? P::R_C + P::MR + 2 : 0))));
-                        bulk_g2s(st, a.a_codes[0] + tok * P::A_C, toks * P::A_C, bar);
-                        bulk_g2s(st + P::K_AM, a.a_meta[0] + tok * P::MR, toks * P::MR, bar);
+                        bulk_g2s(st, c0, toks * P::A_C, bar);
+                        bulk_g2s(st + P::K_AM, c1, toks * P::MR, bar);
                         if (RESID) {
-                            bulk_g2s(st + P::K_RC, a.r_codes[0] + tok * P::R_C, toks * P::R_C, bar);
-                            bulk_g2s(st + P::K_RM, a.r_meta[0] + tok * P::MR, toks * P::MR, bar);
-                            bulk_g2s(st + P::K_CF, a.r_coef[0] + tok, toks * 2, bar);
+                            bulk_g2s(st + P::K_RC, r0, toks * P::R_C, bar);
+                            bulk_g2s(st + P::K_RM, r1, toks * P::MR, bar);
+                            bulk_g2s(st + P::K_CF, r2, toks * 2, bar);
+                            r0 += kItem * P::R_C;
+                            r1 += kItem * P::MR;
+                            r2 += kItem * 2;
                         }
-                    } else if (pass[w] == 1) {
-                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR)));
-                        bulk_g2s(st, a.a_codes[1] + tok * P::A_C, toks * P::A_C, bar);
-                        bulk_g2s(st + P::VA_M, a.a_meta[1] + tok * P::MR, toks * P::MR, bar);
                     } else {
-                        mbar_expect_tx(bar, (uint32_t)(toks * (P::R_C + P::MR)));
-                        bulk_g2s(st, a.r_codes[1] + tok * P::R_C, toks * P::R_C, bar);
-                        bulk_g2s(st + P::VR_M, a.r_meta[1] + tok * P::MR, toks * P::MR, bar);
+                        const int cb = pass == 1 ? P::A_C : P::R_C;
+                        mbar_expect_tx(bar, (uint32_t)(toks * (cb + P::MR)));
+                        bulk_g2s(st, c0, toks * cb, bar);
+                        bulk_g2s(st + cstride, c1, toks * P::MR, bar);
                     }
-                    virt[w] += bytes;
-                    phys[w] += bytes;
-                    it[w]++;
-                    if (++jj[w] == k.nitems) {
-                        jj[w] = 0;
-                        pass[w]++;
-                    }
+                    c0 += cstride;
+                    c1 += c1stride;
+                    virt += bytes;
+                    phys += bytes;
                 }
             }
-            dep(0, 0x7FFFFFFF);
+            dep(0x7FFFFFFF);
+            const int issued = it;
             // drain: every issued copy must have landed before the CTA exits
             // (the consumers stop waiting once the CTA has given up)
-#pragma unroll
-            for (int w = 0; w < NWG; w++) {
-                if (RESID && blockIdx.x * NWG + w < nchunks) mbar_wait<256>(&bar_cf[w], 0, &s_abort);
-                for (int i = max(0, it[w] - kSlots); i < it[w]; i++)
-                    mbar_wait<256>(&bar_full[w][i % kSlots], (i / kSlots) & 1, &s_abort);
-            }
+            if (RESID) mbar_wait<256>(&bar_cf, 0, &s_abort);
+            for (int it = max(0, issued - kSlots); it < issued; it++)
+                mbar_wait<256>(&bar_full[it % kSlots], (it / kSlots) & 1, &s_abort);
         } else {
-            // the other lanes: the bound max |s_hat(V)| of each chunk's V
+            // the other lanes: the bound max |s_hat(V)| of the chunk's V
             // coefficients (for the weights' fixed point), ready before the
             // softmax needs it
             griddep_wait_then_release();
-            for (int w = 0; w < NWG; w++) {
-                const int c = blockIdx.x * NWG + w;
-                if (c >= nchunks) break;
-                unsigned m = 0;
-                if (RESID && mbar_wait<64>(&bar_cf[w], 0, &s_abort)) {
-                    const Chunk k = chunk_of(a, c, npairs);
-                    const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + w * wg_bytes + P::RING);
-                    for (int t = lane - 1; t < k.n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
-                }
-                atomicMax(&s_cfmax[w], m);
-                mbar_arrive(&bar_cfmax[w]);
+            unsigned m = 0;
+            if (RESID && mbar_wait<64>(&bar_cf, 0, &s_abort)) {
+                const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING);
+                for (int t = lane - 1; t < n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
             }
+            atomicMax(&s_cfmax, m);
+            mbar_arrive(&bar_cfmax);
         }
         return;
     }
 
     // ------------------------------------------------------------ consumers
-    const int wg = warp >> 2;                 // consumer warp-group
-    const int cid = blockIdx.x * NWG + wg;    // its chunk
-    if (cid >= nchunks) return;
-    const int lw = warp & 3, ltid = tid & (kConsumers - 1);
-    const Chunk ck = chunk_of(a, cid, npairs);
-    const int b = ck.b, h = ck.h, pair = ck.pair, split = ck.split, n = ck.n, ntiles = ck.ntiles,
-              nitems = ck.nitems;
-    const size_t bh = ck.bh;
-    const int hq0 = h * a.G + pair * GK;
-    uint8_t *ring = smem + wg * wg_bytes;
-    const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(ring + P::RING);        // V coefficients
-    float *s_sc = reinterpret_cast<float *>(ring + P::RING + P::coef_bytes(a.chunk));  // [GK][chunk] logits -> p
-    float *s_P = s_sc + GK * a.chunk;                                                  // [GK][chunk] p * s_hat
-    float(*red)[2 * GK + 2] = s_red[wg];
-
     griddep_wait_then_release();
     // upper bounds of this stream's V scales (anchor; the loop's residual)
     const float vA = e4m3_to_f32((uint32_t)a.vmax_a[bh]);
@@ -596,9 +548,9 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
     if (a.n_new > 0 && split == 0) {
         // fused append: this unit's new tail rows (K and V, 16-byte vectors);
         // the fence before the arrival count below publishes them to the
-        // group that combines
+        // CTA that combines
         const int nvec = a.n_new * 2 * (kHeadDim / 8);
-        for (int i = ltid; i < nvec; i += kConsumers) {
+        for (int i = tid; i < nvec; i += kConsumers) {
             const int vec = i % (kHeadDim / 8), r = i / (kHeadDim / 8), kv = r & 1, t = r >> 1;
             const uint4 *src = reinterpret_cast<const uint4 *>((kv ? a.new_v : a.new_k) +
                                                                (((size_t)b * a.n_new + t) * a.H + h) * kHeadDim);
@@ -612,14 +564,14 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
 
     // q (log2-domain scale folded in) and R q, then 24-bit fixed-point planes
     for (int gq = 0; gq < GK; gq++)
-        s_q[wg][gq][0][ltid] = bf16_to_f32(a.q[((size_t)b * a.Hq + hq0 + gq) * kHeadDim + ltid]) * a.scale_log2;
-    wg_sync(wg);
-    if (RESID && lw < GK) {
-        const int gq = lw;
+        s_q[gq][0][tid] = bf16_to_f32(a.q[((size_t)b * a.Hq + hq0 + gq) * kHeadDim + tid]) * a.scale_log2;
+    consumer_sync();
+    if (RESID && warp < GK) {
+        const int gq = warp;
         float v[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-            v[k] = s_q[wg][gq][0][4 * lane + k];
+            v[k] = s_q[gq][0][4 * lane + k];
             if (a.rotate && sigma_neg(a.sigma, 4 * lane + k)) v[k] = -v[k];
         }
         if (a.rotate) {
@@ -628,66 +580,66 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
             for (int k = 0; k < 4; k++) v[k] *= kRsqrt128;
         }
 #pragma unroll
-        for (int k = 0; k < 4; k++) s_q[wg][gq][1][4 * lane + k] = v[k];
+        for (int k = 0; k < 4; k++) s_q[gq][1][4 * lane + k] = v[k];
     }
-    wg_sync(wg);
+    consumer_sync();
     {
         float mx = 0.f;
         for (int gq = 0; gq < GK; gq++) {
-            mx = fmaxf(mx, fabsf(s_q[wg][gq][0][ltid]));
-            if (RESID) mx = fmaxf(mx, fabsf(s_q[wg][gq][1][ltid]));
+            mx = fmaxf(mx, fabsf(s_q[gq][0][tid]));
+            if (RESID) mx = fmaxf(mx, fabsf(s_q[gq][1][tid]));
         }
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-        if (lane == 0) red[lw][0] = mx;
+        if (lane == 0) s_red[warp][0] = mx;
     }
-    wg_sync(wg);
-    const float qmax = fmaxf(fmaxf(red[0][0], red[1][0]), fmaxf(red[2][0], red[3][0]));
+    consumer_sync();
+    const float qmax = fmaxf(fmaxf(s_red[0][0], s_red[1][0]), fmaxf(s_red[2][0], s_red[3][0]));
     const float qscale = fixed_scale(qmax, 22);  // q_int = round(q * qscale), |q_int| < 2^22
     const float qinv = 1.f / qscale;             // exact (power of two)
-    // Each consumer thread converts element ltid of q (and of R q) and stores
+    // Each consumer thread converts element tid of q (and of R q) and stores
     // its three bytes where the lanes of its segment pick them up as plane
     // words; the integer sum of each segment's 16 values comes from a
     // 16-lane shuffle reduction.
     {
-        const int sg = ltid >> 4, i = ltid & 15;
+        const int sg = tid >> 4, i = tid & 15;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
 #pragma unroll
             for (int ab = 0; ab < (RESID ? 2 : 1); ab++) {
-                const int x = __float2int_rn(s_q[wg][gq][ab][ltid] * qscale);
-                uint8_t *dst = &s_qp[wg][gq][ab][0][sg * 16 + (ab == 0 ? slot_of<BA>(i) : slot_of<BR>(i))];
+                const int x = __float2int_rn(s_q[gq][ab][tid] * qscale);
+                uint8_t *dst = &s_qp[gq][ab][0][sg * 16 + (ab == 0 ? slot_of<BA>(i) : slot_of<BR>(i))];
                 dst[0] = (uint8_t)(x & 0xFF);
                 dst[kHeadDim] = (uint8_t)((x >> 8) & 0xFF);
                 dst[2 * kHeadDim] = (uint8_t)((x >> 16) & 0xFF);
                 int sum = x;
 #pragma unroll
                 for (int m = 1; m < 16; m <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
-                if (i == 0) s_qsum[wg][gq][ab][sg] = sum;
+                if (i == 0) s_qsum[gq][ab][sg] = sum;
             }
         }
     }
-    wg_sync(wg);
+    consumer_sync();
     QPlanes qA[GK], qR[GK];
     float QA[GK], QR[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
 #pragma unroll
         for (int pl = 0; pl < 3; pl++) {
-            const uint4 wa = *reinterpret_cast<const uint4 *>(&s_qp[wg][gq][0][pl][seg * 16]);
+            const uint4 wa = *reinterpret_cast<const uint4 *>(&s_qp[gq][0][pl][seg * 16]);
             qA[gq].p[pl][0] = wa.x;
             qA[gq].p[pl][1] = wa.y;
             qA[gq].p[pl][2] = wa.z;
             qA[gq].p[pl][3] = wa.w;
             if (RESID) {
-                const uint4 wr = *reinterpret_cast<const uint4 *>(&s_qp[wg][gq][1][pl][seg * 16]);
+                const uint4 wr = *reinterpret_cast<const uint4 *>(&s_qp[gq][1][pl][seg * 16]);
                 qR[gq].p[pl][0] = wr.x;
                 qR[gq].p[pl][1] = wr.y;
                 qR[gq].p[pl][2] = wr.z;
                 qR[gq].p[pl][3] = wr.w;
             }
         }
-        QA[gq] = (float)s_qsum[wg][gq][0][seg];
-        QR[gq] = RESID ? (float)s_qsum[wg][gq][1][seg] : 0.f;
+        QA[gq] = (float)s_qsum[gq][0][seg];
+        QR[gq] = RESID ? (float)s_qsum[gq][1][seg] : 0.f;
     }
 
     // ------------------------------------------------------------ pass 1: logits
@@ -696,10 +648,11 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
     const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
     const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
+    const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // ring items per pass
     int c_off = 0;   // ring offset of the current item (the producer's placement rule)
     for (int j = 0; j < nitems; j++) {
         const int slot = j % kSlots;
-        const bool ok = mbar_wait(&bar_full[wg][slot], (j / kSlots) & 1, &s_abort);
+        const bool ok = mbar_wait(&bar_full[slot], (j / kSlots) & 1, &s_abort);
         if (!ok) {
             s_abort = 1;
             atomicExch(a.err, 2);
@@ -711,7 +664,7 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
             if (j * kItemTiles + u >= ntiles) break;   // uniform: a short last item
 #pragma unroll
             for (int k = 0; k < 4; k++) {
-                const int tok = u * kTile + 16 * lw + sub + 4 * k;   // token within the item
+                const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
                 const Seg<BA> ca = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
                 const float2 ma =
                     meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_AM + tok * P::MR + 2 * mg));
@@ -735,14 +688,14 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
                 }
             }
         }
-        mbar_arrive(&bar_empty[wg][slot]);
+        mbar_arrive(&bar_empty[slot]);
         c_off = P::advance(c_off, P::K_BYTES, j + 1 < nitems ? P::K_BYTES : P::VA_BYTES);
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
             const int i = j * kItemTiles + u;
             if (i >= ntiles) break;
-            const int tl = i * kTile + 16 * lw + sub + 4 * kown;
+            const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
                 float r0 = (b4 ? part[u][gq][2] : part[u][gq][0]) +
@@ -763,31 +716,32 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
     for (int gq = 0; gq < GK; gq++) {
         float v = mloc[gq];
         for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
-        if (lane == 0) red[lw][gq] = v;
+        if (lane == 0) s_red[warp][gq] = v;
     }
-    if (RESID && !mbar_wait(&bar_cf[wg], 0, &s_abort)) {
+    if (RESID && !mbar_wait(&bar_cf, 0, &s_abort)) {
         s_abort = 1;
         atomicExch(a.err, 3);
     }
-    wg_sync(wg);
+    consumer_sync();
     float M[GK];
 #pragma unroll
-    for (int gq = 0; gq < GK; gq++) M[gq] = fmaxf(fmaxf(red[0][gq], red[1][gq]), fmaxf(red[2][gq], red[3][gq]));
+    for (int gq = 0; gq < GK; gq++)
+        M[gq] = fmaxf(fmaxf(s_red[0][gq], s_red[1][gq]), fmaxf(s_red[2][gq], s_red[3][gq]));
     // the weights' fixed-point scales: w = P * sc (anchor) or p * sc
     // (residual), |P| <= max|s_hat|, p <= 1, sc <= the stream's largest V
     // scale (powers of two)
-    if (!mbar_wait(&bar_cfmax[wg], 0, &s_abort)) {
+    if (!mbar_wait(&bar_cfmax, 0, &s_abort)) {
         s_abort = 1;
         atomicExch(a.err, 3);
     }
-    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax[wg]) * vA : vA, kWeightTop);
+    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax) * vA : vA, kWeightTop);
     const float cR = fixed_scale(vR, kWeightTop);
     // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V
     // weight), zero beyond the chunk's tokens, stored with their scales
     float lsum[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
-    for (int t = ltid; t < ntiles * kTile; t += kConsumers) {
+    for (int t = tid; t < ntiles * kTile; t += kConsumers) {
         const bool valid = t < n;
         const float shv = RESID ? bf16_to_f32(s_cf[t]) : 1.f;
 #pragma unroll
@@ -802,12 +756,13 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
     for (int gq = 0; gq < GK; gq++) {
         float v = lsum[gq];
         for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-        if (lane == 0) red[lw][GK + gq] = v;   // beside the maxima, which are read until here
+        if (lane == 0) s_red[warp][GK + gq] = v;   // beside the maxima, which are read until here
     }
-    wg_sync(wg);
+    consumer_sync();
     float Lsum[GK];
 #pragma unroll
-    for (int gq = 0; gq < GK; gq++) Lsum[gq] = red[0][GK + gq] + red[1][GK + gq] + red[2][GK + gq] + red[3][GK + gq];
+    for (int gq = 0; gq < GK; gq++)
+        Lsum[gq] = s_red[0][GK + gq] + s_red[1][GK + gq] + s_red[2][GK + gq] + s_red[3][GK + gq];
 
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
     const int npass = RESID ? 2 : 1;
@@ -829,7 +784,7 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
         for (int j = 0; j < nitems; j++) {
             const int it = (1 + vp) * nitems + j;
             const int slot = it % kSlots;
-            if (!mbar_wait(&bar_full[wg][slot], (it / kSlots) & 1, &s_abort)) {
+            if (!mbar_wait(&bar_full[slot], (it / kSlots) & 1, &s_abort)) {
                 s_abort = 1;
                 atomicExch(a.err, 4);
             }
@@ -845,7 +800,7 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
                 Seg<BR> cr[4];
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    const int tok = u * kTile + 16 * lw + sub + 4 * k;   // token within the item
+                    const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
                     if (vp == 0) {
                         ca[k] = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
                         mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VA_M + tok * P::MR + 2 * mg));
@@ -857,7 +812,7 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
                     for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + j * kItem + tok];
                 }
                 if (u == last_u) {   // every read of the item is done: release it
-                    mbar_arrive(&bar_empty[wg][slot]);
+                    mbar_arrive(&bar_empty[slot]);
                     const int cur = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
                     c_off = P::advance(c_off, cur, j + 1 < nitems ? cur : P::VR_BYTES);
                 }
@@ -932,121 +887,110 @@ __global__ void __launch_bounds__(NWG * kConsumers + 32, (min_ctas<GK, NWG>()))
             r2.y = (hb16 ? r1[5] : r1[1]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[1] : r1[5], 16);
             r2.z = (hb16 ? r1[6] : r1[2]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[2] : r1[6], 16);
             r2.w = (hb16 ? r1[7] : r1[3]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[3] : r1[7], 16);
-            *reinterpret_cast<float4 *>(&s_acc[wg][lw][gq][vp][seg * 16 + (hb8 ? 8 : 0) + (hb16 ? 4 : 0)]) = r2;
+            *reinterpret_cast<float4 *>(&s_acc[warp][gq][vp][seg * 16 + (hb8 ? 8 : 0) + (hb16 ? 4 : 0)]) = r2;
         }
     }
 
     // ------------------------------------------------------------ reduce over warps, write the partial
-    wg_sync(wg);
+    consumer_sync();
     float oA[GK], oR[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
-        oA[gq] = s_acc[wg][0][gq][0][ltid] + s_acc[wg][1][gq][0][ltid] + s_acc[wg][2][gq][0][ltid] +
-                 s_acc[wg][3][gq][0][ltid];
-        oR[gq] = RESID ? s_acc[wg][0][gq][1][ltid] + s_acc[wg][1][gq][1][ltid] + s_acc[wg][2][gq][1][ltid] +
-                             s_acc[wg][3][gq][1][ltid]
+        oA[gq] = s_acc[0][gq][0][tid] + s_acc[1][gq][0][tid] + s_acc[2][gq][0][tid] + s_acc[3][gq][0][tid];
+        oR[gq] = RESID ? s_acc[0][gq][1][tid] + s_acc[1][gq][1][tid] + s_acc[2][gq][1][tid] + s_acc[3][gq][1][tid]
                        : 0.f;
     }
     if (RESID && a.rotate) {
         // o += R^T o_rot = sigma . (H o_rot) / sqrt(d)
 #pragma unroll
-        for (int gq = 0; gq < GK; gq++) s_q[wg][gq][1][ltid] = oR[gq];
-        wg_sync(wg);
-        if (lw < GK) {
-            const int gq = lw;
+        for (int gq = 0; gq < GK; gq++) s_q[gq][1][tid] = oR[gq];
+        consumer_sync();
+        if (warp < GK) {
+            const int gq = warp;
             float v[4];
 #pragma unroll
-            for (int k = 0; k < 4; k++) v[k] = s_q[wg][gq][1][4 * lane + k];
+            for (int k = 0; k < 4; k++) v[k] = s_q[gq][1][4 * lane + k];
             wht128_warp<float>(v, lane);
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 float r = v[k] * kRsqrt128;
                 if (sigma_neg(a.sigma, 4 * lane + k)) r = -r;
-                s_q[wg][gq][1][4 * lane + k] = r;
+                s_q[gq][1][4 * lane + k] = r;
             }
         }
-        wg_sync(wg);
+        consumer_sync();
 #pragma unroll
-        for (int gq = 0; gq < GK; gq++) oR[gq] = s_q[wg][gq][1][ltid];
+        for (int gq = 0; gq < GK; gq++) oR[gq] = s_q[gq][1][tid];
     }
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) {
         float *part = a.partials + (((size_t)b * a.Hq + hq0 + gq) * a.splits_max + split) * kPartialStride;
-        part[ltid] = oA[gq] + oR[gq];
-        if (ltid == 0) {
+        part[tid] = oA[gq] + oR[gq];
+        if (tid == 0) {
             part[kHeadDim] = M[gq];
             part[kHeadDim + 1] = Lsum[gq];
         }
     }
 
-    // ------------------------------------------------------------ last chunk of the unit combines
+    // ------------------------------------------------------------ last CTA of the unit combines
     __threadfence();
-    wg_sync(wg);
+    consumer_sync();
     const int unit = (b * a.H + h) * npairs + pair;
-    if (ltid == 0) s_last[wg] = (atomicAdd(&a.counters[unit], 1) == a.S - 1);
-    wg_sync(wg);
-    if (s_last[wg]) {
+    if (tid == 0) s_last = (atomicAdd(&a.counters[unit], 1) == a.S - 1);
+    consumer_sync();
+    if (s_last) {
         __threadfence();
-        if (ltid == 0) a.counters[unit] = 0;   // ready for the next call
+        if (tid == 0) a.counters[unit] = 0;   // ready for the next call
 #pragma unroll 1
         for (int gq = 0; gq < GK; gq++) {
             const size_t row = (size_t)b * a.Hq + hq0 + gq;
             const size_t trow = ((size_t)b * a.tail_cap * a.H + h) * kHeadDim;
             combine_row(a.partials + row * a.splits_max * kPartialStride, a.S, a.q + row * kHeadDim, a.scale_log2,
                         a.tail_k ? a.tail_k + trow : nullptr, a.tail_v ? a.tail_v + trow : nullptr,
-                        (size_t)a.H * kHeadDim, a.n_tail, a.out + row * kHeadDim, ltid, &red[0][0], WgSync{wg});
+                        (size_t)a.H * kHeadDim, a.n_tail, a.out + row * kHeadDim, tid, &s_red[0][0],
+                        ConsumerSync());
         }
     }
-}
-
-template <int GK>
-constexpr int nwg() {
-    return GK == 1 ? RQ_DECODE_NWG1 : RQ_DECODE_NWG2;
 }
 
 template <int GK, int BA, int BR, int GS, bool RESID>
 cudaError_t configure() {
     static bool done[kMaxDevices] = {};   // the largest dynamic shared memory any launch can ask for
     return once_per_device(done, [] {
-        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID, nwg<GK>()>,
+        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)(nwg<GK>() * Plan<BA, BR, GS, RESID>::wg_smem(GK, kMaxChunk)));
+                                    (int)Plan<BA, BR, GS, RESID>::smem(GK, kMaxChunk));
     });
 }
 
 template <int GK, int BA, int BR, int GS, bool RESID>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
-    constexpr int NWG = nwg<GK>();
-    const int nchunks = a.S * a.H * a.B * (a.G / GK);
+    const dim3 grid(a.S, a.H, a.B * (a.G / GK));
     cudaError_t e = configure<GK, BA, BR, GS, RESID>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3((nchunks + NWG - 1) / NWG);
-    lc.blockDim = dim3(NWG * kConsumers + 32);
-    lc.dynamicSmemBytes = NWG * Plan<BA, BR, GS, RESID>::wg_smem(GK, a.chunk);
+    lc.gridDim = grid;
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = Plan<BA, BR, GS, RESID>::smem(GK, a.chunk);
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = RQ_DECODE_PDL ? 1 : 0;
-    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, RESID, NWG>, a);
+    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, RESID>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-// resident chunks per SM: CTAs per SM x warp-groups per CTA
 template <int GK, int BA, int BR, int GS, bool RESID>
 int occupancy_t(int chunk) {
-    constexpr int NWG = nwg<GK>();
     if (configure<GK, BA, BR, GS, RESID>() != cudaSuccess) return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, RESID, NWG>,
-                                                      NWG * kConsumers + 32,
-                                                      NWG * Plan<BA, BR, GS, RESID>::wg_smem(GK, chunk)) !=
-        cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, RESID>, kThreads,
+                                                      Plan<BA, BR, GS, RESID>::smem(GK, chunk)) != cudaSuccess)
         return 1;
-    return n > 0 ? n * NWG : 1;
+    return n > 0 ? n : 1;
 }
 
 // Variant dispatch: one instantiation per (q heads per CTA, bits, group, loop kind).

@@ -107,6 +107,8 @@ struct AppendArgs {
     SeqLens pos0;                              // first token position written, per sequence
     int B, H, n, Tp, tail_cap, nres;           // nres = Lg - 1
     int g, ba, br, rotate;
+    int scale_mode;                            // 0 least squares, 1 norm ratio, 2 none
+    int chained;                               // 1: loop 0 is the anchor, loop l a residual against loop l - 1
     uint32_t sigma[4];
 };
 

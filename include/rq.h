@@ -81,8 +81,32 @@ typedef enum {
  *                    (Sylvester Hadamard; sigma_j = -1 iff the top bit of
  *                    splitmix64(seed + j) is set); 0: R = I
  *   format           rq_format
- *   seed             rotation seed (one rotation per cache, shared by K and
- *                    V, all layers and loops)
+ *   seed             rotation seed (shared by K and V and all loops)
+ *   scale_mode       coefficient of a residual loop (the abstract's scaling
+ *                    ablation): 0 least squares <x, ref>/<ref, ref> (the
+ *                    method), 1 norm ratio |x|/|ref|, 2 none (s = 1); 0 when
+ *                    ref = 0 (modes 0, 1).  Stored in BF16 either way.
+ *   anchor_mode      reference of a residual loop (the abstract's reference
+ *                    ablation): 0 the group's last loop, shared by all other
+ *                    loops (the method: two cache reads per loop); 1 chained:
+ *                    the group's FIRST loop is quantized at anchor_bits and
+ *                    loop l >= 1 is a residual against the reconstruction of
+ *                    loop l - 1, so rebuilding loop l reads l + 1 records.
+ *                    The group is still committed when its last loop is
+ *                    appended.
+ *   rotation_per_layer  0: one rotation per cache; 1: layer i uses the seed
+ *                    seed + i * 2^32 (rotations fixed per layer)
+ *   block_tokens     0: each sequence's records are contiguous (capacity
+ *                    max_tokens); 128 or 256: paged -- records live in
+ *                    blocks of this many tokens drawn from a pool of
+ *                    num_blocks physical blocks per (layer, group), through a
+ *                    per-sequence block table shared by all layers and groups
+ *                    (the library allocates blocks as sequences grow and
+ *                    returns them when sequences shrink; see
+ *                    rq_cache_fork_seq).  RQ_FMT_RESIDUAL only.
+ *   num_blocks       paged: physical blocks per pool (each holds block_tokens
+ *                    tokens of every kv head); 0 otherwise
+ * Fields after `seed` are zero for the method with contiguous records.
  */
 typedef struct rq_config {
     int32_t num_layers;
@@ -100,6 +124,11 @@ typedef struct rq_config {
     int32_t rotate;
     int32_t format;
     uint64_t seed;
+    int32_t scale_mode;
+    int32_t anchor_mode;
+    int32_t rotation_per_layer;
+    int32_t block_tokens;
+    int32_t num_blocks;
 } rq_config;
 
 typedef struct rq_cache rq_cache;

@@ -73,6 +73,12 @@ def lib():
         L.orc_attention.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [ctypes.c_void_p] * 4 + [ctypes.c_int]
         L.orc_mse.restype = ctypes.c_double
         L.orc_mse.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
+        L.orc_encode_modes.restype = None
+        L.orc_encode_modes.argtypes = [ctypes.c_int] * 7 + [ctypes.c_uint64] + [ctypes.c_int] * 2 + \
+            [ctypes.c_void_p] * 11
+        L.orc_reconstruct_modes.restype = None
+        L.orc_reconstruct_modes.argtypes = [ctypes.c_int] * 7 + [ctypes.c_uint64] + [ctypes.c_int] + \
+            [ctypes.c_void_p] * 6
         L.orc_encode_ablation.restype = None
         L.orc_encode_ablation.argtypes = [ctypes.c_int] * 7 + [ctypes.c_uint64] + [ctypes.c_int] * 2 + \
             [ctypes.c_void_p] * 4
@@ -211,6 +217,36 @@ def reconstruct(a_codes, a_meta, r_codes, r_meta, r_coef, L: int, d: int, g: int
     out = np.zeros((L, n, d), np.float64)
     lib().orc_reconstruct(n, L, d, g, ba, br, int(rotate), seed, _p(a_codes), _p(a_meta),
                           _p(r_codes), _p(r_meta), _p(r_coef), _p(out))
+    return out
+
+
+def encode_modes(x_bf16: np.ndarray, g: int, ba: int, br: int, rotate: bool, seed: int, anchor_mode: int,
+                 scale_mode: int) -> Encoded:
+    """Records of the ablation modes in the library's layout (orc_encode_modes):
+    x_bf16 uint16 [L][n][d] in loop order."""
+    x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)
+    L, n, d = x_bf16.shape
+    e = Encoded(n, L, d, g, ba, br)
+    lib().orc_encode_modes(n, L, d, g, ba, br, int(rotate), seed, int(anchor_mode), int(scale_mode), _p(x_bf16),
+                           _p(e.a_codes), _p(e.a_meta), _p(e.r_codes), _p(e.r_meta), _p(e.r_coef),
+                           _p(e.a_eflag), _p(e.a_mflag), _p(e.r_eflag), _p(e.r_mflag), _p(e.r_cflag))
+    return e
+
+
+def reconstruct_modes(a_codes, a_meta, r_codes, r_meta, r_coef, L: int, d: int, g: int, ba: int, br: int,
+                      rotate: bool, seed: int, anchor_mode: int) -> np.ndarray:
+    """float64 [L][n][d] in loop order, from records as encode_modes lays them out."""
+    if anchor_mode == 0:
+        return reconstruct(a_codes, a_meta, r_codes, r_meta, r_coef, L, d, g, ba, br, rotate, seed)
+    a_codes = np.ascontiguousarray(a_codes, np.uint8)
+    a_meta = np.ascontiguousarray(a_meta, np.uint8)
+    r_codes = np.ascontiguousarray(r_codes, np.uint8)
+    r_meta = np.ascontiguousarray(r_meta, np.uint8)
+    r_coef = np.ascontiguousarray(r_coef, np.uint16)
+    n = a_codes.shape[0]
+    out = np.zeros((L, n, d), np.float64)
+    lib().orc_reconstruct_modes(n, L, d, g, ba, br, int(rotate), seed, int(anchor_mode), _p(a_codes), _p(a_meta),
+                                _p(r_codes), _p(r_meta), _p(r_coef), _p(out))
     return out
 
 

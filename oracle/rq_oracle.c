@@ -502,6 +502,127 @@ ORC_EXPORT void orc_reconstruct(int n, int L, int d, int g, int ba, int br, int 
 }
 
 /* ------------------------------------------------------------------ */
+/* Records of one loop group under the ablation modes, in the record     */
+/* layout the CUDA library stores (the abstract's comparison of          */
+/* reference choice and scaling method; see orc_encode_ablation below    */
+/* for the same chain as reconstructions).                               */
+/*   anchor_mode 0: the anchor record holds loop L-1; residual record j  */
+/*                  holds loop j (j < L-1) against a_hat;                */
+/*   anchor_mode 1: the anchor record holds loop 0; residual record j    */
+/*                  holds loop j+1 against the reconstruction of loop j. */
+/*   scale_mode 0 least squares <x, ref>/<ref, ref>, 1 norm ratio        */
+/*   |x|/|ref| (both 0 when ref = 0), 2 none (s = 1).                    */
+/* Outputs and flags as for orc_encode.  anchor_mode 0 with scale_mode 0 */
+/* is orc_encode.                                                        */
+/* ------------------------------------------------------------------ */
+ORC_EXPORT void orc_encode_modes(int n, int L, int d, int g, int ba, int br, int rotate, uint64_t seed,
+                                 int anchor_mode, int scale_mode, const uint16_t *x_bf16,
+                                 uint8_t *a_codes, uint8_t *a_meta,
+                                 uint8_t *r_codes, uint8_t *r_meta, uint16_t *r_coef,
+                                 uint8_t *a_eflag, uint8_t *a_mflag,
+                                 uint8_t *r_eflag, uint8_t *r_mflag, uint8_t *r_cflag)
+{
+    int t, j, i;
+    int G = d / g;
+    size_t ab = (size_t)(d * ba / 8), rb = (size_t)(d * br / 8);
+    const int first = anchor_mode == 0 ? L - 1 : 0;   /* the loop in the anchor record */
+    double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+    double c = orc_rotation_scale(d, rotate);
+    double *x = (double *)malloc(sizeof(double) * (size_t)d);
+    double *ahat = (double *)malloc(sizeof(double) * (size_t)d);
+    double *ref = (double *)malloc(sizeof(double) * (size_t)d);
+    double *r = (double *)malloc(sizeof(double) * (size_t)d);
+    double *y = (double *)malloc(sizeof(double) * (size_t)d);
+    double *yhat = (double *)malloc(sizeof(double) * (size_t)d);
+    double *back = (double *)malloc(sizeof(double) * (size_t)d);
+    orc_rotation_signs_matrix(seed, d, rotate, S);
+    for (t = 0; t < n; t++) {
+        for (i = 0; i < d; i++)
+            x[i] = orc_bf16_value(x_bf16[((size_t)first * n + t) * d + i]);
+        quantize_record(x, d, g, ba, a_codes + (size_t)t * ab, a_meta + (size_t)t * 2 * G,
+                        a_eflag ? a_eflag + (size_t)t * d : NULL,
+                        a_mflag ? a_mflag + (size_t)t * G : NULL);
+        orc_dequant(a_codes + (size_t)t * ab, a_meta + (size_t)t * 2 * G, d, g, ba, ahat);
+        memcpy(ref, ahat, sizeof(double) * (size_t)d);
+        for (j = 0; j < L - 1; j++) {
+            const int loop = anchor_mode == 0 ? j : j + 1;
+            double num = 0.0, den = 0.0, xx = 0.0, s = 0.0, shat;
+            int cnear = 0;
+            uint16_t sbits;
+            size_t rec = (size_t)j * n + t;
+            for (i = 0; i < d; i++)
+                x[i] = orc_bf16_value(x_bf16[((size_t)loop * n + t) * d + i]);
+            for (i = 0; i < d; i++) {
+                num += x[i] * ref[i];
+                den += ref[i] * ref[i];
+                xx += x[i] * x[i];
+            }
+            if (scale_mode == 2)
+                s = 1.0;
+            else if (den != 0.0)
+                s = scale_mode == 0 ? num / den : sqrt(xx) / sqrt(den);
+            sbits = orc_bf16_round(s, &cnear);
+            shat = orc_bf16_value(sbits);
+            r_coef[rec] = sbits;
+            if (r_cflag)
+                r_cflag[rec] = (uint8_t)cnear;
+            for (i = 0; i < d; i++)
+                r[i] = x[i] - shat * ref[i];
+            rotate_vec(S, c, d, r, y);
+            quantize_record(y, d, g, br, r_codes + rec * rb, r_meta + rec * 2 * G,
+                            r_eflag ? r_eflag + rec * d : NULL,
+                            r_mflag ? r_mflag + rec * G : NULL);
+            if (anchor_mode == 1) {
+                /* the next loop's reference: this loop's reconstruction */
+                orc_dequant(r_codes + rec * rb, r_meta + rec * 2 * G, d, g, br, yhat);
+                rotate_back(S, c, d, yhat, back);
+                for (i = 0; i < d; i++)
+                    ref[i] = shat * ref[i] + back[i];
+            }
+        }
+    }
+    free(S); free(x); free(ahat); free(ref); free(r); free(y); free(yhat); free(back);
+}
+
+/* Reconstruction of all L loops from records laid out as orc_encode_modes
+ * writes them: anchor_mode 0 as orc_reconstruct; anchor_mode 1: loop 0 =
+ * a_hat, loop l = s_hat_{l-1} x_hat_{l-1} + R^T y_hat_{l-1} (record l-1).
+ * out [L][n][d] in loop order. */
+ORC_EXPORT void orc_reconstruct_modes(int n, int L, int d, int g, int ba, int br, int rotate, uint64_t seed,
+                                      int anchor_mode, const uint8_t *a_codes, const uint8_t *a_meta,
+                                      const uint8_t *r_codes, const uint8_t *r_meta, const uint16_t *r_coef,
+                                      double *out)
+{
+    int t, l, i;
+    int G = d / g;
+    size_t ab = (size_t)(d * ba / 8), rb = (size_t)(d * br / 8);
+    double *S, *yhat, *back, c;
+    if (anchor_mode == 0) {
+        orc_reconstruct(n, L, d, g, ba, br, rotate, seed, a_codes, a_meta, r_codes, r_meta, r_coef, out);
+        return;
+    }
+    S = (double *)malloc(sizeof(double) * (size_t)d * d);
+    c = orc_rotation_scale(d, rotate);
+    yhat = (double *)malloc(sizeof(double) * (size_t)d);
+    back = (double *)malloc(sizeof(double) * (size_t)d);
+    orc_rotation_signs_matrix(seed, d, rotate, S);
+    for (t = 0; t < n; t++) {
+        orc_dequant(a_codes + (size_t)t * ab, a_meta + (size_t)t * 2 * G, d, g, ba, out + (size_t)t * d);
+        for (l = 1; l < L; l++) {
+            size_t rec = (size_t)(l - 1) * n + t;
+            const double shat = orc_bf16_value(r_coef[rec]);
+            const double *prev = out + ((size_t)(l - 1) * n + t) * d;
+            double *o = out + ((size_t)l * n + t) * d;
+            orc_dequant(r_codes + rec * rb, r_meta + rec * 2 * G, d, g, br, yhat);
+            rotate_back(S, c, d, yhat, back);
+            for (i = 0; i < d; i++)
+                o[i] = shat * prev[i] + back[i];
+        }
+    }
+    free(S); free(yhat); free(back);
+}
+
+/* ------------------------------------------------------------------ */
 /* Ablation encoders (the arXiv abstract's comparison of reference      */
 /* choice and scaling method): encode one loop group of n token-heads   */
 /* and return the reconstruction, for reconstruction-error studies.     */

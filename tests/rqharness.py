@@ -49,7 +49,7 @@ def scale32() -> float:
 
 def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, rotate=True,
           n_tail=0, seed=0x5EED0000, sigma=(0.1, 0.2, 0.3), chunk=128, fmt=rq.RQ_FMT_RESIDUAL,
-          only_layers=None, only_groups=None, max_tokens=None) -> Built:
+          only_layers=None, only_groups=None, max_tokens=None, **modes) -> Built:
     """Fills `layers` x (loops/Lg) groups with T committed tokens (appended in
     chunks through the tail), then n_tail in-flight tokens on every
     non-anchor loop."""
@@ -57,7 +57,7 @@ def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, r
     cfg = rq.make_config(num_layers=layers, num_loops=loops, loops_per_group=Lg, batch=B,
                          max_tokens=max_tokens or max(T, 1), max_tail_tokens=tail_cap, num_kv_heads=H,
                          num_q_heads=Hq, group_size=g, anchor_bits=ba, resid_bits=br, rotate=rotate,
-                         format=fmt, seed=0xA11CE)
+                         format=fmt, seed=0xA11CE, **modes)
     cache = rq.Cache(cfg)
     bt = Built(cache, cfg, seed, T, n_tail)
     for layer in range(layers):
@@ -120,7 +120,22 @@ def oracle_encode(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> orc.
         arrs.append(u.reshape(-1, D))
     x = np.stack(arrs)
     cfg = bt.cfg
-    return orc.encode(x, cfg.group_size, cfg.anchor_bits, cfg.resid_bits, bool(cfg.rotate), cfg.seed)
+    seed = rq.layer_seed(cfg, layer)
+    if cfg.anchor_mode or cfg.scale_mode:
+        return orc.encode_modes(x, cfg.group_size, cfg.anchor_bits, cfg.resid_bits, bool(cfg.rotate), seed,
+                                cfg.anchor_mode, cfg.scale_mode)
+    return orc.encode(x, cfg.group_size, cfg.anchor_bits, cfg.resid_bits, bool(cfg.rotate), seed)
+
+
+def anchor_loop(cfg, grp: int) -> int:
+    """The loop whose K/V the anchor record holds (the last of the group;
+    the first with the chained reference)."""
+    return grp * cfg.loops_per_group + (0 if cfg.anchor_mode else cfg.loops_per_group - 1)
+
+
+def residual_loop(cfg, grp: int, j: int) -> int:
+    """The loop whose K/V residual record j holds."""
+    return grp * cfg.loops_per_group + (j + 1 if cfg.anchor_mode else j)
 
 
 def gpu_records(bt: Built, layer: int, loop: int, kv: int, bh_sel=None):
@@ -156,8 +171,7 @@ def compare_records(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
     Lg = cfg.loops_per_group
     e = oracle_encode(bt, layer, grp, kv, bh_sel)
     res = dict(mismatch=0, tolerated=0, flagged=0, excluded=0, compared=0)
-    anchor_loop = grp * Lg + Lg - 1
-    gc, gm, _ = gpu_records(bt, layer, anchor_loop, kv, bh_sel)
+    gc, gm, _ = gpu_records(bt, layer, anchor_loop(cfg, grp), kv, bh_sel)
     grp_of = np.arange(D) // cfg.group_size
 
     def cmp(gpu_c, gpu_m, orc_c, orc_m, eflag, mflag, bits, skip_rows):
@@ -184,7 +198,7 @@ def compare_records(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
 
     a_tol = cmp(gc, gm, e.a_codes, e.a_meta, e.a_eflag, e.a_mflag, cfg.anchor_bits, np.zeros(len(gc), bool))
     for j in range(Lg - 1):
-        rc, rm, rf = gpu_records(bt, layer, grp * Lg + j, kv, bh_sel)
+        rc, rm, rf = gpu_records(bt, layer, residual_loop(cfg, grp, j), kv, bh_sel)
         cdiff = (rf != e.r_coef[j]) & ~a_tol
         cflag = e.r_cflag[j] != 0
         res["mismatch"] += int((cdiff & ~cflag).sum())
@@ -204,25 +218,26 @@ def reconstruct_gpu(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> np
 def _reconstruct_gpu(bt: Built, layer: int, grp: int, kv: int, bh_sel=None) -> np.ndarray:
     cfg = bt.cfg
     Lg = cfg.loops_per_group
-    ac, am, _ = gpu_records(bt, layer, grp * Lg + Lg - 1, kv, bh_sel)
+    ac, am, _ = gpu_records(bt, layer, anchor_loop(cfg, grp), kv, bh_sel)
     if Lg > 1:
-        rs = [gpu_records(bt, layer, grp * Lg + j, kv, bh_sel) for j in range(Lg - 1)]
+        rs = [gpu_records(bt, layer, residual_loop(cfg, grp, j), kv, bh_sel) for j in range(Lg - 1)]
         rc = np.stack([r[0] for r in rs])
         rm = np.stack([r[1] for r in rs])
         rf = np.stack([r[2] for r in rs])
     else:
         rc = rm = rf = None
-    return orc.reconstruct(ac, am, rc, rm, rf, Lg, D, cfg.group_size, cfg.anchor_bits, cfg.resid_bits,
-                           bool(cfg.rotate), cfg.seed)
+    return orc.reconstruct_modes(ac, am, rc, rm, rf, Lg, D, cfg.group_size, cfg.anchor_bits, cfg.resid_bits,
+                                 bool(cfg.rotate), rq.layer_seed(cfg, layer), cfg.anchor_mode)
 
 
 def mse_check(bt: Built, layer: int, grp: int, kv: int, bh_sel=None):
     cfg = bt.cfg
     e = oracle_encode(bt, layer, grp, kv, bh_sel)
     Lg = cfg.loops_per_group
-    mine = orc.reconstruct(e.a_codes, e.a_meta, e.r_codes if Lg > 1 else None, e.r_meta if Lg > 1 else None,
-                           e.r_coef if Lg > 1 else None, Lg, D, cfg.group_size, cfg.anchor_bits, cfg.resid_bits,
-                           bool(cfg.rotate), cfg.seed)
+    mine = orc.reconstruct_modes(e.a_codes, e.a_meta, e.r_codes if Lg > 1 else None,
+                                 e.r_meta if Lg > 1 else None, e.r_coef if Lg > 1 else None, Lg, D,
+                                 cfg.group_size, cfg.anchor_bits, cfg.resid_bits, bool(cfg.rotate),
+                                 rq.layer_seed(cfg, layer), cfg.anchor_mode)
     gpu = reconstruct_gpu(bt, layer, grp, kv, bh_sel)
     K, V = bt.inputs[(layer, grp)]
     X = K if kv == 0 else V

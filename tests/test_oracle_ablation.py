@@ -149,3 +149,29 @@ def test_study_on_synthetic_loops():
                 ("last", "previous")[am], ("least-squares", "norm-ratio", "none")[sm], k, v, rows[(am, sm, "reads")]))
         for kv in (0, 1):
             assert rows[(am, orc.SCALE_LEAST_SQUARES)][kv] < rows[(am, orc.SCALE_NONE)][kv]
+
+
+@pytest.mark.parametrize("anchor_mode", [orc.ANCHOR_LAST, orc.ANCHOR_PREVIOUS])
+@pytest.mark.parametrize("scale_mode", [orc.SCALE_LEAST_SQUARES, orc.SCALE_NORM_RATIO, orc.SCALE_NONE])
+@pytest.mark.parametrize("rotate", [True, False])
+def test_mode_records_rebuild_the_ablation(anchor_mode, scale_mode, rotate):
+    """The records the oracle lays out for each mode (orc_encode_modes: the
+    anchor record holds the last loop or, chained, the first; residual
+    record j holds loop j or loop j + 1), rebuilt by orc_reconstruct_modes,
+    give the ablation encoder's reconstruction bit for bit, and the stored
+    coefficients are its coefficients; the method's mode gives the method's
+    records."""
+    L = 4
+    x = _correlated(np.random.default_rng(40 + anchor_mode * 3 + scale_mode), L, 29)
+    e = orc.encode_modes(x, 16, 4, 2, rotate, SEED, anchor_mode, scale_mode)
+    xr = orc.reconstruct_modes(e.a_codes, e.a_meta, e.r_codes, e.r_meta, e.r_coef, L, D, 16, 4, 2, rotate, SEED,
+                               anchor_mode)
+    xh, coef, _ = orc.encode_ablation(x, 16, 4, 2, rotate, SEED, anchor_mode, scale_mode)
+    assert np.array_equal(xr, xh)
+    loops = range(L - 1) if anchor_mode == orc.ANCHOR_LAST else range(1, L)
+    for j, loop in enumerate(loops):
+        assert np.array_equal(orc.bf16_bits_to_f64(e.r_coef[j]), coef[loop])
+    if anchor_mode == orc.ANCHOR_LAST and scale_mode == orc.SCALE_LEAST_SQUARES:
+        m = orc.encode(x, 16, 4, 2, rotate, SEED)
+        for f in ("a_codes", "a_meta", "r_codes", "r_meta", "r_coef", "a_eflag", "r_eflag", "r_mflag", "r_cflag"):
+            assert np.array_equal(getattr(e, f), getattr(m, f)), f
