@@ -135,6 +135,9 @@ bool on_cache_device(const rq_cache *c) {
 // Among the admissible split counts the one with the least wave-quantised
 // work (waves x tokens of the largest CTA, plus a fixed per-CTA cost) is
 // taken, waves counted from the kernel's measured occupancy.
+#ifndef RQ_SPLIT_OVERHEAD_TILES
+#define RQ_SPLIT_OVERHEAD_TILES 2
+#endif
 void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *chunk) {
     if (T <= 0) {
         *S = 0;
@@ -151,13 +154,19 @@ void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *
         const int ss = s;
         const int slots = std::max(1, c->occ[which][ch / kTokTile - 1] * c->sms);
         const long waves = ((long)ss * units + slots - 1) / slots;
-        const long cost = waves * (ch + 2 * kTokTile);
+        const long cost = waves * (ch + RQ_SPLIT_OVERHEAD_TILES * kTokTile);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best_s = ss;
             best_ch = ch;
         }
     }
+#ifdef RQ_SPLIT_FORCE_S
+    if (RQ_SPLIT_FORCE_S >= s_lo && RQ_SPLIT_FORCE_S <= std::max(s_lo, s_hi)) {
+        best_s = RQ_SPLIT_FORCE_S;
+        best_ch = (nt + best_s - 1) / best_s * kTokTile;
+    }
+#endif
     *S = best_s;
     *chunk = best_ch;
 }
