@@ -360,7 +360,9 @@ class Cache:
         """Logical records of (layer, loop) as numpy arrays:
         codes [2][B][H][len][bytes], meta [2][B][H][len][2d/g], coef [2][B][H][len] (uint16, residual loops)."""
         cfg = self.cfg
-        anchor = (loop % self.Lg) == self.Lg - 1
+        j = loop % self.Lg
+        # the anchor record holds the group's last loop, or its first under the chained reference
+        anchor = j == (0 if cfg.anchor_mode else self.Lg - 1)
         n = self.length(layer, loop // self.Lg)
         bits = cfg.anchor_bits if anchor else cfg.resid_bits
         codes = np.zeros((2, self.B, self.H, n, HEAD_DIM * bits // 8), np.uint8)

@@ -26,8 +26,8 @@ struct rq_cache {
     // not touched by any append still in flight
     std::vector<int> wstart;
     std::vector<uint32_t> sigma;   // [layer][4]: sign bits of the layer's rotation
-    // resident CTAs per SM for chunk = 64 * (i + 1): [0] anchor loops, [1] residual loops
-    int occ[2][kMaxChunk / kTokTile];
+    // resident CTAs per SM for chunk = 64 * (i + 1), by residual records read (0 .. kMaxChain)
+    int occ[kMaxChain + 1][kMaxChunk / kTokTile];
     // split partials of rq_prefill_attn, allocated on first use and grown on demand
     float *prefill_ws = nullptr;
     size_t prefill_ws_floats = 0;
@@ -339,11 +339,14 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
         const int G = cfg->num_q_heads / cfg->num_kv_heads;
         for (int i = 0; i < kMaxChunk / kTokTile; i++) {
             const int ch = kTokTile * (i + 1);
-            if (cfg->format == RQ_FMT_BF16) {
-                c->occ[0][i] = c->occ[1][i] = decode_bf16_occupancy(G, ch);
-            } else {
-                c->occ[0][i] = decode_rq_occupancy(G, cfg->anchor_bits, cfg->resid_bits, false, cfg->group_size, ch);
-                c->occ[1][i] = decode_rq_occupancy(G, cfg->anchor_bits, cfg->resid_bits, true, cfg->group_size, ch);
+            for (int nr = 0; nr <= kMaxChain; nr++) {
+                if (cfg->format == RQ_FMT_BF16)
+                    c->occ[nr][i] = decode_bf16_occupancy(G, ch);
+                else if (nr <= 1 || (cfg->anchor_mode == 1 && nr < cfg->loops_per_group &&
+                                     decode_rq_supported(cfg->anchor_bits, cfg->resid_bits, nr)))
+                    c->occ[nr][i] = decode_rq_occupancy(G, cfg->anchor_bits, cfg->resid_bits, nr, cfg->group_size, ch);
+                else
+                    c->occ[nr][i] = 1;
             }
         }
         cudaGetLastError();
@@ -493,7 +496,6 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     a.rotate = cfg.rotate;
     a.tail_cap = L.tail_cap;
     std::memcpy(a.sigma, &c->sigma[(size_t)layer * 4], sizeof(a.sigma));
-    bool resid = false;
     if (bf16) {
         a.T = c->len[(size_t)layer * cfg.num_loops + loop];
         fill_lens(seq_lens(c, (size_t)layer * cfg.num_loops + loop), cfg.batch, &a.seqT);
@@ -514,20 +516,23 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
             a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
             a.tail_v = (const uint16_t *)tail_ptr(c, layer, group, j, 1);
         }
+        // residual records read: the loop's own (shared reference), or the
+        // chain of records 0 .. slot (chained reference)
         const int slot = record_slot(L, loop);
-        if (slot >= 0) {
-            if (cfg.anchor_mode == 1) return RQ_ERR_UNSUPPORTED;   // chained reference: rq_decode_attn_chain
-            resid = true;
-            a.vmax_r = vmax_ptr(c, layer, group, slot);
+        const int r0 = cfg.anchor_mode == 1 ? 0 : slot;
+        a.nr = slot < 0 ? 0 : slot - r0 + 1;
+        if (!decode_rq_supported(cfg.anchor_bits, cfg.resid_bits, a.nr)) return RQ_ERR_UNSUPPORTED;
+        for (int r = 0; r < a.nr; r++) {
+            a.vmax_r[r] = vmax_ptr(c, layer, group, r0 + r);
             for (int kv = 0; kv < 2; kv++) {
-                a.r_codes[kv] = resid_codes(c, layer, group, slot, kv);
-                a.r_meta[kv] = resid_meta(c, layer, group, slot, kv);
-                a.r_coef[kv] = (const uint16_t *)resid_coef(c, layer, group, slot, kv);
+                a.r_codes[r][kv] = resid_codes(c, layer, group, r0 + r, kv);
+                a.r_meta[r][kv] = resid_meta(c, layer, group, r0 + r, kv);
+                a.r_coef[r][kv] = (const uint16_t *)resid_coef(c, layer, group, r0 + r, kv);
             }
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
-    choose_splits(c, a.T, units, resid ? 1 : 0, &a.S, &a.chunk);
+    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, &a.S, &a.chunk);
     if (partials) {
         a.splits_max = std::max(a.S, 1);
         if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;
@@ -553,12 +558,12 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         a.n_new = app_n;
         a.tail_pos = nt;
         a.n_tail = nt + app_n;
-        int s = cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st));
+        int s = cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, st));
         if (s == RQ_OK) nt += app_n;
         return s;
     }
     if (!bf16 && a.S > 0)   // the decode kernel merges its splits and the tail itself
-        return cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, resid, st));
+        return cuda_status(launch_decode_rq(a, cfg.anchor_bits, cfg.resid_bits, st));
     if (bf16 && a.S > 0) {
         cudaError_t e = launch_decode_bf16(a, st);
         if (e != cudaSuccess) return RQ_ERR_CUDA;

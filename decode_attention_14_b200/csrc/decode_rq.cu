@@ -127,16 +127,25 @@ __device__ __forceinline__ unsigned long long global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+#ifndef RQ_POLLS_PER_CHECK
+#define RQ_POLLS_PER_CHECK 4
+#endif
 // Bounded wait on an mbarrier phase; gives up after kWaitNs or as soon as
 // another warp of the CTA has given up.  SLEEP_NS > 0 backs off between
-// polls (for waits whose latency does not matter).
+// polls (for waits whose latency does not matter).  The abort flag and the
+// clock are checked once per RQ_POLLS_PER_CHECK polls: a poll is two
+// instructions, the checks several more, and waiting warps share the
+// schedulers with working ones.
 template <unsigned SLEEP_NS = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (;;) {
-        if (SLEEP_NS) __nanosleep(SLEEP_NS);
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll
+        for (int i = 0; i < RQ_POLLS_PER_CHECK; i++) {
+            if (SLEEP_NS) __nanosleep(SLEEP_NS);
+            if (mbar_try_wait(bar, parity)) return true;
+        }
         if (*abort_flag) return false;
         if (global_ns() - t0 > kWaitNs) return false;
     }
@@ -328,25 +337,31 @@ __device__ __forceinline__ float fixed_scale(float bound, int top) {
 // back to back in a byte ring (an item never straddles its end), so the
 // number in flight follows their size: about 4 K items, 7 anchor V items or
 // 12 residual V items at once.
-template <int BA, int BR, int GS, bool RESID>
+template <int BA, int BR, int GS, int NR>
 struct Plan {
+    static constexpr bool RESID = NR > 0;
     static constexpr int A_C = 16 * BA;              // anchor codes per record
     static constexpr int R_C = 16 * BR;              // residual codes per record
     static constexpr int MR = 2 * (kHeadDim / GS);   // meta bytes per record
-    // K item: anchor codes | anchor meta | residual codes | residual meta | coefficients
+    // K item: anchor codes | anchor meta | then per residual record k of the
+    // chain: codes | meta | coefficients
     static constexpr int K_AM = kItem * A_C;
-    static constexpr int K_RC = K_AM + kItem * MR;
-    static constexpr int K_RM = K_RC + (RESID ? kItem * R_C : 0);
-    static constexpr int K_CF = K_RM + (RESID ? kItem * MR : 0);
-    static constexpr int K_BYTES = K_CF + (RESID ? kItem * 2 : 0);
+    static constexpr int K_R0 = K_AM + kItem * MR;
+    static constexpr int K_RS = kItem * (R_C + MR + 2);
+    __host__ __device__ static constexpr int K_RC(int k) { return K_R0 + k * K_RS; }
+    __host__ __device__ static constexpr int K_RM(int k) { return K_RC(k) + kItem * R_C; }
+    __host__ __device__ static constexpr int K_CF(int k) { return K_RM(k) + kItem * MR; }
+    static constexpr int K_BYTES = K_R0 + NR * K_RS;
     // V items: codes | meta, anchor items then residual items
     static constexpr int VA_M = kItem * A_C;
     static constexpr int VA_BYTES = VA_M + kItem * MR;
     static constexpr int VR_M = kItem * R_C;
     static constexpr int VR_BYTES = VR_M + kItem * MR;
-    static constexpr int RING = kRingBytes;
+    // at least two K items in flight
+    static constexpr int RING = 2 * K_BYTES > kRingBytes ? 2 * K_BYTES : kRingBytes;
     static_assert(K_BYTES % 128 == 0 && VA_BYTES % 128 == 0 && VR_BYTES % 128 == 0, "item alignment");
     static_assert(K_BYTES <= RING && VA_BYTES <= RING, "ring too small");
+    // pass 0: K items; pass 1: anchor V items; pass 2 + k: residual V items of record k
     __host__ __device__ static constexpr int item_bytes(int pass) {
         return pass == 0 ? K_BYTES : pass == 1 ? VA_BYTES : VR_BYTES;
     }
@@ -355,23 +370,30 @@ struct Plan {
         off += cur;
         return off + next > RING ? 0 : off;
     }
-    // then: V coefficients [chunk] (RESID), logits/p [GK][chunk], p*s_hat [GK][chunk]
+    // then: V coefficients [NR][chunk], logits -> residual weights of the last
+    // record [GK][chunk], anchor weights [GK][chunk], residual weights of the
+    // other records [NR - 1][GK][chunk]
     __host__ __device__ static int coef_bytes(int chunk) { return RESID ? (chunk * 2 + 127) / 128 * 128 : 0; }
     __host__ __device__ static size_t smem(int GK, int chunk) {
-        return (size_t)RING + coef_bytes(chunk) + (size_t)2 * GK * chunk * sizeof(float);
+        return (size_t)RING + (size_t)NR * coef_bytes(chunk) +
+               (size_t)(1 + (NR > 1 ? NR : 1)) * GK * chunk * sizeof(float);
     }
 };
 
-template <int GK, int BA, int BR, int GS, bool RESID>
+// NR: residual records the loop's reconstruction reads (0 for the anchor's
+// own loop, 1 for the shared reference, 1..3 along a chained reference).
+template <int GK, int BA, int BR, int GS, int NR>
 __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) decode_rq_kernel(const DecodeArgs a) {
-    using P = Plan<BA, BR, GS, RESID>;
+    using P = Plan<BA, BR, GS, NR>;
+    constexpr bool RESID = NR > 0;
+    constexpr int NW = NR > 1 ? NR : 1;   // residual weight arrays
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kSlots];
     __shared__ __align__(8) uint64_t bar_empty[kSlots];
     __shared__ __align__(8) uint64_t bar_cf;
     __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
     __shared__ int s_abort, s_last;
-    __shared__ unsigned s_cfmax;
+    __shared__ unsigned s_cfmax[NW];
     __shared__ float s_q[GK][2][kHeadDim];
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
     __shared__ int s_qsum[GK][2][8];                             // sum of each segment's fixed-point q
@@ -388,9 +410,12 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int ntiles = (n + kTile - 1) / kTile;
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
-    const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);        // V coefficients
-    float *s_sc = reinterpret_cast<float *>(smem + P::RING + P::coef_bytes(a.chunk));  // [GK][chunk] logits -> p
-    float *s_P = s_sc + GK * a.chunk;                                                  // [GK][chunk] p * s_hat
+    const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);   // V coefficients [NR][cstride]
+    const int cstride = P::coef_bytes(a.chunk) / 2;
+    float *s_sc = reinterpret_cast<float *>(smem + P::RING + NR * P::coef_bytes(a.chunk));  // logits -> weights
+    float *s_P = s_sc + GK * a.chunk;                        // [GK][chunk] anchor weights
+    // residual weights of record k: s_sc for the last one, s_P + (k + 1) * GK * chunk for the others
+    auto s_W = [&](int k) { return k == NR - 1 ? s_sc : s_P + (size_t)(k + 1) * GK * a.chunk; };
 
     if (tid == 0) {
         for (int i = 0; i < kSlots; i++) {
@@ -400,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         mbar_init(&bar_cf, 1);
         mbar_init(&bar_cfmax, 31);
         s_abort = 0;
-        s_cfmax = 0;
+        for (int k = 0; k < NW; k++) s_cfmax[k] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -421,8 +446,11 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             };
             dep(RESID && ntiles > 0 ? n : 0);
             if (RESID && ntiles > 0) {
-                mbar_expect_tx(&bar_cf, (uint32_t)(ntiles * kTile * 2));
-                bulk_g2s(smem + P::RING, a.r_coef[1] + tok0, (uint32_t)(ntiles * kTile * 2), &bar_cf);
+                mbar_expect_tx(&bar_cf, (uint32_t)(NR * ntiles * kTile * 2));
+#pragma unroll
+                for (int k = 0; k < NR; k++)
+                    bulk_g2s(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1] + tok0,
+                             (uint32_t)(ntiles * kTile * 2), &bar_cf);
             } else if (RESID) {
                 mbar_arrive(&bar_cf);   // nothing to fetch
             }
@@ -433,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // older item starting below virt + bytes - RING must have been
             // released, and at most kSlots items may be outstanding.  The
             // loop keeps all of this in running counters (no division).
-            const int npass = RESID ? 3 : 2;
+            const int npass = 2 + NR;
             int it = 0, virt = 0, phys = 0;
             const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // items per pass
             int rel = 0, vrel = 0, rphys = 0, ritem = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
@@ -451,13 +479,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     c1 = a.a_meta[1] + tok0 * P::MR;
                     cstride = P::A_C * kItem;
                 } else {
-                    c0 = a.r_codes[1] + tok0 * P::R_C;
-                    c1 = a.r_meta[1] + tok0 * P::MR;
+                    c0 = a.r_codes[pass - 2][1] + tok0 * P::R_C;
+                    c1 = a.r_meta[pass - 2][1] + tok0 * P::MR;
                     cstride = P::R_C * kItem;
                 }
-                const uint8_t *r0 = RESID ? a.r_codes[0] + tok0 * P::R_C : nullptr;
-                const uint8_t *r1 = RESID ? a.r_meta[0] + tok0 * P::MR : nullptr;
-                const uint8_t *r2 = RESID ? reinterpret_cast<const uint8_t *>(a.r_coef[0] + tok0) : nullptr;
                 for (int j = 0; j < nitems; j++, it++) {
                     if (phys + bytes > P::RING) {
                         virt += P::RING - phys;
@@ -494,16 +519,15 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     uint8_t *st = ring + phys;
                     uint64_t *bar = &bar_full[it % kSlots];
                     if (pass == 0) {
-                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + (RESID ? P::R_C + P::MR + 2 : 0))));
+                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2))));
                         bulk_g2s(st, c0, toks * P::A_C, bar);
                         bulk_g2s(st + P::K_AM, c1, toks * P::MR, bar);
-                        if (RESID) {
-                            bulk_g2s(st + P::K_RC, r0, toks * P::R_C, bar);
-                            bulk_g2s(st + P::K_RM, r1, toks * P::MR, bar);
-                            bulk_g2s(st + P::K_CF, r2, toks * 2, bar);
-                            r0 += kItem * P::R_C;
-                            r1 += kItem * P::MR;
-                            r2 += kItem * 2;
+                        const size_t tj = tok0 + (size_t)j * kItem;
+#pragma unroll
+                        for (int k = 0; k < NR; k++) {
+                            bulk_g2s(st + P::K_RC(k), a.r_codes[k][0] + tj * P::R_C, toks * P::R_C, bar);
+                            bulk_g2s(st + P::K_RM(k), a.r_meta[k][0] + tj * P::MR, toks * P::MR, bar);
+                            bulk_g2s(st + P::K_CF(k), a.r_coef[k][0] + tj, toks * 2, bar);
                         }
                     } else {
                         const int cb = pass == 1 ? P::A_C : P::R_C;
@@ -529,12 +553,15 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // coefficients (for the weights' fixed point), ready before the
             // softmax needs it
             griddep_wait_then_release();
-            unsigned m = 0;
             if (RESID && mbar_wait<64>(&bar_cf, 0, &s_abort)) {
-                const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING);
-                for (int t = lane - 1; t < n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
+#pragma unroll
+                for (int k = 0; k < NR; k++) {
+                    const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING + k * P::coef_bytes(a.chunk));
+                    unsigned m = 0;
+                    for (int t = lane - 1; t < n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
+                    atomicMax(&s_cfmax[k], m);
+                }
             }
-            atomicMax(&s_cfmax, m);
             mbar_arrive(&bar_cfmax);
         }
         return;
@@ -544,7 +571,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     griddep_wait_then_release();
     // upper bounds of this stream's V scales (anchor; the loop's residual)
     const float vA = e4m3_to_f32((uint32_t)a.vmax_a[bh]);
-    const float vR = RESID ? e4m3_to_f32((uint32_t)a.vmax_r[bh]) : 0.f;
+    float vR[NW];
+#pragma unroll
+    for (int k = 0; k < NW; k++) vR[k] = RESID ? e4m3_to_f32((uint32_t)a.vmax_r[k][bh]) : 0.f;
     if (a.n_new > 0 && split == 0) {
         // fused append: this unit's new tail rows (K and V, 16-byte vectors);
         // the fence before the arrival count below publishes them to the
@@ -668,23 +697,21 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 const Seg<BA> ca = lds_seg<BA>(st + tok * P::A_C + seg * (2 * BA));
                 const float2 ma =
                     meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_AM + tok * P::MR + 2 * mg));
-                float shat = 1.f;
-                Seg<BR> cr;
-                float2 mr = make_float2(0.f, 0.f);
-                if (RESID) {
-                    cr = lds_seg<BR>(st + P::K_RC + tok * P::R_C + seg * (2 * BR));
-                    mr = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_RM + tok * P::MR + 2 * mg));
-                    shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + P::K_CF + 2 * tok));
-                }
 #pragma unroll
-                for (int gq = 0; gq < GK; gq++) {
-                    const float A = fmaf(ma.y, QA[gq], ma.x * __int2float_rn(dot_seg<BA>(ca, qA[gq])));
-                    float v = A;
-                    if (RESID) {
+                for (int gq = 0; gq < GK; gq++)
+                    part[u][gq][k] = fmaf(ma.y, QA[gq], ma.x * __int2float_rn(dot_seg<BA>(ca, qA[gq])));
+                // along the chain: v <- s_hat_k v + (R q) . y_hat_k  (one step for the shared reference)
+#pragma unroll
+                for (int r = 0; r < NR; r++) {
+                    const Seg<BR> cr = lds_seg<BR>(st + P::K_RC(r) + tok * P::R_C + seg * (2 * BR));
+                    const float2 mr =
+                        meta_pair(*reinterpret_cast<const uint16_t *>(st + P::K_RM(r) + tok * P::MR + 2 * mg));
+                    const float shat = bf16_to_f32(*reinterpret_cast<const uint16_t *>(st + P::K_CF(r) + 2 * tok));
+#pragma unroll
+                    for (int gq = 0; gq < GK; gq++) {
                         const float R = fmaf(mr.y, QR[gq], mr.x * __int2float_rn(dot_seg<BR>(cr, qR[gq])));
-                        v = fmaf(shat, A, R);
+                        part[u][gq][k] = fmaf(shat, part[u][gq][k], R);
                     }
-                    part[u][gq][k] = v;
                 }
             }
         }
@@ -734,22 +761,34 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         s_abort = 1;
         atomicExch(a.err, 3);
     }
-    const float cA = fixed_scale(RESID ? bf16_to_f32((uint16_t)s_cfmax) * vA : vA, kWeightTop);
-    const float cR = fixed_scale(vR, kWeightTop);
-    // p = exp2(z - M) (residual V weight) and P = p * s_hat(V) (anchor V
-    // weight), zero beyond the chunk's tokens, stored with their scales
+    // record k's V weight is p times the product of the V coefficients of
+    // the records after it on the chain (1 for the last), the anchor's p
+    // times the product of all of them; bounds from the coefficients' maxima
+    float cR[NW];
+    float cfprod = 1.f;
+#pragma unroll
+    for (int k = NW - 1; k >= 0; k--) {
+        cR[k] = fixed_scale(cfprod * vR[k], kWeightTop);
+        if (RESID) cfprod *= bf16_to_f32((uint16_t)s_cfmax[k]);
+    }
+    const float cA = fixed_scale(cfprod * vA, kWeightTop);
+    // p = exp2(z - M), zero beyond the chunk's tokens; the weights stored with their scales
     float lsum[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
     for (int t = tid; t < ntiles * kTile; t += kConsumers) {
         const bool valid = t < n;
-        const float shv = RESID ? bf16_to_f32(s_cf[t]) : 1.f;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
             const float p = valid ? exp2f(s_sc[gq * a.chunk + t] - M[gq]) : 0.f;
             lsum[gq] += p;
-            s_sc[gq * a.chunk + t] = p * cR;
-            s_P[gq * a.chunk + t] = p * shv * cA;
+            float pr = p;
+#pragma unroll
+            for (int k = NR - 1; k >= 0; k--) {
+                s_W(k)[gq * a.chunk + t] = pr * cR[k];
+                pr *= bf16_to_f32(s_cf[k * cstride + t]);
+            }
+            s_P[gq * a.chunk + t] = pr * cA;
         }
     }
 #pragma unroll
@@ -765,10 +804,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         Lsum[gq] = s_red[0][GK + gq] + s_red[1][GK + gq] + s_red[2][GK + gq] + s_red[3][GK + gq];
 
     // ------------------------------------------------------------ pass 2: values (anchor, then residual)
-    const int npass = RESID ? 2 : 1;
+    const int npass = 1 + NR;
     for (int vp = 0; vp < npass; vp++) {
-        const float cW = vp == 0 ? cA : cR;   // weights in s_P / s_sc already carry it
-        const float *wsrc = vp == 0 ? s_P : s_sc;
+        const float cW = vp == 0 ? cA : cR[vp - 1];   // the weights already carry it
+        const float *wsrc = vp == 0 ? s_P : s_W(vp - 1);
         unsigned accLo[GK][16];
         int accHi[GK][16];
         float mS[GK];
@@ -887,7 +926,17 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             r2.y = (hb16 ? r1[5] : r1[1]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[1] : r1[5], 16);
             r2.z = (hb16 ? r1[6] : r1[2]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[2] : r1[6], 16);
             r2.w = (hb16 ? r1[7] : r1[3]) + __shfl_xor_sync(0xffffffffu, hb16 ? r1[3] : r1[7], 16);
-            *reinterpret_cast<float4 *>(&s_acc[warp][gq][vp][seg * 16 + (hb8 ? 8 : 0) + (hb16 ? 4 : 0)]) = r2;
+            // residual records after the first add into the rotated basis's slot
+            float4 *dst = reinterpret_cast<float4 *>(
+                &s_acc[warp][gq][vp > 0 ? 1 : 0][seg * 16 + (hb8 ? 8 : 0) + (hb16 ? 4 : 0)]);
+            if (vp >= 2) {
+                const float4 o = *dst;
+                r2.x += o.x;
+                r2.y += o.y;
+                r2.z += o.z;
+                r2.w += o.w;
+            }
+            *dst = r2;
         }
     }
 
@@ -953,86 +1002,96 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     }
 }
 
-template <int GK, int BA, int BR, int GS, bool RESID>
+template <int GK, int BA, int BR, int GS, int NR>
 cudaError_t configure() {
     static bool done[kMaxDevices] = {};   // the largest dynamic shared memory any launch can ask for
     return once_per_device(done, [] {
-        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, RESID>,
+        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, NR>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)Plan<BA, BR, GS, RESID>::smem(GK, kMaxChunk));
+                                    (int)Plan<BA, BR, GS, NR>::smem(GK, kMaxChunk));
     });
 }
 
-template <int GK, int BA, int BR, int GS, bool RESID>
+template <int GK, int BA, int BR, int GS, int NR>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
     const dim3 grid(a.S, a.H, a.B * (a.G / GK));
-    cudaError_t e = configure<GK, BA, BR, GS, RESID>();
+    cudaError_t e = configure<GK, BA, BR, GS, NR>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = grid;
     lc.blockDim = dim3(kThreads);
-    lc.dynamicSmemBytes = Plan<BA, BR, GS, RESID>::smem(GK, a.chunk);
+    lc.dynamicSmemBytes = Plan<BA, BR, GS, NR>::smem(GK, a.chunk);
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = RQ_DECODE_PDL ? 1 : 0;
-    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, RESID>, a);
+    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, NR>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int GK, int BA, int BR, int GS, bool RESID>
+template <int GK, int BA, int BR, int GS, int NR>
 int occupancy_t(int chunk) {
-    if (configure<GK, BA, BR, GS, RESID>() != cudaSuccess) return 1;
+    if (configure<GK, BA, BR, GS, NR>() != cudaSuccess) return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, RESID>, kThreads,
-                                                      Plan<BA, BR, GS, RESID>::smem(GK, chunk)) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, NR>, kThreads,
+                                                      Plan<BA, BR, GS, NR>::smem(GK, chunk)) != cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
 }
 
-// Variant dispatch: one instantiation per (q heads per CTA, bits, group, loop kind).
+// Variant dispatch: one instantiation per (q heads per CTA, bits, group,
+// residual records read).  Chains of two or three records (the chained
+// reference) are built for the method's format, INT4 anchor / INT2 residuals.
 template <int GK, int GS>
 struct Dispatch {
     template <typename F>
-    static auto run(int ba, int br, bool resid, F f) {
-        if (!resid) return ba == 4 ? f.template go<GK, 4, 2, GS, false>() : f.template go<GK, 2, 2, GS, false>();
-        if (ba == 4 && br == 2) return f.template go<GK, 4, 2, GS, true>();
-        if (ba == 4 && br == 4) return f.template go<GK, 4, 4, GS, true>();
-        if (ba == 2 && br == 2) return f.template go<GK, 2, 2, GS, true>();
-        return f.template go<GK, 2, 4, GS, true>();
+    static auto run(int ba, int br, int nr, F f) {
+        if (nr == 0) return ba == 4 ? f.template go<GK, 4, 2, GS, 0>() : f.template go<GK, 2, 2, GS, 0>();
+        if (nr == 2) return f.template go<GK, 4, 2, GS, 2>();
+        if (nr == 3) return f.template go<GK, 4, 2, GS, 3>();
+        if (ba == 4 && br == 2) return f.template go<GK, 4, 2, GS, 1>();
+        if (ba == 4 && br == 4) return f.template go<GK, 4, 4, GS, 1>();
+        if (ba == 2 && br == 2) return f.template go<GK, 2, 2, GS, 1>();
+        return f.template go<GK, 2, 4, GS, 1>();
     }
 };
 
 struct LaunchF {
     const DecodeArgs *a;
     cudaStream_t st;
-    template <int GK, int BA, int BR, int GS, bool RESID>
-    cudaError_t go() const { return launch_t<GK, BA, BR, GS, RESID>(*a, st); }
+    template <int GK, int BA, int BR, int GS, int NR>
+    cudaError_t go() const { return launch_t<GK, BA, BR, GS, NR>(*a, st); }
 };
 struct OccF {
     int chunk;
-    template <int GK, int BA, int BR, int GS, bool RESID>
-    int go() const { return occupancy_t<GK, BA, BR, GS, RESID>(chunk); }
+    template <int GK, int BA, int BR, int GS, int NR>
+    int go() const { return occupancy_t<GK, BA, BR, GS, NR>(chunk); }
 };
 
 template <typename F>
-auto dispatch(int G, int g, int ba, int br, bool resid, F f) {
-    if (G == 1) return g == 16 ? Dispatch<1, 16>::run(ba, br, resid, f) : Dispatch<1, 32>::run(ba, br, resid, f);
-    return g == 16 ? Dispatch<2, 16>::run(ba, br, resid, f) : Dispatch<2, 32>::run(ba, br, resid, f);
+auto dispatch(int G, int g, int ba, int br, int nr, F f) {
+    if (G == 1) return g == 16 ? Dispatch<1, 16>::run(ba, br, nr, f) : Dispatch<1, 32>::run(ba, br, nr, f);
+    return g == 16 ? Dispatch<2, 16>::run(ba, br, nr, f) : Dispatch<2, 32>::run(ba, br, nr, f);
 }
 
 }  // namespace
 
-cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st) {
-    // G = 2, 4, 8 run as pairs of query heads per CTA
-    return dispatch(a.G, a.g, ba, br, resid, LaunchF{&a, st});
+bool decode_rq_supported(int ba, int br, int nr) {
+    return nr >= 0 && nr <= kMaxChain && (nr <= 1 || (ba == 4 && br == 2));
 }
 
-int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk) {
-    return dispatch(G, g, ba, br, resid, OccF{chunk});
+cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, cudaStream_t st) {
+    // G = 2, 4, 8 run as pairs of query heads per CTA
+    if (!decode_rq_supported(ba, br, a.nr)) return cudaErrorInvalidValue;
+    return dispatch(a.G, a.g, ba, br, a.nr, LaunchF{&a, st});
+}
+
+int decode_rq_occupancy(int G, int ba, int br, int nr, int g, int chunk) {
+    if (!decode_rq_supported(ba, br, nr)) return 1;
+    return dispatch(G, g, ba, br, nr, OccF{chunk});
 }
 
 }  // namespace rq

@@ -125,12 +125,16 @@ struct Bf16StoreArgs {
     int B, H, n, Tp;
 };
 
+constexpr int kMaxChain = 3;   // residual records one decode may chain (the chained reference, groups of 4)
+
 struct DecodeArgs {
     // anchor streams (kv 0 = K, 1 = V)
     const uint8_t *a_codes[2], *a_meta[2];
-    // residual streams (null for the anchor loop)
-    const uint8_t *r_codes[2], *r_meta[2];
-    const uint16_t *r_coef[2];
+    // residual streams of the records the loop's reconstruction reads, in
+    // chain order (one for the shared reference; none for the anchor's own loop)
+    const uint8_t *r_codes[kMaxChain][2], *r_meta[kMaxChain][2];
+    const uint16_t *r_coef[kMaxChain][2];
+    int nr;                   // residual records read
     // BF16 format streams
     const uint16_t *bf[2];
     const uint16_t *q;        // [B][Hq][d] bf16
@@ -142,7 +146,7 @@ struct DecodeArgs {
     // largest FP8 scale byte of the anchor V and (residual loops) the loop's
     // residual V stream of every (sequence, kv head), [B][H]: upper bounds of
     // the V scales, from which the weights' fixed point is chosen
-    const int *vmax_a, *vmax_r;
+    const int *vmax_a, *vmax_r[kMaxChain];
     // committed records below token `stable` are not written by any work
     // that may still run when this kernel starts (see the programmatic
     // launch in api.cpp); records from `stable` on are read only after the
@@ -183,11 +187,13 @@ struct CombineArgs {
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st);
 cudaError_t launch_tail_copy(const TailArgs &a, cudaStream_t st);
 cudaError_t launch_bf16_store(const Bf16StoreArgs &a, cudaStream_t st);
-cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, bool resid, cudaStream_t st);
+// a.nr residual records: 0, 1, or (INT4 anchor / INT2 residuals only) 2-3
+bool decode_rq_supported(int ba, int br, int nr);
+cudaError_t launch_decode_rq(const DecodeArgs &a, int ba, int br, cudaStream_t st);
 cudaError_t launch_decode_bf16(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 // resident CTAs per SM of the decode kernels for a given chunk (tokens per CTA)
-int decode_rq_occupancy(int G, int ba, int br, bool resid, int g, int chunk);
+int decode_rq_occupancy(int G, int ba, int br, int nr, int g, int chunk);
 int decode_bf16_occupancy(int G, int chunk);
 
 // rq_decode_attn with the split partials and the combine counters in

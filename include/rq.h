@@ -313,10 +313,13 @@ int rq_cache_truncate_seq(rq_cache *cache, int layer, int group, int seq, int ne
  * Copy the committed records of (layer, loop) to host memory in the logical
  * record format (for tests and inspection; synchronises `stream`):
  * (len = rq_cache_length; rows past a shorter sequence's length hold no token of it)
- *   anchor loop:   host_codes [2][B][H_kv][len][d*anchor_bits/8]  (K then V)
+ * The loop's own record is the anchor record for the group's last loop
+ * (anchor_mode 0) or its first loop (anchor_mode 1), a residual record for
+ * the others; the host buffers must be sized for that kind:
+ *   anchor record: host_codes [2][B][H_kv][len][d*anchor_bits/8]  (K then V)
  *                  host_meta  [2][B][H_kv][len][2*d/g]  ([scale, min] per group)
  *                  host_coef  unused (may be NULL)
- *   other loops:   host_codes [2][B][H_kv][len][d*resid_bits/8]
+ *   residual:      host_codes [2][B][H_kv][len][d*resid_bits/8]
  *                  host_meta  [2][B][H_kv][len][2*d/g]
  *                  host_coef  [2][B][H_kv][len] BF16
  * Code packing: element i at byte i*b/8, bit (i*b)%8, LSB first.

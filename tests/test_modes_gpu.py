@@ -79,5 +79,17 @@ def test_chained_reference_records(scale_mode, rotate):
     l >= 1 a residual against the reconstruction of loop l - 1."""
     bt = H.build(layers=1, loops=4, Lg=4, B=2, T=170, H=2, Hq=4, n_tail=1, rotate=rotate,
                  seed=0x5EEDB200 + scale_mode, anchor_mode=rq.ANCHOR_CHAINED, scale_mode=scale_mode)
-    _check(bt, strict=not rotate, loops=[0])
+    _check(bt, strict=not rotate, loops=range(4))
+    # records read per decode call grow along the chain: anchor, then 1, 2, 3 residuals
+    per = [bt.cache.decode_bytes(0, loop) for loop in range(4)]
+    assert per[0] < per[1] < per[2] < per[3]
+    bt.cache.close()
+
+
+@pytest.mark.parametrize("T,Hq", [(1000, 2), (3000, 8)])
+def test_chained_reference_longer(T, Hq):
+    """Longer caches (several splits, a ragged last tile) and GQA 4."""
+    bt = H.build(layers=1, loops=4, Lg=4, B=1, T=T, H=2, Hq=Hq, n_tail=2, chunk=256, seed=0x5EEDB300 + T,
+                 anchor_mode=rq.ANCHOR_CHAINED)
+    _check(bt, strict=False, loops=range(4))
     bt.cache.close()
