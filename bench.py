@@ -177,10 +177,17 @@ def run_ours(args, cfgd, rank, world, local_rank):
     loops, Lg, B, T, H, Hq = cfgd["loops"], cfgd["Lg"], cfgd["B"], cfgd["T"], cfgd["H"], cfgd["Hq"]
     seed = rank_seed(CONFIG_SEED[name], rank)
     fmt = rq.RQ_FMT_BF16 if args.bf16 else rq.RQ_FMT_RESIDUAL
+    paging = {}
+    if args.paged:
+        # 128-token blocks, the pool sized to the batch, allocation scattered over it
+        paging = dict(block_tokens=128, num_blocks=B * ((T + 127) // 128) + 8)
     cfg = rq.make_config(num_layers=layers, num_loops=loops, loops_per_group=Lg, batch=B, max_tokens=T,
                          max_tail_tokens=FILL_CHUNK, num_kv_heads=H, num_q_heads=Hq, group_size=cfgd["g"],
-                         anchor_bits=cfgd["ba"], resid_bits=cfgd["br"], rotate=True, format=fmt, seed=0xA11CE)
+                         anchor_bits=cfgd["ba"], resid_bits=cfgd["br"], rotate=True, format=fmt, seed=0xA11CE,
+                         anchor_mode=rq.ANCHOR_CHAINED if args.chained else rq.ANCHOR_LAST, **paging)
     cache = rq.Cache(cfg, device=dev)
+    if args.paged:
+        cache.shuffle_free_blocks(0x5EED)
     T0 = T - 1
     groups = loops // Lg
     stream = torch.cuda.current_stream(dev)
@@ -395,6 +402,8 @@ def run_ours(args, cfgd, rank, world, local_rank):
                   else "bf16 in, fp32 math"),
         "data": "synthetic (seeded; anchor N(0,1) with 4 outlier channels x10, loops c*anchor+sigma*N(0,1))",
         "config": dict(workload_config(name, cfgd, layers, world), **{
+                   "paged": "128-token blocks, shuffled pool" if args.paged else None,
+                   "reference": "chained (previous loop)" if args.chained else "shared (last loop)",
                    "step_calls": ("rq_append + rq_decode_attn_bf16" if args.bf16 else
                                   "rq_append + rq_decode_attn" if args.separate_append else "rq_append_decode_attn"),
                    "l2": "inputs larger than L2: %.1f GB of records read per step, loop-major over %d layers"
@@ -404,6 +413,10 @@ def run_ours(args, cfgd, rank, world, local_rank):
                         "bytes_per_step": int(step_decode_bytes), "gbs": round(achieved, 1),
                         "tokens_per_s_decode_only": round(world * B * args.steps / (dec_ms / 1e3), 2)},
         "append": {"ms_per_step_est": round(max(ms_step - dec_ms / args.steps, 0.0), 4)},
+        # records each loop's decode reads per token-head and K|V side: the anchor alone,
+        # or the anchor and residuals (one for the shared reference, the chain for the other)
+        "records_read_per_loop": [1 if args.bf16 else lp % Lg + 1 if args.chained else 2 if lp % Lg < Lg - 1 else 1
+                                  for lp in range(loops)],
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": measured_traffic(name) if not args.bf16 else None,
                      "algorithmic_bytes_per_launch": int(step_decode_bytes / ncalls),
@@ -722,6 +735,29 @@ def run_prefill(args):
     return rows
 
 
+def run_all_configs(args):
+    """One JSON line per workload on one GPU, each measured as the headline
+    is (same step, timed graph, decode-only graph): the compressed cache and
+    the BF16 comparison cache for Ouro 8k b4 and 16k b2/b4, the deep
+    recurrence, and the Ouro 8k b4 step on a paged cache and with the
+    chained reference."""
+    import copy
+    runs = [("ouro8k_b4", {}), ("ouro8k_b4", {"bf16": True}), ("long16k_b2", {}), ("long16k_b2", {"bf16": True}),
+            ("long16k_b4", {}), ("deep", {}), ("ouro8k_b4", {"paged": True}), ("ouro8k_b4", {"chained": True})]
+    for name, flags in runs:
+        a = copy.copy(args)
+        a.config, a.bf16, a.paged, a.chained = name, False, False, False
+        a.no_e2e, a.no_clocks = True, True
+        for k, v in flags.items():
+            setattr(a, k, v)
+        res, cache, _ = run_ours(a, CONFIGS[name], 0, 1, 0)
+        print(json.dumps(res), flush=True)
+        cache.close()
+        del cache
+        import torch
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -742,6 +778,12 @@ def main():
                     help="batch x format sweep of the Ouro shape at T=8192 (one JSON line per row)")
     ap.add_argument("--prefill", default="",
                     help="comma-separated chunk sizes: time rq_prefill_attn on the Ouro shape instead")
+    ap.add_argument("--paged", action="store_true", help="records in a pool of 128-token blocks (block tables)")
+    ap.add_argument("--chained", action="store_true",
+                    help="the chained (previous-loop) reference of the ablation instead of the shared anchor")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="one JSON line per workload (Ouro 8k b4, 16k b2/b4, deep; compressed and BF16; paged; "
+                         "chained) instead of the single headline line")
     ap.add_argument("--profile", action="store_true",
                     help="bracket the timed region with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     args = ap.parse_args()
@@ -754,6 +796,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.all_configs:
+        run_all_configs(args)
         return
     if args.prefill:
         run_prefill(args)

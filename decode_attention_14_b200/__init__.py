@@ -108,6 +108,14 @@ def _load() -> ctypes.CDLL:
     L.rq_decode_bytes.argtypes = [vp, i32, i32]
     L.rq_check.restype = i32
     L.rq_check.argtypes = [vp]
+    L.rq_cache_fork_seq.restype = i32
+    L.rq_cache_fork_seq.argtypes = [vp, i32, i32, vp]
+    L.rq_cache_shuffle_free_blocks.restype = i32
+    L.rq_cache_shuffle_free_blocks.argtypes = [vp, ctypes.c_uint64]
+    L.rq_cache_free_blocks.restype = i32
+    L.rq_cache_free_blocks.argtypes = [vp, ctypes.POINTER(i32)]
+    L.rq_cache_seq_blocks.restype = i32
+    L.rq_cache_seq_blocks.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), i32, ctypes.POINTER(i32)]
     return L
 
 
@@ -263,6 +271,28 @@ def rq_check(h) -> int:
     return lib.rq_check(h)
 
 
+def rq_cache_fork_seq(h, src: int, dst: int, stream=None) -> int:
+    return lib.rq_cache_fork_seq(h, src, dst, ctypes.c_void_p(_stream(stream)))
+
+
+def rq_cache_shuffle_free_blocks(h, seed: int) -> int:
+    return lib.rq_cache_shuffle_free_blocks(h, seed)
+
+
+def rq_cache_free_blocks(h) -> int:
+    n = ctypes.c_int(0)
+    _ok(lib.rq_cache_free_blocks(h, ctypes.byref(n)), "rq_cache_free_blocks")
+    return n.value
+
+
+def rq_cache_seq_blocks(h, seq: int) -> list:
+    n = ctypes.c_int(0)
+    _ok(lib.rq_cache_seq_blocks(h, seq, None, 0, ctypes.byref(n)), "rq_cache_seq_blocks")
+    buf = (ctypes.c_int32 * max(n.value, 1))()
+    _ok(lib.rq_cache_seq_blocks(h, seq, buf, n.value, ctypes.byref(n)), "rq_cache_seq_blocks")
+    return list(buf[:n.value])
+
+
 # ------------------------------------------------------------ convenience
 class Cache:
     """Owns one rq_cache handle (and its arena, a torch uint8 tensor, unless
@@ -355,6 +385,18 @@ class Cache:
 
     def check(self) -> None:
         _ok(rq_check(self.h), "rq_check")
+
+    def fork_seq(self, src: int, dst: int, stream=None) -> None:
+        _ok(rq_cache_fork_seq(self.h, src, dst, stream), "rq_cache_fork_seq")
+
+    def shuffle_free_blocks(self, seed: int) -> None:
+        _ok(rq_cache_shuffle_free_blocks(self.h, seed), "rq_cache_shuffle_free_blocks")
+
+    def free_blocks(self) -> int:
+        return rq_cache_free_blocks(self.h)
+
+    def seq_blocks(self, seq: int) -> list:
+        return rq_cache_seq_blocks(self.h, seq)
 
     def export(self, layer: int, loop: int, stream=None):
         """Logical records of (layer, loop) as numpy arrays:

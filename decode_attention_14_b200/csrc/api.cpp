@@ -31,6 +31,12 @@ struct rq_cache {
     // split partials of rq_prefill_attn, allocated on first use and grown on demand
     float *prefill_ws = nullptr;
     size_t prefill_ws_floats = 0;
+    // paged records: host copy of the block table [B][MB] (-1: no block),
+    // reference counts of the physical blocks (forked sequences share
+    // blocks), and the free list (blocks are taken from its back)
+    std::vector<int> table;
+    std::vector<int> ref;
+    std::vector<int> free_blocks;
 };
 
 namespace {
@@ -102,6 +108,136 @@ int *vmax_ptr(const rq_cache *c, int layer, int group, int r) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? RQ_OK : RQ_ERR_CUDA; }
+
+// Token -> record row mapping of the compressed format.
+Pages pages_of(const rq_cache *c) {
+    const Layout &L = c->lay;
+    Pages p;
+    p.table = L.paged ? (const int *)(c->base + L.off_table) : nullptr;
+    p.mb = L.MB;
+    p.bt = L.BT;
+    p.shift = 0;
+    while (L.paged && (1 << p.shift) < L.BT) p.shift++;
+    return p;
+}
+
+// The record arrays inside one (layer, group) block of the arena, as
+// (offset, bytes per record) pairs (the BF16 tails excluded).
+int record_arrays(const Layout &L, size_t *off, int *rec) {
+    int n = 0;
+    for (int kv = 0; kv < 2; kv++) {
+        const size_t a0 = kv * (L.anchor_codes_bytes + L.anchor_meta_bytes);
+        off[n] = a0;
+        rec[n++] = L.rec.a_codes;
+        off[n] = a0 + L.anchor_codes_bytes;
+        rec[n++] = L.rec.meta;
+    }
+    const size_t side = L.resid_codes_bytes + L.resid_meta_bytes + L.resid_coef_bytes;
+    for (int j = 0; j < L.Lg - 1; j++)
+        for (int kv = 0; kv < 2; kv++) {
+            const size_t r0 = L.anchor_block + (size_t)j * L.resid_block + kv * side;
+            off[n] = r0;
+            rec[n++] = L.rec.r_codes;
+            off[n] = r0 + L.resid_codes_bytes;
+            rec[n++] = L.rec.meta;
+            off[n] = r0 + L.resid_codes_bytes + L.resid_meta_bytes;
+            rec[n++] = 2;
+        }
+    return n;
+}
+
+// Device work of block operations collected on the host: block-table
+// entries to set and whole blocks to copy (copy-on-write of shared blocks).
+struct PendingOps {
+    std::vector<std::pair<int, int>> sets;     // (table index, block)
+    std::vector<std::pair<int, int>> copies;   // (source block, destination block)
+};
+
+int flush_ops(rq_cache *c, const PendingOps &ops, cudaStream_t st) {
+    const Layout &L = c->lay;
+    BlockOpsArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.table = (int *)(c->base + L.off_table);
+    a.records = c->base + L.off_records;
+    a.group_block = L.group_block;
+    a.n_groups = L.cfg.num_layers * L.groups;
+    a.n_arrays = record_arrays(L, a.arr_off, a.arr_rec);
+    a.rows_per_block = (size_t)L.cfg.num_kv_heads * L.BT;
+    size_t i = 0, k = 0;
+    while (i < ops.sets.size() || k < ops.copies.size()) {
+        a.n_sets = a.n_copies = 0;
+        for (; i < ops.sets.size() && a.n_sets < kMaxBlockOps; i++) {
+            a.set_idx[a.n_sets] = ops.sets[i].first;
+            a.set_val[a.n_sets++] = ops.sets[i].second;
+        }
+        for (; k < ops.copies.size() && a.n_copies < kMaxBlockOps; k++) {
+            a.copy_src[a.n_copies] = ops.copies[k].first;
+            a.copy_dst[a.n_copies++] = ops.copies[k].second;
+        }
+        if (launch_block_ops(a, st) != cudaSuccess) return RQ_ERR_CUDA;
+    }
+    return RQ_OK;
+}
+
+// Blocks a sequence needs: those holding any committed token of any
+// (layer, group).
+int blocks_needed(const rq_cache *c, int b) {
+    const Layout &L = c->lay;
+    int mx = 0;
+    for (size_t slot = 0; slot < c->len.size(); slot++) mx = std::max(mx, c->seq[slot * L.cfg.batch + b]);
+    return (mx + L.BT - 1) / L.BT;
+}
+
+// Returns blocks k >= keep of sequence b to the pool (host only: the device
+// table keeps stale entries, never read past a sequence's length).
+void release_blocks(rq_cache *c, int b, int keep) {
+    const Layout &L = c->lay;
+    for (int k = keep; k < L.MB; k++) {
+        int &e = c->table[(size_t)b * L.MB + k];
+        if (e < 0) continue;
+        if (--c->ref[e] == 0) c->free_blocks.push_back(e);
+        e = -1;
+    }
+}
+
+// Before tokens [pos0_b, pos0_b + n) of every sequence are written: every
+// block they fall in is allocated, and a block shared with another sequence
+// is first copied (copy-on-write).  Enqueues the table and copy work on st.
+// All or nothing: on CAPACITY (pool exhausted) the host state is restored.
+int prepare_blocks(rq_cache *c, const SeqLens &pos0, int n, cudaStream_t st) {
+    const Layout &L = c->lay;
+    const std::vector<int> table0 = c->table, ref0 = c->ref, free0 = c->free_blocks;
+    PendingOps ops;
+    for (int b = 0; b < L.cfg.batch; b++) {
+        const int k0 = pos0.v[b] / L.BT, k1 = (pos0.v[b] + n - 1) / L.BT;
+        for (int k = k0; k <= k1; k++) {
+            int &e = c->table[(size_t)b * L.MB + k];
+            if (e >= 0 && c->ref[e] == 1) continue;
+            if (c->free_blocks.empty()) {
+                c->table = table0;
+                c->ref = ref0;
+                c->free_blocks = free0;
+                return RQ_ERR_CAPACITY;
+            }
+            const int nb = c->free_blocks.back();
+            c->free_blocks.pop_back();
+            c->ref[nb] = 1;
+            if (e >= 0) {   // shared: copy, then drop this sequence's reference
+                ops.copies.push_back({e, nb});
+                c->ref[e]--;
+            }
+            e = nb;
+            ops.sets.push_back({b * L.MB + k, nb});
+        }
+    }
+    const int s = flush_ops(c, ops, st);
+    if (s != RQ_OK) {
+        c->table = table0;
+        c->ref = ref0;
+        c->free_blocks = free0;
+    }
+    return s;
+}
 
 // per-sequence lengths of length slot `slot` (= layer * groups + group, or
 // layer * loops + loop for the BF16 format)
@@ -190,7 +326,12 @@ bool make_layout(const rq_config &cfg, Layout *out) {
     L.Tp = (int)align_up((size_t)cfg.max_tokens, kTokTile);
     L.tail_cap = cfg.max_tail_tokens;
     L.splits_max = std::min(kMaxSplits, L.Tp / kTokTile);
-    const size_t bht = B * H * (size_t)L.Tp;
+    L.paged = cfg.block_tokens > 0;
+    L.BT = L.paged ? cfg.block_tokens : L.Tp;
+    L.NBLK = L.paged ? cfg.num_blocks : cfg.batch;
+    L.MB = L.paged ? (cfg.max_tokens + cfg.block_tokens - 1) / cfg.block_tokens : 1;
+    // rows of every record array: blocks x heads x tokens per block
+    const size_t bht = (size_t)L.NBLK * H * (size_t)L.BT;
     if (cfg.format == RQ_FMT_RESIDUAL) {
         L.anchor_codes_bytes = align_up(bht * L.rec.a_codes, kAlign);
         L.anchor_meta_bytes = align_up(bht * L.rec.meta, kAlign);
@@ -217,7 +358,9 @@ bool make_layout(const rq_config &cfg, Layout *out) {
     const size_t vmax_bytes = cfg.format == RQ_FMT_RESIDUAL
                                   ? align_up((size_t)cfg.num_layers * L.groups * L.Lg * B * H * sizeof(int), kAlign)
                                   : 0;
-    L.total = L.off_vmax + vmax_bytes;
+    L.off_table = L.off_vmax + vmax_bytes;
+    const size_t table_bytes = L.paged ? align_up(B * (size_t)L.MB * sizeof(int), kAlign) : 0;
+    L.total = L.off_table + table_bytes;
     *out = L;
     return true;
 }
@@ -255,6 +398,7 @@ int rq_config_check(const rq_config *c) {
     if (c->block_tokens != 0) {
         if (c->block_tokens != 128 && c->block_tokens != 256) return RQ_ERR_UNSUPPORTED;
         if (c->format != RQ_FMT_RESIDUAL) return RQ_ERR_UNSUPPORTED;
+        if (c->loops_per_group > 16) return RQ_ERR_UNSUPPORTED;   // copy-on-write covers groups of up to 16 loops
         if (c->num_blocks < 1) return RQ_ERR_INVALID;
     } else if (c->num_blocks != 0) {
         return RQ_ERR_INVALID;
@@ -335,6 +479,12 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
     c->seq.assign(c->len.size() * (size_t)cfg->batch, 0);
     c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
     c->wstart.assign(c->len.size(), 0x7FFFFFFF);
+    if (L.paged) {
+        c->table.assign((size_t)cfg->batch * L.MB, -1);
+        c->ref.assign(L.NBLK, 0);
+        c->free_blocks.resize(L.NBLK);
+        for (int i = 0; i < L.NBLK; i++) c->free_blocks[i] = L.NBLK - 1 - i;   // block 0 first
+    }
     {
         const int G = cfg->num_q_heads / cfg->num_kv_heads;
         for (int i = 0; i < kMaxChunk / kTokTile; i++) {
@@ -444,7 +594,7 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     a.H = cfg.num_kv_heads;
     a.n = n;
     fill_lens(seq_lens(c, slot), cfg.batch, &a.pos0);
-    a.Tp = L.Tp;
+    a.pg = pages_of(c);
     a.tail_cap = L.tail_cap;
     a.g = cfg.group_size;
     a.ba = cfg.anchor_bits;
@@ -453,6 +603,10 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     a.scale_mode = cfg.scale_mode;
     a.chained = cfg.anchor_mode;
     std::memcpy(a.sigma, &c->sigma[(size_t)layer * 4], sizeof(a.sigma));
+    if (L.paged) {
+        const int sb = prepare_blocks(c, a.pos0, n, st);
+        if (sb != RQ_OK) return sb;
+    }
     int s = cuda_status(launch_append(a, st));
     if (s != RQ_OK) return s;
     int w0 = 0x7FFFFFFF;
@@ -490,6 +644,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     a.Hq = cfg.num_q_heads;
     a.G = cfg.num_q_heads / cfg.num_kv_heads;
     a.Tp = L.Tp;
+    a.pg = pages_of(c);
     a.splits_max = L.splits_max;
     a.g = cfg.group_size;
     a.scale_log2 = resolve_scale(scale) * 1.4426950408889634f;
@@ -719,6 +874,8 @@ int rq_cache_truncate(rq_cache *c, int layer, int group, int new_len) {
     int *v = seq_lens(c, slot), mx = 0;
     for (int b = 0; b < L.cfg.batch; b++) mx = std::max(mx, v[b] = std::min(v[b], new_len));
     c->len[slot] = mx;
+    if (L.paged)
+        for (int b = 0; b < L.cfg.batch; b++) release_blocks(c, b, blocks_needed(c, b));
     return RQ_OK;
 }
 
@@ -738,6 +895,7 @@ int rq_cache_truncate_seq(rq_cache *c, int layer, int group, int seq, int new_le
     int mx = 0;
     for (int b = 0; b < L.cfg.batch; b++) mx = std::max(mx, v[b]);
     c->len[slot] = mx;
+    if (L.paged) release_blocks(c, seq, blocks_needed(c, seq));
     return RQ_OK;
 }
 
@@ -767,20 +925,36 @@ int rq_cache_export(const rq_cache *c, int layer, int loop, void *host_codes, vo
     cudaStream_t st = (cudaStream_t)stream;
     if (len == 0) return RQ_OK;
     const size_t crec = anchor ? L.rec.a_codes : L.rec.r_codes;
+    // one array [blocks][H][BT][rec] -> host [B][H][len][rec]: contiguous
+    // caches copy each sequence's block whole; paged ones every allocated
+    // block of every sequence (rows past a sequence's length are left as they are)
+    auto copy_array = [&](uint8_t *host, const uint8_t *dev, size_t rec) -> cudaError_t {
+        const int H = cfg.num_kv_heads;
+        if (!L.paged)
+            return cudaMemcpy2DAsync(host, len * rec, dev, (size_t)L.BT * rec, len * rec, bh, cudaMemcpyDeviceToHost,
+                                     st);
+        for (int b = 0; b < cfg.batch; b++)
+            for (int k = 0; k * L.BT < len; k++) {
+                const int blk = c->table[(size_t)b * L.MB + k];
+                if (blk < 0) continue;
+                const size_t cnt = std::min(L.BT, len - k * L.BT);
+                cudaError_t e = cudaMemcpy2DAsync(host + ((size_t)b * H * len + (size_t)k * L.BT) * rec, len * rec,
+                                                  dev + (size_t)blk * H * L.BT * rec, (size_t)L.BT * rec, cnt * rec,
+                                                  H, cudaMemcpyDeviceToHost, st);
+                if (e != cudaSuccess) return e;
+            }
+        return cudaSuccess;
+    };
     for (int kv = 0; kv < 2; kv++) {
         const uint8_t *codes = anchor ? anchor_codes(c, layer, group, kv) : resid_codes(c, layer, group, j, kv);
         const uint8_t *meta = anchor ? anchor_meta(c, layer, group, kv) : resid_meta(c, layer, group, j, kv);
         uint8_t *hc = (uint8_t *)host_codes + kv * bh * len * crec;
         uint8_t *hm = (uint8_t *)host_meta + kv * bh * len * L.rec.meta;
-        cudaError_t e = cudaMemcpy2DAsync(hc, len * crec, codes, (size_t)L.Tp * crec, len * crec, bh,
-                                          cudaMemcpyDeviceToHost, st);
-        if (e == cudaSuccess)
-            e = cudaMemcpy2DAsync(hm, len * (size_t)L.rec.meta, meta, (size_t)L.Tp * L.rec.meta,
-                                  len * (size_t)L.rec.meta, bh, cudaMemcpyDeviceToHost, st);
+        cudaError_t e = copy_array(hc, codes, crec);
+        if (e == cudaSuccess) e = copy_array(hm, meta, L.rec.meta);
         if (e == cudaSuccess && !anchor) {
             uint8_t *hf = (uint8_t *)host_coef + kv * bh * len * 2;
-            e = cudaMemcpy2DAsync(hf, len * 2, resid_coef(c, layer, group, j, kv), (size_t)L.Tp * 2, len * 2, bh,
-                                  cudaMemcpyDeviceToHost, st);
+            e = copy_array(hf, resid_coef(c, layer, group, j, kv), 2);
         }
         if (e != cudaSuccess) return RQ_ERR_CUDA;
     }
@@ -813,6 +987,75 @@ size_t rq_decode_bytes(const rq_cache *c, int layer, int loop) {
     if (!is_commit_loop(L, loop))
         tail = (size_t)c->ntail[(size_t)layer * cfg.num_loops + loop] * bh * 2 * kHeadDim * 2;
     return T * cfg.num_kv_heads * per + tail + qo;
+}
+
+int rq_cache_fork_seq(rq_cache *c, int src, int dst, void *stream) {
+    if (!c) return RQ_ERR_INVALID;
+    if (!on_cache_device(c)) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    const rq_config &cfg = L.cfg;
+    if (!L.paged) return RQ_ERR_UNSUPPORTED;
+    if (src < 0 || src >= cfg.batch || dst < 0 || dst >= cfg.batch || src == dst) return RQ_ERR_INVALID;
+    for (int nt : c->ntail)
+        if (nt != 0) return RQ_ERR_STATE;
+    for (size_t slot = 0; slot < c->len.size(); slot++)
+        if (c->seq[slot * cfg.batch + dst] != 0) return RQ_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    PendingOps ops;
+    for (int k = 0; k < L.MB; k++) {
+        const int e = c->table[(size_t)src * L.MB + k];
+        if (e < 0) continue;
+        ops.sets.push_back({dst * L.MB + k, e});
+    }
+    // the largest V scales of dst's streams are src's: [layer][group][Lg][B][H] rows of H ints
+    const size_t H = cfg.num_kv_heads;
+    int *vm = (int *)(c->base + L.off_vmax);
+    const size_t rows = (size_t)cfg.num_layers * L.groups * L.Lg;
+    if (cudaMemcpy2DAsync(vm + dst * H, cfg.batch * H * sizeof(int), vm + src * H, cfg.batch * H * sizeof(int),
+                          H * sizeof(int), rows, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return RQ_ERR_CUDA;
+    int s = flush_ops(c, ops, st);
+    if (s != RQ_OK) return s;
+    for (int k = 0; k < L.MB; k++) {
+        const int e = c->table[(size_t)src * L.MB + k];
+        if (e < 0) continue;
+        c->table[(size_t)dst * L.MB + k] = e;
+        c->ref[e]++;
+    }
+    for (size_t slot = 0; slot < c->len.size(); slot++) c->seq[slot * cfg.batch + dst] = c->seq[slot * cfg.batch + src];
+    return RQ_OK;
+}
+
+int rq_cache_shuffle_free_blocks(rq_cache *c, uint64_t seed) {
+    if (!c) return RQ_ERR_INVALID;
+    if (!c->lay.paged) return RQ_ERR_UNSUPPORTED;
+    // Fisher-Yates with splitmix64 draws
+    std::vector<int> &f = c->free_blocks;
+    for (size_t i = f.size(); i > 1; i--) {
+        const size_t j = (size_t)(splitmix64(seed + i) % i);
+        std::swap(f[i - 1], f[j]);
+    }
+    return RQ_OK;
+}
+
+int rq_cache_free_blocks(const rq_cache *c, int *n) {
+    if (!c || !n) return RQ_ERR_INVALID;
+    if (!c->lay.paged) return RQ_ERR_UNSUPPORTED;
+    *n = (int)c->free_blocks.size();
+    return RQ_OK;
+}
+
+int rq_cache_seq_blocks(const rq_cache *c, int seq, int32_t *host_blocks, int max_blocks, int *n) {
+    if (!c || !n) return RQ_ERR_INVALID;
+    const Layout &L = c->lay;
+    if (!L.paged) return RQ_ERR_UNSUPPORTED;
+    if (seq < 0 || seq >= L.cfg.batch) return RQ_ERR_INVALID;
+    int cnt = 0;
+    while (cnt < L.MB && c->table[(size_t)seq * L.MB + cnt] >= 0) cnt++;
+    *n = cnt;
+    if (host_blocks)
+        for (int k = 0; k < std::min(cnt, max_blocks); k++) host_blocks[k] = c->table[(size_t)seq * L.MB + k];
+    return RQ_OK;
 }
 
 int rq_check(rq_cache *c) {

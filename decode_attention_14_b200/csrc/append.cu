@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendArgs a) {
     load4_bf16(a.x_anchor[kv] + (((size_t)b * a.n + t) * a.H + h) * kHeadDim + lane * 4, x);
     uint32_t s8, m8;
     const uint32_t apack = quantize4(x, a.ba, a.g, lane, ahat, &s8, &m8);
-    const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0.v[b] + t);
+    const size_t rec = rec_row(a.pg, a.H, b, h, a.pos0.v[b] + t);
     const int meta_rec = 2 * (kHeadDim / a.g);
     if (j == a.nres) {
         uint8_t *ac = a.a_codes0 + kv * a.anchor_kv_stride + rec * (kHeadDim * a.ba / 8);
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(128) append_chain_kernel(const AppendArgs a) {
     r /= a.n;
     const int b = (int)(r % a.B);
     const int kv = (int)(r / a.B);
-    const size_t rec = ((size_t)b * a.H + h) * a.Tp + (size_t)(a.pos0.v[b] + t);
+    const size_t rec = rec_row(a.pg, a.H, b, h, a.pos0.v[b] + t);
     const int meta_rec = 2 * (kHeadDim / a.g);
     // loop l's input: the tails hold loops 0 .. nres-1, the call's input the last loop
     auto load_loop = [&](int l, double v[4]) {
@@ -278,7 +278,30 @@ __global__ void bf16_store_kernel(const Bf16StoreArgs a) {
     dst[vec] = src[vec];
 }
 
+// Paged caches: block-table writes (CTA (0, 0)) and block copies (CTA
+// (copy, group x array) copies one block of one record array).
+__global__ void block_ops_kernel(const BlockOpsArgs a) {
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+        for (int i = threadIdx.x; i < a.n_sets; i += blockDim.x) a.table[a.set_idx[i]] = a.set_val[i];
+    const int ci = blockIdx.x;
+    if (ci >= a.n_copies) return;
+    const int g = blockIdx.y / a.n_arrays, arr = blockIdx.y % a.n_arrays;
+    const size_t bytes = a.rows_per_block * a.arr_rec[arr];
+    uint8_t *base = a.records + g * a.group_block + a.arr_off[arr];
+    const uint4 *src = reinterpret_cast<const uint4 *>(base + (size_t)a.copy_src[ci] * bytes);
+    uint4 *dst = reinterpret_cast<uint4 *>(base + (size_t)a.copy_dst[ci] * bytes);
+    for (size_t i = threadIdx.x; i < bytes / 16; i += blockDim.x) dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_block_ops(const BlockOpsArgs &a, cudaStream_t st) {
+    if (a.n_sets == 0 && a.n_copies == 0) return cudaSuccess;
+    const dim3 grid(a.n_copies > 0 ? a.n_copies : 1, a.n_copies > 0 ? a.n_groups * a.n_arrays : 1);
+    if (grid.y > 65535) return cudaErrorInvalidValue;
+    block_ops_kernel<<<grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st) {
     const long long warps = 2LL * a.B * a.n * a.H * (a.chained ? 1 : a.nres + 1);

@@ -65,6 +65,17 @@
 #include "common.cuh"
 #include "rq_internal.h"
 
+#ifdef RQ_FAULT_INJECT
+// Test builds only (never the shipped library): when set, the next decode
+// launch's CTA (0, 0, 0) leaves the mbarrier of its second ring item unarmed
+// -- it issues no copy for it -- so its consumers' bounded wait runs out.
+__device__ int g_rq_fault_once;
+extern "C" int rq_test_arm_fault(void) {
+    const int one = 1;
+    return cudaMemcpyToSymbol(g_rq_fault_once, &one, sizeof(int)) == cudaSuccess ? 0 : -6;
+}
+#endif
+
 namespace rq {
 namespace {
 
@@ -92,7 +103,10 @@ static_assert(kRingBytes % 128 == 0, "ring must be a multiple of 128 bytes");
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
-constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait
+#ifndef RQ_WAIT_NS
+#define RQ_WAIT_NS 1000000000ull
+#endif
+constexpr unsigned long long kWaitNs = RQ_WAIT_NS;      // limit of one wait (1 s by default)
 constexpr int kWeightTop = 22;                          // V weight bound in [2^21, 2^22) (fixed point)
 #ifndef RQ_DECODE_PDL
 #define RQ_DECODE_PDL 1
@@ -393,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     __shared__ __align__(8) uint64_t bar_cf;
     __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
     __shared__ int s_abort, s_last;
+    __shared__ int s_blk[kMaxChunk / kTokTile + 1];   // paged: physical blocks of the chunk
     __shared__ unsigned s_cfmax[NW];
     __shared__ float s_q[GK][2][kHeadDim];
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
@@ -432,12 +447,40 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 
     // ------------------------------------------------------------ producer
     if (warp == 4) {
+        // paged records: the chunk's physical blocks, read once into shared
+        // memory (after the grid dependency wait: the table may just have
+        // been written)
+        const bool paged = a.pg.table != nullptr;
+        const int blk0 = t0 >> a.pg.shift;
+        if (paged) {
+            griddep_wait_then_release();
+            const int nblk = ntiles > 0 ? ((t0 + ntiles * kTile - 1) >> a.pg.shift) - blk0 + 1 : 0;
+            if (lane < nblk) s_blk[lane] = a.pg.table[(size_t)b * a.pg.mb + blk0 + lane];
+            __syncwarp();
+        }
         if (lane == 0) {
-            const size_t tok0 = bh * a.Tp + (size_t)t0;
+            // record row of token t of this (sequence, head)
+            auto row_of = [&](int t) -> size_t {
+                if (!paged) return bh * a.pg.bt + (size_t)t;
+                return (((size_t)s_blk[(t >> a.pg.shift) - blk0] * a.H + h) << a.pg.shift) +
+                       (size_t)(t & (a.pg.bt - 1));
+            };
+            // bulk copies of tokens [t, t + cnt) of an array with rec bytes per
+            // record, one per block the run touches
+            auto copy_run = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
+                const uint8_t *src = static_cast<const uint8_t *>(base);
+                while (cnt > 0) {
+                    const int c = paged ? min(cnt, a.pg.bt - (t & (a.pg.bt - 1))) : cnt;
+                    bulk_g2s(dst, src + row_of(t) * rec, (uint32_t)(c * rec), bar);
+                    dst += c * rec;
+                    t += c;
+                    cnt -= c;
+                }
+            };
             // records of tokens [.., tok_end) may be read before the grid
             // dependency wait only if all of them lie below a.stable (padding
             // beyond the sequence's length is read but never used)
-            bool waited = false;
+            bool waited = paged;
             auto dep = [&](int tok_end) {
                 if (!waited && t0 + tok_end > a.stable) {
                     griddep_wait_then_release();
@@ -449,8 +492,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 mbar_expect_tx(&bar_cf, (uint32_t)(NR * ntiles * kTile * 2));
 #pragma unroll
                 for (int k = 0; k < NR; k++)
-                    bulk_g2s(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1] + tok0,
-                             (uint32_t)(ntiles * kTile * 2), &bar_cf);
+                    copy_run(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1], 2, t0, ntiles * kTile,
+                             &bar_cf);
             } else if (RESID) {
                 mbar_arrive(&bar_cf);   // nothing to fetch
             }
@@ -468,21 +511,6 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             bool ok = true;
             for (int pass = 0; pass < npass && ok; pass++) {
                 const int bytes = P::item_bytes(pass);
-                const uint8_t *c0, *c1 = nullptr;   // code and meta sources of this pass's first tile
-                int cstride = 0, c1stride = P::MR * kItem;
-                if (pass == 0) {
-                    c0 = a.a_codes[0] + tok0 * P::A_C;
-                    c1 = a.a_meta[0] + tok0 * P::MR;
-                    cstride = P::A_C * kItem;
-                } else if (pass == 1) {
-                    c0 = a.a_codes[1] + tok0 * P::A_C;
-                    c1 = a.a_meta[1] + tok0 * P::MR;
-                    cstride = P::A_C * kItem;
-                } else {
-                    c0 = a.r_codes[pass - 2][1] + tok0 * P::R_C;
-                    c1 = a.r_meta[pass - 2][1] + tok0 * P::MR;
-                    cstride = P::R_C * kItem;
-                }
                 for (int j = 0; j < nitems; j++, it++) {
                     if (phys + bytes > P::RING) {
                         virt += P::RING - phys;
@@ -516,27 +544,36 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     }
                     // the last item of a pass may hold fewer tiles: copy only those
                     const int toks = min(kItem, (ntiles - j * kItemTiles) * kTile);
+                    const int tj = t0 + j * kItem;
                     uint8_t *st = ring + phys;
                     uint64_t *bar = &bar_full[it % kSlots];
+#ifdef RQ_FAULT_INJECT
+                    if (it == 1 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 &&
+                        atomicExch(&g_rq_fault_once, 0) == 1) {
+                        virt += bytes;   // the item keeps its place in the ring, unarmed
+                        phys += bytes;
+                        continue;
+                    }
+#endif
                     if (pass == 0) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2))));
-                        bulk_g2s(st, c0, toks * P::A_C, bar);
-                        bulk_g2s(st + P::K_AM, c1, toks * P::MR, bar);
-                        const size_t tj = tok0 + (size_t)j * kItem;
+                        copy_run(st, a.a_codes[0], P::A_C, tj, toks, bar);
+                        copy_run(st + P::K_AM, a.a_meta[0], P::MR, tj, toks, bar);
 #pragma unroll
                         for (int k = 0; k < NR; k++) {
-                            bulk_g2s(st + P::K_RC(k), a.r_codes[k][0] + tj * P::R_C, toks * P::R_C, bar);
-                            bulk_g2s(st + P::K_RM(k), a.r_meta[k][0] + tj * P::MR, toks * P::MR, bar);
-                            bulk_g2s(st + P::K_CF(k), a.r_coef[k][0] + tj, toks * 2, bar);
+                            copy_run(st + P::K_RC(k), a.r_codes[k][0], P::R_C, tj, toks, bar);
+                            copy_run(st + P::K_RM(k), a.r_meta[k][0], P::MR, tj, toks, bar);
+                            copy_run(st + P::K_CF(k), a.r_coef[k][0], 2, tj, toks, bar);
                         }
+                    } else if (pass == 1) {
+                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR)));
+                        copy_run(st, a.a_codes[1], P::A_C, tj, toks, bar);
+                        copy_run(st + P::VA_M, a.a_meta[1], P::MR, tj, toks, bar);
                     } else {
-                        const int cb = pass == 1 ? P::A_C : P::R_C;
-                        mbar_expect_tx(bar, (uint32_t)(toks * (cb + P::MR)));
-                        bulk_g2s(st, c0, toks * cb, bar);
-                        bulk_g2s(st + cstride, c1, toks * P::MR, bar);
+                        mbar_expect_tx(bar, (uint32_t)(toks * (P::R_C + P::MR)));
+                        copy_run(st, a.r_codes[pass - 2][1], P::R_C, tj, toks, bar);
+                        copy_run(st + P::VR_M, a.r_meta[pass - 2][1], P::MR, tj, toks, bar);
                     }
-                    c0 += cstride;
-                    c1 += c1stride;
                     virt += bytes;
                     phys += bytes;
                 }

@@ -43,16 +43,37 @@ struct RecordSizes {
     int meta;      // (d / g) * 2: [scale e4m3, min e4m3] per group
 };
 
+// Token-to-row mapping of the record arrays of one (layer, group).  Each
+// array is [blocks][H_kv][bt][record]: a block holds bt consecutive tokens of
+// one sequence, for every kv head.  Contiguous caches have one block per
+// sequence (block b, bt = the padded capacity Tp); paged caches draw blocks of
+// bt = block_tokens tokens from a pool through a per-sequence block table.
+struct Pages {
+    const int *table;   // [B][mb] physical block of each block of tokens; null: contiguous
+    int mb;             // table entries per sequence
+    int bt;             // tokens per block
+    int shift;          // log2(bt) (paged)
+};
+
+// Row (record index) of token t of (sequence b, kv head h).
+__host__ __device__ inline size_t rec_row(const Pages &p, int H, int b, int h, int t) {
+    if (!p.table) return ((size_t)b * H + h) * p.bt + (size_t)t;
+    return (((size_t)p.table[(size_t)b * p.mb + (t >> p.shift)] * H + h) << p.shift) + (size_t)(t & (p.bt - 1));
+}
+
 // Where every array of the arena lives.  All token streams are laid out
-// [B][H_kv][Tp][record] so that the records of one (sequence, head) are one
-// contiguous, 16-byte-aligned run of Tp records (Tp = max_tokens rounded up
-// to kTokTile).
+// [blocks][H_kv][bt][record] (see Pages): the records of one (block, head)
+// are one contiguous, 16-byte-aligned run.
 struct Layout {
     rq_config cfg;
     RecordSizes rec;
     int groups;          // anchor groups per layer = num_loops / loops_per_group
     int Lg;              // loops per group
-    int Tp;              // padded token capacity of a stream
+    int Tp;              // padded token capacity of a sequence (max_tokens rounded up to kTokTile)
+    bool paged;          // records in a pool of blocks (block_tokens > 0)
+    int BT;              // tokens per block (contiguous: Tp)
+    int NBLK;            // blocks per array (contiguous: B)
+    int MB;              // block-table entries per sequence (contiguous: 1)
     int tail_cap;        // max_tail_tokens
     int splits_max;      // partial slots per (b, q head)
     // residual format: per (layer, group)
@@ -74,6 +95,7 @@ struct Layout {
     size_t off_counters;         // int [B][H_kv]
     size_t off_err;              // int error word (+ pad)
     size_t off_vmax;             // int [layers][groups][Lg][B][H_kv]: largest V scale byte per stream
+    size_t off_table;            // int [B][MB]: block table (paged)
     size_t total;
 };
 
@@ -105,7 +127,8 @@ struct AppendArgs {
     // with atomicMax as records are written
     int *vmax;
     SeqLens pos0;                              // first token position written, per sequence
-    int B, H, n, Tp, tail_cap, nres;           // nres = Lg - 1
+    Pages pg;                                  // token -> record row
+    int B, H, n, tail_cap, nres;               // nres = Lg - 1
     int g, ba, br, rotate;
     int scale_mode;                            // 0 least squares, 1 norm ratio, 2 none
     int chained;                               // 1: loop 0 is the anchor, loop l a residual against loop l - 1
@@ -159,7 +182,8 @@ struct DecodeArgs {
     uint16_t *tail_k_w, *tail_v_w;
     int n_new, tail_pos;
     SeqLens seqT;             // committed tokens of each sequence (T = their maximum)
-    int B, H, Hq, G, T, Tp, S, chunk, splits_max;
+    Pages pg;                 // token -> record row (compressed format)
+    int B, H, Hq, G, T, Tp, S, chunk, splits_max;   // Tp: row stride of the BF16 format
     int g;
     float scale_log2;         // softmax_scale * log2(e)
     int rotate;
@@ -183,6 +207,25 @@ struct CombineArgs {
     int B, H, Hq, G, S, splits_max, n_tail, tail_cap;
     float scale_log2;
 };
+
+// Block-table writes and whole-block copies of a paged cache (copy-on-write
+// of blocks shared by forked sequences), up to kMaxBlockOps of each per launch.
+constexpr int kMaxBlockOps = 32;
+constexpr int kMaxArrays = 4 + 6 * 15;   // record arrays of a loop group of up to 16 loops
+struct BlockOpsArgs {
+    int *table;
+    uint8_t *records;          // start of the record area
+    size_t group_block;        // bytes of one (layer, group) block
+    int n_groups;              // layers x groups
+    int n_arrays;
+    size_t arr_off[kMaxArrays];   // record arrays inside a group block
+    int arr_rec[kMaxArrays];      // their bytes per record
+    size_t rows_per_block;        // H_kv x tokens per block
+    int n_sets, n_copies;
+    int set_idx[kMaxBlockOps], set_val[kMaxBlockOps];
+    int copy_src[kMaxBlockOps], copy_dst[kMaxBlockOps];
+};
+cudaError_t launch_block_ops(const BlockOpsArgs &a, cudaStream_t st);
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st);
 cudaError_t launch_tail_copy(const TailArgs &a, cudaStream_t st);

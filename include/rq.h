@@ -334,6 +334,44 @@ int rq_cache_export(const rq_cache *cache, int layer, int loop, void *host_codes
  * and fp32 out.  Split-combine traffic is not counted.  0 on bad input. */
 size_t rq_decode_bytes(const rq_cache *cache, int layer, int loop);
 
+/*
+ * Paged caches (block_tokens > 0): records live in blocks of block_tokens
+ * tokens (every kv head of one sequence) drawn from a pool of num_blocks per
+ * (layer, group), addressed through a per-sequence block table shared by all
+ * layers and groups -- the layout of a serving engine's paged KV cache (the
+ * ai4snews summary, paragraph 4, integrates the method with vLLM).  The
+ * library owns the pool: rq_append takes blocks from the free list as a
+ * sequence grows past its last block (RQ_ERR_CAPACITY when none is left;
+ * nothing is appended then), and rq_cache_truncate / rq_cache_truncate_seq
+ * return the blocks no (layer, group) of the sequence needs any more.
+ * Blocks carry reference counts: a forked sequence shares its source's
+ * blocks until either sequence writes into a shared one, which is then
+ * copied first (copy-on-write, enqueued on the appending call's stream).
+ * Decode, export and the other calls work on paged caches as on contiguous
+ * ones; rq_prefill_attn returns RQ_ERR_UNSUPPORTED for them.
+ */
+
+/* Makes sequence dst (every committed length 0, no tail tokens in the cache)
+ * a copy of sequence src that shares src's blocks: its committed lengths
+ * become src's, and later appends to either copy the shared block they
+ * write into.  Enqueues a few small copies on `stream`.  Errors: INVALID,
+ * UNSUPPORTED (contiguous cache), STATE (dst not empty, or tails not empty),
+ * CUDA. */
+int rq_cache_fork_seq(rq_cache *cache, int src, int dst, void *stream);
+
+/* Permutes the free list with a seeded Fisher-Yates shuffle (splitmix64
+ * draws), so that later allocations scatter over the pool (tests and
+ * fragmentation studies).  Host only.  Errors: INVALID, UNSUPPORTED. */
+int rq_cache_shuffle_free_blocks(rq_cache *cache, uint64_t seed);
+
+/* Number of free blocks in the pool.  Errors: INVALID, UNSUPPORTED. */
+int rq_cache_free_blocks(const rq_cache *cache, int *n);
+
+/* The physical blocks of sequence seq, in token order: *n receives their
+ * count, host_blocks (may be NULL) the first min(*n, max_blocks) ids.
+ * Errors: INVALID, UNSUPPORTED. */
+int rq_cache_seq_blocks(const rq_cache *cache, int seq, int32_t *host_blocks, int max_blocks, int *n);
+
 /* Reports asynchronous failures: RQ_ERR_TIMEOUT if a kernel's bounded wait
  * gave up (the error word and the split-combine counters -- the cache's and
  * rq_decode_attn_noalloc's on this device -- are then cleared, so later calls

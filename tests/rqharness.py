@@ -49,7 +49,7 @@ def scale32() -> float:
 
 def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, rotate=True,
           n_tail=0, seed=0x5EED0000, sigma=(0.1, 0.2, 0.3), chunk=128, fmt=rq.RQ_FMT_RESIDUAL,
-          only_layers=None, only_groups=None, max_tokens=None, **modes) -> Built:
+          only_layers=None, only_groups=None, max_tokens=None, prepare=None, **modes) -> Built:
     """Fills `layers` x (loops/Lg) groups with T committed tokens (appended in
     chunks through the tail), then n_tail in-flight tokens on every
     non-anchor loop."""
@@ -59,6 +59,8 @@ def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, r
                          num_q_heads=Hq, group_size=g, anchor_bits=ba, resid_bits=br, rotate=rotate,
                          format=fmt, seed=0xA11CE, **modes)
     cache = rq.Cache(cfg)
+    if prepare is not None:
+        prepare(cache)
     bt = Built(cache, cfg, seed, T, n_tail)
     for layer in range(layers):
         if only_layers is not None and layer not in only_layers:
