@@ -298,15 +298,18 @@ class Cache:
     """Owns one rq_cache handle (and its arena, a torch uint8 tensor, unless
     ``library_alloc`` asks the library to cudaMalloc it)."""
 
-    def __init__(self, cfg: rq_config, device=None, library_alloc: bool = False):
+    def __init__(self, cfg: rq_config, device=None, library_alloc: bool = False, arena=None):
+        """arena: an optional caller-owned uint8 CUDA tensor of at least
+        rq_cache_required_bytes(cfg) bytes, 256-byte aligned (for example a
+        view into a larger buffer); by default one is allocated."""
         import torch
         self.cfg = cfg
         self.B, self.H, self.Hq = cfg.batch, cfg.num_kv_heads, cfg.num_q_heads
         self.Lg = cfg.loops_per_group
         _ok(rq_config_check(cfg), "rq_config_check")
         self.nbytes = rq_cache_required_bytes(cfg)
-        self.arena = None
-        if not library_alloc:
+        self.arena = arena
+        if arena is None and not library_alloc:
             self.arena = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
         self.h = rq_cache_create(cfg, self.arena)
 

@@ -25,3 +25,13 @@ _build_library()
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands(request):
+    """After every GPU test: the guard bands around the harness's cache arenas
+    and decode outputs are intact."""
+    yield
+    if request.node.get_closest_marker("gpu") is not None:
+        import rqharness
+        rqharness.check_guards()

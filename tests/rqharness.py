@@ -30,6 +30,44 @@ MSE_REL_TOL = 0.01
 D = 128
 
 
+# ------------------------------------------------------------------ guard bands
+# Every cache the harness creates lives in the middle of a larger buffer
+# whose margins hold a fixed byte pattern, and decode outputs get the same;
+# an autouse fixture (conftest.py) checks after each GPU test that no margin
+# changed -- a write outside the arena or past an output row would.
+GUARD = 4096
+GUARD_BYTE = 0xA5
+_guarded = []
+
+
+def guarded_buffer(nbytes: int, dtype=torch.uint8, device="cuda"):
+    """A tensor view of nbytes (256-byte aligned) inside a buffer with
+    GUARD_BYTE margins of GUARD bytes on both sides."""
+    big = torch.full((nbytes + 2 * GUARD,), GUARD_BYTE, dtype=torch.uint8, device=device)
+    _guarded.append((big, GUARD, nbytes))
+    return big[GUARD:GUARD + nbytes].view(dtype)
+
+
+def guarded_out(shape):
+    n = int(np.prod(shape))
+    return guarded_buffer(4 * n, torch.float32).view(*shape)
+
+
+def check_guards():
+    """Asserts that no margin changed; forgets the buffers."""
+    bad = []
+    for big, off, n in _guarded:
+        host = big.cpu().numpy()
+        if not ((host[:off] == GUARD_BYTE).all() and (host[off + n:] == GUARD_BYTE).all()):
+            bad.append(n)
+    _guarded.clear()
+    assert not bad, f"guard bands overwritten around buffers of {bad} bytes"
+
+
+def guarded_cache(cfg) -> rq.Cache:
+    return rq.Cache(cfg, arena=guarded_buffer(rq.rq_cache_required_bytes(cfg)))
+
+
 @dataclass
 class Built:
     cache: rq.Cache
@@ -58,7 +96,7 @@ def build(*, layers=1, loops=4, Lg=4, B=1, T=256, H=4, Hq=8, g=16, ba=4, br=2, r
                          max_tokens=max_tokens or max(T, 1), max_tail_tokens=tail_cap, num_kv_heads=H,
                          num_q_heads=Hq, group_size=g, anchor_bits=ba, resid_bits=br, rotate=rotate,
                          format=fmt, seed=0xA11CE, **modes)
-    cache = rq.Cache(cfg)
+    cache = guarded_cache(cfg)
     if prepare is not None:
         prepare(cache)
     bt = Built(cache, cfg, seed, T, n_tail)
@@ -98,7 +136,7 @@ def build_from(K, V, *, Hq: int, g=16, ba=4, br=2, rotate=True, T: int, n_tail=0
     cfg = rq.make_config(num_layers=1, num_loops=Lg, loops_per_group=Lg, batch=B, max_tokens=max(T, 1),
                          max_tail_tokens=max(chunk, n_tail, 1), num_kv_heads=Hkv, num_q_heads=Hq, group_size=g,
                          anchor_bits=ba, resid_bits=br, rotate=rotate, seed=0xA11CE)
-    bt = Built(rq.Cache(cfg), cfg, seed, T, n_tail)
+    bt = Built(guarded_cache(cfg), cfg, seed, T, n_tail)
     fill_group(bt, 0, 0, K, V, chunk)
     torch.cuda.synchronize()
     return bt

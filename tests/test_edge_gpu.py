@@ -112,7 +112,7 @@ def check_decode(bt, q_of=None):
     cfg = bt.cfg
     for loop in range(LG):
         q = synth.queries(bt.seed, 0, loop, 0, cfg.batch, cfg.num_q_heads) if q_of is None else q_of(loop)
-        out = bt.cache.decode(0, loop, q).cpu().numpy()
+        out = bt.cache.decode(0, loop, q, out=H.guarded_out((cfg.batch, cfg.num_q_heads, D))).cpu().numpy()
         assert np.isfinite(out).all()
         ref = H.oracle_decode(bt, 0, loop, q)
         rel, mx = H.attn_errors(out, ref, cfg.num_q_heads // cfg.num_kv_heads)

@@ -37,7 +37,7 @@ def _check(bt, strict, loops, layer=0):
         assert abs(g / o - 1.0) <= H.MSE_REL_TOL, (kv, g, o)
     for loop in loops:
         q = synth.queries(bt.seed, layer, loop, 0, cfg.batch, cfg.num_q_heads)
-        out = bt.cache.decode(layer, loop, q).cpu().numpy()
+        out = bt.cache.decode(layer, loop, q, out=H.guarded_out((cfg.batch, cfg.num_q_heads, 128))).cpu().numpy()
         ref = H.oracle_decode(bt, layer, loop, q)
         rel, mx = H.attn_errors(out, ref, cfg.num_q_heads // cfg.num_kv_heads)
         assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (loop, rel, mx)

@@ -39,7 +39,7 @@ def _check(bt, sel=None, loops=range(4)):
     outs = {}
     for loop in loops:
         q = synth.queries(bt.seed, 0, loop, 0, cfg.batch, cfg.num_q_heads)
-        out = bt.cache.decode(0, loop, q)
+        out = bt.cache.decode(0, loop, q, out=H.guarded_out((cfg.batch, cfg.num_q_heads, 128)))
         ref = H.oracle_decode(bt, 0, loop, q, sel)
         rel, mx = H.attn_errors(out.cpu().numpy(), ref, cfg.num_q_heads // cfg.num_kv_heads)
         assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (loop, rel, mx)

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 def _decode_and_check(bt, layer, loop, bh_sel=None, step=0):
     cfg = bt.cfg
     q = synth.queries(bt.seed, layer, loop, step, cfg.batch, cfg.num_q_heads)
-    out = bt.cache.decode(layer, loop, q).cpu().numpy()
+    out = bt.cache.decode(layer, loop, q, out=H.guarded_out((cfg.batch, cfg.num_q_heads, 128))).cpu().numpy()
     ref = H.oracle_decode(bt, layer, loop, q, bh_sel)
     rel, mx = H.attn_errors(out, ref, cfg.num_q_heads // cfg.num_kv_heads)
     assert rel <= H.REL_L2_TOL and mx <= H.MAX_ABS_TOL, (layer, loop, rel, mx)
