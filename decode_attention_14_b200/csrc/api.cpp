@@ -21,6 +21,10 @@ struct rq_cache {
     std::vector<int> len;     // residual: [layer][group]; bf16: [layer][loop]; the longest sequence
     std::vector<int> seq;     // the same, per sequence: [layer][group or loop][batch]
     std::vector<int> ntail;   // [layer][loop]
+    // per length slot: the first token position the most recent record write
+    // (an anchor append) started at, over the sequences; records below it are
+    // not touched by any append still in flight
+    std::vector<int> wstart;
     std::vector<uint32_t> sigma;   // [layer][4]: sign bits of the layer's rotation
     // resident CTAs per SM for chunk = 64 * (i + 1), by residual records read (0 .. kMaxChain)
     int occ[kMaxChain + 1][kMaxChunk / kTokTile];
@@ -303,26 +307,6 @@ void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *
     *chunk = best_ch;
 }
 
-// CTAs per unit of the compressed-cache decode, which share the unit's
-// tiles out dynamically (each takes 128-token items from a counter until
-// none is left or its shared memory -- chunk = kMaxChunk tokens -- is full):
-// enough CTAs to hold every tile, and otherwise as many as fill the resident
-// slots once (more would only wait for items).
-void choose_ctas(const rq_cache *c, int T, int units, int nr, int *S, int *chunk) {
-    *chunk = kMaxChunk;
-    if (T <= 0) {
-        *S = 0;
-        return;
-    }
-    const int nt = (T + kTokTile - 1) / kTokTile;
-    const int items = (nt + 1) / 2;
-    const int need = (nt + kMaxChunk / kTokTile - 1) / (kMaxChunk / kTokTile);
-    const int slots = std::max(1, c->occ[nr][kMaxChunk / kTokTile - 1] * c->sms);
-    int s = std::max(need, std::min(slots / std::max(units, 1), items));
-    s = std::min(s, c->lay.splits_max);
-    *S = std::max(s, 1);
-}
-
 }  // namespace
 
 namespace rq {
@@ -369,7 +353,7 @@ bool make_layout(const rq_config &cfg, Layout *out) {
     L.off_partials = align_up(L.records_bytes, kAlign);
     size_t partial_bytes = align_up(B * Hq * (size_t)L.splits_max * kPartialStride * sizeof(float), kAlign);
     L.off_counters = L.off_partials + partial_bytes;
-    L.off_err = L.off_counters + align_up(2 * B * Hq * sizeof(int), kAlign);   // arrival + tile counters
+    L.off_err = L.off_counters + align_up(B * Hq * sizeof(int), kAlign);
     L.off_vmax = L.off_err + kAlign;
     const size_t vmax_bytes = cfg.format == RQ_FMT_RESIDUAL
                                   ? align_up((size_t)cfg.num_layers * L.groups * L.Lg * B * H * sizeof(int), kAlign)
@@ -494,6 +478,7 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
     c->len.assign((size_t)cfg->num_layers * (cfg->format == RQ_FMT_RESIDUAL ? L.groups : cfg->num_loops), 0);
     c->seq.assign(c->len.size() * (size_t)cfg->batch, 0);
     c->ntail.assign((size_t)cfg->num_layers * cfg->num_loops, 0);
+    c->wstart.assign(c->len.size(), 0x7FFFFFFF);
     if (L.paged) {
         c->table.assign((size_t)cfg->batch * L.MB, -1);
         c->ref.assign(L.NBLK, 0);
@@ -624,6 +609,9 @@ int rq_append(rq_cache *c, int layer, int loop, const void *k, const void *v, in
     }
     int s = cuda_status(launch_append(a, st));
     if (s != RQ_OK) return s;
+    int w0 = 0x7FFFFFFF;
+    for (int b = 0; b < cfg.batch; b++) w0 = std::min(w0, a.pos0.v[b]);
+    c->wstart[slot] = w0;
     grow(c, slot, n);
     for (int jj = 0; jj < L.Lg - 1; jj++) c->ntail[(size_t)layer * cfg.num_loops + group * L.Lg + jj] = 0;
     return RQ_OK;
@@ -650,7 +638,6 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
     a.out = out;
     a.partials = (float *)(c->base + L.off_partials);
     a.counters = (int *)(c->base + L.off_counters);
-    a.tiles = a.counters + (size_t)cfg.batch * cfg.num_q_heads;
     a.err = (int *)(c->base + L.off_err);
     a.B = cfg.batch;
     a.H = cfg.num_kv_heads;
@@ -678,6 +665,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
             a.a_meta[kv] = anchor_meta(c, layer, group, kv);
         }
         a.vmax_a = vmax_ptr(c, layer, group, L.Lg - 1);
+        a.stable = c->wstart[(size_t)layer * L.groups + group];
         if (!is_commit_loop(L, loop)) {
             a.n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
             a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
@@ -699,17 +687,13 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
-    if (bf16)
-        choose_splits(c, a.T, units, 0, &a.S, &a.chunk);
-    else
-        choose_ctas(c, a.T, units, a.nr, &a.S, &a.chunk);
+    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, &a.S, &a.chunk);
     if (partials) {
         a.splits_max = std::max(a.S, 1);
         if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;
         if ((size_t)a.B * a.Hq > max_units) return RQ_ERR_CAPACITY;
         a.partials = partials;
         a.counters = counters;
-        a.tiles = counters + max_units;
     }
     if (app_k) {
         // one launch when the loop keeps the tokens in its tail and the split

@@ -30,28 +30,27 @@
 // which follows the actual V scales, so small-magnitude V keeps its relative
 // precision).
 //
-// Per-group scales, minima, softmax and the final rotation stay in fp32.
-//
 // Programmatic launch.  The kernel may start while the previous kernel on
 // its stream is still running (the host launches it with programmatic stream
-// serialization): it sets up its barriers and then waits for that kernel at
-// a grid-dependency wait before any global access; a thread signals that the
-// next kernel may start only after its own wait has returned, so at most one
-// earlier kernel is ever still running.
+// serialization): the producer streams committed records below a.stable --
+// which no in-flight work writes -- before its grid-dependency wait; every
+// other global access (q, the V scale bounds, records from a.stable on, the
+// tail, partials, counters, out) comes after the wait.  A thread signals
+// that the next kernel may start only after its own wait has returned, so at
+// most one earlier kernel is ever still running.
+// Per-group scales, minima, softmax and the final rotation stay in fp32.
 //
-// Data movement.  The CTAs of one (sequence, kv head) unit share its 64-token
-// tiles out dynamically: each CTA's producer warp takes 128-token items from
-// the unit's atomic counter as long as items are left and its shared memory
-// has room, so CTAs that run faster (on less loaded SMs) take more and the
-// unit's CTAs finish together.  Each item is streamed through a
-// byte-addressed shared-memory ring with 1-D bulk asynchronous copies
-// (cp.async.bulk, completion counted on mbarriers; no multicast): first the
-// K records of every item with the V coefficients of the same tokens (pass
-// 1: logits), a sentinel item marking the end of the CTA's list, then the
-// anchor V codes + meta and the residual V codes + meta of the same items
-// (pass 2: values).  Every mbarrier wait is bounded: on timeout the kernel
-// records an error word, stops issuing copies, drains what it issued and
-// finishes without touching further data.
+// Data movement.  Each CTA owns a chunk of one (sequence, kv head) (the
+// sequence's 64-token tiles dealt evenly over the splits) and streams it in
+// 128-token items through a byte-addressed shared-memory ring filled by one
+// producer warp with 1-D bulk asynchronous copies (cp.async.bulk, completion
+// counted on mbarriers; no multicast): first the K records of every item
+// (pass 1: logits), then the anchor V codes + meta, then the residual V codes
+// + meta (pass 2: values).  Only the V coefficients of the chunk (2 bytes per
+// token) are fetched once up front; the producer warp's other lanes take
+// their maximum for the weights' fixed point.  Every mbarrier wait is
+// bounded: on timeout the kernel records an error word, stops issuing copies,
+// drains what it issued and finishes without touching further data.
 //
 // Split combine.  Each CTA writes its partial (max, sum, o); the last CTA of
 // a (sequence, kv head) -- found with a device-wide counter, no waiting --
@@ -93,7 +92,7 @@ constexpr int kItem = kTile * kItemTiles;          // tokens per ring item
 #define RQ_DECODE_PRODUCER_SLEEP_NS 0
 #endif
 #ifndef RQ_DECODE_RING_BYTES
-#define RQ_DECODE_RING_BYTES 36864
+#define RQ_DECODE_RING_BYTES 39936
 #endif
 #ifndef RQ_DECODE_MIN_CTAS
 #define RQ_DECODE_MIN_CTAS 4
@@ -405,10 +404,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bar_full[kSlots];
     __shared__ __align__(8) uint64_t bar_empty[kSlots];
+    __shared__ __align__(8) uint64_t bar_cf;
+    __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
     __shared__ int s_abort, s_last;
-    __shared__ int s_start[kSlots];            // producer: virtual ring start of the item in each slot
-    __shared__ int s_item_tile[kSlots];        // first tile of the K item in each slot; -1: no more
-    __shared__ int s_list[kMaxChunk / kItem];  // first tiles of this CTA's items, in order
+    __shared__ int s_blk[kMaxChunk / kTokTile + 1];   // paged: physical blocks of the chunk
     __shared__ unsigned s_cfmax[NW];
     __shared__ float s_q[GK][2][kHeadDim];
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
@@ -421,10 +420,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int npairs = a.G / GK;
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int hq0 = h * a.G + pair * GK;
-    const int unit = (b * a.H + h) * npairs + pair;
-    const int Tb = a.seqT.v[b];                     // committed tokens of this sequence
-    const int nt = (Tb + kTile - 1) / kTile;        // its tiles, shared out among the unit's CTAs
-    const int cap = a.chunk / kItem;                // items one CTA may take (its shared-memory capacity)
+    int t0, n;   // this split's tokens of its sequence (none when the sequence is short)
+    split_range(split, a.S, a.seqT.v[b], &t0, &n);
+    const int ntiles = (n + kTile - 1) / kTile;
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
     const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);   // V coefficients [NR][cstride]
@@ -439,6 +437,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             mbar_init(&bar_full[i], 1);
             mbar_init(&bar_empty[i], kConsumers);   // every consumer thread arrives
         }
+        mbar_init(&bar_cf, 1);
+        mbar_init(&bar_cfmax, 31);
         s_abort = 0;
         for (int k = 0; k < NW; k++) s_cfmax[k] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -446,92 +446,126 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     __syncthreads();
 
     // ------------------------------------------------------------ producer
-    // The unit's tiles are shared out dynamically: each item of two tiles
-    // (128 tokens) goes to the CTA that asks for it first (an atomic counter
-    // per unit), so CTAs that run faster take more of them and the unit's
-    // CTAs -- on different SMs -- finish close together.  The K items come
-    // first, then a sentinel item (no bytes) that tells the consumers how many
-    // there were, then the anchor V items and the residual V items of the same
-    // tiles in the same order.
     if (warp == 4) {
-        // everything the producer reads may have been written by the previous
-        // kernel on the stream (records, block table, the tile counters)
-        griddep_wait_then_release();
+        // paged records: the chunk's physical blocks, read once into shared
+        // memory (after the grid dependency wait: the table may just have
+        // been written)
+        const bool paged = a.pg.table != nullptr;
+        const int blk0 = t0 >> a.pg.shift;
+        if (paged) {
+            griddep_wait_then_release();
+            const int nblk = ntiles > 0 ? ((t0 + ntiles * kTile - 1) >> a.pg.shift) - blk0 + 1 : 0;
+            if (lane < nblk) s_blk[lane] = a.pg.table[(size_t)b * a.pg.mb + blk0 + lane];
+            __syncwarp();
+        }
         if (lane == 0) {
-            const bool paged = a.pg.table != nullptr;
-            int blk = 0;   // paged: physical block of the current item (an item never crosses a block)
-            // bulk copy of the records of tokens [t, t + cnt) of an array with rec bytes per record
-            auto copy_run = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
-                const size_t row = paged ? (((size_t)blk * a.H + h) << a.pg.shift) + (size_t)(t & (a.pg.bt - 1))
-                                         : bh * a.pg.bt + (size_t)t;
-                bulk_g2s(dst, static_cast<const uint8_t *>(base) + row * rec, (uint32_t)(cnt * rec), bar);
+            // record row of token t of this (sequence, head)
+            auto row_of = [&](int t) -> size_t {
+                if (!paged) return bh * a.pg.bt + (size_t)t;
+                return (((size_t)s_blk[(t >> a.pg.shift) - blk0] * a.H + h) << a.pg.shift) +
+                       (size_t)(t & (a.pg.bt - 1));
             };
-            auto block_of = [&](int t) { return paged ? a.pg.table[(size_t)b * a.pg.mb + (t >> a.pg.shift)] : 0; };
-            int it = 0, virt = 0, phys = 0, rel = 0;
-            bool ok = true;
-            // ring space for an item of `bytes` at phys (wrapping to 0 if it would straddle the end):
-            // every older item starting below virt + bytes - RING released, at most kSlots outstanding
-            auto make_room = [&](int bytes) {
-                if (phys + bytes > P::RING) {
-                    virt += P::RING - phys;
-                    phys = 0;
+            // bulk copies of tokens [t, t + cnt) of an array with rec bytes per
+            // record, one per block the run touches
+            auto copy_run = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
+                const uint8_t *src = static_cast<const uint8_t *>(base);
+                while (cnt > 0) {
+                    const int c = paged ? min(cnt, a.pg.bt - (t & (a.pg.bt - 1))) : cnt;
+                    bulk_g2s(dst, src + row_of(t) * rec, (uint32_t)(c * rec), bar);
+                    dst += c * rec;
+                    t += c;
+                    cnt -= c;
                 }
-                while (ok && rel < it && (it - rel >= kSlots || s_start[rel % kSlots] < virt + bytes - P::RING)) {
-                    if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
-                                                                &s_abort)) {
-                        ok = false;
+            };
+            // records of tokens [.., tok_end) may be read before the grid
+            // dependency wait only if all of them lie below a.stable (padding
+            // beyond the sequence's length is read but never used)
+            bool waited = paged;
+            auto dep = [&](int tok_end) {
+                if (!waited && t0 + tok_end > a.stable) {
+                    griddep_wait_then_release();
+                    waited = true;
+                }
+            };
+            dep(RESID && ntiles > 0 ? n : 0);
+            if (RESID && ntiles > 0) {
+                mbar_expect_tx(&bar_cf, (uint32_t)(NR * ntiles * kTile * 2));
+#pragma unroll
+                for (int k = 0; k < NR; k++)
+                    copy_run(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1], 2, t0, ntiles * kTile,
+                             &bar_cf);
+            } else if (RESID) {
+                mbar_arrive(&bar_cf);   // nothing to fetch
+            }
+            // Items in order: K items, anchor V items, residual V items.  Item it
+            // occupies [virt, virt + bytes) of an unbounded virtual byte
+            // sequence, padded so that no item straddles the ring's end; its
+            // ring offset is phys = virt mod RING.  Before it is issued, every
+            // older item starting below virt + bytes - RING must have been
+            // released, and at most kSlots items may be outstanding.  The
+            // loop keeps all of this in running counters (no division).
+            const int npass = 2 + NR;
+            int it = 0, virt = 0, phys = 0;
+            const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // items per pass
+            int rel = 0, vrel = 0, rphys = 0, ritem = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
+            bool ok = true;
+            for (int pass = 0; pass < npass && ok; pass++) {
+                const int bytes = P::item_bytes(pass);
+                for (int j = 0; j < nitems; j++, it++) {
+                    if (phys + bytes > P::RING) {
+                        virt += P::RING - phys;
+                        phys = 0;
+                    }
+                    if (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING))
+                        dep(0x7FFFFFFF);   // about to block on the consumers, who run after their wait
+                    dep(min((j + 1) * kItem, n));
+                    while (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING)) {
+                        if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
+                                                                    &s_abort)) {
+                            ok = false;
+                            break;
+                        }
+                        vrel += rbytes;
+                        rphys += rbytes;
+                        if (++ritem == nitems) {
+                            ritem = 0;
+                            rbytes = P::item_bytes(++rpass);
+                        }
+                        if (rphys + rbytes > P::RING) {
+                            vrel += P::RING - rphys;
+                            rphys = 0;
+                        }
+                        rel++;
+                    }
+                    if (!ok) {
                         s_abort = 1;
                         atomicExch(a.err, 1);
+                        break;
                     }
-                    rel++;
-                }
-                s_start[it % kSlots] = virt;
-            };
-            int nitems = 0;
-            int g = (nt > 0 && cap > 0) ? atomicAdd(&a.tiles[unit], kItemTiles) : nt;
-            while (ok && g < nt) {
-                const int toks = min(kItem, (nt - g) * kTile);
-                const int tj = g * kTile;
-                if (paged) blk = block_of(tj);
-                make_room(P::K_BYTES);
-                if (!ok) break;
-                uint8_t *st = ring + phys;
-                uint64_t *bar = &bar_full[it % kSlots];
-                s_list[nitems] = g;
-                s_item_tile[it % kSlots] = g;
-                // K records, and the V coefficients of the same tokens into their own buffer
-                mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2 + 2))));
-                copy_run(st, a.a_codes[0], P::A_C, tj, toks, bar);
-                copy_run(st + P::K_AM, a.a_meta[0], P::MR, tj, toks, bar);
-#pragma unroll
-                for (int k = 0; k < NR; k++) {
-                    copy_run(st + P::K_RC(k), a.r_codes[k][0], P::R_C, tj, toks, bar);
-                    copy_run(st + P::K_RM(k), a.r_meta[k][0], P::MR, tj, toks, bar);
-                    copy_run(st + P::K_CF(k), a.r_coef[k][0], 2, tj, toks, bar);
-                    copy_run(smem + P::RING + k * P::coef_bytes(a.chunk) + nitems * kItem * 2, a.r_coef[k][1], 2, tj,
-                             toks, bar);
-                }
-                virt += P::K_BYTES;
-                phys += P::K_BYTES;
-                it++;
-                nitems++;
-                g = nitems < cap ? atomicAdd(&a.tiles[unit], kItemTiles) : nt;
-            }
-            // the sentinel: no bytes, tile -1
-            make_room(0);
-            s_item_tile[it % kSlots] = -1;
-            mbar_arrive(&bar_full[it % kSlots]);
-            it++;
-            for (int pass = 1; pass < 2 + NR && ok; pass++) {
-                const int bytes = P::item_bytes(pass);
-                for (int jj = 0; jj < nitems; jj++) {
-                    const int tj = s_list[jj] * kTile, toks = min(kItem, (nt - s_list[jj]) * kTile);
-                    if (paged) blk = block_of(tj);
-                    make_room(bytes);
-                    if (!ok) break;
+                    // the last item of a pass may hold fewer tiles: copy only those
+                    const int toks = min(kItem, (ntiles - j * kItemTiles) * kTile);
+                    const int tj = t0 + j * kItem;
                     uint8_t *st = ring + phys;
                     uint64_t *bar = &bar_full[it % kSlots];
-                    if (pass == 1) {
+#ifdef RQ_FAULT_INJECT
+                    if (it == 1 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 &&
+                        atomicExch(&g_rq_fault_once, 0) == 1) {
+                        virt += bytes;   // the item keeps its place in the ring, unarmed
+                        phys += bytes;
+                        continue;
+                    }
+#endif
+                    if (pass == 0) {
+                        mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2))));
+                        copy_run(st, a.a_codes[0], P::A_C, tj, toks, bar);
+                        copy_run(st + P::K_AM, a.a_meta[0], P::MR, tj, toks, bar);
+#pragma unroll
+                        for (int k = 0; k < NR; k++) {
+                            copy_run(st + P::K_RC(k), a.r_codes[k][0], P::R_C, tj, toks, bar);
+                            copy_run(st + P::K_RM(k), a.r_meta[k][0], P::MR, tj, toks, bar);
+                            copy_run(st + P::K_CF(k), a.r_coef[k][0], 2, tj, toks, bar);
+                        }
+                    } else if (pass == 1) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR)));
                         copy_run(st, a.a_codes[1], P::A_C, tj, toks, bar);
                         copy_run(st + P::VA_M, a.a_meta[1], P::MR, tj, toks, bar);
@@ -542,13 +576,30 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     }
                     virt += bytes;
                     phys += bytes;
-                    it++;
                 }
             }
+            dep(0x7FFFFFFF);
+            const int issued = it;
             // drain: every issued copy must have landed before the CTA exits
             // (the consumers stop waiting once the CTA has given up)
-            for (int i = max(0, it - kSlots); i < it; i++)
-                mbar_wait<256>(&bar_full[i % kSlots], (i / kSlots) & 1, &s_abort);
+            if (RESID) mbar_wait<256>(&bar_cf, 0, &s_abort);
+            for (int it = max(0, issued - kSlots); it < issued; it++)
+                mbar_wait<256>(&bar_full[it % kSlots], (it / kSlots) & 1, &s_abort);
+        } else {
+            // the other lanes: the bound max |s_hat(V)| of the chunk's V
+            // coefficients (for the weights' fixed point), ready before the
+            // softmax needs it
+            griddep_wait_then_release();
+            if (RESID && mbar_wait<64>(&bar_cf, 0, &s_abort)) {
+#pragma unroll
+                for (int k = 0; k < NR; k++) {
+                    const uint16_t *cf = reinterpret_cast<const uint16_t *>(smem + P::RING + k * P::coef_bytes(a.chunk));
+                    unsigned m = 0;
+                    for (int t = lane - 1; t < n; t += 31) m = max(m, (unsigned)cf[t] & 0x7FFFu);
+                    atomicMax(&s_cfmax[k], m);
+                }
+            }
+            mbar_arrive(&bar_cfmax);
         }
         return;
     }
@@ -663,33 +714,20 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
     const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
     const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
-    // ring offset of the next item: the end of the previous one, wrapped to 0
-    // when the next would straddle the ring's end (the producer's placement rule)
-    int c_off = 0;
-    auto place = [&](int bytes) {
-        if (c_off + bytes > P::RING) c_off = 0;
-    };
-    int nitems = 0;   // K items this CTA received (known at the sentinel)
-    for (int j = 0;; j++) {
+    const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // ring items per pass
+    int c_off = 0;   // ring offset of the current item (the producer's placement rule)
+    for (int j = 0; j < nitems; j++) {
         const int slot = j % kSlots;
         const bool ok = mbar_wait(&bar_full[slot], (j / kSlots) & 1, &s_abort);
         if (!ok) {
             s_abort = 1;
             atomicExch(a.err, 2);
         }
-        const int tile = ok ? s_item_tile[slot] : -1;
-        if (tile < 0) {   // the sentinel (or a wait that gave up): no more K items
-            mbar_arrive(&bar_empty[slot]);
-            nitems = j;
-            break;
-        }
-        const int itiles = min(kItemTiles, nt - tile);   // tiles in this item
-        place(P::K_BYTES);
         const uint8_t *st = ring + c_off;
         float part[kItemTiles][GK][4];
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
-            if (u >= itiles) break;   // uniform: a short last item
+            if (j * kItemTiles + u >= ntiles) break;   // uniform: a short last item
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
@@ -715,13 +753,13 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             }
         }
         mbar_arrive(&bar_empty[slot]);
-        c_off += P::K_BYTES;
+        c_off = P::advance(c_off, P::K_BYTES, j + 1 < nitems ? P::K_BYTES : P::VA_BYTES);
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
-            if (u >= itiles) break;
-            const int tl = (j * kItemTiles + u) * kTile + 16 * warp + sub + 4 * kown;   // local token
-            const bool valid = (tile + u) * kTile + 16 * warp + sub + 4 * kown < Tb;
+            const int i = j * kItemTiles + u;
+            if (i >= ntiles) break;
+            const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
                 float r0 = (b4 ? part[u][gq][2] : part[u][gq][0]) +
@@ -731,8 +769,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 float r = (b2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, b2 ? r0 : r1, 2);
                 r += __shfl_xor_sync(0xffffffffu, r, 1);
                 r *= qinv;
-                if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;   // tl < cap items * 128 = chunk
-                if (valid) mloc[gq] = fmaxf(mloc[gq], r);
+                if ((seg & 1) == 0) s_sc[gq * a.chunk + tl] = r;   // tl < ntiles*64 <= chunk
+                if (tl < n && ok) mloc[gq] = fmaxf(mloc[gq], r);
             }
         }
     }
@@ -744,17 +782,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
         if (lane == 0) s_red[warp][gq] = v;
     }
-    // the largest |s_hat(V)| of each residual record over this CTA's tokens
-    // (the V coefficients arrived with the K items)
-    const int nloc = nitems * kItem;   // local token slots (the last item may be short)
-    auto local_valid = [&](int t) { return s_list[t / kItem] * kTile + (t % kItem) < Tb; };
-#pragma unroll
-    for (int k = 0; k < NR; k++) {
-        unsigned m = 0;
-        for (int t = tid; t < nloc; t += kConsumers)
-            if (local_valid(t)) m = max(m, (unsigned)s_cf[k * cstride + t] & 0x7FFFu);
-        m = __reduce_max_sync(0xffffffffu, m);
-        if (lane == 0) atomicMax(&s_cfmax[k], m);
+    if (RESID && !mbar_wait(&bar_cf, 0, &s_abort)) {
+        s_abort = 1;
+        atomicExch(a.err, 3);
     }
     consumer_sync();
     float M[GK];
@@ -764,6 +794,10 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     // the weights' fixed-point scales: w = P * sc (anchor) or p * sc
     // (residual), |P| <= max|s_hat|, p <= 1, sc <= the stream's largest V
     // scale (powers of two)
+    if (!mbar_wait(&bar_cfmax, 0, &s_abort)) {
+        s_abort = 1;
+        atomicExch(a.err, 3);
+    }
     // record k's V weight is p times the product of the V coefficients of
     // the records after it on the chain (1 for the last), the anchor's p
     // times the product of all of them; bounds from the coefficients' maxima
@@ -779,8 +813,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     float lsum[GK];
 #pragma unroll
     for (int gq = 0; gq < GK; gq++) lsum[gq] = 0.f;
-    for (int t = tid; t < nloc; t += kConsumers) {
-        const bool valid = local_valid(t);
+    for (int t = tid; t < ntiles * kTile; t += kConsumers) {
+        const bool valid = t < n;
 #pragma unroll
         for (int gq = 0; gq < GK; gq++) {
             const float p = valid ? exp2f(s_sc[gq * a.chunk + t] - M[gq]) : 0.f;
@@ -823,17 +857,15 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 accHi[gq][e] = 0;
             }
         }
-        const int vbytes = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
         for (int j = 0; j < nitems; j++) {
-            const int it = (1 + vp) * nitems + 1 + j;   // after the K items and the sentinel
+            const int it = (1 + vp) * nitems + j;
             const int slot = it % kSlots;
             if (!mbar_wait(&bar_full[slot], (it / kSlots) & 1, &s_abort)) {
                 s_abort = 1;
                 atomicExch(a.err, 4);
             }
-            place(vbytes);
             const uint8_t *st = ring + c_off;
-            const int last_u = min(kItemTiles, nt - s_list[j]) - 1;   // a short last item
+            const int last_u = min(kItemTiles, ntiles - j * kItemTiles) - 1;   // a short last item
 #pragma unroll
             for (int u = 0; u < kItemTiles; u++) {
                 if (u > last_u) break;   // uniform
@@ -857,7 +889,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 }
                 if (u == last_u) {   // every read of the item is done: release it
                     mbar_arrive(&bar_empty[slot]);
-                    c_off += vbytes;
+                    const int cur = vp == 0 ? P::VA_BYTES : P::VR_BYTES;
+                    c_off = P::advance(c_off, cur, j + 1 < nitems ? cur : P::VR_BYTES);
                 }
                 uint32_t hi_any[2] = {0u, 0u};   // per token pair
 #pragma unroll
@@ -988,14 +1021,12 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     // ------------------------------------------------------------ last CTA of the unit combines
     __threadfence();
     consumer_sync();
+    const int unit = (b * a.H + h) * npairs + pair;
     if (tid == 0) s_last = (atomicAdd(&a.counters[unit], 1) == a.S - 1);
     consumer_sync();
     if (s_last) {
         __threadfence();
-        if (tid == 0) {   // ready for the next call
-            a.counters[unit] = 0;
-            a.tiles[unit] = 0;
-        }
+        if (tid == 0) a.counters[unit] = 0;   // ready for the next call
 #pragma unroll 1
         for (int gq = 0; gq < GK; gq++) {
             const size_t row = (size_t)b * a.Hq + hq0 + gq;

@@ -18,8 +18,7 @@
 // contents: calls whose GPU work overlaps (other streams, other threads) race
 // on it and must be ordered by the caller.  The split partials need no
 // clearing (each slot is written before it is read within a call); the last
-// 64 Ki words hold the split-combine arrival counters and the tile counters
-// of up to 32 Ki (sequence, query head) units, zeroed once at set-up and
+// 64 Ki words hold the split-combine counters, zeroed once at set-up and
 // returned to zero by every call.
 #include <mutex>
 
@@ -87,7 +86,6 @@ extern "C" int rq_decode_attn_noalloc(rq_cache *cache, int layer, int loop, cons
     float *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);
     if (st != RQ_OK) return st;
-    // the counter words: arrival counters, then the tile counters of the same units
     return rq::decode_with_scratch(cache, layer, loop, q_bf16, out, softmax_scale, stream, scratch, kPartialFloats,
-                                   reinterpret_cast<int *>(scratch + kPartialFloats), kCounterInts / 2);
+                                   reinterpret_cast<int *>(scratch + kPartialFloats), kCounterInts);
 }

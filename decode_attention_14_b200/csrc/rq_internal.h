@@ -163,7 +163,6 @@ struct DecodeArgs {
     const uint16_t *q;        // [B][Hq][d] bf16
     float *partials;          // [B][Hq][splits_max][kPartialStride]
     int *counters;            // [B * Hq] arrival counters of the fused split combine (zero between calls)
-    int *tiles;               // [B * Hq] next tile of each unit to hand out (zero between calls)
     int *err;                 // device error word (bounded waits that gave up)
     float *out;               // [B][Hq][d] fp32
     const uint16_t *tail_k, *tail_v;   // [B][tail_cap][H][d] BF16 in-flight tokens, or null
@@ -171,6 +170,11 @@ struct DecodeArgs {
     // residual V stream of every (sequence, kv head), [B][H]: upper bounds of
     // the V scales, from which the weights' fixed point is chosen
     const int *vmax_a, *vmax_r[kMaxChain];
+    // committed records below token `stable` are not written by any work
+    // that may still run when this kernel starts (see the programmatic
+    // launch in api.cpp); records from `stable` on are read only after the
+    // kernel's grid-dependency wait
+    int stable;
     int n_tail, tail_cap;
     // fused append: n_new tokens [B][n_new][H][d] written to tail rows
     // tail_pos.. (included in n_tail) by split 0 of each unit before the combine

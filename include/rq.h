@@ -26,7 +26,8 @@
  *   - Ownership: the caller owns q, k, v, out and (optionally) the cache's
  *     device arena; the library owns the host-side handle and, when it
  *     allocated the arena itself, the arena.  Once created, the arena is
- *     written only by this library's calls.
+ *     written only by this library's calls (the decode kernel relies on it:
+ *     see rq_decode_attn).
  */
 #ifndef RQ_H
 #define RQ_H
@@ -191,10 +192,12 @@ int rq_append(rq_cache *cache, int layer, int loop, const void *k_bf16, const vo
  * Keys/values seen: the committed tokens of the loop's group (anchor loop:
  * the dequantized anchor; other loops: s_hat a_hat + R^T r_hat), followed by
  * the loop's BF16 tail tokens.  With no key at all the output is zero.
- * Overlap: the kernel is launched so that its CTAs may be scheduled while
- * the previous work on `stream` is still running (programmatic dependent
- * launch); they wait for that work to complete before touching any global
- * memory, so the observable results are those of plain stream order.
+ * Overlap: the kernel is launched so that it may start while the previous
+ * work on `stream` is still running (programmatic dependent launch).  Before
+ * that work has completed it reads only committed records that no append
+ * enqueued earlier can still be writing; q, the tail, out and everything else
+ * are touched only after it.  The observable results are those of plain
+ * stream order.
  * Errors: INVALID, STATE (wrong format), CUDA.
  */
 int rq_decode_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, float *out,
@@ -268,7 +271,7 @@ int rq_prefill_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, in
  *   Limits: batch * num_q_heads * S * 132 floats must fit in 2^21 - 2^16
  *   floats (the last 2^16 words of the array hold the combine counters), S
  *   being the split count the call chooses (at most ceil(T/64)), and
- *   batch * num_q_heads must not exceed 32768; beyond either the call returns
+ *   batch * num_q_heads must not exceed 65536; beyond either the call returns
  *   RQ_ERR_CAPACITY and enqueues nothing.
  *   The first call on a device looks up the array's device address (and
  *   zeroes its counters, synchronously); make it before any stream capture.
