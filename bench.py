@@ -659,9 +659,26 @@ def run_sweep(args):
     return rows
 
 
-# FP32 lanes x 2 flops x SMs x maximum SM clock of a B200: the ALU roofline of
-# a kernel whose products run as fp32 FMAs
-FP32_PEAK_TFLOPS = 128 * 2 * 148 * 1.965e9 / 1e12
+def _bf16_peak():
+    """Dense BF16 tensor-core peak (TFLOP/s): the measured burst figure, else
+    the pool's earlier measurement."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        if "bf16_tflops" in j:
+            return float(j["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def prefill_mma_flops(n, G, B, H, T, resid):
+    """Tensor-core FLOPs rq_prefill_attn issues: per CTA step (64 query rows x
+    64 committed tokens) 9 (+17 at a residual loop) logit MMAs of 64x64x16
+    and 8 (+8) value MMAs of 64x136x16."""
+    steps = B * H * ((n * G + 63) // 64) * ((T + 63) // 64)
+    logit = (9 + (17 if resid else 0)) * 2 * 64 * 64 * 16
+    value = (8 + (8 if resid else 0)) * 2 * 64 * 136 * 16
+    return steps * (logit + value)
 
 
 def run_prefill(args):
@@ -669,7 +686,9 @@ def run_prefill(args):
     n new tokens per sequence, timed at a residual loop (the chunk in the BF16
     tail) and at the anchor loop (the chunk committed).  One JSON line per
     (n, loop kind).  FLOPs counted: 2 x 128 for q.k and 2 x 128 for p v per
-    (query row, committed token)."""
+    (query row, committed token), against the dense BF16 tensor peak; the
+    line also gives the tensor FLOPs the kernel issues (hi/lo operand
+    splits, minimum columns, rows padded to 64)."""
     import torch
     import decode_attention_14_b200 as rq
     import synth
@@ -721,13 +740,17 @@ def run_prefill(args):
             committed = T if kind == "residual" else T + n
             flops = 4.0 * 128 * n * Hq * B * committed
             tflops = flops / (us * 1e-6) / 1e12
+            mma = prefill_mma_flops(n, Hq // H, B, H, committed, kind == "residual")
+            peak, peak_kind = _bf16_peak()
             row = {"prefill": "ouro8k_b4", "n_tokens": n, "loop": kind, "batch": B, "seq_len": committed,
                    "us_per_call": round(us, 1), "query_tokens_per_s": round(B * n / (us * 1e-6), 1),
                    "decode_bytes_per_call": cache.decode_bytes(0, loop),
-                   "roofline": {"bound": "alu", "achieved": round(tflops, 2), "peak": round(FP32_PEAK_TFLOPS, 1),
-                                "unit": "TFLOP/s", "frac": round(tflops / FP32_PEAK_TFLOPS, 4),
-                                "peak_kind": "fp32 FMA lanes x clock (derived)"},
-                   "timing": "CUDA graph of %d calls, CUDA events" % reps}
+                   "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                                "frac": round(tflops / peak, 4), "peak_kind": peak_kind + " dense bf16 (burst)",
+                                "achieved_counts": "4 x 128 flops per (query row, committed token)",
+                                "mma_tflops": round(mma / (us * 1e-6) / 1e12, 2),
+                                "mma_flops_per_call": mma},
+                   "timing": "CUDA graph of %d calls (attention kernel + split combine), CUDA events" % reps}
             rows.append(row)
             print(json.dumps(row), flush=True)
         cache.check()

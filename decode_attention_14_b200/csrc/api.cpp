@@ -25,6 +25,9 @@ struct rq_cache {
     // (an anchor append) started at, over the sequences; records below it are
     // not touched by any append still in flight
     std::vector<int> wstart;
+    // a block-table change is (or may be) in flight: the next decode reads the
+    // table only after its grid-dependency wait
+    bool table_dirty = false;
     std::vector<uint32_t> sigma;   // [layer][4]: sign bits of the layer's rotation
     // resident CTAs per SM for chunk = 64 * (i + 1), by residual records read (0 .. kMaxChain)
     int occ[kMaxChain + 1][kMaxChunk / kTokTile];
@@ -174,6 +177,7 @@ int flush_ops(rq_cache *c, const PendingOps &ops, cudaStream_t st) {
             a.copy_src[a.n_copies] = ops.copies[k].first;
             a.copy_dst[a.n_copies++] = ops.copies[k].second;
         }
+        c->table_dirty = true;
         if (launch_block_ops(a, st) != cudaSuccess) return RQ_ERR_CUDA;
     }
     return RQ_OK;
@@ -274,19 +278,20 @@ bool on_cache_device(const rq_cache *c) {
 #ifndef RQ_SPLIT_OVERHEAD_TILES
 #define RQ_SPLIT_OVERHEAD_TILES 2
 #endif
-void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *chunk) {
+void choose_splits(const rq_cache *c, int T, int units, int which, int gran, int *S, int *chunk) {
     if (T <= 0) {
         *S = 0;
         *chunk = kTokTile;
         return;
     }
+    const int nt = (T + kTokTile - 1) / kTokTile;
+    const int nu = (nt + gran - 1) / gran;   // granules (kMaxChunk is a whole number of them)
     const int s_lo = (T + kMaxChunk - 1) / kMaxChunk;
-    const int s_hi = std::min(c->lay.splits_max, (T + kTokTile - 1) / kTokTile);
+    const int s_hi = std::min(c->lay.splits_max, nu);
     long best_cost = -1;
     int best_s = s_lo, best_ch = kMaxChunk;
-    const int nt = (T + kTokTile - 1) / kTokTile;
     for (int s = s_lo; s <= std::max(s_lo, s_hi); s++) {
-        const int ch = (nt + s - 1) / s * kTokTile;
+        const int ch = (nu + s - 1) / s * gran * kTokTile;
         const int ss = s;
         const int slots = std::max(1, c->occ[which][ch / kTokTile - 1] * c->sms);
         const long waves = ((long)ss * units + slots - 1) / slots;
@@ -300,7 +305,7 @@ void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *
 #ifdef RQ_SPLIT_FORCE_S
     if (RQ_SPLIT_FORCE_S >= s_lo && RQ_SPLIT_FORCE_S <= std::max(s_lo, s_hi)) {
         best_s = RQ_SPLIT_FORCE_S;
-        best_ch = (nt + best_s - 1) / best_s * kTokTile;
+        best_ch = (nu + best_s - 1) / best_s * gran * kTokTile;
     }
 #endif
     *S = best_s;
@@ -666,6 +671,11 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
         a.vmax_a = vmax_ptr(c, layer, group, L.Lg - 1);
         a.stable = c->wstart[(size_t)layer * L.groups + group];
+        if (L.paged && c->table_dirty) {
+            // the table may have changed in the kernel just before this one
+            a.stable = 0;
+            c->table_dirty = false;
+        }
         if (!is_commit_loop(L, loop)) {
             a.n_tail = c->ntail[(size_t)layer * cfg.num_loops + loop];
             a.tail_k = (const uint16_t *)tail_ptr(c, layer, group, j, 0);
@@ -687,7 +697,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
-    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, &a.S, &a.chunk);
+    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, split_granule(a.pg), &a.S, &a.chunk);
     if (partials) {
         a.splits_max = std::max(a.S, 1);
         if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;
@@ -841,6 +851,7 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
         c->prefill_ws_floats = need;
     }
     a.partials = c->prefill_ws;
+    a.err = (int *)(c->base + L.off_err);
     return cuda_status(launch_prefill(a, cfg.anchor_bits, cfg.resid_bits, (cudaStream_t)stream));
 }
 

@@ -64,6 +64,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "rq_internal.h"
+#include "sync.cuh"
 
 #ifdef RQ_FAULT_INJECT
 // Test builds only (never the shipped library): when set, the next decode
@@ -103,66 +104,15 @@ static_assert(kRingBytes % 128 == 0, "ring must be a multiple of 128 bytes");
 constexpr int kConsumers = 128;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kRsqrt128 = 0.088388347648318440f;
-#ifndef RQ_WAIT_NS
-#define RQ_WAIT_NS 1000000000ull
-#endif
-constexpr unsigned long long kWaitNs = RQ_WAIT_NS;      // limit of one wait (1 s by default)
 constexpr int kWeightTop = 22;                          // V weight bound in [2^21, 2^22) (fixed point)
 #ifndef RQ_DECODE_PDL
 #define RQ_DECODE_PDL 1
 #endif
 
 // ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-#ifndef RQ_POLLS_PER_CHECK
-#define RQ_POLLS_PER_CHECK 4
-#endif
-// Bounded wait on an mbarrier phase; gives up after kWaitNs or as soon as
-// another warp of the CTA has given up.  SLEEP_NS > 0 backs off between
-// polls (for waits whose latency does not matter).  The abort flag and the
-// clock are checked once per RQ_POLLS_PER_CHECK polls: a poll is two
-// instructions, the checks several more, and waiting warps share the
-// schedulers with working ones.
-template <unsigned SLEEP_NS = 0>
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    for (;;) {
-#pragma unroll
-        for (int i = 0; i < RQ_POLLS_PER_CHECK; i++) {
-            if (SLEEP_NS) __nanosleep(SLEEP_NS);
-            if (mbar_try_wait(bar, parity)) return true;
-        }
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitNs) return false;
-    }
 }
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
@@ -421,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int hq0 = h * a.G + pair * GK;
     int t0, n;   // this split's tokens of its sequence (none when the sequence is short)
-    split_range(split, a.S, a.seqT.v[b], &t0, &n);
+    split_range(split, a.S, a.seqT.v[b], &t0, &n, split_granule(a.pg));
     const int ntiles = (n + kTile - 1) / kTile;
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
@@ -448,14 +398,16 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     // ------------------------------------------------------------ producer
     if (warp == 4) {
         // paged records: the chunk's physical blocks, read once into shared
-        // memory (after the grid dependency wait: the table may just have
-        // been written)
+        // memory (through L2).  Before the grid dependency wait only when the
+        // whole chunk lies below a.stable: the host sets a.stable to 0 when a
+        // block-table change may be in flight, so such rows are settled.
         const bool paged = a.pg.table != nullptr;
+        const bool early = paged && t0 + ntiles * kTile <= a.stable;
         const int blk0 = t0 >> a.pg.shift;
         if (paged) {
-            griddep_wait_then_release();
+            if (!early) griddep_wait_then_release();
             const int nblk = ntiles > 0 ? ((t0 + ntiles * kTile - 1) >> a.pg.shift) - blk0 + 1 : 0;
-            if (lane < nblk) s_blk[lane] = a.pg.table[(size_t)b * a.pg.mb + blk0 + lane];
+            if (lane < nblk) s_blk[lane] = __ldcg(a.pg.table + (size_t)b * a.pg.mb + blk0 + lane);
             __syncwarp();
         }
         if (lane == 0) {
@@ -480,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // records of tokens [.., tok_end) may be read before the grid
             // dependency wait only if all of them lie below a.stable (padding
             // beyond the sequence's length is read but never used)
-            bool waited = paged;
+            bool waited = paged && !early;
             auto dep = [&](int tok_end) {
                 if (!waited && t0 + tok_end > a.stable) {
                     griddep_wait_then_release();

@@ -6,25 +6,48 @@
 // loop's BF16 tail tokens]: the n new tokens are the most recent ones,
 // committed already at an anchor loop, in the tail at the other loops.
 //
-// Design.  With n query tokens per sequence the keys are shared by n * G
-// query rows, so a CTA dequantizes each record once into shared memory in
-// fp32 (k_hat = s_hat a_hat + R^T y_hat; the inverse rotation is one warp
-// Walsh-Hadamard transform per token, cheaper than rotating n * G queries
-// once the rows outnumber a few) and runs both products, logits and p V, on
-// the FP32 pipes from shared memory:
-//  - CTA = (split of the committed tokens, kv head, sequence x block of
-//    8 RPW query rows, RPW in {1, 2, 4, 8} the fewest that hold a kv head's
-//    n * G rows), 8 warps; warp w owns rows w, w + 8, ...;
-//  - per 32-token step: dequantize K (warp per token), logits (lane = token,
-//    a row's 32 logits in one warp), online softmax per row, dequantize V,
-//    o += p V (lane = 4 columns of head_dim); the raw records of the next
-//    step are copied into a second shared buffer (cp.async) meanwhile;
-//  - each CTA writes a partial (m, l, o) per row; a second kernel merges the
-//    partials and the tail tokens of each row (combine_row) under the row's
-//    causal limit.
-// This is a CUDA-core kernel: the contraction per step is at most 64 x 32 x
-// 128 twice, on fp32 reconstructions; BF16 tensor-core operands would add a
-// rounding of every reconstructed key and value.
+// Algebra.  A committed token's key and value are k = s a + R^T y (anchor a,
+// rotated residual y, least-squares coefficient s; at an anchor loop k = a),
+// and per quantization group each of a and y is sc * code + mn.  So
+//   q.k   = s (q.(sc code) + sum_g mn_g Q_g) + (Rq).(sc_r code_r) + sum_g mn_rg (Rq)_g
+//   sum_t p_t v_t = A + R^T Y,  A = sum_t (p_t s_t) a_t,  Y = sum_t p_t y_t
+// (Q_g, (Rq)_g: sums of the group's elements).  Every product of that runs on
+// the tensor cores with operands that BF16 holds exactly or nearly so:
+//  - sc * code (a 4-significant-bit FP8 scale times a code below 16) and the
+//    FP8 minima are exact in BF16, and so is q itself;
+//  - Rq, the group sums and the probabilities p and p s are fp32 values
+//    split into a BF16 high part and a BF16 low part (relative 2^-17), whose
+//    two products accumulate into the same fp32 tensor-memory accumulator;
+//  - the minima ride along as extra K columns of the logit products (group
+//    sums of q against the minima of the keys) and as extra N rows of the
+//    value products (probabilities against the minima of the values).
+// R^T is applied once per CTA to the accumulated Y.  Per 64-token step and
+// 64 query rows:
+//   SA = [q | Q_g] [sc code | mn]^T            (9 MMAs of 64x64x16)
+//   SY = [Rq_hi | (Rq)_g] [..]^T + Rq_lo [..]^T (17 MMAs)
+//   OA += (p s)_hi [sc code | mn] + (p s)_lo [..]   (8 MMAs of 64x136x16)
+//   OY += p_hi [sc_r code_r | mn_r] + p_lo [..]     (8 MMAs)
+// with logits scale_log2 (s SA + SY) and a running maximum that is only
+// raised when a row's maximum grows by more than 2^8 (then that row of OA and
+// OY is rescaled in tensor memory); the partial (m, l, o) of each row goes to
+// a second kernel that merges the splits and the tail tokens (combine_row).
+//
+// CTA = (split of the committed tokens, kv head, sequence x block of 64 query
+// rows); 13 warps:
+//  - warps 0-3: softmax -- warp w owns tensor-memory lanes 32w.. and query
+//    rows 16w..16w+15 (the M=64 accumulator layout); loads the logits,
+//    writes the probability operands, rescales, and at the end reads OA and
+//    OY, applies R^T and writes the partial;
+//  - warp 4: allocates tensor memory; one thread issues every MMA;
+//  - warps 5-12: dequantize the step's K and V records (straight from global
+//    memory) into the swizzled operand tiles.
+// Hand-offs go through mbarriers, every wait bounded (error word, abort flag):
+//   kfull/vfull   dequant -> MMA       K / V operands of step j written
+//   cfull[j & 1]  dequant -> softmax   coefficients of step j written
+//   kdone         MMA commit           logits of step j complete (K tile free)
+//   sfree         softmax -> MMA       logits of step j read (SA/SY free)
+//   pfull         softmax -> MMA       probabilities of step j written
+//   odone         MMA commit           values of step j complete (V and P free)
 #include <math_constants.h>
 
 #include <algorithm>
@@ -32,257 +55,551 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "prefill.h"
+#include "sync.cuh"
+#include "tc.cuh"
 
 namespace rq {
 namespace {
 
-constexpr int kThreadsP = 256;
-constexpr int kQStride = kHeadDim + 4;   // float4-aligned query rows
-constexpr int kKStride = kHeadDim + 1;   // lane = token reads a column without bank conflicts
-constexpr int kPStride = kPrefillTile + 1;
-// shared floats of a CTA of `rows` query rows: q, one reconstructed tile, probabilities
-__host__ __device__ constexpr int float_smem(int rows) {
-    return rows * kQStride + kPrefillTile * kKStride + rows * kPStride;
-}
+constexpr int kRows = 64;             // query rows of a CTA (M of every MMA)
+constexpr int kTok = kPrefillTile;    // committed tokens per step
+constexpr int kSoftmaxWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kDeqWarps = 8;
+constexpr int kDeqThreads = 32 * kDeqWarps;
+constexpr int kThreadsP = 32 * (kSoftmaxWarps + 1 + kDeqWarps);
+constexpr int kBlk = kRows * 128;     // one 64-row block of 64 bf16 columns (8 KB)
+static_assert(kTok == kRows, "K/V tiles and query tiles share the 64-row block");
+// Operand tiles: a 3-block tile holds head_dim (blocks 0, 1) and the 16
+// minimum / group-sum columns (first 32 bytes of each row of block 2).
+constexpr int OFF_Q = 0;              // q | Q_g hi, lo
+constexpr int OFF_QRH = 3 * kBlk;     // Rq hi | (Rq)_g hi, lo
+constexpr int OFF_QRL = 6 * kBlk;     // Rq lo
+constexpr int OFF_KA = 8 * kBlk;      // anchor K: sc code | mn, mn
+constexpr int OFF_KY = 11 * kBlk;     // residual K
+constexpr int OFF_VA = 14 * kBlk;     // anchor V (read MN-major)
+constexpr int OFF_VY = 17 * kBlk;     // residual V
+constexpr int OFF_PSH = 20 * kBlk;    // (p s) hi, then lo, p hi, p lo: one block each
+constexpr int kTilesBytes = 24 * kBlk;
+constexpr int kSmemBytes = kTilesBytes + 1024;   // + alignment of the base to 1024
+// tensor-memory columns (fp32): logits of a step, then the value accumulators
+constexpr uint32_t kColSA = 0, kColSY = 64, kColOA = 128, kColOY = 272, kTmemCols = 512;
+constexpr int kOCols = kHeadDim + 8;             // head_dim + one column per group minimum
+constexpr float kRescaleLog2 = 8.f;              // raise a row's maximum only past 2^8
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
 
-// Raw records of one 32-token tile, K then V, each side laid out
-// [anchor codes][anchor meta][residual codes][residual meta][coefficients]
-// (meta sized for the largest, group 16); two such stages are in flight.
-template <int BA, int BR>
-struct Stage {
-    static constexpr int A_C = 16 * BA, R_C = 16 * BR, MR_MAX = 16;
-    static constexpr int SIDE = kPrefillTile * (A_C + R_C + 2 * MR_MAX) + 2 * kPrefillTile;
-    static constexpr int BYTES = 2 * SIDE;
-    static constexpr size_t smem(int rows) { return (size_t)float_smem(rows) * sizeof(float) + 2 * (size_t)BYTES; }
-};
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+__device__ __forceinline__ uint32_t bf16_bits(float x) { return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
+// high and low BF16 parts of x, packed as the low halves of two words
+__device__ __forceinline__ void split_hi_lo(float x, uint32_t &hi, uint32_t &lo) {
+    hi = bf16_bits(x);
+    lo = bf16_bits(x - bf16_val(hi));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
-// bytes (a multiple of 16, both addresses 16-byte aligned) spread over the CTA
-__device__ __forceinline__ void copy_async(uint8_t *dst, const uint8_t *src, int bytes, int tid) {
-    for (int o = 16 * tid; o < bytes; o += 16 * kThreadsP) cp_async16(dst + o, src + o);
+__device__ __forceinline__ void st_shared16(uint8_t *p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_shared8(uint8_t *p, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(p)), "r"(x), "r"(y) : "memory");
 }
 
-// Issue the copies of the tile whose first record is rec0 (a multiple of 32:
-// every source is 16-byte aligned, and a whole tile lies inside the stream's
-// padded capacity).
-template <int BA, int BR>
-__device__ __forceinline__ void stage_tile(const PrefillArgs &a, uint8_t *st, size_t rec0, int MR, bool resid,
-                                           int tid) {
-    using SG = Stage<BA, BR>;
-    constexpr int TT = kPrefillTile;
-#pragma unroll
-    for (int kv = 0; kv < 2; kv++) {
-        uint8_t *d = st + kv * SG::SIDE;
-        copy_async(d, a.a_codes[kv] + rec0 * SG::A_C, TT * SG::A_C, tid);
-        copy_async(d + TT * SG::A_C, a.a_meta[kv] + rec0 * MR, TT * MR, tid);
-        if (resid) {
-            copy_async(d + TT * (SG::A_C + MR), a.r_codes[kv] + rec0 * SG::R_C, TT * SG::R_C, tid);
-            copy_async(d + TT * (SG::A_C + MR + SG::R_C), a.r_meta[kv] + rec0 * MR, TT * MR, tid);
-            copy_async(d + TT * (SG::A_C + SG::R_C + 2 * MR), reinterpret_cast<const uint8_t *>(a.r_coef[kv] + rec0),
-                       2 * TT, tid);
-        }
-    }
-}
-
-// The codes of elements 4 lane .. 4 lane + 3 of a record, LSB first.
+// BF16 pair (128 + code of element 2p, 128 + code of element 2p + 1) of a
+// word of BITS-bit codes, LSB first: 0x4300 is 128.0 with one unit per code.
 template <int BITS>
-__device__ __forceinline__ uint32_t lane_codes(const uint8_t *rec, int lane) {
-    if (BITS == 4) return *reinterpret_cast<const uint16_t *>(rec + 2 * lane);
-    return rec[lane];
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int p) {
+    if (BITS == 4) {
+        const uint32_t t = w >> (8 * p);
+        return 0x43004300u | (t & 0xFu) | ((t & 0xF0u) << 12);
+    }
+    const uint32_t t = w >> (4 * p);
+    return 0x43004300u | (t & 0x3u) | ((t & 0xCu) << 14);
 }
 
-// Reconstruct side kv of the staged tile, tokens 0 .. tn - 1, into rows
-// 0 .. tn - 1 of sK (rows tn .. 31 zeroed); warp per token, lane holds
-// elements 4 lane .. 4 lane + 3.
-template <int BA, int BR>
-__device__ __forceinline__ void dequant_tile(const PrefillArgs &a, const uint8_t *st, int kv, int MR, bool resid,
-                                             int tn, float *sK, int warp, int lane) {
-    using SG = Stage<BA, BR>;
-    constexpr int TT = kPrefillTile;
-    const uint8_t *d = st + kv * SG::SIDE;
-    const int gi = (4 * lane) / a.g;   // quantization group of this lane's elements
+// Dequantize half HALF (head_dim elements 64 HALF .. 64 HALF + 63) of one
+// record into row t of a 3-block operand tile: sc * code per element, exact
+// in BF16 ((128 + code) sc - 128 sc in one rounding); HALF 0 also writes the
+// minimum columns (mn_0 .. mn_{NG-1}, zeros, twice).  A token past the step
+// (ok false) gets a zero row.
+template <int BITS, int GS, int HALF>
+__device__ __forceinline__ void deq_half(uint8_t *tile, int t, const uint8_t *codes, const uint8_t *meta, bool ok) {
+    constexpr int NG = kHeadDim / GS, MR = 2 * NG;
+    uint8_t *row = tile + HALF * kBlk;
+    uint8_t *mrow = tile + 2 * kBlk;
+    if (!ok) {
 #pragma unroll
-    for (int u = warp; u < TT; u += kThreadsP / 32) {
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (u < tn) {
-            const uint32_t w = lane_codes<BA>(d + u * SG::A_C, lane);
-            const uint8_t *mp = d + TT * SG::A_C + u * MR + 2 * gi;
-            const float sc = e4m3_to_f32(mp[0]), mn = e4m3_to_f32(mp[1]);
-#pragma unroll
-            for (int k = 0; k < 4; k++) x[k] = fmaf((float)((w >> (BA * k)) & ((1u << BA) - 1)), sc, mn);
-            if (resid) {
-                const float sh =
-                    bf16_to_f32(reinterpret_cast<const uint16_t *>(d + TT * (SG::A_C + SG::R_C + 2 * MR))[u]);
-                const uint32_t wr = lane_codes<BR>(d + TT * (SG::A_C + MR) + u * SG::R_C, lane);
-                const uint8_t *mr = d + TT * (SG::A_C + MR + SG::R_C) + u * MR + 2 * gi;
-                const float rs = e4m3_to_f32(mr[0]), rm = e4m3_to_f32(mr[1]);
-                float y[4];
-#pragma unroll
-                for (int k = 0; k < 4; k++) y[k] = fmaf((float)((wr >> (BR * k)) & ((1u << BR) - 1)), rs, rm);
-                if (a.rotate) {
-                    // R^T y = diag(sigma) H y / sqrt(d)
-                    wht128_warp(y, lane);
-#pragma unroll
-                    for (int k = 0; k < 4; k++) y[k] *= sigma_neg(a.sigma, 4 * lane + k) ? -kInvSqrtD : kInvSqrtD;
-                }
-#pragma unroll
-                for (int k = 0; k < 4; k++) x[k] = fmaf(sh, x[k], y[k]);
-            }
+        for (int c = 0; c < 8; c++) st_shared16(row + tc::sw_chunk(t, c), 0u, 0u, 0u, 0u);
+        if (HALF == 0) {
+            st_shared16(mrow + tc::sw_chunk(t, 0), 0u, 0u, 0u, 0u);
+            st_shared16(mrow + tc::sw_chunk(t, 1), 0u, 0u, 0u, 0u);
         }
+        return;
+    }
+    // 64 codes: 8 BITS bytes
+    uint32_t w[2 * BITS];
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + 8 * BITS * HALF);
 #pragma unroll
-        for (int k = 0; k < 4; k++) sK[u * kKStride + 4 * lane + k] = x[k];
+        for (int u = 0; u < BITS / 2; u++) {
+            const uint4 v = __ldg(src + u);
+            w[4 * u] = v.x;
+            w[4 * u + 1] = v.y;
+            w[4 * u + 2] = v.z;
+            w[4 * u + 3] = v.w;
+        }
+    }
+    // (scale, minimum) FP8 byte pairs of all groups
+    uint32_t mw[MR / 4];
+    if (MR == 16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(meta));
+        mw[0] = v.x;
+        mw[1 % (MR / 4)] = v.y;
+        mw[2 % (MR / 4)] = v.z;
+        mw[3 % (MR / 4)] = v.w;
+    } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(meta));
+        mw[0] = v.x;
+        mw[1] = v.y;
+    }
+    constexpr int GPH = 64 / GS;   // groups of this half
+#pragma unroll
+    for (int gl = 0; gl < GPH; gl++) {
+        constexpr int CPG = GS / 8;   // 16-byte chunks per group
+        const int gi = HALF * GPH + gl;
+        const uint32_t pr = (mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+        const float sc = e4m3_to_f32(pr & 0xFFu);
+        const uint32_t s2 = bf16_bits(sc) * 0x10001u;
+        const uint32_t nb2 = bf16_bits(-128.f * sc) * 0x10001u;
+#pragma unroll
+        for (int cg = 0; cg < CPG; cg++) {
+            const int c = gl * CPG + cg;   // chunk of the half: elements 8c .. 8c + 7
+            const uint32_t cw = BITS == 4 ? w[c] : (w[c >> 1] >> (16 * (c & 1)));
+            st_shared16(row + tc::sw_chunk(t, c), fma_bf16x2(code_pair<BITS>(cw, 0), s2, nb2),
+                        fma_bf16x2(code_pair<BITS>(cw, 1), s2, nb2), fma_bf16x2(code_pair<BITS>(cw, 2), s2, nb2),
+                        fma_bf16x2(code_pair<BITS>(cw, 3), s2, nb2));
+        }
+    }
+    if (HALF == 0) {
+        uint32_t m[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            uint32_t lo = 0u, hi = 0u;
+            if (2 * k < NG) lo = bf16_bits(e4m3_to_f32((mw[k % (MR / 4)] >> 8) & 0xFFu));
+            if (2 * k + 1 < NG) hi = bf16_bits(e4m3_to_f32((mw[k % (MR / 4)] >> 24) & 0xFFu));
+            m[k] = lo | (hi << 16);
+        }
+        st_shared16(mrow + tc::sw_chunk(t, 0), m[0], m[1], m[2], m[3]);
+        st_shared16(mrow + tc::sw_chunk(t, 1), m[0], m[1], m[2], m[3]);
     }
 }
 
-// RPW query rows per warp (8 RPW per CTA); fewer rows leave room for more CTAs per SM
-template <int BA, int BR, int RPW>
-__global__ void __launch_bounds__(kThreadsP, RPW <= 2 ? 4 : RPW == 4 ? 3 : 2) prefill_rq_kernel(const PrefillArgs a) {
-    using SG = Stage<BA, BR>;
-    constexpr int ROWS = 8 * RPW;
-    extern __shared__ __align__(16) float smem[];
-    float *sQ = smem;                                  // [ROWS][kQStride] q * scale * log2(e)
-    float *sK = sQ + ROWS * kQStride;                  // [32][kKStride] reconstructed K, then V
-    float *sP = sK + kPrefillTile * kKStride;          // [ROWS][kPStride] probabilities of the step
-    uint8_t *sRaw = reinterpret_cast<uint8_t *>(smem + float_smem(ROWS));   // 2 stages of raw records
+// Query operands of the CTA's 64 rows (rows past nr are zero): q and its
+// group sums (hi, lo) into OFF_Q; for a residual loop Rq hi / lo and the
+// group sums of Rq (hi, lo) into OFF_QRH / OFF_QRL.  A warp per row.
+template <int GS, bool RESID>
+__device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm, int b, int h, int r0, int nr,
+                                              int warp, int lane) {
+    constexpr int NG = kHeadDim / GS, LPG = GS / 4;   // lanes per group
+    for (int r = warp; r < kRows; r += kThreadsP / 32) {
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        uint2 raw = make_uint2(0u, 0u);
+        if (r < nr) {
+            const int rg = r0 + r, i = rg / a.G, gq = rg % a.G;
+            const uint16_t *qrow = a.q + (((size_t)b * a.n + i) * a.Hq + h * a.G + gq) * kHeadDim;
+            raw = *reinterpret_cast<const uint2 *>(qrow + 4 * lane);
+            x[0] = bf16_val(raw.x & 0xFFFFu);
+            x[1] = bf16_val(raw.x >> 16);
+            x[2] = bf16_val(raw.y & 0xFFFFu);
+            x[3] = bf16_val(raw.y >> 16);
+        }
+        // elements 4 lane .. 4 lane + 3: block lane / 16, chunk (lane % 16) / 2, half (lane & 1)
+        const uint32_t off = (uint32_t)(lane >> 4) * kBlk + tc::sw_chunk(r, (lane & 15) >> 1) + 8u * (lane & 1);
+        st_shared8(sm + OFF_Q + off, raw.x, raw.y);
+        // group sums (hi, lo) into columns 128 + g and 136 + g
+        auto sums = [&](const float v[4], uint8_t *tile) {
+            float gs = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+            for (int o = 1; o < LPG; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+            uint32_t hi[8], lo[8];
+#pragma unroll
+            for (int g = 0; g < 8; g++) {
+                const float s = __shfl_sync(0xffffffffu, gs, (g % NG) * LPG);
+                split_hi_lo(s, hi[g], lo[g]);
+                if (g >= NG) hi[g] = lo[g] = 0u;
+            }
+            if (lane == 0) {
+                uint8_t *mrow = tile + 2 * kBlk;
+                st_shared16(mrow + tc::sw_chunk(r, 0), hi[0] | hi[1] << 16, hi[2] | hi[3] << 16, hi[4] | hi[5] << 16,
+                            hi[6] | hi[7] << 16);
+                st_shared16(mrow + tc::sw_chunk(r, 1), lo[0] | lo[1] << 16, lo[2] | lo[3] << 16, lo[4] | lo[5] << 16,
+                            lo[6] | lo[7] << 16);
+            }
+        };
+        sums(x, sm + OFF_Q);
+        if (RESID) {
+            // R q = H diag(sigma) q / sqrt(d)
+            float y[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) y[k] = (a.rotate && sigma_neg(a.sigma, 4 * lane + k)) ? -x[k] : x[k];
+            if (a.rotate) {
+                wht128_warp<float>(y, lane);
+#pragma unroll
+                for (int k = 0; k < 4; k++) y[k] *= kInvSqrtD;
+            }
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) split_hi_lo(y[k], hi[k], lo[k]);
+            st_shared8(sm + OFF_QRH + off, hi[0] | hi[1] << 16, hi[2] | hi[3] << 16);
+            st_shared8(sm + OFF_QRL + off, lo[0] | lo[1] << 16, lo[2] | lo[3] << 16);
+            sums(y, sm + OFF_QRH);
+        }
+    }
+}
+
+template <int BA, int BR, int GS, bool RESID>
+__global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar_kfull, bar_vfull, bar_kdone, bar_odone, bar_sfree, bar_pfull, bar_cfull[2];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ float s_cK[2][kTok], s_cV[2][kTok];   // coefficients of the step (1 at an anchor loop)
+    __shared__ float s_ml[kRows][2];                  // running maximum and sum of each row
+
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
+    const uint32_t sbase = smem_u32(sm);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, h = blockIdx.y;
     const int b = blockIdx.z / a.nqb, qb = blockIdx.z % a.nqb;
-    const int r0 = qb * ROWS;                                   // first query row (i * G + gq) of the CTA
-    const int nr = min(ROWS, a.n * a.G - r0);                   // rows of the CTA
+    const int r0 = qb * kRows;
+    const int nr = min(kRows, a.n * a.G - r0);
     const int Tb = a.seqT.v[b];
     int t0, cnt;
     split_range(split, a.S, Tb, &t0, &cnt);
+    const int ntl = cnt > 0 ? (cnt + kTok - 1) / kTok : 0;
     const size_t bh = (size_t)b * a.H + h;
-    const int MR = 2 * (kHeadDim / a.g);
-    const bool resid = a.r_codes[0] != nullptr;
-    const int ntl = (cnt + kPrefillTile - 1) / kPrefillTile;
+    constexpr int MR = 2 * (kHeadDim / GS);
 
-    if (ntl > 0) stage_tile<BA, BR>(a, sRaw, bh * a.Tp + t0, MR, resid, tid);
-    cp_async_commit();
-
-    for (int idx = tid; idx < ROWS * kHeadDim; idx += kThreadsP) {
-        const int r = idx / kHeadDim, d = idx % kHeadDim;
-        float v = 0.f;
-        if (r < nr) {
-            const int rg = r0 + r, i = rg / a.G, gq = rg % a.G;
-            v = bf16_to_f32(a.q[(((size_t)b * a.n + i) * a.Hq + h * a.G + gq) * kHeadDim + d]) * a.scale_log2;
+    if (tid == 0) {
+        mbar_init(&bar_kfull, kDeqThreads);
+        mbar_init(&bar_vfull, kDeqThreads);
+        mbar_init(&bar_kdone, 1);
+        mbar_init(&bar_odone, 1);
+        mbar_init(&bar_sfree, 32 * kSoftmaxWarps);
+        mbar_init(&bar_pfull, 32 * kSoftmaxWarps);
+        mbar_init(&bar_cfull[0], kTok);
+        mbar_init(&bar_cfull[1], kTok);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kMmaWarp) {
+        tc::alloc(&s_tmem, kTmemCols);
+        tc::relinquish();
+    }
+    setup_queries<GS, RESID>(a, sm, b, h, r0, nr, warp, lane);
+    tc::fence_async_smem();
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = s_tmem;
+    volatile int *abort_flag = &s_abort;
+    auto wait = [&](uint64_t *bar, int parity, int code) {
+        if (!mbar_wait(bar, (uint32_t)parity, abort_flag)) {
+            *abort_flag = 1;
+            atomicExch(a.err, code);
         }
-        sQ[r * kQStride + d] = v;
-    }
-    // this warp's rows: warp + 8 j for j < jn
-    const int jn = nr > warp ? (nr - warp + 7) / 8 : 0;
-    int lim[RPW];   // committed tokens each row may see
-    float m[RPW], l[RPW], acc[RPW][4];
-#pragma unroll
-    for (int j = 0; j < RPW; j++) {
-        const int i = (r0 + warp + 8 * j) / a.G;
-        lim[j] = min(Tb, Tb + a.n_tail - a.n + 1 + i);
-        m[j] = -CUDART_INF_F;
-        l[j] = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; k++) acc[j][k] = 0.f;
-    }
+    };
 
-    for (int kt = 0; kt < ntl; kt++) {
-        const int tt = kt * kPrefillTile;
-        const int tn = min(kPrefillTile, cnt - tt);
-        const uint8_t *st = sRaw + (kt & 1) * SG::BYTES;
-        // the next tile's copies overlap this tile's work; its stage was
-        // released by the barrier that ended the step before
-        if (kt + 1 < ntl)
-            stage_tile<BA, BR>(a, sRaw + ((kt + 1) & 1) * SG::BYTES, bh * a.Tp + t0 + tt + kPrefillTile, MR,
-                               resid, tid);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();   // this tile's records (and, first time, sQ) are visible
-        dequant_tile<BA, BR>(a, st, 0, MR, resid, tn, sK, warp, lane);
-        __syncthreads();
-        // logits of token lane for the warp's rows
-        float s[RPW];
+    if (warp < kSoftmaxWarps) {
+        // ------------------------------------------------------- softmax
+        const bool own = lane < 16;                   // lanes 16..31 hold no row (M = 64 layout)
+        const int r = 16 * warp + (lane & 15);
+        const int iq = (r0 + r) / a.G;
+        const int lim = min(Tb, Tb + a.n_tail - a.n + 1 + iq);   // committed tokens the row may see
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        float m_used = -CUDART_INF_F, l = 0.f;
+        for (int j = 0; j < ntl; j++) {
+            const int tt = j * kTok;
+            const int tn = min(kTok, cnt - tt);
+            wait(&bar_cfull[j & 1], (j >> 1) & 1, 21);   // the step's coefficients
+            wait(&bar_kdone, j & 1, 22);
+            tc::fence_after();
+            float s[kTok];
 #pragma unroll
-        for (int j = 0; j < RPW; j++) s[j] = 0.f;
-        const float *kr = sK + lane * kKStride;
-#pragma unroll 2
-        for (int d = 0; d < kHeadDim; d += 4) {
-            const float k0 = kr[d], k1 = kr[d + 1], k2 = kr[d + 2], k3 = kr[d + 3];
+            for (int c = 0; c < kTok; c += 16) {
+                uint32_t va[16], vy[16];
+                tc::ld16(tl + kColSA + c, va);
+                if (RESID) {
+                    tc::ld16(tl + kColSY + c, vy);
+                    tc::wait_ld2(va, vy);
+                } else {
+                    tc::wait_ld(va);
+                }
 #pragma unroll
-            for (int j = 0; j < RPW; j++) {
-                if (j < jn) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(sQ + (warp + 8 * j) * kQStride + d);
-                    s[j] = fmaf(qv.x, k0, fmaf(qv.y, k1, fmaf(qv.z, k2, fmaf(qv.w, k3, s[j]))));
+                for (int k = 0; k < 16; k++) {
+                    const float sa = __uint_as_float(va[k]);
+                    const float x = RESID ? fmaf(s_cK[j & 1][c + k], sa, __uint_as_float(vy[k])) : sa;
+                    s[c + k] = x * a.scale_log2;
+                }
+            }
+            tc::fence_before();
+            mbar_arrive(&bar_sfree);
+            float mx = -CUDART_INF_F;
+#pragma unroll
+            for (int t = 0; t < kTok; t++) {
+                const bool ok = own && t < tn && t0 + tt + t < lim;
+                s[t] = ok ? s[t] : -CUDART_INF_F;
+                mx = fmaxf(mx, s[t]);
+            }
+            // the previous step's values are complete: P is free, O is final
+            if (j > 0) wait(&bar_odone, (j - 1) & 1, 23);
+            tc::fence_after();
+            const bool raise = mx > m_used + kRescaleLog2;   // false while nothing is seen (both -inf)
+            const bool rescale = raise && m_used != -CUDART_INF_F;
+            const float f = rescale ? exp2f(m_used - mx) : 1.f;
+            if (raise) m_used = mx;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // this row's accumulated values times f (rows without a raise times 1)
+#pragma unroll 1
+                for (int c = 0; c < kHeadDim; c += 16) {
+                    uint32_t v[16];
+                    tc::ld16(tl + kColOA + c, v);
+                    tc::wait_ld(v);
+#pragma unroll
+                    for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
+                    tc::st16(tl + kColOA + c, v);
+                    if (RESID) {
+                        tc::ld16(tl + kColOY + c, v);
+                        tc::wait_ld(v);
+#pragma unroll
+                        for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
+                        tc::st16(tl + kColOY + c, v);
+                    }
+                }
+                uint32_t v8[8];
+                tc::ld8(tl + kColOA + kHeadDim, v8);
+                tc::wait_ld8(v8);
+#pragma unroll
+                for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
+                tc::st8(tl + kColOA + kHeadDim, v8);
+                if (RESID) {
+                    tc::ld8(tl + kColOY + kHeadDim, v8);
+                    tc::wait_ld8(v8);
+#pragma unroll
+                    for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
+                    tc::st8(tl + kColOY + kHeadDim, v8);
+                }
+                tc::wait_st();
+            }
+            l *= f;
+            // probabilities of the step, split hi / lo, into the A operands
+            const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
+            uint8_t *prow = sm + OFF_PSH;
+#pragma unroll
+            for (int cc = 0; cc < kTok / 8; cc++) {
+                uint32_t psh[8], psl[8], ph[8], pl[8];
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    const int t = 8 * cc + k;
+                    const float p = exp2f(s[t] - mu);   // 0 for a masked token
+                    l += p;
+                    split_hi_lo(RESID ? p * s_cV[j & 1][t] : p, psh[k], psl[k]);
+                    if (RESID) split_hi_lo(p, ph[k], pl[k]);
+                }
+                if (own) {
+                    const uint32_t o = tc::sw_chunk(r, cc);
+                    st_shared16(prow + o, psh[0] | psh[1] << 16, psh[2] | psh[3] << 16, psh[4] | psh[5] << 16,
+                                psh[6] | psh[7] << 16);
+                    st_shared16(prow + kBlk + o, psl[0] | psl[1] << 16, psl[2] | psl[3] << 16,
+                                psl[4] | psl[5] << 16, psl[6] | psl[7] << 16);
+                    if (RESID) {
+                        st_shared16(prow + 2 * kBlk + o, ph[0] | ph[1] << 16, ph[2] | ph[3] << 16, ph[4] | ph[5] << 16,
+                                    ph[6] | ph[7] << 16);
+                        st_shared16(prow + 3 * kBlk + o, pl[0] | pl[1] << 16, pl[2] | pl[3] << 16,
+                                    pl[4] | pl[5] << 16, pl[6] | pl[7] << 16);
+                    }
+                }
+            }
+            tc::fence_async_smem();
+            tc::fence_before();
+            mbar_arrive(&bar_pfull);
+        }
+        // ------------------------------------------------------- epilogue
+        // Each row's A and Y, plus their group minima, go to shared memory
+        // (the K and V tiles are free once the last values completed); then a
+        // warp per row applies R^T to Y with the in-warp transform and writes
+        // the partial, 4 consecutive elements per lane.
+        constexpr int kEStride = kHeadDim + 4;   // padded rows: the row-per-thread stores do not conflict
+        float *sA = reinterpret_cast<float *>(sm + OFF_KA);
+        float *sY = reinterpret_cast<float *>(sm + OFF_VA);
+        if (ntl > 0) {
+            wait(&bar_odone, (ntl - 1) & 1, 24);
+            tc::fence_after();
+#pragma unroll
+            for (int side = 0; side < (RESID ? 2 : 1); side++) {
+                const uint32_t col = side == 0 ? kColOA : kColOY;
+                float *dst = (side == 0 ? sA : sY) + r * kEStride;
+                uint32_t m8[8];
+                tc::ld8(tl + col + kHeadDim, m8);
+                tc::wait_ld8(m8);
+#pragma unroll
+                for (int c = 0; c < kHeadDim; c += 16) {
+                    uint32_t v[16];
+                    tc::ld16(tl + col + c, v);
+                    tc::wait_ld(v);
+                    const float mn = __uint_as_float(m8[c / GS]);   // a 16-column chunk lies in one group
+                    if (own) {
+#pragma unroll
+                        for (int k = 0; k < 16; k += 4)
+                            *reinterpret_cast<float4 *>(dst + c + k) =
+                                make_float4(__uint_as_float(v[k]) + mn, __uint_as_float(v[k + 1]) + mn,
+                                            __uint_as_float(v[k + 2]) + mn, __uint_as_float(v[k + 3]) + mn);
+                    }
                 }
             }
         }
-        // online softmax per row (log2 domain); masked tokens weigh 0
-        const int tabs = t0 + tt + lane;
-#pragma unroll
-        for (int j = 0; j < RPW; j++) {
-            if (j < jn) {
-                const bool valid = lane < tn && tabs < lim[j];
-                const float z = valid ? s[j] : -CUDART_INF_F;
-                float mx = z;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                const float mn = fmaxf(m[j], mx);
-                float p = 0.f, alpha = 1.f;
-                if (mn != -CUDART_INF_F) {
-                    alpha = exp2f(m[j] - mn);   // 0 while nothing was seen
-                    p = valid ? exp2f(z - mn) : 0.f;
-                }
-                float ps = p;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-                l[j] = fmaf(l[j], alpha, ps);
-                m[j] = mn;
-#pragma unroll
-                for (int k = 0; k < 4; k++) acc[j][k] *= alpha;
-                sP[(warp + 8 * j) * kPStride + lane] = p;
-            }
+        if (own) {
+            s_ml[r][0] = m_used;
+            s_ml[r][1] = l;
         }
-        __syncthreads();   // every logit has read sK; sP is complete
-        dequant_tile<BA, BR>(a, st, 1, MR, resid, tn, sK, warp, lane);
-        __syncthreads();
-        for (int t = 0; t < tn; t++) {
-            const float *vr = sK + t * kKStride;
-            const float v0 = vr[lane], v1 = vr[lane + 32], v2 = vr[lane + 64], v3 = vr[lane + 96];
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        for (int rr = 0; rr < 16; rr++) {
+            const int row = 16 * warp + rr;
+            if (row >= nr) break;
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ntl > 0) {
+                if (RESID) {
+                    // R^T Y = diag(sigma) H Y / sqrt(d)
+                    const float4 y = *reinterpret_cast<const float4 *>(sY + row * kEStride + 4 * lane);
+                    o[0] = y.x;
+                    o[1] = y.y;
+                    o[2] = y.z;
+                    o[3] = y.w;
+                    if (a.rotate) {
+                        wht128_warp<float>(o, lane);
 #pragma unroll
-            for (int j = 0; j < RPW; j++) {
-                if (j < jn) {
-                    const float p = sP[(warp + 8 * j) * kPStride + t];
-                    acc[j][0] = fmaf(p, v0, acc[j][0]);
-                    acc[j][1] = fmaf(p, v1, acc[j][1]);
-                    acc[j][2] = fmaf(p, v2, acc[j][2]);
-                    acc[j][3] = fmaf(p, v3, acc[j][3]);
+                        for (int k = 0; k < 4; k++) o[k] *= sigma_neg(a.sigma, 4 * lane + k) ? -kInvSqrtD : kInvSqrtD;
+                    }
                 }
+                const float4 x = *reinterpret_cast<const float4 *>(sA + row * kEStride + 4 * lane);
+                o[0] += x.x;
+                o[1] += x.y;
+                o[2] += x.z;
+                o[3] += x.w;
             }
-        }
-        __syncthreads();   // sK, sP and this stage are rewritten by the next steps
-    }
-    cp_async_wait<0>();
-
-#pragma unroll
-    for (int j = 0; j < RPW; j++) {
-        if (j < jn) {
-            const int rg = r0 + warp + 8 * j, i = rg / a.G, gq = rg % a.G;
-            const size_t row = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
-            float *part = a.partials + (row * a.S + split) * kPartialStride;
-#pragma unroll
-            for (int k = 0; k < 4; k++) part[lane + 32 * k] = acc[j][k];
+            const int rg = r0 + row, i = rg / a.G, gq = rg % a.G;
+            const size_t prow = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
+            float *part = a.partials + (prow * a.S + split) * kPartialStride;
+            *reinterpret_cast<float4 *>(part + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
             if (lane == 0) {
-                part[kHeadDim] = m[j];
-                part[kHeadDim + 1] = l[j];
+                part[kHeadDim] = ntl > 0 ? s_ml[row][0] : -CUDART_INF_F;
+                part[kHeadDim + 1] = ntl > 0 ? s_ml[row][1] : 0.f;
             }
         }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            constexpr uint32_t idL = tc::idesc_bf16(kRows, kTok, false);
+            constexpr uint32_t idP = tc::idesc_bf16(kRows, kOCols, true);
+            auto kdesc = [&](int off, int kk) { return tc::desc_k(sbase + off + (kk >> 2) * kBlk + (kk & 3) * 32); };
+            auto logits = [&]() {
+#pragma unroll
+                for (int kk = 0; kk < 9; kk++)
+                    tc::mma_bf16(tmem + kColSA, kdesc(OFF_Q, kk), kdesc(OFF_KA, kk), idL, kk > 0);
+                if (RESID) {
+#pragma unroll
+                    for (int kk = 0; kk < 9; kk++)
+                        tc::mma_bf16(tmem + kColSY, kdesc(OFF_QRH, kk), kdesc(OFF_KY, kk), idL, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk++)
+                        tc::mma_bf16(tmem + kColSY, kdesc(OFF_QRL, kk), kdesc(OFF_KY, kk), idL, true);
+                }
+                tc::commit(&bar_kdone);
+            };
+            auto values = [&](int j) {
+#pragma unroll
+                for (int part = 0; part < 2; part++) {
+#pragma unroll
+                    for (int kk = 0; kk < kTok / 16; kk++)
+                        tc::mma_bf16(tmem + kColOA, tc::desc_k(sbase + OFF_PSH + part * kBlk + kk * 32),
+                                     tc::desc_mn(sbase + OFF_VA + kk * 2048, kBlk), idP, j > 0 || part > 0 || kk > 0);
+                    if (RESID) {
+#pragma unroll
+                        for (int kk = 0; kk < kTok / 16; kk++)
+                            tc::mma_bf16(tmem + kColOY, tc::desc_k(sbase + OFF_PSH + (2 + part) * kBlk + kk * 32),
+                                         tc::desc_mn(sbase + OFF_VY + kk * 2048, kBlk), idP,
+                                         j > 0 || part > 0 || kk > 0);
+                    }
+                }
+                tc::commit(&bar_odone);
+            };
+            for (int j = 0; j < ntl; j++) {
+                wait(&bar_kfull, j & 1, 25);
+                if (j > 0) wait(&bar_sfree, (j - 1) & 1, 26);
+                tc::fence_after();
+                logits();
+                if (j > 0) {
+                    wait(&bar_pfull, (j - 1) & 1, 27);
+                    wait(&bar_vfull, (j - 1) & 1, 28);
+                    tc::fence_after();
+                    values(j - 1);
+                }
+            }
+            if (ntl > 0) {
+                wait(&bar_pfull, (ntl - 1) & 1, 27);
+                wait(&bar_vfull, (ntl - 1) & 1, 28);
+                tc::fence_after();
+                values(ntl - 1);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------- dequantize
+        const int dt = tid - 32 * (kSoftmaxWarps + 1);
+        const int part = dt >> 6;   // 0, 1: anchor halves; 2, 3: residual halves
+        const int t = dt & (kTok - 1);
+        for (int j = 0; j < ntl; j++) {
+            const int tt = j * kTok;
+            const bool ok = t < min(kTok, cnt - tt);
+            const size_t rec = bh * a.Tp + t0 + tt + t;
+#pragma unroll
+            for (int kv = 0; kv < 2; kv++) {
+                if (j > 0) wait(kv == 0 ? &bar_kdone : &bar_odone, (j - 1) & 1, 29);
+                uint8_t *ta = sm + (kv == 0 ? OFF_KA : OFF_VA);
+                uint8_t *ty = sm + (kv == 0 ? OFF_KY : OFF_VY);
+                const uint8_t *ac = ok ? a.a_codes[kv] + rec * (16 * BA) : nullptr;
+                const uint8_t *am = ok ? a.a_meta[kv] + rec * MR : nullptr;
+                if (part == 0) deq_half<BA, GS, 0>(ta, t, ac, am, ok);
+                else if (part == 1) deq_half<BA, GS, 1>(ta, t, ac, am, ok);
+                else if (RESID) {
+                    const uint8_t *rc = ok ? a.r_codes[kv] + rec * (16 * BR) : nullptr;
+                    const uint8_t *rm = ok ? a.r_meta[kv] + rec * MR : nullptr;
+                    if (part == 2) deq_half<BR, GS, 0>(ty, t, rc, rm, ok);
+                    else deq_half<BR, GS, 1>(ty, t, rc, rm, ok);
+                }
+                if (kv == 0 && part == 0) {
+                    // slot j & 1 was last read at step j - 2, before the softmax
+                    // released step j - 1's logits, which this step's K waited for
+                    s_cK[j & 1][t] = RESID && ok ? bf16_to_f32(a.r_coef[0][rec]) : 1.f;
+                    s_cV[j & 1][t] = RESID && ok ? bf16_to_f32(a.r_coef[1][rec]) : 1.f;
+                    mbar_arrive(&bar_cfull[j & 1]);
+                }
+                tc::fence_async_smem();
+                mbar_arrive(kv == 0 ? &bar_kfull : &bar_vfull);
+            }
+        }
+    }
+
+    tc::fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc::fence_after();
+        tc::dealloc(tmem, kTmemCols);
     }
 }
 
@@ -306,65 +623,50 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
                 (size_t)a.H * kHeadDim, nt, a.out + row * kHeadDim, threadIdx.x, s_red, Sync128());
 }
 
-template <int BA, int BR, int RPW>
+template <int BA, int BR, int GS, bool RESID>
 struct Variant {
     static cudaError_t configure() {
-        static bool done = false;
-        if (done) return cudaSuccess;
-        cudaError_t e = cudaFuncSetAttribute(prefill_rq_kernel<BA, BR, RPW>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)Stage<BA, BR>::smem(8 * RPW));
-        if (e == cudaSuccess) done = true;
-        return e;
-    }
-    static int occupancy() {
-        static int occ = 0;
-        if (occ == 0 && configure() == cudaSuccess &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prefill_rq_kernel<BA, BR, RPW>, kThreadsP,
-                                                          Stage<BA, BR>::smem(8 * RPW)) != cudaSuccess)
-            occ = 0;
-        return occ > 0 ? occ : 1;
+        static bool done[kMaxDevices];
+        return once_per_device(done, [] {
+            return cudaFuncSetAttribute(prefill_tc_kernel<BA, BR, GS, RESID>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        });
     }
     static cudaError_t launch(const PrefillArgs &a, cudaStream_t st) {
         cudaError_t e = configure();
         if (e != cudaSuccess) return e;
         if (a.S > 0)
-            prefill_rq_kernel<BA, BR, RPW>
-                <<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, Stage<BA, BR>::smem(8 * RPW), st>>>(a);
+            prefill_tc_kernel<BA, BR, GS, RESID><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, kSmemBytes, st>>>(a);
         return cudaGetLastError();
     }
 };
 
-// f(Variant) for the (bits, rows per warp) of a
-template <typename F>
-auto with_variant(int ba, int br, int rpw, F f) -> decltype(f(Variant<4, 2, 1>())) {
-#define RQ_PREFILL_RPW(BA, BR)                      \
-    switch (rpw) {                                  \
-        case 1: return f(Variant<BA, BR, 1>());     \
-        case 2: return f(Variant<BA, BR, 2>());     \
-        case 4: return f(Variant<BA, BR, 4>());     \
-        default: return f(Variant<BA, BR, 8>());    \
-    }
-    if (ba == 2 && br == 2) RQ_PREFILL_RPW(2, 2)
-    if (ba == 4 && br == 4) RQ_PREFILL_RPW(4, 4)
-    RQ_PREFILL_RPW(4, 2)
-#undef RQ_PREFILL_RPW
+template <int BA, int BR, int GS>
+cudaError_t launch_bits(const PrefillArgs &a, cudaStream_t st) {
+    return a.r_codes[0] ? Variant<BA, BR, GS, true>::launch(a, st) : Variant<BA, BR, GS, false>::launch(a, st);
+}
+
+template <int GS>
+cudaError_t launch_group(const PrefillArgs &a, int ba, int br, cudaStream_t st) {
+    if (ba == 2 && br == 2) return launch_bits<2, 2, GS>(a, st);
+    if (ba == 4 && br == 4) return launch_bits<4, 4, GS>(a, st);
+    return launch_bits<4, 2, GS>(a, st);
 }
 
 }  // namespace
 
-// Rows per warp: the fewest that hold every query row of a kv head (at most
-// 8, 64 rows per CTA).  Splits: the count with the least wave-quantised work
-// (waves x 64-token tiles of the largest split, plus one tile of fixed cost),
-// waves counted from the variant's measured occupancy.
+// Row blocks of 64 query rows per kv head; splits: the count with the least
+// wave-quantised work (waves x 64-token steps of the largest split, plus one
+// step of fixed cost), one CTA per SM (the tiles take 193 KB of shared memory
+// and the accumulators all 512 tensor-memory columns).
 void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
+    (void)ba;
+    (void)br;
     const int nq = a->n * a->G;
-    a->rpw = nq <= 8 ? 1 : nq <= 16 ? 2 : nq <= 32 ? 4 : 8;
-    a->nqb = (nq + 8 * a->rpw - 1) / (8 * a->rpw);
+    a->nqb = (nq + kRows - 1) / kRows;
     a->S = 0;
     if (T <= 0) return;
-    const int occ = with_variant(ba, br, a->rpw, [](auto v) { return decltype(v)::occupancy(); });
-    const long slots = (long)std::max(1, occ) * std::max(1, sms);
+    const long slots = (long)std::max(1, sms);
     const long units = (long)a->B * a->H * a->nqb;
     const int nt = (T + kTokTile - 1) / kTokTile;
     long best = -1;
@@ -380,7 +682,8 @@ void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
 
 cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st) {
     if (!((ba == 4 && br == 2) || (ba == 2 && br == 2) || (ba == 4 && br == 4))) return cudaErrorInvalidValue;
-    cudaError_t e = with_variant(ba, br, a.rpw, [&](auto v) { return decltype(v)::launch(a, st); });
+    if (a.g != 16 && a.g != 32) return cudaErrorInvalidValue;
+    cudaError_t e = a.g == 16 ? launch_group<16>(a, ba, br, st) : launch_group<32>(a, ba, br, st);
     if (e != cudaSuccess) return e;
     prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
     return cudaGetLastError();

@@ -6,7 +6,7 @@
 
 namespace rq {
 
-constexpr int kPrefillTile = 32;   // committed tokens per step of a CTA
+constexpr int kPrefillTile = 64;   // committed tokens per step of a CTA (one split granule)
 
 // Causal attention of the n most recent tokens of every sequence: query row
 // (i, hq) of sequence b (i < n) sees the first T_b + n_tail - n + 1 + i tokens
@@ -22,14 +22,15 @@ struct PrefillArgs {
     float *out;                        // [B][n][Hq][d] fp32
     SeqLens seqT;                      // committed tokens of each sequence
     int B, H, Hq, G, n, n_tail, tail_cap, Tp, S;
-    int rpw, nqb;                      // query rows per warp (8 per CTA), row blocks per kv head
+    int nqb;                           // blocks of 64 query rows per kv head
     int g;                             // quantization group size
     float scale_log2;                  // softmax_scale * log2(e)
     int rotate;
     uint32_t sigma[4];
+    int *err;                          // device error word (bounded waits that gave up)
 };
 
-// Sets a->rpw, a->nqb and the split count a->S over the committed tokens (T
+// Sets a->nqb and the split count a->S over the committed tokens (T
 // = the longest sequence); a->B, H, G and n must be set.
 void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms);
 cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st);

@@ -312,8 +312,9 @@ def oracle_decode(bt: Built, layer: int, loop: int, q_bf16: torch.Tensor, bh_sel
             u = synth.bf16_to_u16(X[j][:, :T]).transpose(0, 2, 1, 3)
             vals = orc.bf16_bits_to_f64(np.stack([u[b, h] for (b, h) in sel]))     # [nsel][T][d]
         else:
-            rec = reconstruct_gpu(bt, layer, grp, kv, sel)[j].reshape(len(sel), T, D)
-            vals = rec
+            # exported records span the group's longest sequence; keep the first T tokens
+            rec = reconstruct_gpu(bt, layer, grp, kv, sel)[j].reshape(len(sel), -1, D)
+            vals = rec[:, :T]
         if n_tail:
             tu = synth.bf16_to_u16(X[j][:, T:T + n_tail]).transpose(0, 2, 1, 3)
             tv = orc.bf16_bits_to_f64(np.stack([tu[b, h] for (b, h) in sel]))

@@ -6,7 +6,8 @@ Through the C ABI, against the fp64 oracle and against contiguous caches:
   * a paged cache with a shuffled free list (every sequence's blocks
     scattered over the pool) holds records bit-identical to the oracle's and
     to a contiguous cache fed the same inputs, and decodes to the same
-    outputs, bit for bit, with ragged per-sequence lengths;
+    outputs up to the summation order (a paged cache's splits start on
+    block boundaries), with ragged per-sequence lengths;
   * forking a sequence shares its blocks; the first append into a shared
     block copies it (copy-on-write), leaving the other sequence's records
     untouched;
@@ -63,14 +64,18 @@ def test_paged_equals_contiguous_and_oracle(bt_tokens):
         for x, y in zip(a, b):
             assert (x is None and y is None) or np.array_equal(x, y)
         q = synth.queries(paged.seed, 0, loop, 0, 3, 4)
-        assert torch.equal(out_p[loop], flat.cache.decode(0, loop, q))
+        # same records; the splits differ (block-aligned), hence the order of
+        # the fixed-point sums: agreement to the kernel's own rounding
+        o_f = flat.cache.decode(0, loop, q)
+        d = (out_p[loop] - o_f).double()
+        assert float(d.norm() / o_f.double().norm()) <= 1e-4 and float(d.abs().max()) <= 4e-4, loop
     paged.cache.close()
     flat.cache.close()
 
 
 def test_paged_ragged_and_truncation_returns_blocks():
     bt = H.build(layers=1, loops=4, Lg=4, B=3, T=600, H=2, Hq=2, n_tail=0, chunk=128, seed=0x5EEDC100,
-                 block_tokens=128, num_blocks=20, prepare=_shuffled(6))
+                 max_tokens=640, block_tokens=128, num_blocks=20, prepare=_shuffled(6))
     c = bt.cache
     free0 = c.free_blocks()
     assert free0 == 20 - 3 * 5
