@@ -278,20 +278,19 @@ bool on_cache_device(const rq_cache *c) {
 #ifndef RQ_SPLIT_OVERHEAD_TILES
 #define RQ_SPLIT_OVERHEAD_TILES 2
 #endif
-void choose_splits(const rq_cache *c, int T, int units, int which, int gran, int *S, int *chunk) {
+void choose_splits(const rq_cache *c, int T, int units, int which, int *S, int *chunk) {
     if (T <= 0) {
         *S = 0;
         *chunk = kTokTile;
         return;
     }
-    const int nt = (T + kTokTile - 1) / kTokTile;
-    const int nu = (nt + gran - 1) / gran;   // granules (kMaxChunk is a whole number of them)
     const int s_lo = (T + kMaxChunk - 1) / kMaxChunk;
-    const int s_hi = std::min(c->lay.splits_max, nu);
+    const int s_hi = std::min(c->lay.splits_max, (T + kTokTile - 1) / kTokTile);
     long best_cost = -1;
     int best_s = s_lo, best_ch = kMaxChunk;
+    const int nt = (T + kTokTile - 1) / kTokTile;
     for (int s = s_lo; s <= std::max(s_lo, s_hi); s++) {
-        const int ch = (nu + s - 1) / s * gran * kTokTile;
+        const int ch = (nt + s - 1) / s * kTokTile;
         const int ss = s;
         const int slots = std::max(1, c->occ[which][ch / kTokTile - 1] * c->sms);
         const long waves = ((long)ss * units + slots - 1) / slots;
@@ -305,7 +304,7 @@ void choose_splits(const rq_cache *c, int T, int units, int which, int gran, int
 #ifdef RQ_SPLIT_FORCE_S
     if (RQ_SPLIT_FORCE_S >= s_lo && RQ_SPLIT_FORCE_S <= std::max(s_lo, s_hi)) {
         best_s = RQ_SPLIT_FORCE_S;
-        best_ch = (nu + best_s - 1) / best_s * gran * kTokTile;
+        best_ch = (nt + best_s - 1) / best_s * kTokTile;
     }
 #endif
     *S = best_s;
@@ -697,7 +696,7 @@ static int decode_common(rq_cache *c, int layer, int loop, const void *q, float 
         }
     }
     const int units = a.B * a.H * (a.G > 2 ? a.G / 2 : 1);
-    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, split_granule(a.pg), &a.S, &a.chunk);
+    choose_splits(c, a.T, units, bf16 ? 0 : a.nr, &a.S, &a.chunk);
     if (partials) {
         a.splits_max = std::max(a.S, 1);
         if ((size_t)a.B * a.Hq * a.splits_max * kPartialStride > partial_floats) return RQ_ERR_CAPACITY;

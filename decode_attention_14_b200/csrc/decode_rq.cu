@@ -371,8 +371,13 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     const int b = blockIdx.z / npairs, pair = blockIdx.z % npairs;
     const int hq0 = h * a.G + pair * GK;
     int t0, n;   // this split's tokens of its sequence (none when the sequence is short)
-    split_range(split, a.S, a.seqT.v[b], &t0, &n, split_granule(a.pg));
+    split_range(split, a.S, a.seqT.v[b], &t0, &n);
     const int ntiles = (n + kTile - 1) / kTile;
+    // paged: ring items start on item-size boundaries of the sequence (a
+    // split may begin inside one), so that no item straddles two blocks; the
+    // item grid then begins sh tiles before the split, which stay empty
+    const int sh = (a.pg.table != nullptr && ntiles > 0) ? (t0 / kTile) % kItemTiles : 0;
+    const int ntv = ntiles + sh;   // tiles of the item grid
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
     const uint16_t *s_cf = reinterpret_cast<const uint16_t *>(smem + P::RING);   // V coefficients [NR][cstride]
@@ -458,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             // loop keeps all of this in running counters (no division).
             const int npass = 2 + NR;
             int it = 0, virt = 0, phys = 0;
-            const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // items per pass
+            const int nitems = (ntv + kItemTiles - 1) / kItemTiles;   // items per pass
             int rel = 0, vrel = 0, rphys = 0, ritem = 0, rpass = 0, rbytes = P::K_BYTES;   // oldest unreleased item
             bool ok = true;
             for (int pass = 0; pass < npass && ok; pass++) {
@@ -470,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                     }
                     if (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING))
                         dep(0x7FFFFFFF);   // about to block on the consumers, who run after their wait
-                    dep(min((j + 1) * kItem, n));
+                    dep(min((j + 1) * kItem - sh * kTile, n));
                     while (rel < it && (it - rel >= kSlots || vrel < virt + bytes - P::RING)) {
                         if (!mbar_wait<RQ_DECODE_PRODUCER_SLEEP_NS>(&bar_empty[rel % kSlots], (rel / kSlots) & 1,
                                                                     &s_abort)) {
@@ -494,9 +499,12 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         atomicExch(a.err, 1);
                         break;
                     }
-                    // the last item of a pass may hold fewer tiles: copy only those
-                    const int toks = min(kItem, (ntiles - j * kItemTiles) * kTile);
-                    const int tj = t0 + j * kItem;
+                    // the first and the last item of a pass may hold fewer tiles:
+                    // copy only those, to their places in the item
+                    const int v0 = max(j * kItemTiles, sh), v1 = min((j + 1) * kItemTiles, ntv);
+                    const int toks = (v1 - v0) * kTile;
+                    const int tj = t0 + (v0 - sh) * kTile;
+                    const int skip = (v0 - j * kItemTiles) * kTile;   // empty token slots before them
                     uint8_t *st = ring + phys;
                     uint64_t *bar = &bar_full[it % kSlots];
 #ifdef RQ_FAULT_INJECT
@@ -509,22 +517,22 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #endif
                     if (pass == 0) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2))));
-                        copy_run(st, a.a_codes[0], P::A_C, tj, toks, bar);
-                        copy_run(st + P::K_AM, a.a_meta[0], P::MR, tj, toks, bar);
+                        copy_run(st + skip * P::A_C, a.a_codes[0], P::A_C, tj, toks, bar);
+                        copy_run(st + P::K_AM + skip * P::MR, a.a_meta[0], P::MR, tj, toks, bar);
 #pragma unroll
                         for (int k = 0; k < NR; k++) {
-                            copy_run(st + P::K_RC(k), a.r_codes[k][0], P::R_C, tj, toks, bar);
-                            copy_run(st + P::K_RM(k), a.r_meta[k][0], P::MR, tj, toks, bar);
-                            copy_run(st + P::K_CF(k), a.r_coef[k][0], 2, tj, toks, bar);
+                            copy_run(st + P::K_RC(k) + skip * P::R_C, a.r_codes[k][0], P::R_C, tj, toks, bar);
+                            copy_run(st + P::K_RM(k) + skip * P::MR, a.r_meta[k][0], P::MR, tj, toks, bar);
+                            copy_run(st + P::K_CF(k) + skip * 2, a.r_coef[k][0], 2, tj, toks, bar);
                         }
                     } else if (pass == 1) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR)));
-                        copy_run(st, a.a_codes[1], P::A_C, tj, toks, bar);
-                        copy_run(st + P::VA_M, a.a_meta[1], P::MR, tj, toks, bar);
+                        copy_run(st + skip * P::A_C, a.a_codes[1], P::A_C, tj, toks, bar);
+                        copy_run(st + P::VA_M + skip * P::MR, a.a_meta[1], P::MR, tj, toks, bar);
                     } else {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::R_C + P::MR)));
-                        copy_run(st, a.r_codes[pass - 2][1], P::R_C, tj, toks, bar);
-                        copy_run(st + P::VR_M, a.r_meta[pass - 2][1], P::MR, tj, toks, bar);
+                        copy_run(st + skip * P::R_C, a.r_codes[pass - 2][1], P::R_C, tj, toks, bar);
+                        copy_run(st + P::VR_M + skip * P::MR, a.r_meta[pass - 2][1], P::MR, tj, toks, bar);
                     }
                     virt += bytes;
                     phys += bytes;
@@ -666,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     for (int gq = 0; gq < GK; gq++) mloc[gq] = -CUDART_INF_F;
     const bool b4 = (seg & 4) != 0, b2 = (seg & 2) != 0;
     const int kown = (b4 ? 2 : 0) + (b2 ? 1 : 0);   // token (of 4) this lane ends up owning
-    const int nitems = (ntiles + kItemTiles - 1) / kItemTiles;   // ring items per pass
+    const int nitems = (ntv + kItemTiles - 1) / kItemTiles;   // ring items per pass
     int c_off = 0;   // ring offset of the current item (the producer's placement rule)
     for (int j = 0; j < nitems; j++) {
         const int slot = j % kSlots;
@@ -679,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         float part[kItemTiles][GK][4];
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
-            if (j * kItemTiles + u >= ntiles) break;   // uniform: a short last item
+            if (j * kItemTiles + u >= ntv) break;   // uniform: a short last item
+            if (j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
@@ -709,8 +718,9 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         // reduce the 4 tokens' partials over the 8 segment lanes: lanes 2k, 2k+1 end with token k
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
-            const int i = j * kItemTiles + u;
-            if (i >= ntiles) break;
+            if (j * kItemTiles + u >= ntv) break;
+            if (j * kItemTiles + u < sh) continue;
+            const int i = j * kItemTiles + u - sh;   // tile of the chunk
             const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
             for (int gq = 0; gq < GK; gq++) {
@@ -817,10 +827,11 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 atomicExch(a.err, 4);
             }
             const uint8_t *st = ring + c_off;
-            const int last_u = min(kItemTiles, ntiles - j * kItemTiles) - 1;   // a short last item
+            const int last_u = min(kItemTiles, ntv - j * kItemTiles) - 1;   // a short last item
 #pragma unroll
             for (int u = 0; u < kItemTiles; u++) {
                 if (u > last_u) break;   // uniform
+                if (j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
                 uint32_t wlo[GK][2], whi[GK][2];
                 float2 mm[4];
                 float W[GK][4];
@@ -837,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         mm[k] = meta_pair(*reinterpret_cast<const uint16_t *>(st + P::VR_M + tok * P::MR + 2 * mg));
                     }
 #pragma unroll
-                    for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + j * kItem + tok];
+                    for (int gq = 0; gq < GK; gq++) W[gq][k] = wsrc[gq * a.chunk + j * kItem + tok - sh * kTile];
                 }
                 if (u == last_u) {   // every read of the item is done: release it
                     mbar_arrive(&bar_empty[slot]);

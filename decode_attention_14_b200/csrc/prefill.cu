@@ -79,8 +79,9 @@ constexpr int OFF_KA = 8 * kBlk;      // anchor K: sc code | mn, mn
 constexpr int OFF_KY = 11 * kBlk;     // residual K
 constexpr int OFF_VA = 14 * kBlk;     // anchor V (read MN-major)
 constexpr int OFF_VY = 17 * kBlk;     // residual V
-constexpr int OFF_PSH = 20 * kBlk;    // (p s) hi, then lo, p hi, p lo: one block each
-constexpr int kTilesBytes = 24 * kBlk;
+constexpr int OFF_P = 20 * kBlk;      // two buffers of [(p s) hi, (p s) lo, p hi, p lo], a block each
+constexpr int kPBytes = 4 * kBlk;
+constexpr int kTilesBytes = 28 * kBlk;
 constexpr int kSmemBytes = kTilesBytes + 1024;   // + alignment of the base to 1024
 // tensor-memory columns (fp32): logits of a step, then the value accumulators
 constexpr uint32_t kColSA = 0, kColSY = 64, kColOA = 128, kColOY = 272, kTmemCols = 512;
@@ -94,6 +95,17 @@ __device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_floa
 __device__ __forceinline__ void split_hi_lo(float x, uint32_t &hi, uint32_t &lo) {
     hi = bf16_bits(x);
     lo = bf16_bits(x - bf16_val(hi));
+}
+// (x0, x1) to BF16 pairs, element 0 in the low half: one rounding each
+__device__ __forceinline__ uint32_t bf16x2_rn(float x0, float x1) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x1), "f"(x0));
+    return d;
+}
+// high and low BF16 parts of (x0, x1) as two BF16 pairs
+__device__ __forceinline__ void split_hi_lo2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = bf16x2_rn(x0, x1);
+    lo = bf16x2_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
 }
 __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
@@ -120,14 +132,51 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w, int p) {
     return 0x43004300u | (t & 0x3u) | ((t & 0xCu) << 14);
 }
 
-// Dequantize half HALF (head_dim elements 64 HALF .. 64 HALF + 63) of one
-// record into row t of a 3-block operand tile: sc * code per element, exact
-// in BF16 ((128 + code) sc - 128 sc in one rounding); HALF 0 also writes the
-// minimum columns (mn_0 .. mn_{NG-1}, zeros, twice).  A token past the step
-// (ok false) gets a zero row.
+// Raw bytes of half a record (head_dim elements 64 h .. 64 h + 63): its
+// codes (8 BITS bytes) and the (scale, minimum) FP8 pairs of every group.
+struct RawHalf {
+    uint32_t w[8];
+    uint32_t mw[4];
+};
+
+// Loads half `h` of a record (nothing, zeros, for a token past the step).
+template <int BITS, int GS>
+__device__ __forceinline__ void load_half(const uint8_t *codes, const uint8_t *meta, int h, bool ok, RawHalf &r) {
+    constexpr int MR = 2 * (kHeadDim / GS);
+#pragma unroll
+    for (int i = 0; i < 8; i++) r.w[i] = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; i++) r.mw[i] = 0u;
+    if (!ok) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(codes + 8 * BITS * h);
+#pragma unroll
+    for (int u = 0; u < BITS / 2; u++) {
+        const uint4 v = __ldg(src + u);
+        r.w[4 * u] = v.x;
+        r.w[4 * u + 1] = v.y;
+        r.w[4 * u + 2] = v.z;
+        r.w[4 * u + 3] = v.w;
+    }
+    if (MR == 16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(meta));
+        r.mw[0] = v.x;
+        r.mw[1] = v.y;
+        r.mw[2] = v.z;
+        r.mw[3] = v.w;
+    } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(meta));
+        r.mw[0] = v.x;
+        r.mw[1] = v.y;
+    }
+}
+
+// Writes half HALF of a loaded record into row t of a 3-block operand tile:
+// sc * code per element, exact in BF16 ((128 + code) sc - 128 sc in one
+// rounding); HALF 0 also writes the minimum columns (mn_0 .. mn_{NG-1},
+// zeros, twice).  A token past the step (ok false) gets a zero row.
 template <int BITS, int GS, int HALF>
-__device__ __forceinline__ void deq_half(uint8_t *tile, int t, const uint8_t *codes, const uint8_t *meta, bool ok) {
-    constexpr int NG = kHeadDim / GS, MR = 2 * NG;
+__device__ __forceinline__ void store_half(uint8_t *tile, int t, const RawHalf &r, bool ok) {
+    constexpr int NG = kHeadDim / GS;
     uint8_t *row = tile + HALF * kBlk;
     uint8_t *mrow = tile + 2 * kBlk;
     if (!ok) {
@@ -139,48 +188,33 @@ __device__ __forceinline__ void deq_half(uint8_t *tile, int t, const uint8_t *co
         }
         return;
     }
-    // 64 codes: 8 BITS bytes
-    uint32_t w[2 * BITS];
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(codes + 8 * BITS * HALF);
-#pragma unroll
-        for (int u = 0; u < BITS / 2; u++) {
-            const uint4 v = __ldg(src + u);
-            w[4 * u] = v.x;
-            w[4 * u + 1] = v.y;
-            w[4 * u + 2] = v.z;
-            w[4 * u + 3] = v.w;
-        }
-    }
-    // (scale, minimum) FP8 byte pairs of all groups
-    uint32_t mw[MR / 4];
-    if (MR == 16) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(meta));
-        mw[0] = v.x;
-        mw[1 % (MR / 4)] = v.y;
-        mw[2 % (MR / 4)] = v.z;
-        mw[3 % (MR / 4)] = v.w;
-    } else {
-        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(meta));
-        mw[0] = v.x;
-        mw[1] = v.y;
-    }
     constexpr int GPH = 64 / GS;   // groups of this half
 #pragma unroll
     for (int gl = 0; gl < GPH; gl++) {
         constexpr int CPG = GS / 8;   // 16-byte chunks per group
         const int gi = HALF * GPH + gl;
-        const uint32_t pr = (mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+        const uint32_t pr = (r.mw[gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
         const float sc = e4m3_to_f32(pr & 0xFFu);
         const uint32_t s2 = bf16_bits(sc) * 0x10001u;
         const uint32_t nb2 = bf16_bits(-128.f * sc) * 0x10001u;
 #pragma unroll
         for (int cg = 0; cg < CPG; cg++) {
             const int c = gl * CPG + cg;   // chunk of the half: elements 8c .. 8c + 7
-            const uint32_t cw = BITS == 4 ? w[c] : (w[c >> 1] >> (16 * (c & 1)));
-            st_shared16(row + tc::sw_chunk(t, c), fma_bf16x2(code_pair<BITS>(cw, 0), s2, nb2),
-                        fma_bf16x2(code_pair<BITS>(cw, 1), s2, nb2), fma_bf16x2(code_pair<BITS>(cw, 2), s2, nb2),
-                        fma_bf16x2(code_pair<BITS>(cw, 3), s2, nb2));
+            uint32_t q[4];
+            if (BITS == 4) {
+                // even elements in the bytes of lo, odd ones in the bytes of hi;
+                // byte k of each into the low byte of one half of pair k
+                const uint32_t lo = r.w[c] & 0x0F0F0F0Fu, hi = (r.w[c] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+                    q[k] = (__byte_perm(lo, hi, (uint32_t)(k | ((4 + k) << 8))) & 0x00FF00FFu) | 0x43004300u;
+            } else {
+                const uint32_t cw = r.w[c >> 1] >> (16 * (c & 1));
+#pragma unroll
+                for (int k = 0; k < 4; k++) q[k] = code_pair<BITS>(cw, k);
+            }
+            st_shared16(row + tc::sw_chunk(t, c), fma_bf16x2(q[0], s2, nb2), fma_bf16x2(q[1], s2, nb2),
+                        fma_bf16x2(q[2], s2, nb2), fma_bf16x2(q[3], s2, nb2));
         }
     }
     if (HALF == 0) {
@@ -188,8 +222,8 @@ __device__ __forceinline__ void deq_half(uint8_t *tile, int t, const uint8_t *co
 #pragma unroll
         for (int k = 0; k < 4; k++) {
             uint32_t lo = 0u, hi = 0u;
-            if (2 * k < NG) lo = bf16_bits(e4m3_to_f32((mw[k % (MR / 4)] >> 8) & 0xFFu));
-            if (2 * k + 1 < NG) hi = bf16_bits(e4m3_to_f32((mw[k % (MR / 4)] >> 24) & 0xFFu));
+            if (2 * k < NG) lo = bf16_bits(e4m3_to_f32((r.mw[k] >> 8) & 0xFFu));
+            if (2 * k + 1 < NG) hi = bf16_bits(e4m3_to_f32((r.mw[k] >> 24) & 0xFFu));
             m[k] = lo | (hi << 16);
         }
         st_shared16(mrow + tc::sw_chunk(t, 0), m[0], m[1], m[2], m[3]);
@@ -204,18 +238,29 @@ template <int GS, bool RESID>
 __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm, int b, int h, int r0, int nr,
                                               int warp, int lane) {
     constexpr int NG = kHeadDim / GS, LPG = GS / 4;   // lanes per group
-    for (int r = warp; r < kRows; r += kThreadsP / 32) {
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        uint2 raw = make_uint2(0u, 0u);
+    constexpr int kWarps = kThreadsP / 32, kRowsPerWarp = (kRows + kWarps - 1) / kWarps;
+    // all of this warp's rows are fetched first, so that their latencies overlap
+    uint2 raws[kRowsPerWarp];
+#pragma unroll
+    for (int u = 0; u < kRowsPerWarp; u++) {
+        const int r = warp + u * kWarps;
+        raws[u] = make_uint2(0u, 0u);
         if (r < nr) {
             const int rg = r0 + r, i = rg / a.G, gq = rg % a.G;
             const uint16_t *qrow = a.q + (((size_t)b * a.n + i) * a.Hq + h * a.G + gq) * kHeadDim;
-            raw = *reinterpret_cast<const uint2 *>(qrow + 4 * lane);
-            x[0] = bf16_val(raw.x & 0xFFFFu);
-            x[1] = bf16_val(raw.x >> 16);
-            x[2] = bf16_val(raw.y & 0xFFFFu);
-            x[3] = bf16_val(raw.y >> 16);
+            raws[u] = __ldg(reinterpret_cast<const uint2 *>(qrow + 4 * lane));
         }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowsPerWarp; u++) {
+        const int r = warp + u * kWarps;
+        if (r >= kRows) break;
+        const uint2 raw = raws[u];
+        float x[4];
+        x[0] = bf16_val(raw.x & 0xFFFFu);
+        x[1] = bf16_val(raw.x >> 16);
+        x[2] = bf16_val(raw.y & 0xFFFFu);
+        x[3] = bf16_val(raw.y >> 16);
         // elements 4 lane .. 4 lane + 3: block lane / 16, chunk (lane % 16) / 2, half (lane & 1)
         const uint32_t off = (uint32_t)(lane >> 4) * kBlk + tc::sw_chunk(r, (lane & 15) >> 1) + 8u * (lane & 1);
         st_shared8(sm + OFF_Q + off, raw.x, raw.y);
@@ -263,7 +308,7 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
 template <int BA, int BR, int GS, bool RESID>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar_kfull, bar_vfull, bar_kdone, bar_odone, bar_sfree, bar_pfull, bar_cfull[2];
+    __shared__ uint64_t bar_kfull, bar_vfull, bar_kdone, bar_sfree, bar_cfull[2], bar_pfull[2], bar_odone[2];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_cK[2][kTok], s_cV[2][kTok];   // coefficients of the step (1 at an anchor loop)
@@ -289,11 +334,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         mbar_init(&bar_kfull, kDeqThreads);
         mbar_init(&bar_vfull, kDeqThreads);
         mbar_init(&bar_kdone, 1);
-        mbar_init(&bar_odone, 1);
         mbar_init(&bar_sfree, 32 * kSoftmaxWarps);
-        mbar_init(&bar_pfull, 32 * kSoftmaxWarps);
-        mbar_init(&bar_cfull[0], kTok);
-        mbar_init(&bar_cfull[1], kTok);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&bar_cfull[i], kTok);
+            mbar_init(&bar_pfull[i], 32 * kSoftmaxWarps);
+            mbar_init(&bar_odone[i], 1);
+        }
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -314,28 +360,38 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             atomicExch(a.err, code);
         }
     };
+    // Phases.  kfull, vfull, kdone, sfree complete once per step; cfull[i],
+    // pfull[i] and odone[i] once per step of parity i (their k-th completion
+    // belongs to step 2k + i).  No barrier can run two phases ahead of a
+    // waiter (each next phase needs work the waiter has not released yet).
 
     if (warp < kSoftmaxWarps) {
         // ------------------------------------------------------- softmax
-        const bool own = lane < 16;                   // lanes 16..31 hold no row (M = 64 layout)
+        // Thread (w, i): row r = 16 w + (i mod 16) -- tensor-memory lane 32 w
+        // + (i mod 16) of the M = 64 layout -- and half hf = i / 16 of every
+        // range of columns it reads (the 16x32bx2 access: the upper 16
+        // threads read the same lanes at a column offset).
+        const int hf = lane >> 4;
         const int r = 16 * warp + (lane & 15);
         const int iq = (r0 + r) / a.G;
         const int lim = min(Tb, Tb + a.n_tail - a.n + 1 + iq);   // committed tokens the row may see
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-        float m_used = -CUDART_INF_F, l = 0.f;
+        constexpr int kHalf = kTok / 2;                          // tokens of a thread per step
+        float m_used = -CUDART_INF_F, l = 0.f;                   // l: this thread's half of the row's sum
         for (int j = 0; j < ntl; j++) {
             const int tt = j * kTok;
             const int tn = min(kTok, cnt - tt);
-            wait(&bar_cfull[j & 1], (j >> 1) & 1, 21);   // the step's coefficients
+            const int pb = j & 1;   // probability buffer of the step
+            wait(&bar_cfull[pb], (j >> 1) & 1, 21);   // the step's coefficients
             wait(&bar_kdone, j & 1, 22);
             tc::fence_after();
-            float s[kTok];
+            float s[kHalf];
 #pragma unroll
-            for (int c = 0; c < kTok; c += 16) {
+            for (int c = 0; c < kHalf; c += 16) {
                 uint32_t va[16], vy[16];
-                tc::ld16(tl + kColSA + c, va);
+                tc::ld16x2<kHalf>(tl + kColSA + c, va);
                 if (RESID) {
-                    tc::ld16(tl + kColSY + c, vy);
+                    tc::ld16x2<kHalf>(tl + kColSY + c, vy);
                     tc::wait_ld2(va, vy);
                 } else {
                     tc::wait_ld(va);
@@ -343,7 +399,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
 #pragma unroll
                 for (int k = 0; k < 16; k++) {
                     const float sa = __uint_as_float(va[k]);
-                    const float x = RESID ? fmaf(s_cK[j & 1][c + k], sa, __uint_as_float(vy[k])) : sa;
+                    const float x = RESID ? fmaf(s_cK[pb][kHalf * hf + c + k], sa, __uint_as_float(vy[k])) : sa;
                     s[c + k] = x * a.scale_log2;
                 }
             }
@@ -351,84 +407,89 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             mbar_arrive(&bar_sfree);
             float mx = -CUDART_INF_F;
 #pragma unroll
-            for (int t = 0; t < kTok; t++) {
-                const bool ok = own && t < tn && t0 + tt + t < lim;
-                s[t] = ok ? s[t] : -CUDART_INF_F;
-                mx = fmaxf(mx, s[t]);
+            for (int k = 0; k < kHalf; k++) {
+                const int t = kHalf * hf + k;
+                const bool ok = t < tn && t0 + tt + t < lim;
+                s[k] = ok ? s[k] : -CUDART_INF_F;
+                mx = fmaxf(mx, s[k]);
             }
-            // the previous step's values are complete: P is free, O is final
-            if (j > 0) wait(&bar_odone, (j - 1) & 1, 23);
-            tc::fence_after();
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));   // the row's maximum
             const bool raise = mx > m_used + kRescaleLog2;   // false while nothing is seen (both -inf)
             const bool rescale = raise && m_used != -CUDART_INF_F;
             const float f = rescale ? exp2f(m_used - mx) : 1.f;
             if (raise) m_used = mx;
+            // this step's probability buffer was last read by the values of step j - 2
+            if (j >= 2) wait(&bar_odone[pb], ((j >> 1) - 1) & 1, 23);
             if (__any_sync(0xffffffffu, rescale)) {
-                // this row's accumulated values times f (rows without a raise times 1)
+                // O must be final: the values of step j - 1 complete
+                if (j >= 1) wait(&bar_odone[pb ^ 1], ((j - 1) >> 1) & 1, 23);
+                tc::fence_after();
+                // this row's accumulated values times f (rows without a raise
+                // times 1); the two threads of a row take columns c and c + 64
 #pragma unroll 1
-                for (int c = 0; c < kHeadDim; c += 16) {
+                for (int c = 0; c < kHeadDim / 2; c += 16) {
                     uint32_t v[16];
-                    tc::ld16(tl + kColOA + c, v);
+                    tc::ld16x2<kHeadDim / 2>(tl + kColOA + c, v);
                     tc::wait_ld(v);
 #pragma unroll
                     for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
-                    tc::st16(tl + kColOA + c, v);
+                    tc::st16x2<kHeadDim / 2>(tl + kColOA + c, v);
                     if (RESID) {
-                        tc::ld16(tl + kColOY + c, v);
+                        tc::ld16x2<kHeadDim / 2>(tl + kColOY + c, v);
                         tc::wait_ld(v);
 #pragma unroll
                         for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
-                        tc::st16(tl + kColOY + c, v);
+                        tc::st16x2<kHeadDim / 2>(tl + kColOY + c, v);
                     }
                 }
+                // the minimum columns (the upper threads' 8 columns after them are unused)
                 uint32_t v8[8];
-                tc::ld8(tl + kColOA + kHeadDim, v8);
+                tc::ld8x2<8>(tl + kColOA + kHeadDim, v8);
                 tc::wait_ld8(v8);
 #pragma unroll
                 for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
-                tc::st8(tl + kColOA + kHeadDim, v8);
+                tc::st8x2<8>(tl + kColOA + kHeadDim, v8);
                 if (RESID) {
-                    tc::ld8(tl + kColOY + kHeadDim, v8);
+                    tc::ld8x2<8>(tl + kColOY + kHeadDim, v8);
                     tc::wait_ld8(v8);
 #pragma unroll
                     for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
-                    tc::st8(tl + kColOY + kHeadDim, v8);
+                    tc::st8x2<8>(tl + kColOY + kHeadDim, v8);
                 }
                 tc::wait_st();
             }
             l *= f;
             // probabilities of the step, split hi / lo, into the A operands
             const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
-            uint8_t *prow = sm + OFF_PSH;
+            uint8_t *prow = sm + OFF_P + pb * kPBytes;
 #pragma unroll
-            for (int cc = 0; cc < kTok / 8; cc++) {
-                uint32_t psh[8], psl[8], ph[8], pl[8];
+            for (int cc = 0; cc < kHalf / 8; cc++) {
+                uint32_t psh[4], psl[4], ph[4], pl[4];
 #pragma unroll
-                for (int k = 0; k < 8; k++) {
-                    const int t = 8 * cc + k;
-                    const float p = exp2f(s[t] - mu);   // 0 for a masked token
-                    l += p;
-                    split_hi_lo(RESID ? p * s_cV[j & 1][t] : p, psh[k], psl[k]);
-                    if (RESID) split_hi_lo(p, ph[k], pl[k]);
-                }
-                if (own) {
-                    const uint32_t o = tc::sw_chunk(r, cc);
-                    st_shared16(prow + o, psh[0] | psh[1] << 16, psh[2] | psh[3] << 16, psh[4] | psh[5] << 16,
-                                psh[6] | psh[7] << 16);
-                    st_shared16(prow + kBlk + o, psl[0] | psl[1] << 16, psl[2] | psl[3] << 16,
-                                psl[4] | psl[5] << 16, psl[6] | psl[7] << 16);
+                for (int k = 0; k < 8; k += 2) {
+                    const int t = kHalf * hf + 8 * cc + k;
+                    const float p0 = exp2f(s[8 * cc + k] - mu), p1 = exp2f(s[8 * cc + k + 1] - mu);   // 0 if masked
+                    l += p0 + p1;
                     if (RESID) {
-                        st_shared16(prow + 2 * kBlk + o, ph[0] | ph[1] << 16, ph[2] | ph[3] << 16, ph[4] | ph[5] << 16,
-                                    ph[6] | ph[7] << 16);
-                        st_shared16(prow + 3 * kBlk + o, pl[0] | pl[1] << 16, pl[2] | pl[3] << 16,
-                                    pl[4] | pl[5] << 16, pl[6] | pl[7] << 16);
+                        split_hi_lo2(p0 * s_cV[pb][t], p1 * s_cV[pb][t + 1], psh[k / 2], psl[k / 2]);
+                        split_hi_lo2(p0, p1, ph[k / 2], pl[k / 2]);
+                    } else {
+                        split_hi_lo2(p0, p1, psh[k / 2], psl[k / 2]);
                     }
+                }
+                const uint32_t o = tc::sw_chunk(r, (kHalf / 8) * hf + cc);
+                st_shared16(prow + o, psh[0], psh[1], psh[2], psh[3]);
+                st_shared16(prow + kBlk + o, psl[0], psl[1], psl[2], psl[3]);
+                if (RESID) {
+                    st_shared16(prow + 2 * kBlk + o, ph[0], ph[1], ph[2], ph[3]);
+                    st_shared16(prow + 3 * kBlk + o, pl[0], pl[1], pl[2], pl[3]);
                 }
             }
             tc::fence_async_smem();
             tc::fence_before();
-            mbar_arrive(&bar_pfull);
+            mbar_arrive(&bar_pfull[pb]);
         }
+        l += __shfl_xor_sync(0xffffffffu, l, 16);   // the row's sum
         // ------------------------------------------------------- epilogue
         // Each row's A and Y, plus their group minima, go to shared memory
         // (the K and V tiles are free once the last values completed); then a
@@ -438,32 +499,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         float *sA = reinterpret_cast<float *>(sm + OFF_KA);
         float *sY = reinterpret_cast<float *>(sm + OFF_VA);
         if (ntl > 0) {
-            wait(&bar_odone, (ntl - 1) & 1, 24);
+            // the last values complete (and with them every earlier MMA)
+            wait(&bar_odone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, 24);
             tc::fence_after();
 #pragma unroll
             for (int side = 0; side < (RESID ? 2 : 1); side++) {
                 const uint32_t col = side == 0 ? kColOA : kColOY;
-                float *dst = (side == 0 ? sA : sY) + r * kEStride;
+                float *dst = (side == 0 ? sA : sY) + r * kEStride + (kHeadDim / 2) * hf;
+                // the row's group minima (read by the lower thread of the pair)
                 uint32_t m8[8];
-                tc::ld8(tl + col + kHeadDim, m8);
+                tc::ld8x2<8>(tl + col + kHeadDim, m8);
                 tc::wait_ld8(m8);
 #pragma unroll
-                for (int c = 0; c < kHeadDim; c += 16) {
-                    uint32_t v[16];
-                    tc::ld16(tl + col + c, v);
-                    tc::wait_ld(v);
-                    const float mn = __uint_as_float(m8[c / GS]);   // a 16-column chunk lies in one group
-                    if (own) {
+                for (int k = 0; k < 8; k++) m8[k] = __shfl_sync(0xffffffffu, m8[k], lane & 15);
 #pragma unroll
-                        for (int k = 0; k < 16; k += 4)
-                            *reinterpret_cast<float4 *>(dst + c + k) =
-                                make_float4(__uint_as_float(v[k]) + mn, __uint_as_float(v[k + 1]) + mn,
-                                            __uint_as_float(v[k + 2]) + mn, __uint_as_float(v[k + 3]) + mn);
-                    }
+                for (int c = 0; c < kHeadDim / 2; c += 16) {
+                    uint32_t v[16];
+                    tc::ld16x2<kHeadDim / 2>(tl + col + c, v);
+                    tc::wait_ld(v);
+                    // a 16-column chunk lies in one group
+                    const float mn = __uint_as_float(hf ? m8[(kHeadDim / 2 + c) / GS] : m8[c / GS]);
+#pragma unroll
+                    for (int k = 0; k < 16; k += 4)
+                        *reinterpret_cast<float4 *>(dst + c + k) =
+                            make_float4(__uint_as_float(v[k]) + mn, __uint_as_float(v[k + 1]) + mn,
+                                        __uint_as_float(v[k + 2]) + mn, __uint_as_float(v[k + 3]) + mn);
                 }
             }
         }
-        if (own) {
+        if (hf == 0) {
             s_ml[r][0] = m_used;
             s_ml[r][1] = l;
         }
@@ -503,95 +567,137 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------- MMA issue
+        // One thread; the logits of step j + 1 and the values of step j are
+        // issued in whichever order their operands become ready.
         if (lane == 0) {
             constexpr uint32_t idL = tc::idesc_bf16(kRows, kTok, false);
             constexpr uint32_t idP = tc::idesc_bf16(kRows, kOCols, true);
-            auto kdesc = [&](int off, int kk) { return tc::desc_k(sbase + off + (kk >> 2) * kBlk + (kk & 3) * 32); };
+            // descriptors of the operand tiles; the start address advances in
+            // 16-byte units (32 bytes per K step inside a block, kBlk across)
+            const uint64_t dQ = tc::desc_k(sbase + OFF_Q), dQRH = tc::desc_k(sbase + OFF_QRH),
+                           dQRL = tc::desc_k(sbase + OFF_QRL), dKA = tc::desc_k(sbase + OFF_KA),
+                           dKY = tc::desc_k(sbase + OFF_KY), dP = tc::desc_k(sbase + OFF_P),
+                           dVA = tc::desc_mn(sbase + OFF_VA, kBlk), dVY = tc::desc_mn(sbase + OFF_VY, kBlk);
+            auto kstep = [](int kk) { return (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4); };
             auto logits = [&]() {
 #pragma unroll
-                for (int kk = 0; kk < 9; kk++)
-                    tc::mma_bf16(tmem + kColSA, kdesc(OFF_Q, kk), kdesc(OFF_KA, kk), idL, kk > 0);
+                for (int kk = 0; kk < 9; kk++) tc::mma_bf16(tmem + kColSA, dQ + kstep(kk), dKA + kstep(kk), idL, kk > 0);
                 if (RESID) {
 #pragma unroll
                     for (int kk = 0; kk < 9; kk++)
-                        tc::mma_bf16(tmem + kColSY, kdesc(OFF_QRH, kk), kdesc(OFF_KY, kk), idL, kk > 0);
+                        tc::mma_bf16(tmem + kColSY, dQRH + kstep(kk), dKY + kstep(kk), idL, kk > 0);
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++)
-                        tc::mma_bf16(tmem + kColSY, kdesc(OFF_QRL, kk), kdesc(OFF_KY, kk), idL, true);
+                    for (int kk = 0; kk < 8; kk++) tc::mma_bf16(tmem + kColSY, dQRL + kstep(kk), dKY + kstep(kk), idL, true);
                 }
                 tc::commit(&bar_kdone);
             };
             auto values = [&](int j) {
+                const uint64_t pbuf = dP + (uint64_t)(((j & 1) * kPBytes) >> 4);
 #pragma unroll
                 for (int part = 0; part < 2; part++) {
 #pragma unroll
                     for (int kk = 0; kk < kTok / 16; kk++)
-                        tc::mma_bf16(tmem + kColOA, tc::desc_k(sbase + OFF_PSH + part * kBlk + kk * 32),
-                                     tc::desc_mn(sbase + OFF_VA + kk * 2048, kBlk), idP, j > 0 || part > 0 || kk > 0);
+                        tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((part * kBlk + kk * 32) >> 4),
+                                     dVA + (uint64_t)((kk * 2048) >> 4), idP, j > 0 || part > 0 || kk > 0);
                     if (RESID) {
 #pragma unroll
                         for (int kk = 0; kk < kTok / 16; kk++)
-                            tc::mma_bf16(tmem + kColOY, tc::desc_k(sbase + OFF_PSH + (2 + part) * kBlk + kk * 32),
-                                         tc::desc_mn(sbase + OFF_VY + kk * 2048, kBlk), idP,
-                                         j > 0 || part > 0 || kk > 0);
+                            tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)(((2 + part) * kBlk + kk * 32) >> 4),
+                                         dVY + (uint64_t)((kk * 2048) >> 4), idP, j > 0 || part > 0 || kk > 0);
                     }
                 }
-                tc::commit(&bar_odone);
+                tc::commit(&bar_odone[j & 1]);
             };
-            for (int j = 0; j < ntl; j++) {
-                wait(&bar_kfull, j & 1, 25);
-                if (j > 0) wait(&bar_sfree, (j - 1) & 1, 26);
-                tc::fence_after();
-                logits();
-                if (j > 0) {
-                    wait(&bar_pfull, (j - 1) & 1, 27);
-                    wait(&bar_vfull, (j - 1) & 1, 28);
+            int nl = 0, nv = 0;   // steps whose logits / values are issued
+            unsigned long long idle0 = 0;
+            while (nv < ntl) {
+                bool did = false;
+                if (nl < ntl && mbar_test(&bar_kfull, nl & 1) &&
+                    (nl == 0 || mbar_test(&bar_sfree, (nl - 1) & 1))) {
                     tc::fence_after();
-                    values(j - 1);
+                    logits();
+                    nl++;
+                    did = true;
                 }
-            }
-            if (ntl > 0) {
-                wait(&bar_pfull, (ntl - 1) & 1, 27);
-                wait(&bar_vfull, (ntl - 1) & 1, 28);
-                tc::fence_after();
-                values(ntl - 1);
+                if (nv < nl && mbar_test(&bar_pfull[nv & 1], (nv >> 1) & 1) && mbar_test(&bar_vfull, nv & 1)) {
+                    tc::fence_after();
+                    values(nv);
+                    nv++;
+                    did = true;
+                }
+                if (did) {
+                    idle0 = 0;
+                } else if (idle0 == 0) {
+                    idle0 = global_ns();
+                } else if (*abort_flag || global_ns() - idle0 > kWaitNs) {
+                    *abort_flag = 1;
+                    atomicExch(a.err, 25);
+                    break;
+                }
             }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------- dequantize
+        // Thread (part, t): token t of the step, half (part & 1) of its
+        // anchor (part < 2) or residual record.  The records of step j + 1
+        // are loaded into registers while the tiles of step j are in use.
         const int dt = tid - 32 * (kSoftmaxWarps + 1);
         const int part = dt >> 6;   // 0, 1: anchor halves; 2, 3: residual halves
         const int t = dt & (kTok - 1);
-        for (int j = 0; j < ntl; j++) {
-            const int tt = j * kTok;
-            const bool ok = t < min(kTok, cnt - tt);
-            const size_t rec = bh * a.Tp + t0 + tt + t;
-#pragma unroll
-            for (int kv = 0; kv < 2; kv++) {
-                if (j > 0) wait(kv == 0 ? &bar_kdone : &bar_odone, (j - 1) & 1, 29);
-                uint8_t *ta = sm + (kv == 0 ? OFF_KA : OFF_VA);
-                uint8_t *ty = sm + (kv == 0 ? OFF_KY : OFF_VY);
-                const uint8_t *ac = ok ? a.a_codes[kv] + rec * (16 * BA) : nullptr;
-                const uint8_t *am = ok ? a.a_meta[kv] + rec * MR : nullptr;
-                if (part == 0) deq_half<BA, GS, 0>(ta, t, ac, am, ok);
-                else if (part == 1) deq_half<BA, GS, 1>(ta, t, ac, am, ok);
-                else if (RESID) {
-                    const uint8_t *rc = ok ? a.r_codes[kv] + rec * (16 * BR) : nullptr;
-                    const uint8_t *rm = ok ? a.r_meta[kv] + rec * MR : nullptr;
-                    if (part == 2) deq_half<BR, GS, 0>(ty, t, rc, rm, ok);
-                    else deq_half<BR, GS, 1>(ty, t, rc, rm, ok);
+        auto load = [&](int j, int kv, RawHalf &r, uint16_t *cf) {
+            const bool ok = t < min(kTok, cnt - j * kTok);
+            const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok + t;
+            if (part < 2) {
+                load_half<BA, GS>(ok ? a.a_codes[kv] + rec * (16 * BA) : nullptr, ok ? a.a_meta[kv] + rec * MR : nullptr,
+                                  part, ok, r);
+                if (RESID && part == 0 && kv == 0) {
+                    cf[0] = ok ? __ldg(a.r_coef[0] + rec) : 0;
+                    cf[1] = ok ? __ldg(a.r_coef[1] + rec) : 0;
                 }
-                if (kv == 0 && part == 0) {
-                    // slot j & 1 was last read at step j - 2, before the softmax
-                    // released step j - 1's logits, which this step's K waited for
-                    s_cK[j & 1][t] = RESID && ok ? bf16_to_f32(a.r_coef[0][rec]) : 1.f;
-                    s_cV[j & 1][t] = RESID && ok ? bf16_to_f32(a.r_coef[1][rec]) : 1.f;
-                    mbar_arrive(&bar_cfull[j & 1]);
-                }
-                tc::fence_async_smem();
-                mbar_arrive(kv == 0 ? &bar_kfull : &bar_vfull);
+            } else if (RESID) {
+                load_half<BR, GS>(ok ? a.r_codes[kv] + rec * (16 * BR) : nullptr, ok ? a.r_meta[kv] + rec * MR : nullptr,
+                                  part - 2, ok, r);
             }
+        };
+        auto store = [&](int j, int kv, const RawHalf &r) {
+            const bool ok = t < min(kTok, cnt - j * kTok);
+            uint8_t *ta = sm + (kv == 0 ? OFF_KA : OFF_VA);
+            uint8_t *ty = sm + (kv == 0 ? OFF_KY : OFF_VY);
+            if (part == 0) store_half<BA, GS, 0>(ta, t, r, ok);
+            else if (part == 1) store_half<BA, GS, 1>(ta, t, r, ok);
+            else if (RESID) {
+                if (part == 2) store_half<BR, GS, 0>(ty, t, r, ok);
+                else store_half<BR, GS, 1>(ty, t, r, ok);
+            }
+        };
+        RawHalf rk, rv;
+        uint16_t cf[2] = {0, 0};
+        if (ntl > 0) {
+            load(0, 0, rk, cf);
+            load(0, 1, rv, cf);
+        }
+        for (int j = 0; j < ntl; j++) {
+            const bool ok = t < min(kTok, cnt - j * kTok);
+            // K of step j (its tile was released by step j - 1's logits)
+            if (j > 0) wait(&bar_kdone, (j - 1) & 1, 29);
+            store(j, 0, rk);
+            if (part == 0) {
+                // slot j & 1 was last read at step j - 2, before the softmax
+                // released step j - 1's logits, which this step's K waited for
+                s_cK[j & 1][t] = RESID && ok ? bf16_to_f32(cf[0]) : 1.f;
+                s_cV[j & 1][t] = RESID && ok ? bf16_to_f32(cf[1]) : 1.f;
+                mbar_arrive(&bar_cfull[j & 1]);
+            }
+            tc::fence_async_smem();
+            mbar_arrive(&bar_kfull);
+            if (j + 1 < ntl) load(j + 1, 0, rk, cf);
+            // V of step j (its tile was released by step j - 1's values)
+            if (j > 0) wait(&bar_odone[(j - 1) & 1], ((j - 1) >> 1) & 1, 29);
+            store(j, 1, rv);
+            tc::fence_async_smem();
+            mbar_arrive(&bar_vfull);
+            if (j + 1 < ntl) load(j + 1, 1, rv, cf);
         }
     }
 
@@ -656,9 +762,12 @@ cudaError_t launch_group(const PrefillArgs &a, int ba, int br, cudaStream_t st) 
 }  // namespace
 
 // Row blocks of 64 query rows per kv head; splits: the count with the least
-// wave-quantised work (waves x 64-token steps of the largest split, plus one
-// step of fixed cost), one CTA per SM (the tiles take 193 KB of shared memory
+// wave-quantised work (waves x 64-token steps of the largest split, plus a
+// fixed cost of RQ_PREFILL_STEP_OVERHEAD steps per CTA), one CTA per SM (the tiles take 193 KB of shared memory
 // and the accumulators all 512 tensor-memory columns).
+#ifndef RQ_PREFILL_STEP_OVERHEAD
+#define RQ_PREFILL_STEP_OVERHEAD 1
+#endif
 void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
     (void)ba;
     (void)br;
@@ -672,7 +781,7 @@ void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
     long best = -1;
     for (int S = 1; S <= std::min(nt, kMaxSplits); S++) {
         const long waves = (S * units + slots - 1) / slots;
-        const long cost = waves * ((nt + S - 1) / S + 1);
+        const long cost = waves * ((nt + S - 1) / S + RQ_PREFILL_STEP_OVERHEAD);
         if (best < 0 || cost < best) {
             best = cost;
             a->S = S;

@@ -190,22 +190,14 @@ struct DecodeArgs {
     uint32_t sigma[4];
 };
 
-// Tokens [*t0, *t0 + *n) of split `split` of S: the ceil(T/64) tiles, in
-// granules of `gran` tiles (a paged cache's block, so that no split starts
-// inside a block), are dealt out evenly (granule counts differ by at most
-// one; chunk >= the largest).
-__host__ __device__ inline void split_range(int split, int S, int T, int *t0, int *n, int gran = 1) {
+// Tokens [*t0, *t0 + *n) of split `split` of S: the ceil(T/64) tiles are
+// dealt out evenly (tile counts differ by at most one; chunk >= the largest).
+__host__ __device__ inline void split_range(int split, int S, int T, int *t0, int *n) {
     const int nt = (T + kTokTile - 1) / kTokTile;
-    const int nu = (nt + gran - 1) / gran;
-    const int lo = (int)((long long)split * nu / S) * gran;
-    int hi = (int)((long long)(split + 1) * nu / S) * gran;
-    hi = hi < nt ? hi : nt;
+    const int lo = (int)((long long)split * nt / S), hi = (int)((long long)(split + 1) * nt / S);
     *t0 = lo * kTokTile;
     *n = (hi * kTokTile < T ? hi * kTokTile : T) - *t0;
-    if (*n < 0) *n = 0;
 }
-// Tiles per split granule of a record layout: one block of a paged cache.
-__host__ __device__ inline int split_granule(const Pages &p) { return p.table ? p.bt / kTokTile : 1; }
 
 struct CombineArgs {
     const float *partials;
