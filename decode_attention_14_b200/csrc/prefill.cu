@@ -62,32 +62,35 @@ namespace rq {
 namespace {
 
 constexpr int kRows = 64;             // query rows of a CTA (M of every MMA)
-constexpr int kTok = kPrefillTile;    // committed tokens per step
+constexpr int kTok = kPrefillTile;    // committed tokens per step (N of the logits, K of the values)
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kDeqWarps = 8;
 constexpr int kDeqThreads = 32 * kDeqWarps;
 constexpr int kThreadsP = 32 * (kSoftmaxWarps + 1 + kDeqWarps);
-constexpr int kBlk = kRows * 128;     // one 64-row block of 64 bf16 columns (8 KB)
-static_assert(kTok == kRows, "K/V tiles and query tiles share the 64-row block");
-// Operand tiles: a 3-block tile holds head_dim (blocks 0, 1) and the 16
-// minimum / group-sum columns (first 32 bytes of each row of block 2).
-constexpr int OFF_Q = 0;              // q | Q_g hi, lo
-constexpr int OFF_QRH = 3 * kBlk;     // Rq hi | (Rq)_g hi, lo
-constexpr int OFF_QRL = 6 * kBlk;     // Rq lo
-constexpr int OFF_KA = 8 * kBlk;      // anchor K: sc code | mn, mn
-constexpr int OFF_KY = 11 * kBlk;     // residual K
-constexpr int OFF_VA = 14 * kBlk;     // anchor V (read MN-major)
-constexpr int OFF_VY = 17 * kBlk;     // residual V
-constexpr int OFF_P = 20 * kBlk;      // two buffers of [(p s) hi, (p s) lo, p hi, p lo], a block each
-constexpr int kPBytes = 4 * kBlk;
-constexpr int kTilesBytes = 28 * kBlk;
+constexpr int kQBlk = kRows * 128;    // a 64-row block of 64 bf16 columns (8 KB): query-side operands
+constexpr int kTBlk = kTok * 128;     // a block of the step's token rows (4 KB): key / value operands
+static_assert(kDeqThreads == 2 * 4 * kTok, "a dequantizing thread per (K or V, record half, token)");
+// Operand tiles of 3 blocks hold head_dim (blocks 0, 1) and the 16 minimum /
+// group-sum columns (first 32 bytes of each row of block 2).  K, V and the
+// probabilities are double-buffered by step parity.
+constexpr int OFF_Q = 0;                 // q | Q_g hi, lo
+constexpr int OFF_QRH = 3 * kQBlk;       // Rq hi | (Rq)_g hi, lo
+constexpr int OFF_QRL = 6 * kQBlk;       // Rq lo
+constexpr int OFF_K = 8 * kQBlk;         // per buffer: anchor K (sc code | mn, mn), then residual K
+constexpr int kKVBytes = 6 * kTBlk;
+constexpr int OFF_V = OFF_K + 2 * kKVBytes;   // per buffer: anchor V, then residual V (read MN-major)
+constexpr int OFF_P = OFF_V + 2 * kKVBytes;   // per buffer: (p s) hi, (p s) lo, p hi, p lo, a block each
+constexpr int kPBytes = 4 * kQBlk;
+constexpr int kTilesBytes = OFF_P + 2 * kPBytes;
 constexpr int kSmemBytes = kTilesBytes + 1024;   // + alignment of the base to 1024
-// tensor-memory columns (fp32): logits of a step, then the value accumulators
-constexpr uint32_t kColSA = 0, kColSY = 64, kColOA = 128, kColOY = 272, kTmemCols = 512;
+// tensor-memory columns (fp32): the logits SA, SY of each step buffer, then
+// the value accumulators OA, OY
+constexpr uint32_t kColS = 0, kColOA = 128, kColOY = 272, kTmemCols = 512;
 constexpr int kOCols = kHeadDim + 8;             // head_dim + one column per group minimum
 constexpr float kRescaleLog2 = 8.f;              // raise a row's maximum only past 2^8
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
+static_assert(2 * 2 * kTok <= (int)kColOA, "two buffers of SA, SY fit before OA");
 
 __device__ __forceinline__ uint32_t bf16_bits(float x) { return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 __device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
@@ -115,6 +118,9 @@ __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t 
 __device__ __forceinline__ void st_shared16(uint8_t *p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
+}
+__device__ __forceinline__ void st_shared_u16(uint8_t *p, uint32_t x) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(smem_u32(p)), "h"((unsigned short)x) : "memory");
 }
 __device__ __forceinline__ void st_shared8(uint8_t *p, uint32_t x, uint32_t y) {
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(p)), "r"(x), "r"(y) : "memory");
@@ -174,11 +180,11 @@ __device__ __forceinline__ void load_half(const uint8_t *codes, const uint8_t *m
 // sc * code per element, exact in BF16 ((128 + code) sc - 128 sc in one
 // rounding); HALF 0 also writes the minimum columns (mn_0 .. mn_{NG-1},
 // zeros, twice).  A token past the step (ok false) gets a zero row.
-template <int BITS, int GS, int HALF>
+template <int BITS, int GS, int HALF, int BLK>
 __device__ __forceinline__ void store_half(uint8_t *tile, int t, const RawHalf &r, bool ok) {
     constexpr int NG = kHeadDim / GS;
-    uint8_t *row = tile + HALF * kBlk;
-    uint8_t *mrow = tile + 2 * kBlk;
+    uint8_t *row = tile + HALF * BLK;
+    uint8_t *mrow = tile + 2 * BLK;
     if (!ok) {
 #pragma unroll
         for (int c = 0; c < 8; c++) st_shared16(row + tc::sw_chunk(t, c), 0u, 0u, 0u, 0u);
@@ -262,26 +268,27 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
         x[2] = bf16_val(raw.y & 0xFFFFu);
         x[3] = bf16_val(raw.y >> 16);
         // elements 4 lane .. 4 lane + 3: block lane / 16, chunk (lane % 16) / 2, half (lane & 1)
-        const uint32_t off = (uint32_t)(lane >> 4) * kBlk + tc::sw_chunk(r, (lane & 15) >> 1) + 8u * (lane & 1);
+        const uint32_t off = (uint32_t)(lane >> 4) * kQBlk + tc::sw_chunk(r, (lane & 15) >> 1) + 8u * (lane & 1);
         st_shared8(sm + OFF_Q + off, raw.x, raw.y);
         // group sums (hi, lo) into columns 128 + g and 136 + g
         auto sums = [&](const float v[4], uint8_t *tile) {
             float gs = (v[0] + v[1]) + (v[2] + v[3]);
 #pragma unroll
             for (int o = 1; o < LPG; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-            uint32_t hi[8], lo[8];
-#pragma unroll
-            for (int g = 0; g < 8; g++) {
-                const float s = __shfl_sync(0xffffffffu, gs, (g % NG) * LPG);
-                split_hi_lo(s, hi[g], lo[g]);
-                if (g >= NG) hi[g] = lo[g] = 0u;
+            uint8_t *mrow = tile + 2 * kQBlk;
+            if (NG < 8) {   // unused group columns are zero
+                if (lane == 0) {
+                    st_shared16(mrow + tc::sw_chunk(r, 0), 0u, 0u, 0u, 0u);
+                    st_shared16(mrow + tc::sw_chunk(r, 1), 0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
             }
-            if (lane == 0) {
-                uint8_t *mrow = tile + 2 * kBlk;
-                st_shared16(mrow + tc::sw_chunk(r, 0), hi[0] | hi[1] << 16, hi[2] | hi[3] << 16, hi[4] | hi[5] << 16,
-                            hi[6] | hi[7] << 16);
-                st_shared16(mrow + tc::sw_chunk(r, 1), lo[0] | lo[1] << 16, lo[2] | lo[3] << 16, lo[4] | lo[5] << 16,
-                            lo[6] | lo[7] << 16);
+            if (lane % LPG == 0) {   // the group's first lane holds its sum
+                const int g = lane / LPG;
+                uint32_t hi, lo;
+                split_hi_lo(gs, hi, lo);
+                st_shared_u16(mrow + tc::sw_chunk(r, 0) + 2 * g, hi);
+                st_shared_u16(mrow + tc::sw_chunk(r, 1) + 2 * g, lo);
             }
         };
         sums(x, sm + OFF_Q);
@@ -308,10 +315,13 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
 template <int BA, int BR, int GS, bool RESID>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bar_kfull, bar_vfull, bar_kdone, bar_sfree, bar_cfull[2], bar_pfull[2], bar_odone[2];
+    // per step buffer b = j & 1 (k-th completion: step 2k + b); cfull per
+    // coefficient slot j & 3 (k-th completion: step 4k + slot)
+    __shared__ uint64_t bar_kfull[2], bar_vfull[2], bar_kdone[2], bar_sfree[2], bar_pfull[2], bar_odone[2];
+    __shared__ uint64_t bar_cfull[4];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_cK[2][kTok], s_cV[2][kTok];   // coefficients of the step (1 at an anchor loop)
+    __shared__ float s_cK[4][kTok], s_cV[4][kTok];   // coefficients of a step (1 at an anchor loop)
     __shared__ float s_ml[kRows][2];                  // running maximum and sum of each row
 
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -331,15 +341,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
     constexpr int MR = 2 * (kHeadDim / GS);
 
     if (tid == 0) {
-        mbar_init(&bar_kfull, kDeqThreads);
-        mbar_init(&bar_vfull, kDeqThreads);
-        mbar_init(&bar_kdone, 1);
-        mbar_init(&bar_sfree, 32 * kSoftmaxWarps);
         for (int i = 0; i < 2; i++) {
-            mbar_init(&bar_cfull[i], kTok);
+            mbar_init(&bar_kfull[i], kDeqThreads / 2);
+            mbar_init(&bar_vfull[i], kDeqThreads / 2);
+            mbar_init(&bar_kdone[i], 1);
+            mbar_init(&bar_sfree[i], 32 * kSoftmaxWarps);
             mbar_init(&bar_pfull[i], 32 * kSoftmaxWarps);
             mbar_init(&bar_odone[i], 1);
         }
+        for (int i = 0; i < 4; i++) mbar_init(&bar_cfull[i], kTok);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -360,10 +370,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             atomicExch(a.err, code);
         }
     };
-    // Phases.  kfull, vfull, kdone, sfree complete once per step; cfull[i],
-    // pfull[i] and odone[i] once per step of parity i (their k-th completion
-    // belongs to step 2k + i).  No barrier can run two phases ahead of a
-    // waiter (each next phase needs work the waiter has not released yet).
+    // No barrier runs two of its phases ahead of a waiter: each next phase
+    // needs work that the waiter itself releases later (the hand-offs below).
 
     if (warp < kSoftmaxWarps) {
         // ------------------------------------------------------- softmax
@@ -381,30 +389,34 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         for (int j = 0; j < ntl; j++) {
             const int tt = j * kTok;
             const int tn = min(kTok, cnt - tt);
-            const int pb = j & 1;   // probability buffer of the step
-            wait(&bar_cfull[pb], (j >> 1) & 1, 21);   // the step's coefficients
-            wait(&bar_kdone, j & 1, 22);
+            const int pb = j & 1;   // step buffer
+            const int cs = j & 3;   // coefficient slot
+            wait(&bar_cfull[cs], (j >> 2) & 1, 21);
+            wait(&bar_kdone[pb], (j >> 1) & 1, 22);
             tc::fence_after();
-            float s[kHalf];
-#pragma unroll
-            for (int c = 0; c < kHalf; c += 16) {
+            // logits, and this thread's V coefficients, read before the
+            // logits buffer and the coefficient slot are released
+            float s[kHalf], cv[kHalf];
+            {
                 uint32_t va[16], vy[16];
-                tc::ld16x2<kHalf>(tl + kColSA + c, va);
+                const uint32_t cS = kColS + pb * 2 * kTok;
+                tc::ld16x2<kHalf>(tl + cS, va);
                 if (RESID) {
-                    tc::ld16x2<kHalf>(tl + kColSY + c, vy);
+                    tc::ld16x2<kHalf>(tl + cS + kTok, vy);
                     tc::wait_ld2(va, vy);
                 } else {
                     tc::wait_ld(va);
                 }
 #pragma unroll
-                for (int k = 0; k < 16; k++) {
+                for (int k = 0; k < kHalf; k++) {
                     const float sa = __uint_as_float(va[k]);
-                    const float x = RESID ? fmaf(s_cK[pb][kHalf * hf + c + k], sa, __uint_as_float(vy[k])) : sa;
-                    s[c + k] = x * a.scale_log2;
+                    const float x = RESID ? fmaf(s_cK[cs][kHalf * hf + k], sa, __uint_as_float(vy[k])) : sa;
+                    s[k] = x * a.scale_log2;
+                    cv[k] = RESID ? s_cV[cs][kHalf * hf + k] : 1.f;
                 }
             }
             tc::fence_before();
-            mbar_arrive(&bar_sfree);
+            mbar_arrive(&bar_sfree[pb]);
             float mx = -CUDART_INF_F;
 #pragma unroll
             for (int k = 0; k < kHalf; k++) {
@@ -460,6 +472,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             }
             l *= f;
             // probabilities of the step, split hi / lo, into the A operands
+            // (K = the step's 32 tokens: the first 64 bytes of each 128-byte row)
             const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
             uint8_t *prow = sm + OFF_P + pb * kPBytes;
 #pragma unroll
@@ -467,11 +480,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 uint32_t psh[4], psl[4], ph[4], pl[4];
 #pragma unroll
                 for (int k = 0; k < 8; k += 2) {
-                    const int t = kHalf * hf + 8 * cc + k;
-                    const float p0 = exp2f(s[8 * cc + k] - mu), p1 = exp2f(s[8 * cc + k + 1] - mu);   // 0 if masked
+                    const int u = 8 * cc + k;
+                    const float p0 = exp2f(s[u] - mu), p1 = exp2f(s[u + 1] - mu);   // 0 if masked
                     l += p0 + p1;
                     if (RESID) {
-                        split_hi_lo2(p0 * s_cV[pb][t], p1 * s_cV[pb][t + 1], psh[k / 2], psl[k / 2]);
+                        split_hi_lo2(p0 * cv[u], p1 * cv[u + 1], psh[k / 2], psl[k / 2]);
                         split_hi_lo2(p0, p1, ph[k / 2], pl[k / 2]);
                     } else {
                         split_hi_lo2(p0, p1, psh[k / 2], psl[k / 2]);
@@ -479,10 +492,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 }
                 const uint32_t o = tc::sw_chunk(r, (kHalf / 8) * hf + cc);
                 st_shared16(prow + o, psh[0], psh[1], psh[2], psh[3]);
-                st_shared16(prow + kBlk + o, psl[0], psl[1], psl[2], psl[3]);
+                st_shared16(prow + kQBlk + o, psl[0], psl[1], psl[2], psl[3]);
                 if (RESID) {
-                    st_shared16(prow + 2 * kBlk + o, ph[0], ph[1], ph[2], ph[3]);
-                    st_shared16(prow + 3 * kBlk + o, pl[0], pl[1], pl[2], pl[3]);
+                    st_shared16(prow + 2 * kQBlk + o, ph[0], ph[1], ph[2], ph[3]);
+                    st_shared16(prow + 3 * kQBlk + o, pl[0], pl[1], pl[2], pl[3]);
                 }
             }
             tc::fence_async_smem();
@@ -496,8 +509,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         // warp per row applies R^T to Y with the in-warp transform and writes
         // the partial, 4 consecutive elements per lane.
         constexpr int kEStride = kHeadDim + 4;   // padded rows: the row-per-thread stores do not conflict
-        float *sA = reinterpret_cast<float *>(sm + OFF_KA);
-        float *sY = reinterpret_cast<float *>(sm + OFF_VA);
+        static_assert(kRows * kEStride * 4 <= 2 * kKVBytes, "staging fits in the K (and the V) tiles");
+        float *sA = reinterpret_cast<float *>(sm + OFF_K);
+        float *sY = reinterpret_cast<float *>(sm + OFF_V);
         if (ntl > 0) {
             // the last values complete (and with them every earlier MMA)
             wait(&bar_odone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, 24);
@@ -567,43 +581,47 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------- MMA issue
-        // One thread; the logits of step j + 1 and the values of step j are
-        // issued in whichever order their operands become ready.
+        // One thread; the logits of the next steps and the values of the
+        // current one are issued in whichever order their operands are ready.
         if (lane == 0) {
             constexpr uint32_t idL = tc::idesc_bf16(kRows, kTok, false);
             constexpr uint32_t idP = tc::idesc_bf16(kRows, kOCols, true);
             // descriptors of the operand tiles; the start address advances in
-            // 16-byte units (32 bytes per K step inside a block, kBlk across)
+            // 16-byte units (32 bytes per K step inside a block, a block across)
             const uint64_t dQ = tc::desc_k(sbase + OFF_Q), dQRH = tc::desc_k(sbase + OFF_QRH),
-                           dQRL = tc::desc_k(sbase + OFF_QRL), dKA = tc::desc_k(sbase + OFF_KA),
-                           dKY = tc::desc_k(sbase + OFF_KY), dP = tc::desc_k(sbase + OFF_P),
-                           dVA = tc::desc_mn(sbase + OFF_VA, kBlk), dVY = tc::desc_mn(sbase + OFF_VY, kBlk);
-            auto kstep = [](int kk) { return (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4); };
-            auto logits = [&]() {
+                           dQRL = tc::desc_k(sbase + OFF_QRL), dK = tc::desc_k(sbase + OFF_K),
+                           dP = tc::desc_k(sbase + OFF_P), dV = tc::desc_mn(sbase + OFF_V, kTBlk);
+            auto kq = [](int kk) { return (uint64_t)(((kk >> 2) * kQBlk + (kk & 3) * 32) >> 4); };
+            auto kt = [](int kk) { return (uint64_t)(((kk >> 2) * kTBlk + (kk & 3) * 32) >> 4); };
+            auto logits = [&](int j) {
+                const uint64_t ka = dK + (uint64_t)(((j & 1) * kKVBytes) >> 4);
+                const uint64_t ky = ka + (uint64_t)((3 * kTBlk) >> 4);
+                const uint32_t cS = tmem + kColS + (j & 1) * 2 * kTok;
 #pragma unroll
-                for (int kk = 0; kk < 9; kk++) tc::mma_bf16(tmem + kColSA, dQ + kstep(kk), dKA + kstep(kk), idL, kk > 0);
+                for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idL, kk > 0);
                 if (RESID) {
 #pragma unroll
-                    for (int kk = 0; kk < 9; kk++)
-                        tc::mma_bf16(tmem + kColSY, dQRH + kstep(kk), dKY + kstep(kk), idL, kk > 0);
+                    for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS + kTok, dQRH + kq(kk), ky + kt(kk), idL, kk > 0);
 #pragma unroll
-                    for (int kk = 0; kk < 8; kk++) tc::mma_bf16(tmem + kColSY, dQRL + kstep(kk), dKY + kstep(kk), idL, true);
+                    for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS + kTok, dQRL + kq(kk), ky + kt(kk), idL, true);
                 }
-                tc::commit(&bar_kdone);
+                tc::commit(&bar_kdone[j & 1]);
             };
             auto values = [&](int j) {
                 const uint64_t pbuf = dP + (uint64_t)(((j & 1) * kPBytes) >> 4);
+                const uint64_t va = dV + (uint64_t)(((j & 1) * kKVBytes) >> 4);
+                const uint64_t vy = va + (uint64_t)((3 * kTBlk) >> 4);
 #pragma unroll
                 for (int part = 0; part < 2; part++) {
 #pragma unroll
                     for (int kk = 0; kk < kTok / 16; kk++)
-                        tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((part * kBlk + kk * 32) >> 4),
-                                     dVA + (uint64_t)((kk * 2048) >> 4), idP, j > 0 || part > 0 || kk > 0);
+                        tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((part * kQBlk + kk * 32) >> 4),
+                                     va + (uint64_t)((kk * 16 * 128) >> 4), idP, j > 0 || part > 0 || kk > 0);
                     if (RESID) {
 #pragma unroll
                         for (int kk = 0; kk < kTok / 16; kk++)
-                            tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)(((2 + part) * kBlk + kk * 32) >> 4),
-                                         dVY + (uint64_t)((kk * 2048) >> 4), idP, j > 0 || part > 0 || kk > 0);
+                            tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)(((2 + part) * kQBlk + kk * 32) >> 4),
+                                         vy + (uint64_t)((kk * 16 * 128) >> 4), idP, j > 0 || part > 0 || kk > 0);
                     }
                 }
                 tc::commit(&bar_odone[j & 1]);
@@ -612,14 +630,17 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             unsigned long long idle0 = 0;
             while (nv < ntl) {
                 bool did = false;
-                if (nl < ntl && mbar_test(&bar_kfull, nl & 1) &&
-                    (nl == 0 || mbar_test(&bar_sfree, (nl - 1) & 1))) {
+                // logits of step nl: its K written, its logits buffer read by the softmax of step nl - 2
+                if (nl < ntl && mbar_test(&bar_kfull[nl & 1], (nl >> 1) & 1) &&
+                    (nl < 2 || mbar_test(&bar_sfree[nl & 1], ((nl >> 1) - 1) & 1))) {
                     tc::fence_after();
-                    logits();
+                    logits(nl);
                     nl++;
                     did = true;
                 }
-                if (nv < nl && mbar_test(&bar_pfull[nv & 1], (nv >> 1) & 1) && mbar_test(&bar_vfull, nv & 1)) {
+                // values of step nv: its probabilities and V written
+                if (nv < nl && mbar_test(&bar_pfull[nv & 1], (nv >> 1) & 1) &&
+                    mbar_test(&bar_vfull[nv & 1], (nv >> 1) & 1)) {
                     tc::fence_after();
                     values(nv);
                     nv++;
@@ -639,65 +660,55 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         __syncwarp();
     } else {
         // ------------------------------------------------------- dequantize
-        // Thread (part, t): token t of the step, half (part & 1) of its
-        // anchor (part < 2) or residual record.  The records of step j + 1
-        // are loaded into registers while the tiles of step j are in use.
+        // Thread (side, part, t): token t of the step, K (side 0) or V, half
+        // (part & 1) of its anchor (part < 2) or residual record.  The record
+        // of step j + 1 is loaded into registers while step j's is written.
         const int dt = tid - 32 * (kSoftmaxWarps + 1);
-        const int part = dt >> 6;   // 0, 1: anchor halves; 2, 3: residual halves
-        const int t = dt & (kTok - 1);
-        auto load = [&](int j, int kv, RawHalf &r, uint16_t *cf) {
+        const int side = dt / (4 * kTok);
+        const int part = (dt / kTok) & 3;   // 0, 1: anchor halves; 2, 3: residual halves
+        const int t = dt % kTok;
+        auto load = [&](int j, RawHalf &r, uint16_t *cf) {
             const bool ok = t < min(kTok, cnt - j * kTok);
             const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok + t;
             if (part < 2) {
-                load_half<BA, GS>(ok ? a.a_codes[kv] + rec * (16 * BA) : nullptr, ok ? a.a_meta[kv] + rec * MR : nullptr,
-                                  part, ok, r);
-                if (RESID && part == 0 && kv == 0) {
+                load_half<BA, GS>(ok ? a.a_codes[side] + rec * (16 * BA) : nullptr,
+                                  ok ? a.a_meta[side] + rec * MR : nullptr, part, ok, r);
+                if (RESID && part == 0 && side == 0) {
                     cf[0] = ok ? __ldg(a.r_coef[0] + rec) : 0;
                     cf[1] = ok ? __ldg(a.r_coef[1] + rec) : 0;
                 }
             } else if (RESID) {
-                load_half<BR, GS>(ok ? a.r_codes[kv] + rec * (16 * BR) : nullptr, ok ? a.r_meta[kv] + rec * MR : nullptr,
-                                  part - 2, ok, r);
+                load_half<BR, GS>(ok ? a.r_codes[side] + rec * (16 * BR) : nullptr,
+                                  ok ? a.r_meta[side] + rec * MR : nullptr, part - 2, ok, r);
             }
         };
-        auto store = [&](int j, int kv, const RawHalf &r) {
-            const bool ok = t < min(kTok, cnt - j * kTok);
-            uint8_t *ta = sm + (kv == 0 ? OFF_KA : OFF_VA);
-            uint8_t *ty = sm + (kv == 0 ? OFF_KY : OFF_VY);
-            if (part == 0) store_half<BA, GS, 0>(ta, t, r, ok);
-            else if (part == 1) store_half<BA, GS, 1>(ta, t, r, ok);
-            else if (RESID) {
-                if (part == 2) store_half<BR, GS, 0>(ty, t, r, ok);
-                else store_half<BR, GS, 1>(ty, t, r, ok);
-            }
-        };
-        RawHalf rk, rv;
+        RawHalf raw;
         uint16_t cf[2] = {0, 0};
-        if (ntl > 0) {
-            load(0, 0, rk, cf);
-            load(0, 1, rv, cf);
-        }
+        if (ntl > 0) load(0, raw, cf);
         for (int j = 0; j < ntl; j++) {
             const bool ok = t < min(kTok, cnt - j * kTok);
-            // K of step j (its tile was released by step j - 1's logits)
-            if (j > 0) wait(&bar_kdone, (j - 1) & 1, 29);
-            store(j, 0, rk);
-            if (part == 0) {
-                // slot j & 1 was last read at step j - 2, before the softmax
-                // released step j - 1's logits, which this step's K waited for
-                s_cK[j & 1][t] = RESID && ok ? bf16_to_f32(cf[0]) : 1.f;
-                s_cV[j & 1][t] = RESID && ok ? bf16_to_f32(cf[1]) : 1.f;
-                mbar_arrive(&bar_cfull[j & 1]);
+            const int pb = j & 1;
+            // the buffer was last read by the logits (K) / values (V) of step j - 2
+            if (j >= 2) wait(side == 0 ? &bar_kdone[pb] : &bar_odone[pb], ((j >> 1) - 1) & 1, 29);
+            uint8_t *ta = sm + (side == 0 ? OFF_K : OFF_V) + pb * kKVBytes;
+            uint8_t *ty = ta + 3 * kTBlk;
+            if (part == 0) store_half<BA, GS, 0, kTBlk>(ta, t, raw, ok);
+            else if (part == 1) store_half<BA, GS, 1, kTBlk>(ta, t, raw, ok);
+            else if (RESID) {
+                if (part == 2) store_half<BR, GS, 0, kTBlk>(ty, t, raw, ok);
+                else store_half<BR, GS, 1, kTBlk>(ty, t, raw, ok);
+            }
+            if (side == 0 && part == 0) {
+                // slot j & 3 was last read by the softmax of step j - 4, before
+                // it released the logits of that step, which the logits of
+                // step j - 2 (hence this K buffer) waited for
+                s_cK[j & 3][t] = RESID && ok ? bf16_to_f32(cf[0]) : 1.f;
+                s_cV[j & 3][t] = RESID && ok ? bf16_to_f32(cf[1]) : 1.f;
+                mbar_arrive(&bar_cfull[j & 3]);
             }
             tc::fence_async_smem();
-            mbar_arrive(&bar_kfull);
-            if (j + 1 < ntl) load(j + 1, 0, rk, cf);
-            // V of step j (its tile was released by step j - 1's values)
-            if (j > 0) wait(&bar_odone[(j - 1) & 1], ((j - 1) >> 1) & 1, 29);
-            store(j, 1, rv);
-            tc::fence_async_smem();
-            mbar_arrive(&bar_vfull);
-            if (j + 1 < ntl) load(j + 1, 1, rv, cf);
+            mbar_arrive(side == 0 ? &bar_kfull[pb] : &bar_vfull[pb]);
+            if (j + 1 < ntl) load(j + 1, raw, cf);
         }
     }
 

@@ -6,7 +6,7 @@
 
 namespace rq {
 
-constexpr int kPrefillTile = 64;   // committed tokens per step of a CTA (one split granule)
+constexpr int kPrefillTile = 32;   // committed tokens per step of a CTA
 
 // Causal attention of the n most recent tokens of every sequence: query row
 // (i, hq) of sequence b (i < n) sees the first T_b + n_tail - n + 1 + i tokens
