@@ -68,20 +68,24 @@ constexpr int kMmaWarp = 4;
 constexpr int kDeqWarps = 8;
 constexpr int kDeqThreads = 32 * kDeqWarps;
 constexpr int kThreadsP = 32 * (kSoftmaxWarps + 1 + kDeqWarps);
-constexpr int kQBlk = kRows * 128;    // a 64-row block of 64 bf16 columns (8 KB): query-side operands
+constexpr int kQBlk = kRows * 128;    // a 64-row block of 64 bf16 columns (8 KB): q
+constexpr int kSBlk = 2 * kQBlk;      // a 128-row block (16 KB): stacked high / low operands (M = 128)
 constexpr int kTBlk = kTok * 128;     // a block of the step's token rows (4 KB): key / value operands
 static_assert(kDeqThreads == 2 * 4 * kTok, "a dequantizing thread per (K or V, record half, token)");
 // Operand tiles of 3 blocks hold head_dim (blocks 0, 1) and the 16 minimum /
-// group-sum columns (first 32 bytes of each row of block 2).  K, V and the
-// probabilities are double-buffered by step parity.
-constexpr int OFF_Q = 0;                 // q | Q_g hi, lo
-constexpr int OFF_QRH = 3 * kQBlk;       // Rq hi | (Rq)_g hi, lo
-constexpr int OFF_QRL = 6 * kQBlk;       // Rq lo
-constexpr int OFF_K = 8 * kQBlk;         // per buffer: anchor K (sc code | mn, mn), then residual K
+// group-sum columns (the first 32 bytes of each row of block 2).  Operands
+// with a BF16 high and low part are stacked as the two halves of an M = 128
+// operand: row 32 (r / 16) + r % 16 holds the high part of query row r, the
+// row 16 after it the low part, so that both land in the tensor-memory lanes
+// of the warp that owns row r.  K, V and the probabilities are
+// double-buffered by step parity.
+constexpr int OFF_Q = 0;                 // q (blocks 0, 1; its group sums: chunks 2, 3 of block 2 of OFF_QR)
+constexpr int OFF_QR = 2 * kQBlk;        // stacked Rq hi / lo | (Rq)_g hi, lo on the high rows
+constexpr int OFF_K = OFF_QR + 3 * kSBlk;   // per buffer: anchor K (sc code | mn, mn), then residual K
 constexpr int kKVBytes = 6 * kTBlk;
 constexpr int OFF_V = OFF_K + 2 * kKVBytes;   // per buffer: anchor V, then residual V (read MN-major)
-constexpr int OFF_P = OFF_V + 2 * kKVBytes;   // per buffer: (p s) hi, (p s) lo, p hi, p lo, a block each
-constexpr int kPBytes = 4 * kQBlk;
+constexpr int OFF_P = OFF_V + 2 * kKVBytes;   // per buffer: stacked (p s) hi / lo, then stacked p hi / lo
+constexpr int kPBytes = 2 * kSBlk;
 constexpr int kTilesBytes = OFF_P + 2 * kPBytes;
 constexpr int kSmemBytes = kTilesBytes + 1024;   // + alignment of the base to 1024
 // tensor-memory columns (fp32): the logits SA, SY of each step buffer, then
@@ -237,14 +241,17 @@ __device__ __forceinline__ void store_half(uint8_t *tile, int t, const RawHalf &
     }
 }
 
-// Query operands of the CTA's 64 rows (rows past nr are zero): q and its
-// group sums (hi, lo) into OFF_Q; for a residual loop Rq hi / lo and the
-// group sums of Rq (hi, lo) into OFF_QRH / OFF_QRL.  A warp per row.
+// Query operands of the CTA's 64 rows (rows past nr are zero): q into OFF_Q
+// and its group sums (hi, lo) into chunks 2, 3 of row r of block 2 of the
+// stacked tile; for a residual loop Rq hi / lo into the stacked tile's high
+// and low rows and the group sums of Rq (hi, lo) into chunks 0, 1 of the
+// high row (zero on the low row).  A warp per row.
 template <int GS, bool RESID>
 __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm, int b, int h, int r0, int nr,
                                               int warp, int lane) {
     constexpr int NG = kHeadDim / GS, LPG = GS / 4;   // lanes per group
     constexpr int kWarps = kThreadsP / 32, kRowsPerWarp = (kRows + kWarps - 1) / kWarps;
+    uint8_t *mblk = sm + OFF_QR + 2 * kSBlk;          // block 2 of the stacked tile
     // all of this warp's rows are fetched first, so that their latencies overlap
     uint2 raws[kRowsPerWarp];
 #pragma unroll
@@ -257,6 +264,26 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
             raws[u] = __ldg(reinterpret_cast<const uint2 *>(qrow + 4 * lane));
         }
     }
+    // group sums of v (hi, lo) as elements g of chunks c0 and c0 + 1 of row `row` of block 2
+    auto sums = [&](const float v[4], int row, int c0) {
+        float gs = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+        if (NG < 8) {   // unused group columns are zero
+            if (lane == 0) {
+                st_shared16(mblk + tc::sw_chunk(row, c0), 0u, 0u, 0u, 0u);
+                st_shared16(mblk + tc::sw_chunk(row, c0 + 1), 0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+        if (lane % LPG == 0) {   // the group's first lane holds its sum
+            const int g = lane / LPG;
+            uint32_t hi, lo;
+            split_hi_lo(gs, hi, lo);
+            st_shared_u16(mblk + tc::sw_chunk(row, c0) + 2 * g, hi);
+            st_shared_u16(mblk + tc::sw_chunk(row, c0 + 1) + 2 * g, lo);
+        }
+    };
 #pragma unroll
     for (int u = 0; u < kRowsPerWarp; u++) {
         const int r = warp + u * kWarps;
@@ -268,30 +295,10 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
         x[2] = bf16_val(raw.y & 0xFFFFu);
         x[3] = bf16_val(raw.y >> 16);
         // elements 4 lane .. 4 lane + 3: block lane / 16, chunk (lane % 16) / 2, half (lane & 1)
-        const uint32_t off = (uint32_t)(lane >> 4) * kQBlk + tc::sw_chunk(r, (lane & 15) >> 1) + 8u * (lane & 1);
-        st_shared8(sm + OFF_Q + off, raw.x, raw.y);
-        // group sums (hi, lo) into columns 128 + g and 136 + g
-        auto sums = [&](const float v[4], uint8_t *tile) {
-            float gs = (v[0] + v[1]) + (v[2] + v[3]);
-#pragma unroll
-            for (int o = 1; o < LPG; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-            uint8_t *mrow = tile + 2 * kQBlk;
-            if (NG < 8) {   // unused group columns are zero
-                if (lane == 0) {
-                    st_shared16(mrow + tc::sw_chunk(r, 0), 0u, 0u, 0u, 0u);
-                    st_shared16(mrow + tc::sw_chunk(r, 1), 0u, 0u, 0u, 0u);
-                }
-                __syncwarp();
-            }
-            if (lane % LPG == 0) {   // the group's first lane holds its sum
-                const int g = lane / LPG;
-                uint32_t hi, lo;
-                split_hi_lo(gs, hi, lo);
-                st_shared_u16(mrow + tc::sw_chunk(r, 0) + 2 * g, hi);
-                st_shared_u16(mrow + tc::sw_chunk(r, 1) + 2 * g, lo);
-            }
-        };
-        sums(x, sm + OFF_Q);
+        const int ch = (lane & 15) >> 1;
+        const uint32_t in = 8u * (lane & 1);
+        st_shared8(sm + OFF_Q + (lane >> 4) * kQBlk + tc::sw_chunk(r, ch) + in, raw.x, raw.y);
+        sums(x, r, 2);
         if (RESID) {
             // R q = H diag(sigma) q / sqrt(d)
             float y[4];
@@ -305,9 +312,15 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) split_hi_lo(y[k], hi[k], lo[k]);
-            st_shared8(sm + OFF_QRH + off, hi[0] | hi[1] << 16, hi[2] | hi[3] << 16);
-            st_shared8(sm + OFF_QRL + off, lo[0] | lo[1] << 16, lo[2] | lo[3] << 16);
-            sums(y, sm + OFF_QRH);
+            const int rh = 32 * (r / 16) + r % 16, rl = rh + 16;   // stacked rows
+            uint8_t *blk = sm + OFF_QR + (lane >> 4) * kSBlk;
+            st_shared8(blk + tc::sw_chunk(rh, ch) + in, hi[0] | hi[1] << 16, hi[2] | hi[3] << 16);
+            st_shared8(blk + tc::sw_chunk(rl, ch) + in, lo[0] | lo[1] << 16, lo[2] | lo[3] << 16);
+            sums(y, rh, 0);
+            if (lane == 0) {
+                st_shared16(mblk + tc::sw_chunk(rl, 0), 0u, 0u, 0u, 0u);
+                st_shared16(mblk + tc::sw_chunk(rl, 1), 0u, 0u, 0u, 0u);
+            }
         }
     }
 }
@@ -375,12 +388,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
 
     if (warp < kSoftmaxWarps) {
         // ------------------------------------------------------- softmax
-        // Thread (w, i): row r = 16 w + (i mod 16) -- tensor-memory lane 32 w
-        // + (i mod 16) of the M = 64 layout -- and half hf = i / 16 of every
-        // range of columns it reads (the 16x32bx2 access: the upper 16
-        // threads read the same lanes at a column offset).
-        const int hf = lane >> 4;
-        const int r = 16 * warp + (lane & 15);
+        // Thread (w, i + 16 hf) owns query row r = 16 w + i and the tokens
+        // 16 hf .. 16 hf + 15 of each step.  SA (M = 64 layout: row r in
+        // lane 32 w + i) is read with the 16x32bx2 access, which gives each
+        // thread its own tokens; SY and the values (M = 128, stacked) hold
+        // row r's high part in lane 32 w + i and its low part in lane
+        // 32 w + 16 + i, i.e. thread hf = 0 reads the high, hf = 1 the low
+        // part, and the pair exchanges the halves of the other's tokens.
+        const int hf = lane >> 4, i16 = lane & 15;
+        const int r = 16 * warp + i16;
         const int iq = (r0 + r) / a.G;
         const int lim = min(Tb, Tb + a.n_tail - a.n + 1 + iq);   // committed tokens the row may see
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
@@ -398,22 +414,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             // logits buffer and the coefficient slot are released
             float s[kHalf], cv[kHalf];
             {
-                uint32_t va[16], vy[16];
                 const uint32_t cS = kColS + pb * 2 * kTok;
-                tc::ld16x2<kHalf>(tl + cS, va);
+                uint32_t sa[16];
+                tc::ld16x2<kHalf>(tl + cS, sa);
                 if (RESID) {
-                    tc::ld16x2<kHalf>(tl + cS + kTok, vy);
-                    tc::wait_ld2(va, vy);
+                    uint32_t y0[16], y1[16];
+                    tc::ld16(tl + cS + kTok, y0);        // this lane's part of SY, tokens 0..15
+                    tc::ld16(tl + cS + kTok + 16, y1);   // tokens 16..31
+                    tc::wait_ld3(sa, y0, y1);
+#pragma unroll
+                    for (int k = 0; k < kHalf; k++) {
+                        const float own = __uint_as_float(hf ? y1[k] : y0[k]);
+                        const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(hf ? y0[k] : y1[k]), 16);
+                        s[k] = fmaf(s_cK[cs][kHalf * hf + k], __uint_as_float(sa[k]), own + other) * a.scale_log2;
+                    }
                 } else {
-                    tc::wait_ld(va);
+                    tc::wait_ld(sa);
+#pragma unroll
+                    for (int k = 0; k < kHalf; k++) s[k] = __uint_as_float(sa[k]) * a.scale_log2;
                 }
 #pragma unroll
-                for (int k = 0; k < kHalf; k++) {
-                    const float sa = __uint_as_float(va[k]);
-                    const float x = RESID ? fmaf(s_cK[cs][kHalf * hf + k], sa, __uint_as_float(vy[k])) : sa;
-                    s[k] = x * a.scale_log2;
-                    cv[k] = RESID ? s_cV[cs][kHalf * hf + k] : 1.f;
-                }
+                for (int k = 0; k < kHalf; k++) cv[k] = RESID ? s_cV[cs][kHalf * hf + k] : 1.f;
             }
             tc::fence_before();
             mbar_arrive(&bar_sfree[pb]);
@@ -436,45 +457,46 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 // O must be final: the values of step j - 1 complete
                 if (j >= 1) wait(&bar_odone[pb ^ 1], ((j - 1) >> 1) & 1, 23);
                 tc::fence_after();
-                // this row's accumulated values times f (rows without a raise
-                // times 1); the two threads of a row take columns c and c + 64
+                // this lane's part (high or low) of the row's accumulated
+                // values times f (rows without a raise times 1)
 #pragma unroll 1
-                for (int c = 0; c < kHeadDim / 2; c += 16) {
+                for (int c = 0; c < kHeadDim; c += 16) {
                     uint32_t v[16];
-                    tc::ld16x2<kHeadDim / 2>(tl + kColOA + c, v);
+                    tc::ld16(tl + kColOA + c, v);
                     tc::wait_ld(v);
 #pragma unroll
                     for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
-                    tc::st16x2<kHeadDim / 2>(tl + kColOA + c, v);
+                    tc::st16(tl + kColOA + c, v);
                     if (RESID) {
-                        tc::ld16x2<kHeadDim / 2>(tl + kColOY + c, v);
+                        tc::ld16(tl + kColOY + c, v);
                         tc::wait_ld(v);
 #pragma unroll
                         for (int k = 0; k < 16; k++) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
-                        tc::st16x2<kHeadDim / 2>(tl + kColOY + c, v);
+                        tc::st16(tl + kColOY + c, v);
                     }
                 }
-                // the minimum columns (the upper threads' 8 columns after them are unused)
                 uint32_t v8[8];
-                tc::ld8x2<8>(tl + kColOA + kHeadDim, v8);
+                tc::ld8(tl + kColOA + kHeadDim, v8);
                 tc::wait_ld8(v8);
 #pragma unroll
                 for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
-                tc::st8x2<8>(tl + kColOA + kHeadDim, v8);
+                tc::st8(tl + kColOA + kHeadDim, v8);
                 if (RESID) {
-                    tc::ld8x2<8>(tl + kColOY + kHeadDim, v8);
+                    tc::ld8(tl + kColOY + kHeadDim, v8);
                     tc::wait_ld8(v8);
 #pragma unroll
                     for (int k = 0; k < 8; k++) v8[k] = __float_as_uint(__uint_as_float(v8[k]) * f);
-                    tc::st8x2<8>(tl + kColOY + kHeadDim, v8);
+                    tc::st8(tl + kColOY + kHeadDim, v8);
                 }
                 tc::wait_st();
             }
             l *= f;
-            // probabilities of the step, split hi / lo, into the A operands
-            // (K = the step's 32 tokens: the first 64 bytes of each 128-byte row)
+            // probabilities of the step, split hi / lo, into the stacked A
+            // operands (K = the step's 32 tokens: the first 64 bytes of each
+            // 128-byte row)
             const float mu = m_used == -CUDART_INF_F ? 0.f : m_used;
             uint8_t *prow = sm + OFF_P + pb * kPBytes;
+            const int rh = 32 * warp + i16, rl = rh + 16;
 #pragma unroll
             for (int cc = 0; cc < kHalf / 8; cc++) {
                 uint32_t psh[4], psl[4], ph[4], pl[4];
@@ -490,12 +512,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                         split_hi_lo2(p0, p1, psh[k / 2], psl[k / 2]);
                     }
                 }
-                const uint32_t o = tc::sw_chunk(r, (kHalf / 8) * hf + cc);
-                st_shared16(prow + o, psh[0], psh[1], psh[2], psh[3]);
-                st_shared16(prow + kQBlk + o, psl[0], psl[1], psl[2], psl[3]);
+                const int c = (kHalf / 8) * hf + cc;
+                st_shared16(prow + tc::sw_chunk(rh, c), psh[0], psh[1], psh[2], psh[3]);
+                st_shared16(prow + tc::sw_chunk(rl, c), psl[0], psl[1], psl[2], psl[3]);
                 if (RESID) {
-                    st_shared16(prow + 2 * kQBlk + o, ph[0], ph[1], ph[2], ph[3]);
-                    st_shared16(prow + 3 * kQBlk + o, pl[0], pl[1], pl[2], pl[3]);
+                    st_shared16(prow + kSBlk + tc::sw_chunk(rh, c), ph[0], ph[1], ph[2], ph[3]);
+                    st_shared16(prow + kSBlk + tc::sw_chunk(rl, c), pl[0], pl[1], pl[2], pl[3]);
                 }
             }
             tc::fence_async_smem();
@@ -504,10 +526,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         }
         l += __shfl_xor_sync(0xffffffffu, l, 16);   // the row's sum
         // ------------------------------------------------------- epilogue
-        // Each row's A and Y, plus their group minima, go to shared memory
-        // (the K and V tiles are free once the last values completed); then a
-        // warp per row applies R^T to Y with the in-warp transform and writes
-        // the partial, 4 consecutive elements per lane.
+        // Each row's A and Y (high + low parts, plus their group minima) go
+        // to shared memory (the K and V tiles are free once the last values
+        // completed); then a warp per row applies R^T to Y with the in-warp
+        // transform and writes the partial, 4 consecutive elements per lane.
         constexpr int kEStride = kHeadDim + 4;   // padded rows: the row-per-thread stores do not conflict
         static_assert(kRows * kEStride * 4 <= 2 * kKVBytes, "staging fits in the K (and the V) tiles");
         float *sA = reinterpret_cast<float *>(sm + OFF_K);
@@ -519,25 +541,32 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
 #pragma unroll
             for (int side = 0; side < (RESID ? 2 : 1); side++) {
                 const uint32_t col = side == 0 ? kColOA : kColOY;
-                float *dst = (side == 0 ? sA : sY) + r * kEStride + (kHeadDim / 2) * hf;
-                // the row's group minima (read by the lower thread of the pair)
+                float *dst = (side == 0 ? sA : sY) + r * kEStride + 8 * hf;
+                // the row's group minima: high + low lane
                 uint32_t m8[8];
-                tc::ld8x2<8>(tl + col + kHeadDim, m8);
+                tc::ld8(tl + col + kHeadDim, m8);
                 tc::wait_ld8(m8);
+                float mn8[8];
 #pragma unroll
-                for (int k = 0; k < 8; k++) m8[k] = __shfl_sync(0xffffffffu, m8[k], lane & 15);
+                for (int k = 0; k < 8; k++)
+                    mn8[k] = __uint_as_float(m8[k]) + __shfl_xor_sync(0xffffffffu, __uint_as_float(m8[k]), 16);
 #pragma unroll
-                for (int c = 0; c < kHeadDim / 2; c += 16) {
+                for (int c = 0; c < kHeadDim; c += 16) {
                     uint32_t v[16];
-                    tc::ld16x2<kHeadDim / 2>(tl + col + c, v);
+                    tc::ld16(tl + col + c, v);
                     tc::wait_ld(v);
-                    // a 16-column chunk lies in one group
-                    const float mn = __uint_as_float(hf ? m8[(kHeadDim / 2 + c) / GS] : m8[c / GS]);
+                    float w[16];
 #pragma unroll
-                    for (int k = 0; k < 16; k += 4)
-                        *reinterpret_cast<float4 *>(dst + c + k) =
-                            make_float4(__uint_as_float(v[k]) + mn, __uint_as_float(v[k + 1]) + mn,
-                                        __uint_as_float(v[k + 2]) + mn, __uint_as_float(v[k + 3]) + mn);
+                    for (int k = 0; k < 16; k++)
+                        w[k] = __uint_as_float(v[k]) + __shfl_xor_sync(0xffffffffu, __uint_as_float(v[k]), 16);
+                    // a 16-column chunk lies in one group; thread hf stores its 8 columns
+                    const float mn = mn8[c / GS];
+#pragma unroll
+                    for (int k = 0; k < 8; k += 4) {
+                        const float a0 = hf ? w[8 + k] : w[k], a1 = hf ? w[9 + k] : w[k + 1];
+                        const float a2 = hf ? w[10 + k] : w[k + 2], a3 = hf ? w[11 + k] : w[k + 3];
+                        *reinterpret_cast<float4 *>(dst + c + k) = make_float4(a0 + mn, a1 + mn, a2 + mn, a3 + mn);
+                    }
                 }
             }
         }
@@ -584,26 +613,27 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         // One thread; the logits of the next steps and the values of the
         // current one are issued in whichever order their operands are ready.
         if (lane == 0) {
-            constexpr uint32_t idL = tc::idesc_bf16(kRows, kTok, false);
-            constexpr uint32_t idP = tc::idesc_bf16(kRows, kOCols, true);
+            constexpr uint32_t idA = tc::idesc_bf16(kRows, kTok, false);          // SA: q (M = 64)
+            constexpr uint32_t idY = tc::idesc_bf16(2 * kRows, kTok, false);      // SY: stacked Rq (M = 128)
+            constexpr uint32_t idV = tc::idesc_bf16(2 * kRows, kOCols, true);     // OA, OY: stacked p (M = 128)
             // descriptors of the operand tiles; the start address advances in
             // 16-byte units (32 bytes per K step inside a block, a block across)
-            const uint64_t dQ = tc::desc_k(sbase + OFF_Q), dQRH = tc::desc_k(sbase + OFF_QRH),
-                           dQRL = tc::desc_k(sbase + OFF_QRL), dK = tc::desc_k(sbase + OFF_K),
+            const uint64_t dQ = tc::desc_k(sbase + OFF_Q), dQm = tc::desc_k(sbase + OFF_QR + 2 * kSBlk + 32),
+                           dR = tc::desc_k(sbase + OFF_QR), dK = tc::desc_k(sbase + OFF_K),
                            dP = tc::desc_k(sbase + OFF_P), dV = tc::desc_mn(sbase + OFF_V, kTBlk);
             auto kq = [](int kk) { return (uint64_t)(((kk >> 2) * kQBlk + (kk & 3) * 32) >> 4); };
+            auto ks = [](int kk) { return (uint64_t)(((kk >> 2) * kSBlk + (kk & 3) * 32) >> 4); };
             auto kt = [](int kk) { return (uint64_t)(((kk >> 2) * kTBlk + (kk & 3) * 32) >> 4); };
             auto logits = [&](int j) {
                 const uint64_t ka = dK + (uint64_t)(((j & 1) * kKVBytes) >> 4);
                 const uint64_t ky = ka + (uint64_t)((3 * kTBlk) >> 4);
                 const uint32_t cS = tmem + kColS + (j & 1) * 2 * kTok;
 #pragma unroll
-                for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idL, kk > 0);
+                for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idA, kk > 0);
+                tc::mma_bf16(cS, dQm, ka + kt(8), idA, true);   // the group sums of q against the minima
                 if (RESID) {
 #pragma unroll
-                    for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS + kTok, dQRH + kq(kk), ky + kt(kk), idL, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS + kTok, dQRL + kq(kk), ky + kt(kk), idL, true);
+                    for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS + kTok, dR + ks(kk), ky + kt(kk), idY, kk > 0);
                 }
                 tc::commit(&bar_kdone[j & 1]);
             };
@@ -612,17 +642,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 const uint64_t va = dV + (uint64_t)(((j & 1) * kKVBytes) >> 4);
                 const uint64_t vy = va + (uint64_t)((3 * kTBlk) >> 4);
 #pragma unroll
-                for (int part = 0; part < 2; part++) {
+                for (int kk = 0; kk < kTok / 16; kk++)
+                    tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((kk * 32) >> 4),
+                                 va + (uint64_t)((kk * 16 * 128) >> 4), idV, j > 0 || kk > 0);
+                if (RESID) {
 #pragma unroll
                     for (int kk = 0; kk < kTok / 16; kk++)
-                        tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((part * kQBlk + kk * 32) >> 4),
-                                     va + (uint64_t)((kk * 16 * 128) >> 4), idP, j > 0 || part > 0 || kk > 0);
-                    if (RESID) {
-#pragma unroll
-                        for (int kk = 0; kk < kTok / 16; kk++)
-                            tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)(((2 + part) * kQBlk + kk * 32) >> 4),
-                                         vy + (uint64_t)((kk * 16 * 128) >> 4), idP, j > 0 || part > 0 || kk > 0);
-                    }
+                        tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)((kSBlk + kk * 32) >> 4),
+                                     vy + (uint64_t)((kk * 16 * 128) >> 4), idV, j > 0 || kk > 0);
                 }
                 tc::commit(&bar_odone[j & 1]);
             };

@@ -169,6 +169,10 @@ __device__ __forceinline__ void wait_ld2(uint32_t (&v)[16], uint32_t (&w)[16]) {
                  :
                  : "memory");
 }
+__device__ __forceinline__ void wait_ld3(uint32_t (&u)[16], uint32_t (&v)[16], uint32_t (&w)[16]) {
+    wait_ld2(u, v);
+    wait_ld(w);
+}
 __device__ __forceinline__ void wait_ld8(uint32_t (&v)[8]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7])
