@@ -33,12 +33,14 @@
 // a second kernel that merges the splits and the tail tokens (combine_row).
 //
 // CTA = (split of the committed tokens, kv head, sequence x block of 64 query
-// rows); 13 warps:
+// rows); 14 warps:
 //  - warps 0-3: softmax -- warp w owns tensor-memory lanes 32w.. and query
 //    rows 16w..16w+15 (the M=64 accumulator layout); loads the logits,
 //    writes the probability operands, rescales, and at the end reads OA and
 //    OY, applies R^T and writes the partial;
-//  - warp 4: allocates tensor memory; one thread issues every MMA;
+//  - warps 4 and 13: one thread each issues the MMAs of the anchor side
+//    (SA, OA) and of the residual side (SY, OY); warp 4 allocates tensor
+//    memory;
 //  - warps 5-12: dequantize the step's K and V records (straight from global
 //    memory) into the swizzled operand tiles.
 // Hand-offs go through mbarriers, every wait bounded (error word, abort flag):
@@ -64,10 +66,12 @@ namespace {
 constexpr int kRows = 64;             // query rows of a CTA (M of every MMA)
 constexpr int kTok = kPrefillTile;    // committed tokens per step (N of the logits, K of the values)
 constexpr int kSoftmaxWarps = 4;
-constexpr int kMmaWarp = 4;
+constexpr int kMmaWarp = 4;            // issues the anchor-side MMAs (SA, OA); allocates tensor memory
+constexpr int kMmaWarpY = 13;          // issues the residual-side MMAs (SY, OY)
 constexpr int kDeqWarps = 8;
 constexpr int kDeqThreads = 32 * kDeqWarps;
-constexpr int kThreadsP = 32 * (kSoftmaxWarps + 1 + kDeqWarps);
+constexpr int kThreadsP = 32 * (kSoftmaxWarps + 2 + kDeqWarps);
+static_assert(kMmaWarpY == kSoftmaxWarps + 1 + kDeqWarps, "the second MMA warp follows the dequantizing warps");
 constexpr int kQBlk = kRows * 128;    // a 64-row block of 64 bf16 columns (8 KB): q
 constexpr int kSBlk = 2 * kQBlk;      // a 128-row block (16 KB): stacked high / low operands (M = 128)
 constexpr int kTBlk = kTok * 128;     // a block of the step's token rows (4 KB): key / value operands
@@ -357,10 +361,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         for (int i = 0; i < 2; i++) {
             mbar_init(&bar_kfull[i], kDeqThreads / 2);
             mbar_init(&bar_vfull[i], kDeqThreads / 2);
-            mbar_init(&bar_kdone[i], 1);
+            mbar_init(&bar_kdone[i], RESID ? 2 : 1);   // one commit per MMA-issuing thread
             mbar_init(&bar_sfree[i], 32 * kSoftmaxWarps);
             mbar_init(&bar_pfull[i], 32 * kSoftmaxWarps);
-            mbar_init(&bar_odone[i], 1);
+            mbar_init(&bar_odone[i], RESID ? 2 : 1);
         }
         for (int i = 0; i < 4; i++) mbar_init(&bar_cfull[i], kTok);
         s_abort = 0;
@@ -608,11 +612,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 part[kHeadDim + 1] = ntl > 0 ? s_ml[row][1] : 0.f;
             }
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kMmaWarpY) {
         // ------------------------------------------------------- MMA issue
-        // One thread; the logits of the next steps and the values of the
+        // Two threads, in different warps (one thread issues a tcgen05.mma
+        // every ~57 cycles at best; two reach the shared-memory bandwidth of
+        // the operands): the anchor side (SA, OA) and the residual side (SY,
+        // OY, residual loops only).  Each commits to kdone / odone, which
+        // count both.  The logits of the next steps and the values of the
         // current one are issued in whichever order their operands are ready.
-        if (lane == 0) {
+        const bool yside = warp == kMmaWarpY;
+        if (lane == 0 && (RESID || !yside)) {
             constexpr uint32_t idA = tc::idesc_bf16(kRows, kTok, false);          // SA: q (M = 64)
             constexpr uint32_t idY = tc::idesc_bf16(2 * kRows, kTok, false);      // SY: stacked Rq (M = 128)
             constexpr uint32_t idV = tc::idesc_bf16(2 * kRows, kOCols, true);     // OA, OY: stacked p (M = 128)
@@ -628,29 +637,24 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 const uint64_t ka = dK + (uint64_t)(((j & 1) * kKVBytes) >> 4);
                 const uint64_t ky = ka + (uint64_t)((3 * kTBlk) >> 4);
                 const uint32_t cS = tmem + kColS + (j & 1) * 2 * kTok;
+                if (!yside) {
 #pragma unroll
-                for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idA, kk > 0);
-                tc::mma_bf16(cS, dQm, ka + kt(8), idA, true);   // the group sums of q against the minima
-                if (RESID) {
+                    for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idA, kk > 0);
+                    tc::mma_bf16(cS, dQm, ka + kt(8), idA, true);   // the group sums of q against the minima
+                } else {
 #pragma unroll
                     for (int kk = 0; kk < 9; kk++) tc::mma_bf16(cS + kTok, dR + ks(kk), ky + kt(kk), idY, kk > 0);
                 }
                 tc::commit(&bar_kdone[j & 1]);
             };
             auto values = [&](int j) {
-                const uint64_t pbuf = dP + (uint64_t)(((j & 1) * kPBytes) >> 4);
-                const uint64_t va = dV + (uint64_t)(((j & 1) * kKVBytes) >> 4);
-                const uint64_t vy = va + (uint64_t)((3 * kTBlk) >> 4);
+                const uint64_t pbuf = dP + (uint64_t)(((j & 1) * kPBytes + (yside ? kSBlk : 0)) >> 4);
+                const uint64_t vv = dV + (uint64_t)(((j & 1) * kKVBytes + (yside ? 3 * kTBlk : 0)) >> 4);
+                const uint32_t cO = tmem + (yside ? kColOY : kColOA);
 #pragma unroll
                 for (int kk = 0; kk < kTok / 16; kk++)
-                    tc::mma_bf16(tmem + kColOA, pbuf + (uint64_t)((kk * 32) >> 4),
-                                 va + (uint64_t)((kk * 16 * 128) >> 4), idV, j > 0 || kk > 0);
-                if (RESID) {
-#pragma unroll
-                    for (int kk = 0; kk < kTok / 16; kk++)
-                        tc::mma_bf16(tmem + kColOY, pbuf + (uint64_t)((kSBlk + kk * 32) >> 4),
-                                     vy + (uint64_t)((kk * 16 * 128) >> 4), idV, j > 0 || kk > 0);
-                }
+                    tc::mma_bf16(cO, pbuf + (uint64_t)((kk * 32) >> 4), vv + (uint64_t)((kk * 16 * 128) >> 4), idV,
+                                 j > 0 || kk > 0);
                 tc::commit(&bar_odone[j & 1]);
             };
             int nl = 0, nv = 0;   // steps whose logits / values are issued
