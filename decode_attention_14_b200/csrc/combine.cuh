@@ -12,29 +12,17 @@
 
 namespace rq {
 
-// Run by 128 threads (thread `tid` owns element tid of the row).  `sync` is a
-// barrier over exactly those threads; `red` is 4 floats of shared memory.
-// `part` points at slot 0 of this row's partials (stride kPartialStride); it
-// is read with L1-bypassing loads because other CTAs wrote it.
-template <typename Sync>
-__device__ __forceinline__ void combine_row(const float *part, int S, const uint16_t *q_row, float scale_log2,
-                                            const uint16_t *tail_k, const uint16_t *tail_v, size_t tail_stride,
-                                            int n_tail, float *out_row, int tid, float *red, Sync sync) {
-    const int lane = tid & 31, warp = tid >> 5;
-    // q and the first tail token are fetched first, so that their latency
-    // overlaps the partials' (L2 loads: the tail rows may have been written
-    // during this kernel by another CTA)
-    float q = 0.f, k0 = 0.f, v0 = 0.f;
-    if (n_tail > 0) {
-        q = bf16_to_f32(q_row[tid]) * scale_log2;
-        k0 = bf16_to_f32(__ldcg(tail_k + tid));
-        v0 = bf16_to_f32(__ldcg(tail_v + tid));
-    }
-    // partials, kBatch splits per round of loads (one round for up to kBatch
-    // splits): the batch's maximum, the running sums rescaled to it, then the
-    // batch folded in (a split with no key has m = -inf: weight 0)
+// The split partials of a row merged into (M, l, o) for element tid:
+// kBatch splits per round of loads (one round for up to kBatch splits), the
+// batch's maximum, the running sums rescaled to it, then the batch folded in
+// (a split with no key has m = -inf: weight 0).  `part` points at slot 0 of
+// the row's partials (stride kPartialStride); it is read with L1-bypassing
+// loads because other CTAs wrote it.
+__device__ __forceinline__ void merge_partials(const float *part, int S, int tid, float &M, float &l, float &o) {
     constexpr int kBatch = 16;
-    float M = -CUDART_INF_F, l = 0.f, o = 0.f;
+    M = -CUDART_INF_F;
+    l = 0.f;
+    o = 0.f;
     for (int s0 = 0; s0 < S; s0 += kBatch) {
         float m[kBatch], ls[kBatch], os[kBatch];
 #pragma unroll
@@ -60,6 +48,26 @@ __device__ __forceinline__ void combine_row(const float *part, int S, const uint
         }
         M = Mn;
     }
+}
+
+// Run by 128 threads (thread `tid` owns element tid of the row).  `sync` is a
+// barrier over exactly those threads; `red` is 4 floats of shared memory.
+template <typename Sync>
+__device__ __forceinline__ void combine_row(const float *part, int S, const uint16_t *q_row, float scale_log2,
+                                            const uint16_t *tail_k, const uint16_t *tail_v, size_t tail_stride,
+                                            int n_tail, float *out_row, int tid, float *red, Sync sync) {
+    const int lane = tid & 31, warp = tid >> 5;
+    // q and the first tail token are fetched first, so that their latency
+    // overlaps the partials' (L2 loads: the tail rows may have been written
+    // during this kernel by another CTA)
+    float q = 0.f, k0 = 0.f, v0 = 0.f;
+    if (n_tail > 0) {
+        q = bf16_to_f32(q_row[tid]) * scale_log2;
+        k0 = bf16_to_f32(__ldcg(tail_k + tid));
+        v0 = bf16_to_f32(__ldcg(tail_v + tid));
+    }
+    float M, l, o;
+    merge_partials(part, S, tid, M, l, o);
     // tail tokens, folded in one by one with the running-max rule
     for (int j = 0; j < n_tail; j++) {
         const size_t row = (size_t)j * tail_stride;

@@ -48,4 +48,33 @@ __device__ __forceinline__ void wht128_warp(T v[4], int lane) {
     }
 }
 
+// The transform of two 128-vectors at once (independent shuffle chains
+// interleaved).
+template <typename T>
+__device__ __forceinline__ void wht128_warp2(T u[4], T v[4], int lane) {
+    {
+        T a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+        u[0] = a0 + a2;
+        u[2] = a0 - a2;
+        u[1] = a1 + a3;
+        u[3] = a1 - a3;
+        T b0 = v[0] + v[1], b1 = v[0] - v[1], b2 = v[2] + v[3], b3 = v[2] - v[3];
+        v[0] = b0 + b2;
+        v[2] = b0 - b2;
+        v[1] = b1 + b3;
+        v[3] = b1 - b3;
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const T ou = __shfl_xor_sync(0xffffffffu, u[k], m);
+            const T ov = __shfl_xor_sync(0xffffffffu, v[k], m);
+            u[k] = upper ? (ou - u[k]) : (u[k] + ou);
+            v[k] = upper ? (ov - v[k]) : (v[k] + ov);
+        }
+    }
+}
+
 }  // namespace rq

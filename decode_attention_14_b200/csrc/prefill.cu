@@ -30,7 +30,7 @@
 // with logits scale_log2 (s SA + SY) and a running maximum that is only
 // raised when a row's maximum grows by more than 2^8 (then that row of OA and
 // OY is rescaled in tensor memory); the partial (m, l, o) of each row goes to
-// a second kernel that merges the splits and the tail tokens (combine_row).
+// a second kernel that merges the splits and the tail tokens.
 //
 // CTA = (split of the committed tokens, kv head, sequence x block of 64 query
 // rows); 14 warps:
@@ -117,6 +117,12 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float x0, float x1) {
 __device__ __forceinline__ void split_hi_lo2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
     hi = bf16x2_rn(x0, x1);
     lo = bf16x2_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+}
+// 2^x on the multi-function unit (relative error ~2^-22; 0 for x = -inf)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
     __shared__ uint64_t bar_cfull[4];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_cK[4][kTok], s_cV[4][kTok];   // coefficients of a step (1 at an anchor loop)
+    __shared__ __align__(16) float s_cK[4][kTok], s_cV[4][kTok];   // coefficients of a step (1 at an anchor loop)
     __shared__ float s_ml[kRows][2];                  // running maximum and sum of each row
 
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -426,30 +432,55 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                     tc::ld16(tl + cS + kTok, y0);        // this lane's part of SY, tokens 0..15
                     tc::ld16(tl + cS + kTok + 16, y1);   // tokens 16..31
                     tc::wait_ld3(sa, y0, y1);
+                    float ck[kHalf];
+                    const float4 *c4 = reinterpret_cast<const float4 *>(&s_cK[cs][kHalf * hf]);
+#pragma unroll
+                    for (int k = 0; k < kHalf; k += 4) {
+                        const float4 v = c4[k / 4];
+                        ck[k] = v.x;
+                        ck[k + 1] = v.y;
+                        ck[k + 2] = v.z;
+                        ck[k + 3] = v.w;
+                    }
 #pragma unroll
                     for (int k = 0; k < kHalf; k++) {
                         const float own = __uint_as_float(hf ? y1[k] : y0[k]);
                         const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(hf ? y0[k] : y1[k]), 16);
-                        s[k] = fmaf(s_cK[cs][kHalf * hf + k], __uint_as_float(sa[k]), own + other) * a.scale_log2;
+                        s[k] = fmaf(ck[k], __uint_as_float(sa[k]), own + other) * a.scale_log2;
                     }
                 } else {
                     tc::wait_ld(sa);
 #pragma unroll
                     for (int k = 0; k < kHalf; k++) s[k] = __uint_as_float(sa[k]) * a.scale_log2;
                 }
+                if (RESID) {
+                    const float4 *c4 = reinterpret_cast<const float4 *>(&s_cV[cs][kHalf * hf]);
 #pragma unroll
-                for (int k = 0; k < kHalf; k++) cv[k] = RESID ? s_cV[cs][kHalf * hf + k] : 1.f;
+                    for (int k = 0; k < kHalf; k += 4) {
+                        const float4 v = c4[k / 4];
+                        cv[k] = v.x;
+                        cv[k + 1] = v.y;
+                        cv[k + 2] = v.z;
+                        cv[k + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kHalf; k++) cv[k] = 1.f;
+                }
             }
             tc::fence_before();
             mbar_arrive(&bar_sfree[pb]);
             float mx = -CUDART_INF_F;
+            if (tn < kTok || t0 + tt + kTok > lim) {   // the step's end is not visible to the row
 #pragma unroll
-            for (int k = 0; k < kHalf; k++) {
-                const int t = kHalf * hf + k;
-                const bool ok = t < tn && t0 + tt + t < lim;
-                s[k] = ok ? s[k] : -CUDART_INF_F;
-                mx = fmaxf(mx, s[k]);
+                for (int k = 0; k < kHalf; k++) {
+                    const int t = kHalf * hf + k;
+                    const bool ok = t < tn && t0 + tt + t < lim;
+                    s[k] = ok ? s[k] : -CUDART_INF_F;
+                }
             }
+#pragma unroll
+            for (int k = 0; k < kHalf; k++) mx = fmaxf(mx, s[k]);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));   // the row's maximum
             const bool raise = mx > m_used + kRescaleLog2;   // false while nothing is seen (both -inf)
             const bool rescale = raise && m_used != -CUDART_INF_F;
@@ -507,7 +538,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
 #pragma unroll
                 for (int k = 0; k < 8; k += 2) {
                     const int u = 8 * cc + k;
-                    const float p0 = exp2f(s[u] - mu), p1 = exp2f(s[u + 1] - mu);   // 0 if masked
+                    const float p0 = ex2(s[u] - mu), p1 = ex2(s[u + 1] - mu);   // 0 if masked
                     l += p0 + p1;
                     if (RESID) {
                         split_hi_lo2(p0 * cv[u], p1 * cv[u + 1], psh[k / 2], psl[k / 2]);
@@ -532,8 +563,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         // ------------------------------------------------------- epilogue
         // Each row's A and Y (high + low parts, plus their group minima) go
         // to shared memory (the K and V tiles are free once the last values
-        // completed); then a warp per row applies R^T to Y with the in-warp
-        // transform and writes the partial, 4 consecutive elements per lane.
+        // completed), with the row's running maximum and sum.
         constexpr int kEStride = kHeadDim + 4;   // padded rows: the row-per-thread stores do not conflict
         static_assert(kRows * kEStride * 4 <= 2 * kKVBytes, "staging fits in the K (and the V) tiles");
         float *sA = reinterpret_cast<float *>(sm + OFF_K);
@@ -577,40 +607,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         if (hf == 0) {
             s_ml[r][0] = m_used;
             s_ml[r][1] = l;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
-        for (int rr = 0; rr < 16; rr++) {
-            const int row = 16 * warp + rr;
-            if (row >= nr) break;
-            float o[4] = {0.f, 0.f, 0.f, 0.f};
-            if (ntl > 0) {
-                if (RESID) {
-                    // R^T Y = diag(sigma) H Y / sqrt(d)
-                    const float4 y = *reinterpret_cast<const float4 *>(sY + row * kEStride + 4 * lane);
-                    o[0] = y.x;
-                    o[1] = y.y;
-                    o[2] = y.z;
-                    o[3] = y.w;
-                    if (a.rotate) {
-                        wht128_warp<float>(o, lane);
-#pragma unroll
-                        for (int k = 0; k < 4; k++) o[k] *= sigma_neg(a.sigma, 4 * lane + k) ? -kInvSqrtD : kInvSqrtD;
-                    }
-                }
-                const float4 x = *reinterpret_cast<const float4 *>(sA + row * kEStride + 4 * lane);
-                o[0] += x.x;
-                o[1] += x.y;
-                o[2] += x.z;
-                o[3] += x.w;
-            }
-            const int rg = r0 + row, i = rg / a.G, gq = rg % a.G;
-            const size_t prow = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
-            float *part = a.partials + (prow * a.S + split) * kPartialStride;
-            *reinterpret_cast<float4 *>(part + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-            if (lane == 0) {
-                part[kHeadDim] = ntl > 0 ? s_ml[row][0] : -CUDART_INF_F;
-                part[kHeadDim + 1] = ntl > 0 ? s_ml[row][1] : 0.f;
-            }
         }
     } else if (warp == kMmaWarp || warp == kMmaWarpY) {
         // ------------------------------------------------------- MMA issue
@@ -743,32 +739,129 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         }
     }
 
+    // ------------------------------------------------------- partials
+    // Every warp takes rows of the staged A and Y (warp w: rows w, w + 14,
+    // ...; two rows at a time, so that their transforms overlap), applies
+    // R^T to Y with the in-warp transform and writes the row's partial
+    // (m, l, o), 4 consecutive elements per lane.
     tc::fence_before();
     __syncthreads();
+    {
+        constexpr int kEStride = kHeadDim + 4;
+        const float *sA = reinterpret_cast<const float *>(sm + OFF_K);
+        const float *sY = reinterpret_cast<const float *>(sm + OFF_V);
+        constexpr int kWarps = kThreadsP / 32;
+        for (int row0 = warp; row0 < nr; row0 += 2 * kWarps) {
+            float o[2][4];
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const int row = min(row0 + u * kWarps, kRows - 1);   // a row past nr is computed, not written
+#pragma unroll
+                for (int k = 0; k < 4; k++) o[u][k] = 0.f;
+                if (ntl > 0 && RESID) {
+                    const float4 y = *reinterpret_cast<const float4 *>(sY + row * kEStride + 4 * lane);
+                    o[u][0] = y.x;
+                    o[u][1] = y.y;
+                    o[u][2] = y.z;
+                    o[u][3] = y.w;
+                }
+            }
+            if (ntl > 0 && RESID && a.rotate) {
+                // R^T Y = diag(sigma) H Y / sqrt(d)
+                wht128_warp2<float>(o[0], o[1], lane);
+#pragma unroll
+                for (int u = 0; u < 2; u++)
+#pragma unroll
+                    for (int k = 0; k < 4; k++) o[u][k] *= sigma_neg(a.sigma, 4 * lane + k) ? -kInvSqrtD : kInvSqrtD;
+            }
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const int row = row0 + u * kWarps;
+                if (row >= nr) break;
+                if (ntl > 0) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sA + row * kEStride + 4 * lane);
+                    o[u][0] += x.x;
+                    o[u][1] += x.y;
+                    o[u][2] += x.z;
+                    o[u][3] += x.w;
+                }
+                const int rg = r0 + row, i = rg / a.G, gq = rg % a.G;
+                const size_t prow = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
+                float *part = a.partials + (prow * a.S + split) * kPartialStride;
+                *reinterpret_cast<float4 *>(part + 4 * lane) = make_float4(o[u][0], o[u][1], o[u][2], o[u][3]);
+                if (lane == 0) {
+                    part[kHeadDim] = ntl > 0 ? s_ml[row][0] : -CUDART_INF_F;
+                    part[kHeadDim + 1] = ntl > 0 ? s_ml[row][1] : 0.f;
+                }
+            }
+        }
+    }
     if (warp == kMmaWarp) {
         tc::fence_after();
         tc::dealloc(tmem, kTmemCols);
     }
 }
 
-struct Sync128 {
-    __device__ __forceinline__ void operator()() const { __syncthreads(); }
-};
-
-// One CTA per (q head, query token, sequence): the row's partials, then the
-// tail tokens it may see.
+// One CTA per (q head, query token, sequence): the row's split partials,
+// then the tail tokens it may see, 128 at a time: their logits (a warp per
+// token, 4 elements per lane), the chunk's maximum, then o += sum 2^(z - M) v
+// with thread tid owning element tid.
 __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs a) {
+    constexpr int kChunk = 128;
+    __shared__ float s_z[kChunk];
     __shared__ float s_red[4];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hq = blockIdx.x, i = blockIdx.y, b = blockIdx.z;
     const int h = hq / a.G;
     const size_t row = ((size_t)b * a.n + i) * a.Hq + hq;
     // of [committed, tail] the row sees T_b + n_tail - n + 1 + i tokens: all
     // committed ones when the new tokens are in the tail
     const int nt = a.tail_k ? max(0, a.n_tail - a.n + 1 + i) : 0;
-    const size_t trow = ((size_t)b * a.tail_cap * a.H + h) * kHeadDim;
-    combine_row(a.partials + row * a.S * kPartialStride, a.S, a.q + row * kHeadDim, a.scale_log2,
-                a.tail_k ? a.tail_k + trow : nullptr, a.tail_v ? a.tail_v + trow : nullptr,
-                (size_t)a.H * kHeadDim, nt, a.out + row * kHeadDim, threadIdx.x, s_red, Sync128());
+    const size_t tstride = (size_t)a.H * kHeadDim;
+    const uint16_t *tk = a.tail_k ? a.tail_k + ((size_t)b * a.tail_cap * a.H + h) * kHeadDim : nullptr;
+    const uint16_t *tv = a.tail_v ? a.tail_v + ((size_t)b * a.tail_cap * a.H + h) * kHeadDim : nullptr;
+    float q4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (nt > 0) {
+        const uint2 qr = *reinterpret_cast<const uint2 *>(a.q + row * kHeadDim + 4 * lane);
+        q4[0] = bf16_to_f32(qr.x & 0xFFFFu) * a.scale_log2;
+        q4[1] = bf16_to_f32(qr.x >> 16) * a.scale_log2;
+        q4[2] = bf16_to_f32(qr.y & 0xFFFFu) * a.scale_log2;
+        q4[3] = bf16_to_f32(qr.y >> 16) * a.scale_log2;
+    }
+    float M, l, o;
+    merge_partials(a.partials + row * a.S * kPartialStride, a.S, tid, M, l, o);
+    for (int c0 = 0; c0 < nt; c0 += kChunk) {
+        const int cn = min(kChunk, nt - c0);
+        // logits of the chunk (L2 loads: the tail rows may just have been written)
+        for (int jj = warp; jj < cn; jj += 4) {
+            const uint2 kr = __ldcg(reinterpret_cast<const uint2 *>(tk + (size_t)(c0 + jj) * tstride + 4 * lane));
+            float z = q4[0] * bf16_to_f32(kr.x & 0xFFFFu);
+            z = fmaf(q4[1], bf16_to_f32(kr.x >> 16), z);
+            z = fmaf(q4[2], bf16_to_f32(kr.y & 0xFFFFu), z);
+            z = fmaf(q4[3], bf16_to_f32(kr.y >> 16), z);
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+            if (lane == 0) s_z[jj] = z;
+        }
+        __syncthreads();
+        float mc = tid < cn ? s_z[tid] : -CUDART_INF_F;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, m));
+        if (lane == 0) s_red[warp] = mc;
+        __syncthreads();
+        const float Mn = fmaxf(M, fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3])));
+        const float c = exp2f(M - Mn);   // 0 while M = -inf
+        l *= c;
+        o *= c;
+        for (int j = 0; j < cn; j++) {
+            const float w = exp2f(s_z[j] - Mn);
+            l += w;
+            o = fmaf(w, bf16_to_f32(__ldcg(tv + (size_t)(c0 + j) * tstride + tid)), o);
+        }
+        M = Mn;
+        __syncthreads();   // s_z and s_red are rewritten by the next chunk
+    }
+    a.out[row * kHeadDim + tid] = (l > 0.f) ? o / l : 0.f;
 }
 
 template <int BA, int BR, int GS, bool RESID>
@@ -808,7 +901,7 @@ cudaError_t launch_group(const PrefillArgs &a, int ba, int br, cudaStream_t st) 
 // fixed cost of RQ_PREFILL_STEP_OVERHEAD steps per CTA), one CTA per SM (the tiles take 193 KB of shared memory
 // and the accumulators all 512 tensor-memory columns).
 #ifndef RQ_PREFILL_STEP_OVERHEAD
-#define RQ_PREFILL_STEP_OVERHEAD 1
+#define RQ_PREFILL_STEP_OVERHEAD 3
 #endif
 void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
     (void)ba;
