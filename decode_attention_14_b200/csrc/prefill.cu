@@ -690,10 +690,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         // Thread (side, part, t): token t of the step, K (side 0) or V, half
         // (part & 1) of its anchor (part < 2) or residual record.  The record
         // of step j + 1 is loaded into registers while step j's is written.
-        const int dt = tid - 32 * (kSoftmaxWarps + 1);
-        const int side = dt / (4 * kTok);
-        const int part = (dt / kTok) & 3;   // 0, 1: anchor halves; 2, 3: residual halves
-        const int t = dt % kTok;
+        // A warp per (side, part), a lane per token; the roles are dealt so
+        // that every scheduler (warp index mod 4) gets one anchor half and one
+        // (costlier) residual half.
+        static_assert(kTok == 32, "a lane per token of the step");
+        const int dq = warp - (kSoftmaxWarps + 1);   // 0 .. 7
+        const int side = dq >> 2;
+        const int part = (0x31201302u >> (4 * dq)) & 0xF;   // 2, 0, 3, 1, 0, 2, 1, 3
+        const int t = lane;
         auto load = [&](int j, RawHalf &r, uint16_t *cf) {
             const bool ok = t < min(kTok, cnt - j * kTok);
             const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok + t;
@@ -833,6 +837,7 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
     for (int c0 = 0; c0 < nt; c0 += kChunk) {
         const int cn = min(kChunk, nt - c0);
         // logits of the chunk (L2 loads: the tail rows may just have been written)
+#pragma unroll 4
         for (int jj = warp; jj < cn; jj += 4) {
             const uint2 kr = __ldcg(reinterpret_cast<const uint2 *>(tk + (size_t)(c0 + jj) * tstride + 4 * lane));
             float z = q4[0] * bf16_to_f32(kr.x & 0xFFFFu);
@@ -853,6 +858,7 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
         const float c = exp2f(M - Mn);   // 0 while M = -inf
         l *= c;
         o *= c;
+#pragma unroll 8
         for (int j = 0; j < cn; j++) {
             const float w = exp2f(s_z[j] - Mn);
             l += w;

@@ -166,6 +166,31 @@ def test_prefill_many_query_rows():
     cache.check()
 
 
+def test_prefill_long_chunk_in_the_tail():
+    """A 150-token chunk in the tail of loop 1: 150 query rows per kv head
+    (three 64-row blocks), and tails longer than one 128-token batch of the
+    combine kernel; then committed at the anchor loop."""
+    B, Hkv, T, n = 2, 2, 700, 150
+    bt = H.build(layers=1, loops=4, Lg=4, B=B, T=T, H=Hkv, Hq=Hkv, n_tail=0, chunk=256, seed=0x5EED9250,
+                 max_tokens=T + n)
+    cache, cfg = bt.cache, bt.cfg
+    sel = [(b, h) for b in range(B) for h in range(Hkv)]
+    K, V = _recon(cache, cfg, 0, 0)
+    nk, nv = _new_tokens(61, 4, B, n, Hkv)
+    cache.append(0, 0, nk[0], nv[0])
+    cache.append(0, 1, nk[1], nv[1])
+    q = _queries(450, B, n, Hkv)
+    out = cache.prefill(0, 1, q).cpu().numpy()
+    _check(out, _reference(K[1], V[1], q, [T] * B, n, 1, sel, (_f64(nk[1]), _f64(nv[1]))), 1)
+    cache.append(0, 2, nk[2], nv[2])
+    cache.append(0, 3, nk[3], nv[3])
+    K, V = _recon(cache, cfg, 0, 0)
+    q = _queries(451, B, n, Hkv)
+    out = cache.prefill(0, 3, q).cpu().numpy()
+    _check(out, _reference(K[3], V[3], q, [T + n] * B, 0, 1, sel), 1)
+    cache.check()
+
+
 def test_prefill_one_token_is_decode():
     B, Hkv, Hq, T = 2, 2, 4, 200
     bt = H.build(layers=1, loops=4, Lg=4, B=B, T=T, H=Hkv, Hq=Hq, n_tail=1, chunk=64, seed=0x5EED9300)
