@@ -359,7 +359,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
     const int Tb = a.seqT.v[b];
     int t0, cnt;
     split_range(split, a.S, Tb, &t0, &cnt);
-    const int ntl = cnt > 0 ? (cnt + kTok - 1) / kTok : 0;
+    // committed steps, then (last split of each sequence and kv head) steps
+    // over the loop's BF16 tail tokens: an anchor-like step with the tokens'
+    // K and V as exact BF16 operands, coefficient 1 and no residual part
+    const int ntc = cnt > 0 ? (cnt + kTok - 1) / kTok : 0;
+    const bool tail_here = a.tail_in_kernel && a.tail_k != nullptr && split == a.S - 1;
+    const int ntl = ntc + (tail_here ? (a.n_tail + kTok - 1) / kTok : 0);
     const size_t bh = (size_t)b * a.H + h;
     constexpr int MR = 2 * (kHeadDim / GS);
 
@@ -409,6 +414,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         const int r = 16 * warp + i16;
         const int iq = (r0 + r) / a.G;
         const int lim = min(Tb, Tb + a.n_tail - a.n + 1 + iq);   // committed tokens the row may see
+        const int ltail = min(a.n_tail, max(0, a.n_tail - a.n + 1 + iq));   // tail tokens it may see
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
         constexpr int kHalf = kTok / 2;                          // tokens of a thread per step
         float m_used = -CUDART_INF_F, l = 0.f;                   // l: this thread's half of the row's sum
@@ -422,12 +428,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             tc::fence_after();
             // logits, and this thread's V coefficients, read before the
             // logits buffer and the coefficient slot are released
+            const bool tstep = j >= ntc;   // a tail step (warp-uniform)
             float s[kHalf], cv[kHalf];
             {
                 const uint32_t cS = kColS + pb * 2 * kTok;
                 uint32_t sa[16];
                 tc::ld16x2<kHalf>(tl + cS, sa);
-                if (RESID) {
+                if (RESID && !tstep) {
                     uint32_t y0[16], y1[16];
                     tc::ld16(tl + cS + kTok, y0);        // this lane's part of SY, tokens 0..15
                     tc::ld16(tl + cS + kTok + 16, y1);   // tokens 16..31
@@ -471,12 +478,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             tc::fence_before();
             mbar_arrive(&bar_sfree[pb]);
             float mx = -CUDART_INF_F;
-            if (tn < kTok || t0 + tt + kTok > lim) {   // the step's end is not visible to the row
+            if (!tstep) {
+                if (tn < kTok || t0 + tt + kTok > lim) {   // the step's end is not visible to the row
 #pragma unroll
-                for (int k = 0; k < kHalf; k++) {
-                    const int t = kHalf * hf + k;
-                    const bool ok = t < tn && t0 + tt + t < lim;
-                    s[k] = ok ? s[k] : -CUDART_INF_F;
+                    for (int k = 0; k < kHalf; k++) {
+                        const int t = kHalf * hf + k;
+                        const bool ok = t < tn && t0 + tt + t < lim;
+                        s[k] = ok ? s[k] : -CUDART_INF_F;
+                    }
+                }
+            } else {
+                const int jt0 = (j - ntc) * kTok;   // first tail token of the step
+                if (jt0 + kTok > ltail) {
+#pragma unroll
+                    for (int k = 0; k < kHalf; k++) {
+                        const bool ok = jt0 + kHalf * hf + k < ltail;
+                        s[k] = ok ? s[k] : -CUDART_INF_F;
+                    }
                 }
             }
 #pragma unroll
@@ -573,7 +591,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             wait(&bar_odone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, 24);
             tc::fence_after();
 #pragma unroll
-            for (int side = 0; side < (RESID ? 2 : 1); side++) {
+            // OY holds something only if a committed step ran (tail steps add nothing to it)
+            for (int side = 0; side < ((RESID && ntc > 0) ? 2 : 1); side++) {
                 const uint32_t col = side == 0 ? kColOA : kColOY;
                 float *dst = (side == 0 ? sA : sY) + r * kEStride + 8 * hf;
                 // the row's group minima: high + low lane
@@ -633,7 +652,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 const uint64_t ka = dK + (uint64_t)(((j & 1) * kKVBytes) >> 4);
                 const uint64_t ky = ka + (uint64_t)((3 * kTBlk) >> 4);
                 const uint32_t cS = tmem + kColS + (j & 1) * 2 * kTok;
-                if (!yside) {
+                if (yside && j >= ntc) {
+                    // a tail step has no residual part: nothing to issue
+                } else if (!yside) {
 #pragma unroll
                     for (int kk = 0; kk < 8; kk++) tc::mma_bf16(cS, dQ + kq(kk), ka + kt(kk), idA, kk > 0);
                     tc::mma_bf16(cS, dQm, ka + kt(8), idA, true);   // the group sums of q against the minima
@@ -647,10 +668,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 const uint64_t pbuf = dP + (uint64_t)(((j & 1) * kPBytes + (yside ? kSBlk : 0)) >> 4);
                 const uint64_t vv = dV + (uint64_t)(((j & 1) * kKVBytes + (yside ? 3 * kTBlk : 0)) >> 4);
                 const uint32_t cO = tmem + (yside ? kColOY : kColOA);
+                if (!(yside && j >= ntc)) {
 #pragma unroll
-                for (int kk = 0; kk < kTok / 16; kk++)
-                    tc::mma_bf16(cO, pbuf + (uint64_t)((kk * 32) >> 4), vv + (uint64_t)((kk * 16 * 128) >> 4), idV,
-                                 j > 0 || kk > 0);
+                    for (int kk = 0; kk < kTok / 16; kk++)
+                        tc::mma_bf16(cO, pbuf + (uint64_t)((kk * 32) >> 4), vv + (uint64_t)((kk * 16 * 128) >> 4),
+                                     idV, j > 0 || kk > 0);
+                }
                 tc::commit(&bar_odone[j & 1]);
             };
             int nl = 0, nv = 0;   // steps whose logits / values are issued
@@ -715,15 +738,35 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         };
         RawHalf raw;
         uint16_t cf[2] = {0, 0};
-        if (ntl > 0) load(0, raw, cf);
+        if (ntc > 0) load(0, raw, cf);
         for (int j = 0; j < ntl; j++) {
-            const bool ok = t < min(kTok, cnt - j * kTok);
+            const bool tstep = j >= ntc;
+            const bool ok = !tstep && t < min(kTok, cnt - j * kTok);
             const int pb = j & 1;
             // the buffer was last read by the logits (K) / values (V) of step j - 2
             if (j >= 2) wait(side == 0 ? &bar_kdone[pb] : &bar_odone[pb], ((j >> 1) - 1) & 1, 29);
             uint8_t *ta = sm + (side == 0 ? OFF_K : OFF_V) + pb * kKVBytes;
             uint8_t *ty = ta + 3 * kTBlk;
-            if (part == 0) store_half<BA, GS, 0, kTBlk>(ta, t, raw, ok);
+            if (tstep) {
+                // tail token jt's K or V half, BF16 as it is; minima zero
+                if (part < 2) {
+                    const int jt = (j - ntc) * kTok + t;
+                    const bool tok = jt < a.n_tail;
+                    const uint16_t *src =
+                        (side == 0 ? a.tail_k : a.tail_v) + (((size_t)b * a.tail_cap + (tok ? jt : 0)) * a.H + h) * kHeadDim;
+                    uint8_t *row = ta + part * kTBlk;
+#pragma unroll
+                    for (int c = 0; c < 8; c++) {
+                        const uint4 v = tok ? __ldcg(reinterpret_cast<const uint4 *>(src + 64 * part) + c)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+                        st_shared16(row + tc::sw_chunk(t, c), v.x, v.y, v.z, v.w);
+                    }
+                    if (part == 0) {
+                        st_shared16(ta + 2 * kTBlk + tc::sw_chunk(t, 0), 0u, 0u, 0u, 0u);
+                        st_shared16(ta + 2 * kTBlk + tc::sw_chunk(t, 1), 0u, 0u, 0u, 0u);
+                    }
+                }
+            } else if (part == 0) store_half<BA, GS, 0, kTBlk>(ta, t, raw, ok);
             else if (part == 1) store_half<BA, GS, 1, kTBlk>(ta, t, raw, ok);
             else if (RESID) {
                 if (part == 2) store_half<BR, GS, 0, kTBlk>(ty, t, raw, ok);
@@ -739,7 +782,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             }
             tc::fence_async_smem();
             mbar_arrive(side == 0 ? &bar_kfull[pb] : &bar_vfull[pb]);
-            if (j + 1 < ntl) load(j + 1, raw, cf);
+            if (j + 1 < ntc) load(j + 1, raw, cf);
         }
     }
 
@@ -762,7 +805,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                 const int row = min(row0 + u * kWarps, kRows - 1);   // a row past nr is computed, not written
 #pragma unroll
                 for (int k = 0; k < 4; k++) o[u][k] = 0.f;
-                if (ntl > 0 && RESID) {
+                if (ntc > 0 && RESID) {
                     const float4 y = *reinterpret_cast<const float4 *>(sY + row * kEStride + 4 * lane);
                     o[u][0] = y.x;
                     o[u][1] = y.y;
@@ -770,7 +813,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                     o[u][3] = y.w;
                 }
             }
-            if (ntl > 0 && RESID && a.rotate) {
+            if (ntc > 0 && RESID && a.rotate) {
                 // R^T Y = diag(sigma) H Y / sqrt(d)
                 wht128_warp2<float>(o[0], o[1], lane);
 #pragma unroll
@@ -820,7 +863,7 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
     const size_t row = ((size_t)b * a.n + i) * a.Hq + hq;
     // of [committed, tail] the row sees T_b + n_tail - n + 1 + i tokens: all
     // committed ones when the new tokens are in the tail
-    const int nt = a.tail_k ? max(0, a.n_tail - a.n + 1 + i) : 0;
+    const int nt = (a.tail_k && !a.tail_in_kernel) ? max(0, a.n_tail - a.n + 1 + i) : 0;
     const size_t tstride = (size_t)a.H * kHeadDim;
     const uint16_t *tk = a.tail_k ? a.tail_k + ((size_t)b * a.tail_cap * a.H + h) * kHeadDim : nullptr;
     const uint16_t *tv = a.tail_v ? a.tail_v + ((size_t)b * a.tail_cap * a.H + h) * kHeadDim : nullptr;
@@ -915,7 +958,9 @@ void prefill_plan(PrefillArgs *a, int T, int ba, int br, int sms) {
     const int nq = a->n * a->G;
     a->nqb = (nq + kRows - 1) / kRows;
     a->S = 0;
-    if (T <= 0) return;
+    a->tail_in_kernel = 0;
+    if (T <= 0) return;   // nothing committed: the combine kernel takes the tail
+    a->tail_in_kernel = 1;
     const long slots = (long)std::max(1, sms);
     const long units = (long)a->B * a->H * a->nqb;
     const int nt = (T + kTokTile - 1) / kTokTile;

@@ -28,6 +28,7 @@ struct PrefillArgs {
     int rotate;
     uint32_t sigma[4];
     int *err;                          // device error word (bounded waits that gave up)
+    int tail_in_kernel;                // the attention kernel (last split) takes the tail tokens
 };
 
 // Sets a->nqb and the split count a->S over the committed tokens (T
