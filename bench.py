@@ -672,13 +672,19 @@ def _bf16_peak():
 
 
 def prefill_mma_flops(n, G, B, H, T, resid):
-    """Tensor-core FLOPs rq_prefill_attn issues: per CTA step (64 query rows x
-    64 committed tokens) 9 (+17 at a residual loop) logit MMAs of 64x64x16
-    and 8 (+8) value MMAs of 64x136x16."""
-    steps = B * H * ((n * G + 63) // 64) * ((T + 63) // 64)
-    logit = (9 + (17 if resid else 0)) * 2 * 64 * 64 * 16
-    value = (8 + (8 if resid else 0)) * 2 * 64 * 136 * 16
-    return steps * (logit + value)
+    """Tensor-core FLOPs rq_prefill_attn issues.  A CTA takes 64 query rows
+    and steps over 32 committed tokens at a time: 9 logit MMAs of 64x32x16
+    and 2 value MMAs of 128x136x16 (the probabilities' high and low parts
+    stacked) on the anchor side, and at a residual loop as many again on the
+    residual side with the logit MMAs also at M = 128 (Rq's high and low
+    parts stacked).  At a residual loop the n new tokens sit in the BF16
+    tail, which the last split takes as anchor-side steps."""
+    units = B * H * ((n * G + 63) // 64)
+    anchor = 9 * 2 * 64 * 32 * 16 + 2 * 2 * 128 * 136 * 16
+    residual = 9 * 2 * 128 * 32 * 16 + 2 * 2 * 128 * 136 * 16
+    committed = units * ((T + 31) // 32) * (anchor + (residual if resid else 0))
+    tail = units * ((n + 31) // 32) * anchor if resid else 0
+    return committed + tail
 
 
 def run_prefill(args):

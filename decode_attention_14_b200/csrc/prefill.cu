@@ -21,12 +21,13 @@
 //  - the minima ride along as extra K columns of the logit products (group
 //    sums of q against the minima of the keys) and as extra N rows of the
 //    value products (probabilities against the minima of the values).
-// R^T is applied once per CTA to the accumulated Y.  Per 64-token step and
-// 64 query rows:
-//   SA = [q | Q_g] [sc code | mn]^T            (9 MMAs of 64x64x16)
-//   SY = [Rq_hi | (Rq)_g] [..]^T + Rq_lo [..]^T (17 MMAs)
-//   OA += (p s)_hi [sc code | mn] + (p s)_lo [..]   (8 MMAs of 64x136x16)
-//   OY += p_hi [sc_r code_r | mn_r] + p_lo [..]     (8 MMAs)
+// R^T is applied once per CTA to the accumulated Y.  Per 32-token step and
+// 64 query rows (operands with a high and a low part stacked as M = 128):
+//   SA = [q | Q_g] [sc code | mn]^T                      (9 MMAs of 64x32x16)
+//   SY = [Rq | (Rq)_g]_hi,lo [sc_r code_r | mn_r]^T      (9 MMAs of 128x32x16)
+//   OA += (p s)_hi,lo [sc code | mn]                     (2 MMAs of 128x136x16)
+//   OY += p_hi,lo [sc_r code_r | mn_r]                   (2 MMAs of 128x136x16)
+// (the two row halves of SY, OA, OY are summed when they are read back)
 // with logits scale_log2 (s SA + SY) and a running maximum that is only
 // raised when a row's maximum grows by more than 2^8 (then that row of OA and
 // OY is rescaled in tensor memory); the partial (m, l, o) of each row goes to
@@ -45,7 +46,7 @@
 //    memory) into the swizzled operand tiles.
 // Hand-offs go through mbarriers, every wait bounded (error word, abort flag):
 //   kfull/vfull   dequant -> MMA       K / V operands of step j written
-//   cfull[j & 1]  dequant -> softmax   coefficients of step j written
+//   cfull[j & 3]  dequant -> softmax   coefficients of step j written
 //   kdone         MMA commit           logits of step j complete (K tile free)
 //   sfree         softmax -> MMA       logits of step j read (SA/SY free)
 //   pfull         softmax -> MMA       probabilities of step j written
