@@ -43,7 +43,8 @@
 //    (SA, OA) and of the residual side (SY, OY); warp 4 allocates tensor
 //    memory;
 //  - warps 5-12: dequantize the step's K and V records (straight from global
-//    memory) into the swizzled operand tiles.
+//    memory; the anchor records brought into L2 two steps ahead) into the
+//    swizzled operand tiles.
 // Hand-offs go through mbarriers, every wait bounded (error word, abort flag):
 //   kfull/vfull   dequant -> MMA       K / V operands of step j written
 //   cfull[j & 3]  dequant -> softmax   coefficients of step j written
@@ -65,6 +66,10 @@ namespace rq {
 namespace {
 
 constexpr int kRows = 64;             // query rows of a CTA (M of every MMA)
+#ifndef RQ_PREFILL_PREFETCH
+#define RQ_PREFILL_PREFETCH 2
+#endif
+constexpr int kPrefetchSteps = RQ_PREFILL_PREFETCH;   // steps of records brought into L2 ahead of their loads (0: none)
 constexpr int kTok = kPrefillTile;    // committed tokens per step (N of the logits, K of the values)
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = 4;            // issues the anchor-side MMAs (SA, OA); allocates tensor memory
@@ -140,17 +145,19 @@ __device__ __forceinline__ void st_shared_u16(uint8_t *p, uint32_t x) {
 __device__ __forceinline__ void st_shared8(uint8_t *p, uint32_t x, uint32_t y) {
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(p)), "r"(x), "r"(y) : "memory");
 }
+// Bulk prefetch of [p, p + bytes) from global memory into L2 (p 16-byte
+// aligned, bytes a multiple of 16); nothing waits for it.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
-// BF16 pair (128 + code of element 2p, 128 + code of element 2p + 1) of a
-// word of BITS-bit codes, LSB first: 0x4300 is 128.0 with one unit per code.
+// BF16 pair (128 + code x, 128 + code y): x in bits 0 .. BITS-1 of byte b of
+// wx, y in the same bits of byte b of wy (0x4300 is 128.0 with one unit per
+// code; one byte permute and one mask-and-or).
 template <int BITS>
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, int p) {
-    if (BITS == 4) {
-        const uint32_t t = w >> (8 * p);
-        return 0x43004300u | (t & 0xFu) | ((t & 0xF0u) << 12);
-    }
-    const uint32_t t = w >> (4 * p);
-    return 0x43004300u | (t & 0x3u) | ((t & 0xCu) << 14);
+__device__ __forceinline__ uint32_t code_pair(uint32_t wx, uint32_t wy, int b) {
+    constexpr uint32_t m = BITS == 4 ? 0x000F000Fu : 0x00030003u;
+    return (__byte_perm(wx, wy, (uint32_t)(b | ((4 + b) << 8))) & m) | 0x43004300u;
 }
 
 // Raw bytes of half a record (head_dim elements 64 h .. 64 h + 63): its
@@ -223,16 +230,20 @@ __device__ __forceinline__ void store_half(uint8_t *tile, int t, const RawHalf &
             const int c = gl * CPG + cg;   // chunk of the half: elements 8c .. 8c + 7
             uint32_t q[4];
             if (BITS == 4) {
-                // even elements in the bytes of lo, odd ones in the bytes of hi;
-                // byte k of each into the low byte of one half of pair k
-                const uint32_t lo = r.w[c] & 0x0F0F0F0Fu, hi = (r.w[c] >> 4) & 0x0F0F0F0Fu;
+                // pair k: element 8c + 2k in the low nibble of byte k of the
+                // word, element 8c + 2k + 1 in its high nibble
+                const uint32_t w = r.w[c];
 #pragma unroll
-                for (int k = 0; k < 4; k++)
-                    q[k] = (__byte_perm(lo, hi, (uint32_t)(k | ((4 + k) << 8))) & 0x00FF00FFu) | 0x43004300u;
+                for (int k = 0; k < 4; k++) q[k] = code_pair<4>(w, w >> 4, k);
             } else {
-                const uint32_t cw = r.w[c >> 1] >> (16 * (c & 1));
+                // pair k: elements 8c + 2k, 8c + 2k + 1 in bits 4(k & 1) ..
+                // 4(k & 1) + 3 of byte 2(c & 1) + k / 2 of the word
+                const uint32_t w = r.w[c >> 1];
 #pragma unroll
-                for (int k = 0; k < 4; k++) q[k] = code_pair<BITS>(cw, k);
+                for (int k = 0; k < 4; k++) {
+                    const int b = 2 * (c & 1) + (k >> 1);
+                    q[k] = (k & 1) ? code_pair<2>(w >> 4, w >> 6, b) : code_pair<2>(w, w >> 2, b);
+                }
             }
             st_shared16(row + tc::sw_chunk(t, c), fma_bf16x2(q[0], s2, nb2), fma_bf16x2(q[1], s2, nb2),
                         fma_bf16x2(q[2], s2, nb2), fma_bf16x2(q[3], s2, nb2));
@@ -737,9 +748,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
                                   ok ? a.r_meta[side] + rec * MR : nullptr, part - 2, ok, r);
             }
         };
+        // Lane 0 of the warps of part 0 brings the anchor records (codes and
+        // meta) of step j + 1 + kPrefetchSteps of its side into L2 while step
+        // j is written, so that the register loads of that step find them
+        // there: a whole step (the padded token capacity of a sequence is a
+        // multiple of 64 tokens, so a full step never leaves it).  The
+        // residual records are not prefetched: that made residual loops
+        // slower 1 or 2 steps ahead and gained nothing 3 steps ahead.
+        auto prefetch = [&](int j) {
+            if (kPrefetchSteps <= 0 || lane != 0 || part != 0 || j >= ntc) return;
+            const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok;
+            prefetch_l2(a.a_codes[side] + rec * (16 * BA), kTok * 16 * BA);
+            prefetch_l2(a.a_meta[side] + rec * MR, kTok * MR);
+        };
         RawHalf raw;
         uint16_t cf[2] = {0, 0};
         if (ntc > 0) load(0, raw, cf);
+        for (int i = 1; i <= kPrefetchSteps; i++) prefetch(i);
         for (int j = 0; j < ntl; j++) {
             const bool tstep = j >= ntc;
             const bool ok = !tstep && t < min(kTok, cnt - j * kTok);
@@ -784,6 +809,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             tc::fence_async_smem();
             mbar_arrive(side == 0 ? &bar_kfull[pb] : &bar_vfull[pb]);
             if (j + 1 < ntc) load(j + 1, raw, cf);
+            prefetch(j + 1 + kPrefetchSteps);
         }
     }
 
