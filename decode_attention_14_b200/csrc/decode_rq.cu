@@ -346,7 +346,9 @@ struct Plan {
 
 // NR: residual records the loop's reconstruction reads (0 for the anchor's
 // own loop, 1 for the shared reference, 1..3 along a chained reference).
-template <int GK, int BA, int BR, int GS, int NR>
+// PG: records in a pool of blocks behind a block table (a.pg.table set); the
+// contiguous instantiation carries none of the block arithmetic.
+template <int GK, int BA, int BR, int GS, int NR, bool PG>
 __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) decode_rq_kernel(const DecodeArgs a) {
     using P = Plan<BA, BR, GS, NR>;
     constexpr bool RESID = NR > 0;
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     __shared__ __align__(8) uint64_t bar_cf;
     __shared__ __align__(8) uint64_t bar_cfmax;   // the chunk's max |s_hat(V)| is known
     __shared__ int s_abort, s_last;
-    __shared__ int s_blk[kMaxChunk / kTokTile + 1];   // paged: physical blocks of the chunk
+    __shared__ int s_blk[PG ? kMaxChunk / kTokTile + 1 : 1];   // paged: physical blocks of the chunk
     __shared__ unsigned s_cfmax[NW];
     __shared__ float s_q[GK][2][kHeadDim];
     __shared__ __align__(16) uint8_t s_qp[GK][2][3][kHeadDim];   // q byte planes, [plane][segment][word][byte]
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     // paged: ring items start on item-size boundaries of the sequence (a
     // split may begin inside one), so that no item straddles two blocks; the
     // item grid then begins sh tiles before the split, which stay empty
-    const int sh = (a.pg.table != nullptr && ntiles > 0) ? (t0 / kTile) % kItemTiles : 0;
+    const int sh = (PG && ntiles > 0) ? (t0 / kTile) % kItemTiles : 0;
     const int ntv = ntiles + sh;   // tiles of the item grid
     const size_t bh = (size_t)b * a.H + h;
     uint8_t *ring = smem;
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
         // memory (through L2).  Before the grid dependency wait only when the
         // whole chunk lies below a.stable: the host sets a.stable to 0 when a
         // block-table change may be in flight, so such rows are settled.
-        const bool paged = a.pg.table != nullptr;
+        constexpr bool paged = PG;
         const bool early = paged && t0 + ntiles * kTile <= a.stable;
         const int blk0 = t0 >> a.pg.shift;
         if (paged) {
@@ -688,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
             if (j * kItemTiles + u >= ntv) break;   // uniform: a short last item
-            if (j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
+            if (PG && j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 const int tok = u * kTile + 16 * warp + sub + 4 * k;   // token within the item
@@ -719,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
         for (int u = 0; u < kItemTiles; u++) {
             if (j * kItemTiles + u >= ntv) break;
-            if (j * kItemTiles + u < sh) continue;
+            if (PG && j * kItemTiles + u < sh) continue;
             const int i = j * kItemTiles + u - sh;   // tile of the chunk
             const int tl = i * kTile + 16 * warp + sub + 4 * kown;
 #pragma unroll
@@ -831,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
 #pragma unroll
             for (int u = 0; u < kItemTiles; u++) {
                 if (u > last_u) break;   // uniform
-                if (j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
+                if (PG && j * kItemTiles + u < sh) continue;   // uniform: an empty first tile
                 uint32_t wlo[GK][2], whi[GK][2];
                 float2 mm[4];
                 float W[GK][4];
@@ -1002,20 +1004,20 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
     }
 }
 
-template <int GK, int BA, int BR, int GS, int NR>
+template <int GK, int BA, int BR, int GS, int NR, bool PG>
 cudaError_t configure() {
     static bool done[kMaxDevices] = {};   // the largest dynamic shared memory any launch can ask for
     return once_per_device(done, [] {
-        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, NR>,
+        return cudaFuncSetAttribute(decode_rq_kernel<GK, BA, BR, GS, NR, PG>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)Plan<BA, BR, GS, NR>::smem(GK, kMaxChunk));
     });
 }
 
-template <int GK, int BA, int BR, int GS, int NR>
+template <int GK, int BA, int BR, int GS, int NR, bool PG>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
     const dim3 grid(a.S, a.H, a.B * (a.G / GK));
-    cudaError_t e = configure<GK, BA, BR, GS, NR>();
+    cudaError_t e = configure<GK, BA, BR, GS, NR, PG>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = grid;
@@ -1027,16 +1029,16 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = RQ_DECODE_PDL ? 1 : 0;
-    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, NR>, a);
+    e = cudaLaunchKernelEx(&lc, decode_rq_kernel<GK, BA, BR, GS, NR, PG>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-template <int GK, int BA, int BR, int GS, int NR>
+template <int GK, int BA, int BR, int GS, int NR, bool PG>
 int occupancy_t(int chunk) {
-    if (configure<GK, BA, BR, GS, NR>() != cudaSuccess) return 1;
+    if (configure<GK, BA, BR, GS, NR, PG>() != cudaSuccess) return 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, NR>, kThreads,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_rq_kernel<GK, BA, BR, GS, NR, PG>, kThreads,
                                                       Plan<BA, BR, GS, NR>::smem(GK, chunk)) != cudaSuccess)
         return 1;
     return n > 0 ? n : 1;
@@ -1063,12 +1065,14 @@ struct LaunchF {
     const DecodeArgs *a;
     cudaStream_t st;
     template <int GK, int BA, int BR, int GS, int NR>
-    cudaError_t go() const { return launch_t<GK, BA, BR, GS, NR>(*a, st); }
+    cudaError_t go() const {
+        return a->pg.table ? launch_t<GK, BA, BR, GS, NR, true>(*a, st) : launch_t<GK, BA, BR, GS, NR, false>(*a, st);
+    }
 };
 struct OccF {
     int chunk;
     template <int GK, int BA, int BR, int GS, int NR>
-    int go() const { return occupancy_t<GK, BA, BR, GS, NR>(chunk); }
+    int go() const { return occupancy_t<GK, BA, BR, GS, NR, false>(chunk); }   // same resources paged or not
 };
 
 template <typename F>
