@@ -34,6 +34,10 @@ struct rq_cache {
     // split partials of rq_prefill_attn, allocated on first use and grown on demand
     float *prefill_ws = nullptr;
     size_t prefill_ws_floats = 0;
+    // arrival counters of rq_prefill_attn's row blocks (zeroed once; every
+    // launch leaves them at zero)
+    int *prefill_cnt = nullptr;
+    size_t prefill_cnt_n = 0;
     // paged records: host copy of the block table [B][MB] (-1: no block),
     // reference counts of the physical blocks (forked sequences share
     // blocks), and the free list (blocks are taken from its back)
@@ -519,11 +523,12 @@ int rq_cache_create(const rq_config *cfg, void *dev_mem, size_t bytes, rq_cache 
 int rq_cache_destroy(rq_cache *c) {
     if (!c) return RQ_OK;
     int st = RQ_OK;
-    if (c->owned || c->prefill_ws) {
+    if (c->owned || c->prefill_ws || c->prefill_cnt) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = RQ_ERR_CUDA;
     }
     if (c->owned) cudaFree(c->base);
     if (c->prefill_ws) cudaFree(c->prefill_ws);
+    if (c->prefill_cnt) cudaFree(c->prefill_cnt);
     delete c;
     return st;
 }
@@ -850,6 +855,30 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
         c->prefill_ws_floats = need;
     }
     a.partials = c->prefill_ws;
+    a.counters = nullptr;
+    if (a.S > 0) {
+        const size_t units = (size_t)a.B * a.H * a.nqb;
+        if (units > c->prefill_cnt_n) {
+            if (c->prefill_cnt) {
+                if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
+                cudaFree(c->prefill_cnt);
+                c->prefill_cnt = nullptr;
+                c->prefill_cnt_n = 0;
+            }
+            void *p = nullptr;
+            if (cudaMalloc(&p, units * sizeof(int)) != cudaSuccess) {
+                cudaGetLastError();
+                return RQ_ERR_NOMEM;
+            }
+            if (cudaMemset(p, 0, units * sizeof(int)) != cudaSuccess) {
+                cudaFree(p);
+                return RQ_ERR_CUDA;
+            }
+            c->prefill_cnt = (int *)p;
+            c->prefill_cnt_n = units;
+        }
+        a.counters = c->prefill_cnt;
+    }
     a.err = (int *)(c->base + L.off_err);
     return cuda_status(launch_prefill(a, cfg.anchor_bits, cfg.resid_bits, (cudaStream_t)stream));
 }

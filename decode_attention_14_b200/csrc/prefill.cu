@@ -31,7 +31,9 @@
 // with logits scale_log2 (s SA + SY) and a running maximum that is only
 // raised when a row's maximum grows by more than 2^8 (then that row of OA and
 // OY is rescaled in tensor memory); the partial (m, l, o) of each row goes to
-// a second kernel that merges the splits and the tail tokens.
+// global memory, and the last split of each row block to finish merges them
+// (a second kernel does, with the tail tokens, only when nothing is
+// committed and this kernel does not run).
 //
 // CTA = (split of the committed tokens, kv head, sequence x block of 64 query
 // rows); 14 warps:
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
     __shared__ uint64_t bar_kfull[2], bar_vfull[2], bar_kdone[2], bar_sfree[2], bar_pfull[2], bar_odone[2];
     __shared__ uint64_t bar_cfull[4];
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
+    __shared__ int s_abort, s_last;
     __shared__ __align__(16) float s_cK[4][kTok], s_cV[4][kTok];   // coefficients of a step (1 at an anchor loop)
     __shared__ float s_ml[kRows][2];                  // running maximum and sum of each row
 
@@ -870,6 +872,43 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
             }
         }
     }
+    // ------------------------------------------------------- split merge
+    // The last split of the row block to arrive merges every split's partial
+    // of its rows (a split with no key has m = -inf: weight 0) and writes the
+    // output rows; it leaves the counter at zero for the next launch.
+    if (a.counters) {
+        __threadfence();
+        __syncthreads();
+        const int unit = (b * a.H + h) * a.nqb + qb;
+        if (tid == 0) s_last = atomicAdd(a.counters + unit, 1) == a.S - 1;
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int row = warp; row < nr; row += kThreadsP / 32) {
+                const int rg = r0 + row, i = rg / a.G, gq = rg % a.G;
+                const size_t prow = ((size_t)b * a.n + i) * a.Hq + h * a.G + gq;
+                const float *part = a.partials + prow * a.S * kPartialStride;
+                float M = -CUDART_INF_F, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int sp = 0; sp < a.S; sp++) {
+                    const float *p = part + (size_t)sp * kPartialStride;
+                    const float m = __ldcg(p + kHeadDim), ls = __ldcg(p + kHeadDim + 1);
+                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(p) + lane);
+                    if (m == -CUDART_INF_F) continue;   // uniform over the warp
+                    const float Mn = fmaxf(M, m);
+                    const float c0 = exp2f(M - Mn), c = exp2f(m - Mn);   // c0 = 0 while M = -inf
+                    l = fmaf(ls, c, l * c0);
+                    o[0] = fmaf(v.x, c, o[0] * c0);
+                    o[1] = fmaf(v.y, c, o[1] * c0);
+                    o[2] = fmaf(v.z, c, o[2] * c0);
+                    o[3] = fmaf(v.w, c, o[3] * c0);
+                    M = Mn;
+                }
+                *reinterpret_cast<float4 *>(a.out + prow * kHeadDim + 4 * lane) =
+                    l > 0.f ? make_float4(o[0] / l, o[1] / l, o[2] / l, o[3] / l) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (tid == 0) a.counters[unit] = 0;
+        }
+    }
     if (warp == kMmaWarp) {
         tc::fence_after();
         tc::dealloc(tmem, kTmemCols);
@@ -1007,7 +1046,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, int ba, int br, cudaStream_t st
     if (a.g != 16 && a.g != 32) return cudaErrorInvalidValue;
     cudaError_t e = a.g == 16 ? launch_group<16>(a, ba, br, st) : launch_group<32>(a, ba, br, st);
     if (e != cudaSuccess) return e;
-    prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
+    if (!a.counters) prefill_combine_kernel<<<dim3(a.Hq, a.n, a.B), 128, 0, st>>>(a);
     return cudaGetLastError();
 }
 

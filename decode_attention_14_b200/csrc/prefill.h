@@ -28,6 +28,9 @@ struct PrefillArgs {
     int rotate;
     uint32_t sigma[4];
     int *err;                          // device error word (bounded waits that gave up)
+    int *counters;                     // [B][H][nqb] split arrivals (zero between calls): the last
+                                       // split of a row block merges the partials; null: the
+                                       // combine kernel merges them
     int tail_in_kernel;                // the attention kernel (last split) takes the tail tokens
 };
 
