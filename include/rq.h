@@ -244,11 +244,13 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
  * tail at the other loops -- and each sees itself and the ones before it.
  * The split partials live in a device buffer the cache allocates on the
  * first call (and grows when a later call needs more:
- * batch * n_tokens * num_q_heads * splits * 132 floats), freed by
- * rq_cache_destroy; that allocation synchronises the device, so make the
- * first call of a size before any stream capture.  Calls on one cache share
- * the buffer: calls whose work overlaps (other streams) must be ordered by
- * the caller.
+ * batch * n_tokens * num_q_heads * splits * 132 floats), and the arrival
+ * counters of the splits (batch * num_kv_heads * ceil(n_tokens * G / 64)
+ * ints, zeroed when allocated and left at zero by every call) in a second
+ * one; both are freed by rq_cache_destroy.  Those allocations synchronise the
+ * device, so make the first call of a size before any stream capture.  Calls
+ * on one cache share the buffers: calls whose work overlaps (other streams)
+ * must be ordered by the caller.
  * Errors: INVALID (null pointer, n_tokens < 1, index out of range), STATE
  * (wrong format, or a sequence holds fewer than n_tokens tokens),
  * UNSUPPORTED (n_tokens > 65535, or an INT2 anchor with INT4 residuals --
