@@ -245,7 +245,8 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
  * The split partials live in a device buffer the cache allocates on the
  * first call (and grows when a later call needs more:
  * batch * n_tokens * num_q_heads * splits * 132 floats), and the arrival
- * counters of the splits (batch * num_kv_heads * ceil(n_tokens * G / 64)
+ * counters of the splits (batch * num_kv_heads *
+ * ceil(n_tokens * num_q_heads / num_kv_heads / 64)
  * ints, zeroed when allocated and left at zero by every call) in a second
  * one; both are freed by rq_cache_destroy.  Those allocations synchronise the
  * device, so make the first call of a size before any stream capture.  Calls
