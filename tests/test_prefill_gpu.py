@@ -191,6 +191,34 @@ def test_prefill_long_chunk_in_the_tail():
     cache.check()
 
 
+def test_prefill_repeated_calls_and_growing_row_blocks():
+    """The last split of a row block merges the partials, found with arrival
+    counters that every call leaves at zero: on one cache with many splits per
+    row block, repeated calls give bit-identical outputs, also after a call
+    with more row blocks (the counter buffer grows) and back, and both sizes
+    match the oracle."""
+    B, Hkv, Hq, T, nb = 2, 2, 4, 3000, 40   # nb * G = 80 query rows per kv head: two row blocks
+    G = Hq // Hkv
+    bt = H.build(layers=1, loops=2, Lg=2, B=B, T=T, H=Hkv, Hq=Hq, n_tail=0, chunk=128, seed=0x5EED9400,
+                 max_tokens=T + nb)
+    cache, cfg = bt.cache, bt.cfg
+    sel = [(b, h) for b in range(B) for h in range(Hkv)]
+    K, V = _recon(cache, cfg, 0, 0)
+    nk, nv = _new_tokens(71, 2, B, nb, Hkv)
+    cache.append(0, 0, nk[0], nv[0])   # in loop 0's tail
+    tail = (_f64(nk[0]), _f64(nv[0]))
+    q_small, q_big = _queries(500, B, 4, Hq), _queries(501, B, nb, Hq)
+    o1 = cache.prefill(0, 0, q_small)
+    o2 = cache.prefill(0, 0, q_small)
+    o3 = cache.prefill(0, 0, q_big)
+    o4 = cache.prefill(0, 0, q_small)
+    o5 = cache.prefill(0, 0, q_big)
+    assert torch.equal(o1, o2) and torch.equal(o1, o4) and torch.equal(o3, o5)
+    _check(o1.cpu().numpy(), _reference(K[0], V[0], q_small, [T] * B, nb, G, sel, tail), G)
+    _check(o3.cpu().numpy(), _reference(K[0], V[0], q_big, [T] * B, nb, G, sel, tail), G)
+    cache.check()
+
+
 def test_prefill_one_token_is_decode():
     B, Hkv, Hq, T = 2, 2, 4, 200
     bt = H.build(layers=1, loops=4, Lg=4, B=B, T=T, H=Hkv, Hq=Hq, n_tail=1, chunk=64, seed=0x5EED9300)
