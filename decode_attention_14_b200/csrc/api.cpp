@@ -796,15 +796,16 @@ int rq_prefill_attn(rq_cache *c, int layer, int loop, const void *q, int n, floa
     if (layer < 0 || layer >= cfg.num_layers || loop < 0 || loop >= cfg.num_loops) return RQ_ERR_INVALID;
     if (cfg.format != RQ_FMT_RESIDUAL) return RQ_ERR_STATE;
     // the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4,
-    // the last-loop reference and contiguous records
+    // the last-loop reference (contiguous or paged records)
     if (cfg.anchor_bits == 2 && cfg.resid_bits == 4) return RQ_ERR_UNSUPPORTED;
-    if (cfg.anchor_mode != 0 || cfg.block_tokens != 0) return RQ_ERR_UNSUPPORTED;
+    if (cfg.anchor_mode != 0) return RQ_ERR_UNSUPPORTED;
     PrefillArgs a;
     std::memset(&a, 0, sizeof(a));
     const int group = loop / L.Lg, j = loop % L.Lg;
     const size_t slot = (size_t)layer * L.groups + group;
     const int T = c->len[slot];
     fill_lens(seq_lens(c, slot), cfg.batch, &a.seqT);
+    a.pg = pages_of(c);
     for (int kv = 0; kv < 2; kv++) {
         a.a_codes[kv] = anchor_codes(c, layer, group, kv);
         a.a_meta[kv] = anchor_meta(c, layer, group, kv);

@@ -349,7 +349,9 @@ __device__ __forceinline__ void setup_queries(const PrefillArgs &a, uint8_t *sm,
     }
 }
 
-template <int BA, int BR, int GS, bool RESID>
+// PG: records in a pool of blocks behind a block table (a.pg.table set); the
+// contiguous instantiation carries none of the block arithmetic.
+template <int BA, int BR, int GS, bool RESID, bool PG>
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // per step buffer b = j & 1 (k-th completion: step 2k + b); cfull per
@@ -735,9 +737,18 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         const int side = dq >> 2;
         const int part = (0x31201302u >> (4 * dq)) & 0xF;   // 2, 0, 3, 1, 0, 2, 1, 3
         const int t = lane;
+        // record row of the first token of committed step j (a step lies in
+        // one block of a paged cache: splits start on 64-token tiles and
+        // blocks hold 128 or 256 tokens)
+        auto step_row = [&](int j) -> size_t {
+            const int tok = t0 + j * kTok;
+            if (!PG) return bh * a.Tp + (size_t)tok;
+            const int blk = __ldg(a.pg.table + (size_t)b * a.pg.mb + (tok >> a.pg.shift));
+            return (((size_t)blk * a.H + h) << a.pg.shift) + (size_t)(tok & (a.pg.bt - 1));
+        };
         auto load = [&](int j, RawHalf &r, uint16_t *cf) {
             const bool ok = t < min(kTok, cnt - j * kTok);
-            const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok + t;
+            const size_t rec = step_row(j) + t;
             if (part < 2) {
                 load_half<BA, GS>(ok ? a.a_codes[side] + rec * (16 * BA) : nullptr,
                                   ok ? a.a_meta[side] + rec * MR : nullptr, part, ok, r);
@@ -754,12 +765,13 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_tc_kernel(const PrefillA
         // meta) of step j + 1 + kPrefetchSteps of its side into L2 while step
         // j is written, so that the register loads of that step find them
         // there: a whole step (the padded token capacity of a sequence is a
-        // multiple of 64 tokens, so a full step never leaves it).  The
+        // multiple of 64 tokens and a block holds 128 or 256, so a full step
+        // never leaves the sequence's records or its block).  The
         // residual records are not prefetched: that made residual loops
         // slower 1 or 2 steps ahead and gained nothing 3 steps ahead.
         auto prefetch = [&](int j) {
             if (kPrefetchSteps <= 0 || lane != 0 || part != 0 || j >= ntc) return;
-            const size_t rec = bh * a.Tp + t0 + (size_t)j * kTok;
+            const size_t rec = step_row(j);
             prefetch_l2(a.a_codes[side] + rec * (16 * BA), kTok * 16 * BA);
             prefetch_l2(a.a_meta[side] + rec * MR, kTok * MR);
         };
@@ -979,12 +991,12 @@ __global__ void __launch_bounds__(128) prefill_combine_kernel(const PrefillArgs 
     a.out[row * kHeadDim + tid] = (l > 0.f) ? o / l : 0.f;
 }
 
-template <int BA, int BR, int GS, bool RESID>
+template <int BA, int BR, int GS, bool RESID, bool PG>
 struct Variant {
     static cudaError_t configure() {
         static bool done[kMaxDevices];
         return once_per_device(done, [] {
-            return cudaFuncSetAttribute(prefill_tc_kernel<BA, BR, GS, RESID>,
+            return cudaFuncSetAttribute(prefill_tc_kernel<BA, BR, GS, RESID, PG>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         });
     }
@@ -992,14 +1004,16 @@ struct Variant {
         cudaError_t e = configure();
         if (e != cudaSuccess) return e;
         if (a.S > 0)
-            prefill_tc_kernel<BA, BR, GS, RESID><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, kSmemBytes, st>>>(a);
+            prefill_tc_kernel<BA, BR, GS, RESID, PG><<<dim3(a.S, a.H, a.B * a.nqb), kThreadsP, kSmemBytes, st>>>(a);
         return cudaGetLastError();
     }
 };
 
 template <int BA, int BR, int GS>
 cudaError_t launch_bits(const PrefillArgs &a, cudaStream_t st) {
-    return a.r_codes[0] ? Variant<BA, BR, GS, true>::launch(a, st) : Variant<BA, BR, GS, false>::launch(a, st);
+    if (a.pg.table)
+        return a.r_codes[0] ? Variant<BA, BR, GS, true, true>::launch(a, st) : Variant<BA, BR, GS, false, true>::launch(a, st);
+    return a.r_codes[0] ? Variant<BA, BR, GS, true, false>::launch(a, st) : Variant<BA, BR, GS, false, false>::launch(a, st);
 }
 
 template <int GS>

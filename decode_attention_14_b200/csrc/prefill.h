@@ -21,6 +21,7 @@ struct PrefillArgs {
     float *partials;                   // [B][n][Hq][S][kPartialStride]
     float *out;                        // [B][n][Hq][d] fp32
     SeqLens seqT;                      // committed tokens of each sequence
+    Pages pg;                          // token -> record row (contiguous: row bh * Tp + t)
     int B, H, Hq, G, n, n_tail, tail_cap, Tp, S;
     int nqb;                           // blocks of 64 query rows per kv head
     int g;                             // quantization group size

@@ -254,8 +254,9 @@ int rq_decode_attn_bf16(rq_cache *cache, int layer, int loop, const void *q_bf16
  * must be ordered by the caller.
  * Errors: INVALID (null pointer, n_tokens < 1, index out of range), STATE
  * (wrong format, or a sequence holds fewer than n_tokens tokens),
- * UNSUPPORTED (n_tokens > 65535, or an INT2 anchor with INT4 residuals --
- * the multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4),
+ * UNSUPPORTED (n_tokens > 65535, an INT2 anchor with INT4 residuals -- the
+ * multi-token kernel is built for INT4/INT2, INT2/INT2 and INT4/INT4 -- or
+ * the chained, previous-loop reference),
  * NOMEM, CUDA.  UNSUPPORTED is returned before any allocation.
  */
 int rq_prefill_attn(rq_cache *cache, int layer, int loop, const void *q_bf16, int n_tokens, float *out,
@@ -350,8 +351,8 @@ size_t rq_decode_bytes(const rq_cache *cache, int layer, int loop);
  * Blocks carry reference counts: a forked sequence shares its source's
  * blocks until either sequence writes into a shared one, which is then
  * copied first (copy-on-write, enqueued on the appending call's stream).
- * Decode, export and the other calls work on paged caches as on contiguous
- * ones; rq_prefill_attn returns RQ_ERR_UNSUPPORTED for them.
+ * Decode, rq_prefill_attn, export and the other calls work on paged caches
+ * as on contiguous ones.
  */
 
 /* Makes sequence dst (every committed length 0, no tail tokens in the cache)

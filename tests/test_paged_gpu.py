@@ -161,3 +161,33 @@ def test_paged_ouro_8k_batch4_sampled():
                  block_tokens=128, num_blocks=4 * 64 + 8, prepare=_shuffled(12))
     _check(bt, sel=[(0, 3), (3, 12)])
     bt.cache.close()
+
+
+@pytest.mark.parametrize("bt_tokens", [128, 256])
+def test_paged_prefill_equals_contiguous(bt_tokens):
+    """rq_prefill_attn on a paged cache (blocks scattered over the pool) gives
+    the contiguous cache's outputs bit for bit, with the new tokens in a
+    residual loop's tail and committed at the anchor loop: the same records,
+    splits and steps (a 32-token step lies inside one block)."""
+    B, Hkv, Hq, T, n = 3, 2, 4, 700, 24
+    kw = dict(layers=1, loops=4, Lg=4, B=B, T=T, H=Hkv, Hq=Hq, n_tail=0, chunk=100,
+              seed=0x5EEDC400 + bt_tokens, max_tokens=T + n)
+    paged = H.build(block_tokens=bt_tokens, num_blocks=40, prepare=_shuffled(9), **kw)
+    flat = H.build(**kw)
+    blocks = paged.cache.seq_blocks(1)
+    assert any(b2 != b1 + 1 for b1, b2 in zip(blocks, blocks[1:]))    # scattered over the pool
+    g = torch.Generator(device="cuda").manual_seed(bt_tokens)
+    K = torch.randn((4, B, n, Hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((4, B, n, Hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((B, n, Hq, 128), generator=g, device="cuda").to(torch.bfloat16)
+    for bt in (paged, flat):
+        bt.cache.append(0, 0, K[0], V[0])
+    outs = [bt.cache.prefill(0, 0, q) for bt in (paged, flat)]
+    assert torch.equal(outs[0], outs[1])
+    for bt in (paged, flat):
+        for j in range(1, 4):
+            bt.cache.append(0, j, K[j], V[j])
+    outs = [bt.cache.prefill(0, 3, q) for bt in (paged, flat)]
+    assert torch.equal(outs[0], outs[1])
+    paged.cache.check()
+    flat.cache.check()
