@@ -688,7 +688,8 @@ def prefill_mma_flops(n, G, B, H, T, resid):
 
 
 def run_prefill(args):
-    """rq_prefill_attn on the Ouro-1.4B-shaped cache (B = 4, T = 8192, H = 16):
+    """rq_prefill_attn on the Ouro-1.4B-shaped cache (B = 4, T = 8192, H = 16;
+    with --paged in 128-token blocks scattered over the pool):
     n new tokens per sequence, timed at a residual loop (the chunk in the BF16
     tail) and at the anchor loop (the chunk committed).  One JSON line per
     (n, loop kind).  FLOPs counted: 2 x 128 for q.k and 2 x 128 for p v per
@@ -706,9 +707,15 @@ def run_prefill(args):
     reps = 10
     rows = []
     for n in [int(x) for x in args.prefill.split(",")]:
+        paging = {}
+        if args.paged:   # 128-token blocks, allocation scattered over the pool
+            paging = dict(block_tokens=128, num_blocks=B * ((T + n + 127) // 128) + 8)
         cfg = rq.make_config(num_layers=1, num_loops=loops, loops_per_group=Lg, batch=B, max_tokens=T + n,
-                             max_tail_tokens=max(FILL_CHUNK, n), num_kv_heads=H, num_q_heads=Hq, seed=0xA11CE)
+                             max_tail_tokens=max(FILL_CHUNK, n), num_kv_heads=H, num_q_heads=Hq, seed=0xA11CE,
+                             **paging)
         cache = rq.Cache(cfg, device=dev)
+        if args.paged:
+            cache.shuffle_free_blocks(0x5EED)
         seed = 0x5EED0007 + n
         for t0 in range(0, T, FILL_CHUNK):
             Kg, Vg = synth.group_kv(seed, 0, 0, Lg, base["sigma"], B, FILL_CHUNK, H, t0=t0, device=dev)
@@ -749,6 +756,7 @@ def run_prefill(args):
             mma = prefill_mma_flops(n, Hq // H, B, H, committed, kind == "residual")
             peak, peak_kind = _bf16_peak()
             row = {"prefill": "ouro8k_b4", "n_tokens": n, "loop": kind, "batch": B, "seq_len": committed,
+                   "paged": "128-token blocks, shuffled pool" if args.paged else None,
                    "us_per_call": round(us, 1), "query_tokens_per_s": round(B * n / (us * 1e-6), 1),
                    "decode_bytes_per_call": cache.decode_bytes(0, loop),
                    "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
