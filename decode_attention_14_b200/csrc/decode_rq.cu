@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
             };
             // bulk copies of tokens [t, t + cnt) of an array with rec bytes per
             // record, one per block the run touches
-            auto copy_run = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
+            auto copy_rows = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
                 const uint8_t *src = static_cast<const uint8_t *>(base);
                 while (cnt > 0) {
                     const int c = paged ? min(cnt, a.pg.bt - (t & (a.pg.bt - 1))) : cnt;
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                 mbar_expect_tx(&bar_cf, (uint32_t)(NR * ntiles * kTile * 2));
 #pragma unroll
                 for (int k = 0; k < NR; k++)
-                    copy_run(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1], 2, t0, ntiles * kTile,
+                    copy_rows(smem + P::RING + k * P::coef_bytes(a.chunk), a.r_coef[k][1], 2, t0, ntiles * kTile,
                              &bar_cf);
             } else if (RESID) {
                 mbar_arrive(&bar_cf);   // nothing to fetch
@@ -517,6 +517,17 @@ __global__ void __launch_bounds__(kThreads, GK == 1 ? RQ_DECODE_MIN_CTAS : 3) de
                         continue;
                     }
 #endif
+                    // paged: one run per stream, at a row found once per item (an
+                    // item lies inside one block: items follow the 128-token grid,
+                    // blocks hold 128 or 256 tokens)
+                    const size_t prow = PG ? row_of(tj) : 0;
+                    auto copy_run = [&](uint8_t *dst, const void *base, int rec, int t, int cnt, uint64_t *bar) {
+                        if (PG) {
+                            bulk_g2s(dst, static_cast<const uint8_t *>(base) + prow * rec, (uint32_t)(cnt * rec), bar);
+                        } else {
+                            copy_rows(dst, base, rec, t, cnt, bar);
+                        }
+                    };
                     if (pass == 0) {
                         mbar_expect_tx(bar, (uint32_t)(toks * (P::A_C + P::MR + NR * (P::R_C + P::MR + 2))));
                         copy_run(st + skip * P::A_C, a.a_codes[0], P::A_C, tj, toks, bar);
