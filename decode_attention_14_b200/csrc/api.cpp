@@ -1114,8 +1114,22 @@ int rq_check(rq_cache *c) {
         // happened.
         cudaMemset(c->base + c->lay.off_counters, 0, c->lay.off_err + sizeof(int) - c->lay.off_counters);
         noalloc_reset_counters();
+        if (c->prefill_cnt) cudaMemset(c->prefill_cnt, 0, c->prefill_cnt_n * sizeof(int));
         if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
         return RQ_ERR_TIMEOUT;
+    }
+    // every completed rq_prefill_attn leaves its split-arrival counters at zero
+    if (c->prefill_cnt) {
+        std::vector<int> cnt(c->prefill_cnt_n);
+        if (cudaMemcpy(cnt.data(), c->prefill_cnt, cnt.size() * sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+            return RQ_ERR_CUDA;
+        for (int v : cnt) {
+            if (v != 0) {
+                cudaMemset(c->prefill_cnt, 0, c->prefill_cnt_n * sizeof(int));
+                if (cudaDeviceSynchronize() != cudaSuccess) return RQ_ERR_CUDA;
+                return RQ_ERR_STATE;
+            }
+        }
     }
     return RQ_OK;
 }

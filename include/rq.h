@@ -377,9 +377,11 @@ int rq_cache_free_blocks(const rq_cache *cache, int *n);
 int rq_cache_seq_blocks(const rq_cache *cache, int seq, int32_t *host_blocks, int max_blocks, int *n);
 
 /* Reports asynchronous failures: RQ_ERR_TIMEOUT if a kernel's bounded wait
- * gave up (the error word and the split-combine counters -- the cache's and
- * rq_decode_attn_noalloc's on this device -- are then cleared, so later calls
- * start clean), RQ_ERR_CUDA if the context holds a sticky error, else RQ_OK.
+ * gave up (the error word and the split-combine counters -- the cache's,
+ * rq_prefill_attn's and rq_decode_attn_noalloc's on this device -- are then
+ * cleared, so later calls start clean), RQ_ERR_CUDA if the context holds a
+ * sticky error, RQ_ERR_STATE if rq_prefill_attn's split-arrival counters are
+ * not all zero after its calls completed (they are cleared), else RQ_OK.
  * Synchronises the device. */
 int rq_check(rq_cache *cache);
 
